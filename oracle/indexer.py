@@ -1,0 +1,208 @@
+"""fp64 oracle of the indexer hot path (test infrastructure only; see the package header).
+
+Everything here follows "ADIndex: Layer-Adaptive Sparse Attention Indexing via Group-Level
+Distillation" (arXiv 2611.12956v1), cited as "ADIndex" with section and equation. All
+arrays are float64 real values (operand codes are decoded by ``oracle.fp_formats`` first);
+positions are absolute token positions (0-based).
+
+Readings taken where the page is garbled or silent (each one is also listed in the design
+notes of the repository):
+  * Eq. (1): the gate w multiplies ReLU(q.k) per head and the heads are summed; no 1/sqrt(d)
+    or other scale appears, so none is applied. w may have any sign.
+  * Causal visibility includes the query's own position: key s is visible to a query at
+    position p iff s <= p.
+  * Top-K ties are broken by ascending position; rows with fewer than K visible keys return
+    all of them. Results are sets; order carries no meaning.
+  * Group mode has two readings of the bank (Eq. 13) and the candidate set (Eq. 14):
+      "paper"  - anchor a = the group's first query; scan s <= a; bank = Top-B; query i adds
+                 the post-anchor positions a+1..i. Groups with a + 1 <= B and incomplete
+                 trailing groups use the plain indexer (§4.3 "Shared Token Bank
+                 Construction" and "Application to Prefill and MTP").
+      "window" - scan s < a; bank = Top-(B-G) of the scan plus the group's own window
+                 a..a+G-1 (total B); query i's candidates are the bank entries <= i.
+                 Incomplete trailing groups use the plain indexer.
+"""
+
+from dataclasses import dataclass
+
+import numpy as np
+
+
+# ---------------------------------------------------------------------------------------
+# Eq. (1) and Eq. (2)
+# ---------------------------------------------------------------------------------------
+
+def score_keys(q_t, w_t, keys):
+    """ADIndex §3, Eq. (1) for one query against an explicit list of key vectors.
+
+    q_t [H, d], w_t [H], keys [n, d]  ->  I [n] with I[s] = sum_j w_t[j] * max(0, q_t[j] . keys[s]).
+    """
+    q_t = np.asarray(q_t, dtype=np.float64)
+    keys = np.asarray(keys, dtype=np.float64)
+    if keys.shape[0] == 0:
+        return np.zeros(0)
+    logits = q_t @ keys.T                     # [H, n], one dot product per (head, key)
+    return np.asarray(w_t, dtype=np.float64) @ np.maximum(logits, 0.0)
+
+
+def indexer_scores(q, w, k, pos):
+    """Eq. (1) over the causal prefix of every query: I [T, S], -inf where s > pos[t].
+
+    q [T, H, d], w [T, H], k [S, d], pos [T] (absolute position of each query row).
+    """
+    T, S = q.shape[0], k.shape[0]
+    out = np.full((T, S), -np.inf)
+    for t in range(T):
+        n = min(int(pos[t]) + 1, S)
+        out[t, :n] = score_keys(q[t], w[t], k[:n])
+    return out
+
+
+def topk(scores, K, positions=None):
+    """ADIndex §3, Eq. (2): the min(K, n) highest-scoring candidates.
+
+    ``scores`` [n] are candidate scores, ``positions`` [n] their key positions (defaults to
+    0..n-1). Order: score descending, then position ascending. Returns positions, in that
+    order.
+    """
+    scores = np.asarray(scores, dtype=np.float64)
+    if positions is None:
+        positions = np.arange(scores.shape[0])
+    positions = np.asarray(positions, dtype=np.int64)
+    if not np.all(np.isfinite(scores)):
+        raise ValueError("oracle requires finite scores")
+    order = np.lexsort((positions, -scores))
+    return positions[order[: min(int(K), scores.shape[0])]]
+
+
+def flat_topk_row(q_t, w_t, k, p, K):
+    """Plain DSA indexer for one query at position p: Top-K over keys s <= p (Eqs. 1-2)."""
+    n = min(int(p) + 1, k.shape[0])
+    return topk(score_keys(q_t, w_t, k[:n]), K)
+
+
+def flat_topk(q, w, k, pos, K, rows=None):
+    """Plain DSA indexer: {row: Top-K positions} for the requested rows (all by default)."""
+    rows = range(q.shape[0]) if rows is None else rows
+    return {int(t): flat_topk_row(q[t], w[t], k, pos[t], K) for t in rows}
+
+
+# ---------------------------------------------------------------------------------------
+# Group plan: which keys each stage of the group procedure scores (§4.3, Appendix A.2)
+# ---------------------------------------------------------------------------------------
+
+@dataclass(frozen=True)
+class GroupPlan:
+    """One query group of the procedure.
+
+    kind      "bank" (shared bank + refinement) or "flat" (plain indexer for every member)
+    rows      query rows of the members (consecutive)
+    anchor    position of the first member
+    scan_n    keys scanned by the group query: positions 0..scan_n-1
+    bank_k    size of the scan Top-K kept in the bank
+    post_lo   first position added to every member i's candidates (post_lo..pos_i)
+    """
+    kind: str
+    rows: tuple
+    anchor: int
+    scan_n: int = 0
+    bank_k: int = 0
+    post_lo: int = 0
+
+
+def plan_groups(T, q_pos0, G, B, mode, fallback="group"):
+    """Split T query rows (row t at position q_pos0 + t) into consecutive groups of G.
+
+    mode      "paper" or "window" (see the module header)
+    fallback  "group":  prefill rule - a group falls back when its anchor's visible prefix
+                        a + 1 does not exceed the budget B, or when it is incomplete
+                        (ADIndex §4.3, "Application to Prefill and MTP").
+              "window": MTP rule - the whole window falls back when the first query's
+                        visible prefix q_pos0 + 1 does not exceed B (§4.3 and Appendix A.2,
+                        "Bank Sharing During MTP Target Verification").
+    """
+    if mode not in ("paper", "window"):
+        raise ValueError(mode)
+    plans = []
+    whole_window_flat = fallback == "window" and (q_pos0 + 1) <= B
+    for g0 in range(0, T, G):
+        rows = tuple(range(g0, min(g0 + G, T)))
+        a = q_pos0 + g0
+        incomplete = len(rows) < G
+        if mode == "paper":
+            short = (a + 1) <= B if fallback == "group" else whole_window_flat
+            if incomplete or short:
+                plans.append(GroupPlan("flat", rows, a))
+            else:
+                plans.append(GroupPlan("bank", rows, a, scan_n=a + 1, bank_k=B, post_lo=a + 1))
+        else:
+            if incomplete or whole_window_flat:
+                plans.append(GroupPlan("flat", rows, a))
+            else:
+                plans.append(GroupPlan("bank", rows, a, scan_n=a, bank_k=B - G, post_lo=a))
+    return plans
+
+
+def token_bank(qbar_g, wbar_g, k, plan):
+    """ADIndex §4.3, Eq. (13): the shared bank of one group.
+
+    Scores the scanned prefix once with the group query (Eq. (8) has the same form as
+    Eq. (1)) and keeps its Top-``bank_k`` positions.
+    """
+    n = min(plan.scan_n, k.shape[0])
+    return topk(score_keys(qbar_g, wbar_g, k[:n]), plan.bank_k)
+
+
+def refine_row(q_i, w_i, k, bank, post_lo, p_i, K):
+    """ADIndex §4.3, Eq. (14): Top-K of the original indexer over C_i = bank U {post_lo..p_i}."""
+    cand = np.union1d(np.asarray(bank, dtype=np.int64), np.arange(post_lo, int(p_i) + 1))
+    cand = cand[cand <= p_i]
+    return topk(score_keys(q_i, w_i, k[cand]), K, positions=cand)
+
+
+def group_topk(q, w, k, qbar, wbar, q_pos0, G, B, K, mode, rows=None, fallback="group"):
+    """Prefill in group mode: {row: Top-K positions}; group g uses qbar[g], wbar[g].
+
+    Banks are only built for groups that own a requested row.
+    """
+    want = None if rows is None else set(int(r) for r in rows)
+    out, banks = {}, {}
+    for gi, plan in enumerate(plan_groups(q.shape[0], q_pos0, G, B, mode, fallback)):
+        todo = [t for t in plan.rows if want is None or t in want]
+        if not todo:
+            continue
+        if plan.kind == "flat":
+            for t in todo:
+                out[t] = flat_topk_row(q[t], w[t], k, q_pos0 + t, K)
+            continue
+        bank = token_bank(qbar[gi], wbar[gi], k, plan)
+        banks[gi] = bank
+        for t in todo:
+            out[t] = refine_row(q[t], w[t], k, bank, plan.post_lo, q_pos0 + t, K)
+    return out, banks
+
+
+# ---------------------------------------------------------------------------------------
+# Decode (one query per sequence, each sequence with its own key cache)
+# ---------------------------------------------------------------------------------------
+
+def decode_topk(q, w, caches, seq_len, K):
+    """Plain indexer at decode: row b sits at position seq_len[b]-1 of its own cache."""
+    return {b: flat_topk_row(q[b], w[b], caches[b], int(seq_len[b]) - 1, K)
+            for b in range(q.shape[0])}
+
+
+def decode_bank(qbar, wbar, caches, seq_len, B):
+    """Bank refresh at decode: Eq. (13) with the anchor at the refreshing query's position
+    a = seq_len[b]-1, i.e. Top-B of the group query's scores over s <= a."""
+    return {b: token_bank(qbar[b], wbar[b], caches[b],
+                          GroupPlan("bank", (b,), int(seq_len[b]) - 1,
+                                    scan_n=int(seq_len[b]), bank_k=B))
+            for b in range(qbar.shape[0])}
+
+
+def decode_refine(q, w, caches, seq_len, banks, anchors, K):
+    """Decode step reusing a bank: Eq. (14) with C = bank U {a+1 .. seq_len[b]-1}."""
+    return {b: refine_row(q[b], w[b], caches[b], banks[b], int(anchors[b]) + 1,
+                          int(seq_len[b]) - 1, K)
+            for b in range(q.shape[0])}

@@ -1,0 +1,289 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself.
+
+Sources: "ADIndex: Layer-Adaptive Sparse Attention Indexing via Group-Level Distillation"
+(arXiv 2611.12956v1) - §3 Eqs. (1)-(2), §1 (exact recovery when the bank holds the Top-K),
+§4.3 Eqs. (13)-(14) and the fallback rules, Appendix A and Table 5 (score counts) - plus
+library routines (torch's bf16 / float8 conversions, numpy's stable argsort) and brute force.
+"""
+
+import itertools
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import cost_model, fp_formats
+from oracle import indexer as ox
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------------------------------
+# operand decoding
+# ---------------------------------------------------------------------------------------
+
+def test_bf16_decode_matches_torch_on_every_code():
+    codes = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = torch.from_numpy(codes.view(np.int16)).view(torch.bfloat16).double().numpy()
+    got = fp_formats.bf16_bits_to_f64(codes)
+    nan = np.isnan(ref)
+    assert np.array_equal(nan, np.isnan(got))
+    assert np.array_equal(ref[~nan], got[~nan])
+
+
+def test_e4m3_decode_matches_torch_on_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    got = fp_formats.e4m3_to_f64(codes)
+    nan = np.isnan(ref)
+    assert np.array_equal(nan, np.isnan(got))
+    assert nan.sum() == 2  # 0x7F and 0xFF
+    assert np.array_equal(ref[~nan], got[~nan])
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9  # largest finite, smallest subnormal
+
+
+def test_dequantize_applies_per_row_scale():
+    codes = np.array([[0x38, 0xB8], [0x40, 0x00]], dtype=np.uint8)  # 1, -1 ; 2, 0
+    got = fp_formats.dequantize(codes, np.array([0.5, 3.0], dtype=np.float32), "e4m3")
+    assert np.array_equal(got, [[0.5, -0.5], [6.0, 0.0]])
+
+
+# ---------------------------------------------------------------------------------------
+# Eq. (1): hand-computed values and closed forms
+# ---------------------------------------------------------------------------------------
+
+Q2 = np.array([[1.0, 2.0], [-1.0, 1.0]])          # H = 2 heads, d = 2
+K3 = np.array([[3.0, -1.0], [0.0, 1.0], [-2.0, -2.0]])
+
+
+def test_score_hand_values():
+    # head 0 dots: 1, 2, -6 -> ReLU 1, 2, 0 ; head 1 dots: -4, 1, 0 -> ReLU 0, 1, 0
+    # I = 0.5 * [1, 2, 0] + 2 * [0, 1, 0]
+    assert np.array_equal(ox.score_keys(Q2, [0.5, 2.0], K3), [0.5, 3.0, 0.0])
+
+
+def test_score_negative_gate_keeps_relu_per_head():
+    # ReLU before the gate: a negative gate can make a score negative
+    assert np.array_equal(ox.score_keys(Q2, [-1.0, 1.0], K3), [-1.0, -1.0, 0.0])
+
+
+def test_score_all_negative_logits_is_zero():
+    k = -np.abs(np.random.default_rng(0).normal(size=(5, 2)))
+    q = np.abs(np.random.default_rng(1).normal(size=(3, 2)))
+    assert np.array_equal(ox.score_keys(q, [1.0, 2.0, 3.0], k), np.zeros(5))
+
+
+def test_score_single_head_unit_gate_is_dot_product():
+    rng = np.random.default_rng(2)
+    q = rng.normal(size=(1, 16))
+    k = rng.normal(size=(40, 16))
+    k[np.dot(k, q[0]) < 0] *= -1                     # make every dot product positive
+    assert np.allclose(ox.score_keys(q, [1.0], k), np.dot(k, q[0]), rtol=1e-14, atol=0)
+
+
+def test_score_positive_scales_factor_out():
+    rng = np.random.default_rng(3)
+    q, w, k = rng.normal(size=(4, 8)), rng.normal(size=4), rng.normal(size=(10, 8))
+    got = ox.score_keys(q * 0.25, w, k * 8.0)
+    assert np.allclose(got, 2.0 * ox.score_keys(q, w, k), rtol=1e-13, atol=1e-13)
+
+
+def test_indexer_scores_causal_mask():
+    rng = np.random.default_rng(4)
+    T, H, d = 6, 2, 4
+    q, w, k = rng.normal(size=(T, H, d)), rng.random((T, H)), rng.normal(size=(T, d))
+    I = ox.indexer_scores(q, w, k, np.arange(T))
+    for t in range(T):
+        assert np.all(np.isfinite(I[t, : t + 1])) and np.all(I[t, t + 1:] == -np.inf)
+        # brute force: per head, per key, written out
+        for s in range(t + 1):
+            ref = sum(w[t, j] * max(0.0, sum(q[t, j, x] * k[s, x] for x in range(d)))
+                      for j in range(H))
+            assert abs(I[t, s] - ref) <= 1e-12 * max(1.0, abs(ref))
+
+
+# ---------------------------------------------------------------------------------------
+# Eq. (2): Top-K
+# ---------------------------------------------------------------------------------------
+
+def test_topk_brute_force_small():
+    rng = np.random.default_rng(5)
+    for n in range(1, 10):
+        for K in range(1, 5):
+            sc = rng.normal(size=n)
+            got = set(ox.topk(sc, K).tolist())
+            best = None
+            for sub in itertools.combinations(range(n), min(K, n)):
+                rest = [s for s in range(n) if s not in sub]
+                if not rest or min(sc[list(sub)]) >= max(sc[rest]):
+                    best = set(sub)
+            assert got == best
+
+
+def test_topk_matches_stable_argsort_with_ties():
+    sc = np.array([3.0, 1.0, 3.0, 2.0, 3.0, 1.0, 2.0])
+    for K in range(1, 8):
+        ref = np.argsort(-sc, kind="stable")[:K]
+        assert np.array_equal(ox.topk(sc, K), ref)
+
+
+def test_flat_topk_causal_counts():
+    rng = np.random.default_rng(6)
+    T, H, d, K = 12, 2, 4, 4
+    q, w, k = rng.normal(size=(T, H, d)), rng.random((T, H)), rng.normal(size=(T, d))
+    res = ox.flat_topk(q, w, k, np.arange(T), K)
+    for t, idx in res.items():
+        assert len(idx) == min(K, t + 1) == len(set(idx.tolist()))
+        assert idx.max() <= t
+        if t + 1 <= K:
+            assert sorted(idx.tolist()) == list(range(t + 1))
+
+
+def test_topk_permutation_equivariance_and_monotonicity():
+    rng = np.random.default_rng(7)
+    H, d, S, K = 3, 8, 40, 6
+    q, w, k = rng.normal(size=(H, d)), rng.random(H), rng.normal(size=(S, d))
+    base = set(ox.flat_topk_row(q, w, k, S - 1, K).tolist())
+    perm = rng.permutation(S)
+    permuted = set(ox.flat_topk_row(q, w, k[perm], S - 1, K).tolist())
+    assert {int(perm[i]) for i in permuted} == base
+    sc = ox.score_keys(q, w, k)
+    chosen = sorted(base)[0]
+    unchosen = [s for s in range(S) if s not in base][0]
+    k2 = k.copy()
+    k2[chosen] *= 1.5 if sc[chosen] > 0 else 1.0       # raise a selected score
+    k2[unchosen] *= 0.5 if sc[unchosen] > 0 else 1.0   # lower an unselected one
+    assert set(ox.flat_topk_row(q, w, k2, S - 1, K).tolist()) == base
+
+
+# ---------------------------------------------------------------------------------------
+# Eqs. (13)-(14): bank and refinement
+# ---------------------------------------------------------------------------------------
+
+def _prob(T=48, H=3, Hg=2, d=8, G=8, seed=8):
+    rng = np.random.default_rng(seed)
+    q, w, k = rng.normal(size=(T, H, d)), rng.random((T, H)), rng.normal(size=(T, d))
+    qbar, wbar = rng.normal(size=(T // G, Hg, d)), rng.random((T // G, Hg))
+    return q, w, k, qbar, wbar
+
+
+def test_refine_exact_recovery_when_bank_holds_topk():
+    q, w, k, *_ = _prob()
+    rng = np.random.default_rng(9)
+    K = 5
+    for i in range(10, 48):
+        full = ox.flat_topk_row(q[i], w[i], k, i, K)
+        extra = rng.choice(i, size=3, replace=False)
+        bank = np.union1d(full, extra)
+        got = ox.refine_row(q[i], w[i], k, bank, i + 1, i, K)
+        assert set(got.tolist()) == set(full.tolist())
+
+
+@pytest.mark.parametrize("mode", ["paper", "window"])
+def test_large_bank_equals_flat(mode):
+    q, w, k, qbar, wbar = _prob()
+    T, K, G = 48, 5, 8
+    flat = ox.flat_topk(q, w, k, np.arange(T), K)
+    got, _ = ox.group_topk(q, w, k, qbar, wbar, 0, G, B=T + G, K=K, mode=mode)
+    for t in range(T):
+        assert set(got[t].tolist()) == set(flat[t].tolist())
+
+
+def test_window_group_of_one_is_flat():
+    q, w, k, _, _ = _prob()
+    T, K = 48, 5
+    rng = np.random.default_rng(10)
+    qbar, wbar = rng.normal(size=(T, 2, 8)), rng.random((T, 2))
+    flat = ox.flat_topk(q, w, k, np.arange(T), K)
+    got, _ = ox.group_topk(q, w, k, qbar, wbar, 0, 1, B=T + 1, K=K, mode="window")
+    assert all(set(got[t].tolist()) == set(flat[t].tolist()) for t in range(T))
+
+
+def test_candidates_stay_causal_and_in_bank():
+    q, w, k, qbar, wbar = _prob()
+    T, K, G, B = 48, 4, 8, 12
+    for mode in ("paper", "window"):
+        got, banks = ox.group_topk(q, w, k, qbar, wbar, 0, G, B, K, mode)
+        plans = ox.plan_groups(T, 0, G, B, mode)
+        for gi, plan in enumerate(plans):
+            for t in plan.rows:
+                idx = got[t]
+                assert len(idx) == len(set(idx.tolist())) and idx.max() <= t
+                if plan.kind == "bank":
+                    allowed = set(banks[gi].tolist()) | set(range(plan.post_lo, t + 1))
+                    assert set(idx.tolist()) <= allowed
+                    assert len(banks[gi]) == min(plan.bank_k, plan.scan_n)
+                    assert banks[gi].max(initial=-1) < plan.scan_n
+
+
+def test_paper_fallback_rule():
+    plans = ox.plan_groups(T=40, q_pos0=0, G=8, B=16, mode="paper")
+    # anchors 0, 8, 16, 24, 32: reuse needs a + 1 > 16; the last group is complete
+    assert [p.kind for p in plans] == ["flat", "flat", "bank", "bank", "bank"]
+    plans = ox.plan_groups(T=36, q_pos0=0, G=8, B=16, mode="paper")
+    assert plans[-1].kind == "flat" and len(plans[-1].rows) == 4   # incomplete group
+    # MTP: the whole window falls back when its first query sees <= B keys
+    assert all(p.kind == "flat" for p in ox.plan_groups(16, 15, 4, 16, "paper", "window"))
+    assert all(p.kind == "bank" for p in ox.plan_groups(16, 16, 4, 16, "paper", "window"))
+
+
+def test_decode_bank_reuse_matches_definitions():
+    rng = np.random.default_rng(11)
+    Bs, H, Hg, d, S, K, B = 3, 3, 2, 8, 60, 5, 10
+    caches = rng.normal(size=(Bs, S, d))
+    q, w = rng.normal(size=(Bs, H, d)), rng.random((Bs, H))
+    qbar, wbar = rng.normal(size=(Bs, Hg, d)), rng.random((Bs, Hg))
+    n0 = np.array([50, 40, 55])
+    banks = ox.decode_bank(qbar, wbar, caches, n0, B)
+    flat = ox.decode_topk(q, w, caches, n0 + 4, K)
+    # a bank as large as the prefix makes reuse exact
+    big = ox.decode_bank(qbar, wbar, caches, n0, S)
+    got = ox.decode_refine(q, w, caches, n0 + 4, big, n0 - 1, K)
+    assert all(set(got[b].tolist()) == set(flat[b].tolist()) for b in range(Bs))
+    got = ox.decode_refine(q, w, caches, n0 + 4, banks, n0 - 1, K)
+    for b in range(Bs):
+        allowed = set(banks[b].tolist()) | set(range(n0[b], n0[b] + 4))
+        assert set(got[b].tolist()) <= allowed and len(got[b]) == K
+
+
+# ---------------------------------------------------------------------------------------
+# Appendix A: the procedure's score counts reproduce Table 5
+# ---------------------------------------------------------------------------------------
+
+def _table5():
+    rows = []
+    with open(os.path.join(GOLDEN, "table5_speedups.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                p, G, P, *vals = line.split()
+                rows.append((p, int(G), int(P) * 1024, [float(v) for v in vals]))
+    return rows
+
+
+def test_group_cost_matches_eq17():
+    # one bank group with anchor visible prefix N: N + G P + G (G - 1) / 2
+    G, P, a = 16, 4096, 10000
+    plan = ox.plan_groups(G, a, G, P, "paper")
+    assert len(plan) == 1 and plan[0].kind == "bank"
+    assert cost_model.plan_cost(plan, a) == (a + 1) + G * P + G * (G - 1) // 2
+
+
+def test_table5_reproduced_by_the_group_plan():
+    rows = _table5()
+    assert len(rows) == 27
+    ctx = [16 * 1024, 32 * 1024, 64 * 1024, 128 * 1024]
+    cache = {}
+    for panel, G, P, vals in rows:
+        for L, ref in zip(ctx, vals):
+            key = (L, G, P)
+            if key not in cache:
+                cache[key] = cost_model.speedups(L, G, P)
+            got = cache[key]["abc".index(panel)]
+            if panel == "b":
+                # Eqs. (20)-(21) are discrete: same 2-decimal value
+                assert round(got, 2) == pytest.approx(ref, abs=1e-9), (panel, G, P, L, got)
+            else:
+                # (a) and (c) use the integral of Eq. (19); the discrete count differs from it
+                # by less than one unit in the last printed digit
+                assert abs(got - ref) <= 0.0101, (panel, G, P, L, got)
