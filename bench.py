@@ -1,0 +1,497 @@
+#!/usr/bin/env python
+"""Throughput of the indexer hot path on B200: query-key scores/s and Top-K queries/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--rows]
+
+One step = one pass of the flat DSA indexer (score, Eq. (1), + per-query Top-K, Eq. (2))
+over the DSA-shaped prefill workload: T = 16384 causal queries, H_I = 64 heads, d = 128,
+K = 2048, bf16 operands on anchor-structured synthetic data. Inputs are resident in HBM
+before the timed region and larger than L2 (q alone is 256 MiB), so no L2 flush is needed.
+Under torchrun each rank runs its own replica of the workload (weak scaling, no collective
+on the data path); the time is the max over ranks.
+
+--rows also times the other hot-path rows on their own workloads (FP8 flat prefill, ADIndex
+group mode on 64K tokens, decode with an FP8 key cache, decode with bank reuse) and adds
+them under "rows". --impl reference times the fp64 CPU oracle on the host cores instead.
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FLAT = dict(T=16384, H=64, d=128, K=2048, seed=1)
+GROUP = dict(T=65536, H=64, d=128, K=2048, G=64, B=8192, Hg=16, seed=2)
+DECODE = dict(Bs=32, S=131072, H=64, d=128, K=2048, Hg=16, B=8192, G=16, seed=3)
+
+
+def flat_pairs(T, q_pos0=0):
+    return sum(q_pos0 + t + 1 for t in range(T)) if q_pos0 else T * (T + 1) // 2
+
+
+# ---------------------------------------------------------------------------------------
+# infrastructure
+# ---------------------------------------------------------------------------------------
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x):
+        if not self.pg:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+class Clocks:
+    """Samples SM clocks and throttle reasons with nvidia-smi while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc:
+            time.sleep(0.3)
+            self.proc.terminate()
+            self.proc.wait()
+
+    def summary(self):
+        self.f.seek(0)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.f.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.f.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"],
+                    bf16_sustained=p.get("bf16_tflops_sustained"), source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def kernel_traffic(name):
+    """Per-launch DRAM bytes from the committed ncu summary of a kernel, if it was taken on
+    the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{name}.md")
+    src = os.path.join(ROOT, "sparse_attention_token_indexer_b200", "csrc", "score_sm100.cu")
+    if not os.path.exists(path):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    vals = {}
+    for line in open(path):
+        if ":" in line and line.startswith("- "):
+            k, v = line[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("source_sha256_16") != h:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch_full_size"])
+    except (KeyError, ValueError):
+        return None
+
+
+class StageTimer:
+    """CUDA events the library records around its scoring and selection kernels."""
+
+    def __init__(self, lib, steps):
+        import ctypes
+        self.ctypes, self.lib = ctypes, lib
+        self.ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+        for evs in self.ev:          # torch creates the CUDA event on its first record
+            for e in evs:
+                e.record()
+        torch.cuda.synchronize()
+        self.arr = []
+        for evs in self.ev:
+            a = (ctypes.c_void_p * 4)(*[e.cuda_event for e in evs])
+            self.arr.append(a)
+
+    def arm(self, i):
+        self.lib.adx_set_timing_events(self.arr[i], 4)
+
+    def disarm(self):
+        self.lib.adx_set_timing_events(None, 0)
+
+    def ms(self, a, b):
+        return [evs[a].elapsed_time(evs[b]) for evs in self.ev]
+
+
+def timed(fn, steps, warmup, dist, stage_timer=None):
+    """W untimed steps, then exactly K timed steps between barriers; returns ms per step
+    (max over ranks) and the library's launch count inside the timed region."""
+    from sparse_attention_token_indexer_b200 import _lib
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = _lib.lib().adx_launch_count()
+    start.record(s)
+    for i in range(steps):
+        if stage_timer:
+            stage_timer.arm(i)
+        fn()
+    end.record(s)
+    if stage_timer:
+        stage_timer.disarm()
+    torch.cuda.synchronize()
+    launches = _lib.lib().adx_launch_count() - n0
+    dist.barrier()
+    ms = dist.max(start.elapsed_time(end)) / steps
+    return ms, launches
+
+
+# ---------------------------------------------------------------------------------------
+# workloads (our CUDA path)
+# ---------------------------------------------------------------------------------------
+
+def run_flat(args, dist, dtype="bf16", clocks=None):
+    from sparse_attention_token_indexer_b200 import _lib, indexer, inputs
+    c = FLAT
+    p = inputs.anchor_prefill(c["T"], c["H"], c["d"], c["K"], seed=c["seed"], device="cuda",
+                              dtype=dtype)
+    ws = indexer.Workspace("cuda")
+    idx = torch.empty(c["T"], c["K"], dtype=torch.int32, device="cuda")
+
+    def step():
+        _call_prefill(p, c["K"], idx, ws)
+
+    timer = StageTimer(_lib.lib(), args.steps)
+    if clocks is not None:
+        with clocks:
+            ms, launches = timed(step, args.steps, args.warmup, dist, timer)
+    else:
+        ms, launches = timed(step, args.steps, args.warmup, dist, timer)
+    score_ms = statistics.mean(timer.ms(0, 1))
+    select_ms = statistics.mean(timer.ms(2, 3))
+    pairs = flat_pairs(c["T"])
+    return dict(p=p, ms=ms, launches=launches, score_ms=score_ms, select_ms=select_ms,
+                pairs=pairs, flops=pairs * 2 * c["H"] * c["d"], rows=c["T"])
+
+
+def _call_prefill(p, K, idx, ws):
+    import ctypes
+    from sparse_attention_token_indexer_b200 import _lib as L, indexer
+    ops = indexer.make_operands(p["q"], p["w"], p["k"], p["q_scale"], p["k_scale"], p["q_pos0"])
+    buf = ws.get(indexer.workspace_size(L.ADX_OP_PREFILL, ops, K))
+    L.check("adx_index_prefill", L.lib().adx_index_prefill(
+        ctypes.byref(ops), K, ctypes.c_void_p(idx.data_ptr()), None, None, 0,
+        ctypes.c_void_p(buf.data_ptr()), buf.numel(),
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)))
+
+
+def run_e2e(args, dist, p):
+    """Same step through the public API with host buffers: pinned H2D of the inputs, the
+    indexer, and D2H of the Top-K indices, every step inside the timed region."""
+    from sparse_attention_token_indexer_b200 import indexer
+    c = FLAT
+    host = {k: p[k].cpu().pin_memory() for k in ("q", "w", "k")}
+    dev = {k: torch.empty_like(p[k]) for k in ("q", "w", "k")}
+    out_h = torch.empty(c["T"], c["K"], dtype=torch.int32).pin_memory()
+    idx = torch.empty(c["T"], c["K"], dtype=torch.int32, device="cuda")
+    ws = indexer.Workspace("cuda")
+    q = dict(p)
+
+    def step():
+        for k in dev:
+            dev[k].copy_(host[k], non_blocking=True)
+        q.update(dev)
+        _call_prefill(q, c["K"], idx, ws)
+        out_h.copy_(idx, non_blocking=True)
+
+    ms, _ = timed(step, args.steps, args.warmup, dist)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+    return ms, h2d, d2h
+
+
+def run_group(args, dist):
+    from sparse_attention_token_indexer_b200 import indexer, inputs
+    c = GROUP
+    p = inputs.group_prefill(c["T"], c["H"], c["d"], c["K"], c["G"], c["B"], c["Hg"],
+                             seed=c["seed"], device="cuda")
+    ws = indexer.Workspace("cuda")
+
+    def step():
+        bank = indexer.group_bank(p["qbar"], p["wbar"], p["k"], c["G"], c["B"], "window",
+                                  ws=ws)
+        indexer.bank_refine(p["q"], p["w"], p["k"], bank, c["G"], c["B"], "window", c["K"],
+                            ws=ws)
+
+    ms, launches = timed(step, max(2, args.steps // 2), args.warmup, dist)
+    G, B, T = c["G"], c["B"], c["T"]
+    scan = sum(g * G for g in range(T // G))
+    refine = sum(min(B - G, g * G) * G + G * (G + 1) // 2 for g in range(T // G))
+    return dict(ms=ms, launches=launches, scan_pairs=scan, refine_pairs=refine, rows=T,
+                flops=scan * 2 * c["Hg"] * c["d"] + refine * 2 * c["H"] * c["d"])
+
+
+def run_decode(args, dist):
+    from sparse_attention_token_indexer_b200 import indexer, inputs
+    c = DECODE
+    prob = inputs.decode_problem(c["Bs"], c["S"], c["H"], c["d"], c["K"], c["Hg"],
+                                 steps=c["G"], seed=c["seed"], device="cuda")
+    ws = indexer.Workspace("cuda")
+    seq0 = inputs.decode_seq_len(prob, 0)
+    q0, w0 = prob["q_steps"][0], prob["w_steps"][0]
+
+    def flat_step():
+        indexer.index_decode(q0, w0, prob["k"], seq0, c["K"], k_scale=prob["k_scale"], ws=ws)
+
+    ms_flat, l_flat = timed(flat_step, args.steps, args.warmup, dist)
+    seqs = [inputs.decode_seq_len(prob, r) for r in range(c["G"])]
+
+    def cycle():
+        qb = prob["q_steps"][0][:, : c["Hg"]].contiguous()
+        wb = prob["w_steps"][0][:, : c["Hg"]].contiguous()
+        bank = indexer.group_bank(qb, wb, prob["k"], c["G"], c["B"], "paper",
+                                  k_scale=prob["k_scale"], seq_len=seqs[0], ws=ws)
+        for r in range(c["G"]):
+            indexer.bank_refine(prob["q_steps"][r], prob["w_steps"][r], prob["k"], bank, c["G"],
+                                c["B"], "paper", c["K"], k_scale=prob["k_scale"],
+                                seq_len=seqs[r], ws=ws)
+
+    ms_cycle, l_cycle = timed(cycle, max(2, args.steps // 4), 1, dist)
+    key_bytes = c["d"] + 4
+    return dict(ms_flat=ms_flat, launches_flat=l_flat, ms_cycle=ms_cycle, launches_cycle=l_cycle,
+                bytes_flat=c["Bs"] * c["S"] * key_bytes, steps_per_cycle=c["G"])
+
+
+# ---------------------------------------------------------------------------------------
+# the oracle on the host cores
+# ---------------------------------------------------------------------------------------
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n and n[0]:
+            return int(n[0])
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def oracle_sample(p, K, seconds, seed=0):
+    """Times the oracle on flat rows drawn across the causal triangle until `seconds` of
+    CPU work are done; returns (pairs scored, rows completed, elapsed seconds)."""
+    from oracle import fp_formats
+    from oracle import indexer as ox
+
+    def f64(t, scale=None):
+        t = t.detach().cpu()
+        if t.dtype == torch.bfloat16:
+            return fp_formats.bf16_bits_to_f64(t.view(torch.int16).numpy().view(np.uint16))
+        return fp_formats.dequantize(t.numpy(), scale.detach().cpu().numpy(), "e4m3")
+
+    q64 = f64(p["q"], p["q_scale"])
+    k64 = f64(p["k"], p["k_scale"])
+    w64 = p["w"].double().cpu().numpy()
+    rng = np.random.default_rng(seed)
+    T = q64.shape[0]
+    pairs = rows = 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < seconds or rows < 4:
+        t = int(rng.integers(T))
+        ox.flat_topk_row(q64[t], w64[t], k64, p["q_pos0"] + t, K)
+        pairs += p["q_pos0"] + t + 1
+        rows += 1
+    return pairs, rows, time.perf_counter() - t0
+
+
+# ---------------------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--rows", action="store_true", help="also time the other hot-path rows")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    dist = Dist()
+    torch.cuda.set_device(dist.local)
+    config = {"workload": "dsa_flat_prefill_T16384_H64_d128_K2048", "T": FLAT["T"],
+              "H_I": FLAT["H"], "d": FLAT["d"], "K": FLAT["K"], "seq_len": FLAT["T"],
+              "global_batch": dist.world, "parallelism": f"replicas{dist.world}",
+              "l2": "inputs larger than L2 (q 256 MiB, scores 1 GiB)"}
+
+    if args.impl == "reference":
+        if dist.rank != 0:
+            dist.close()
+            return
+        from sparse_attention_token_indexer_b200 import inputs
+        p = inputs.anchor_prefill(FLAT["T"], FLAT["H"], FLAT["d"], FLAT["K"], seed=FLAT["seed"])
+        per = max(1.0, args.cpu_seconds / max(args.steps, 1))
+        for _ in range(args.warmup):
+            oracle_sample(p, FLAT["K"], 0.2)
+        tot_pairs = tot_rows = 0
+        tot_s = 0.0
+        for i in range(args.steps):
+            pr, rw, s = oracle_sample(p, FLAT["K"], per, seed=i)
+            tot_pairs, tot_rows, tot_s = tot_pairs + pr, tot_rows + rw, tot_s + s
+        value = tot_pairs / tot_s
+        line = {"impl": "reference", "metric": "indexer query-key scores/s", "value": value,
+                "unit": "scores/s", "n_gpus": dist.world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f64", "data": "synthetic", "config": config,
+                "topk_queries_per_s": tot_rows / tot_s,
+                "cpu_baseline": {"value": value, "unit": "scores/s", "cores": cpu_cores(),
+                                 "kind": "oracle",
+                                 "sample": f"{tot_rows} flat rows drawn uniformly over the "
+                                           f"causal triangle, {tot_s:.1f} s"},
+                "e2e": {"value": value, "unit": "scores/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        dist.close()
+        return
+
+    from sparse_attention_token_indexer_b200 import build
+    build.build()
+    pk = peaks()
+    clocks = Clocks(dist.local)
+    flat = run_flat(args, dist, "bf16", clocks)
+    clk = clocks.summary()
+    value = dist.world * flat["pairs"] / (flat["ms"] * 1e-3)
+    score_tflops = flat["flops"] / (flat["score_ms"] * 1e-3) / 1e12
+    e2e_ms, h2d, d2h = run_e2e(args, dist, flat["p"])
+    line = {
+        "metric": "indexer query-key scores/s", "value": value, "unit": "scores/s",
+        "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": flat["ms"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (anchor-structured, seeded)",
+        "config": config,
+        "topk_queries_per_s": dist.world * flat["rows"] / (flat["ms"] * 1e-3),
+        "stage_ms": {"score": flat["score_ms"], "select": flat["select_ms"]},
+        "roofline": {"kernel": "score_kernel (tcgen05, bf16)", "bound": "tensor",
+                     "achieved": score_tflops, "peak": pk["bf16"], "unit": "TFLOP/s",
+                     "frac": score_tflops / pk["bf16"],
+                     "peak_source": f"{pk['source']} bf16 burst",
+                     "traffic": kernel_traffic("score_kernel_flat_prefill_T16384_bf16")},
+        "e2e": {"value": dist.world * flat["pairs"] / (e2e_ms * 1e-3), "unit": "scores/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": flat["launches"],
+        "clocks": clk,
+    }
+    del flat["p"]
+    if args.rows:
+        rows = {}
+        f8 = run_flat(args, dist, "e4m3")
+        f8.pop("p")
+        rows["flat_prefill_e4m3"] = {
+            "scores_per_s": f8["pairs"] / (f8["ms"] * 1e-3), "ms_per_step": f8["ms"],
+            "score_ms": f8["score_ms"], "select_ms": f8["select_ms"],
+            "score_tflops": f8["flops"] / (f8["score_ms"] * 1e-3) / 1e12,
+            "peak_tflops_e4m3": 2 * pk["bf16"], "gpu_launches": f8["launches"]}
+        g = run_group(args, dist)
+        rows["group_mode_T65536"] = {
+            "ms_per_step": g["ms"], "scan_pairs": g["scan_pairs"],
+            "refine_pairs": g["refine_pairs"],
+            "scores_per_s": (g["scan_pairs"] + g["refine_pairs"]) / (g["ms"] * 1e-3),
+            "topk_queries_per_s": g["rows"] / (g["ms"] * 1e-3),
+            "tflops": g["flops"] / (g["ms"] * 1e-3) / 1e12, "gpu_launches": g["launches"]}
+        dcd = run_decode(args, dist)
+        rows["decode_Bs32_S131072_e4m3"] = {
+            "ms_per_step": dcd["ms_flat"],
+            "scores_per_s": DECODE["Bs"] * DECODE["S"] / (dcd["ms_flat"] * 1e-3),
+            "topk_queries_per_s": DECODE["Bs"] / (dcd["ms_flat"] * 1e-3),
+            "hbm_gbs": dcd["bytes_flat"] / (dcd["ms_flat"] * 1e-3) / 1e9,
+            "hbm_frac": dcd["bytes_flat"] / (dcd["ms_flat"] * 1e-3) / 1e9 / pk["hbm"],
+            "gpu_launches": dcd["launches_flat"]}
+        rows["decode_bank_reuse_cycle16"] = {
+            "ms_per_cycle": dcd["ms_cycle"],
+            "ms_per_step": dcd["ms_cycle"] / dcd["steps_per_cycle"],
+            "topk_queries_per_s": DECODE["Bs"] * dcd["steps_per_cycle"] / (dcd["ms_cycle"] * 1e-3),
+            "gpu_launches": dcd["launches_cycle"]}
+        line["rows"] = rows
+    if dist.rank == 0 and dist.world == 1:
+        pr, rw, s = oracle_sample(_cpu_copy_inputs(), FLAT["K"], args.cpu_seconds)
+        line["cpu_baseline"] = {"value": pr / s, "unit": "scores/s", "cores": cpu_cores(),
+                                "kind": "oracle",
+                                "sample": f"{rw} flat rows drawn uniformly over the causal "
+                                          f"triangle of the same workload, {s:.1f} s"}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.close()
+
+
+def _cpu_copy_inputs():
+    from sparse_attention_token_indexer_b200 import inputs
+    return inputs.anchor_prefill(FLAT["T"], FLAT["H"], FLAT["d"], FLAT["K"], seed=FLAT["seed"],
+                                 device="cuda", dtype="bf16")
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,172 @@
+/*
+ * adx.h - C ABI of the B200 (sm_100a) sparse-attention token indexer.
+ *
+ * The library computes the DeepSeek Sparse Attention token indexer and ADIndex's
+ * group-shared variant of it, as defined in "ADIndex: Layer-Adaptive Sparse Attention
+ * Indexing via Group-Level Distillation" (arXiv 2611.12956v1):
+ *
+ *   score      I[t,s] = sum_j w[t,j] * ReLU(q[t,j] . k[s])          (§3, Eq. (1))
+ *   selection  T_t = TopK_{s <= pos(t)} I[t,s]                        (§3, Eq. (2))
+ *   bank       P = TopK over the group query's scores of a scan      (§4.3, Eq. (13))
+ *   refine     T_i = TopK_{s in C_i} I[i,s], C_i = bank U post-anchor (§4.3, Eq. (14))
+ *
+ * Conventions shared by every entry point
+ *  - Every pointer argument is a DEVICE pointer unless stated otherwise. The caller owns
+ *    all memory; the library allocates nothing, keeps no state between calls besides
+ *    cached device properties, and launches all work asynchronously on `stream` (a
+ *    cudaStream_t passed as void*; NULL = the legacy default stream).
+ *  - Argument errors are detected on the host and returned before any launch.
+ *  - Errors the device detects (a bounded wait that ran out) are recorded in a status word
+ *    at the start of the workspace and reported by adx_read_device_status(). The word is
+ *    sticky: it holds the first error since the workspace was zeroed or last read. Zero the
+ *    workspace's first ADX_STATUS_BYTES once before the first call.
+ *  - Positions are absolute token positions starting at 0. Key s is visible to a query at
+ *    position p iff s <= p.
+ *  - Output rows hold key positions (int32) in ascending candidate order (flat: ascending
+ *    position), padded with -1 when fewer than K keys are visible; the optional score
+ *    outputs hold the matching fp32 scores, padded with -inf. Ties at the K-th score are
+ *    broken towards the lower candidate index.
+ *  - Operands: bf16, or FP8-e4m3 codes (uint8) with one fp32 scale per token row (a query
+ *    token's scale covers all its heads). Score arithmetic is fp32 with fp32 tensor-core
+ *    accumulation.
+ */
+#ifndef ADX_H_
+#define ADX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ADX_ABI_VERSION 1
+#define ADX_STATUS_BYTES 256
+
+typedef enum {
+  ADX_OK = 0,
+  ADX_EINVAL = 1,        /* bad argument (null pointer, size or range) */
+  ADX_EUNSUPPORTED = 2,  /* shape/dtype combination without a compiled kernel */
+  ADX_EWORKSPACE = 3,    /* workspace too small (see adx_workspace_size) */
+  ADX_ECUDA = 4,         /* a CUDA runtime call or launch failed */
+  ADX_EOVERFLOW = 5,     /* an internal buffer would overflow */
+  ADX_ETIMEOUT = 6       /* a device-side bounded wait ran out (device status only) */
+} adx_status;
+
+typedef enum { ADX_BF16 = 0, ADX_E4M3 = 1 } adx_dtype;
+
+/* Readings of the shared bank (ADIndex §4.3). For a group whose first query sits at
+ * position a and whose members are a .. a+G-1:
+ *   ADX_BANK_PAPER  - the group query scans s <= a; the bank keeps the B best; member i adds
+ *                     the post-anchor positions a+1 .. i (Eqs. (13)-(14)). Bank width B+G-1.
+ *   ADX_BANK_WINDOW - the group query scans s < a; the bank keeps the B-G best plus the
+ *                     group's window a .. a+G-1; member i uses the bank entries <= i.
+ *                     Bank width B. */
+typedef enum { ADX_BANK_PAPER = 0, ADX_BANK_WINDOW = 1 } adx_bank_mode;
+
+typedef enum {
+  ADX_OP_PREFILL = 0,
+  ADX_OP_DECODE = 1,
+  ADX_OP_GROUP_BANK = 2,
+  ADX_OP_BANK_REFINE = 3
+} adx_op;
+
+/* One indexer operand set.
+ *
+ * Prefill layout (seq_len == NULL): T query rows at positions q_pos0 .. q_pos0+T-1 share
+ *   one key array k [S, d]; requires 0 <= q_pos0 and q_pos0 + T <= S.
+ * Decode layout (seq_len != NULL): row t owns key cache t of k [T, S, d] (S = capacity)
+ *   and sits at position seq_len[t] - 1; requires 1 <= seq_len[t] <= S (not checked on the
+ *   host: seq_len lives on the device).
+ *
+ * q        [T, H, d] row-major, bf16 or e4m3 codes (q_dtype)
+ * q_scale  [T] fp32, required iff q_dtype == ADX_E4M3
+ * w        [T, H] fp32 gates, any sign
+ * k        key rows of d elements, bf16 or e4m3 codes (k_dtype); 16-byte aligned
+ * k_scale  one fp32 per key row, required iff k_dtype == ADX_E4M3
+ * Supported: H in {4, 8, 16, 32, 64}; d = 128 (bf16 or e4m3) or d = 64 (bf16 only);
+ * q_dtype == k_dtype, except bf16 queries with an e4m3 key cache in the decode layout (the
+ * queries are then quantised to e4m3 per token inside the call). */
+typedef struct {
+  int32_t q_dtype;
+  int32_t k_dtype;
+  const void* q;
+  const float* q_scale;
+  const float* w;
+  const void* k;
+  const float* k_scale;
+  int32_t T, H, d, S;
+  int64_t q_pos0;
+  const int32_t* seq_len;
+} adx_operands;
+
+/* Bytes of workspace `op` needs for these operands (K: Top-K size; B, G, mode: bank
+ * parameters, ignored by the flat ops). Returns 0 for invalid or unsupported arguments. */
+size_t adx_workspace_size(int32_t op, const adx_operands* ops, int32_t K, int32_t B, int32_t G,
+                          int32_t mode);
+
+/* Columns of a bank row for (B, G, mode): B + G - 1 (PAPER) or B (WINDOW). */
+int32_t adx_bank_width(int32_t B, int32_t G, int32_t mode);
+
+/* Flat causal indexer over a prefix (ADIndex §3, Eqs. (1)-(2)); prefill layout.
+ * topk_idx    [T, K] int32 out
+ * topk_score  [T, K] fp32 out, or NULL
+ * scores_out  [T, scores_ld] fp32 out, or NULL: every score I[t, s] (s <= pos(t); -inf for
+ *             invisible keys up to the tile end). scores_ld >= S rounded up to 128.
+ * ws          workspace of ws_bytes >= adx_workspace_size(ADX_OP_PREFILL, ...) */
+adx_status adx_index_prefill(const adx_operands* ops, int32_t K, int32_t* topk_idx,
+                             float* topk_score, float* scores_out, int64_t scores_ld, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/* Flat indexer for one query per sequence against that sequence's key cache (§3,
+ * Eqs. (1)-(2), one decode step); decode layout. topk_idx [T, K], topk_score [T, K] or NULL. */
+adx_status adx_index_decode(const adx_operands* ops, int32_t K, int32_t* topk_idx,
+                            float* topk_score, void* ws, size_t ws_bytes, void* stream);
+
+/* Shared token banks (ADIndex §4.3, Eq. (13)); `grp` holds the group queries: q = q-bar
+ * [Ng, H_g, d], w = w-bar [Ng, H_g], with Ng = grp->T.
+ *  prefill layout: group g has members at positions q_pos0 + g*G .. q_pos0 + g*G + G-1.
+ *  decode layout:  group g is sequence g, refreshed at position seq_len[g]-1 and reused by
+ *                  the next G-1 decode steps; mode must be ADX_BANK_PAPER.
+ * bank_idx [Ng, adx_bank_width(B, G, mode)] int32 out: the scan's Top-B (PAPER) or Top-(B-G)
+ * (WINDOW) positions in ascending order, -1 padded when fewer keys were scanned, followed by
+ * the group's post-anchor positions (PAPER: a+1 .. a+G-1; WINDOW: a .. a+G-1). */
+adx_status adx_group_bank(const adx_operands* grp, int32_t G, int32_t B, int32_t mode,
+                          int32_t* bank_idx, void* ws, size_t ws_bytes, void* stream);
+
+/* Query-specific refinement (ADIndex §4.3, Eq. (14)) with the full indexer `full`.
+ *  prefill layout: the floor(T/G) complete groups use bank row g = row // G; the rows of an
+ *                  incomplete trailing group use the flat indexer (§4.3, "Application to
+ *                  Prefill and MTP").
+ *  decode layout:  row t uses bank row t; candidates are its bank entries <= seq_len[t]-1.
+ * bank_idx as written by adx_group_bank with the same (G, B, mode) and layout.
+ * topk_idx [T, K] out; topk_score [T, K] or NULL. */
+adx_status adx_bank_refine(const adx_operands* full, int32_t G, int32_t B, int32_t mode,
+                           const int32_t* bank_idx, int32_t K, int32_t* topk_idx,
+                           float* topk_score, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, returns the device status recorded in `ws` (ADX_OK if none) and
+ * clears it. */
+adx_status adx_read_device_status(void* ws, void* stream);
+
+/* Static description of a status code. */
+const char* adx_status_string(adx_status s);
+
+/* ADX_ABI_VERSION of the built library. */
+int32_t adx_abi_version(void);
+
+/* Instrumentation (no counterpart in the paper). When `events` (n cudaEvent_t handles,
+ * host array, owned by the caller) is set, later calls on this host thread record
+ * events[0] / events[1] on their stream right before / after each scoring-kernel launch and
+ * events[2] / events[3] before / after each Top-K selection; later records overwrite
+ * earlier ones. NULL switches it off. */
+void adx_set_timing_events(void* const* events, int32_t n);
+
+/* Number of kernels this library has launched in the process so far. */
+int64_t adx_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ADX_H_ */

@@ -1,0 +1,682 @@
+// C ABI of the indexer library: argument validation, workspace layout, TMA descriptors and
+// the launch sequence of each entry point. Every step of the computation runs in this
+// library's kernels; this file only plans and launches them.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/adx.h"
+#include "adx_internal.h"
+
+namespace adx {
+namespace {
+
+constexpr size_t kAlign = 256;
+
+// Optional instrumentation (adx_set_timing_events / adx_launch_count).
+thread_local void* const* g_events = nullptr;
+thread_local int g_n_events = 0;
+std::atomic<long long> g_launches{0};
+
+void mark(int i, cudaStream_t s) {
+  if (g_events != nullptr && i < g_n_events && g_events[i] != nullptr)
+    cudaEventRecord(static_cast<cudaEvent_t>(g_events[i]), s);
+}
+
+cudaError_t counted(cudaError_t e, int n = 1) {
+  if (e == cudaSuccess) g_launches += n;
+  return e;
+}
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per device-side wait
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int64_t ld_for(int64_t n) { return (n + kTileM - 1) / kTileM * kTileM; }
+
+struct Carve {
+  uint8_t* base;
+  size_t off = 0;
+  explicit Carve(void* p) : base(static_cast<uint8_t*>(p)) {}
+  template <class T>
+  T* take(size_t bytes) {
+    T* p = reinterpret_cast<T*>(base ? base + off : nullptr);
+    off += align_up(bytes, kAlign);
+    return p;
+  }
+};
+
+// ------------------------------------------------------------------------------------
+// device properties and the driver's tensor-map encoder
+// ------------------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encoder() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  static int cache[64] = {0};
+  if (dev < 0 || dev >= 64) return 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// 2-D map over `rows` rows of `d` elements (1 or 2 bytes), 128-byte swizzled boxes of
+// (128 bytes) x box_rows.
+bool encode_rows(CUtensorMap* m, const void* base, bool one_byte, int d, int64_t rows,
+                 int box_rows) {
+  EncodeTiledFn enc = encoder();
+  if (!enc || rows <= 0 || rows > INT32_MAX) return false;
+  if (reinterpret_cast<uintptr_t>(base) % 16 != 0) return false;
+  const int esz = one_byte ? 1 : 2;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * esz};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esz), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, one_byte ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+             const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------------------------
+// validation
+// ------------------------------------------------------------------------------------
+adx_status check_operands(const adx_operands* o, bool decode) {
+  if (!o || !o->q || !o->w || !o->k) return ADX_EINVAL;
+  if (o->T <= 0 || o->H <= 0 || o->d <= 0 || o->S <= 0) return ADX_EINVAL;
+  if ((o->q_dtype != ADX_BF16 && o->q_dtype != ADX_E4M3) ||
+      (o->k_dtype != ADX_BF16 && o->k_dtype != ADX_E4M3))
+    return ADX_EINVAL;
+  if ((o->q_dtype == ADX_E4M3) != (o->q_scale != nullptr)) return ADX_EINVAL;
+  if ((o->k_dtype == ADX_E4M3) != (o->k_scale != nullptr)) return ADX_EINVAL;
+  if (decode != (o->seq_len != nullptr)) return ADX_EINVAL;
+  if (!decode && (o->q_pos0 < 0 || o->q_pos0 + o->T > o->S)) return ADX_EINVAL;
+  if (o->q_dtype != o->k_dtype && !(decode && o->q_dtype == ADX_BF16 && o->k_dtype == ADX_E4M3))
+    return ADX_EUNSUPPORTED;
+  if (!score_config_supported(o->k_dtype == ADX_E4M3, o->H, o->d)) return ADX_EUNSUPPORTED;
+  if (static_cast<int64_t>(o->T) * o->H > INT32_MAX) return ADX_EINVAL;
+  if (decode && static_cast<int64_t>(o->T) * o->S > INT32_MAX) return ADX_EINVAL;
+  return ADX_OK;
+}
+
+bool fp8_keys(const adx_operands* o) { return o->k_dtype == ADX_E4M3; }
+int row_bytes(const adx_operands* o) { return o->d * (fp8_keys(o) ? 1 : 2); }
+bool quantise_q(const adx_operands* o) { return o->q_dtype == ADX_BF16 && o->k_dtype == ADX_E4M3; }
+
+// split of a long row into segments for a two-stage select (few long rows)
+void plan_split(int64_t rows, int64_t n, int K, int& n_seg, int& seg_len) {
+  n_seg = 1;
+  seg_len = static_cast<int>(std::min<int64_t>(n, INT32_MAX));
+  const int sms = std::max(sm_count(), 1);
+  if (rows >= sms || n < 8ll * K) return;
+  const int64_t want = (2ll * sms + rows - 1) / rows;
+  const int64_t most = n / (4ll * K);
+  n_seg = static_cast<int>(std::max<int64_t>(1, std::min(want, most)));
+  if (n_seg == 1) return;
+  seg_len = static_cast<int>(align_up((n + n_seg - 1) / n_seg, 4));
+  n_seg = static_cast<int>((n + seg_len - 1) / seg_len);
+}
+
+// ------------------------------------------------------------------------------------
+// building blocks
+// ------------------------------------------------------------------------------------
+struct ScorePlan {
+  ScoreArgs a{};
+  bool fp8 = false;
+  int H = 0, d = 0, tok = 0;
+};
+
+// Chooses the key-chunk size and the persistent grid for a score launch.
+void finish_plan(ScorePlan& p, int64_t max_tiles_per_block) {
+  const int bps = score_blocks_per_sm(p.fp8, p.H, p.d, p.tok);
+  const int grid_cap = std::max(1, sm_count() * std::max(bps, 1));
+  const int64_t blocks = static_cast<int64_t>(p.a.row_blocks_per_batch) * p.a.n_batches;
+  // aim for >= 4 items per CTA, chunks of 8..32 tiles
+  int64_t chunk = max_tiles_per_block;
+  const int64_t want_items = 4ll * grid_cap;
+  if (blocks * ((max_tiles_per_block + chunk - 1) / chunk) < want_items)
+    chunk = std::max<int64_t>(8, (blocks * max_tiles_per_block + want_items - 1) / want_items);
+  chunk = std::min<int64_t>(chunk, 32);
+  chunk = std::max<int64_t>(1, std::min(chunk, max_tiles_per_block));
+  p.a.chunk_tiles = static_cast<int>(chunk);
+  p.a.chunks_per_block = static_cast<int>((max_tiles_per_block + chunk - 1) / chunk);
+  p.a.n_items = static_cast<int>(blocks * p.a.chunks_per_block);
+}
+
+adx_status run_score(const ScorePlan& p, const void* q_codes, const void* keys, int64_t key_rows,
+                     cudaStream_t s) {
+  CUtensorMap tq, tk;
+  const int n = p.tok * p.H;
+  if (!encode_rows(&tq, q_codes, p.fp8, p.d, static_cast<int64_t>(p.a.R) * p.H, n))
+    return ADX_EINVAL;
+  if (!encode_rows(&tk, keys, p.fp8, p.d, key_rows, kTileM)) return ADX_EINVAL;
+  if (p.a.n_items <= 0) return ADX_OK;
+  const int bps = score_blocks_per_sm(p.fp8, p.H, p.d, p.tok);
+  const int grid = std::min<int64_t>(p.a.n_items, static_cast<int64_t>(sm_count()) * bps);
+  if (grid <= 0) return ADX_EUNSUPPORTED;
+  mark(0, s);
+  const cudaError_t e = counted(launch_score(tq, tk, p.a, p.fp8, p.H, p.d, p.tok, grid, s));
+  mark(1, s);
+  if (e == cudaErrorNotSupported) return ADX_EUNSUPPORTED;
+  return e == cudaSuccess ? ADX_OK : ADX_ECUDA;
+}
+
+size_t select_scratch_bytes(int64_t rows, int64_t n, int K) {
+  int n_seg, seg_len;
+  plan_split(rows, n, K, n_seg, seg_len);
+  if (n_seg == 1) return 0;
+  const size_t c = static_cast<size_t>(rows) * n_seg * K;
+  return align_up(c * 4, kAlign) * 2;
+}
+
+// Top-K per row of a score matrix, split into two stages when there are few long rows.
+adx_status run_select(SelectArgs a, int64_t n_max, Carve& cv, DeviceStatus* st, cudaStream_t s) {
+  a.status = st;
+  int n_seg, seg_len;
+  plan_split(a.rows, n_max, a.K, n_seg, seg_len);
+  mark(2, s);
+  if (n_seg == 1) {
+    a.n_seg = 1;
+    a.seg_len = static_cast<int32_t>(std::min<int64_t>(n_max, INT32_MAX));
+    const cudaError_t e = counted(launch_select(a, s));
+    mark(3, s);
+    return e == cudaSuccess ? ADX_OK : ADX_ECUDA;
+  }
+  const size_t c = static_cast<size_t>(a.rows) * n_seg * a.K;
+  float* cv_val = cv.take<float>(c * 4);
+  int32_t* cv_idx = cv.take<int32_t>(c * 4);
+  SelectArgs s1 = a;
+  s1.n_seg = n_seg;
+  s1.seg_len = seg_len;
+  s1.idx_map = nullptr;
+  s1.out_idx = cv_idx;
+  s1.out_val = cv_val;
+  s1.out_ld = a.K;
+  if (counted(launch_select(s1, s)) != cudaSuccess) return ADX_ECUDA;
+  SelectArgs s2 = a;
+  s2.vals = cv_val;
+  s2.in_idx = cv_idx;
+  s2.ld = static_cast<int64_t>(n_seg) * a.K;
+  s2.len_mode = 0;
+  s2.len_fixed = static_cast<int32_t>(s2.ld);
+  s2.len_cap = s2.len_fixed;
+  s2.n_seg = 1;
+  s2.seg_len = s2.len_fixed;
+  const cudaError_t e = counted(launch_select(s2, s));
+  mark(3, s);
+  return e == cudaSuccess ? ADX_OK : ADX_ECUDA;
+}
+
+// ---- flat prefill ------------------------------------------------------------------
+size_t ws_flat(const adx_operands* o, int K, bool scores_external) {
+  size_t b = kStatusBytes;
+  if (!scores_external) b += align_up(static_cast<size_t>(o->T) * ld_for(o->S) * 4, kAlign);
+  b += select_scratch_bytes(o->T, o->S, K);
+  return b;
+}
+
+adx_status run_flat(const adx_operands* o, int K, int32_t* topk_idx, float* topk_score,
+                    float* scores_ext, int64_t scores_ld, Carve& cv, DeviceStatus* st,
+                    cudaStream_t s) {
+  const bool fp8 = fp8_keys(o);
+  const int64_t ld = scores_ext ? scores_ld : ld_for(o->S);
+  float* scores = scores_ext ? scores_ext : cv.take<float>(static_cast<size_t>(o->T) * ld * 4);
+  ScorePlan p;
+  p.fp8 = fp8;
+  p.H = o->H;
+  p.d = o->d;
+  p.tok = score_tokens_per_tile(o->H);
+  ScoreArgs& a = p.a;
+  a.w = o->w;
+  a.q_scale = o->q_scale;
+  a.k_scale = o->k_scale;
+  a.scores = scores;
+  a.score_ld = ld;
+  a.pos_base = o->q_pos0;
+  a.pos_step = 1;
+  a.R = o->T;
+  a.rows_per_batch = o->T;
+  a.n_batches = 1;
+  a.key_batch_stride = 0;
+  a.keys_per_batch = o->S;
+  a.row_blocks_per_batch = (o->T + p.tok - 1) / p.tok;
+  a.reverse_order = 1;
+  a.status = st;
+  a.timeout_ns = kTimeoutNs;
+  const int64_t max_keys = std::min<int64_t>(o->S, o->q_pos0 + o->T);
+  finish_plan(p, (max_keys + kTileM - 1) / kTileM);
+  adx_status r = run_score(p, o->q, o->k, o->S, s);
+  if (r != ADX_OK) return r;
+  SelectArgs sa{};
+  sa.vals = scores;
+  sa.ld = ld;
+  sa.rows_per_batch = o->T;
+  sa.len_mode = 1;
+  sa.len_cap = o->S;
+  sa.pos_base = o->q_pos0;
+  sa.pos_step = 1;
+  sa.K = K;
+  sa.out_idx = topk_idx;
+  sa.out_val = topk_score;
+  sa.out_ld = K;
+  sa.rows = o->T;
+  return run_select(sa, max_keys, cv, st, s);
+}
+
+// ---- decode-layout scoring (one query per key cache) --------------------------------
+size_t ws_rowwise_q8(const adx_operands* o) {
+  if (!quantise_q(o)) return 0;
+  return align_up(static_cast<size_t>(o->T) * o->H * o->d, kAlign) +
+         align_up(static_cast<size_t>(o->T) * 4, kAlign);
+}
+
+// Quantises bf16 queries when the keys are e4m3; returns the query codes/scales to use.
+adx_status prepare_q(const adx_operands* o, Carve& cv, const void*& q, const float*& q_scale,
+                     cudaStream_t s) {
+  q = o->q;
+  q_scale = o->q_scale;
+  if (!quantise_q(o)) return ADX_OK;
+  uint8_t* codes = cv.take<uint8_t>(static_cast<size_t>(o->T) * o->H * o->d);
+  float* sc = cv.take<float>(static_cast<size_t>(o->T) * 4);
+  if (counted(launch_quantize_rows_e4m3(static_cast<const uint16_t*>(o->q), o->T,
+                                        static_cast<int64_t>(o->H) * o->d, codes, sc, s)) !=
+      cudaSuccess)
+    return ADX_ECUDA;
+  q = codes;
+  q_scale = sc;
+  return ADX_OK;
+}
+
+ScorePlan rowwise_plan(const adx_operands* o, const float* q_scale, float* scores, int64_t ld) {
+  ScorePlan p;
+  p.fp8 = fp8_keys(o);
+  p.H = o->H;
+  p.d = o->d;
+  p.tok = 1;
+  ScoreArgs& a = p.a;
+  a.w = o->w;
+  a.q_scale = q_scale;
+  a.k_scale = o->k_scale;
+  a.seq_len = o->seq_len;
+  a.scores = scores;
+  a.score_ld = ld;
+  a.R = o->T;
+  a.rows_per_batch = 1;
+  a.n_batches = o->T;
+  a.key_batch_stride = o->S;
+  a.keys_per_batch = o->S;
+  a.row_blocks_per_batch = 1;
+  a.timeout_ns = kTimeoutNs;
+  return p;
+}
+
+size_t ws_decode(const adx_operands* o, int K) {
+  return kStatusBytes + ws_rowwise_q8(o) +
+         align_up(static_cast<size_t>(o->T) * ld_for(o->S) * 4, kAlign) +
+         select_scratch_bytes(o->T, o->S, K);
+}
+
+// ---- group bank ---------------------------------------------------------------------
+struct BankShape {
+  int bank_k, post_count, post_start_off, width;
+  int64_t scan_pos_off;  // scan row position = anchor + scan_pos_off
+};
+
+BankShape bank_shape(int B, int G, int mode) {
+  BankShape b{};
+  if (mode == ADX_BANK_PAPER) {
+    b.bank_k = B;
+    b.post_count = G - 1;
+    b.post_start_off = 1;
+    b.scan_pos_off = 0;
+  } else {
+    b.bank_k = B - G;
+    b.post_count = G;
+    b.post_start_off = 0;
+    b.scan_pos_off = -1;
+  }
+  b.width = b.bank_k + b.post_count;
+  return b;
+}
+
+adx_status check_bank_args(const adx_operands* o, int G, int B, int mode) {
+  if (G <= 0 || B <= 0) return ADX_EINVAL;
+  if (mode != ADX_BANK_PAPER && mode != ADX_BANK_WINDOW) return ADX_EINVAL;
+  if (mode == ADX_BANK_WINDOW && B <= G) return ADX_EINVAL;
+  if (o->seq_len != nullptr && mode != ADX_BANK_PAPER) return ADX_EUNSUPPORTED;
+  return ADX_OK;
+}
+
+size_t ws_bank(const adx_operands* o, int G, int B, int mode) {
+  const BankShape bs = bank_shape(B, G, mode);
+  return kStatusBytes + ws_rowwise_q8(o) +
+         align_up(static_cast<size_t>(o->T) * ld_for(o->S) * 4, kAlign) +
+         select_scratch_bytes(o->T, o->S, bs.bank_k);
+}
+
+// ---- refine -------------------------------------------------------------------------
+size_t ws_refine(const adx_operands* o, int G, int B, int mode, int K) {
+  const BankShape bs = bank_shape(B, G, mode);
+  const int64_t bcp = ld_for(bs.width);
+  const bool dec = o->seq_len != nullptr;
+  const int64_t ng = dec ? o->T : o->T / G;
+  const int64_t rows = dec ? o->T : ng * G;
+  size_t b = kStatusBytes + ws_rowwise_q8(o);
+  b += align_up(static_cast<size_t>(ng) * bcp * row_bytes(o), kAlign);  // packed keys
+  b += align_up(static_cast<size_t>(ng) * bcp * 4, kAlign) * 2;          // scales, positions
+  b += align_up(static_cast<size_t>(rows) * bcp * 4, kAlign);             // scores
+  b += select_scratch_bytes(rows, bcp, K);
+  if (!dec && rows < o->T) {
+    adx_operands tail = *o;
+    tail.T = static_cast<int32_t>(o->T - rows);
+    b += ws_flat(&tail, K, false) - kStatusBytes;
+  }
+  return b;
+}
+
+}  // namespace
+}  // namespace adx
+
+using namespace adx;
+
+extern "C" {
+
+int32_t adx_abi_version(void) { return ADX_ABI_VERSION; }
+
+void adx_set_timing_events(void* const* events, int32_t n) {
+  g_events = (events != nullptr && n > 0) ? events : nullptr;
+  g_n_events = g_events ? n : 0;
+}
+
+int64_t adx_launch_count(void) { return g_launches.load(); }
+
+int32_t adx_bank_width(int32_t B, int32_t G, int32_t mode) {
+  if (B <= 0 || G <= 0 || (mode != ADX_BANK_PAPER && mode != ADX_BANK_WINDOW)) return 0;
+  if (mode == ADX_BANK_WINDOW && B <= G) return 0;
+  return bank_shape(B, G, mode).width;
+}
+
+const char* adx_status_string(adx_status s) {
+  switch (s) {
+    case ADX_OK: return "ok";
+    case ADX_EINVAL: return "invalid argument";
+    case ADX_EUNSUPPORTED: return "unsupported shape or dtype";
+    case ADX_EWORKSPACE: return "workspace too small";
+    case ADX_ECUDA: return "CUDA error";
+    case ADX_EOVERFLOW: return "internal buffer overflow";
+    case ADX_ETIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+size_t adx_workspace_size(int32_t op, const adx_operands* ops, int32_t K, int32_t B, int32_t G,
+                          int32_t mode) {
+  if (!ops) return 0;
+  switch (op) {
+    case ADX_OP_PREFILL:
+      if (K <= 0 || check_operands(ops, false) != ADX_OK) return 0;
+      return ws_flat(ops, K, false);
+    case ADX_OP_DECODE:
+      if (K <= 0 || check_operands(ops, true) != ADX_OK) return 0;
+      return ws_decode(ops, K);
+    case ADX_OP_GROUP_BANK:
+      if (check_operands(ops, ops->seq_len != nullptr) != ADX_OK ||
+          check_bank_args(ops, G, B, mode) != ADX_OK)
+        return 0;
+      return ws_bank(ops, G, B, mode);
+    case ADX_OP_BANK_REFINE:
+      if (K <= 0 || check_operands(ops, ops->seq_len != nullptr) != ADX_OK ||
+          check_bank_args(ops, G, B, mode) != ADX_OK)
+        return 0;
+      return ws_refine(ops, G, B, mode, K);
+    default:
+      return 0;
+  }
+}
+
+adx_status adx_index_prefill(const adx_operands* o, int32_t K, int32_t* topk_idx,
+                             float* topk_score, float* scores_out, int64_t scores_ld, void* ws,
+                             size_t ws_bytes, void* stream) {
+  adx_status r = check_operands(o, false);
+  if (r != ADX_OK) return r;
+  if (K <= 0 || !topk_idx || !ws) return ADX_EINVAL;
+  if (scores_out && scores_ld < ld_for(o->S)) return ADX_EINVAL;
+  if (ws_bytes < ws_flat(o, K, scores_out != nullptr)) return ADX_EWORKSPACE;
+  Carve cv(ws);
+  DeviceStatus* st = cv.take<DeviceStatus>(kStatusBytes);
+  return run_flat(o, K, topk_idx, topk_score, scores_out, scores_ld, cv, st,
+                  static_cast<cudaStream_t>(stream));
+}
+
+adx_status adx_index_decode(const adx_operands* o, int32_t K, int32_t* topk_idx,
+                            float* topk_score, void* ws, size_t ws_bytes, void* stream) {
+  adx_status r = check_operands(o, true);
+  if (r != ADX_OK) return r;
+  if (K <= 0 || !topk_idx || !ws) return ADX_EINVAL;
+  if (ws_bytes < ws_decode(o, K)) return ADX_EWORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Carve cv(ws);
+  DeviceStatus* st = cv.take<DeviceStatus>(kStatusBytes);
+  const void* q;
+  const float* q_scale;
+  if ((r = prepare_q(o, cv, q, q_scale, s)) != ADX_OK) return r;
+  const int64_t ld = ld_for(o->S);
+  float* scores = cv.take<float>(static_cast<size_t>(o->T) * ld * 4);
+  ScorePlan p = rowwise_plan(o, q_scale, scores, ld);
+  p.a.status = st;
+  finish_plan(p, (o->S + kTileM - 1) / kTileM);
+  if ((r = run_score(p, q, o->k, static_cast<int64_t>(o->T) * o->S, s)) != ADX_OK) return r;
+  SelectArgs sa{};
+  sa.vals = scores;
+  sa.ld = ld;
+  sa.rows_per_batch = 1;
+  sa.len_mode = 2;
+  sa.len_cap = o->S;
+  sa.seq_len = o->seq_len;
+  sa.K = K;
+  sa.out_idx = topk_idx;
+  sa.out_val = topk_score;
+  sa.out_ld = K;
+  sa.rows = o->T;
+  return run_select(sa, o->S, cv, st, s);
+}
+
+adx_status adx_group_bank(const adx_operands* o, int32_t G, int32_t B, int32_t mode,
+                          int32_t* bank_idx, void* ws, size_t ws_bytes, void* stream) {
+  if (!o) return ADX_EINVAL;
+  const bool dec = o->seq_len != nullptr;
+  adx_status r = check_operands(o, dec);
+  if (r != ADX_OK) return r;
+  if ((r = check_bank_args(o, G, B, mode)) != ADX_OK) return r;
+  if (!bank_idx || !ws) return ADX_EINVAL;
+  if (ws_bytes < ws_bank(o, G, B, mode)) return ADX_EWORKSPACE;
+  if (!dec && o->q_pos0 + static_cast<int64_t>(o->T - 1) * G >= o->S) return ADX_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const BankShape bs = bank_shape(B, G, mode);
+  Carve cv(ws);
+  DeviceStatus* st = cv.take<DeviceStatus>(kStatusBytes);
+  const int64_t ld = ld_for(o->S);
+  SelectArgs sa{};
+  if (dec) {
+    const void* q;
+    const float* q_scale;
+    if ((r = prepare_q(o, cv, q, q_scale, s)) != ADX_OK) return r;
+    float* scores = cv.take<float>(static_cast<size_t>(o->T) * ld * 4);
+    ScorePlan p = rowwise_plan(o, q_scale, scores, ld);
+    p.a.status = st;
+    finish_plan(p, (o->S + kTileM - 1) / kTileM);
+    if ((r = run_score(p, q, o->k, static_cast<int64_t>(o->T) * o->S, s)) != ADX_OK) return r;
+    sa.vals = scores;
+    sa.len_mode = 2;
+    sa.seq_len = o->seq_len;
+  } else {
+    float* scores = cv.take<float>(static_cast<size_t>(o->T) * ld * 4);
+    ScorePlan p;
+    p.fp8 = fp8_keys(o);
+    p.H = o->H;
+    p.d = o->d;
+    p.tok = score_tokens_per_tile(o->H);
+    ScoreArgs& a = p.a;
+    a.w = o->w;
+    a.q_scale = o->q_scale;
+    a.k_scale = o->k_scale;
+    a.scores = scores;
+    a.score_ld = ld;
+    a.pos_base = o->q_pos0 + bs.scan_pos_off;
+    a.pos_step = G;
+    a.R = o->T;
+    a.rows_per_batch = o->T;
+    a.n_batches = 1;
+    a.keys_per_batch = o->S;
+    a.row_blocks_per_batch = (o->T + p.tok - 1) / p.tok;
+    a.reverse_order = 1;
+    a.status = st;
+    a.timeout_ns = kTimeoutNs;
+    const int64_t last = o->q_pos0 + bs.scan_pos_off + static_cast<int64_t>(o->T - 1) * G;
+    const int64_t max_keys = std::max<int64_t>(0, std::min<int64_t>(o->S, last + 1));
+    finish_plan(p, std::max<int64_t>(1, (max_keys + kTileM - 1) / kTileM));
+    if ((r = run_score(p, o->q, o->k, o->S, s)) != ADX_OK) return r;
+    sa.vals = scores;
+    sa.len_mode = 1;
+    sa.pos_base = o->q_pos0 + bs.scan_pos_off;
+    sa.pos_step = G;
+  }
+  sa.ld = ld;
+  sa.rows_per_batch = 1;
+  sa.len_cap = o->S;
+  sa.K = bs.bank_k;
+  sa.out_idx = bank_idx;
+  sa.out_ld = bs.width;
+  sa.rows = o->T;
+  if ((r = run_select(sa, o->S, cv, st, s)) != ADX_OK) return r;
+  if (counted(launch_fill_post_anchor(bank_idx, o->T, bs.width, bs.bank_k, bs.post_count,
+                                      o->q_pos0, G, o->seq_len, bs.post_start_off, s)) !=
+      cudaSuccess)
+    return ADX_ECUDA;
+  return ADX_OK;
+}
+
+adx_status adx_bank_refine(const adx_operands* o, int32_t G, int32_t B, int32_t mode,
+                           const int32_t* bank_idx, int32_t K, int32_t* topk_idx,
+                           float* topk_score, void* ws, size_t ws_bytes, void* stream) {
+  if (!o) return ADX_EINVAL;
+  const bool dec = o->seq_len != nullptr;
+  adx_status r = check_operands(o, dec);
+  if (r != ADX_OK) return r;
+  if ((r = check_bank_args(o, G, B, mode)) != ADX_OK) return r;
+  if (K <= 0 || !bank_idx || !topk_idx || !ws) return ADX_EINVAL;
+  if (ws_bytes < ws_refine(o, G, B, mode, K)) return ADX_EWORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const BankShape bs = bank_shape(B, G, mode);
+  const int64_t bcp = ld_for(bs.width);
+  const int64_t ng = dec ? o->T : o->T / G;
+  const int64_t rows = dec ? o->T : ng * G;
+  if (ng * bcp > INT32_MAX) return ADX_EINVAL;
+  Carve cv(ws);
+  DeviceStatus* st = cv.take<DeviceStatus>(kStatusBytes);
+  const void* q;
+  const float* q_scale;
+  if ((r = prepare_q(o, cv, q, q_scale, s)) != ADX_OK) return r;
+  if (rows > 0) {
+    const int rb = row_bytes(o);
+    uint8_t* packed = cv.take<uint8_t>(static_cast<size_t>(ng) * bcp * rb);
+    float* pscale = cv.take<float>(static_cast<size_t>(ng) * bcp * 4);
+    int32_t* ppos = cv.take<int32_t>(static_cast<size_t>(ng) * bcp * 4);
+    float* scores = cv.take<float>(static_cast<size_t>(rows) * bcp * 4);
+    if (counted(launch_pack_candidates(o->k, o->k_scale, o->S, dec ? 1 : 0, o->S, bank_idx,
+                               static_cast<int32_t>(ng), bs.width, static_cast<int32_t>(bcp), rb,
+                               packed, fp8_keys(o) ? pscale : nullptr, ppos, s)) != cudaSuccess)
+      return ADX_ECUDA;
+    ScorePlan p;
+    if (dec) {
+      p = rowwise_plan(o, q_scale, scores, bcp);
+    } else {
+      p.fp8 = fp8_keys(o);
+      p.H = o->H;
+      p.d = o->d;
+      p.tok = score_tokens_per_tile(o->H);
+      p.a.w = o->w;
+      p.a.q_scale = q_scale;
+      p.a.scores = scores;
+      p.a.score_ld = bcp;
+      p.a.pos_base = o->q_pos0;
+      p.a.pos_step = 1;
+      p.a.R = static_cast<int32_t>(rows);
+      p.a.rows_per_batch = G;
+      p.a.n_batches = static_cast<int32_t>(ng);
+      p.a.row_blocks_per_batch = (G + p.tok - 1) / p.tok;
+      p.a.timeout_ns = kTimeoutNs;
+    }
+    p.a.k_scale = fp8_keys(o) ? pscale : nullptr;
+    p.a.key_pos = ppos;
+    p.a.key_batch_stride = bcp;
+    p.a.keys_per_batch = static_cast<int32_t>(bcp);
+    p.a.status = st;
+    finish_plan(p, bcp / kTileM);
+    if ((r = run_score(p, q, packed, ng * bcp, s)) != ADX_OK) return r;
+    SelectArgs sa{};
+    sa.vals = scores;
+    sa.ld = bcp;
+    sa.idx_map = ppos;
+    sa.map_stride = bcp;
+    sa.rows_per_batch = dec ? 1 : G;
+    sa.len_mode = 0;
+    sa.len_fixed = static_cast<int32_t>(bcp);
+    sa.len_cap = static_cast<int32_t>(bcp);
+    sa.K = K;
+    sa.out_idx = topk_idx;
+    sa.out_val = topk_score;
+    sa.out_ld = K;
+    sa.rows = static_cast<int32_t>(rows);
+    if ((r = run_select(sa, bcp, cv, st, s)) != ADX_OK) return r;
+  }
+  if (!dec && rows < o->T) {
+    // incomplete trailing group: the plain indexer on those rows
+    adx_operands tail = *o;
+    tail.T = static_cast<int32_t>(o->T - rows);
+    tail.q = static_cast<const uint8_t*>(o->q) +
+             rows * o->H * o->d * (o->q_dtype == ADX_E4M3 ? 1 : 2);
+    tail.q_scale = o->q_scale ? o->q_scale + rows : nullptr;
+    tail.w = o->w + rows * o->H;
+    tail.q_pos0 = o->q_pos0 + rows;
+    return run_flat(&tail, K, topk_idx + rows * K, topk_score ? topk_score + rows * K : nullptr,
+                    nullptr, 0, cv, st, s);
+  }
+  return ADX_OK;
+}
+
+adx_status adx_read_device_status(void* ws, void* stream) {
+  if (!ws) return ADX_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ADX_ECUDA;
+  DeviceStatus h{};
+  if (cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return ADX_ECUDA;
+  if (cudaMemset(ws, 0, sizeof(h)) != cudaSuccess) return ADX_ECUDA;
+  return static_cast<adx_status>(h.code);
+}
+
+}  // extern "C"

@@ -1,0 +1,99 @@
+// Internal declarations shared by the library's translation units (not part of the ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace adx {
+
+// Device status word at the start of every workspace (sticky until read).
+struct DeviceStatus {
+  int32_t code;    // 0 = ok, otherwise an adx_status value
+  int32_t where;   // which kernel raised it
+  int32_t info0;
+  int32_t info1;
+};
+constexpr size_t kStatusBytes = 256;
+constexpr int kWhereScore = 1;
+constexpr int kWhereSelect = 2;
+
+constexpr int kTileM = 128;  // keys per MMA tile (TMEM lanes)
+
+// Work decomposition and epilogue parameters of the scoring kernel.
+//
+// Query rows r = 0..R-1 are split into batches of rows_per_batch rows; every batch owns a
+// key range of keys_per_batch rows in the key tensor map, starting at row
+// b * key_batch_stride. The position of row r is seq_len[b] - 1 when seq_len is given
+// (decode), else pos_base + r * pos_step. Key c of batch b sits at position key_pos[...]
+// when key_pos is given (packed candidate lists), else at position c.
+struct ScoreArgs {
+  const float* w;          // [R, H] gates
+  const float* q_scale;    // [R] or null
+  const float* k_scale;    // [n_batches * key_batch_stride] or null
+  const int32_t* key_pos;  // [n_batches * key_batch_stride] or null
+  const int32_t* seq_len;  // [n_batches] or null
+  float* scores;           // [R, score_ld]
+  int64_t score_ld;
+  int64_t pos_base;
+  int32_t pos_step;
+  int32_t R;
+  int32_t rows_per_batch;
+  int32_t n_batches;
+  int64_t key_batch_stride;
+  int32_t keys_per_batch;
+  int32_t row_blocks_per_batch;
+  int32_t chunks_per_block;
+  int32_t chunk_tiles;
+  int32_t n_items;
+  int32_t reverse_order;
+  DeviceStatus* status;
+  uint64_t timeout_ns;
+};
+
+// Row-wise Top-K over a score matrix (radix select).
+struct SelectArgs {
+  const float* vals;       // [rows, ld]
+  int64_t ld;
+  const int32_t* in_idx;   // [rows, ld] element ids (second stage of a split select) or null
+  const int32_t* idx_map;  // position of element c of row r: idx_map[(r / rows_per_batch) * map_stride + c], or null
+  int64_t map_stride;
+  int32_t rows_per_batch;
+  // row length: len_mode 0 -> fixed len_fixed; 1 -> min(len_cap, pos_base + r*pos_step + 1);
+  //             2 -> min(len_cap, seq_len[r / rows_per_batch])
+  int32_t len_mode;
+  int32_t len_fixed;
+  int32_t len_cap;
+  int64_t pos_base;
+  int32_t pos_step;
+  const int32_t* seq_len;
+  int32_t K;
+  int32_t n_seg;           // split each row into n_seg segments of seg_len (first stage)
+  int32_t seg_len;
+  int32_t* out_idx;        // [rows * n_seg, out_ld]
+  float* out_val;          // same layout, or null
+  int64_t out_ld;
+  int32_t rows;
+  DeviceStatus* status;
+};
+
+// Launchers (return a cudaError_t from the launch).
+cudaError_t launch_score(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const ScoreArgs& a,
+                         bool fp8, int H, int d, int tok, int grid, cudaStream_t s);
+int score_tokens_per_tile(int H);  // tokens per N tile for a head count (0 = unsupported)
+bool score_config_supported(bool fp8, int H, int d);
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t s);
+cudaError_t launch_quantize_rows_e4m3(const uint16_t* x_bf16, int64_t rows, int64_t cols,
+                                      uint8_t* codes, float* scale, cudaStream_t s);
+cudaError_t launch_pack_candidates(const void* k, const float* k_scale, int64_t key_batch_stride,
+                                   int32_t per_group_keys, int32_t S_valid, const int32_t* cand,
+                                   int32_t n_groups, int32_t n_cand, int32_t n_cand_pad,
+                                   int32_t row_bytes, void* packed, float* packed_scale,
+                                   int32_t* packed_pos, cudaStream_t s);
+cudaError_t launch_fill_post_anchor(int32_t* bank, int32_t n_groups, int32_t bank_w,
+                                    int32_t first_col, int32_t count, int64_t pos_base,
+                                    int32_t pos_step, const int32_t* seq_len, int32_t start_off,
+                                    cudaStream_t s);
+int score_blocks_per_sm(bool fp8, int H, int d, int tok);
+
+}  // namespace adx

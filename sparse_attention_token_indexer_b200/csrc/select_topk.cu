@@ -1,0 +1,215 @@
+// Row-wise Top-K selection (ADIndex, arXiv 2611.12956v1, §3 Eq. (2), and the bank Top-P
+// of Eq. (13)) as an exact radix select.
+//
+// Each CTA owns one row (or one segment of a row, for the first stage of a split select).
+// Scores are mapped to order-preserving 32-bit keys; the K-th largest key is found digit by
+// digit (12 + 12 + 8 bits) with shared-memory histograms, and a last pass writes every
+// element above the threshold plus the lowest-indexed elements equal to it, in index order,
+// using block-wide prefix sums (warp shuffles) for the output slots. -inf marks a masked
+// (invisible) key and NaN is treated the same way: neither is ever selected. Rows with fewer
+// than K valid elements return all of them, padded with index -1 and score -inf.
+#include <cstdint>
+
+#include "adx_internal.h"
+
+namespace adx {
+
+namespace {
+
+constexpr int kSelThreads = 512;
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kBins = 4096;
+
+__device__ __forceinline__ uint32_t order_key(float v) {
+  const uint32_t b = __float_as_uint(v);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ bool is_valid(float v) { return !(v != v) && v != -INFINITY; }
+
+// Inclusive prefix sum over the block (all threads participate); also returns the total.
+__device__ __forceinline__ uint32_t block_inclusive_scan(uint32_t x, uint32_t* warp_tot,
+                                                         uint32_t& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t t = lane < kSelWarps ? warp_tot[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    if (lane < kSelWarps) warp_tot[lane] = t;  // inclusive warp prefix
+  }
+  __syncthreads();
+  const uint32_t before = warp == 0 ? 0u : warp_tot[warp - 1];
+  total = warp_tot[kSelWarps - 1];
+  __syncthreads();  // warp_tot may be reused right after
+  return x + before;
+}
+
+struct RowInfo {
+  int64_t lo, hi;  // element range of this CTA
+};
+
+__device__ __forceinline__ int64_t row_length(const SelectArgs& a, int r) {
+  int64_t n;
+  if (a.len_mode == 0) {
+    n = a.len_fixed;
+  } else if (a.len_mode == 1) {
+    n = a.pos_base + static_cast<int64_t>(r) * a.pos_step + 1;
+  } else {
+    n = a.seq_len[r / a.rows_per_batch];
+  }
+  if (n > a.len_cap) n = a.len_cap;
+  return n < 0 ? 0 : n;
+}
+
+__global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a) {
+  __shared__ uint32_t hist[kBins];
+  __shared__ uint32_t warp_tot[32];
+  __shared__ uint32_t sh_bin, sh_above;
+
+  const int seg = blockIdx.x % a.n_seg;
+  const int r = blockIdx.x / a.n_seg;
+  if (r >= a.rows) return;
+  const int64_t n = row_length(a, r);
+  const int64_t lo = static_cast<int64_t>(seg) * a.seg_len;
+  const int64_t hi = a.n_seg == 1 ? n : min(n, lo + a.seg_len);
+  const float* vals = a.vals + static_cast<int64_t>(r) * a.ld;
+  const int32_t* in_idx = a.in_idx ? a.in_idx + static_cast<int64_t>(r) * a.ld : nullptr;
+  const int32_t* map =
+      a.idx_map ? a.idx_map + static_cast<int64_t>(r / a.rows_per_batch) * a.map_stride : nullptr;
+  const int64_t out_base = (static_cast<int64_t>(r) * a.n_seg + seg) * a.out_ld;
+  const int K = a.K;
+
+  // ---- radix passes: find the K-th largest key digit by digit -------------------------
+  // After the passes: elements whose top (32 - shift) key bits are > prefix are selected;
+  // those equal to prefix are selected while their tie rank is < need.
+  uint32_t prefix = 0;
+  int shift = 32;            // number of low key bits not yet resolved
+  uint32_t need = K;
+  bool take_all = false;
+  const int widths[3] = {12, 12, 8};
+  for (int p = 0; p < 3; ++p) {
+    const int wbits = widths[p];
+    const int nb = 1 << wbits;
+    const int nshift = shift - wbits;
+    for (int i = threadIdx.x; i < nb; i += kSelThreads) hist[i] = 0;
+    __syncthreads();
+    for (int64_t i = lo + threadIdx.x; i < hi; i += kSelThreads) {
+      const float v = vals[i];
+      if (!is_valid(v)) continue;
+      const uint32_t u = order_key(v);
+      if (shift < 32 && (u >> shift) != prefix) continue;
+      atomicAdd(&hist[(u >> nshift) & (nb - 1)], 1u);
+    }
+    __syncthreads();
+    // thread t owns the bins nb-1-(t*bpt) .. nb-(t+1)*bpt, i.e. thread 0 the highest ones
+    const int bpt = nb >= kSelThreads ? nb / kSelThreads : 1;
+    const bool owner = threadIdx.x * bpt < nb;
+    uint32_t mine = 0;
+    if (owner)
+      for (int j = 0; j < bpt; ++j) mine += hist[nb - 1 - (threadIdx.x * bpt + j)];
+    uint32_t total;
+    const uint32_t incl = block_inclusive_scan(mine, warp_tot, total);
+    if (p == 0 && total <= static_cast<uint32_t>(K)) {
+      take_all = true;  // every valid element is selected
+      break;
+    }
+    const uint32_t excl = incl - mine;
+    if (owner && excl < need && need <= incl) {
+      uint32_t above = excl;
+      for (int j = 0; j < bpt; ++j) {
+        const int bin = nb - 1 - (threadIdx.x * bpt + j);
+        const uint32_t h = hist[bin];
+        if (above + h >= need) {
+          sh_bin = static_cast<uint32_t>(bin);
+          sh_above = above;
+          break;
+        }
+        above += h;
+      }
+    }
+    __syncthreads();
+    const uint32_t bin = sh_bin;
+    need -= sh_above;
+    const uint32_t in_bin = hist[bin];
+    prefix = (shift < 32 ? (prefix << wbits) : 0u) | bin;
+    shift = nshift;
+    __syncthreads();
+    if (in_bin == need) break;  // the whole bin is taken: no further digits needed
+  }
+
+  // ---- output pass, in index order ----------------------------------------------------
+  uint32_t eq_carry = 0, sel_carry = 0;
+  constexpr int V = 4;
+  for (int64_t base = lo; base < hi; base += static_cast<int64_t>(kSelThreads) * V) {
+    float v[V];
+    uint32_t gt_mask = 0, eq_mask = 0;
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      const int64_t i = base + threadIdx.x * V + j;
+      v[j] = i < hi ? vals[i] : -INFINITY;
+      if (!is_valid(v[j])) continue;
+      if (take_all) {
+        gt_mask |= 1u << j;
+        continue;
+      }
+      const uint32_t top = order_key(v[j]) >> shift;
+      if (top > prefix) gt_mask |= 1u << j;
+      else if (top == prefix) eq_mask |= 1u << j;
+    }
+    uint32_t eq_tot;
+    const uint32_t n_eq = __popc(eq_mask);
+    const uint32_t eq_excl = block_inclusive_scan(n_eq, warp_tot, eq_tot) - n_eq + eq_carry;
+    uint32_t sel_mask = gt_mask;
+    uint32_t rank = eq_excl;
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      if (eq_mask & (1u << j)) {
+        if (rank < need) sel_mask |= 1u << j;
+        ++rank;
+      }
+    }
+    uint32_t sel_tot;
+    const uint32_t n_sel = __popc(sel_mask);
+    uint32_t slot = block_inclusive_scan(n_sel, warp_tot, sel_tot) - n_sel + sel_carry;
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      if (sel_mask & (1u << j)) {
+        const int64_t i = base + threadIdx.x * V + j;
+        int32_t id = in_idx ? in_idx[i] : static_cast<int32_t>(i);
+        if (map != nullptr && id >= 0) id = map[id];
+        if (slot < static_cast<uint32_t>(K)) {
+          a.out_idx[out_base + slot] = id;
+          if (a.out_val) a.out_val[out_base + slot] = v[j];
+        }
+        ++slot;
+      }
+    }
+    eq_carry += eq_tot;
+    sel_carry += sel_tot;
+  }
+  for (int64_t j = sel_carry + threadIdx.x; j < K; j += kSelThreads) {
+    a.out_idx[out_base + j] = -1;
+    if (a.out_val) a.out_val[out_base + j] = -INFINITY;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
+  const int64_t grid = static_cast<int64_t>(a.rows) * a.n_seg;
+  if (grid <= 0) return cudaSuccess;
+  select_kernel<<<static_cast<unsigned>(grid), kSelThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace adx

@@ -1,0 +1,173 @@
+"""Python entry points of the indexer: argument marshalling onto the C ABI (include/adx.h).
+
+Every computation runs in libadx.so's CUDA kernels; this module only checks tensor
+properties, allocates outputs and workspaces with PyTorch and passes raw device pointers
+and the current CUDA stream. There is no CPU or PyTorch fallback.
+
+Tensors: q [T, H, d] bf16 or uint8 (e4m3 codes, then q_scale [T] fp32); w [T, H] fp32;
+k [S, d] (prefill layout) or [T, S, d] (decode layout, with seq_len [T] int32 on the
+device), bf16 or uint8 e4m3 codes with k_scale fp32 of one value per key row.
+"""
+
+import ctypes
+
+import torch
+
+from . import _lib as L
+
+PAPER, WINDOW = L.ADX_BANK_PAPER, L.ADX_BANK_WINDOW
+
+
+def _mode(mode):
+    if isinstance(mode, str):
+        return {"paper": PAPER, "window": WINDOW}[mode]
+    return int(mode)
+
+
+def _dtype(t):
+    if t.dtype == torch.bfloat16:
+        return L.ADX_BF16
+    if t.dtype == torch.uint8:
+        return L.ADX_E4M3
+    raise TypeError(f"operand dtype {t.dtype}: expected bfloat16 or uint8 (e4m3 codes)")
+
+
+def _dev(t, name, dtype=None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def make_operands(q, w, k, q_scale=None, k_scale=None, q_pos0=0, seq_len=None):
+    """adx_operands for these tensors (prefill layout, or decode layout when seq_len is set)."""
+    _dev(q, "q"), _dev(w, "w", torch.float32), _dev(k, "k")
+    _dev(q_scale, "q_scale", torch.float32), _dev(k_scale, "k_scale", torch.float32)
+    _dev(seq_len, "seq_len", torch.int32)
+    T, H, d = q.shape
+    S = k.shape[-2]
+    o = L.Operands()
+    o.q_dtype, o.k_dtype = _dtype(q), _dtype(k)
+    o.q, o.q_scale, o.w = q.data_ptr(), _p(q_scale), w.data_ptr()
+    o.k, o.k_scale = k.data_ptr(), _p(k_scale)
+    o.T, o.H, o.d, o.S = T, H, d, S
+    o.q_pos0 = int(q_pos0)
+    o.seq_len = _p(seq_len)
+    return o
+
+
+class Workspace:
+    """Grow-only device workspace; its status word starts zeroed (torch.zeros)."""
+
+    def __init__(self, device=None):
+        self.device = device
+        self.buf = None
+
+    def get(self, nbytes):
+        nbytes = max(int(nbytes), L.ADX_STATUS_BYTES)
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.zeros(nbytes, dtype=torch.uint8, device=self.device or "cuda")
+        return self.buf
+
+
+_default_ws = {}
+
+
+def _ws(ws, device):
+    if ws is not None:
+        return ws
+    key = torch.device(device).index
+    if key not in _default_ws:
+        _default_ws[key] = Workspace(device)
+    return _default_ws[key]
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def workspace_size(op, ops, K=0, B=0, G=0, mode=PAPER):
+    n = L.lib().adx_workspace_size(op, ctypes.byref(ops), K, B, G, _mode(mode))
+    if n == 0:
+        raise L.AdxError("adx_workspace_size", L.ADX_EINVAL)
+    return n
+
+
+def index_prefill(q, w, k, K, q_scale=None, k_scale=None, q_pos0=0, with_scores=False,
+                  all_scores=False, ws=None, stream=None):
+    """Flat causal indexer (Eqs. (1)-(2)). Returns (topk_idx [T, K] int32,
+    topk_score [T, K] fp32 or None, scores [T, ld] fp32 or None)."""
+    ops = make_operands(q, w, k, q_scale, k_scale, q_pos0)
+    T, S = ops.T, ops.S
+    idx = torch.empty(T, K, dtype=torch.int32, device=q.device)
+    sc = torch.empty(T, K, dtype=torch.float32, device=q.device) if with_scores else None
+    full, ld = None, 0
+    if all_scores:
+        ld = (S + 127) // 128 * 128
+        full = torch.empty(T, ld, dtype=torch.float32, device=q.device)
+    buf = _ws(ws, q.device).get(workspace_size(L.ADX_OP_PREFILL, ops, K))
+    L.check("adx_index_prefill", L.lib().adx_index_prefill(
+        ctypes.byref(ops), K, _p(idx), _p(sc), _p(full), ld, _p(buf), buf.numel(),
+        _stream(stream)))
+    return idx, sc, full
+
+
+def index_decode(q, w, k, seq_len, K, q_scale=None, k_scale=None, with_scores=False, ws=None,
+                 stream=None):
+    """One decode step of the flat indexer: row t scores its own cache k[t]."""
+    ops = make_operands(q, w, k, q_scale, k_scale, 0, seq_len)
+    idx = torch.empty(ops.T, K, dtype=torch.int32, device=q.device)
+    sc = torch.empty(ops.T, K, dtype=torch.float32, device=q.device) if with_scores else None
+    buf = _ws(ws, q.device).get(workspace_size(L.ADX_OP_DECODE, ops, K))
+    L.check("adx_index_decode", L.lib().adx_index_decode(
+        ctypes.byref(ops), K, _p(idx), _p(sc), _p(buf), buf.numel(), _stream(stream)))
+    return idx, sc
+
+
+def bank_width(B, G, mode):
+    return L.lib().adx_bank_width(B, G, _mode(mode))
+
+
+def group_bank(qbar, wbar, k, G, B, mode, qbar_scale=None, k_scale=None, q_pos0=0,
+               seq_len=None, ws=None, stream=None):
+    """Shared token banks (Eq. (13)) of Ng = qbar.shape[0] groups -> bank [Ng, width] int32."""
+    ops = make_operands(qbar, wbar, k, qbar_scale, k_scale, q_pos0, seq_len)
+    m = _mode(mode)
+    bank = torch.empty(ops.T, bank_width(B, G, m), dtype=torch.int32, device=qbar.device)
+    buf = _ws(ws, qbar.device).get(workspace_size(L.ADX_OP_GROUP_BANK, ops, 0, B, G, m))
+    L.check("adx_group_bank", L.lib().adx_group_bank(
+        ctypes.byref(ops), G, B, m, _p(bank), _p(buf), buf.numel(), _stream(stream)))
+    return bank
+
+
+def bank_refine(q, w, k, bank, G, B, mode, K, q_scale=None, k_scale=None, q_pos0=0,
+                seq_len=None, with_scores=False, ws=None, stream=None):
+    """Query-specific refinement (Eq. (14)) -> (topk_idx [T, K], topk_score or None)."""
+    ops = make_operands(q, w, k, q_scale, k_scale, q_pos0, seq_len)
+    _dev(bank, "bank", torch.int32)
+    m = _mode(mode)
+    idx = torch.empty(ops.T, K, dtype=torch.int32, device=q.device)
+    sc = torch.empty(ops.T, K, dtype=torch.float32, device=q.device) if with_scores else None
+    buf = _ws(ws, q.device).get(workspace_size(L.ADX_OP_BANK_REFINE, ops, K, B, G, m))
+    L.check("adx_bank_refine", L.lib().adx_bank_refine(
+        ctypes.byref(ops), G, B, m, _p(bank), K, _p(idx), _p(sc), _p(buf), buf.numel(),
+        _stream(stream)))
+    return idx, sc
+
+
+def read_device_status(ws=None, device=None, stream=None):
+    """Synchronises and returns (and clears) the device status of a workspace (0 = ok)."""
+    w = _ws(ws, device or torch.device("cuda"))
+    if w.buf is None:
+        return L.ADX_OK
+    return L.lib().adx_read_device_status(_p(w.buf), _stream(stream))

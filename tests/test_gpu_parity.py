@@ -1,0 +1,273 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle on the same seeded inputs.
+
+Scores must agree within rtol * max(|I|, F) (2e-2 bf16, 6e-2 e4m3; see tests/parity.py);
+Top-K sets must agree except at keys within that tolerance of the oracle's K-th score.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import indexer as ox
+from sparse_attention_token_indexer_b200 import build, indexer, inputs
+
+from parity import RTOL, check_scores, check_topk, f64, score_floor
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    build.build()
+    yield
+    assert indexer.read_device_status() == 0
+
+
+def _to_cuda(p):
+    return {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in p.items()}
+
+
+def _flat_reference(q64, w64, k64, pos, rows):
+    """Per requested row: visible positions, oracle scores, score floors."""
+    out = {}
+    for t in rows:
+        n = min(int(pos[t]) + 1, k64.shape[0])
+        keys = k64[:n]
+        out[t] = (np.arange(n), ox.score_keys(q64[t], w64[t], keys),
+                  score_floor(q64[t], w64[t], keys))
+    return out
+
+
+def _check_flat(p, idx, sc, rows, what):
+    q64, k64 = f64(p["q"], p["q_scale"]), f64(p["k"], p["k_scale"])
+    w64 = p["w"].double().cpu().numpy()
+    pos = p["q_pos0"] + np.arange(p["T"])
+    ref = _flat_reference(q64, w64, k64, pos, rows)
+    idx, sc = idx.cpu().numpy(), None if sc is None else sc.cpu().numpy()
+    for t in rows:
+        cpos, cs, cf = ref[t]
+        check_topk(idx[t], cpos, cs, cf, p["K"], RTOL[p["dtype"]],
+                   None if sc is None else sc[t], f"{what} row {t}")
+    return ref
+
+
+def _rows_sample(T, K, n=40, seed=0):
+    rng = np.random.default_rng(seed)
+    fixed = {0, 1, 2, T - 1, T - 2, min(K - 1, T - 1), min(K, T - 1), min(K + 1, T - 1)}
+    return sorted(fixed | set(rng.choice(T, size=min(n, T), replace=False).tolist()))
+
+
+# ---------------------------------------------------------------------------------------
+# flat prefill
+# ---------------------------------------------------------------------------------------
+
+def test_tiny_prefill_every_score_and_row():
+    p = _to_cuda(inputs.tiny_prefill(seed=0))
+    idx, sc, full = indexer.index_prefill(p["q"], p["w"], p["k"], p["K"], with_scores=True,
+                                          all_scores=True)
+    torch.cuda.synchronize()
+    q64, k64, w64 = f64(p["q"]), f64(p["k"]), p["w"].double().cpu().numpy()
+    T = p["T"]
+    ref = ox.indexer_scores(q64, w64, k64, np.arange(T))
+    got = full.cpu().numpy()[:, :T]
+    vis = np.isfinite(ref)
+    # invisible keys are -inf up to the end of the row's own 128-key tile (entries past the
+    # last tile of a row block are not written)
+    for t in range(T):
+        end = min(T, (t // 128 + 1) * 128)
+        assert np.all(np.isneginf(got[t, t + 1:end])), f"row {t}: invisible keys must be -inf"
+    floor = np.stack([score_floor(q64[t], w64[t], k64) for t in range(T)])
+    check_scores(got[vis], ref[vis], floor[vis], RTOL["bf16"], "tiny scores")
+    _check_flat(p, idx, sc, range(T), "tiny")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_anchor_prefill_all_rows(dtype):
+    p = _to_cuda(inputs.anchor_prefill(1000, H=64, d=128, K=256, seed=11, dtype=dtype))
+    idx, sc, _ = indexer.index_prefill(p["q"], p["w"], p["k"], p["K"], p["q_scale"],
+                                       p["k_scale"], with_scores=True)
+    _check_flat(p, idx, sc, range(p["T"]), f"anchor {dtype}")
+
+
+@pytest.mark.parametrize("H,d", [(16, 128), (4, 128), (64, 64)])
+def test_other_head_counts(H, d):
+    p = _to_cuda(inputs.anchor_prefill(600, H=H, d=d, K=100, seed=12))
+    idx, sc, _ = indexer.index_prefill(p["q"], p["w"], p["k"], p["K"], with_scores=True)
+    _check_flat(p, idx, sc, range(p["T"]), f"H={H} d={d}")
+
+
+def test_chunked_prefill_with_offset():
+    p = _to_cuda(inputs.anchor_prefill(700, H=64, d=128, K=512, seed=13, S=3000))
+    assert p["q_pos0"] == 2300
+    idx, sc, _ = indexer.index_prefill(p["q"], p["w"], p["k"], p["K"], q_pos0=p["q_pos0"],
+                                       with_scores=True)
+    _check_flat(p, idx, sc, _rows_sample(700, 512), "chunk")
+
+
+def test_short_rows_return_every_visible_key():
+    p = _to_cuda(inputs.anchor_prefill(130, H=64, d=128, K=200, seed=14))
+    idx, _, _ = indexer.index_prefill(p["q"], p["w"], p["k"], p["K"])
+    idx = idx.cpu().numpy()
+    for t in range(130):
+        assert sorted(idx[t][idx[t] >= 0].tolist()) == list(range(t + 1))
+        assert np.all(idx[t][t + 1:] == -1)
+    p1 = _to_cuda(inputs.anchor_prefill(1, H=64, d=128, K=8, seed=15))
+    idx, _, _ = indexer.index_prefill(p1["q"], p1["w"], p1["k"], 8)
+    assert idx.cpu().tolist() == [[0] + [-1] * 7]
+
+
+def test_negative_gates():
+    p = _to_cuda(inputs.anchor_prefill(300, H=64, d=128, K=64, seed=16))
+    p["w"] = p["w"] - 0.5 / 64          # mixed signs
+    idx, sc, _ = indexer.index_prefill(p["q"], p["w"], p["k"], p["K"], with_scores=True)
+    _check_flat(p, idx, sc, range(300), "signed gates")
+
+
+# ---------------------------------------------------------------------------------------
+# group bank + refinement
+# ---------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode", ["window", "paper"])
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_group_bank_and_refine(mode, dtype):
+    T, G, B, K, Hg = 1536 + 37, 64, 512, 128, 16
+    p = _to_cuda(inputs.group_prefill(T, H=64, d=128, K=K, G=G, B=B, Hg=Hg, seed=21,
+                                      dtype=dtype))
+    rtol = RTOL[dtype]
+    bank = indexer.group_bank(p["qbar"], p["wbar"], p["k"], G, B, mode, p["qbar_scale"],
+                              p["k_scale"])
+    idx, sc = indexer.bank_refine(p["q"], p["w"], p["k"], bank, G, B, mode, K, p["q_scale"],
+                                  p["k_scale"], with_scores=True)
+    torch.cuda.synchronize()
+    q64, k64 = f64(p["q"], p["q_scale"]), f64(p["k"], p["k_scale"])
+    w64 = p["w"].double().cpu().numpy()
+    qb64, wb64 = f64(p["qbar"], p["qbar_scale"]), p["wbar"].double().cpu().numpy()
+    bank = bank.cpu().numpy()
+    idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+    plans = ox.plan_groups(T, 0, G, B, mode)
+    bank_k = B if mode == "paper" else B - G
+    assert bank.shape[1] == indexer.bank_width(B, G, mode)
+    n_complete = T // G
+    for g in range(n_complete):
+        a = g * G
+        scan_n = a + 1 if mode == "paper" else a
+        # stage 1: the bank's scan part against Eq. (13) with the oracle's group scores
+        keys = k64[:scan_n]
+        bs = ox.score_keys(qb64[g], wb64[g], keys)
+        bf = score_floor(qb64[g], wb64[g], keys)
+        check_topk(bank[g, :bank_k], np.arange(scan_n), bs, bf, bank_k, rtol, what=f"bank {g}")
+        post = bank[g, bank_k:]
+        lo = a + 1 if mode == "paper" else a
+        assert post.tolist() == list(range(lo, lo + len(post)))
+        # stage 2: refinement over the GPU's own bank (stage isolation)
+        scan_part = bank[g, :bank_k]
+        scan_part = scan_part[scan_part >= 0]
+        for i in range(a, a + G, 7 if g % 3 else 1):
+            cand = np.union1d(scan_part, np.arange(lo, i + 1))
+            cand = cand[cand <= i]
+            cs = ox.score_keys(q64[i], w64[i], k64[cand])
+            cf = score_floor(q64[i], w64[i], k64[cand])
+            check_topk(idx[i], cand, cs, cf, K, rtol, sc[i], f"refine row {i}")
+    # the incomplete trailing group uses the plain indexer
+    pos = np.arange(T)
+    tail = list(range(n_complete * G, T))
+    ref = _flat_reference(q64, w64, k64, pos, tail)
+    for t in tail:
+        cpos, cs, cf = ref[t]
+        check_topk(idx[t], cpos, cs, cf, K, rtol, sc[t], f"tail row {t}")
+    # paper fallback groups (a + 1 <= B) give the plain indexer's result exactly
+    if mode == "paper":
+        flat_idx, _, _ = indexer.index_prefill(p["q"], p["w"], p["k"], K, p["q_scale"],
+                                               p["k_scale"])
+        flat_idx = flat_idx.cpu().numpy()
+        for plan in plans:
+            if plan.kind == "flat":
+                for t in plan.rows:
+                    assert set(idx[t].tolist()) == set(flat_idx[t].tolist()), t
+
+
+# ---------------------------------------------------------------------------------------
+# decode
+# ---------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("k_dtype", ["e4m3", "bf16"])
+def test_decode_flat(k_dtype):
+    prob = inputs.decode_problem(Bs=4, S=5000, H=64, d=128, K=256, Hg=16, steps=1, seed=31,
+                                 k_dtype=k_dtype, device="cuda")
+    seq_len = torch.tensor([5000, 4097, 129, 1], dtype=torch.int32, device="cuda")
+    q, w = prob["q_steps"][0], prob["w_steps"][0]
+    idx, sc = indexer.index_decode(q, w, prob["k"], seq_len, 256, k_scale=prob["k_scale"],
+                                   with_scores=True)
+    torch.cuda.synchronize()
+    q64, w64 = f64(q), w.double().cpu().numpy()
+    k64 = f64(prob["k"].reshape(-1, 128), None if prob["k_scale"] is None
+              else prob["k_scale"].reshape(-1)).reshape(4, -1, 128)
+    idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+    for b, n in enumerate(seq_len.tolist()):
+        keys = k64[b, :n]
+        check_topk(idx[b], np.arange(n), ox.score_keys(q64[b], w64[b], keys),
+                   score_floor(q64[b], w64[b], keys), 256, RTOL[k_dtype], sc[b], f"decode {b}")
+
+
+def test_decode_bank_reuse():
+    Bs, S, K, B, G = 4, 6000, 256, 1024, 16
+    prob = inputs.decode_problem(Bs=Bs, S=S, H=64, d=128, K=K, Hg=16, steps=G, seed=32,
+                                 device="cuda")
+    k, ks = prob["k"], prob["k_scale"]
+    seq0 = inputs.decode_seq_len(prob, 0)
+    qbar, wbar = prob["q_steps"][0][:, :16].contiguous(), prob["w_steps"][0][:, :16].contiguous()
+    bank = indexer.group_bank(qbar, wbar, k, G, B, "paper", k_scale=ks, seq_len=seq0)
+    k64 = f64(k.reshape(-1, 128), ks.reshape(-1)).reshape(Bs, -1, 128)
+    qb64, wb64 = f64(qbar), wbar.double().cpu().numpy()
+    bank_np = bank.cpu().numpy()
+    assert bank_np.shape == (Bs, B + G - 1)
+    for b in range(Bs):
+        keys = k64[b, :S]
+        check_topk(bank_np[b, :B], np.arange(S), ox.score_keys(qb64[b], wb64[b], keys),
+                   score_floor(qb64[b], wb64[b], keys), B, RTOL["e4m3"], what=f"dbank {b}")
+        assert bank_np[b, B:].tolist() == list(range(S, S + G - 1))
+    for step in (0, 1, 5, G - 1):
+        seq = inputs.decode_seq_len(prob, step)
+        q, w = prob["q_steps"][step], prob["w_steps"][step]
+        idx, sc = indexer.bank_refine(q, w, k, bank, G, B, "paper", K, k_scale=ks,
+                                      seq_len=seq, with_scores=True)
+        idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+        q64, w64 = f64(q), w.double().cpu().numpy()
+        pos = S + step - 1
+        for b in range(Bs):
+            cand = np.union1d(bank_np[b, :B], np.arange(S, pos + 1))
+            cand = cand[(cand >= 0) & (cand <= pos)]
+            keys = k64[b, cand]
+            check_topk(idx[b], cand, ox.score_keys(q64[b], w64[b], keys),
+                       score_floor(q64[b], w64[b], keys), K, RTOL["e4m3"], sc[b],
+                       f"dref step {step} seq {b}")
+
+
+# ---------------------------------------------------------------------------------------
+# full-size workloads, sampled rows, in the configuration bench.py times
+# ---------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_full_size_flat_prefill_sampled(dtype):
+    T, K = 16384, 2048
+    p = inputs.anchor_prefill(T, H=64, d=128, K=K, seed=1, device="cuda", dtype=dtype)
+    idx, sc, _ = indexer.index_prefill(p["q"], p["w"], p["k"], K, p["q_scale"], p["k_scale"],
+                                       with_scores=True)
+    _check_flat(p, idx, sc, _rows_sample(T, K, n=24, seed=3), f"full {dtype}")
+
+
+def test_full_size_decode_sampled():
+    Bs, S, K = 32, 131072, 2048
+    prob = inputs.decode_problem(Bs=Bs, S=S, H=64, d=128, K=K, Hg=16, steps=1, seed=3,
+                                 device="cuda")
+    seq = inputs.decode_seq_len(prob, 0)
+    q, w = prob["q_steps"][0], prob["w_steps"][0]
+    idx, sc = indexer.index_decode(q, w, prob["k"], seq, K, k_scale=prob["k_scale"],
+                                   with_scores=True)
+    idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+    q64, w64 = f64(q), w.double().cpu().numpy()
+    for b in (0, 17, 31):
+        keys = f64(prob["k"][b], prob["k_scale"][b])
+        check_topk(idx[b], np.arange(S), ox.score_keys(q64[b], w64[b], keys),
+                   score_floor(q64[b], w64[b], keys), K, RTOL["e4m3"], sc[b], f"dfull {b}")
