@@ -33,6 +33,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 FLAT = dict(T=16384, H=64, d=128, K=2048, seed=1)
+# smaller flat case for ncu captures: its operands (q 128 MiB, scores 256 MiB) still exceed L2
+FLAT_SMALL = dict(T=8192, H=64, d=128, K=2048, seed=1)
 GROUP = dict(T=65536, H=64, d=128, K=2048, G=64, B=8192, Hg=16, seed=2)
 DECODE = dict(Bs=32, S=131072, H=64, d=128, K=2048, Hg=16, B=8192, G=16, seed=3)
 
@@ -215,7 +217,7 @@ def timed(fn, steps, warmup, dist, stage_timer=None):
 
 def run_flat(args, dist, dtype="bf16", clocks=None):
     from sparse_attention_token_indexer_b200 import _lib, indexer, inputs
-    c = FLAT
+    c = FLAT_SMALL if args.case == "flat_small" else FLAT
     p = inputs.anchor_prefill(c["T"], c["H"], c["d"], c["K"], seed=c["seed"], device="cuda",
                               dtype=dtype)
     ws = indexer.Workspace("cuda")
@@ -319,7 +321,7 @@ def run_decode(args, dist):
                                 c["B"], "paper", c["K"], k_scale=prob["k_scale"],
                                 seq_len=seqs[r], ws=ws)
 
-    ms_cycle, l_cycle = timed(cycle, max(2, args.steps // 4), 1, dist)
+    ms_cycle, l_cycle = timed(cycle, max(2, args.steps // 4), args.warmup, dist)
     key_bytes = c["d"] + 4
     return dict(ms_flat=ms_flat, launches_flat=l_flat, ms_cycle=ms_cycle, launches_cycle=l_cycle,
                 bytes_flat=c["Bs"] * c["S"] * key_bytes, steps_per_cycle=c["G"])
@@ -377,11 +379,17 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--rows", action="store_true", help="also time the other hot-path rows")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--case", default="flat", choices=["flat", "flat_small"],
+                    help="flat_small: T = 8192, for profiler captures")
+    ap.add_argument("--dtype", default="bf16", choices=["bf16", "e4m3"])
+    ap.add_argument("--quick", action="store_true",
+                    help="time the kernels only (no e2e, rows or CPU baseline): for profiling")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
     dist = Dist()
-    torch.cuda.set_device(dist.local)
+    if args.impl == "ours":
+        torch.cuda.set_device(dist.local)
     config = {"workload": "dsa_flat_prefill_T16384_H64_d128_K2048", "T": FLAT["T"],
               "H_I": FLAT["H"], "d": FLAT["d"], "K": FLAT["K"], "seq_len": FLAT["T"],
               "global_batch": dist.world, "parallelism": f"replicas{dist.world}",
@@ -422,8 +430,16 @@ def main():
     build.build()
     pk = peaks()
     clocks = Clocks(dist.local)
-    flat = run_flat(args, dist, "bf16", clocks)
+    flat = run_flat(args, dist, args.dtype, clocks)
     clk = clocks.summary()
+    if args.quick:
+        if dist.rank == 0:
+            print(json.dumps({"case": args.case, "dtype": args.dtype, "ms_per_step": flat["ms"],
+                              "score_ms": flat["score_ms"], "select_ms": flat["select_ms"],
+                              "score_tflops": flat["flops"] / flat["score_ms"] / 1e9,
+                              "gpu_launches": flat["launches"], "clocks": clk}), flush=True)
+        dist.close()
+        return
     value = dist.world * flat["pairs"] / (flat["ms"] * 1e-3)
     score_tflops = flat["flops"] / (flat["score_ms"] * 1e-3) / 1e12
     e2e_ms, h2d, d2h = run_e2e(args, dist, flat["p"])

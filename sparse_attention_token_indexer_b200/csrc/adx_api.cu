@@ -148,7 +148,27 @@ struct ScorePlan {
   ScoreArgs a{};
   bool fp8 = false;
   int H = 0, d = 0, tok = 0;
+  const void* qf = nullptr;  // gate-folded bf16 queries (rows with neg_row == 0), or null
 };
+
+// Workspace bytes of the gate-folded copy of R bf16 query rows.
+size_t ws_fold(int64_t R, int H, int d) {
+  return align_up(static_cast<size_t>(R) * H * d * 2, kAlign) + align_up(static_cast<size_t>(R), kAlign);
+}
+
+// bf16 queries against bf16 keys: writes w-folded queries and per-row sign flags into the
+// workspace and records them in the plan.
+adx_status prepare_fold(ScorePlan& p, const void* q, const float* w, int64_t R, Carve& cv,
+                        cudaStream_t s) {
+  uint16_t* qf = cv.take<uint16_t>(static_cast<size_t>(R) * p.H * p.d * 2);
+  int8_t* neg = cv.take<int8_t>(static_cast<size_t>(R));
+  if (counted(launch_fold_gates_bf16(static_cast<const uint16_t*>(q), w, R, p.H, p.d, qf, neg,
+                                     s)) != cudaSuccess)
+    return ADX_ECUDA;
+  p.qf = qf;
+  p.a.neg_row = neg;
+  return ADX_OK;
+}
 
 // Chooses the key-chunk size and the persistent grid for a score launch.
 void finish_plan(ScorePlan& p, int64_t max_tiles_per_block) {
@@ -169,17 +189,23 @@ void finish_plan(ScorePlan& p, int64_t max_tiles_per_block) {
 
 adx_status run_score(const ScorePlan& p, const void* q_codes, const void* keys, int64_t key_rows,
                      cudaStream_t s) {
-  CUtensorMap tq, tk;
+  CUtensorMap tq, tqf, tk;
   const int n = p.tok * p.H;
   if (!encode_rows(&tq, q_codes, p.fp8, p.d, static_cast<int64_t>(p.a.R) * p.H, n))
     return ADX_EINVAL;
+  if (p.qf != nullptr) {
+    if (!encode_rows(&tqf, p.qf, false, p.d, static_cast<int64_t>(p.a.R) * p.H, n))
+      return ADX_EINVAL;
+  } else {
+    tqf = tq;
+  }
   if (!encode_rows(&tk, keys, p.fp8, p.d, key_rows, kTileM)) return ADX_EINVAL;
   if (p.a.n_items <= 0) return ADX_OK;
   const int bps = score_blocks_per_sm(p.fp8, p.H, p.d, p.tok);
   const int grid = std::min<int64_t>(p.a.n_items, static_cast<int64_t>(sm_count()) * bps);
   if (grid <= 0) return ADX_EUNSUPPORTED;
   mark(0, s);
-  const cudaError_t e = counted(launch_score(tq, tk, p.a, p.fp8, p.H, p.d, p.tok, grid, s));
+  const cudaError_t e = counted(launch_score(tq, tqf, tk, p.a, p.fp8, p.H, p.d, p.tok, grid, s));
   mark(1, s);
   if (e == cudaErrorNotSupported) return ADX_EUNSUPPORTED;
   return e == cudaSuccess ? ADX_OK : ADX_ECUDA;
@@ -232,8 +258,11 @@ adx_status run_select(SelectArgs a, int64_t n_max, Carve& cv, DeviceStatus* st, 
 }
 
 // ---- flat prefill ------------------------------------------------------------------
+bool foldable(const adx_operands* o) { return o->q_dtype == ADX_BF16 && o->k_dtype == ADX_BF16; }
+
 size_t ws_flat(const adx_operands* o, int K, bool scores_external) {
   size_t b = kStatusBytes;
+  if (foldable(o)) b += ws_fold(o->T, o->H, o->d);
   if (!scores_external) b += align_up(static_cast<size_t>(o->T) * ld_for(o->S) * 4, kAlign);
   b += select_scratch_bytes(o->T, o->S, K);
   return b;
@@ -269,7 +298,9 @@ adx_status run_flat(const adx_operands* o, int K, int32_t* topk_idx, float* topk
   a.timeout_ns = kTimeoutNs;
   const int64_t max_keys = std::min<int64_t>(o->S, o->q_pos0 + o->T);
   finish_plan(p, (max_keys + kTileM - 1) / kTileM);
-  adx_status r = run_score(p, o->q, o->k, o->S, s);
+  adx_status r = ADX_OK;
+  if (foldable(o) && (r = prepare_fold(p, o->q, o->w, o->T, cv, s)) != ADX_OK) return r;
+  r = run_score(p, o->q, o->k, o->S, s);
   if (r != ADX_OK) return r;
   SelectArgs sa{};
   sa.vals = scores;
@@ -335,7 +366,7 @@ ScorePlan rowwise_plan(const adx_operands* o, const float* q_scale, float* score
 }
 
 size_t ws_decode(const adx_operands* o, int K) {
-  return kStatusBytes + ws_rowwise_q8(o) +
+  return kStatusBytes + ws_rowwise_q8(o) + (foldable(o) ? ws_fold(o->T, o->H, o->d) : 0) +
          align_up(static_cast<size_t>(o->T) * ld_for(o->S) * 4, kAlign) +
          select_scratch_bytes(o->T, o->S, K);
 }
@@ -373,7 +404,7 @@ adx_status check_bank_args(const adx_operands* o, int G, int B, int mode) {
 
 size_t ws_bank(const adx_operands* o, int G, int B, int mode) {
   const BankShape bs = bank_shape(B, G, mode);
-  return kStatusBytes + ws_rowwise_q8(o) +
+  return kStatusBytes + ws_rowwise_q8(o) + (foldable(o) ? ws_fold(o->T, o->H, o->d) : 0) +
          align_up(static_cast<size_t>(o->T) * ld_for(o->S) * 4, kAlign) +
          select_scratch_bytes(o->T, o->S, bs.bank_k);
 }
@@ -386,6 +417,7 @@ size_t ws_refine(const adx_operands* o, int G, int B, int mode, int K) {
   const int64_t ng = dec ? o->T : o->T / G;
   const int64_t rows = dec ? o->T : ng * G;
   size_t b = kStatusBytes + ws_rowwise_q8(o);
+  if (foldable(o)) b += ws_fold(rows, o->H, o->d);
   b += align_up(static_cast<size_t>(ng) * bcp * row_bytes(o), kAlign);  // packed keys
   b += align_up(static_cast<size_t>(ng) * bcp * 4, kAlign) * 2;          // scales, positions
   b += align_up(static_cast<size_t>(rows) * bcp * 4, kAlign);             // scores
@@ -489,6 +521,7 @@ adx_status adx_index_decode(const adx_operands* o, int32_t K, int32_t* topk_idx,
   ScorePlan p = rowwise_plan(o, q_scale, scores, ld);
   p.a.status = st;
   finish_plan(p, (o->S + kTileM - 1) / kTileM);
+  if (foldable(o) && (r = prepare_fold(p, o->q, o->w, o->T, cv, s)) != ADX_OK) return r;
   if ((r = run_score(p, q, o->k, static_cast<int64_t>(o->T) * o->S, s)) != ADX_OK) return r;
   SelectArgs sa{};
   sa.vals = scores;
@@ -529,6 +562,7 @@ adx_status adx_group_bank(const adx_operands* o, int32_t G, int32_t B, int32_t m
     ScorePlan p = rowwise_plan(o, q_scale, scores, ld);
     p.a.status = st;
     finish_plan(p, (o->S + kTileM - 1) / kTileM);
+    if (foldable(o) && (r = prepare_fold(p, o->q, o->w, o->T, cv, s)) != ADX_OK) return r;
     if ((r = run_score(p, q, o->k, static_cast<int64_t>(o->T) * o->S, s)) != ADX_OK) return r;
     sa.vals = scores;
     sa.len_mode = 2;
@@ -559,6 +593,7 @@ adx_status adx_group_bank(const adx_operands* o, int32_t G, int32_t B, int32_t m
     const int64_t last = o->q_pos0 + bs.scan_pos_off + static_cast<int64_t>(o->T - 1) * G;
     const int64_t max_keys = std::max<int64_t>(0, std::min<int64_t>(o->S, last + 1));
     finish_plan(p, std::max<int64_t>(1, (max_keys + kTileM - 1) / kTileM));
+    if (foldable(o) && (r = prepare_fold(p, o->q, o->w, o->T, cv, s)) != ADX_OK) return r;
     if ((r = run_score(p, o->q, o->k, o->S, s)) != ADX_OK) return r;
     sa.vals = scores;
     sa.len_mode = 1;
@@ -637,6 +672,7 @@ adx_status adx_bank_refine(const adx_operands* o, int32_t G, int32_t B, int32_t 
     p.a.keys_per_batch = static_cast<int32_t>(bcp);
     p.a.status = st;
     finish_plan(p, bcp / kTileM);
+    if (foldable(o) && (r = prepare_fold(p, q, o->w, rows, cv, s)) != ADX_OK) return r;
     if ((r = run_score(p, q, packed, ng * bcp, s)) != ADX_OK) return r;
     SelectArgs sa{};
     sa.vals = scores;

@@ -33,6 +33,7 @@ struct ScoreArgs {
   const float* k_scale;    // [n_batches * key_batch_stride] or null
   const int32_t* key_pos;  // [n_batches * key_batch_stride] or null
   const int32_t* seq_len;  // [n_batches] or null
+  const int8_t* neg_row;   // [R]: 1 = row has a negative gate; null = no folded queries
   float* scores;           // [R, score_ld]
   int64_t score_ld;
   int64_t pos_base;
@@ -78,8 +79,11 @@ struct SelectArgs {
 };
 
 // Launchers (return a cudaError_t from the launch).
-cudaError_t launch_score(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const ScoreArgs& a,
-                         bool fp8, int H, int d, int tok, int grid, cudaStream_t s);
+// tm_qf maps the gate-folded queries (used for row blocks whose rows all have neg_row == 0);
+// pass tm_q again when there are none.
+cudaError_t launch_score(const CUtensorMap& tm_q, const CUtensorMap& tm_qf, const CUtensorMap& tm_k,
+                         const ScoreArgs& a, bool fp8, int H, int d, int tok, int grid,
+                         cudaStream_t s);
 int score_tokens_per_tile(int H);  // tokens per N tile for a head count (0 = unsupported)
 bool score_config_supported(bool fp8, int H, int d);
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s);
@@ -95,5 +99,7 @@ cudaError_t launch_fill_post_anchor(int32_t* bank, int32_t n_groups, int32_t ban
                                     int32_t pos_step, const int32_t* seq_len, int32_t start_off,
                                     cudaStream_t s);
 int score_blocks_per_sm(bool fp8, int H, int d, int tok);
+cudaError_t launch_fold_gates_bf16(const uint16_t* q, const float* w, int64_t rows, int H, int d,
+                                   uint16_t* qf, int8_t* neg_row, cudaStream_t s);
 
 }  // namespace adx

@@ -3,6 +3,8 @@
 //  * candidate packing: gather each group's candidate key rows (and scales, positions) into
 //    a contiguous block so that refinement streams them with tiled TMA loads
 //    (ADIndex, arXiv 2611.12956v1, §4.3 Eq. (14): C_i = bank U post-anchor positions);
+//  * gate folding for bf16 queries with non-negative gates (w * ReLU(x) = ReLU(w * x)), so
+//    the scoring epilogue needs no gate loads;
 //  * post-anchor columns of a bank: the positions every member of a group adds to the
 //    shared bank (Eq. (14)), stored beside the bank so refinement needs no extra inputs.
 #include <cuda_bf16.h>
@@ -86,7 +88,45 @@ __global__ void fill_post_kernel(int32_t* bank, int32_t n_groups, int32_t bank_w
   bank[static_cast<int64_t>(g) * bank_w + first_col + j] = static_cast<int32_t>(anchor + start_off + j);
 }
 
+// q'[r, j, :] = bf16(w[r, j] * q[r, j, :]) for rows whose gates are all >= 0, where
+// w * ReLU(q . k) = ReLU((w q) . k); neg_row[r] = 1 marks rows with a negative gate (their
+// folded copy is not used).
+__global__ void __launch_bounds__(256)
+fold_gates_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w, int H, int d,
+                  __nv_bfloat16* __restrict__ qf, int8_t* __restrict__ neg_row) {
+  const int64_t r = blockIdx.x;
+  const float* wr = w + r * H;
+  int neg = 0;
+  for (int j = threadIdx.x; j < H; j += blockDim.x) neg |= wr[j] < 0.f;
+  neg = __syncthreads_or(neg);
+  if (threadIdx.x == 0) neg_row[r] = static_cast<int8_t>(neg != 0);
+  if (neg) return;
+  const int64_t n = static_cast<int64_t>(H) * d;
+  const uint4* src = reinterpret_cast<const uint4*>(q + r * n);
+  uint4* dst = reinterpret_cast<uint4*>(qf + r * n);
+  for (int64_t i = threadIdx.x; i < n / 8; i += blockDim.x) {
+    const float g = wr[(i * 8) / d];
+    uint4 v = src[i];
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float2 f = __bfloat1622float2(h[u]);
+      h[u] = __floats2bfloat162_rn(f.x * g, f.y * g);
+    }
+    dst[i] = v;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_fold_gates_bf16(const uint16_t* q, const float* w, int64_t rows, int H, int d,
+                                   uint16_t* qf, int8_t* neg_row, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  fold_gates_kernel<<<static_cast<unsigned>(rows), 256, 0, s>>>(
+      reinterpret_cast<const __nv_bfloat16*>(q), w, H, d, reinterpret_cast<__nv_bfloat16*>(qf),
+      neg_row);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_quantize_rows_e4m3(const uint16_t* x_bf16, int64_t rows, int64_t cols,
                                       uint8_t* codes, float* scale, cudaStream_t s) {

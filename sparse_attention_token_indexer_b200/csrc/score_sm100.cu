@@ -14,9 +14,11 @@
 // heads of every token in registers - ReLU, gate and head sum never leave the SM, so the
 // per-head logits [T, H, S] are never written anywhere.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and issues the
-// MMAs (one thread), warps 2-5 run the epilogue. The grid is persistent: CTA c takes work
-// items c, c + gridDim.x, ... where an item is (row block, chunk of key tiles).
+// Warp roles: warp 0 issues TMA loads, warp 1 allocates TMEM and issues the MMAs (one
+// thread), the remaining one or two warpgroups run the epilogue (each owns half of the
+// tile's query tokens). The grid is persistent and statically balanced: all (row block,
+// key tile) pairs are laid end to end, longest rows first, and every CTA takes an equal
+// contiguous share, loading a row block's queries once for its whole run of key tiles.
 #include <cuda_bf16.h>
 
 #include "adx_internal.h"
@@ -26,8 +28,7 @@ namespace adx {
 
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kEpiWarps = 4;
+constexpr int kMaxThreads = 320;
 
 __host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 __host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
@@ -47,6 +48,19 @@ struct Cfg {
   static constexpr int KC = DB / 128;        // 128-byte K chunks
   static constexpr int ELEMS_PER_CHUNK = FP8 ? 128 : 64;
   static constexpr int KSTEPS = DB / 32;     // 32 bytes of K per MMA instruction
+  // Epilogue warpgroups. With two and few tokens per tile (BUF_SPLIT), warpgroup g owns
+  // TMEM accumulator buffer g and reduces every other tile, all of its tokens, so each warp
+  // has two MMA periods per tile; with many tokens per tile the two warpgroups split the
+  // tokens of every tile instead (keeps the per-thread accumulators in registers).
+  static constexpr int EG = TOK >= 2 ? 2 : 1;
+  static constexpr bool BUF_SPLIT = false;
+  static constexpr int EPI_WARPS = 4 * EG;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int TOKG = BUF_SPLIT ? TOK : TOK / EG;  // tokens one warp reduces per tile
+  static constexpr int NG = TOKG * H;        // accumulator columns one warp reads per tile
+  static constexpr int CW = NG < 32 ? NG : 32;  // TMEM columns per load
+  static constexpr int NCH = NG / CW;        // loads per tile per thread
+  static constexpr int NP = (H >= 16 && TOKG <= 4) ? 4 : 1;  // partial sums per token
   static constexpr int QBYTES = N * DB;
   static constexpr int KBYTES = kTileM * DB;
   static constexpr int ST = cmin(8, (200 * 1024 - QBYTES) / KBYTES);
@@ -55,18 +69,25 @@ struct Cfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = QBYTES;
   static constexpr int OFF_W = OFF_K + ST * KBYTES;
-  static constexpr int OFF_BAR = OFF_W + kEpiWarps * N * 4;  // one gate copy per epilogue warp
+  static constexpr int OFF_BAR = OFF_W + EPI_WARPS * NG * 4;  // one gate copy per epilogue warp
   static constexpr int NBAR = 2 * ST + 2 * ACC + 3;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
+  static constexpr int OFF_SCAN = OFF_MISC + 64;
+  static constexpr int SMEM = OFF_SCAN + 8 * (THREADS / 32) + 1024;  // + alignment slack
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "invalid MMA N");
   static_assert(DB % 128 == 0, "rows must be a multiple of 128 bytes");
   static_assert(QBYTES % 1024 == 0 && KBYTES % 1024 == 0, "alignment");
   static_assert(ST >= 2, "not enough shared memory for a pipeline");
+  static_assert(NG % CW == 0 && CW % 4 == 0 && (H >= 32 ? H % CW == 0 : CW % H == 0),
+                "epilogue chunking");
+  static_assert(THREADS <= kMaxThreads, "block size");
+  static_assert(!BUF_SPLIT || EG == ACC, "one accumulator buffer per epilogue warpgroup");
 };
 
-struct Item {
-  int b, row0, row_end, t_begin, t_end, nkeys;
+// One row block of the work: TOK consecutive query rows of one key batch and the key
+// tiles they need.
+struct Block {
+  int b, row0, row_end, nkeys, ntiles;
   int64_t key_row0;  // first key row of the batch in the key tensor map
 };
 
@@ -75,17 +96,19 @@ __device__ __forceinline__ int64_t row_position(const ScoreArgs& a, int r) {
   return a.pos_base + static_cast<int64_t>(r) * a.pos_step;
 }
 
+// Row block number i of the schedule (longest first for a causal prefix).
 template <int TOK>
-__device__ __forceinline__ bool decode_item(const ScoreArgs& a, int it, Item& x) {
-  const int kc = it % a.chunks_per_block;
-  int rbg = it / a.chunks_per_block;
-  const int total_rb = a.row_blocks_per_batch * a.n_batches;
-  if (a.reverse_order) rbg = total_rb - 1 - rbg;
+__device__ __forceinline__ void block_info(const ScoreArgs& a, int i, Block& x) {
+  const int nb = a.row_blocks_per_batch * a.n_batches;
+  const int rbg = a.reverse_order ? nb - 1 - i : i;
   x.b = rbg / a.row_blocks_per_batch;
   const int rb = rbg % a.row_blocks_per_batch;
   x.row0 = x.b * a.rows_per_batch + rb * TOK;
   x.row_end = min(min(x.row0 + TOK, (x.b + 1) * a.rows_per_batch), a.R);
-  if (x.row0 >= x.row_end) return false;
+  x.key_row0 = static_cast<int64_t>(x.b) * a.key_batch_stride;
+  x.nkeys = 0;
+  x.ntiles = 0;
+  if (x.row0 >= x.row_end) return;
   int64_t nk;
   if (a.key_pos != nullptr) {
     nk = a.keys_per_batch;
@@ -94,13 +117,62 @@ __device__ __forceinline__ bool decode_item(const ScoreArgs& a, int it, Item& x)
   } else {
     nk = min(row_position(a, x.row_end - 1) + 1, static_cast<int64_t>(a.keys_per_batch));
   }
-  if (nk <= 0) return false;
+  if (nk <= 0) return;
   x.nkeys = static_cast<int>(nk);
-  const int ntiles = (x.nkeys + kTileM - 1) / kTileM;
-  x.t_begin = kc * a.chunk_tiles;
-  x.t_end = min(x.t_begin + a.chunk_tiles, ntiles);
-  x.key_row0 = static_cast<int64_t>(x.b) * a.key_batch_stride;
-  return x.t_begin < x.t_end;
+  x.ntiles = (x.nkeys + kTileM - 1) / kTileM;
+}
+
+// Balanced static partition: all (row block, key tile) pairs laid end to end in schedule
+// order; CTA c owns the tiles [c*W/grid, (c+1)*W/grid). Computed once per CTA by all its
+// threads; returns the first row block touching the range and the tile offset it starts at.
+template <class C>
+__device__ __forceinline__ void partition(const ScoreArgs& a, int64_t* scan_s, int64_t& start,
+                                          int64_t& end, int& b0, int64_t& base0) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NW = C::THREADS / 32;
+  const int nb = a.row_blocks_per_batch * a.n_batches;
+  const int per = (nb + C::THREADS - 1) / C::THREADS;
+  const int lo = min(nb, tid * per), hi = min(nb, lo + per);
+  int64_t mine = 0;
+  for (int i = lo; i < hi; ++i) {
+    Block x;
+    block_info<C::TOK>(a, i, x);
+    mine += x.ntiles;
+  }
+  int64_t incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) scan_s[warp] = incl;
+  __syncthreads();
+  int64_t before = 0, total = 0;
+  for (int w = 0; w < NW; ++w) {
+    const int64_t v = scan_s[w];
+    if (w < warp) before += v;
+    total += v;
+  }
+  const int64_t excl = before + incl - mine;
+  start = static_cast<int64_t>(blockIdx.x) * total / gridDim.x;
+  end = static_cast<int64_t>(blockIdx.x + 1) * total / gridDim.x;
+  __syncthreads();  // everyone has read scan_s
+  if (start < end && excl <= start && start < excl + mine) {
+    int64_t cum = excl;
+    for (int i = lo; i < hi; ++i) {
+      Block x;
+      block_info<C::TOK>(a, i, x);
+      if (start < cum + x.ntiles) {
+        scan_s[0] = i;
+        scan_s[1] = cum;
+        break;
+      }
+      cum += x.ntiles;
+    }
+  }
+  __syncthreads();
+  b0 = start < end ? static_cast<int>(scan_s[0]) : 0;
+  base0 = start < end ? scan_s[1] : 0;
 }
 
 __device__ __forceinline__ void raise_timeout(const ScoreArgs& a, int role) {
@@ -118,10 +190,61 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
   (void)mbar_wait(bar, parity, &never, timeout_ns);
 }
 
+template <int CW>
+__device__ __forceinline__ void tmem_ld_chunk(uint32_t taddr, float (&v)[CW]) {
+  if constexpr (CW == 32) {
+    tmem_ld32(taddr, v);
+  } else {
+    tmem_ld16(taddr, v);
+  }
+}
+
+// ReLU, gate and head sum of one chunk of accumulator columns (group-local columns
+// c0 .. c0+CW-1), as packed fp32x2 FMAs into independent partial sums.
 template <class C>
-__global__ void __launch_bounds__(kThreads, 1)
-score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-             const ScoreArgs a) {
+__device__ __forceinline__ void reduce_chunk(const float (&v)[C::CW], const float* w, int c0,
+                                             float2 (&acc)[C::TOKG][C::NP]) {
+#pragma unroll
+  for (int i = 0; i < C::CW; i += 4) {
+    const int col = c0 + i;
+    const int tt = col / C::H;
+    const int m = (col % C::H) / 2;
+    const float4 w4 = *reinterpret_cast<const float4*>(w + col);
+    const float2 r01 = make_float2(fmaxf(v[i], 0.f), fmaxf(v[i + 1], 0.f));
+    const float2 r23 = make_float2(fmaxf(v[i + 2], 0.f), fmaxf(v[i + 3], 0.f));
+    acc[tt][m % C::NP] = __ffma2_rn(r01, make_float2(w4.x, w4.y), acc[tt][m % C::NP]);
+    acc[tt][(m + 1) % C::NP] =
+        __ffma2_rn(r23, make_float2(w4.z, w4.w), acc[tt][(m + 1) % C::NP]);
+  }
+}
+
+// Gate-folded variant of reduce_chunk: the queries were pre-multiplied by their (non-negative)
+// gates, so a column's contribution is just ReLU(x).
+template <class C>
+__device__ __forceinline__ void reduce_chunk_folded(const float (&v)[C::CW], int c0,
+                                                    float2 (&acc)[C::TOKG][C::NP]) {
+#pragma unroll
+  for (int i = 0; i < C::CW; i += 2) {
+    const int col = c0 + i;
+    const int tt = col / C::H;
+    const int m = (col % C::H) / 2;
+    acc[tt][m % C::NP] =
+        __fadd2_rn(acc[tt][m % C::NP], make_float2(fmaxf(v[i], 0.f), fmaxf(v[i + 1], 0.f)));
+  }
+}
+
+// True when every row of the block has non-negative gates and folded queries exist.
+__device__ __forceinline__ bool block_folded(const ScoreArgs& a, const Block& x) {
+  if (a.neg_row == nullptr) return false;
+  int neg = 0;
+  for (int r = x.row0; r < x.row_end; ++r) neg |= a.neg_row[r];
+  return neg == 0;
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
+score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qf,
+             const __grid_constant__ CUtensorMap tm_k, const ScoreArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -138,6 +261,7 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   uint64_t* drain = q_full + 2;
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_s = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  int64_t* scan_s = reinterpret_cast<int64_t*>(smem + C::OFF_SCAN);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -149,7 +273,7 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     }
     for (int i = 0; i < C::ACC; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], kEpiWarps);
+      mbar_init(&acc_empty[i], C::BUF_SPLIT ? 4 : C::EPI_WARPS);
     }
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
@@ -157,16 +281,21 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     *abort_s = 0;
     fence_mbarrier_init();
     tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_qf);
     tma_prefetch_desc(&tm_k);
   }
   if (warp == 1) {
     tmem_alloc(tmem_base_s, C::TMEM_COLS);
     tmem_relinquish();
   }
+  int64_t start, end, base0;
+  int b0;
+  partition<C>(a, scan_s, start, end, b0, base0);  // contains __syncthreads
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_base_s;
+  const int nblocks = a.row_blocks_per_batch * a.n_batches;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -176,20 +305,26 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       uint32_t q_phase = 0;
       bool q_loaded = false;
       uint32_t issued_mask = 0, issued_parity = 0;
-      for (int it = blockIdx.x; it < a.n_items && !*abort_s; it += gridDim.x) {
-        Item x;
-        if (!decode_item<C::TOK>(a, it, x)) continue;
+      int64_t cum = base0;
+      for (int bi = b0; bi < nblocks && cum < end && !*abort_s; ++bi) {
+        Block x;
+        block_info<C::TOK>(a, bi, x);
+        const int64_t t_lo = max(start - cum, int64_t(0));
+        const int64_t t_hi = min(end - cum, static_cast<int64_t>(x.ntiles));
+        cum += x.ntiles;
+        if (t_lo >= t_hi) continue;
         if (q_loaded) {
           if (!mbar_wait(q_empty, q_phase ^ 1u, abort_s, a.timeout_ns)) break;
         }
+        const CUtensorMap* qmap = block_folded(a, x) ? &tm_qf : &tm_q;
         mbar_arrive_expect_tx(q_full, C::QBYTES);
 #pragma unroll
         for (int kc = 0; kc < C::KC; ++kc)
-          tma_load_2d(q_s + kc * C::N * 128, &tm_q, q_full, kc * C::ELEMS_PER_CHUNK,
+          tma_load_2d(q_s + kc * C::N * 128, qmap, q_full, kc * C::ELEMS_PER_CHUNK,
                       x.row0 * C::H);
         q_loaded = true;
         q_phase ^= 1u;
-        for (int t = x.t_begin; t < x.t_end; ++t) {
+        for (int t = static_cast<int>(t_lo); t < static_cast<int>(t_hi); ++t) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_s, a.timeout_ns)) break;
           mbar_arrive_expect_tx(&full[stage], C::KBYTES);
           const int32_t y = static_cast<int32_t>(x.key_row0 + static_cast<int64_t>(t) * kTileM);
@@ -221,15 +356,20 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       int acc = 0;
       uint32_t acc_phase = 0;
       bool any = false;
-      for (int it = blockIdx.x; it < a.n_items && !*abort_s; it += gridDim.x) {
-        Item x;
-        if (!decode_item<C::TOK>(a, it, x)) continue;
+      int64_t cum = base0;
+      for (int bi = b0; bi < nblocks && cum < end && !*abort_s; ++bi) {
+        Block x;
+        block_info<C::TOK>(a, bi, x);
+        const int64_t t_lo = max(start - cum, int64_t(0));
+        const int64_t t_hi = min(end - cum, static_cast<int64_t>(x.ntiles));
+        cum += x.ntiles;
+        if (t_lo >= t_hi) continue;
         if (!mbar_wait(q_full, q_phase, abort_s, a.timeout_ns)) break;
         q_phase ^= 1u;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(q_s);
         bool ok = true;
-        for (int t = x.t_begin; t < x.t_end; ++t) {
+        for (int t = static_cast<int>(t_lo); t < static_cast<int>(t_hi); ++t) {
           if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_s, a.timeout_ns) ||
               !mbar_wait(&full[stage], phase, abort_s, a.timeout_ns)) {
             ok = false;
@@ -257,7 +397,7 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             acc_phase ^= 1u;
           }
         }
-        umma_commit(q_empty);  // Q buffer is free once this item's MMAs complete
+        umma_commit(q_empty);  // Q buffer is free once this block's MMAs complete
         if (!ok) break;
       }
       if (*abort_s) raise_timeout(a, 1);
@@ -268,20 +408,28 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     }
   } else {
     // ------------------------------------------------------------------ epilogue
-    const int ew = warp - 2;                  // 0..3
+    const int ew = warp - 2;                  // 0 .. EPI_WARPS-1
+    const int grp = ew / 4;                   // epilogue warpgroup
     const int lq = warp & 3;                  // TMEM lane quadrant this warp may access
     const int m = lq * 32 + lane;             // key row within the tile = TMEM lane
-    constexpr int CW = C::N < 32 ? C::N : 32; // TMEM columns per load
-    float* w_w = w_s + ew * C::N;             // this warp's copy of the gates
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    for (int it = blockIdx.x; it < a.n_items && !*abort_s; it += gridDim.x) {
-      Item x;
-      if (!decode_item<C::TOK>(a, it, x)) continue;
-      // gates of this item's rows, with the per-token query scale folded in
+    float* w_w = w_s + ew * C::NG;            // this warp's copy of the gates
+    const int tok0 = C::BUF_SPLIT ? 0 : grp * C::TOKG;  // first token this warp reduces
+    int64_t gi = 0;                           // tile counter of this CTA (selects the buffer)
+    int64_t cum = base0;
+    for (int bi = b0; bi < nblocks && cum < end && !*abort_s; ++bi) {
+      Block x;
+      block_info<C::TOK>(a, bi, x);
+      const int64_t t_lo = max(start - cum, int64_t(0));
+      const int64_t t_hi = min(end - cum, static_cast<int64_t>(x.ntiles));
+      cum += x.ntiles;
+      if (t_lo >= t_hi) continue;
+      // gates of this block's rows, with the per-token query scale folded in (not needed
+      // when the queries carry their gates already)
+      const bool folded = block_folded(a, x);
       __syncwarp();
-      for (int i = lane; i < C::N; i += 32) {
-        const int r = x.row0 + i / C::H;
+      const int rowg = x.row0 + tok0;
+      for (int i = lane; i < C::NG && !folded; i += 32) {
+        const int r = rowg + i / C::H;
         float wv = 0.f;
         if (r < x.row_end) {
           wv = a.w[static_cast<int64_t>(r) * C::H + (i % C::H)];
@@ -290,13 +438,16 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         w_w[i] = wv;
       }
       __syncwarp();
-      int64_t rpos[C::TOK];
+      int32_t rpos[C::TOKG];
 #pragma unroll
-      for (int tt = 0; tt < C::TOK; ++tt)
-        rpos[tt] = (x.row0 + tt < x.row_end) ? row_position(a, x.row0 + tt) : -1;
+      for (int tt = 0; tt < C::TOKG; ++tt)
+        rpos[tt] = (rowg + tt < x.row_end) ? static_cast<int32_t>(row_position(a, rowg + tt)) : -1;
 
       bool ok = true;
-      for (int t = x.t_begin; t < x.t_end; ++t) {
+      for (int t = static_cast<int>(t_lo); t < static_cast<int>(t_hi); ++t, ++gi) {
+        const int acc = static_cast<int>(gi % C::ACC);
+        if (C::BUF_SPLIT && acc != grp) continue;  // the other warpgroup's tile
+        const uint32_t acc_phase = static_cast<uint32_t>((gi / C::ACC) & 1);
         int got = 0;
         if (lane == 0) got = mbar_wait(&acc_full[acc], acc_phase, abort_s, a.timeout_ns) ? 1 : 0;
         got = __shfl_sync(0xffffffffu, got, 0);
@@ -314,39 +465,54 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           if (a.key_pos != nullptr) kpos = a.key_pos[kr];
           if (a.k_scale != nullptr) ks = a.k_scale[kr];
         }
-        float accum[C::TOK];
+        float2 part[C::TOKG][C::NP];
 #pragma unroll
-        for (int tt = 0; tt < C::TOK; ++tt) accum[tt] = 0.f;
-        const uint32_t taddr =
-            tmem_base + (static_cast<uint32_t>(lq * 32) << 16) + static_cast<uint32_t>(acc * C::N);
+        for (int tt = 0; tt < C::TOKG; ++tt)
 #pragma unroll
-        for (int c0 = 0; c0 < C::N; c0 += CW) {
-          float v[CW];
-          if constexpr (CW == 32) {
-            tmem_ld32(taddr + c0, v);
-          } else {
-            tmem_ld16(taddr + c0, v);
+          for (int p = 0; p < C::NP; ++p) part[tt][p] = make_float2(0.f, 0.f);
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(lq * 32) << 16) +
+                               static_cast<uint32_t>(acc * C::N + tok0 * C::H);
+        // software pipeline: the next chunk's TMEM load is in flight while this one reduces
+        float va[C::CW], vb[C::CW];
+        tmem_ld_chunk<C::CW>(taddr, va);
+        tmem_wait_ld();
+        if (folded) {
+#pragma unroll
+          for (int ch = 0; ch < C::NCH; ++ch) {
+            if (ch % 2 == 0) {
+              if (ch + 1 < C::NCH) tmem_ld_chunk<C::CW>(taddr + (ch + 1) * C::CW, vb);
+              reduce_chunk_folded<C>(va, ch * C::CW, part);
+            } else {
+              if (ch + 1 < C::NCH) tmem_ld_chunk<C::CW>(taddr + (ch + 1) * C::CW, va);
+              reduce_chunk_folded<C>(vb, ch * C::CW, part);
+            }
+            if (ch + 1 < C::NCH) tmem_wait_ld();
           }
-          tmem_wait_ld();
+        } else {
 #pragma unroll
-          for (int i = 0; i < CW; ++i) {
-            const int col = c0 + i;
-            accum[col / C::H] = fmaf(w_w[col], fmaxf(v[i], 0.f), accum[col / C::H]);
+          for (int ch = 0; ch < C::NCH; ++ch) {
+            if (ch % 2 == 0) {
+              if (ch + 1 < C::NCH) tmem_ld_chunk<C::CW>(taddr + (ch + 1) * C::CW, vb);
+              reduce_chunk<C>(va, w_w, ch * C::CW, part);
+            } else {
+              if (ch + 1 < C::NCH) tmem_ld_chunk<C::CW>(taddr + (ch + 1) * C::CW, va);
+              reduce_chunk<C>(vb, w_w, ch * C::CW, part);
+            }
+            if (ch + 1 < C::NCH) tmem_wait_ld();
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[acc]);
-        if (++acc == C::ACC) {
-          acc = 0;
-          acc_phase ^= 1u;
-        }
 #pragma unroll
-        for (int tt = 0; tt < C::TOK; ++tt) {
-          const int r = x.row0 + tt;
+        for (int tt = 0; tt < C::TOKG; ++tt) {
+          const int r = rowg + tt;
           if (r < x.row_end) {
+            float sc = 0.f;
+#pragma unroll
+            for (int p = 0; p < C::NP; ++p) sc += part[tt][p].x + part[tt][p].y;
             const bool vis = key_ok && kpos <= rpos[tt];
-            a.scores[static_cast<int64_t>(r) * a.score_ld + c] = vis ? ks * accum[tt] : -INFINITY;
+            a.scores[static_cast<int64_t>(r) * a.score_ld + c] = vis ? ks * sc : -INFINITY;
           }
         }
       }
@@ -365,12 +531,12 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 }
 
 template <class C>
-cudaError_t launch_cfg(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const ScoreArgs& a,
-                       int grid, cudaStream_t s) {
+cudaError_t launch_cfg(const CUtensorMap& tm_q, const CUtensorMap& tm_qf, const CUtensorMap& tm_k,
+                       const ScoreArgs& a, int grid, cudaStream_t s) {
   auto kern = score_kernel<C>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, C::SMEM, s>>>(tm_q, tm_k, a);
+  kern<<<grid, C::THREADS, C::SMEM, s>>>(tm_q, tm_qf, tm_k, a);
   return cudaGetLastError();
 }
 
@@ -405,11 +571,12 @@ bool score_config_supported(bool fp8, int H, int d) {
 
 // tok: tokens per N tile; either score_tokens_per_tile(H) (prefill) or 1 (one query per
 // key batch: decode and its bank refresh).
-cudaError_t launch_score(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const ScoreArgs& a,
-                         bool fp8, int H, int d, int tok, int grid, cudaStream_t s) {
+cudaError_t launch_score(const CUtensorMap& tm_q, const CUtensorMap& tm_qf, const CUtensorMap& tm_k,
+                         const ScoreArgs& a, bool fp8, int H, int d, int tok, int grid,
+                         cudaStream_t s) {
 #define ADX_CASE(FP, HH, TT, DD)                                                        \
   if (fp8 == FP && H == HH && tok == TT && d == DD)                                     \
-    return launch_cfg<Cfg<HH, TT, (FP ? DD : 2 * DD), FP>>(tm_q, tm_k, a, grid, s);
+    return launch_cfg<Cfg<HH, TT, (FP ? DD : 2 * DD), FP>>(tm_q, tm_qf, tm_k, a, grid, s);
   ADX_SCORE_CONFIGS(ADX_CASE)
 #undef ADX_CASE
   return cudaErrorNotSupported;

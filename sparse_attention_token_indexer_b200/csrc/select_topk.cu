@@ -103,12 +103,12 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a)
     const int nshift = shift - wbits;
     for (int i = threadIdx.x; i < nb; i += kSelThreads) hist[i] = 0;
     __syncthreads();
-    for (int64_t i = lo + threadIdx.x; i < hi; i += kSelThreads) {
-      const float v = vals[i];
-      if (!is_valid(v)) continue;
+    for (int64_t base = lo; base < hi; base += kSelThreads) {
+      const int64_t i = base + threadIdx.x;
+      const float v = i < hi ? vals[i] : -INFINITY;
       const uint32_t u = order_key(v);
-      if (shift < 32 && (u >> shift) != prefix) continue;
-      atomicAdd(&hist[(u >> nshift) & (nb - 1)], 1u);
+      if (is_valid(v) && (shift >= 32 || (u >> shift) == prefix))
+        atomicAdd(&hist[(u >> nshift) & (nb - 1)], 1u);
     }
     __syncthreads();
     // thread t owns the bins nb-1-(t*bpt) .. nb-(t+1)*bpt, i.e. thread 0 the highest ones
@@ -203,12 +203,223 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a)
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// Rows of at most kRegItems * kSelThreads elements: the whole row lives in registers (each
+// thread a contiguous run of kRegItems elements), so global memory is read once; the digit
+// passes work on registers and one block-wide scan of (above, equal) counts gives every
+// thread its output slots in index order.
+// ---------------------------------------------------------------------------------------
+constexpr int kRegItems = 32;
+constexpr int kRegCapacity = kRegItems * kSelThreads;
+
+__device__ __forceinline__ unsigned long long block_exclusive_scan64(unsigned long long x,
+                                                                    unsigned long long* warp_tot,
+                                                                    unsigned long long& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned long long incl = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  unsigned long long before = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < kSelWarps; ++w) {
+    const unsigned long long v = warp_tot[w];
+    if (w < warp) before += v;
+    tot += v;
+  }
+  total = tot;
+  __syncthreads();
+  return before + incl - x;
+}
+
+__global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const SelectArgs a) {
+  __shared__ uint32_t hist[kBins];
+  __shared__ uint32_t warp_tot[32];
+  __shared__ uint32_t red_min[kSelWarps], red_max[kSelWarps], red_cnt[kSelWarps];
+  __shared__ unsigned long long warp_tot64[kSelWarps];
+  __shared__ uint32_t sh_bin, sh_above;
+
+  const int seg = blockIdx.x % a.n_seg;
+  const int r = blockIdx.x / a.n_seg;
+  if (r >= a.rows) return;
+  const int64_t n = row_length(a, r);
+  const int64_t lo = static_cast<int64_t>(seg) * a.seg_len;
+  const int64_t hi = a.n_seg == 1 ? n : min(n, lo + a.seg_len);
+  const int64_t len = hi > lo ? hi - lo : 0;
+  const float* vals = a.vals + static_cast<int64_t>(r) * a.ld + lo;
+  const int32_t* in_idx = a.in_idx ? a.in_idx + static_cast<int64_t>(r) * a.ld + lo : nullptr;
+  const int32_t* map =
+      a.idx_map ? a.idx_map + static_cast<int64_t>(r / a.rows_per_batch) * a.map_stride : nullptr;
+  const int64_t out_base = (static_cast<int64_t>(r) * a.n_seg + seg) * a.out_ld;
+  const int K = a.K;
+
+  // ---- load: thread t owns elements [t*kRegItems, (t+1)*kRegItems) of the segment ------
+  uint32_t key[kRegItems];
+  const int64_t my0 = static_cast<int64_t>(threadIdx.x) * kRegItems;
+  const bool vec = ((reinterpret_cast<uintptr_t>(vals) & 15) == 0);
+#pragma unroll
+  for (int j = 0; j < kRegItems; j += 4) {
+    float v[4];
+    const int64_t i0 = my0 + j;
+    if (vec && i0 + 4 <= len) {
+      const float4 f = *reinterpret_cast<const float4*>(vals + i0);
+      v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+    } else {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = (i0 + u < len) ? vals[i0 + u] : -INFINITY;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) key[j + u] = is_valid(v[u]) ? order_key(v[u]) : 0u;  // 0 = invalid
+  }
+
+  // ---- common high bits of the valid keys: the first digit starts below them ----------
+  uint32_t kmin = 0xffffffffu, kmax = 0u, nval = 0u;
+#pragma unroll
+  for (int j = 0; j < kRegItems; ++j) {
+    if (key[j] != 0u) {
+      kmin = min(kmin, key[j]);
+      kmax = max(kmax, key[j]);
+      ++nval;
+    }
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  nval = __reduce_add_sync(0xffffffffu, nval);
+  if ((threadIdx.x & 31) == 0) {
+    red_min[threadIdx.x >> 5] = kmin;
+    red_max[threadIdx.x >> 5] = kmax;
+    red_cnt[threadIdx.x >> 5] = nval;
+  }
+  __syncthreads();
+  kmin = 0xffffffffu;
+  kmax = 0u;
+  nval = 0u;
+#pragma unroll
+  for (int w = 0; w < kSelWarps; ++w) {
+    kmin = min(kmin, red_min[w]);
+    kmax = max(kmax, red_max[w]);
+    nval += red_cnt[w];
+  }
+
+  uint32_t prefix = 0;
+  int shift = 32;            // number of low key bits not yet resolved
+  uint32_t need = K;
+  bool take_all = nval <= static_cast<uint32_t>(K);
+  if (!take_all) {
+    const uint32_t diff = kmin ^ kmax;
+    shift = diff == 0u ? 0 : 32 - __clz(diff);  // bits above `shift` are common to all keys
+    prefix = shift >= 32 ? 0u : (kmax >> shift);
+  }
+#pragma unroll 1
+  while (!take_all && shift > 0) {
+    const int wbits = min(12, shift);
+    const int nb = 1 << wbits;
+    const int nshift = shift - wbits;
+    for (int i = threadIdx.x; i < nb; i += kSelThreads) hist[i] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kRegItems; ++j) {
+      const uint32_t u = key[j];
+      if (u != 0u && (shift >= 32 || (u >> shift) == prefix))
+        atomicAdd(&hist[(u >> nshift) & (nb - 1)], 1u);
+    }
+    __syncthreads();
+    const int bpt = nb >= kSelThreads ? nb / kSelThreads : 1;
+    const bool owner = threadIdx.x * bpt < nb;
+    uint32_t mine = 0;
+    if (owner)
+      for (int j = 0; j < bpt; ++j) mine += hist[nb - 1 - (threadIdx.x * bpt + j)];
+    uint32_t total;
+    const uint32_t incl = block_inclusive_scan(mine, warp_tot, total);
+    const uint32_t excl = incl - mine;
+    if (owner && excl < need && need <= incl) {
+      uint32_t above = excl;
+      for (int j = 0; j < bpt; ++j) {
+        const int bin = nb - 1 - (threadIdx.x * bpt + j);
+        const uint32_t h = hist[bin];
+        if (above + h >= need) {
+          sh_bin = static_cast<uint32_t>(bin);
+          sh_above = above;
+          break;
+        }
+        above += h;
+      }
+    }
+    __syncthreads();
+    const uint32_t bin = sh_bin;
+    need -= sh_above;
+    const uint32_t in_bin = hist[bin];
+    prefix = (shift < 32 ? (prefix << wbits) : 0u) | bin;
+    shift = nshift;
+    __syncthreads();
+    if (in_bin == need) break;
+  }
+
+  // ---- output: one scan of (above, equal) counts, then each thread writes its run ------
+  uint32_t gt_mask = 0, eq_mask = 0;
+#pragma unroll
+  for (int j = 0; j < kRegItems; ++j) {
+    const uint32_t u = key[j];
+    if (u == 0u) continue;
+    if (take_all) {
+      gt_mask |= 1u << j;
+      continue;
+    }
+    const uint32_t top = u >> shift;
+    if (top > prefix) gt_mask |= 1u << j;
+    else if (top == prefix) eq_mask |= 1u << j;
+  }
+  unsigned long long tot;
+  const unsigned long long packed =
+      (static_cast<unsigned long long>(__popc(gt_mask)) << 32) | __popc(eq_mask);
+  const unsigned long long ex = block_exclusive_scan64(packed, warp_tot64, tot);
+  const uint32_t gt_before = static_cast<uint32_t>(ex >> 32);
+  const uint32_t eq_before = static_cast<uint32_t>(ex & 0xffffffffu);
+  const uint32_t n_sel_total =
+      static_cast<uint32_t>(tot >> 32) + min(static_cast<uint32_t>(tot & 0xffffffffu), need);
+  uint32_t slot = gt_before + min(eq_before, need);
+  uint32_t eq_rank = eq_before;
+#pragma unroll
+  for (int j = 0; j < kRegItems; ++j) {
+    bool sel = (gt_mask >> j) & 1u;
+    if ((eq_mask >> j) & 1u) {
+      sel = eq_rank < need;
+      ++eq_rank;
+    }
+    if (sel) {
+      const int64_t i = my0 + j;
+      int32_t id = in_idx ? in_idx[i] : static_cast<int32_t>(lo + i);
+      if (map != nullptr && id >= 0) id = map[id];
+      if (slot < static_cast<uint32_t>(K)) {
+        a.out_idx[out_base + slot] = id;
+        if (a.out_val) {
+          const uint32_t u = key[j];
+          a.out_val[out_base + slot] = __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+        }
+      }
+      ++slot;
+    }
+  }
+  for (int64_t j = n_sel_total + threadIdx.x; j < K; j += kSelThreads) {
+    a.out_idx[out_base + j] = -1;
+    if (a.out_val) a.out_val[out_base + j] = -INFINITY;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
   const int64_t grid = static_cast<int64_t>(a.rows) * a.n_seg;
   if (grid <= 0) return cudaSuccess;
-  select_kernel<<<static_cast<unsigned>(grid), kSelThreads, 0, s>>>(a);
+  const int64_t seg = a.n_seg == 1 ? a.len_cap : a.seg_len;
+  if (seg <= kRegCapacity)
+    select_reg_kernel<<<static_cast<unsigned>(grid), kSelThreads, 0, s>>>(a);
+  else
+    select_kernel<<<static_cast<unsigned>(grid), kSelThreads, 0, s>>>(a);
   return cudaGetLastError();
 }
 
