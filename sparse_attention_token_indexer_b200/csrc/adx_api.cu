@@ -228,7 +228,9 @@ adx_status run_select(SelectArgs a, int64_t n_max, Carve& cv, DeviceStatus* st, 
   if (n_seg == 1) {
     a.n_seg = 1;
     a.seg_len = static_cast<int32_t>(std::min<int64_t>(n_max, INT32_MAX));
-    const cudaError_t e = counted(launch_select(a, s));
+    int nl = 0;
+    const cudaError_t e0 = launch_select(a, s, &nl);
+    const cudaError_t e = counted(e0, nl);
     mark(3, s);
     return e == cudaSuccess ? ADX_OK : ADX_ECUDA;
   }
@@ -242,7 +244,9 @@ adx_status run_select(SelectArgs a, int64_t n_max, Carve& cv, DeviceStatus* st, 
   s1.out_idx = cv_idx;
   s1.out_val = cv_val;
   s1.out_ld = a.K;
-  if (counted(launch_select(s1, s)) != cudaSuccess) return ADX_ECUDA;
+  int nl = 0;
+  const cudaError_t e1 = launch_select(s1, s, &nl);
+  if (counted(e1, nl) != cudaSuccess) return ADX_ECUDA;
   SelectArgs s2 = a;
   s2.vals = cv_val;
   s2.in_idx = cv_idx;
@@ -252,7 +256,8 @@ adx_status run_select(SelectArgs a, int64_t n_max, Carve& cv, DeviceStatus* st, 
   s2.len_cap = s2.len_fixed;
   s2.n_seg = 1;
   s2.seg_len = s2.len_fixed;
-  const cudaError_t e = counted(launch_select(s2, s));
+  const cudaError_t e2 = launch_select(s2, s, &nl);
+  const cudaError_t e = counted(e2, nl);
   mark(3, s);
   return e == cudaSuccess ? ADX_OK : ADX_ECUDA;
 }

@@ -86,7 +86,8 @@ cudaError_t launch_score(const CUtensorMap& tm_q, const CUtensorMap& tm_qf, cons
                          cudaStream_t s);
 int score_tokens_per_tile(int H);  // tokens per N tile for a head count (0 = unsupported)
 bool score_config_supported(bool fp8, int H, int d);
-cudaError_t launch_select(const SelectArgs& a, cudaStream_t s);
+// Launches one to three kernels (row-length classes); *launched receives how many.
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launched);
 cudaError_t launch_quantize_rows_e4m3(const uint16_t* x_bf16, int64_t rows, int64_t cols,
                                       uint8_t* codes, float* scale, cudaStream_t s);
 cudaError_t launch_pack_candidates(const void* k, const float* k_scale, int64_t key_batch_stride,

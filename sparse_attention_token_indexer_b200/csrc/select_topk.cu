@@ -8,6 +8,7 @@
 // using block-wide prefix sums (warp shuffles) for the output slots. -inf marks a masked
 // (invisible) key and NaN is treated the same way: neither is ever selected. Rows with fewer
 // than K valid elements return all of them, padded with index -1 and score -inf.
+#include <algorithm>
 #include <cstdint>
 
 #include "adx_internal.h"
@@ -204,17 +205,19 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a)
 }
 
 // ---------------------------------------------------------------------------------------
-// Rows of at most kRegItems * kSelThreads elements: the whole row lives in registers (each
+// Rows of at most kRegItems * THREADS elements: the whole row lives in registers (each
 // thread a contiguous run of kRegItems elements), so global memory is read once; the digit
 // passes work on registers and one block-wide scan of (above, equal) counts gives every
-// thread its output slots in index order.
+// thread its output slots in index order. The CTA size (and digit width) is chosen per row
+// length class, so short rows of a causal prefix do not pay for long ones.
 // ---------------------------------------------------------------------------------------
 constexpr int kRegItems = 32;
-constexpr int kRegCapacity = kRegItems * kSelThreads;
 
+template <int THREADS>
 __device__ __forceinline__ unsigned long long block_exclusive_scan64(unsigned long long x,
                                                                     unsigned long long* warp_tot,
                                                                     unsigned long long& total) {
+  constexpr int NW = THREADS / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   unsigned long long incl = x;
 #pragma unroll
@@ -226,7 +229,7 @@ __device__ __forceinline__ unsigned long long block_exclusive_scan64(unsigned lo
   __syncthreads();
   unsigned long long before = 0, tot = 0;
 #pragma unroll
-  for (int w = 0; w < kSelWarps; ++w) {
+  for (int w = 0; w < NW; ++w) {
     const unsigned long long v = warp_tot[w];
     if (w < warp) before += v;
     tot += v;
@@ -236,16 +239,19 @@ __device__ __forceinline__ unsigned long long block_exclusive_scan64(unsigned lo
   return before + incl - x;
 }
 
-__global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const SelectArgs a) {
-  __shared__ uint32_t hist[kBins];
-  __shared__ uint32_t warp_tot[32];
-  __shared__ uint32_t red_min[kSelWarps], red_max[kSelWarps], red_cnt[kSelWarps];
-  __shared__ unsigned long long warp_tot64[kSelWarps];
+template <int THREADS, int DIGIT>
+__global__ void __launch_bounds__(THREADS) select_reg_kernel(const SelectArgs a, int row0) {
+  constexpr int NW = THREADS / 32;
+  constexpr int NB = 1 << DIGIT;
+  __shared__ uint32_t hist[NB];
+  __shared__ unsigned long long warp_tot64[NW];
+  __shared__ uint32_t red_min[NW], red_max[NW], red_cnt[NW];
   __shared__ uint32_t sh_bin, sh_above;
 
   const int seg = blockIdx.x % a.n_seg;
-  const int r = blockIdx.x / a.n_seg;
+  const int r = row0 + static_cast<int>(blockIdx.x / a.n_seg);
   if (r >= a.rows) return;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t n = row_length(a, r);
   const int64_t lo = static_cast<int64_t>(seg) * a.seg_len;
   const int64_t hi = a.n_seg == 1 ? n : min(n, lo + a.seg_len);
@@ -261,6 +267,7 @@ __global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const SelectArg
   uint32_t key[kRegItems];
   const int64_t my0 = static_cast<int64_t>(threadIdx.x) * kRegItems;
   const bool vec = ((reinterpret_cast<uintptr_t>(vals) & 15) == 0);
+  uint32_t kmin = 0xffffffffu, kmax = 0u, nval = 0u;
 #pragma unroll
   for (int j = 0; j < kRegItems; j += 4) {
     float v[4];
@@ -273,33 +280,30 @@ __global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const SelectArg
       for (int u = 0; u < 4; ++u) v[u] = (i0 + u < len) ? vals[i0 + u] : -INFINITY;
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) key[j + u] = is_valid(v[u]) ? order_key(v[u]) : 0u;  // 0 = invalid
-  }
-
-  // ---- common high bits of the valid keys: the first digit starts below them ----------
-  uint32_t kmin = 0xffffffffu, kmax = 0u, nval = 0u;
-#pragma unroll
-  for (int j = 0; j < kRegItems; ++j) {
-    if (key[j] != 0u) {
-      kmin = min(kmin, key[j]);
-      kmax = max(kmax, key[j]);
-      ++nval;
+    for (int u = 0; u < 4; ++u) {
+      const bool ok = is_valid(v[u]);
+      const uint32_t k = ok ? order_key(v[u]) : 0u;  // 0 = invalid (valid keys are > 0)
+      key[j + u] = k;
+      kmin = ok ? min(kmin, k) : kmin;
+      kmax = max(kmax, k);
+      nval += ok;
     }
   }
+  // common high bits of the valid keys: the first digit starts right below them
   kmin = __reduce_min_sync(0xffffffffu, kmin);
   kmax = __reduce_max_sync(0xffffffffu, kmax);
   nval = __reduce_add_sync(0xffffffffu, nval);
-  if ((threadIdx.x & 31) == 0) {
-    red_min[threadIdx.x >> 5] = kmin;
-    red_max[threadIdx.x >> 5] = kmax;
-    red_cnt[threadIdx.x >> 5] = nval;
+  if (lane == 0) {
+    red_min[warp] = kmin;
+    red_max[warp] = kmax;
+    red_cnt[warp] = nval;
   }
   __syncthreads();
   kmin = 0xffffffffu;
   kmax = 0u;
   nval = 0u;
 #pragma unroll
-  for (int w = 0; w < kSelWarps; ++w) {
+  for (int w = 0; w < NW; ++w) {
     kmin = min(kmin, red_min[w]);
     kmax = max(kmax, red_max[w]);
     nval += red_cnt[w];
@@ -308,7 +312,7 @@ __global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const SelectArg
   uint32_t prefix = 0;
   int shift = 32;            // number of low key bits not yet resolved
   uint32_t need = K;
-  bool take_all = nval <= static_cast<uint32_t>(K);
+  const bool take_all = nval <= static_cast<uint32_t>(K);
   if (!take_all) {
     const uint32_t diff = kmin ^ kmax;
     shift = diff == 0u ? 0 : 32 - __clz(diff);  // bits above `shift` are common to all keys
@@ -316,10 +320,10 @@ __global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const SelectArg
   }
 #pragma unroll 1
   while (!take_all && shift > 0) {
-    const int wbits = min(12, shift);
+    const int wbits = min(DIGIT, shift);
     const int nb = 1 << wbits;
     const int nshift = shift - wbits;
-    for (int i = threadIdx.x; i < nb; i += kSelThreads) hist[i] = 0;
+    for (int i = threadIdx.x; i < nb; i += THREADS) hist[i] = 0;
     __syncthreads();
 #pragma unroll
     for (int j = 0; j < kRegItems; ++j) {
@@ -328,15 +332,15 @@ __global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const SelectArg
         atomicAdd(&hist[(u >> nshift) & (nb - 1)], 1u);
     }
     __syncthreads();
-    const int bpt = nb >= kSelThreads ? nb / kSelThreads : 1;
+    // thread t owns bins nb-1-t*bpt .. : thread 0 the highest ones
+    const int bpt = nb >= THREADS ? nb / THREADS : 1;
     const bool owner = threadIdx.x * bpt < nb;
     uint32_t mine = 0;
     if (owner)
       for (int j = 0; j < bpt; ++j) mine += hist[nb - 1 - (threadIdx.x * bpt + j)];
-    uint32_t total;
-    const uint32_t incl = block_inclusive_scan(mine, warp_tot, total);
-    const uint32_t excl = incl - mine;
-    if (owner && excl < need && need <= incl) {
+    unsigned long long tot64;
+    const uint32_t excl = static_cast<uint32_t>(block_exclusive_scan64<THREADS>(mine, warp_tot64, tot64));
+    if (owner && excl < need && need <= excl + mine) {
       uint32_t above = excl;
       for (int j = 0; j < bpt; ++j) {
         const int bin = nb - 1 - (threadIdx.x * bpt + j);
@@ -356,7 +360,7 @@ __global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const SelectArg
     prefix = (shift < 32 ? (prefix << wbits) : 0u) | bin;
     shift = nshift;
     __syncthreads();
-    if (in_bin == need) break;
+    if (in_bin == need) break;  // the whole bin is taken: no further digits needed
   }
 
   // ---- output: one scan of (above, equal) counts, then each thread writes its run ------
@@ -369,14 +373,14 @@ __global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const SelectArg
       gt_mask |= 1u << j;
       continue;
     }
-    const uint32_t top = u >> shift;
+    const uint32_t top = shift >= 32 ? 0u : (u >> shift);
     if (top > prefix) gt_mask |= 1u << j;
     else if (top == prefix) eq_mask |= 1u << j;
   }
   unsigned long long tot;
   const unsigned long long packed =
       (static_cast<unsigned long long>(__popc(gt_mask)) << 32) | __popc(eq_mask);
-  const unsigned long long ex = block_exclusive_scan64(packed, warp_tot64, tot);
+  const unsigned long long ex = block_exclusive_scan64<THREADS>(packed, warp_tot64, tot);
   const uint32_t gt_before = static_cast<uint32_t>(ex >> 32);
   const uint32_t eq_before = static_cast<uint32_t>(ex & 0xffffffffu);
   const uint32_t n_sel_total =
@@ -404,23 +408,52 @@ __global__ void __launch_bounds__(kSelThreads) select_reg_kernel(const SelectArg
       ++slot;
     }
   }
-  for (int64_t j = n_sel_total + threadIdx.x; j < K; j += kSelThreads) {
+  for (int64_t j = n_sel_total + threadIdx.x; j < K; j += THREADS) {
     a.out_idx[out_base + j] = -1;
     if (a.out_val) a.out_val[out_base + j] = -INFINITY;
   }
 }
 
+template <int THREADS, int DIGIT>
+cudaError_t launch_reg(const SelectArgs& a, int row0, int row1, cudaStream_t s, int* launched) {
+  const int64_t grid = static_cast<int64_t>(row1 - row0) * a.n_seg;
+  if (grid <= 0) return cudaSuccess;
+  select_reg_kernel<THREADS, DIGIT><<<static_cast<unsigned>(grid), THREADS, 0, s>>>(a, row0);
+  ++*launched;
+  return cudaGetLastError();
+}
+
 }  // namespace
 
-cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launched) {
+  *launched = 0;
   const int64_t grid = static_cast<int64_t>(a.rows) * a.n_seg;
   if (grid <= 0) return cudaSuccess;
   const int64_t seg = a.n_seg == 1 ? a.len_cap : a.seg_len;
-  if (seg <= kRegCapacity)
-    select_reg_kernel<<<static_cast<unsigned>(grid), kSelThreads, 0, s>>>(a);
-  else
+  constexpr int64_t c128 = 128 * kRegItems, c256 = 256 * kRegItems, c512 = 512 * kRegItems;
+  if (seg > c512) {
     select_kernel<<<static_cast<unsigned>(grid), kSelThreads, 0, s>>>(a);
-  return cudaGetLastError();
+    *launched = 1;
+    return cudaGetLastError();
+  }
+  // rows of a causal prefix grow with the row index: split the launch by length class
+  int r128 = 0, r256 = 0;
+  if (a.len_mode == 1 && a.n_seg == 1 && a.pos_step > 0) {
+    auto rows_upto = [&](int64_t cap) {  // first row whose length exceeds cap
+      const int64_t r = (cap - 1 - a.pos_base) / a.pos_step + 1;
+      return static_cast<int>(std::max<int64_t>(0, std::min<int64_t>(a.rows, r)));
+    };
+    r128 = rows_upto(c128);
+    r256 = std::max(r128, rows_upto(c256));
+  } else if (seg <= c128) {
+    r128 = r256 = a.rows;
+  } else if (seg <= c256) {
+    r256 = a.rows;
+  }
+  cudaError_t e;
+  if ((e = launch_reg<128, 10>(a, 0, r128, s, launched)) != cudaSuccess) return e;
+  if ((e = launch_reg<256, 11>(a, r128, r256, s, launched)) != cudaSuccess) return e;
+  return launch_reg<512, 12>(a, r256, a.rows, s, launched);
 }
 
 }  // namespace adx
