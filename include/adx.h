@@ -165,6 +165,24 @@ void adx_set_timing_events(void* const* events, int32_t n);
 /* Number of kernels this library has launched in the process so far. */
 int64_t adx_launch_count(void);
 
+/* Bytes of the fixed device scratch array behind adx_index_prefill_noalloc. */
+#define ADX_STATIC_SCRATCH_BYTES (32u << 20)
+
+/* adx_index_prefill for callers that cannot allocate device memory (an engine that plans all
+ * device buffers ahead in its own arena, a plugin host without an allocator, plain C code):
+ * same operands, outputs and results as adx_index_prefill, but no workspace argument. The
+ * paper has no counterpart; this exists only for such callers.
+ * Scratch is a fixed array of ADX_STATIC_SCRATCH_BYTES inside the library; every GPU that
+ * loads the library holds it until the process exits. Problems that need more (see
+ * adx_workspace_size(ADX_OP_PREFILL, ...)) return ADX_EWORKSPACE before any launch; nothing is
+ * ever allocated. The first call on a device looks up the array's device address with that
+ * device current: make it before any stream capture. All calls on a device share the array,
+ * so calls that overlap on the GPU race; serialise them. Each call clears the status word on
+ * `stream` first; device_status (a device int32, or NULL) receives the call's device status
+ * (ADX_OK or ADX_ETIMEOUT) asynchronously on `stream`. */
+adx_status adx_index_prefill_noalloc(const adx_operands* ops, int32_t K, int32_t* topk_idx,
+                                     float* topk_score, int32_t* device_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

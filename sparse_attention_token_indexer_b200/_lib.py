@@ -17,7 +17,8 @@ ADX_STATUS_BYTES = 256
 # every extern "C" symbol include/adx.h declares
 EXPORTS = ("adx_abi_version", "adx_bank_width", "adx_status_string", "adx_workspace_size",
            "adx_index_prefill", "adx_index_decode", "adx_group_bank", "adx_bank_refine",
-           "adx_read_device_status", "adx_set_timing_events", "adx_launch_count")
+           "adx_read_device_status", "adx_set_timing_events", "adx_launch_count",
+           "adx_index_prefill_noalloc")
 
 
 class Operands(ctypes.Structure):
@@ -62,6 +63,7 @@ def _declare(lib):
         "adx_read_device_status": (ctypes.c_int, [VP, VP]),
         "adx_set_timing_events": (None, [ctypes.POINTER(VP), I32]),
         "adx_launch_count": (I64, []),
+        "adx_index_prefill_noalloc": (ctypes.c_int, [P, I32, VP, VP, VP, VP]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

@@ -14,7 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libadx.so")
-SOURCES = ["adx_api.cu", "score_sm100.cu", "select_topk.cu", "aux_kernels.cu"]
+SOURCES = ["adx_api.cu", "score_sm100.cu", "select_topk.cu", "aux_kernels.cu", "adx_noalloc.cu"]
 HEADERS = ["adx_internal.h", "sm100_ptx.cuh"]
 
 
