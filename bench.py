@@ -281,19 +281,39 @@ def run_group(args, dist):
     p = inputs.group_prefill(c["T"], c["H"], c["d"], c["K"], c["G"], c["B"], c["Hg"],
                              seed=c["seed"], device="cuda")
     ws = indexer.Workspace("cuda")
+    steps = max(2, args.steps // 2)
+    from sparse_attention_token_indexer_b200 import _lib
+    tb, tr = StageTimer(_lib.lib(), steps), StageTimer(_lib.lib(), steps)
+    it = [0]
 
     def step():
+        i = it[0]
+        if 0 <= i < steps:
+            tb.arm(i)
         bank = indexer.group_bank(p["qbar"], p["wbar"], p["k"], c["G"], c["B"], "window",
                                   ws=ws)
+        if 0 <= i < steps:
+            tr.arm(i)
         indexer.bank_refine(p["q"], p["w"], p["k"], bank, c["G"], c["B"], "window", c["K"],
                             ws=ws)
+        tr.disarm()
+        it[0] += 1
 
-    ms, launches = timed(step, max(2, args.steps // 2), args.warmup, dist)
+    for _ in range(args.warmup):
+        it[0] = -1
+        step()
+    it[0] = 0
+    ms, launches = timed(step, steps, 0, dist)
+    stages = {"bank_score_ms": statistics.mean(tb.ms(0, 1)),
+              "bank_select_ms": statistics.mean(tb.ms(2, 3)),
+              "refine_score_ms": statistics.mean(tr.ms(0, 1)),
+              "refine_select_ms": statistics.mean(tr.ms(2, 3))}
     G, B, T = c["G"], c["B"], c["T"]
     scan = sum(g * G for g in range(T // G))
     refine = sum(min(B - G, g * G) * G + G * (G + 1) // 2 for g in range(T // G))
     return dict(ms=ms, launches=launches, scan_pairs=scan, refine_pairs=refine, rows=T,
-                flops=scan * 2 * c["Hg"] * c["d"] + refine * 2 * c["H"] * c["d"])
+                flops=scan * 2 * c["Hg"] * c["d"] + refine * 2 * c["H"] * c["d"], stages=stages,
+                refine_tflops=refine * 2 * c["H"] * c["d"] / (stages["refine_score_ms"] * 1e-3) / 1e12)
 
 
 def run_decode(args, dist):
@@ -308,7 +328,10 @@ def run_decode(args, dist):
     def flat_step():
         indexer.index_decode(q0, w0, prob["k"], seq0, c["K"], k_scale=prob["k_scale"], ws=ws)
 
-    ms_flat, l_flat = timed(flat_step, args.steps, args.warmup, dist)
+    from sparse_attention_token_indexer_b200 import _lib
+    td = StageTimer(_lib.lib(), args.steps)
+    ms_flat, l_flat = timed(flat_step, args.steps, args.warmup, dist, td)
+    dstages = {"score_ms": statistics.mean(td.ms(0, 1)), "select_ms": statistics.mean(td.ms(2, 3))}
     seqs = [inputs.decode_seq_len(prob, r) for r in range(c["G"])]
 
     def cycle():
@@ -324,7 +347,7 @@ def run_decode(args, dist):
     ms_cycle, l_cycle = timed(cycle, max(2, args.steps // 4), args.warmup, dist)
     key_bytes = c["d"] + 4
     return dict(ms_flat=ms_flat, launches_flat=l_flat, ms_cycle=ms_cycle, launches_cycle=l_cycle,
-                bytes_flat=c["Bs"] * c["S"] * key_bytes, steps_per_cycle=c["G"])
+                bytes_flat=c["Bs"] * c["S"] * key_bytes, steps_per_cycle=c["G"], stages=dstages)
 
 
 # ---------------------------------------------------------------------------------------
@@ -477,7 +500,8 @@ def main():
             "refine_pairs": g["refine_pairs"],
             "scores_per_s": (g["scan_pairs"] + g["refine_pairs"]) / (g["ms"] * 1e-3),
             "topk_queries_per_s": g["rows"] / (g["ms"] * 1e-3),
-            "tflops": g["flops"] / (g["ms"] * 1e-3) / 1e12, "gpu_launches": g["launches"]}
+            "tflops": g["flops"] / (g["ms"] * 1e-3) / 1e12, "gpu_launches": g["launches"],
+            "stage_ms": g["stages"], "refine_score_tflops": g["refine_tflops"]}
         dcd = run_decode(args, dist)
         rows["decode_Bs32_S131072_e4m3"] = {
             "ms_per_step": dcd["ms_flat"],
@@ -485,7 +509,8 @@ def main():
             "topk_queries_per_s": DECODE["Bs"] / (dcd["ms_flat"] * 1e-3),
             "hbm_gbs": dcd["bytes_flat"] / (dcd["ms_flat"] * 1e-3) / 1e9,
             "hbm_frac": dcd["bytes_flat"] / (dcd["ms_flat"] * 1e-3) / 1e9 / pk["hbm"],
-            "gpu_launches": dcd["launches_flat"]}
+            "score_kernel_hbm_gbs": dcd["bytes_flat"] / (dcd["stages"]["score_ms"] * 1e-3) / 1e9,
+            "stage_ms": dcd["stages"], "gpu_launches": dcd["launches_flat"]}
         rows["decode_bank_reuse_cycle16"] = {
             "ms_per_cycle": dcd["ms_cycle"],
             "ms_per_step": dcd["ms_cycle"] / dcd["steps_per_cycle"],
