@@ -125,7 +125,6 @@ adx_status check_operands(const adx_operands* o, bool decode) {
 
 bool fp8_keys(const adx_operands* o) { return o->k_dtype == ADX_E4M3; }
 int row_bytes(const adx_operands* o) { return o->d * (fp8_keys(o) ? 1 : 2); }
-bool quantise_q(const adx_operands* o) { return o->q_dtype == ADX_BF16 && o->k_dtype == ADX_E4M3; }
 
 // split of a long row into segments for a two-stage select (few long rows)
 void plan_split(int64_t rows, int64_t n, int K, int& n_seg, int& seg_len) {
@@ -142,32 +141,59 @@ void plan_split(int64_t rows, int64_t n, int K, int& n_seg, int& seg_len) {
 }
 
 // ------------------------------------------------------------------------------------
+// query preparation: the scoring kernel reads prepared query rows (gate-folded where all
+// gates of the row are >= 0, else as given; e4m3 with per-row scales for e4m3 keys)
+// ------------------------------------------------------------------------------------
+struct Prepared {
+  const void* q = nullptr;
+  const float* q_scale = nullptr;
+  const int8_t* fold = nullptr;
+};
+
+size_t ws_prepare(const adx_operands* o, int64_t R) {
+  const bool out8 = fp8_keys(o);
+  return align_up(static_cast<size_t>(R) * o->H * o->d * (out8 ? 1 : 2), kAlign) +
+         (out8 ? align_up(static_cast<size_t>(R) * 4, kAlign) : 0) +
+         align_up(static_cast<size_t>(R), kAlign);
+}
+
+// R rows of q / q_scale / w starting at the given pointers.
+adx_status prepare(const adx_operands* o, const void* q, const float* q_scale, const float* w,
+                   int64_t R, Carve& cv, cudaStream_t s, Prepared& out) {
+  const bool in8 = o->q_dtype == ADX_E4M3, out8 = fp8_keys(o);
+  void* qo = cv.take<uint8_t>(static_cast<size_t>(R) * o->H * o->d * (out8 ? 1 : 2));
+  float* so = out8 ? cv.take<float>(static_cast<size_t>(R) * 4) : nullptr;
+  int8_t* fl = cv.take<int8_t>(static_cast<size_t>(R));
+  if (counted(launch_prepare_q(q, q_scale, in8, out8, w, R, o->H, o->d, qo, so, fl, s)) !=
+      cudaSuccess)
+    return ADX_ECUDA;
+  out.q = qo;
+  out.q_scale = so;
+  out.fold = fl;
+  return ADX_OK;
+}
+
+// ------------------------------------------------------------------------------------
 // building blocks
 // ------------------------------------------------------------------------------------
 struct ScorePlan {
   ScoreArgs a{};
   bool fp8 = false;
   int H = 0, d = 0, tok = 0;
-  const void* qf = nullptr;  // gate-folded bf16 queries (rows with neg_row == 0), or null
 };
 
-// Workspace bytes of the gate-folded copy of R bf16 query rows.
-size_t ws_fold(int64_t R, int H, int d) {
-  return align_up(static_cast<size_t>(R) * H * d * 2, kAlign) + align_up(static_cast<size_t>(R), kAlign);
-}
-
-// bf16 queries against bf16 keys: writes w-folded queries and per-row sign flags into the
-// workspace and records them in the plan.
-adx_status prepare_fold(ScorePlan& p, const void* q, const float* w, int64_t R, Carve& cv,
-                        cudaStream_t s) {
-  uint16_t* qf = cv.take<uint16_t>(static_cast<size_t>(R) * p.H * p.d * 2);
-  int8_t* neg = cv.take<int8_t>(static_cast<size_t>(R));
-  if (counted(launch_fold_gates_bf16(static_cast<const uint16_t*>(q), w, R, p.H, p.d, qf, neg,
-                                     s)) != cudaSuccess)
-    return ADX_ECUDA;
-  p.qf = qf;
-  p.a.neg_row = neg;
-  return ADX_OK;
+ScorePlan base_plan(const adx_operands* o, const Prepared& pq, int tok) {
+  ScorePlan p;
+  p.fp8 = fp8_keys(o);
+  p.H = o->H;
+  p.d = o->d;
+  p.tok = tok;
+  p.a.w = o->w;
+  p.a.q_scale = pq.q_scale;
+  p.a.k_scale = o->k_scale;
+  p.a.fold_flag = pq.fold;
+  p.a.timeout_ns = kTimeoutNs;
+  return p;
 }
 
 // Chooses the key-chunk size and the persistent grid for a score launch.
@@ -175,7 +201,6 @@ void finish_plan(ScorePlan& p, int64_t max_tiles_per_block) {
   const int bps = score_blocks_per_sm(p.fp8, p.H, p.d, p.tok);
   const int grid_cap = std::max(1, sm_count() * std::max(bps, 1));
   const int64_t blocks = static_cast<int64_t>(p.a.row_blocks_per_batch) * p.a.n_batches;
-  // aim for >= 4 items per CTA, chunks of 8..32 tiles
   int64_t chunk = max_tiles_per_block;
   const int64_t want_items = 4ll * grid_cap;
   if (blocks * ((max_tiles_per_block + chunk - 1) / chunk) < want_items)
@@ -189,23 +214,17 @@ void finish_plan(ScorePlan& p, int64_t max_tiles_per_block) {
 
 adx_status run_score(const ScorePlan& p, const void* q_codes, const void* keys, int64_t key_rows,
                      cudaStream_t s) {
-  CUtensorMap tq, tqf, tk;
+  CUtensorMap tq, tk;
   const int n = p.tok * p.H;
   if (!encode_rows(&tq, q_codes, p.fp8, p.d, static_cast<int64_t>(p.a.R) * p.H, n))
     return ADX_EINVAL;
-  if (p.qf != nullptr) {
-    if (!encode_rows(&tqf, p.qf, false, p.d, static_cast<int64_t>(p.a.R) * p.H, n))
-      return ADX_EINVAL;
-  } else {
-    tqf = tq;
-  }
   if (!encode_rows(&tk, keys, p.fp8, p.d, key_rows, kTileM)) return ADX_EINVAL;
   if (p.a.n_items <= 0) return ADX_OK;
   const int bps = score_blocks_per_sm(p.fp8, p.H, p.d, p.tok);
   const int grid = std::min<int64_t>(p.a.n_items, static_cast<int64_t>(sm_count()) * bps);
   if (grid <= 0) return ADX_EUNSUPPORTED;
   mark(0, s);
-  const cudaError_t e = counted(launch_score(tq, tqf, tk, p.a, p.fp8, p.H, p.d, p.tok, grid, s));
+  const cudaError_t e = counted(launch_score(tq, tk, p.a, p.fp8, p.H, p.d, p.tok, grid, s));
   mark(1, s);
   if (e == cudaErrorNotSupported) return ADX_EUNSUPPORTED;
   return e == cudaSuccess ? ADX_OK : ADX_ECUDA;
@@ -263,11 +282,8 @@ adx_status run_select(SelectArgs a, int64_t n_max, Carve& cv, DeviceStatus* st, 
 }
 
 // ---- flat prefill ------------------------------------------------------------------
-bool foldable(const adx_operands* o) { return o->q_dtype == ADX_BF16 && o->k_dtype == ADX_BF16; }
-
 size_t ws_flat(const adx_operands* o, int K, bool scores_external) {
-  size_t b = kStatusBytes;
-  if (foldable(o)) b += ws_fold(o->T, o->H, o->d);
+  size_t b = kStatusBytes + ws_prepare(o, o->T);
   if (!scores_external) b += align_up(static_cast<size_t>(o->T) * ld_for(o->S) * 4, kAlign);
   b += select_scratch_bytes(o->T, o->S, K);
   return b;
@@ -276,18 +292,13 @@ size_t ws_flat(const adx_operands* o, int K, bool scores_external) {
 adx_status run_flat(const adx_operands* o, int K, int32_t* topk_idx, float* topk_score,
                     float* scores_ext, int64_t scores_ld, Carve& cv, DeviceStatus* st,
                     cudaStream_t s) {
-  const bool fp8 = fp8_keys(o);
+  Prepared pq;
+  adx_status r = prepare(o, o->q, o->q_scale, o->w, o->T, cv, s, pq);
+  if (r != ADX_OK) return r;
   const int64_t ld = scores_ext ? scores_ld : ld_for(o->S);
   float* scores = scores_ext ? scores_ext : cv.take<float>(static_cast<size_t>(o->T) * ld * 4);
-  ScorePlan p;
-  p.fp8 = fp8;
-  p.H = o->H;
-  p.d = o->d;
-  p.tok = score_tokens_per_tile(o->H);
+  ScorePlan p = base_plan(o, pq, score_tokens_per_tile(o->H));
   ScoreArgs& a = p.a;
-  a.w = o->w;
-  a.q_scale = o->q_scale;
-  a.k_scale = o->k_scale;
   a.scores = scores;
   a.score_ld = ld;
   a.pos_base = o->q_pos0;
@@ -295,18 +306,13 @@ adx_status run_flat(const adx_operands* o, int K, int32_t* topk_idx, float* topk
   a.R = o->T;
   a.rows_per_batch = o->T;
   a.n_batches = 1;
-  a.key_batch_stride = 0;
   a.keys_per_batch = o->S;
   a.row_blocks_per_batch = (o->T + p.tok - 1) / p.tok;
   a.reverse_order = 1;
   a.status = st;
-  a.timeout_ns = kTimeoutNs;
   const int64_t max_keys = std::min<int64_t>(o->S, o->q_pos0 + o->T);
   finish_plan(p, (max_keys + kTileM - 1) / kTileM);
-  adx_status r = ADX_OK;
-  if (foldable(o) && (r = prepare_fold(p, o->q, o->w, o->T, cv, s)) != ADX_OK) return r;
-  r = run_score(p, o->q, o->k, o->S, s);
-  if (r != ADX_OK) return r;
+  if ((r = run_score(p, pq.q, o->k, o->S, s)) != ADX_OK) return r;
   SelectArgs sa{};
   sa.vals = scores;
   sa.ld = ld;
@@ -324,39 +330,9 @@ adx_status run_flat(const adx_operands* o, int K, int32_t* topk_idx, float* topk
 }
 
 // ---- decode-layout scoring (one query per key cache) --------------------------------
-size_t ws_rowwise_q8(const adx_operands* o) {
-  if (!quantise_q(o)) return 0;
-  return align_up(static_cast<size_t>(o->T) * o->H * o->d, kAlign) +
-         align_up(static_cast<size_t>(o->T) * 4, kAlign);
-}
-
-// Quantises bf16 queries when the keys are e4m3; returns the query codes/scales to use.
-adx_status prepare_q(const adx_operands* o, Carve& cv, const void*& q, const float*& q_scale,
-                     cudaStream_t s) {
-  q = o->q;
-  q_scale = o->q_scale;
-  if (!quantise_q(o)) return ADX_OK;
-  uint8_t* codes = cv.take<uint8_t>(static_cast<size_t>(o->T) * o->H * o->d);
-  float* sc = cv.take<float>(static_cast<size_t>(o->T) * 4);
-  if (counted(launch_quantize_rows_e4m3(static_cast<const uint16_t*>(o->q), o->T,
-                                        static_cast<int64_t>(o->H) * o->d, codes, sc, s)) !=
-      cudaSuccess)
-    return ADX_ECUDA;
-  q = codes;
-  q_scale = sc;
-  return ADX_OK;
-}
-
-ScorePlan rowwise_plan(const adx_operands* o, const float* q_scale, float* scores, int64_t ld) {
-  ScorePlan p;
-  p.fp8 = fp8_keys(o);
-  p.H = o->H;
-  p.d = o->d;
-  p.tok = 1;
+ScorePlan rowwise_plan(const adx_operands* o, const Prepared& pq, float* scores, int64_t ld) {
+  ScorePlan p = base_plan(o, pq, 1);
   ScoreArgs& a = p.a;
-  a.w = o->w;
-  a.q_scale = q_scale;
-  a.k_scale = o->k_scale;
   a.seq_len = o->seq_len;
   a.scores = scores;
   a.score_ld = ld;
@@ -366,12 +342,11 @@ ScorePlan rowwise_plan(const adx_operands* o, const float* q_scale, float* score
   a.key_batch_stride = o->S;
   a.keys_per_batch = o->S;
   a.row_blocks_per_batch = 1;
-  a.timeout_ns = kTimeoutNs;
   return p;
 }
 
 size_t ws_decode(const adx_operands* o, int K) {
-  return kStatusBytes + ws_rowwise_q8(o) + (foldable(o) ? ws_fold(o->T, o->H, o->d) : 0) +
+  return kStatusBytes + ws_prepare(o, o->T) +
          align_up(static_cast<size_t>(o->T) * ld_for(o->S) * 4, kAlign) +
          select_scratch_bytes(o->T, o->S, K);
 }
@@ -409,7 +384,7 @@ adx_status check_bank_args(const adx_operands* o, int G, int B, int mode) {
 
 size_t ws_bank(const adx_operands* o, int G, int B, int mode) {
   const BankShape bs = bank_shape(B, G, mode);
-  return kStatusBytes + ws_rowwise_q8(o) + (foldable(o) ? ws_fold(o->T, o->H, o->d) : 0) +
+  return kStatusBytes + ws_prepare(o, o->T) +
          align_up(static_cast<size_t>(o->T) * ld_for(o->S) * 4, kAlign) +
          select_scratch_bytes(o->T, o->S, bs.bank_k);
 }
@@ -421,8 +396,7 @@ size_t ws_refine(const adx_operands* o, int G, int B, int mode, int K) {
   const bool dec = o->seq_len != nullptr;
   const int64_t ng = dec ? o->T : o->T / G;
   const int64_t rows = dec ? o->T : ng * G;
-  size_t b = kStatusBytes + ws_rowwise_q8(o);
-  if (foldable(o)) b += ws_fold(rows, o->H, o->d);
+  size_t b = kStatusBytes + ws_prepare(o, rows);
   b += align_up(static_cast<size_t>(ng) * bcp * row_bytes(o), kAlign);  // packed keys
   b += align_up(static_cast<size_t>(ng) * bcp * 4, kAlign) * 2;          // scales, positions
   b += align_up(static_cast<size_t>(rows) * bcp * 4, kAlign);             // scores
@@ -518,16 +492,14 @@ adx_status adx_index_decode(const adx_operands* o, int32_t K, int32_t* topk_idx,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   Carve cv(ws);
   DeviceStatus* st = cv.take<DeviceStatus>(kStatusBytes);
-  const void* q;
-  const float* q_scale;
-  if ((r = prepare_q(o, cv, q, q_scale, s)) != ADX_OK) return r;
+  Prepared pq;
+  if ((r = prepare(o, o->q, o->q_scale, o->w, o->T, cv, s, pq)) != ADX_OK) return r;
   const int64_t ld = ld_for(o->S);
   float* scores = cv.take<float>(static_cast<size_t>(o->T) * ld * 4);
-  ScorePlan p = rowwise_plan(o, q_scale, scores, ld);
+  ScorePlan p = rowwise_plan(o, pq, scores, ld);
   p.a.status = st;
   finish_plan(p, (o->S + kTileM - 1) / kTileM);
-  if (foldable(o) && (r = prepare_fold(p, o->q, o->w, o->T, cv, s)) != ADX_OK) return r;
-  if ((r = run_score(p, q, o->k, static_cast<int64_t>(o->T) * o->S, s)) != ADX_OK) return r;
+  if ((r = run_score(p, pq.q, o->k, static_cast<int64_t>(o->T) * o->S, s)) != ADX_OK) return r;
   SelectArgs sa{};
   sa.vals = scores;
   sa.ld = ld;
@@ -557,32 +529,21 @@ adx_status adx_group_bank(const adx_operands* o, int32_t G, int32_t B, int32_t m
   const BankShape bs = bank_shape(B, G, mode);
   Carve cv(ws);
   DeviceStatus* st = cv.take<DeviceStatus>(kStatusBytes);
+  Prepared pq;
+  if ((r = prepare(o, o->q, o->q_scale, o->w, o->T, cv, s, pq)) != ADX_OK) return r;
   const int64_t ld = ld_for(o->S);
+  float* scores = cv.take<float>(static_cast<size_t>(o->T) * ld * 4);
   SelectArgs sa{};
   if (dec) {
-    const void* q;
-    const float* q_scale;
-    if ((r = prepare_q(o, cv, q, q_scale, s)) != ADX_OK) return r;
-    float* scores = cv.take<float>(static_cast<size_t>(o->T) * ld * 4);
-    ScorePlan p = rowwise_plan(o, q_scale, scores, ld);
+    ScorePlan p = rowwise_plan(o, pq, scores, ld);
     p.a.status = st;
     finish_plan(p, (o->S + kTileM - 1) / kTileM);
-    if (foldable(o) && (r = prepare_fold(p, o->q, o->w, o->T, cv, s)) != ADX_OK) return r;
-    if ((r = run_score(p, q, o->k, static_cast<int64_t>(o->T) * o->S, s)) != ADX_OK) return r;
-    sa.vals = scores;
+    if ((r = run_score(p, pq.q, o->k, static_cast<int64_t>(o->T) * o->S, s)) != ADX_OK) return r;
     sa.len_mode = 2;
     sa.seq_len = o->seq_len;
   } else {
-    float* scores = cv.take<float>(static_cast<size_t>(o->T) * ld * 4);
-    ScorePlan p;
-    p.fp8 = fp8_keys(o);
-    p.H = o->H;
-    p.d = o->d;
-    p.tok = score_tokens_per_tile(o->H);
+    ScorePlan p = base_plan(o, pq, score_tokens_per_tile(o->H));
     ScoreArgs& a = p.a;
-    a.w = o->w;
-    a.q_scale = o->q_scale;
-    a.k_scale = o->k_scale;
     a.scores = scores;
     a.score_ld = ld;
     a.pos_base = o->q_pos0 + bs.scan_pos_off;
@@ -594,17 +555,15 @@ adx_status adx_group_bank(const adx_operands* o, int32_t G, int32_t B, int32_t m
     a.row_blocks_per_batch = (o->T + p.tok - 1) / p.tok;
     a.reverse_order = 1;
     a.status = st;
-    a.timeout_ns = kTimeoutNs;
     const int64_t last = o->q_pos0 + bs.scan_pos_off + static_cast<int64_t>(o->T - 1) * G;
     const int64_t max_keys = std::max<int64_t>(0, std::min<int64_t>(o->S, last + 1));
     finish_plan(p, std::max<int64_t>(1, (max_keys + kTileM - 1) / kTileM));
-    if (foldable(o) && (r = prepare_fold(p, o->q, o->w, o->T, cv, s)) != ADX_OK) return r;
-    if ((r = run_score(p, o->q, o->k, o->S, s)) != ADX_OK) return r;
-    sa.vals = scores;
+    if ((r = run_score(p, pq.q, o->k, o->S, s)) != ADX_OK) return r;
     sa.len_mode = 1;
     sa.pos_base = o->q_pos0 + bs.scan_pos_off;
     sa.pos_step = G;
   }
+  sa.vals = scores;
   sa.ld = ld;
   sa.rows_per_batch = 1;
   sa.len_cap = o->S;
@@ -638,29 +597,24 @@ adx_status adx_bank_refine(const adx_operands* o, int32_t G, int32_t B, int32_t 
   if (ng * bcp > INT32_MAX) return ADX_EINVAL;
   Carve cv(ws);
   DeviceStatus* st = cv.take<DeviceStatus>(kStatusBytes);
-  const void* q;
-  const float* q_scale;
-  if ((r = prepare_q(o, cv, q, q_scale, s)) != ADX_OK) return r;
   if (rows > 0) {
+    Prepared pq;
+    if ((r = prepare(o, o->q, o->q_scale, o->w, rows, cv, s, pq)) != ADX_OK) return r;
     const int rb = row_bytes(o);
     uint8_t* packed = cv.take<uint8_t>(static_cast<size_t>(ng) * bcp * rb);
     float* pscale = cv.take<float>(static_cast<size_t>(ng) * bcp * 4);
     int32_t* ppos = cv.take<int32_t>(static_cast<size_t>(ng) * bcp * 4);
     float* scores = cv.take<float>(static_cast<size_t>(rows) * bcp * 4);
     if (counted(launch_pack_candidates(o->k, o->k_scale, o->S, dec ? 1 : 0, o->S, bank_idx,
-                               static_cast<int32_t>(ng), bs.width, static_cast<int32_t>(bcp), rb,
-                               packed, fp8_keys(o) ? pscale : nullptr, ppos, s)) != cudaSuccess)
+                                       static_cast<int32_t>(ng), bs.width,
+                                       static_cast<int32_t>(bcp), rb, packed,
+                                       fp8_keys(o) ? pscale : nullptr, ppos, s)) != cudaSuccess)
       return ADX_ECUDA;
     ScorePlan p;
     if (dec) {
-      p = rowwise_plan(o, q_scale, scores, bcp);
+      p = rowwise_plan(o, pq, scores, bcp);
     } else {
-      p.fp8 = fp8_keys(o);
-      p.H = o->H;
-      p.d = o->d;
-      p.tok = score_tokens_per_tile(o->H);
-      p.a.w = o->w;
-      p.a.q_scale = q_scale;
+      p = base_plan(o, pq, score_tokens_per_tile(o->H));
       p.a.scores = scores;
       p.a.score_ld = bcp;
       p.a.pos_base = o->q_pos0;
@@ -669,7 +623,7 @@ adx_status adx_bank_refine(const adx_operands* o, int32_t G, int32_t B, int32_t 
       p.a.rows_per_batch = G;
       p.a.n_batches = static_cast<int32_t>(ng);
       p.a.row_blocks_per_batch = (G + p.tok - 1) / p.tok;
-      p.a.timeout_ns = kTimeoutNs;
+      p.a.round_robin = 1;  // a group's row blocks run together and share its packed keys
     }
     p.a.k_scale = fp8_keys(o) ? pscale : nullptr;
     p.a.key_pos = ppos;
@@ -677,8 +631,7 @@ adx_status adx_bank_refine(const adx_operands* o, int32_t G, int32_t B, int32_t 
     p.a.keys_per_batch = static_cast<int32_t>(bcp);
     p.a.status = st;
     finish_plan(p, bcp / kTileM);
-    if (foldable(o) && (r = prepare_fold(p, q, o->w, rows, cv, s)) != ADX_OK) return r;
-    if ((r = run_score(p, q, packed, ng * bcp, s)) != ADX_OK) return r;
+    if ((r = run_score(p, pq.q, packed, ng * bcp, s)) != ADX_OK) return r;
     SelectArgs sa{};
     sa.vals = scores;
     sa.ld = bcp;

@@ -33,7 +33,7 @@ struct ScoreArgs {
   const float* k_scale;    // [n_batches * key_batch_stride] or null
   const int32_t* key_pos;  // [n_batches * key_batch_stride] or null
   const int32_t* seq_len;  // [n_batches] or null
-  const int8_t* neg_row;   // [R]: 1 = row has a negative gate; null = no folded queries
+  const int8_t* fold_flag; // [R]: 1 = the row's queries carry its gates already; null = none do
   float* scores;           // [R, score_ld]
   int64_t score_ld;
   int64_t pos_base;
@@ -48,6 +48,10 @@ struct ScoreArgs {
   int32_t chunk_tiles;
   int32_t n_items;
   int32_t reverse_order;
+  // 1: CTA c takes whole row blocks c, c + grid, ... (for equal-length row blocks: the row
+  // blocks of one key batch then run at the same time and share its keys through L2);
+  // 0: balanced contiguous ranges of (row block, key tile) pairs.
+  int32_t round_robin;
   DeviceStatus* status;
   uint64_t timeout_ns;
 };
@@ -79,17 +83,12 @@ struct SelectArgs {
 };
 
 // Launchers (return a cudaError_t from the launch).
-// tm_qf maps the gate-folded queries (used for row blocks whose rows all have neg_row == 0);
-// pass tm_q again when there are none.
-cudaError_t launch_score(const CUtensorMap& tm_q, const CUtensorMap& tm_qf, const CUtensorMap& tm_k,
-                         const ScoreArgs& a, bool fp8, int H, int d, int tok, int grid,
-                         cudaStream_t s);
+cudaError_t launch_score(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const ScoreArgs& a,
+                         bool fp8, int H, int d, int tok, int grid, cudaStream_t s);
 int score_tokens_per_tile(int H);  // tokens per N tile for a head count (0 = unsupported)
 bool score_config_supported(bool fp8, int H, int d);
 // Launches one to three kernels (row-length classes); *launched receives how many.
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launched);
-cudaError_t launch_quantize_rows_e4m3(const uint16_t* x_bf16, int64_t rows, int64_t cols,
-                                      uint8_t* codes, float* scale, cudaStream_t s);
 cudaError_t launch_pack_candidates(const void* k, const float* k_scale, int64_t key_batch_stride,
                                    int32_t per_group_keys, int32_t S_valid, const int32_t* cand,
                                    int32_t n_groups, int32_t n_cand, int32_t n_cand_pad,
@@ -100,7 +99,10 @@ cudaError_t launch_fill_post_anchor(int32_t* bank, int32_t n_groups, int32_t ban
                                     int32_t pos_step, const int32_t* seq_len, int32_t start_off,
                                     cudaStream_t s);
 int score_blocks_per_sm(bool fp8, int H, int d, int tok);
-cudaError_t launch_fold_gates_bf16(const uint16_t* q, const float* w, int64_t rows, int H, int d,
-                                   uint16_t* qf, int8_t* neg_row, cudaStream_t s);
+// Writes the prepared query rows (gate-folded where all gates are >= 0, else as given), with
+// fold flags and, for e4m3 output, one scale per row.
+cudaError_t launch_prepare_q(const void* q, const float* q_scale, bool in_e4m3, bool out_e4m3,
+                             const float* w, int64_t rows, int H, int d, void* q_out,
+                             float* q_scale_out, int8_t* fold_flag, cudaStream_t s);
 
 }  // namespace adx

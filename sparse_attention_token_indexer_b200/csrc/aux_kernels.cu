@@ -1,10 +1,10 @@
 // Small memory-bound helpers of the indexer path:
-//  * per-token FP8-e4m3 quantisation of bf16 queries (decode with an e4m3 key cache);
 //  * candidate packing: gather each group's candidate key rows (and scales, positions) into
 //    a contiguous block so that refinement streams them with tiled TMA loads
 //    (ADIndex, arXiv 2611.12956v1, §4.3 Eq. (14): C_i = bank U post-anchor positions);
-//  * gate folding for bf16 queries with non-negative gates (w * ReLU(x) = ReLU(w * x)), so
-//    the scoring epilogue needs no gate loads;
+//  * query preparation: gate folding for rows with non-negative gates
+//    (w * ReLU(x) = ReLU(w * x)), so the scoring epilogue needs no gate loads for them, and
+//    e4m3 (re)quantisation;
 //  * post-anchor columns of a bank: the positions every member of a group adds to the
 //    shared bank (Eq. (14)), stored beside the bank so refinement needs no extra inputs.
 #include <cuda_bf16.h>
@@ -17,38 +17,6 @@
 namespace adx {
 
 namespace {
-
-constexpr int kQuantThreads = 256;
-
-__global__ void __launch_bounds__(kQuantThreads)
-quantize_rows_kernel(const __nv_bfloat16* __restrict__ x, int64_t cols, uint8_t* __restrict__ codes,
-                     float* __restrict__ scale) {
-  __shared__ float red[kQuantThreads / 32];
-  const int64_t row = blockIdx.x;
-  const __nv_bfloat16* xr = x + row * cols;
-  float amax = 0.f;
-  for (int64_t i = threadIdx.x; i < cols; i += kQuantThreads)
-    amax = fmaxf(amax, fabsf(__bfloat162float(xr[i])));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    float v = threadIdx.x < kQuantThreads / 32 ? red[threadIdx.x] : 0.f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    if (threadIdx.x == 0) red[0] = v;
-  }
-  __syncthreads();
-  const float m = red[0];
-  const float s = m > 0.f ? m / 448.f : 1.f;
-  if (threadIdx.x == 0) scale[row] = s;
-  uint8_t* cr = codes + row * cols;
-  for (int64_t i = threadIdx.x; i < cols; i += kQuantThreads) {
-    const float y = __bfloat162float(xr[i]) / s;
-    cr[i] = static_cast<uint8_t>(__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3));
-  }
-}
 
 // One thread per 16-byte piece of a packed candidate row.
 __global__ void pack_kernel(const uint8_t* __restrict__ k, const float* __restrict__ k_scale,
@@ -88,51 +56,110 @@ __global__ void fill_post_kernel(int32_t* bank, int32_t n_groups, int32_t bank_w
   bank[static_cast<int64_t>(g) * bank_w + first_col + j] = static_cast<int32_t>(anchor + start_off + j);
 }
 
-// q'[r, j, :] = bf16(w[r, j] * q[r, j, :]) for rows whose gates are all >= 0, where
-// w * ReLU(q . k) = ReLU((w q) . k); neg_row[r] = 1 marks rows with a negative gate (their
-// folded copy is not used).
+// Query preparation for the scoring kernel, one CTA per query row. A row whose gates are all
+// >= 0 is stored gate-folded, w[r, j] * q[r, j, :], because w * ReLU(q . k) = ReLU((w q) . k)
+// for w >= 0; the scoring epilogue then needs no gates for it. Any other row is stored as
+// given. fold_flag[r] = 1 marks a folded row. Output codes are bf16 (bf16 input) or e4m3 with
+// a new per-row scale (e4m3 input, or bf16 input quantised for an e4m3 key cache).
+template <bool IN_E4M3>
+__device__ __forceinline__ void load8(const void* q, int64_t e, float sin, float (&x)[8]) {
+  if constexpr (IN_E4M3) {
+    const uint2 v = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint8_t*>(q) + e);
+    const __nv_fp8_e4m3* c = reinterpret_cast<const __nv_fp8_e4m3*>(&v);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) x[u] = static_cast<float>(c[u]) * sin;
+  } else {
+    const uint4 v = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(q) + e);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float2 f = __bfloat1622float2(h[u]);
+      x[2 * u] = f.x;
+      x[2 * u + 1] = f.y;
+    }
+  }
+}
+
+template <bool IN_E4M3, bool OUT_E4M3>
 __global__ void __launch_bounds__(256)
-fold_gates_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w, int H, int d,
-                  __nv_bfloat16* __restrict__ qf, int8_t* __restrict__ neg_row) {
+prepare_q_kernel(const void* __restrict__ q_in, const float* __restrict__ q_scale_in,
+                 const float* __restrict__ w, int H, int d, void* __restrict__ q_out,
+                 float* __restrict__ q_scale_out, int8_t* __restrict__ fold_flag) {
+  __shared__ float red[8];
   const int64_t r = blockIdx.x;
   const float* wr = w + r * H;
   int neg = 0;
   for (int j = threadIdx.x; j < H; j += blockDim.x) neg |= wr[j] < 0.f;
-  neg = __syncthreads_or(neg);
-  if (threadIdx.x == 0) neg_row[r] = static_cast<int8_t>(neg != 0);
-  if (neg) return;
+  const bool fold = __syncthreads_or(neg) == 0;
+  if (threadIdx.x == 0) fold_flag[r] = fold ? 1 : 0;
   const int64_t n = static_cast<int64_t>(H) * d;
-  const uint4* src = reinterpret_cast<const uint4*>(q + r * n);
-  uint4* dst = reinterpret_cast<uint4*>(qf + r * n);
-  for (int64_t i = threadIdx.x; i < n / 8; i += blockDim.x) {
-    const float g = wr[(i * 8) / d];
-    uint4 v = src[i];
-    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float2 f = __bfloat1622float2(h[u]);
-      h[u] = __floats2bfloat162_rn(f.x * g, f.y * g);
+  const int64_t base = r * n;
+  const float sin = IN_E4M3 ? q_scale_in[r] : 1.f;
+  if constexpr (IN_E4M3 && OUT_E4M3) {
+    if (!fold) {  // keep the given codes and scale
+      const uint2* in = reinterpret_cast<const uint2*>(reinterpret_cast<const uint8_t*>(q_in) + base);
+      uint2* out = reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(q_out) + base);
+      for (int64_t i = threadIdx.x; i < n / 8; i += blockDim.x) out[i] = in[i];
+      if (threadIdx.x == 0) q_scale_out[r] = sin;
+      return;
     }
-    dst[i] = v;
+  }
+  // element groups of 8 share one head (d is a multiple of 8)
+  float sc = 1.f;
+  if constexpr (OUT_E4M3) {
+    float amax = 0.f;
+    for (int64_t i = threadIdx.x; i < n / 8; i += blockDim.x) {
+      float x[8];
+      load8<IN_E4M3>(q_in, base + i * 8, sin, x);
+      const float g = fold ? wr[(i * 8) / d] : 1.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) amax = fmaxf(amax, fabsf(x[u] * g));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    float m = 0.f;
+    for (int i2 = 0; i2 < static_cast<int>(blockDim.x / 32); ++i2) m = fmaxf(m, red[i2]);
+    sc = m > 0.f ? m / 448.f : 1.f;
+    if (threadIdx.x == 0) q_scale_out[r] = sc;
+  }
+  for (int64_t i = threadIdx.x; i < n / 8; i += blockDim.x) {
+    float x[8];
+    load8<IN_E4M3>(q_in, base + i * 8, sin, x);
+    const float g = fold ? wr[(i * 8) / d] : 1.f;
+    if constexpr (OUT_E4M3) {
+      uint2 v;
+      uint8_t* c = reinterpret_cast<uint8_t*>(&v);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        c[u] = static_cast<uint8_t>(__nv_cvt_float_to_fp8((x[u] * g) / sc, __NV_SATFINITE, __NV_E4M3));
+      reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(q_out) + base)[i] = v;
+    } else {
+      uint4 v;
+      __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) h[u] = __floats2bfloat162_rn(x[2 * u] * g, x[2 * u + 1] * g);
+      reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(q_out) + base)[i] = v;
+    }
   }
 }
 
 }  // namespace
 
-cudaError_t launch_fold_gates_bf16(const uint16_t* q, const float* w, int64_t rows, int H, int d,
-                                   uint16_t* qf, int8_t* neg_row, cudaStream_t s) {
+cudaError_t launch_prepare_q(const void* q, const float* q_scale, bool in_e4m3, bool out_e4m3,
+                             const float* w, int64_t rows, int H, int d, void* q_out,
+                             float* q_scale_out, int8_t* fold_flag, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
-  fold_gates_kernel<<<static_cast<unsigned>(rows), 256, 0, s>>>(
-      reinterpret_cast<const __nv_bfloat16*>(q), w, H, d, reinterpret_cast<__nv_bfloat16*>(qf),
-      neg_row);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_quantize_rows_e4m3(const uint16_t* x_bf16, int64_t rows, int64_t cols,
-                                      uint8_t* codes, float* scale, cudaStream_t s) {
-  if (rows <= 0) return cudaSuccess;
-  quantize_rows_kernel<<<static_cast<unsigned>(rows), kQuantThreads, 0, s>>>(
-      reinterpret_cast<const __nv_bfloat16*>(x_bf16), cols, codes, scale);
+  const unsigned g = static_cast<unsigned>(rows);
+  if (!in_e4m3 && !out_e4m3)
+    prepare_q_kernel<false, false><<<g, 256, 0, s>>>(q, q_scale, w, H, d, q_out, q_scale_out, fold_flag);
+  else if (in_e4m3 && out_e4m3)
+    prepare_q_kernel<true, true><<<g, 256, 0, s>>>(q, q_scale, w, H, d, q_out, q_scale_out, fold_flag);
+  else if (!in_e4m3 && out_e4m3)
+    prepare_q_kernel<false, true><<<g, 256, 0, s>>>(q, q_scale, w, H, d, q_out, q_scale_out, fold_flag);
+  else
+    return cudaErrorNotSupported;
   return cudaGetLastError();
 }
 

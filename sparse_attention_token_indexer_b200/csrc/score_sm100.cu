@@ -175,6 +175,42 @@ __device__ __forceinline__ void partition(const ScoreArgs& a, int64_t* scan_s, i
   base0 = start < end ? scan_s[1] : 0;
 }
 
+// The sequence of (row block, key tile range) a CTA works through; identical in every role.
+struct WorkIter {
+  int64_t start, end, cum;
+  int bi, nblocks;
+  bool rr;
+
+  template <int TOK>
+  __device__ __forceinline__ bool next(const ScoreArgs& a, Block& x, int& t_lo, int& t_hi) {
+    if (rr) {
+      while (bi < nblocks) {
+        block_info<TOK>(a, bi, x);
+        bi += gridDim.x;
+        if (x.ntiles > 0) {
+          t_lo = 0;
+          t_hi = x.ntiles;
+          return true;
+        }
+      }
+      return false;
+    }
+    while (bi < nblocks && cum < end) {
+      block_info<TOK>(a, bi, x);
+      ++bi;
+      const int64_t lo = max(start - cum, int64_t(0));
+      const int64_t hi = min(end - cum, static_cast<int64_t>(x.ntiles));
+      cum += x.ntiles;
+      if (lo < hi) {
+        t_lo = static_cast<int>(lo);
+        t_hi = static_cast<int>(hi);
+        return true;
+      }
+    }
+    return false;
+  }
+};
+
 __device__ __forceinline__ void raise_timeout(const ScoreArgs& a, int role) {
   if (a.status != nullptr && atomicCAS(&a.status->code, 0, 6 /* ADX_ETIMEOUT */) == 0) {
     a.status->where = kWhereScore;
@@ -233,18 +269,18 @@ __device__ __forceinline__ void reduce_chunk_folded(const float (&v)[C::CW], int
   }
 }
 
-// True when every row of the block has non-negative gates and folded queries exist.
+// True when the queries of every row of the block carry their gates already.
 __device__ __forceinline__ bool block_folded(const ScoreArgs& a, const Block& x) {
-  if (a.neg_row == nullptr) return false;
-  int neg = 0;
-  for (int r = x.row0; r < x.row_end; ++r) neg |= a.neg_row[r];
-  return neg == 0;
+  if (a.fold_flag == nullptr) return false;
+  int all = 1;
+  for (int r = x.row0; r < x.row_end; ++r) all &= a.fold_flag[r];
+  return all != 0;
 }
 
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
-score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qf,
-             const __grid_constant__ CUtensorMap tm_k, const ScoreArgs a) {
+score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+             const ScoreArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -281,21 +317,21 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     *abort_s = 0;
     fence_mbarrier_init();
     tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_qf);
     tma_prefetch_desc(&tm_k);
   }
   if (warp == 1) {
     tmem_alloc(tmem_base_s, C::TMEM_COLS);
     tmem_relinquish();
   }
-  int64_t start, end, base0;
-  int b0;
-  partition<C>(a, scan_s, start, end, b0, base0);  // contains __syncthreads
+  int64_t start = 0, end = 0, base0 = 0;
+  int b0 = blockIdx.x;
+  if (!a.round_robin) partition<C>(a, scan_s, start, end, b0, base0);  // contains __syncthreads
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_base_s;
   const int nblocks = a.row_blocks_per_batch * a.n_batches;
+  const WorkIter work0{start, end, base0, b0, nblocks, a.round_robin != 0};
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -305,26 +341,21 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       uint32_t q_phase = 0;
       bool q_loaded = false;
       uint32_t issued_mask = 0, issued_parity = 0;
-      int64_t cum = base0;
-      for (int bi = b0; bi < nblocks && cum < end && !*abort_s; ++bi) {
-        Block x;
-        block_info<C::TOK>(a, bi, x);
-        const int64_t t_lo = max(start - cum, int64_t(0));
-        const int64_t t_hi = min(end - cum, static_cast<int64_t>(x.ntiles));
-        cum += x.ntiles;
-        if (t_lo >= t_hi) continue;
+      WorkIter work = work0;
+      Block x;
+      int t_lo, t_hi;
+      while (!*abort_s && work.next<C::TOK>(a, x, t_lo, t_hi)) {
         if (q_loaded) {
           if (!mbar_wait(q_empty, q_phase ^ 1u, abort_s, a.timeout_ns)) break;
         }
-        const CUtensorMap* qmap = block_folded(a, x) ? &tm_qf : &tm_q;
         mbar_arrive_expect_tx(q_full, C::QBYTES);
 #pragma unroll
         for (int kc = 0; kc < C::KC; ++kc)
-          tma_load_2d(q_s + kc * C::N * 128, qmap, q_full, kc * C::ELEMS_PER_CHUNK,
+          tma_load_2d(q_s + kc * C::N * 128, &tm_q, q_full, kc * C::ELEMS_PER_CHUNK,
                       x.row0 * C::H);
         q_loaded = true;
         q_phase ^= 1u;
-        for (int t = static_cast<int>(t_lo); t < static_cast<int>(t_hi); ++t) {
+        for (int t = t_lo; t < t_hi; ++t) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_s, a.timeout_ns)) break;
           mbar_arrive_expect_tx(&full[stage], C::KBYTES);
           const int32_t y = static_cast<int32_t>(x.key_row0 + static_cast<int64_t>(t) * kTileM);
@@ -356,20 +387,16 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       int acc = 0;
       uint32_t acc_phase = 0;
       bool any = false;
-      int64_t cum = base0;
-      for (int bi = b0; bi < nblocks && cum < end && !*abort_s; ++bi) {
-        Block x;
-        block_info<C::TOK>(a, bi, x);
-        const int64_t t_lo = max(start - cum, int64_t(0));
-        const int64_t t_hi = min(end - cum, static_cast<int64_t>(x.ntiles));
-        cum += x.ntiles;
-        if (t_lo >= t_hi) continue;
+      WorkIter work = work0;
+      Block x;
+      int t_lo, t_hi;
+      while (!*abort_s && work.next<C::TOK>(a, x, t_lo, t_hi)) {
         if (!mbar_wait(q_full, q_phase, abort_s, a.timeout_ns)) break;
         q_phase ^= 1u;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(q_s);
         bool ok = true;
-        for (int t = static_cast<int>(t_lo); t < static_cast<int>(t_hi); ++t) {
+        for (int t = t_lo; t < t_hi; ++t) {
           if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_s, a.timeout_ns) ||
               !mbar_wait(&full[stage], phase, abort_s, a.timeout_ns)) {
             ok = false;
@@ -415,16 +442,13 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     float* w_w = w_s + ew * C::NG;            // this warp's copy of the gates
     const int tok0 = C::BUF_SPLIT ? 0 : grp * C::TOKG;  // first token this warp reduces
     int64_t gi = 0;                           // tile counter of this CTA (selects the buffer)
-    int64_t cum = base0;
-    for (int bi = b0; bi < nblocks && cum < end && !*abort_s; ++bi) {
-      Block x;
-      block_info<C::TOK>(a, bi, x);
-      const int64_t t_lo = max(start - cum, int64_t(0));
-      const int64_t t_hi = min(end - cum, static_cast<int64_t>(x.ntiles));
-      cum += x.ntiles;
-      if (t_lo >= t_hi) continue;
-      // gates of this block's rows, with the per-token query scale folded in (not needed
-      // when the queries carry their gates already)
+    WorkIter work = work0;
+    Block x;
+    int t_lo, t_hi;
+    while (!*abort_s && work.next<C::TOK>(a, x, t_lo, t_hi)) {
+      // Gates of this block's rows with the per-token query scale folded in; a row whose
+      // queries carry their gates already gets gate 1. When every row of the block does, the
+      // epilogue needs no gates at all and applies only the per-token scale.
       const bool folded = block_folded(a, x);
       __syncwarp();
       const int rowg = x.row0 + tok0;
@@ -432,19 +456,24 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         const int r = rowg + i / C::H;
         float wv = 0.f;
         if (r < x.row_end) {
-          wv = a.w[static_cast<int64_t>(r) * C::H + (i % C::H)];
+          const bool fr = a.fold_flag != nullptr && a.fold_flag[r];
+          wv = fr ? 1.f : a.w[static_cast<int64_t>(r) * C::H + (i % C::H)];
           if (a.q_scale != nullptr) wv *= a.q_scale[r];
         }
         w_w[i] = wv;
       }
       __syncwarp();
       int32_t rpos[C::TOKG];
+      float tokf[C::TOKG];
 #pragma unroll
-      for (int tt = 0; tt < C::TOKG; ++tt)
-        rpos[tt] = (rowg + tt < x.row_end) ? static_cast<int32_t>(row_position(a, rowg + tt)) : -1;
+      for (int tt = 0; tt < C::TOKG; ++tt) {
+        const bool in = rowg + tt < x.row_end;
+        rpos[tt] = in ? static_cast<int32_t>(row_position(a, rowg + tt)) : -1;
+        tokf[tt] = (folded && in && a.q_scale != nullptr) ? a.q_scale[rowg + tt] : 1.f;
+      }
 
       bool ok = true;
-      for (int t = static_cast<int>(t_lo); t < static_cast<int>(t_hi); ++t, ++gi) {
+      for (int t = t_lo; t < t_hi; ++t, ++gi) {
         const int acc = static_cast<int>(gi % C::ACC);
         if (C::BUF_SPLIT && acc != grp) continue;  // the other warpgroup's tile
         const uint32_t acc_phase = static_cast<uint32_t>((gi / C::ACC) & 1);
@@ -512,7 +541,7 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll
             for (int p = 0; p < C::NP; ++p) sc += part[tt][p].x + part[tt][p].y;
             const bool vis = key_ok && kpos <= rpos[tt];
-            a.scores[static_cast<int64_t>(r) * a.score_ld + c] = vis ? ks * sc : -INFINITY;
+            a.scores[static_cast<int64_t>(r) * a.score_ld + c] = vis ? (ks * tokf[tt]) * sc : -INFINITY;
           }
         }
       }
@@ -531,12 +560,12 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 }
 
 template <class C>
-cudaError_t launch_cfg(const CUtensorMap& tm_q, const CUtensorMap& tm_qf, const CUtensorMap& tm_k,
-                       const ScoreArgs& a, int grid, cudaStream_t s) {
+cudaError_t launch_cfg(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const ScoreArgs& a,
+                       int grid, cudaStream_t s) {
   auto kern = score_kernel<C>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<grid, C::THREADS, C::SMEM, s>>>(tm_q, tm_qf, tm_k, a);
+  kern<<<grid, C::THREADS, C::SMEM, s>>>(tm_q, tm_k, a);
   return cudaGetLastError();
 }
 
@@ -571,12 +600,11 @@ bool score_config_supported(bool fp8, int H, int d) {
 
 // tok: tokens per N tile; either score_tokens_per_tile(H) (prefill) or 1 (one query per
 // key batch: decode and its bank refresh).
-cudaError_t launch_score(const CUtensorMap& tm_q, const CUtensorMap& tm_qf, const CUtensorMap& tm_k,
-                         const ScoreArgs& a, bool fp8, int H, int d, int tok, int grid,
-                         cudaStream_t s) {
+cudaError_t launch_score(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const ScoreArgs& a,
+                         bool fp8, int H, int d, int tok, int grid, cudaStream_t s) {
 #define ADX_CASE(FP, HH, TT, DD)                                                        \
   if (fp8 == FP && H == HH && tok == TT && d == DD)                                     \
-    return launch_cfg<Cfg<HH, TT, (FP ? DD : 2 * DD), FP>>(tm_q, tm_qf, tm_k, a, grid, s);
+    return launch_cfg<Cfg<HH, TT, (FP ? DD : 2 * DD), FP>>(tm_q, tm_k, a, grid, s);
   ADX_SCORE_CONFIGS(ADX_CASE)
 #undef ADX_CASE
   return cudaErrorNotSupported;

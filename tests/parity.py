@@ -55,17 +55,16 @@ def check_topk(got_idx, cand_pos, cand_scores, cand_floor, K, rtol, got_scores=N
     where = {int(p): i for i, p in enumerate(cand_pos)}
     missing = [int(p) for p in valid if int(p) not in where]
     assert not missing, f"{what}: indices outside the candidate set: {missing[:5]}"
-    if n <= K:
-        return
-    order = np.lexsort((np.asarray(cand_pos), -np.asarray(cand_scores)))
-    ref_set = set(int(cand_pos[i]) for i in order[:K])
-    theta = cand_scores[order[K - 1]]
-    for p in set(valid.tolist()) ^ ref_set:
-        i = where[p]
-        tol = rtol * max(abs(cand_scores[i]), cand_floor[i])
-        assert abs(cand_scores[i] - theta) <= tol, (
-            f"{what}: key {p} (oracle score {cand_scores[i]:.6g}) differs from the oracle set "
-            f"but is not within {tol:.3g} of the K-th score {theta:.6g}")
+    if n > K:
+        order = np.lexsort((np.asarray(cand_pos), -np.asarray(cand_scores)))
+        ref_set = set(int(cand_pos[i]) for i in order[:K])
+        theta = cand_scores[order[K - 1]]
+        for p in set(valid.tolist()) ^ ref_set:
+            i = where[p]
+            tol = rtol * max(abs(cand_scores[i]), cand_floor[i])
+            assert abs(cand_scores[i] - theta) <= tol, (
+                f"{what}: key {p} (oracle score {cand_scores[i]:.6g}) differs from the oracle "
+                f"set but is not within {tol:.3g} of the K-th score {theta:.6g}")
     if got_scores is not None:
         gs = np.asarray(got_scores, dtype=np.float64)[: m]
         idx = [where[int(p)] for p in valid]
