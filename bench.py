@@ -316,7 +316,7 @@ def run_group(args, dist):
                 refine_tflops=refine * 2 * c["H"] * c["d"] / (stages["refine_score_ms"] * 1e-3) / 1e12)
 
 
-def run_decode(args, dist):
+def run_decode(args, dist, cycle=True):
     from sparse_attention_token_indexer_b200 import indexer, inputs
     c = DECODE
     prob = inputs.decode_problem(c["Bs"], c["S"], c["H"], c["d"], c["K"], c["Hg"],
@@ -332,6 +332,10 @@ def run_decode(args, dist):
     td = StageTimer(_lib.lib(), args.steps)
     ms_flat, l_flat = timed(flat_step, args.steps, args.warmup, dist, td)
     dstages = {"score_ms": statistics.mean(td.ms(0, 1)), "select_ms": statistics.mean(td.ms(2, 3))}
+    key_bytes = c["d"] + 4
+    if not cycle:
+        return dict(ms_flat=ms_flat, launches_flat=l_flat, bytes_flat=c["Bs"] * c["S"] * key_bytes,
+                    stages=dstages)
     seqs = [inputs.decode_seq_len(prob, r) for r in range(c["G"])]
 
     def cycle():
@@ -402,8 +406,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--rows", action="store_true", help="also time the other hot-path rows")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--case", default="flat", choices=["flat", "flat_small"],
-                    help="flat_small: T = 8192, for profiler captures")
+    ap.add_argument("--case", default="flat", choices=["flat", "flat_small", "decode"],
+                    help="flat_small: T = 8192, for profiler captures; decode: the decode "
+                         "workload alone (with --quick)")
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "e4m3"])
     ap.add_argument("--quick", action="store_true",
                     help="time the kernels only (no e2e, rows or CPU baseline): for profiling")
@@ -453,6 +458,15 @@ def main():
     build.build()
     pk = peaks()
     clocks = Clocks(dist.local)
+    if args.case == "decode" and args.quick:
+        dcd = run_decode(args, dist, cycle=False)
+        if dist.rank == 0:
+            print(json.dumps({"case": "decode", "ms_per_step": dcd["ms_flat"],
+                              "stage_ms": dcd["stages"],
+                              "hbm_gbs": dcd["bytes_flat"] / (dcd["ms_flat"] * 1e-3) / 1e9,
+                              "gpu_launches": dcd["launches_flat"]}), flush=True)
+        dist.close()
+        return
     flat = run_flat(args, dist, args.dtype, clocks)
     clk = clocks.summary()
     if args.quick:

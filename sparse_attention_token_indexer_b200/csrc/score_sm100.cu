@@ -472,8 +472,26 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         tokf[tt] = (folded && in && a.q_scale != nullptr) ? a.q_scale[rowg + tt] : 1.f;
       }
 
+      // per-key scale and position of the next tile, loaded one tile ahead so their
+      // latency hides behind the current tile's wait and reduction
+      auto key_meta = [&](int t, float& ks, int64_t& kpos) {
+        const int c = t * kTileM + m;
+        kpos = c;
+        ks = 1.f;
+        if (c < x.nkeys) {
+          const int64_t kr = x.key_row0 + c;
+          if (a.key_pos != nullptr) kpos = a.key_pos[kr];
+          if (a.k_scale != nullptr) ks = a.k_scale[kr];
+        }
+      };
+      float ks_next;
+      int64_t kpos_next;
+      key_meta(t_lo, ks_next, kpos_next);
       bool ok = true;
       for (int t = t_lo; t < t_hi; ++t, ++gi) {
+        const float ks = ks_next;
+        const int64_t kpos = kpos_next;
+        if (t + 1 < t_hi) key_meta(t + 1, ks_next, kpos_next);
         const int acc = static_cast<int>(gi % C::ACC);
         if (C::BUF_SPLIT && acc != grp) continue;  // the other warpgroup's tile
         const uint32_t acc_phase = static_cast<uint32_t>((gi / C::ACC) & 1);
@@ -487,13 +505,6 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         tc_fence_after();
         const int c = t * kTileM + m;  // key index within the batch
         const bool key_ok = c < x.nkeys;
-        int64_t kpos = c;
-        float ks = 1.f;
-        if (key_ok) {
-          const int64_t kr = x.key_row0 + c;
-          if (a.key_pos != nullptr) kpos = a.key_pos[kr];
-          if (a.k_scale != nullptr) ks = a.k_scale[kr];
-        }
         float2 part[C::TOKG][C::NP];
 #pragma unroll
         for (int tt = 0; tt < C::TOKG; ++tt)
