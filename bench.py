@@ -37,6 +37,7 @@ FLAT = dict(T=16384, H=64, d=128, K=2048, seed=1)
 FLAT_SMALL = dict(T=8192, H=64, d=128, K=2048, seed=1)
 GROUP = dict(T=65536, H=64, d=128, K=2048, G=64, B=8192, Hg=16, seed=2)
 DECODE = dict(Bs=32, S=131072, H=64, d=128, K=2048, Hg=16, B=8192, G=16, seed=3)
+CHUNKED = dict(S=262144, chunk=4096, H=64, d=128, K=2048, G=64, B=8192, Hg=16, seed=4)
 
 
 def flat_pairs(T, q_pos0=0):
@@ -354,6 +355,46 @@ def run_decode(args, dist, cycle=True):
                 bytes_flat=c["Bs"] * c["S"] * key_bytes, steps_per_cycle=c["G"], stages=dstages)
 
 
+def run_chunked(args, dist):
+    """256K-token prefill in query chunks of 4096 against the growing causal key cache, flat
+    and in group mode (window bank, G = 64, B = 8192); one step = all 64 chunks."""
+    from sparse_attention_token_indexer_b200 import indexer, inputs
+    c = CHUNKED
+    S, ch, G = c["S"], c["chunk"], c["G"]
+    st = inputs.AnchorStructure(c["d"], c["seed"], "cuda")
+    k = st.keys(S).to(torch.bfloat16).contiguous()
+    q = torch.empty(S, c["H"], c["d"], dtype=torch.bfloat16, device="cuda")
+    for c0 in range(0, S, 16384):  # generate in slices to bound the fp32 temporaries
+        q[c0:c0 + 16384] = st.queries(16384, c["H"], pos0=c0).to(torch.bfloat16)
+    w = st.gates(S, c["H"])
+    qbar, wbar = inputs.mean_pool_group_queries(q, w, G, c["Hg"])
+    qbar = qbar.to(torch.bfloat16).contiguous()
+    ws = indexer.Workspace("cuda")
+    idx = torch.empty(ch, c["K"], dtype=torch.int32, device="cuda")
+    gpc = ch // G
+
+    def flat_pass():
+        for c0 in range(0, S, ch):
+            _call_prefill({"q": q[c0:c0 + ch], "w": w[c0:c0 + ch], "k": k, "q_scale": None,
+                           "k_scale": None, "q_pos0": c0}, c["K"], idx, ws)
+
+    def group_pass():
+        for c0 in range(0, S, ch):
+            g0 = c0 // G
+            bank = indexer.group_bank(qbar[g0:g0 + gpc], wbar[g0:g0 + gpc], k, G, c["B"],
+                                      "window", q_pos0=c0, ws=ws)
+            indexer.bank_refine(q[c0:c0 + ch], w[c0:c0 + ch], k, bank, G, c["B"], "window",
+                                c["K"], q_pos0=c0, ws=ws)
+
+    ms_flat, l_flat = timed(flat_pass, 1, args.warmup, dist)
+    ms_grp, l_grp = timed(group_pass, 1, args.warmup, dist)
+    pairs = S * (S + 1) // 2
+    scan = sum(g * G for g in range(S // G))
+    refine = sum(min(c["B"] - G, g * G) * G + G * (G + 1) // 2 for g in range(S // G))
+    return dict(ms_flat=ms_flat, ms_group=ms_grp, l_flat=l_flat, l_group=l_grp, pairs=pairs,
+                scan=scan, refine=refine, rows=S)
+
+
 # ---------------------------------------------------------------------------------------
 # the oracle on the host cores
 # ---------------------------------------------------------------------------------------
@@ -525,6 +566,17 @@ def main():
             "hbm_frac": dcd["bytes_flat"] / (dcd["ms_flat"] * 1e-3) / 1e9 / pk["hbm"],
             "score_kernel_hbm_gbs": dcd["bytes_flat"] / (dcd["stages"]["score_ms"] * 1e-3) / 1e9,
             "stage_ms": dcd["stages"], "gpu_launches": dcd["launches_flat"]}
+        ck = run_chunked(args, dist)
+        rows["chunked_prefill_S262144_flat"] = {
+            "ms_per_pass": ck["ms_flat"], "scores_per_s": ck["pairs"] / (ck["ms_flat"] * 1e-3),
+            "topk_queries_per_s": ck["rows"] / (ck["ms_flat"] * 1e-3),
+            "tflops": ck["pairs"] * 2 * CHUNKED["H"] * CHUNKED["d"] / (ck["ms_flat"] * 1e-3) / 1e12,
+            "gpu_launches": ck["l_flat"]}
+        rows["chunked_prefill_S262144_group"] = {
+            "ms_per_pass": ck["ms_group"],
+            "scores_per_s": (ck["scan"] + ck["refine"]) / (ck["ms_group"] * 1e-3),
+            "topk_queries_per_s": ck["rows"] / (ck["ms_group"] * 1e-3),
+            "speedup_vs_flat": ck["ms_flat"] / ck["ms_group"], "gpu_launches": ck["l_group"]}
         rows["decode_bank_reuse_cycle16"] = {
             "ms_per_cycle": dcd["ms_cycle"],
             "ms_per_step": dcd["ms_cycle"] / dcd["steps_per_cycle"],

@@ -271,3 +271,40 @@ def test_full_size_decode_sampled():
         keys = f64(prob["k"][b], prob["k_scale"][b])
         check_topk(idx[b], np.arange(S), ox.score_keys(q64[b], w64[b], keys),
                    score_floor(q64[b], w64[b], keys), K, RTOL["e4m3"], sc[b], f"dfull {b}")
+
+
+@pytest.mark.parametrize("mode", ["window", "paper"])
+def test_group_mode_on_a_later_chunk(mode):
+    """Group mode for one query chunk of a longer prefix (q_pos0 > 0), as chunked prefill
+    runs it; includes an incomplete trailing group."""
+    S, T, q_pos0, G, B, K, Hg = 3000, 64 * 9 + 21, 2300, 64, 512, 128, 16
+    p = _to_cuda(inputs.anchor_prefill(T, H=64, d=128, K=K, seed=23, S=S, q_pos0=q_pos0))
+    qbar, wbar = inputs.mean_pool_group_queries(p["q"].float(), p["w"], G, Hg)
+    qbar = qbar.to(torch.bfloat16).contiguous()
+    bank = indexer.group_bank(qbar, wbar, p["k"], G, B, mode, q_pos0=q_pos0)
+    idx, sc = indexer.bank_refine(p["q"], p["w"], p["k"], bank, G, B, mode, K, q_pos0=q_pos0,
+                                  with_scores=True)
+    torch.cuda.synchronize()
+    q64, k64, w64 = f64(p["q"]), f64(p["k"]), p["w"].double().cpu().numpy()
+    qb64, wb64 = f64(qbar), wbar.double().cpu().numpy()
+    bank, idx, sc = bank.cpu().numpy(), idx.cpu().numpy(), sc.cpu().numpy()
+    bank_k = B if mode == "paper" else B - G
+    for g in range(T // G):
+        a = q_pos0 + g * G
+        scan_n = a + 1 if mode == "paper" else a
+        keys = k64[:scan_n]
+        check_topk(bank[g, :bank_k], np.arange(scan_n), ox.score_keys(qb64[g], wb64[g], keys),
+                   score_floor(qb64[g], wb64[g], keys), bank_k, RTOL["bf16"], what=f"bank {g}")
+        lo = a + 1 if mode == "paper" else a
+        scan_part = bank[g, :bank_k][bank[g, :bank_k] >= 0]
+        for r in range(g * G, g * G + G, 5):
+            i = q_pos0 + r
+            cand = np.union1d(scan_part, np.arange(lo, i + 1))
+            cand = cand[cand <= i]
+            check_topk(idx[r], cand, ox.score_keys(q64[r], w64[r], k64[cand]),
+                       score_floor(q64[r], w64[r], k64[cand]), K, RTOL["bf16"], sc[r],
+                       f"refine row {r}")
+    for r in range(T // G * G, T):
+        n = q_pos0 + r + 1
+        check_topk(idx[r], np.arange(n), ox.score_keys(q64[r], w64[r], k64[:n]),
+                   score_floor(q64[r], w64[r], k64[:n]), K, RTOL["bf16"], sc[r], f"tail {r}")
