@@ -57,9 +57,13 @@ class Dist:
         if self.world > 1:
             import datetime
             import torch.distributed as dist
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local))
+            timeout = datetime.timedelta(seconds=120)
+            if torch.cuda.is_available():
+                torch.cuda.set_device(self.local)
+                dist.init_process_group("nccl", timeout=timeout,
+                                        device_id=torch.device("cuda", self.local))
+            else:  # host-only ranks (the oracle arm, or tests without a GPU)
+                dist.init_process_group("gloo", timeout=timeout)
             self.pg = dist
 
     def barrier(self):
@@ -69,7 +73,8 @@ class Dist:
     def max(self, x):
         if not self.pg:
             return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 

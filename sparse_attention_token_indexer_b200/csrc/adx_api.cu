@@ -17,7 +17,7 @@ namespace adx {
 namespace {
 
 constexpr size_t kAlign = 256;
-constexpr int64_t kSelectRegCapacity = 16384;  // longest row the register-resident select holds
+constexpr int64_t kSelectRegCapacity = 32768;  // longest row the register-resident select holds
 
 // Optional instrumentation (adx_set_timing_events / adx_launch_count).
 thread_local void* const* g_events = nullptr;
@@ -135,9 +135,11 @@ void plan_split(int64_t rows, int64_t n, int K, int& n_seg, int& seg_len) {
   if (rows >= sms || n < 8ll * K) return;
   const int64_t want = (2ll * sms + rows - 1) / rows;
   const int64_t most = n / (4ll * K);
-  // keep the second stage (n_seg * K candidates per row) inside the register-resident select
+  // keep the second stage (n_seg * K candidates per row) inside the register-resident select,
+  // and the segments too when possible
   const int64_t fit = std::max<int64_t>(2, kSelectRegCapacity / K);
-  n_seg = static_cast<int>(std::max<int64_t>(1, std::min(std::min(want, most), fit)));
+  const int64_t need = (n + kSelectRegCapacity - 1) / kSelectRegCapacity;
+  n_seg = static_cast<int>(std::max<int64_t>(need, std::min(std::min(want, most), fit)));
   if (n_seg == 1) return;
   seg_len = static_cast<int>(align_up((n + n_seg - 1) / n_seg, 4));
   n_seg = static_cast<int>((n + seg_len - 1) / seg_len);

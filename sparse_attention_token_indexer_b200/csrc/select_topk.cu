@@ -239,10 +239,15 @@ __device__ __forceinline__ unsigned long long block_exclusive_scan64(unsigned lo
   return before + incl - x;
 }
 
+// Outputs of a row are staged in shared memory (up to this K) and written with coalesced
+// stores; per-thread runs of slots would otherwise scatter every store instruction.
+constexpr int kStageMaxK = 4096;
+
 template <int THREADS, int DIGIT>
-__global__ void __launch_bounds__(THREADS) select_reg_kernel(const SelectArgs a, int row0) {
+__global__ void __launch_bounds__(THREADS, 1024 / THREADS) select_reg_kernel(const SelectArgs a, int row0) {
   constexpr int NW = THREADS / 32;
   constexpr int NB = 1 << DIGIT;
+  extern __shared__ __align__(16) uint8_t stage_smem[];
   __shared__ uint32_t hist[NB];
   __shared__ unsigned long long warp_tot64[NW];
   __shared__ uint32_t red_min[NW], red_max[NW], red_cnt[NW];
@@ -387,6 +392,9 @@ __global__ void __launch_bounds__(THREADS) select_reg_kernel(const SelectArgs a,
       static_cast<uint32_t>(tot >> 32) + min(static_cast<uint32_t>(tot & 0xffffffffu), need);
   uint32_t slot = gt_before + min(eq_before, need);
   uint32_t eq_rank = eq_before;
+  const bool staged = K <= kStageMaxK;
+  int32_t* st_idx = reinterpret_cast<int32_t*>(stage_smem);
+  uint32_t* st_key = reinterpret_cast<uint32_t*>(st_idx + (staged ? K : 0));
 #pragma unroll
   for (int j = 0; j < kRegItems; ++j) {
     bool sel = (gt_mask >> j) & 1u;
@@ -395,17 +403,36 @@ __global__ void __launch_bounds__(THREADS) select_reg_kernel(const SelectArgs a,
       ++eq_rank;
     }
     if (sel) {
-      const int64_t i = my0 + j;
-      int32_t id = in_idx ? in_idx[i] : static_cast<int32_t>(lo + i);
-      if (map != nullptr && id >= 0) id = map[id];
       if (slot < static_cast<uint32_t>(K)) {
-        a.out_idx[out_base + slot] = id;
-        if (a.out_val) {
-          const uint32_t u = key[j];
-          a.out_val[out_base + slot] = __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+        if (staged) {
+          st_idx[slot] = static_cast<int32_t>(my0 + j);
+          st_key[slot] = key[j];
+        } else {
+          const int64_t i = my0 + j;
+          int32_t id = in_idx ? in_idx[i] : static_cast<int32_t>(lo + i);
+          if (map != nullptr && id >= 0) id = map[id];
+          a.out_idx[out_base + slot] = id;
+          if (a.out_val) {
+            const uint32_t u = key[j];
+            a.out_val[out_base + slot] = __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+          }
         }
       }
       ++slot;
+    }
+  }
+  if (staged) {
+    __syncthreads();
+    const uint32_t n_out = min(n_sel_total, static_cast<uint32_t>(K));
+    for (uint32_t sl = threadIdx.x; sl < n_out; sl += THREADS) {
+      const int32_t i = st_idx[sl];
+      int32_t id = in_idx ? in_idx[i] : static_cast<int32_t>(lo + i);
+      if (map != nullptr && id >= 0) id = map[id];
+      a.out_idx[out_base + sl] = id;
+      if (a.out_val) {
+        const uint32_t u = st_key[sl];
+        a.out_val[out_base + sl] = __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+      }
     }
   }
   for (int64_t j = n_sel_total + threadIdx.x; j < K; j += THREADS) {
@@ -418,7 +445,14 @@ template <int THREADS, int DIGIT>
 cudaError_t launch_reg(const SelectArgs& a, int row0, int row1, cudaStream_t s, int* launched) {
   const int64_t grid = static_cast<int64_t>(row1 - row0) * a.n_seg;
   if (grid <= 0) return cudaSuccess;
-  select_reg_kernel<THREADS, DIGIT><<<static_cast<unsigned>(grid), THREADS, 0, s>>>(a, row0);
+  const size_t smem = a.K <= kStageMaxK ? static_cast<size_t>(a.K) * 8 : 0;
+  auto kern = select_reg_kernel<THREADS, DIGIT>;
+  if (smem > 0) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  kern<<<static_cast<unsigned>(grid), THREADS, smem, s>>>(a, row0);
   ++*launched;
   return cudaGetLastError();
 }
@@ -430,14 +464,15 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launched) {
   const int64_t grid = static_cast<int64_t>(a.rows) * a.n_seg;
   if (grid <= 0) return cudaSuccess;
   const int64_t seg = a.n_seg == 1 ? a.len_cap : a.seg_len;
-  constexpr int64_t c128 = 128 * kRegItems, c256 = 256 * kRegItems, c512 = 512 * kRegItems;
-  if (seg > c512) {
+  constexpr int64_t c128 = 128 * kRegItems, c256 = 256 * kRegItems, c512 = 512 * kRegItems,
+                    c1024 = 1024 * kRegItems;
+  if (seg > c1024) {
     select_kernel<<<static_cast<unsigned>(grid), kSelThreads, 0, s>>>(a);
     *launched = 1;
     return cudaGetLastError();
   }
   // rows of a causal prefix grow with the row index: split the launch by length class
-  int r128 = 0, r256 = 0;
+  int r128 = 0, r256 = 0, r512 = 0;
   if (a.len_mode == 1 && a.n_seg == 1 && a.pos_step > 0) {
     auto rows_upto = [&](int64_t cap) {  // first row whose length exceeds cap
       const int64_t r = (cap - 1 - a.pos_base) / a.pos_step + 1;
@@ -445,15 +480,19 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launched) {
     };
     r128 = rows_upto(c128);
     r256 = std::max(r128, rows_upto(c256));
+    r512 = std::max(r256, rows_upto(c512));
   } else if (seg <= c128) {
-    r128 = r256 = a.rows;
+    r128 = r256 = r512 = a.rows;
   } else if (seg <= c256) {
-    r256 = a.rows;
+    r256 = r512 = a.rows;
+  } else if (seg <= c512) {
+    r512 = a.rows;
   }
   cudaError_t e;
   if ((e = launch_reg<128, 10>(a, 0, r128, s, launched)) != cudaSuccess) return e;
   if ((e = launch_reg<256, 11>(a, r128, r256, s, launched)) != cudaSuccess) return e;
-  return launch_reg<512, 12>(a, r256, a.rows, s, launched);
+  if ((e = launch_reg<512, 12>(a, r256, r512, s, launched)) != cudaSuccess) return e;
+  return launch_reg<1024, 12>(a, r512, a.rows, s, launched);
 }
 
 }  // namespace adx
