@@ -48,12 +48,14 @@ struct Cfg {
   static constexpr int KC = DB / 128;        // 128-byte K chunks
   static constexpr int ELEMS_PER_CHUNK = FP8 ? 128 : 64;
   static constexpr int KSTEPS = DB / 32;     // 32 bytes of K per MMA instruction
-  // Epilogue warpgroups. With two and few tokens per tile (BUF_SPLIT), warpgroup g owns
-  // TMEM accumulator buffer g and reduces every other tile, all of its tokens, so each warp
-  // has two MMA periods per tile; with many tokens per tile the two warpgroups split the
-  // tokens of every tile instead (keeps the per-thread accumulators in registers).
-  static constexpr int EG = TOK >= 2 ? 2 : 1;
-  static constexpr bool BUF_SPLIT = false;
+  // Epilogue warpgroups. With one query token per tile (BUF_SPLIT), the tiles go round the
+  // warpgroups: warpgroup g reduces the tiles whose accumulator buffer index is g modulo EG,
+  // all heads of the one token, so each warp has EG MMA periods per tile (a single warpgroup
+  // cannot keep up with the key stream there). With several tokens per tile the two
+  // warpgroups split the tokens of every tile instead (keeps the per-thread partial sums in
+  // registers).
+  static constexpr bool BUF_SPLIT = TOK == 1;
+  static constexpr int EG = 2;
   static constexpr int EPI_WARPS = 4 * EG;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr int TOKG = BUF_SPLIT ? TOK : TOK / EG;  // tokens one warp reduces per tile
@@ -64,7 +66,7 @@ struct Cfg {
   static constexpr int QBYTES = N * DB;
   static constexpr int KBYTES = kTileM * DB;
   static constexpr int ST = cmin(8, (200 * 1024 - QBYTES) / KBYTES);
-  static constexpr int ACC = 2;
+  static constexpr int ACC = BUF_SPLIT ? 2 * EG : 2;  // accumulator buffers in TMEM
   static constexpr int TMEM_COLS = pow2ceil(cmax(32, ACC * N));
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = QBYTES;
@@ -81,7 +83,7 @@ struct Cfg {
   static_assert(NG % CW == 0 && CW % 4 == 0 && (H >= 32 ? H % CW == 0 : CW % H == 0),
                 "epilogue chunking");
   static_assert(THREADS <= kMaxThreads, "block size");
-  static_assert(!BUF_SPLIT || EG == ACC, "one accumulator buffer per epilogue warpgroup");
+  static_assert(ACC % EG == 0, "every epilogue warpgroup owns the same number of buffers");
 };
 
 // One row block of the work: TOK consecutive query rows of one key batch and the key
@@ -484,17 +486,24 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           if (a.k_scale != nullptr) ks = a.k_scale[kr];
         }
       };
-      float ks_next;
-      int64_t kpos_next;
-      key_meta(t_lo, ks_next, kpos_next);
+      // tile t of this range is the CTA's tile number g = gi_lo + (t - t_lo); it lands in
+      // accumulator buffer g % ACC, and with BUF_SPLIT only the warpgroup g % EG reduces it
+      const int64_t gi_lo = gi;
+      gi += t_hi - t_lo;
+      constexpr int TSTEP = C::BUF_SPLIT ? C::EG : 1;
+      int t0 = t_lo;
+      if (C::BUF_SPLIT) t0 += static_cast<int>(((grp - gi_lo) % C::EG + C::EG) % C::EG);
+      float ks_next = 1.f;
+      int64_t kpos_next = 0;
+      if (t0 < t_hi) key_meta(t0, ks_next, kpos_next);
       bool ok = true;
-      for (int t = t_lo; t < t_hi; ++t, ++gi) {
+      for (int t = t0; t < t_hi; t += TSTEP) {
         const float ks = ks_next;
         const int64_t kpos = kpos_next;
-        if (t + 1 < t_hi) key_meta(t + 1, ks_next, kpos_next);
-        const int acc = static_cast<int>(gi % C::ACC);
-        if (C::BUF_SPLIT && acc != grp) continue;  // the other warpgroup's tile
-        const uint32_t acc_phase = static_cast<uint32_t>((gi / C::ACC) & 1);
+        if (t + TSTEP < t_hi) key_meta(t + TSTEP, ks_next, kpos_next);
+        const int64_t g = gi_lo + (t - t_lo);
+        const int acc = static_cast<int>(g % C::ACC);
+        const uint32_t acc_phase = static_cast<uint32_t>((g / C::ACC) & 1);
         int got = 0;
         if (lane == 0) got = mbar_wait(&acc_full[acc], acc_phase, abort_s, a.timeout_ns) ? 1 : 0;
         got = __shfl_sync(0xffffffffu, got, 0);
