@@ -236,6 +236,7 @@ adx_status run_score(const ScorePlan& p, const void* q_codes, const void* keys, 
 }
 
 size_t select_scratch_bytes(int64_t rows, int64_t n, int K) {
+  if (select_cluster_ctas(rows, n, K, sm_count()) > 0) return 0;
   int n_seg, seg_len;
   plan_split(rows, n, K, n_seg, seg_len);
   if (n_seg == 1) return 0;
@@ -243,9 +244,22 @@ size_t select_scratch_bytes(int64_t rows, int64_t n, int K) {
   return align_up(c * 4, kAlign) * 2;
 }
 
-// Top-K per row of a score matrix, split into two stages when there are few long rows.
+// Top-K per row of a score matrix. Few long rows go to the cluster select (one cluster of
+// CTAs per row) when a cluster holds the row, else to a two-stage split.
 adx_status run_select(SelectArgs a, int64_t n_max, Carve& cv, DeviceStatus* st, cudaStream_t s) {
   a.status = st;
+  n_max = std::max<int64_t>(n_max, a.len_cap);
+  const int ctas = select_cluster_ctas(a.rows, n_max, a.K, sm_count());
+  if (ctas > 0) {
+    a.n_seg = 1;
+    a.seg_len = static_cast<int32_t>(std::min<int64_t>(n_max, INT32_MAX));
+    mark(2, s);
+    int nl = 0;
+    const cudaError_t e0 = launch_select_cluster(a, ctas, s, &nl);
+    const cudaError_t e = counted(e0, nl);
+    mark(3, s);
+    return e == cudaSuccess ? ADX_OK : ADX_ECUDA;
+  }
   int n_seg, seg_len;
   plan_split(a.rows, n_max, a.K, n_seg, seg_len);
   mark(2, s);

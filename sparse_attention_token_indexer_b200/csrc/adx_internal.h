@@ -89,6 +89,11 @@ int score_tokens_per_tile(int H);  // tokens per N tile for a head count (0 = un
 bool score_config_supported(bool fp8, int H, int d);
 // Launches one to three kernels (row-length classes); *launched receives how many.
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launched);
+// Few long rows: CTAs per row of the cluster select (one thread-block cluster per row, the
+// row held in registers across the cluster), or 0 when it does not apply.
+int select_cluster_ctas(int64_t rows, int64_t n_max, int K, int sms);
+// One launch of the cluster select with `ctas` CTAs per row (a.n_seg must be 1).
+cudaError_t launch_select_cluster(const SelectArgs& a, int ctas, cudaStream_t s, int* launched);
 cudaError_t launch_pack_candidates(const void* k, const float* k_scale, int64_t key_batch_stride,
                                    int32_t per_group_keys, int32_t S_valid, const int32_t* cand,
                                    int32_t n_groups, int32_t n_cand, int32_t n_cand_pad,

@@ -8,12 +8,17 @@
 // using block-wide prefix sums (warp shuffles) for the output slots. -inf marks a masked
 // (invisible) key and NaN is treated the same way: neither is ever selected. Rows with fewer
 // than K valid elements return all of them, padded with index -1 and score -inf.
+#include <cooperative_groups.h>
+
 #include <algorithm>
 #include <cstdint>
+#include <type_traits>
 
 #include "adx_internal.h"
 
 namespace adx {
+
+namespace cg = cooperative_groups;
 
 namespace {
 
@@ -205,13 +210,25 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a)
 }
 
 // ---------------------------------------------------------------------------------------
-// Rows of at most kRegItems * THREADS elements: the whole row lives in registers (each
-// thread a contiguous run of kRegItems elements), so global memory is read once; the digit
-// passes work on registers and one block-wide scan of (above, equal) counts gives every
-// thread its output slots in index order. The CTA size (and digit width) is chosen per row
-// length class, so short rows of a causal prefix do not pay for long ones.
+// Register-resident select: each thread holds a contiguous run of ITEMS elements of its
+// CTA's part of the row, so global memory is read once; the digit passes work on registers
+// and one block-wide scan of (above, equal) counts gives every thread its output slots in
+// index order. The CTA size (and digit width) is chosen per row-length class, so short rows
+// of a causal prefix do not pay for long ones.
+//
+// CLUSTER: one thread-block cluster per row, for few long rows. The row is cut into one
+// contiguous slice per CTA of the cluster; the valid-key range, the digit histograms and the
+// per-CTA output counts are combined through distributed shared memory, so every CTA of the
+// cluster takes the same decisions and writes its own share of the output slots. Histograms
+// alternate between two buffers: a CTA clears a buffer only after a cluster barrier that every
+// other CTA reaches after its last read of that buffer, so one barrier per digit suffices.
+// All CTAs of a cluster compute the same row length, key range and bins, so they pass the
+// same cluster barriers.
 // ---------------------------------------------------------------------------------------
-constexpr int kRegItems = 32;
+constexpr int kRegItems = 32;      // elements per thread of the row-per-CTA classes
+constexpr int kClusterItems = 36;  // elements per thread of the cluster class
+constexpr int kClusterThreads = 512;
+constexpr int kClusterMaxCtas = 8;  // portable cluster size
 
 template <int THREADS>
 __device__ __forceinline__ unsigned long long block_exclusive_scan64(unsigned long long x,
@@ -243,23 +260,46 @@ __device__ __forceinline__ unsigned long long block_exclusive_scan64(unsigned lo
 // stores; per-thread runs of slots would otherwise scatter every store instruction.
 constexpr int kStageMaxK = 4096;
 
-template <int THREADS, int DIGIT>
-__global__ void __launch_bounds__(THREADS, 1024 / THREADS) select_reg_kernel(const SelectArgs a, int row0) {
+template <int ITEMS>
+using ItemMask = typename std::conditional<(ITEMS > 32), unsigned long long, uint32_t>::type;
+
+template <int THREADS, int DIGIT, int ITEMS, bool CLUSTER>
+__global__ void __launch_bounds__(THREADS, 1024 / THREADS)
+select_reg_kernel(const SelectArgs a, int row0) {
   constexpr int NW = THREADS / 32;
   constexpr int NB = 1 << DIGIT;
+  constexpr int NH = CLUSTER ? 2 : 1;  // histogram buffers
+  using Mask = ItemMask<ITEMS>;
   extern __shared__ __align__(16) uint8_t stage_smem[];
-  __shared__ uint32_t hist[NB];
+  __shared__ __align__(16) uint32_t hist[NH][NB];
   __shared__ unsigned long long warp_tot64[NW];
   __shared__ uint32_t red_min[NW], red_max[NW], red_cnt[NW];
-  __shared__ uint32_t sh_bin, sh_above;
+  __shared__ uint32_t sh_bin, sh_above, sh_inbin;
+  __shared__ uint32_t cl_red[3];         // this CTA's (min, max, count) of valid keys
+  __shared__ unsigned long long cl_tot;  // this CTA's packed (above, equal) counts
+  __shared__ uint32_t cl_part[NH][CLUSTER ? THREADS : 1];  // per-thread bin-range counts
 
-  const int seg = blockIdx.x % a.n_seg;
-  const int r = row0 + static_cast<int>(blockIdx.x / a.n_seg);
-  if (r >= a.rows) return;
+  int r, seg = 0, nparts = 1, part = 0;
+  if constexpr (CLUSTER) {
+    nparts = static_cast<int>(cg::this_cluster().num_blocks());
+    part = static_cast<int>(cg::this_cluster().block_rank());
+    r = row0 + static_cast<int>(blockIdx.x) / nparts;  // cluster c covers CTAs c*nparts ..
+  } else {
+    seg = blockIdx.x % a.n_seg;
+    r = row0 + static_cast<int>(blockIdx.x / a.n_seg);
+  }
+  if (r >= a.rows) return;  // the same for every CTA of a cluster
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t n = row_length(a, r);
-  const int64_t lo = static_cast<int64_t>(seg) * a.seg_len;
-  const int64_t hi = a.n_seg == 1 ? n : min(n, lo + a.seg_len);
+  int64_t lo, hi;
+  if (CLUSTER) {
+    const int64_t per = ((n + nparts - 1) / nparts + 3) & ~static_cast<int64_t>(3);
+    lo = min(n, static_cast<int64_t>(part) * per);
+    hi = min(n, lo + per);
+  } else {
+    lo = static_cast<int64_t>(seg) * a.seg_len;
+    hi = a.n_seg == 1 ? n : min(n, lo + a.seg_len);
+  }
   const int64_t len = hi > lo ? hi - lo : 0;
   const float* vals = a.vals + static_cast<int64_t>(r) * a.ld + lo;
   const int32_t* in_idx = a.in_idx ? a.in_idx + static_cast<int64_t>(r) * a.ld + lo : nullptr;
@@ -268,13 +308,13 @@ __global__ void __launch_bounds__(THREADS, 1024 / THREADS) select_reg_kernel(con
   const int64_t out_base = (static_cast<int64_t>(r) * a.n_seg + seg) * a.out_ld;
   const int K = a.K;
 
-  // ---- load: thread t owns elements [t*kRegItems, (t+1)*kRegItems) of the segment ------
-  uint32_t key[kRegItems];
-  const int64_t my0 = static_cast<int64_t>(threadIdx.x) * kRegItems;
+  // ---- load: thread t owns elements [t*ITEMS, (t+1)*ITEMS) of this CTA's range -------------
+  uint32_t key[ITEMS];
+  const int64_t my0 = static_cast<int64_t>(threadIdx.x) * ITEMS;
   const bool vec = ((reinterpret_cast<uintptr_t>(vals) & 15) == 0);
   uint32_t kmin = 0xffffffffu, kmax = 0u, nval = 0u;
 #pragma unroll
-  for (int j = 0; j < kRegItems; j += 4) {
+  for (int j = 0; j < ITEMS; j += 4) {
     float v[4];
     const int64_t i0 = my0 + j;
     if (vec && i0 + 4 <= len) {
@@ -313,6 +353,27 @@ __global__ void __launch_bounds__(THREADS, 1024 / THREADS) select_reg_kernel(con
     kmax = max(kmax, red_max[w]);
     nval += red_cnt[w];
   }
+  if constexpr (CLUSTER) {
+    if (threadIdx.x == 0) {
+      cl_red[0] = kmin;
+      cl_red[1] = kmax;
+      cl_red[2] = nval;
+    }
+    cg::this_cluster().sync();
+    kmin = 0xffffffffu;
+    kmax = 0u;
+    nval = 0u;
+    // fixed trip count: the remote loads of all CTAs are in flight together
+#pragma unroll
+    for (int c = 0; c < kClusterMaxCtas; ++c) {
+      if (c < nparts) {
+        const uint32_t* rc = cg::this_cluster().map_shared_rank(cl_red, c);
+        kmin = min(kmin, rc[0]);
+        kmax = max(kmax, rc[1]);
+        nval += rc[2];
+      }
+    }
+  }
 
   uint32_t prefix = 0;
   int shift = 32;            // number of low key bits not yet resolved
@@ -323,80 +384,144 @@ __global__ void __launch_bounds__(THREADS, 1024 / THREADS) select_reg_kernel(con
     shift = diff == 0u ? 0 : 32 - __clz(diff);  // bits above `shift` are common to all keys
     prefix = shift >= 32 ? 0u : (kmax >> shift);
   }
+  int hb = 0;
 #pragma unroll 1
   while (!take_all && shift > 0) {
     const int wbits = min(DIGIT, shift);
     const int nb = 1 << wbits;
     const int nshift = shift - wbits;
-    for (int i = threadIdx.x; i < nb; i += THREADS) hist[i] = 0;
+    uint32_t* h = hist[hb];
+    for (int i = threadIdx.x; i < nb; i += THREADS) h[i] = 0;
     __syncthreads();
 #pragma unroll
-    for (int j = 0; j < kRegItems; ++j) {
+    for (int j = 0; j < ITEMS; ++j) {
       const uint32_t u = key[j];
       if (u != 0u && (shift >= 32 || (u >> shift) == prefix))
-        atomicAdd(&hist[(u >> nshift) & (nb - 1)], 1u);
+        atomicAdd(&h[(u >> nshift) & (nb - 1)], 1u);
     }
     __syncthreads();
-    // thread t owns bins nb-1-t*bpt .. : thread 0 the highest ones
+    // thread t owns bins nb-1-t*bpt .. nb-(t+1)*bpt: thread 0 the highest ones
     const int bpt = nb >= THREADS ? nb / THREADS : 1;
     const bool owner = threadIdx.x * bpt < nb;
+    const int b0 = nb - (threadIdx.x + 1) * bpt;  // lowest bin of this thread
     uint32_t mine = 0;
-    if (owner)
-      for (int j = 0; j < bpt; ++j) mine += hist[nb - 1 - (threadIdx.x * bpt + j)];
+    if (owner) {
+      if (bpt % 4 == 0) {
+        for (int q = 0; q < bpt; q += 4) {
+          const uint4 v4 = *reinterpret_cast<const uint4*>(h + b0 + q);
+          mine += v4.x + v4.y + v4.z + v4.w;
+        }
+      } else {
+        for (int j = 0; j < bpt; ++j) mine += h[b0 + j];
+      }
+    }
+    if constexpr (CLUSTER) {
+      // the row's count of this thread's bins: the same thread's partial in every CTA
+      cl_part[hb][threadIdx.x] = mine;
+      cg::this_cluster().sync();
+      mine = 0;
+#pragma unroll
+      for (int c = 0; c < kClusterMaxCtas; ++c)
+        if (c < nparts) mine += cg::this_cluster().map_shared_rank(cl_part[hb], c)[threadIdx.x];
+    }
     unsigned long long tot64;
     const uint32_t excl = static_cast<uint32_t>(block_exclusive_scan64<THREADS>(mine, warp_tot64, tot64));
     if (owner && excl < need && need <= excl + mine) {
-      uint32_t above = excl;
-      for (int j = 0; j < bpt; ++j) {
-        const int bin = nb - 1 - (threadIdx.x * bpt + j);
-        const uint32_t h = hist[bin];
-        if (above + h >= need) {
-          sh_bin = static_cast<uint32_t>(bin);
-          sh_above = above;
-          break;
+      // the row's count of each of this thread's bins, highest bin first
+      constexpr int BPT = NB >= THREADS ? NB / THREADS : 1;
+      uint32_t cnt[BPT];
+#pragma unroll
+      for (int j = 0; j < BPT; ++j) cnt[j] = 0;
+      if constexpr (CLUSTER) {
+#pragma unroll
+        for (int c = 0; c < kClusterMaxCtas; ++c) {
+          if (c < nparts) {
+            const uint32_t* hc = cg::this_cluster().map_shared_rank(h, c);
+#pragma unroll
+            for (int j = 0; j < BPT; ++j)
+              if (j < bpt) cnt[j] += hc[b0 + bpt - 1 - j];
+          }
         }
-        above += h;
+      } else {
+#pragma unroll
+        for (int j = 0; j < BPT; ++j)
+          if (j < bpt) cnt[j] = h[b0 + bpt - 1 - j];
+      }
+      uint32_t above = excl;
+#pragma unroll
+      for (int j = 0; j < BPT; ++j) {
+        if (j < bpt && above < need) {
+          if (above + cnt[j] >= need) {
+            sh_bin = static_cast<uint32_t>(b0 + bpt - 1 - j);
+            sh_above = above;
+            sh_inbin = cnt[j];
+          }
+          above += cnt[j];
+        }
       }
     }
     __syncthreads();
     const uint32_t bin = sh_bin;
     need -= sh_above;
-    const uint32_t in_bin = hist[bin];
+    const uint32_t in_bin = sh_inbin;
     prefix = (shift < 32 ? (prefix << wbits) : 0u) | bin;
     shift = nshift;
-    __syncthreads();
+    if (CLUSTER) hb ^= 1;
     if (in_bin == need) break;  // the whole bin is taken: no further digits needed
   }
 
   // ---- output: one scan of (above, equal) counts, then each thread writes its run ------
-  uint32_t gt_mask = 0, eq_mask = 0;
+  Mask gt_mask = 0, eq_mask = 0;
 #pragma unroll
-  for (int j = 0; j < kRegItems; ++j) {
+  for (int j = 0; j < ITEMS; ++j) {
     const uint32_t u = key[j];
     if (u == 0u) continue;
     if (take_all) {
-      gt_mask |= 1u << j;
+      gt_mask |= Mask(1) << j;
       continue;
     }
     const uint32_t top = shift >= 32 ? 0u : (u >> shift);
-    if (top > prefix) gt_mask |= 1u << j;
-    else if (top == prefix) eq_mask |= 1u << j;
+    if (top > prefix) gt_mask |= Mask(1) << j;
+    else if (top == prefix) eq_mask |= Mask(1) << j;
   }
+  constexpr unsigned long long kLow = 0xffffffffull;
   unsigned long long tot;
   const unsigned long long packed =
-      (static_cast<unsigned long long>(__popc(gt_mask)) << 32) | __popc(eq_mask);
+      (static_cast<unsigned long long>(__popcll(gt_mask)) << 32) | __popcll(eq_mask);
   const unsigned long long ex = block_exclusive_scan64<THREADS>(packed, warp_tot64, tot);
-  const uint32_t gt_before = static_cast<uint32_t>(ex >> 32);
-  const uint32_t eq_before = static_cast<uint32_t>(ex & 0xffffffffu);
+  // packed counts of the CTAs before this one (cluster) and of the whole row
+  unsigned long long off = 0, all = tot;
+  if constexpr (CLUSTER) {
+    if (threadIdx.x == 0) cl_tot = tot;
+    cg::this_cluster().sync();
+    all = 0;
+#pragma unroll
+    for (int c = 0; c < kClusterMaxCtas; ++c) {
+      if (c < nparts) {
+        const unsigned long long v = *cg::this_cluster().map_shared_rank(&cl_tot, c);
+        if (c < part) off += v;
+        all += v;
+      }
+    }
+    // no CTA leaves while another may still read its shared memory
+    cg::this_cluster().sync();
+  }
+  const uint32_t gt_before = static_cast<uint32_t>((off + ex) >> 32);
+  const uint32_t eq_before = static_cast<uint32_t>((off + ex) & kLow);
   const uint32_t n_sel_total =
-      static_cast<uint32_t>(tot >> 32) + min(static_cast<uint32_t>(tot & 0xffffffffu), need);
+      static_cast<uint32_t>(all >> 32) + min(static_cast<uint32_t>(all & kLow), need);
+  // first output slot of this CTA and its number of selected elements
+  const uint32_t eq_off = static_cast<uint32_t>(off & kLow);
+  const uint32_t cta_slot0 = static_cast<uint32_t>(off >> 32) + min(eq_off, need);
+  const uint32_t cta_sel = static_cast<uint32_t>(tot >> 32) +
+                           min(eq_off + static_cast<uint32_t>(tot & kLow), need) - min(eq_off, need);
   uint32_t slot = gt_before + min(eq_before, need);
   uint32_t eq_rank = eq_before;
   const bool staged = K <= kStageMaxK;
   int32_t* st_idx = reinterpret_cast<int32_t*>(stage_smem);
   uint32_t* st_key = reinterpret_cast<uint32_t*>(st_idx + (staged ? K : 0));
 #pragma unroll
-  for (int j = 0; j < kRegItems; ++j) {
+  for (int j = 0; j < ITEMS; ++j) {
     bool sel = (gt_mask >> j) & 1u;
     if ((eq_mask >> j) & 1u) {
       sel = eq_rank < need;
@@ -405,8 +530,8 @@ __global__ void __launch_bounds__(THREADS, 1024 / THREADS) select_reg_kernel(con
     if (sel) {
       if (slot < static_cast<uint32_t>(K)) {
         if (staged) {
-          st_idx[slot] = static_cast<int32_t>(my0 + j);
-          st_key[slot] = key[j];
+          st_idx[slot - cta_slot0] = static_cast<int32_t>(my0 + j);
+          st_key[slot - cta_slot0] = key[j];
         } else {
           const int64_t i = my0 + j;
           int32_t id = in_idx ? in_idx[i] : static_cast<int32_t>(lo + i);
@@ -423,19 +548,22 @@ __global__ void __launch_bounds__(THREADS, 1024 / THREADS) select_reg_kernel(con
   }
   if (staged) {
     __syncthreads();
-    const uint32_t n_out = min(n_sel_total, static_cast<uint32_t>(K));
+    const uint32_t n_out =
+        cta_slot0 >= static_cast<uint32_t>(K) ? 0u : min(cta_sel, static_cast<uint32_t>(K) - cta_slot0);
     for (uint32_t sl = threadIdx.x; sl < n_out; sl += THREADS) {
       const int32_t i = st_idx[sl];
       int32_t id = in_idx ? in_idx[i] : static_cast<int32_t>(lo + i);
       if (map != nullptr && id >= 0) id = map[id];
-      a.out_idx[out_base + sl] = id;
+      a.out_idx[out_base + cta_slot0 + sl] = id;
       if (a.out_val) {
         const uint32_t u = st_key[sl];
-        a.out_val[out_base + sl] = __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+        a.out_val[out_base + cta_slot0 + sl] =
+            __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
       }
     }
   }
-  for (int64_t j = n_sel_total + threadIdx.x; j < K; j += THREADS) {
+  for (int64_t j = n_sel_total + static_cast<int64_t>(part) * THREADS + threadIdx.x; j < K;
+       j += static_cast<int64_t>(THREADS) * nparts) {
     a.out_idx[out_base + j] = -1;
     if (a.out_val) a.out_val[out_base + j] = -INFINITY;
   }
@@ -446,7 +574,7 @@ cudaError_t launch_reg(const SelectArgs& a, int row0, int row1, cudaStream_t s, 
   const int64_t grid = static_cast<int64_t>(row1 - row0) * a.n_seg;
   if (grid <= 0) return cudaSuccess;
   const size_t smem = a.K <= kStageMaxK ? static_cast<size_t>(a.K) * 8 : 0;
-  auto kern = select_reg_kernel<THREADS, DIGIT>;
+  auto kern = select_reg_kernel<THREADS, DIGIT, kRegItems, false>;
   if (smem > 0) {
     const cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -458,6 +586,47 @@ cudaError_t launch_reg(const SelectArgs& a, int row0, int row1, cudaStream_t s, 
 }
 
 }  // namespace
+
+int select_cluster_ctas(int64_t rows, int64_t n_max, int K, int sms) {
+  constexpr int64_t cap = static_cast<int64_t>(kClusterThreads) * kClusterItems;
+  if (rows <= 0 || rows >= sms || n_max <= 8ll * K) return 0;
+  const int64_t need = (n_max + cap - 1) / cap;
+  if (need > kClusterMaxCtas) return 0;
+  const int64_t fill = (2ll * sms) / rows;       // two CTAs of this class fit on an SM
+  const int64_t useful = (n_max + 4095) / 4096;  // at least 4096 elements per CTA
+  const int64_t cl = std::max(need, std::min(std::min(fill, useful), int64_t(kClusterMaxCtas)));
+  return cl > 1 ? static_cast<int>(cl) : 0;
+}
+
+cudaError_t launch_select_cluster(const SelectArgs& a, int ctas, cudaStream_t s, int* launched) {
+  *launched = 0;
+  if (a.rows <= 0) return cudaSuccess;
+  if (a.n_seg != 1 || ctas < 2 || ctas > kClusterMaxCtas ||
+      static_cast<int64_t>(a.len_cap) > static_cast<int64_t>(ctas) * kClusterThreads * kClusterItems)
+    return cudaErrorInvalidValue;
+  auto kern = select_reg_kernel<kClusterThreads, 12, kClusterItems, true>;
+  const size_t smem = a.K <= kStageMaxK ? static_cast<size_t>(a.K) * 8 : 0;
+  if (smem > 0) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(a.rows) * static_cast<unsigned>(ctas), 1, 1);
+  cfg.blockDim = dim3(kClusterThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(ctas);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a, 0);
+  *launched = 1;
+  return e;
+}
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launched) {
   *launched = 0;

@@ -210,6 +210,39 @@ def test_decode_flat(k_dtype):
                    score_floor(q64[b], w64[b], keys), 256, RTOL[k_dtype], sc[b], f"decode {b}")
 
 
+@pytest.mark.parametrize("S", [12000, 40000])
+def test_decode_long_rows_with_ties(S):
+    """Few long rows: each row is selected by one cluster of CTAs (3 and 8 CTAs for these
+    lengths), the row cut into one slice per CTA. Keys tied at the threshold lie in every
+    slice; the lowest positions among them must be the ones taken."""
+    Bs, K = 3, 512
+    prob = inputs.decode_problem(Bs=Bs, S=S, H=64, d=128, K=K, Hg=16, steps=1, seed=33,
+                                 device="cuda")
+    k, ks = prob["k"], prob["k_scale"]
+    q, w = prob["q_steps"][0], prob["w_steps"][0]
+    seq_len = torch.tensor([S, S * 4 // 7 + 3, 2], dtype=torch.int32, device="cuda")
+    # sequence 0: 300 keys far above the rest and 1500 exact copies of one key below them
+    q64, w64 = f64(q), w.double().cpu().numpy()
+    base = ox.score_keys(q64[0], w64[0], f64(k[0, :S], ks[0, :S]))
+    top = int(np.argmax(base))
+    rng = np.random.default_rng(7)
+    pos = rng.choice(S, size=1800, replace=False)
+    p_hi, p_tie = np.sort(pos[:300]), np.sort(pos[300:])
+    row, scale = k[0, top].clone(), float(ks[0, top])
+    for ps, mult in ((p_hi, 8.0), (p_tie, 4.0)):
+        sel = torch.as_tensor(ps, device="cuda")
+        k[0, sel] = row
+        ks[0, sel] = scale * mult
+    idx, sc = indexer.index_decode(q, w, k, seq_len, K, k_scale=ks, with_scores=True)
+    idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+    expect = set(p_hi.tolist()) | set(p_tie[: K - len(p_hi)].tolist())
+    assert set(idx[0].tolist()) == expect
+    for b, n in enumerate(seq_len.tolist()):
+        keys = f64(k[b, :n], ks[b, :n])
+        check_topk(idx[b], np.arange(n), ox.score_keys(q64[b], w64[b], keys),
+                   score_floor(q64[b], w64[b], keys), K, RTOL["e4m3"], sc[b], f"dlong {b}")
+
+
 def test_decode_bank_reuse():
     Bs, S, K, B, G = 4, 6000, 256, 1024, 16
     prob = inputs.decode_problem(Bs=Bs, S=S, H=64, d=128, K=K, Hg=16, steps=G, seed=32,
