@@ -259,9 +259,17 @@ __device__ __forceinline__ unsigned long long block_exclusive_scan64(unsigned lo
 // Outputs of a row are staged in shared memory (up to this K) and written with coalesced
 // stores; per-thread runs of slots would otherwise scatter every store instruction.
 constexpr int kStageMaxK = 4096;
+// When at most kGatherMax keys remain in the threshold bin they are gathered into shared
+// memory and the selection finishes there: by counting (each key's rank among them) up to
+// kCountMax keys, by 8-bit digit passes over the gathered keys beyond that.
+constexpr int kCountMax = 128;
+constexpr int kGatherMax = 2048;
 
 template <int ITEMS>
 using ItemMask = typename std::conditional<(ITEMS > 32), unsigned long long, uint32_t>::type;
+
+__device__ __forceinline__ int lowest_set_bit(uint32_t m) { return __ffs(m) - 1; }
+__device__ __forceinline__ int lowest_set_bit(unsigned long long m) { return __ffsll(m) - 1; }
 
 template <int THREADS, int DIGIT, int ITEMS, bool CLUSTER>
 __global__ void __launch_bounds__(THREADS, 1024 / THREADS)
@@ -278,6 +286,10 @@ select_reg_kernel(const SelectArgs a, int row0) {
   __shared__ uint32_t cl_red[3];         // this CTA's (min, max, count) of valid keys
   __shared__ unsigned long long cl_tot;  // this CTA's packed (above, equal) counts
   __shared__ uint32_t cl_part[NH][CLUSTER ? THREADS : 1];  // per-thread bin-range counts
+  __shared__ uint32_t sh_ccount, sh_theta, sh_needt;
+  __shared__ uint32_t c_key[kGatherMax];               // this CTA's keys of the threshold bin
+  __shared__ uint32_t c_off[kClusterMaxCtas + 1];       // where each CTA's keys go in c_all
+  __shared__ uint32_t h_small[256];                     // digit histogram of gathered keys
 
   int r, seg = 0, nparts = 1, part = 0;
   if constexpr (CLUSTER) {
@@ -290,6 +302,7 @@ select_reg_kernel(const SelectArgs a, int row0) {
   }
   if (r >= a.rows) return;  // the same for every CTA of a cluster
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) sh_ccount = 0;
   const int64_t n = row_length(a, r);
   int64_t lo, hi;
   if (CLUSTER) {
@@ -385,6 +398,7 @@ select_reg_kernel(const SelectArgs a, int row0) {
     prefix = shift >= 32 ? 0u : (kmax >> shift);
   }
   int hb = 0;
+  bool first = true;
 #pragma unroll 1
   while (!take_all && shift > 0) {
     const int wbits = min(DIGIT, shift);
@@ -393,11 +407,19 @@ select_reg_kernel(const SelectArgs a, int row0) {
     uint32_t* h = hist[hb];
     for (int i = threadIdx.x; i < nb; i += THREADS) h[i] = 0;
     __syncthreads();
+    if (first) {
+      // every valid key carries the common prefix
 #pragma unroll
-    for (int j = 0; j < ITEMS; ++j) {
-      const uint32_t u = key[j];
-      if (u != 0u && (shift >= 32 || (u >> shift) == prefix))
-        atomicAdd(&h[(u >> nshift) & (nb - 1)], 1u);
+      for (int j = 0; j < ITEMS; ++j) {
+        const uint32_t u = key[j];
+        if (u != 0u) atomicAdd(&h[(u >> nshift) & (nb - 1)], 1u);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < ITEMS; ++j) {
+        const uint32_t u = key[j];
+        if (u != 0u && (u >> shift) == prefix) atomicAdd(&h[(u >> nshift) & (nb - 1)], 1u);
+      }
     }
     __syncthreads();
     // thread t owns bins nb-1-t*bpt .. nb-(t+1)*bpt: thread 0 the highest ones
@@ -467,7 +489,112 @@ select_reg_kernel(const SelectArgs a, int row0) {
     prefix = (shift < 32 ? (prefix << wbits) : 0u) | bin;
     shift = nshift;
     if (CLUSTER) hb ^= 1;
+    first = false;
     if (in_bin == need) break;  // the whole bin is taken: no further digits needed
+    if (shift > 0 && in_bin <= static_cast<uint32_t>(kGatherMax)) {
+      // Few keys left in the threshold bin: gather them into shared memory and finish the
+      // selection there instead of more passes over the whole row.
+#pragma unroll
+      for (int j = 0; j < ITEMS; ++j) {
+        const uint32_t u = key[j];
+        if (u != 0u && (u >> shift) == prefix) c_key[atomicAdd(&sh_ccount, 1u)] = u;
+      }
+      const uint32_t m = in_bin;
+      const uint32_t* ck = c_key;
+      if constexpr (CLUSTER) {
+        cg::this_cluster().sync();
+        if (threadIdx.x == 0) {
+          uint32_t o = 0;
+          for (int c = 0; c < nparts; ++c) {
+            c_off[c] = o;
+            o += *cg::this_cluster().map_shared_rank(&sh_ccount, c);
+          }
+          c_off[nparts] = o;
+        }
+        __syncthreads();
+        // the cluster's keys, gathered into the output staging area (not yet in use)
+        uint32_t* c_all = reinterpret_cast<uint32_t*>(stage_smem);
+        for (uint32_t i = threadIdx.x; i < m; i += THREADS) {
+          int c = 0;
+          while (c + 1 < nparts && c_off[c + 1] <= i) ++c;
+          c_all[i] = cg::this_cluster().map_shared_rank(c_key, c)[i - c_off[c]];
+        }
+        ck = c_all;
+      }
+      __syncthreads();
+      if (m <= static_cast<uint32_t>(kCountMax)) {
+        // the threshold key is the candidate with fewer than `need` keys above it and at
+        // least `need` at or above it
+        if (threadIdx.x < m) {
+          const uint32_t kc = ck[threadIdx.x];
+          uint32_t gt = 0, ge = 0;
+#pragma unroll 8
+          for (uint32_t j = 0; j < m; ++j) {
+            const uint32_t v = ck[j];
+            gt += v > kc;
+            ge += v >= kc;
+          }
+          if (gt < need && need <= ge) {
+            sh_theta = kc;
+            sh_needt = need - gt;
+          }
+        }
+        __syncthreads();
+        prefix = sh_theta;
+        need = sh_needt;
+        shift = 0;
+      } else {
+#pragma unroll 1
+        while (shift > 0) {
+          const int wb = min(8, shift);
+          const int nbs = 1 << wb;
+          const int ns = shift - wb;
+          for (int i = threadIdx.x; i < nbs; i += THREADS) h_small[i] = 0;
+          __syncthreads();
+          for (uint32_t i = threadIdx.x; i < m; i += THREADS) {
+            const uint32_t u = ck[i];
+            if ((u >> shift) == prefix) atomicAdd(&h_small[(u >> ns) & (nbs - 1)], 1u);
+          }
+          __syncthreads();
+          if (warp == 0) {
+            // lane l owns bins nbs-1-l*bpl .. nbs-(l+1)*bpl: lane 0 the highest ones
+            const int bpl = nbs >= 32 ? nbs / 32 : 1;
+            const bool own = lane * bpl < nbs;
+            const int lb0 = nbs - (lane + 1) * bpl;
+            uint32_t c = 0;
+            if (own)
+              for (int q = 0; q < bpl; ++q) c += h_small[lb0 + q];
+            uint32_t incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+              const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+              if (lane >= o) incl += y;
+            }
+            if (own && incl - c < need && need <= incl) {
+              uint32_t above = incl - c;
+              for (int q = bpl - 1; q >= 0; --q) {
+                const uint32_t hc = h_small[lb0 + q];
+                if (above + hc >= need) {
+                  sh_bin = static_cast<uint32_t>(lb0 + q);
+                  sh_above = above;
+                  sh_inbin = hc;
+                  break;
+                }
+                above += hc;
+              }
+            }
+          }
+          __syncthreads();
+          need -= sh_above;
+          prefix = (prefix << wb) | sh_bin;
+          shift = ns;
+          const uint32_t ib = sh_inbin;
+          __syncthreads();  // h_small and the shared results are rewritten by the next digit
+          if (ib == need) break;
+        }
+      }
+      break;
+    }
   }
 
   // ---- output: one scan of (above, equal) counts, then each thread writes its run ------
@@ -516,35 +643,33 @@ select_reg_kernel(const SelectArgs a, int row0) {
   const uint32_t cta_sel = static_cast<uint32_t>(tot >> 32) +
                            min(eq_off + static_cast<uint32_t>(tot & kLow), need) - min(eq_off, need);
   uint32_t slot = gt_before + min(eq_before, need);
-  uint32_t eq_rank = eq_before;
+  // the equal keys this thread takes: its lowest-indexed ones, up to need over the row
+  const uint32_t eq_take =
+      need > eq_before ? min(need - eq_before, static_cast<uint32_t>(__popcll(eq_mask))) : 0u;
+  Mask sel = gt_mask;
+  {
+    Mask rest = eq_mask;
+    for (uint32_t q = 0; q < eq_take; ++q) {
+      const Mask low = rest & (~rest + 1);
+      sel |= low;
+      rest ^= low;
+    }
+  }
   const bool staged = K <= kStageMaxK;
   int32_t* st_idx = reinterpret_cast<int32_t*>(stage_smem);
-  uint32_t* st_key = reinterpret_cast<uint32_t*>(st_idx + (staged ? K : 0));
-#pragma unroll
-  for (int j = 0; j < ITEMS; ++j) {
-    bool sel = (gt_mask >> j) & 1u;
-    if ((eq_mask >> j) & 1u) {
-      sel = eq_rank < need;
-      ++eq_rank;
+  // selected elements in index order; scores are read back from the row (still in cache)
+  while (sel != 0 && slot < static_cast<uint32_t>(K)) {
+    const int64_t i = my0 + lowest_set_bit(sel);
+    sel &= sel - 1;
+    if (staged) {
+      st_idx[slot - cta_slot0] = static_cast<int32_t>(i);
+    } else {
+      int32_t id = in_idx ? in_idx[i] : static_cast<int32_t>(lo + i);
+      if (map != nullptr && id >= 0) id = map[id];
+      a.out_idx[out_base + slot] = id;
+      if (a.out_val) a.out_val[out_base + slot] = vals[i];
     }
-    if (sel) {
-      if (slot < static_cast<uint32_t>(K)) {
-        if (staged) {
-          st_idx[slot - cta_slot0] = static_cast<int32_t>(my0 + j);
-          st_key[slot - cta_slot0] = key[j];
-        } else {
-          const int64_t i = my0 + j;
-          int32_t id = in_idx ? in_idx[i] : static_cast<int32_t>(lo + i);
-          if (map != nullptr && id >= 0) id = map[id];
-          a.out_idx[out_base + slot] = id;
-          if (a.out_val) {
-            const uint32_t u = key[j];
-            a.out_val[out_base + slot] = __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
-          }
-        }
-      }
-      ++slot;
-    }
+    ++slot;
   }
   if (staged) {
     __syncthreads();
@@ -555,11 +680,7 @@ select_reg_kernel(const SelectArgs a, int row0) {
       int32_t id = in_idx ? in_idx[i] : static_cast<int32_t>(lo + i);
       if (map != nullptr && id >= 0) id = map[id];
       a.out_idx[out_base + cta_slot0 + sl] = id;
-      if (a.out_val) {
-        const uint32_t u = st_key[sl];
-        a.out_val[out_base + cta_slot0 + sl] =
-            __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
-      }
+      if (a.out_val) a.out_val[out_base + cta_slot0 + sl] = vals[i];
     }
   }
   for (int64_t j = n_sel_total + static_cast<int64_t>(part) * THREADS + threadIdx.x; j < K;
@@ -573,7 +694,7 @@ template <int THREADS, int DIGIT>
 cudaError_t launch_reg(const SelectArgs& a, int row0, int row1, cudaStream_t s, int* launched) {
   const int64_t grid = static_cast<int64_t>(row1 - row0) * a.n_seg;
   if (grid <= 0) return cudaSuccess;
-  const size_t smem = a.K <= kStageMaxK ? static_cast<size_t>(a.K) * 8 : 0;
+  const size_t smem = a.K <= kStageMaxK ? static_cast<size_t>(a.K) * 4 : 0;
   auto kern = select_reg_kernel<THREADS, DIGIT, kRegItems, false>;
   if (smem > 0) {
     const cudaError_t e =
@@ -605,7 +726,9 @@ cudaError_t launch_select_cluster(const SelectArgs& a, int ctas, cudaStream_t s,
       static_cast<int64_t>(a.len_cap) > static_cast<int64_t>(ctas) * kClusterThreads * kClusterItems)
     return cudaErrorInvalidValue;
   auto kern = select_reg_kernel<kClusterThreads, 12, kClusterItems, true>;
-  const size_t smem = a.K <= kStageMaxK ? static_cast<size_t>(a.K) * 8 : 0;
+  // output staging, which first holds the gathered keys of the threshold bin
+  const size_t smem = std::max<size_t>(a.K <= kStageMaxK ? static_cast<size_t>(a.K) * 4 : 0,
+                                       static_cast<size_t>(kGatherMax) * 4);
   if (smem > 0) {
     const cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));

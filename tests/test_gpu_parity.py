@@ -124,6 +124,41 @@ def test_negative_gates():
     _check_flat(p, idx, sc, range(300), "signed gates")
 
 
+def test_exact_ties_take_the_lowest_positions():
+    """Every key is one of 24 copies of one vector scaled by powers of two (exact in bf16 and
+    in every product), so each query's scores take 24 exact values in a fixed order, a factor
+    2 apart (or are all zero). One copy holds 60 % of the positions.
+    Across rows the K-th score is shared by tens to thousands of keys: the select resolves
+    the threshold by counting, by digits over the gathered keys of the threshold bin, or by
+    more passes over the whole row. Its set must equal the oracle's exactly: every key above
+    the K-th score and the lowest positions among the keys equal to it."""
+    T, K, nd, big = 16384, 2048, 24, 3
+    p = inputs.anchor_prefill(T, H=64, d=128, K=K, seed=18, device="cuda")
+    rng = np.random.default_rng(9)
+    which = np.where(rng.random(T) < 0.6, big, rng.integers(0, nd, T))
+    scales = torch.tensor([2.0 ** (nd - 13 - i) for i in range(nd)])
+    v = p["k"][0].float().cpu()
+    distinct = (scales[:, None] * v[None, :]).to(torch.bfloat16)     # [nd, d], decreasing
+    k = distinct[torch.as_tensor(which)].contiguous().cuda()
+    idx, sc, _ = indexer.index_prefill(p["q"], p["w"], k, K, with_scores=True)
+    idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+    q64, w64, d64 = f64(p["q"]), p["w"].double().cpu().numpy(), f64(distinct)
+    # rows 3042 .. 3322 leave 1878 .. 2045 keys in the threshold bin (gathered digits)
+    rows = sorted(set(_rows_sample(T, K, n=80, seed=5)) | set(range(3042, 3330, 40)) |
+                  {2100, 2500, 3500, 4000, 8000, 12000, 16383})
+    for t in rows:
+        vals = ox.score_keys(q64[t], w64[t], d64)
+        sv = np.sort(vals)
+        assert np.all(sv == 0) or np.allclose(sv[1:] / sv[:-1], 2.0), t
+        n = t + 1
+        row = vals[which[:n]]
+        order = np.lexsort((np.arange(n), -row))
+        m = min(K, n)
+        assert set(idx[t][:m].tolist()) == set(order[:m].tolist()), f"row {t}"
+        assert np.all(idx[t][m:] == -1)
+        assert np.all(np.diff(idx[t][:m]) > 0), f"row {t}: positions not ascending"
+
+
 # ---------------------------------------------------------------------------------------
 # group bank + refinement
 # ---------------------------------------------------------------------------------------
