@@ -226,6 +226,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a)
 // same cluster barriers.
 // ---------------------------------------------------------------------------------------
 constexpr int kRegItems = 32;      // elements per thread of the row-per-CTA classes
+constexpr int kWideItems = 36;     // ... of the 256-thread class for rows just above 8192
 constexpr int kClusterItems = 36;  // elements per thread of the cluster class
 constexpr int kClusterThreads = 512;
 constexpr int kClusterMaxCtas = 8;  // portable cluster size
@@ -690,12 +691,12 @@ select_reg_kernel(const SelectArgs a, int row0) {
   }
 }
 
-template <int THREADS, int DIGIT>
+template <int THREADS, int DIGIT, int ITEMS = kRegItems>
 cudaError_t launch_reg(const SelectArgs& a, int row0, int row1, cudaStream_t s, int* launched) {
   const int64_t grid = static_cast<int64_t>(row1 - row0) * a.n_seg;
   if (grid <= 0) return cudaSuccess;
   const size_t smem = a.K <= kStageMaxK ? static_cast<size_t>(a.K) * 4 : 0;
-  auto kern = select_reg_kernel<THREADS, DIGIT, kRegItems, false>;
+  auto kern = select_reg_kernel<THREADS, DIGIT, ITEMS, false>;
   if (smem > 0) {
     const cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -756,35 +757,40 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launched) {
   const int64_t grid = static_cast<int64_t>(a.rows) * a.n_seg;
   if (grid <= 0) return cudaSuccess;
   const int64_t seg = a.n_seg == 1 ? a.len_cap : a.seg_len;
-  constexpr int64_t c128 = 128 * kRegItems, c256 = 256 * kRegItems, c512 = 512 * kRegItems,
-                    c1024 = 1024 * kRegItems;
+  // row-length classes (CTA size x elements per thread): 128x32, 256x32, 256x36, 512x32,
+  // 1024x32; 256x36 takes rows just above 8192 (a bank of 8192 plus a window) at four CTAs
+  // per SM instead of half-empty 512-thread CTAs at two
+  constexpr int NC = 4;
+  constexpr int64_t cap[NC] = {128 * kRegItems, 256 * kRegItems, 256 * kWideItems,
+                               512 * kRegItems};
+  constexpr int64_t c1024 = 1024 * kRegItems;
   if (seg > c1024) {
     select_kernel<<<static_cast<unsigned>(grid), kSelThreads, 0, s>>>(a);
     *launched = 1;
     return cudaGetLastError();
   }
-  // rows of a causal prefix grow with the row index: split the launch by length class
-  int r128 = 0, r256 = 0, r512 = 0;
+  int end[NC];  // rows [end[c-1], end[c]) go to class c, rows from end[NC-1] on to 1024x32
   if (a.len_mode == 1 && a.n_seg == 1 && a.pos_step > 0) {
-    auto rows_upto = [&](int64_t cap) {  // first row whose length exceeds cap
-      const int64_t r = (cap - 1 - a.pos_base) / a.pos_step + 1;
-      return static_cast<int>(std::max<int64_t>(0, std::min<int64_t>(a.rows, r)));
+    // rows of a causal prefix grow with the row index: split the launch by length class
+    auto rows_upto = [&](int64_t c) {  // number of leading rows of length <= c
+      const int64_t num = c - 1 - a.pos_base;
+      if (num < 0) return 0;
+      return static_cast<int>(std::min<int64_t>(a.rows, num / a.pos_step + 1));
     };
-    r128 = rows_upto(c128);
-    r256 = std::max(r128, rows_upto(c256));
-    r512 = std::max(r256, rows_upto(c512));
-  } else if (seg <= c128) {
-    r128 = r256 = r512 = a.rows;
-  } else if (seg <= c256) {
-    r256 = r512 = a.rows;
-  } else if (seg <= c512) {
-    r512 = a.rows;
+    for (int c = 0; c < NC; ++c) end[c] = std::max(c ? end[c - 1] : 0, rows_upto(cap[c]));
+  } else {
+    int first = NC;  // smallest class that holds every row
+    for (int c = NC - 1; c >= 0; --c)
+      if (seg <= cap[c]) first = c;
+    for (int c = 0; c < NC; ++c) end[c] = c >= first ? a.rows : 0;
   }
   cudaError_t e;
-  if ((e = launch_reg<128, 10>(a, 0, r128, s, launched)) != cudaSuccess) return e;
-  if ((e = launch_reg<256, 11>(a, r128, r256, s, launched)) != cudaSuccess) return e;
-  if ((e = launch_reg<512, 12>(a, r256, r512, s, launched)) != cudaSuccess) return e;
-  return launch_reg<1024, 12>(a, r512, a.rows, s, launched);
+  if ((e = launch_reg<128, 10>(a, 0, end[0], s, launched)) != cudaSuccess) return e;
+  if ((e = launch_reg<256, 11>(a, end[0], end[1], s, launched)) != cudaSuccess) return e;
+  if ((e = launch_reg<256, 11, kWideItems>(a, end[1], end[2], s, launched)) != cudaSuccess)
+    return e;
+  if ((e = launch_reg<512, 12>(a, end[2], end[3], s, launched)) != cudaSuccess) return e;
+  return launch_reg<1024, 12>(a, end[3], a.rows, s, launched);
 }
 
 }  // namespace adx

@@ -341,6 +341,31 @@ def test_full_size_decode_sampled():
                    score_floor(q64[b], w64[b], keys), K, RTOL["e4m3"], sc[b], f"dfull {b}")
 
 
+@pytest.mark.parametrize("q_pos0", [4096, 8192])
+def test_bank_rows_starting_past_a_select_class(q_pos0):
+    """Bank scan rows grow by G per group; when the first one is just longer than a select
+    class holds (4097 and 8193 keys here), it must still go to a class that holds it. The
+    key at the last scanned position is planted far above the rest, so a bank that drops
+    it fails."""
+    G, B, Hg, T = 64, 512, 16, 3 * 64
+    S = q_pos0 + T
+    p = _to_cuda(inputs.anchor_prefill(T, H=64, d=128, K=B, seed=24, S=S, q_pos0=q_pos0))
+    qbar, wbar = inputs.mean_pool_group_queries(p["q"].float(), p["w"], G, Hg)
+    qbar = qbar.to(torch.bfloat16).contiguous()
+    qb64, wb64 = f64(qbar), wbar.double().cpu().numpy()
+    base = ox.score_keys(qb64[0], wb64[0], f64(p["k"][:q_pos0]))
+    p["k"][q_pos0] = (p["k"][int(np.argmax(base))].float() * 4).to(torch.bfloat16)
+    bank = indexer.group_bank(qbar, wbar, p["k"], G, B, "paper", q_pos0=q_pos0)
+    bank = bank.cpu().numpy()
+    k64 = f64(p["k"])
+    assert q_pos0 in bank[0, :B].tolist()
+    for g in range(T // G):
+        scan_n = q_pos0 + g * G + 1
+        keys = k64[:scan_n]
+        check_topk(bank[g, :B], np.arange(scan_n), ox.score_keys(qb64[g], wb64[g], keys),
+                   score_floor(qb64[g], wb64[g], keys), B, RTOL["bf16"], what=f"bank {g}")
+
+
 @pytest.mark.parametrize("mode", ["window", "paper"])
 def test_group_mode_on_a_later_chunk(mode):
     """Group mode for one query chunk of a longer prefix (q_pos0 > 0), as chunked prefill
