@@ -192,7 +192,9 @@ class StageTimer:
 
 def timed(fn, steps, warmup, dist, stage_timer=None):
     """W untimed steps, then exactly K timed steps between barriers; returns ms per step
-    (max over ranks) and the library's launch count inside the timed region."""
+    (max over ranks) and the library's launch count inside the timed region. With a stage
+    timer, K more steps follow with the library's stage events armed: those events are extra
+    stream operations between its kernels, so the timed steps run without them."""
     from sparse_attention_token_indexer_b200 import _lib
     for _ in range(warmup):
         fn()
@@ -203,17 +205,19 @@ def timed(fn, steps, warmup, dist, stage_timer=None):
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n0 = _lib.lib().adx_launch_count()
     start.record(s)
-    for i in range(steps):
-        if stage_timer:
-            stage_timer.arm(i)
+    for _ in range(steps):
         fn()
     end.record(s)
-    if stage_timer:
-        stage_timer.disarm()
     torch.cuda.synchronize()
     launches = _lib.lib().adx_launch_count() - n0
     dist.barrier()
     ms = dist.max(start.elapsed_time(end)) / steps
+    if stage_timer:
+        for i in range(steps):
+            stage_timer.arm(i)
+            fn()
+        stage_timer.disarm()
+        torch.cuda.synchronize()
     return ms, launches
 
 
