@@ -80,69 +80,107 @@ __device__ __forceinline__ void load8(const void* q, int64_t e, float sin, float
   }
 }
 
-template <bool IN_E4M3, bool OUT_E4M3>
-__global__ void __launch_bounds__(256)
+// THREADS threads per row; each thread holds up to G = 1024 / THREADS groups of 8 elements
+// in registers (rows of up to 8192 elements), so the row is read once and every load of a
+// thread is in flight together.
+template <bool IN_E4M3, bool OUT_E4M3, int THREADS>
+__global__ void __launch_bounds__(THREADS)
 prepare_q_kernel(const void* __restrict__ q_in, const float* __restrict__ q_scale_in,
                  const float* __restrict__ w, int H, int d, void* __restrict__ q_out,
                  float* __restrict__ q_scale_out, int8_t* __restrict__ fold_flag) {
-  __shared__ float red[8];
+  constexpr int G = 1024 / THREADS;
+  __shared__ float red[THREADS / 32];
   const int64_t r = blockIdx.x;
   const float* wr = w + r * H;
+  const int ng = H * d / 8;  // groups of 8 elements; a group lies within one head
+  const int64_t base = r * static_cast<int64_t>(H) * d;
+  const float sin = IN_E4M3 ? q_scale_in[r] : 1.f;
+  float x[G][8], g[G];
   int neg = 0;
-  for (int j = threadIdx.x; j < H; j += blockDim.x) neg |= wr[j] < 0.f;
+#pragma unroll
+  for (int k = 0; k < G; ++k) {
+    const int i = threadIdx.x + k * THREADS;
+    g[k] = 1.f;
+    if (i < ng) {
+      load8<IN_E4M3>(q_in, base + static_cast<int64_t>(i) * 8, sin, x[k]);
+      g[k] = wr[(i * 8) / d];
+      neg |= g[k] < 0.f;
+    }
+  }
+  // every head has d/8 groups, so the threads together have seen every gate of the row
   const bool fold = __syncthreads_or(neg) == 0;
   if (threadIdx.x == 0) fold_flag[r] = fold ? 1 : 0;
-  const int64_t n = static_cast<int64_t>(H) * d;
-  const int64_t base = r * n;
-  const float sin = IN_E4M3 ? q_scale_in[r] : 1.f;
   if constexpr (IN_E4M3 && OUT_E4M3) {
     if (!fold) {  // keep the given codes and scale
       const uint2* in = reinterpret_cast<const uint2*>(reinterpret_cast<const uint8_t*>(q_in) + base);
       uint2* out = reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(q_out) + base);
-      for (int64_t i = threadIdx.x; i < n / 8; i += blockDim.x) out[i] = in[i];
+      for (int i = threadIdx.x; i < ng; i += THREADS) out[i] = in[i];
       if (threadIdx.x == 0) q_scale_out[r] = sin;
       return;
     }
   }
-  // element groups of 8 share one head (d is a multiple of 8)
+  if (!fold) {
+#pragma unroll
+    for (int k = 0; k < G; ++k) g[k] = 1.f;
+  }
   float sc = 1.f;
   if constexpr (OUT_E4M3) {
     float amax = 0.f;
-    for (int64_t i = threadIdx.x; i < n / 8; i += blockDim.x) {
-      float x[8];
-      load8<IN_E4M3>(q_in, base + i * 8, sin, x);
-      const float g = fold ? wr[(i * 8) / d] : 1.f;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) amax = fmaxf(amax, fabsf(x[u] * g));
-    }
+    for (int k = 0; k < G; ++k)
+      if (threadIdx.x + k * THREADS < ng)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) amax = fmaxf(amax, fabsf(x[k][u] * g[k]));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
     __syncthreads();
     float m = 0.f;
-    for (int i2 = 0; i2 < static_cast<int>(blockDim.x / 32); ++i2) m = fmaxf(m, red[i2]);
+#pragma unroll
+    for (int i2 = 0; i2 < THREADS / 32; ++i2) m = fmaxf(m, red[i2]);
     sc = m > 0.f ? m / 448.f : 1.f;
     if (threadIdx.x == 0) q_scale_out[r] = sc;
   }
-  for (int64_t i = threadIdx.x; i < n / 8; i += blockDim.x) {
-    float x[8];
-    load8<IN_E4M3>(q_in, base + i * 8, sin, x);
-    const float g = fold ? wr[(i * 8) / d] : 1.f;
+#pragma unroll
+  for (int k = 0; k < G; ++k) {
+    const int i = threadIdx.x + k * THREADS;
+    if (i >= ng) continue;
     if constexpr (OUT_E4M3) {
       uint2 v;
       uint8_t* c = reinterpret_cast<uint8_t*>(&v);
 #pragma unroll
       for (int u = 0; u < 8; ++u)
-        c[u] = static_cast<uint8_t>(__nv_cvt_float_to_fp8((x[u] * g) / sc, __NV_SATFINITE, __NV_E4M3));
+        c[u] = static_cast<uint8_t>(
+            __nv_cvt_float_to_fp8((x[k][u] * g[k]) / sc, __NV_SATFINITE, __NV_E4M3));
       reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(q_out) + base)[i] = v;
     } else {
       uint4 v;
       __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) h[u] = __floats2bfloat162_rn(x[2 * u] * g, x[2 * u + 1] * g);
+      for (int u = 0; u < 4; ++u)
+        h[u] = __floats2bfloat162_rn(x[k][2 * u] * g[k], x[k][2 * u + 1] * g[k]);
       reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(q_out) + base)[i] = v;
     }
   }
+}
+
+template <bool IN_E4M3, bool OUT_E4M3>
+cudaError_t launch_prepare_rows(const void* q, const float* q_scale, const float* w, int64_t rows,
+                                int H, int d, void* q_out, float* q_scale_out, int8_t* fold_flag,
+                                cudaStream_t s) {
+  // few rows (decode): spread each row over more threads
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return cudaErrorUnknown;
+  const unsigned g = static_cast<unsigned>(rows);
+  if (rows < 2ll * sms)
+    prepare_q_kernel<IN_E4M3, OUT_E4M3, 1024>
+        <<<g, 1024, 0, s>>>(q, q_scale, w, H, d, q_out, q_scale_out, fold_flag);
+  else
+    prepare_q_kernel<IN_E4M3, OUT_E4M3, 256>
+        <<<g, 256, 0, s>>>(q, q_scale, w, H, d, q_out, q_scale_out, fold_flag);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -151,16 +189,17 @@ cudaError_t launch_prepare_q(const void* q, const float* q_scale, bool in_e4m3, 
                              const float* w, int64_t rows, int H, int d, void* q_out,
                              float* q_scale_out, int8_t* fold_flag, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
-  const unsigned g = static_cast<unsigned>(rows);
+  if (static_cast<int64_t>(H) * d > 8192 || d % 8 != 0) return cudaErrorNotSupported;
   if (!in_e4m3 && !out_e4m3)
-    prepare_q_kernel<false, false><<<g, 256, 0, s>>>(q, q_scale, w, H, d, q_out, q_scale_out, fold_flag);
-  else if (in_e4m3 && out_e4m3)
-    prepare_q_kernel<true, true><<<g, 256, 0, s>>>(q, q_scale, w, H, d, q_out, q_scale_out, fold_flag);
-  else if (!in_e4m3 && out_e4m3)
-    prepare_q_kernel<false, true><<<g, 256, 0, s>>>(q, q_scale, w, H, d, q_out, q_scale_out, fold_flag);
-  else
-    return cudaErrorNotSupported;
-  return cudaGetLastError();
+    return launch_prepare_rows<false, false>(q, q_scale, w, rows, H, d, q_out, q_scale_out,
+                                             fold_flag, s);
+  if (in_e4m3 && out_e4m3)
+    return launch_prepare_rows<true, true>(q, q_scale, w, rows, H, d, q_out, q_scale_out,
+                                           fold_flag, s);
+  if (!in_e4m3 && out_e4m3)
+    return launch_prepare_rows<false, true>(q, q_scale, w, rows, H, d, q_out, q_scale_out,
+                                            fold_flag, s);
+  return cudaErrorNotSupported;
 }
 
 cudaError_t launch_pack_candidates(const void* k, const float* k_scale, int64_t key_batch_stride,
