@@ -124,6 +124,28 @@ def test_negative_gates():
     _check_flat(p, idx, sc, range(300), "signed gates")
 
 
+def test_rows_where_most_scores_are_exactly_zero():
+    """A ReLU sum is exactly 0 for a key no head responds to. Here 85 % of the keys are -e_0
+    and every query head has a positive first component, so most of each row scores exactly
+    0: the row minimum holds most keys (counted apart from the histogram atomics), and in
+    many rows the K-th score is 0 itself."""
+    T, K = 3000, 256
+    p = _to_cuda(inputs.anchor_prefill(T, H=64, d=128, K=K, seed=19))
+    q = p["q"].float()
+    q[..., 0] = q[..., 0].abs() + 3.0
+    p["q"] = q.to(torch.bfloat16).contiguous()
+    rng = np.random.default_rng(11)
+    dead = torch.as_tensor(rng.random(T) < 0.85, device="cuda")
+    k = p["k"].clone()
+    k[dead] = 0
+    k[dead, 0] = -1.0
+    p["k"] = k
+    idx, sc, _ = indexer.index_prefill(p["q"], p["w"], p["k"], K, with_scores=True)
+    ref = _check_flat(p, idx, sc, _rows_sample(T, K, n=60, seed=6), "zeros")
+    zero_rows = [t for t, (_, cs, _) in ref.items() if len(cs) > K and np.sort(cs)[-K] == 0]
+    assert len(zero_rows) >= 5, "the K-th score is 0 in too few sampled rows"
+
+
 def test_exact_ties_take_the_lowest_positions():
     """Every key is one of 24 copies of one vector scaled by powers of two (exact in bf16 and
     in every product), so each query's scores take 24 exact values in a fixed order, a factor
