@@ -373,20 +373,28 @@ select_reg_kernel(const SelectArgs a, int row0) {
       cl_red[1] = kmax;
       cl_red[2] = nval;
     }
-    cg::this_cluster().sync();
-    kmin = 0xffffffffu;
-    kmax = 0u;
-    nval = 0u;
-    // fixed trip count: the remote loads of all CTAs are in flight together
-#pragma unroll
-    for (int c = 0; c < kClusterMaxCtas; ++c) {
-      if (c < nparts) {
-        const uint32_t* rc = cg::this_cluster().map_shared_rank(cl_red, c);
-        kmin = min(kmin, rc[0]);
-        kmax = max(kmax, rc[1]);
-        nval += rc[2];
+    cg::this_cluster().sync();  // also a CTA barrier: red_* are free again
+    if (warp == 0) {  // lane c reads CTA c's values
+      uint32_t mn = 0xffffffffu, mx = 0u, nv = 0u;
+      if (lane < nparts) {
+        const uint32_t* rc = cg::this_cluster().map_shared_rank(cl_red, lane);
+        mn = rc[0];
+        mx = rc[1];
+        nv = rc[2];
+      }
+      mn = __reduce_min_sync(0xffffffffu, mn);
+      mx = __reduce_max_sync(0xffffffffu, mx);
+      nv = __reduce_add_sync(0xffffffffu, nv);
+      if (lane == 0) {
+        red_min[0] = mn;
+        red_max[0] = mx;
+        red_cnt[0] = nv;
       }
     }
+    __syncthreads();
+    kmin = red_min[0];
+    kmax = red_max[0];
+    nval = red_cnt[0];
   }
 
   uint32_t prefix = 0;
@@ -449,9 +457,67 @@ select_reg_kernel(const SelectArgs a, int row0) {
     }
     unsigned long long tot64;
     const uint32_t excl = static_cast<uint32_t>(block_exclusive_scan64<THREADS>(mine, warp_tot64, tot64));
-    if (owner && excl < need && need <= excl + mine) {
+    const bool finder = owner && excl < need && need <= excl + mine;
+    constexpr int BPT = NB >= THREADS ? NB / THREADS : 1;
+    if constexpr (CLUSTER && BPT == 8 && kClusterMaxCtas == 8) {
+      // The finder's warp reads the finder's bins from every CTA together: lane 8*c4 + j
+      // loads bin j of CTAs c4 and c4 + 4; shuffles add the CTAs up.
+      const unsigned fm = __ballot_sync(0xffffffffu, finder);
+      if (fm != 0u && bpt == BPT) {
+        const int fl = __ffs(fm) - 1;
+        const int fb0 = __shfl_sync(0xffffffffu, b0, fl);
+        const int c4 = lane >> 3, j = lane & 7;
+        const int bin = fb0 + BPT - 1 - j;
+        uint32_t v = 0;
+        if (c4 < nparts) v += cg::this_cluster().map_shared_rank(h, c4)[bin];
+        if (c4 + 4 < nparts) v += cg::this_cluster().map_shared_rank(h, c4 + 4)[bin];
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        uint32_t cnt[BPT];
+#pragma unroll
+        for (int q = 0; q < BPT; ++q) cnt[q] = __shfl_sync(0xffffffffu, v, q);
+        if (lane == fl) {
+          uint32_t above = excl;
+#pragma unroll
+          for (int q = 0; q < BPT; ++q) {
+            if (above < need) {
+              if (above + cnt[q] >= need) {
+                sh_bin = static_cast<uint32_t>(fb0 + BPT - 1 - q);
+                sh_above = above;
+                sh_inbin = cnt[q];
+              }
+              above += cnt[q];
+            }
+          }
+        }
+      } else if (finder) {
+        uint32_t cnt[BPT];
+#pragma unroll
+        for (int q = 0; q < BPT; ++q) cnt[q] = 0;
+#pragma unroll
+        for (int c = 0; c < kClusterMaxCtas; ++c) {
+          if (c < nparts) {
+            const uint32_t* hc = cg::this_cluster().map_shared_rank(h, c);
+#pragma unroll
+            for (int q = 0; q < BPT; ++q)
+              if (q < bpt) cnt[q] += hc[b0 + bpt - 1 - q];
+          }
+        }
+        uint32_t above = excl;
+#pragma unroll
+        for (int q = 0; q < BPT; ++q) {
+          if (q < bpt && above < need) {
+            if (above + cnt[q] >= need) {
+              sh_bin = static_cast<uint32_t>(b0 + bpt - 1 - q);
+              sh_above = above;
+              sh_inbin = cnt[q];
+            }
+            above += cnt[q];
+          }
+        }
+      }
+    } else if (finder) {
       // the row's count of each of this thread's bins, highest bin first
-      constexpr int BPT = NB >= THREADS ? NB / THREADS : 1;
       uint32_t cnt[BPT];
 #pragma unroll
       for (int j = 0; j < BPT; ++j) cnt[j] = 0;
@@ -504,13 +570,16 @@ select_reg_kernel(const SelectArgs a, int row0) {
       const uint32_t* ck = c_key;
       if constexpr (CLUSTER) {
         cg::this_cluster().sync();
-        if (threadIdx.x == 0) {
-          uint32_t o = 0;
-          for (int c = 0; c < nparts; ++c) {
-            c_off[c] = o;
-            o += *cg::this_cluster().map_shared_rank(&sh_ccount, c);
+        if (warp == 0) {  // lane c reads CTA c's count
+          const uint32_t cnt =
+              lane < nparts ? *cg::this_cluster().map_shared_rank(&sh_ccount, lane) : 0u;
+          uint32_t incl = cnt;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
           }
-          c_off[nparts] = o;
+          if (lane <= nparts) c_off[lane] = incl - cnt;
         }
         __syncthreads();
         // the cluster's keys, gathered into the output staging area (not yet in use)
@@ -621,18 +690,25 @@ select_reg_kernel(const SelectArgs a, int row0) {
   unsigned long long off = 0, all = tot;
   if constexpr (CLUSTER) {
     if (threadIdx.x == 0) cl_tot = tot;
-    cg::this_cluster().sync();
-    all = 0;
+    cg::this_cluster().sync();  // also a CTA barrier: warp_tot64 is free again
+    if (warp == 0) {  // lane c reads CTA c's counts
+      const unsigned long long v =
+          lane < nparts ? *cg::this_cluster().map_shared_rank(&cl_tot, lane) : 0ull;
+      unsigned long long lower = lane < part ? v : 0ull, sum = v;
 #pragma unroll
-    for (int c = 0; c < kClusterMaxCtas; ++c) {
-      if (c < nparts) {
-        const unsigned long long v = *cg::this_cluster().map_shared_rank(&cl_tot, c);
-        if (c < part) off += v;
-        all += v;
+      for (int o = 16; o > 0; o >>= 1) {
+        lower += __shfl_xor_sync(0xffffffffu, lower, o);
+        sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      }
+      if (lane == 0) {
+        warp_tot64[0] = lower;
+        warp_tot64[1] = sum;
       }
     }
-    // no CTA leaves while another may still read its shared memory
+    // no CTA leaves while another may still read its shared memory; also a CTA barrier
     cg::this_cluster().sync();
+    off = warp_tot64[0];
+    all = warp_tot64[1];
   }
   const uint32_t gt_before = static_cast<uint32_t>((off + ex) >> 32);
   const uint32_t eq_before = static_cast<uint32_t>((off + ex) & kLow);
