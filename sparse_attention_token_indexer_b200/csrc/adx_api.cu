@@ -223,7 +223,8 @@ adx_status run_score(const ScorePlan& p, const void* q_codes, const void* keys, 
   const int n = p.tok * p.H;
   if (!encode_rows(&tq, q_codes, p.fp8, p.d, static_cast<int64_t>(p.a.R) * p.H, n))
     return ADX_EINVAL;
-  if (!encode_rows(&tk, keys, p.fp8, p.d, key_rows, kTileM)) return ADX_EINVAL;
+  // gathered keys (tile::gather4) need one-row boxes
+  if (!encode_rows(&tk, keys, p.fp8, p.d, key_rows, p.a.key_idx ? 1 : kTileM)) return ADX_EINVAL;
   if (p.a.n_items <= 0) return ADX_OK;
   const int bps = score_blocks_per_sm(p.fp8, p.H, p.d, p.tok);
   const int grid = std::min<int64_t>(p.a.n_items, static_cast<int64_t>(sm_count()) * bps);
@@ -416,8 +417,10 @@ size_t ws_refine(const adx_operands* o, int G, int B, int mode, int K) {
   const int64_t ng = dec ? o->T : o->T / G;
   const int64_t rows = dec ? o->T : ng * G;
   size_t b = kStatusBytes + ws_prepare(o, rows);
-  b += align_up(static_cast<size_t>(ng) * bcp * row_bytes(o), kAlign);  // packed keys
-  b += align_up(static_cast<size_t>(ng) * bcp * 4, kAlign) * 2;          // scales, positions
+  if (!dec) {  // packed candidate keys, scales, positions (decode gathers them instead)
+    b += align_up(static_cast<size_t>(ng) * bcp * row_bytes(o), kAlign);
+    b += align_up(static_cast<size_t>(ng) * bcp * 4, kAlign) * 2;
+  }
   b += align_up(static_cast<size_t>(rows) * bcp * 4, kAlign);             // scores
   b += select_scratch_bytes(rows, bcp, K);
   if (!dec && rows < o->T) {
@@ -619,23 +622,34 @@ adx_status adx_bank_refine(const adx_operands* o, int32_t G, int32_t B, int32_t 
   if (rows > 0) {
     Prepared pq;
     if ((r = prepare(o, o->q, o->q_scale, o->w, rows, cv, s, pq)) != ADX_OK) return r;
-    const int rb = row_bytes(o);
-    uint8_t* packed = cv.take<uint8_t>(static_cast<size_t>(ng) * bcp * rb);
-    float* pscale = cv.take<float>(static_cast<size_t>(ng) * bcp * 4);
-    int32_t* ppos = cv.take<int32_t>(static_cast<size_t>(ng) * bcp * 4);
     float* scores = cv.take<float>(static_cast<size_t>(rows) * bcp * 4);
-    if (counted(launch_pack_candidates(o->k, o->k_scale, o->S, dec ? 1 : 0, o->S, bank_idx,
-                                       static_cast<int32_t>(ng), bs.width,
-                                       static_cast<int32_t>(bcp), rb, packed,
-                                       fp8_keys(o) ? pscale : nullptr, ppos, s)) != cudaSuccess)
-      return ADX_ECUDA;
     ScorePlan p;
+    const void* keys = o->k;
+    int64_t key_rows = 0;
+    const int32_t* slot_pos = bank_idx;  // candidate slot -> key position, for the select
+    int64_t slot_stride = bs.width;
     if (dec) {
+      // one query per group: its candidate keys are gathered straight from its own
+      // sequence (tile::gather4), slot c of sequence g at position bank_idx[g, c]
       p = rowwise_plan(o, pq, scores, bcp);
+      p.a.key_idx = bank_idx;
+      p.a.key_idx_stride = bs.width;
+      p.a.n_idx = bs.width;
+      p.a.S_valid = o->S;
+      key_rows = static_cast<int64_t>(o->T) * o->S;
     } else {
+      // G queries share a group's candidates: pack them once into contiguous rows, which
+      // every row block of the group then streams with whole-tile loads
+      const int rb = row_bytes(o);
+      uint8_t* packed = cv.take<uint8_t>(static_cast<size_t>(ng) * bcp * rb);
+      float* pscale = cv.take<float>(static_cast<size_t>(ng) * bcp * 4);
+      int32_t* ppos = cv.take<int32_t>(static_cast<size_t>(ng) * bcp * 4);
+      if (counted(launch_pack_candidates(o->k, o->k_scale, o->S, 0, o->S, bank_idx,
+                                         static_cast<int32_t>(ng), bs.width,
+                                         static_cast<int32_t>(bcp), rb, packed,
+                                         fp8_keys(o) ? pscale : nullptr, ppos, s)) != cudaSuccess)
+        return ADX_ECUDA;
       p = base_plan(o, pq, score_tokens_per_tile(o->H));
-      p.a.scores = scores;
-      p.a.score_ld = bcp;
       p.a.pos_base = o->q_pos0;
       p.a.pos_step = 1;
       p.a.R = static_cast<int32_t>(rows);
@@ -643,19 +657,25 @@ adx_status adx_bank_refine(const adx_operands* o, int32_t G, int32_t B, int32_t 
       p.a.n_batches = static_cast<int32_t>(ng);
       p.a.row_blocks_per_batch = (G + p.tok - 1) / p.tok;
       p.a.round_robin = 1;  // a group's row blocks run together and share its packed keys
+      p.a.scores = scores;
+      p.a.score_ld = bcp;
+      p.a.k_scale = fp8_keys(o) ? pscale : nullptr;
+      p.a.key_pos = ppos;
+      keys = packed;
+      key_rows = ng * bcp;
+      slot_pos = ppos;
+      slot_stride = bcp;
     }
-    p.a.k_scale = fp8_keys(o) ? pscale : nullptr;
-    p.a.key_pos = ppos;
-    p.a.key_batch_stride = bcp;
+    p.a.key_batch_stride = dec ? o->S : bcp;
     p.a.keys_per_batch = static_cast<int32_t>(bcp);
     p.a.status = st;
     finish_plan(p, bcp / kTileM);
-    if ((r = run_score(p, pq.q, packed, ng * bcp, s)) != ADX_OK) return r;
+    if ((r = run_score(p, pq.q, keys, key_rows, s)) != ADX_OK) return r;
     SelectArgs sa{};
     sa.vals = scores;
     sa.ld = bcp;
-    sa.idx_map = ppos;
-    sa.map_stride = bcp;
+    sa.idx_map = slot_pos;
+    sa.map_stride = slot_stride;
     sa.rows_per_batch = dec ? 1 : G;
     sa.len_mode = 0;
     sa.len_fixed = static_cast<int32_t>(bcp);

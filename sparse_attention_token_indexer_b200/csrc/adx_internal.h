@@ -26,12 +26,20 @@ constexpr int kTileM = 128;  // keys per MMA tile (TMEM lanes)
 // key range of keys_per_batch rows in the key tensor map, starting at row
 // b * key_batch_stride. The position of row r is seq_len[b] - 1 when seq_len is given
 // (decode), else pos_base + r * pos_step. Key c of batch b sits at position key_pos[...]
-// when key_pos is given (packed candidate lists), else at position c.
+// when key_pos is given (packed candidate lists), at the position the index list gives for
+// slot c with gathered keys (key_idx), else at position c.
 struct ScoreArgs {
   const float* w;          // [R, H] gates
   const float* q_scale;    // [R] or null
   const float* k_scale;    // [n_batches * key_batch_stride] or null
   const int32_t* key_pos;  // [n_batches * key_batch_stride] or null
+  // Gathered keys (a key tensor map with one-row boxes): slot c < keys_per_batch of batch b is
+  // the key at position key_idx[b * key_idx_stride + c] (c < n_idx) of the batch's key range;
+  // a negative position, one >= S_valid, or c >= n_idx is no key. Null: contiguous key rows.
+  const int32_t* key_idx;
+  int64_t key_idx_stride;
+  int32_t n_idx;
+  int32_t S_valid;
   const int32_t* seq_len;  // [n_batches] or null
   const int8_t* fold_flag; // [R]: 1 = the row's queries carry its gates already; null = none do
   float* scores;           // [R, score_ld]
@@ -85,6 +93,7 @@ struct SelectArgs {
 // Launchers (return a cudaError_t from the launch).
 cudaError_t launch_score(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const ScoreArgs& a,
                          bool fp8, int H, int d, int tok, int grid, cudaStream_t s);
+// tm_k must have one-row boxes when a.key_idx is set (gathered keys).
 int score_tokens_per_tile(int H);  // tokens per N tile for a head count (0 = unsupported)
 bool score_config_supported(bool fp8, int H, int d);
 // Launches one to three kernels (row-length classes); *launched receives how many.

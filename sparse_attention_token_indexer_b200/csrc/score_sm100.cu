@@ -38,12 +38,13 @@ __host__ __device__ constexpr int pow2ceil(int x) {
   return p;
 }
 
-template <int H_, int TOK_, int DB_, bool FP8_>
+template <int H_, int TOK_, int DB_, bool FP8_, bool GATHER_ = false>
 struct Cfg {
   static constexpr int H = H_;
   static constexpr int TOK = TOK_;
   static constexpr int DB = DB_;             // bytes per q/k row (d * element size)
   static constexpr bool FP8 = FP8_;
+  static constexpr bool GATHER = GATHER_;    // key tiles gathered row by row (tile::gather4)
   static constexpr int N = TOK * H;          // MMA N
   static constexpr int KC = DB / 128;        // 128-byte K chunks
   static constexpr int ELEMS_PER_CHUNK = FP8 ? 128 : 64;
@@ -75,7 +76,9 @@ struct Cfg {
   static constexpr int NBAR = 2 * ST + 2 * ACC + 3;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_SCAN = OFF_MISC + 64;
-  static constexpr int SMEM = OFF_SCAN + 8 * (THREADS / 32) + 1024;  // + alignment slack
+  // gathered key rows of a tile, read as 16-byte vectors
+  static constexpr int OFF_IDX = (OFF_SCAN + 8 * (THREADS / 32) + 15) / 16 * 16;
+  static constexpr int SMEM = OFF_IDX + (GATHER ? kTileM * 4 : 0) + 1024;  // + alignment slack
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "invalid MMA N");
   static_assert(DB % 128 == 0, "rows must be a multiple of 128 bytes");
   static_assert(QBYTES % 1024 == 0 && KBYTES % 1024 == 0, "alignment");
@@ -84,6 +87,7 @@ struct Cfg {
                 "epilogue chunking");
   static_assert(THREADS <= kMaxThreads, "block size");
   static_assert(ACC % EG == 0, "every epilogue warpgroup owns the same number of buffers");
+  static_assert(OFF_IDX % 16 == 0 && OFF_BAR % 8 == 0 && OFF_K % 1024 == 0, "alignment");
 };
 
 // One row block of the work: TOK consecutive query rows of one key batch and the key
@@ -112,7 +116,7 @@ __device__ __forceinline__ void block_info(const ScoreArgs& a, int i, Block& x) 
   x.ntiles = 0;
   if (x.row0 >= x.row_end) return;
   int64_t nk;
-  if (a.key_pos != nullptr) {
+  if (a.key_pos != nullptr || a.key_idx != nullptr) {
     nk = a.keys_per_batch;
   } else if (a.seq_len != nullptr) {
     nk = min(static_cast<int64_t>(a.seq_len[x.b]), static_cast<int64_t>(a.keys_per_batch));
@@ -335,7 +339,90 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   const int nblocks = a.row_blocks_per_batch * a.n_batches;
   const WorkIter work0{start, end, base0, b0, nblocks, a.round_robin != 0};
 
-  if (warp == 0) {
+  if (warp == 0 && C::GATHER) {
+    // ---------------------------------------------- TMA producer, gathered key rows
+    // The warp reads a tile's 128 key positions (4 per lane) into shared memory; lane 0
+    // waits for the stage, then issues 32 four-row gathers per 128-byte column chunk.
+    int32_t* idx_s = reinterpret_cast<int32_t*>(smem + C::OFF_IDX);
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t q_phase = 0;
+    bool q_loaded = false;
+    uint32_t issued_mask = 0, issued_parity = 0;
+    WorkIter work = work0;
+    Block x;
+    int t_lo, t_hi;
+    int ok = 1;
+    while (ok && !*abort_s && work.next<C::TOK>(a, x, t_lo, t_hi)) {
+      if (lane == 0) {
+        if (q_loaded && !mbar_wait(q_empty, q_phase ^ 1u, abort_s, a.timeout_ns)) {
+          ok = 0;
+        } else {
+          mbar_arrive_expect_tx(q_full, C::QBYTES);
+#pragma unroll
+          for (int kc = 0; kc < C::KC; ++kc)
+            tma_load_2d(q_s + kc * C::N * 128, &tm_q, q_full, kc * C::ELEMS_PER_CHUNK,
+                        x.row0 * C::H);
+          q_loaded = true;
+          q_phase ^= 1u;
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      const int32_t* kidx = a.key_idx + static_cast<int64_t>(x.b) * a.key_idx_stride;
+      // rows of tile t held by this lane (tile rows lane*4 .. lane*4+3); a slot with no key
+      // loads some row of the range, and the epilogue masks it
+      auto tile_rows = [&](int t, int32_t (&r)[4]) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = t * kTileM + lane * 4 + u;
+          const int32_t p = c < a.n_idx ? kidx[c] : -1;
+          const bool v = p >= 0 && p < a.S_valid;
+          r[u] = static_cast<int32_t>(x.key_row0 + (v ? p : 0));
+        }
+      };
+      int32_t nxt[4];
+      if (t_lo < t_hi) tile_rows(t_lo, nxt);
+      for (int t = t_lo; t < t_hi; ++t) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) idx_s[lane * 4 + u] = nxt[u];
+        if (t + 1 < t_hi) tile_rows(t + 1, nxt);  // in flight while lane 0 issues this tile
+        __syncwarp();
+        if (lane == 0) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_s, a.timeout_ns)) {
+            ok = 0;
+          } else {
+            mbar_arrive_expect_tx(&full[stage], C::KBYTES);
+#pragma unroll
+            for (int kc = 0; kc < C::KC; ++kc) {
+#pragma unroll 8
+              for (int g = 0; g < kTileM / 4; ++g) {
+                const int4 rr = *reinterpret_cast<const int4*>(idx_s + 4 * g);
+                tma_gather4_2d(k_s + stage * C::KBYTES + kc * kTileM * 128 + g * 512, &tm_k,
+                               &full[stage], kc * C::ELEMS_PER_CHUNK, rr.x, rr.y, rr.z, rr.w);
+              }
+            }
+            issued_mask |= 1u << stage;
+            issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);  // also: lane 0 has read idx_s
+        if (!ok) break;
+        if (++stage == C::ST) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (lane == 0) {
+      if (*abort_s) raise_timeout(a, 0);
+      // drain: every issued copy must land before the CTA may exit
+      for (int s2 = 0; s2 < C::ST; ++s2)
+        if (issued_mask & (1u << s2))
+          drain_wait(&full[s2], (issued_parity >> s2) & 1u, a.timeout_ns);
+      if (q_loaded) drain_wait(q_full, q_phase ^ 1u, a.timeout_ns);
+    }
+  } else if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int stage = 0;
@@ -480,7 +567,16 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         const int c = t * kTileM + m;
         kpos = c;
         ks = 1.f;
-        if (c < x.nkeys) {
+        if constexpr (C::GATHER) {
+          kpos = INT64_MAX;  // no key: never visible
+          if (c < x.nkeys && c < a.n_idx) {
+            const int32_t p = a.key_idx[static_cast<int64_t>(x.b) * a.key_idx_stride + c];
+            if (p >= 0 && p < a.S_valid) {
+              kpos = p;
+              if (a.k_scale != nullptr) ks = a.k_scale[x.key_row0 + p];
+            }
+          }
+        } else if (c < x.nkeys) {
           const int64_t kr = x.key_row0 + c;
           if (a.key_pos != nullptr) kpos = a.key_pos[kr];
           if (a.k_scale != nullptr) ks = a.k_scale[kr];
@@ -622,9 +718,11 @@ bool score_config_supported(bool fp8, int H, int d) {
 // key batch: decode and its bank refresh).
 cudaError_t launch_score(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const ScoreArgs& a,
                          bool fp8, int H, int d, int tok, int grid, cudaStream_t s) {
+  const bool gather = a.key_idx != nullptr;
 #define ADX_CASE(FP, HH, TT, DD)                                                        \
   if (fp8 == FP && H == HH && tok == TT && d == DD)                                     \
-    return launch_cfg<Cfg<HH, TT, (FP ? DD : 2 * DD), FP>>(tm_q, tm_k, a, grid, s);
+    return gather ? launch_cfg<Cfg<HH, TT, (FP ? DD : 2 * DD), FP, true>>(tm_q, tm_k, a, grid, s) \
+                  : launch_cfg<Cfg<HH, TT, (FP ? DD : 2 * DD), FP>>(tm_q, tm_k, a, grid, s);
   ADX_SCORE_CONFIGS(ADX_CASE)
 #undef ADX_CASE
   return cudaErrorNotSupported;

@@ -96,6 +96,19 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// Four rows y0..y3 (any order, any distance) of a 2D tensor map whose box is one row high,
+// columns x .. x + box width, written to consecutive rows of smem_dst with the map's swizzle.
+__device__ __forceinline__ void tma_gather4_2d(void* smem_dst, const CUtensorMap* map,
+                                               uint64_t* bar, int32_t x, int32_t y0, int32_t y1,
+                                               int32_t y2, int32_t y3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
+      ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
+        "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
+      : "memory");
+}
+
 // ------------------------------------------------------------------------------------
 // tcgen05
 // ------------------------------------------------------------------------------------
