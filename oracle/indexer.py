@@ -206,3 +206,29 @@ def decode_refine(q, w, caches, seq_len, banks, anchors, K):
     return {b: refine_row(q[b], w[b], caches[b], banks[b], int(anchors[b]) + 1,
                           int(seq_len[b]) - 1, K)
             for b in range(q.shape[0])}
+
+
+# ---------------------------------------------------------------------------------------
+# MTP target verification (one window of m queries per sequence)
+# ---------------------------------------------------------------------------------------
+
+def mtp_topk(q, w, caches, qbar, wbar, seq_len, m, G, P, K):
+    """ADIndex §4.3 ("Application to Prefill and MTP") and Appendix A.2 ("Bank Sharing During
+    MTP Target Verification"): each sequence b verifies a window of m queries, rows
+    b*m .. b*m+m-1 of q, w. Its cache holds seq_len[b] keys, the window's own included, so
+    window query j sits at position seq_len[b] - m + j and the first one sees
+    N_b = seq_len[b] - m + 1 keys. The window is split into m/G groups of G queries (group
+    queries qbar[b*m/G + g], wbar[...]), each with its own bank of P keys built over the
+    history visible to its anchor, the group's first query. When N_b <= P the whole window
+    uses the plain indexer instead (window-level fallback). Returns {row: Top-K positions}.
+    """
+    out = {}
+    gps = m // G
+    for b in range(len(caches)):
+        q_pos0 = int(seq_len[b]) - m
+        res, _ = group_topk(q[b * m:(b + 1) * m], w[b * m:(b + 1) * m], caches[b],
+                            qbar[b * gps:(b + 1) * gps], wbar[b * gps:(b + 1) * gps], q_pos0,
+                            G, P, K, "paper", fallback="window")
+        for j, v in res.items():
+            out[b * m + j] = v
+    return out

@@ -287,3 +287,59 @@ def test_table5_reproduced_by_the_group_plan():
                 # (a) and (c) use the integral of Eq. (19); the discrete count differs from it
                 # by less than one unit in the last printed digit
                 assert abs(got - ref) <= 0.0101, (panel, G, P, L, got)
+
+
+# ---------------------------------------------------------------------------------------
+# MTP target verification (ADIndex §4.3 and Appendix A.2)
+# ---------------------------------------------------------------------------------------
+
+def _relu_scores(qh, wh, keys):
+    """Eq. (1) written out with einsum, independent of the oracle's score_keys."""
+    return (np.maximum(np.einsum("hd,nd->hn", qh, keys), 0.0) * wh[:, None]).sum(axis=0)
+
+
+def test_mtp_window_fallback_is_flat_even_past_the_budget():
+    """N <= P sends the whole window to the plain indexer, also for groups whose anchors
+    already see more than P keys (the per-group prefill rule would bank those)."""
+    rng = np.random.default_rng(40)
+    m, G, P, K, H, d = 16, 4, 40, 8, 3, 8
+    N = P - 2
+    n = N + m - 1
+    k = rng.standard_normal((n, d))
+    q = rng.standard_normal((m, H, d))
+    w = rng.random((m, H))
+    qbar, wbar = -q[::G], w[::G]        # banks that prefer the keys the rows like least
+    out = ox.mtp_topk(q, w, [k], qbar, wbar, [n], m, G, P, K)
+    for j in range(m):
+        p = n - m + j
+        s = _relu_scores(q[j], w[j], k[:p + 1])
+        ref = sorted(range(p + 1), key=lambda x: (-s[x], x))[:K]
+        assert set(out[j]) == set(ref)
+    per_group, _ = ox.group_topk(q, w, k, qbar, wbar, n - m, G, P, K, "paper", fallback="group")
+    assert any(set(per_group[j]) != set(out[j]) for j in range(m))
+
+
+def test_mtp_banked_window_matches_the_equations():
+    """N > P: group g of sequence b has its anchor at seq_len[b] - m + g*G, a bank of the P
+    best keys (group query, s <= anchor) and candidates bank U {anchor+1 .. own position}."""
+    rng = np.random.default_rng(41)
+    m, G, P, K, H, Hg, d = 16, 8, 20, 6, 4, 2, 8
+    seq_len = [60, 91]
+    caches = [rng.standard_normal((n, d)) for n in seq_len]
+    q = rng.standard_normal((2 * m, H, d))
+    w = rng.random((2 * m, H))
+    qbar = rng.standard_normal((2 * m // G, Hg, d))
+    wbar = rng.random((2 * m // G, Hg))
+    out = ox.mtp_topk(q, w, caches, qbar, wbar, seq_len, m, G, P, K)
+    for b, n in enumerate(seq_len):
+        k = caches[b]
+        for g in range(m // G):
+            a = n - m + g * G
+            sb = _relu_scores(qbar[b * (m // G) + g], wbar[b * (m // G) + g], k[:a + 1])
+            bank = sorted(range(a + 1), key=lambda x: (-sb[x], x))[:P]
+            for j in range(g * G, g * G + G):
+                p = n - m + j
+                cand = sorted(set(bank) | set(range(a + 1, p + 1)))
+                s = _relu_scores(q[b * m + j], w[b * m + j], k[cand])
+                ref = [cand[i] for i in sorted(range(len(cand)), key=lambda x: (-s[x], cand[x]))[:K]]
+                assert set(out[b * m + j]) == set(ref), (b, j)
