@@ -145,6 +145,33 @@ adx_status adx_bank_refine(const adx_operands* full, int32_t G, int32_t B, int32
                            const int32_t* bank_idx, int32_t K, int32_t* topk_idx,
                            float* topk_score, void* ws, size_t ws_bytes, void* stream);
 
+/* MTP target verification (ADIndex §4.3, "Application to Prefill and MTP", and Appendix A.2,
+ * "Bank Sharing During MTP Target Verification"): each of Bs sequences verifies a window of
+ * m draft tokens in one call.
+ * full  the full indexer in an MTP layout: q [Bs*m, H, d], w [Bs*m, H] (row b*m + j = window
+ *       query j of sequence b), k [Bs, S, d] key caches (S = capacity) with k_scale [Bs, S]
+ *       for e4m3, seq_len [Bs] device: keys in sequence b's cache, the window's own included,
+ *       so query j sits at position seq_len[b] - m + j (requires m <= seq_len[b] <= S, not
+ *       checked on the host). bf16 queries with an e4m3 cache are quantised inside the call.
+ * grp   the group queries: q = q-bar [Bs*m/G, H_g, d], q_scale, w = w-bar [Bs*m/G, H_g]
+ *       (group g of sequence b is row b*m/G + g), q_dtype, H = H_g; its key fields, S, T and
+ *       seq_len are not used (the keys are full's).
+ * The window is split into m/G groups of G consecutive queries (m % G == 0, G >= 4, m <= 64);
+ * group g's anchor is its first query. When the window's first query sees more than P keys,
+ * every group builds a bank of the P best keys over the history its anchor sees (group query,
+ * Eq. (13)) and each member refines over bank U {anchor+1 .. own position} (Eq. (14));
+ * otherwise the whole window uses the plain indexer (window-level fallback).
+ * topk_idx [Bs*m, K] int32 out (ascending positions, -1 padded); topk_score [Bs*m, K] or NULL.
+ * bank_out [Bs*m/G, P+m-1] int32 out, or NULL: each group's candidate positions - a banked
+ *       window's bank (ascending, -1 padded) then its post-anchor positions, a falling-back
+ *       window's every position up to its last member's - then -1 padding.
+ * ws    workspace of ws_bytes >= adx_mtp_workspace_size(full, grp, m, G, P, K). */
+size_t adx_mtp_workspace_size(const adx_operands* full, const adx_operands* grp, int32_t m,
+                              int32_t G, int32_t P, int32_t K);
+adx_status adx_index_mtp(const adx_operands* full, const adx_operands* grp, int32_t m, int32_t G,
+                         int32_t P, int32_t K, int32_t* topk_idx, float* topk_score,
+                         int32_t* bank_out, void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, returns the device status recorded in `ws` (ADX_OK if none) and
  * clears it. */
 adx_status adx_read_device_status(void* ws, void* stream);

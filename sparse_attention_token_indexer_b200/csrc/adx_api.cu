@@ -431,6 +431,51 @@ size_t ws_refine(const adx_operands* o, int G, int B, int mode, int K) {
   return b;
 }
 
+// ---- MTP target verification ----------------------------------------------------------
+struct MtpShape {
+  int64_t Bs, ng, width, bcp;
+  int gps;
+};
+
+// Validates an MTP call and builds the group operand set over full's keys.
+adx_status mtp_check(const adx_operands* full, const adx_operands* grp, int m, int G, int P,
+                     int K, MtpShape& sh, adx_operands& gops) {
+  if (!full || !grp || !full->seq_len) return ADX_EINVAL;
+  adx_status r = check_operands(full, true);
+  if (r != ADX_OK) return r;
+  if (m <= 0 || m > 64 || G < 4 || m % G != 0 || P <= 0 || K <= 0) return ADX_EINVAL;
+  if (full->T % m != 0) return ADX_EINVAL;
+  sh.Bs = full->T / m;
+  sh.gps = m / G;
+  sh.ng = sh.Bs * sh.gps;
+  sh.width = static_cast<int64_t>(P) + m - 1;
+  sh.bcp = ld_for(sh.width);
+  if (sh.ng * sh.width > INT32_MAX || sh.Bs * full->S > INT32_MAX) return ADX_EINVAL;
+  gops = *full;
+  gops.q_dtype = grp->q_dtype;
+  gops.q = grp->q;
+  gops.q_scale = grp->q_scale;
+  gops.w = grp->w;
+  gops.H = grp->H;
+  gops.T = static_cast<int32_t>(sh.ng);
+  if (grp->d != full->d || grp->T != sh.ng) return ADX_EINVAL;
+  return check_operands(&gops, true);
+}
+
+size_t ws_mtp(const adx_operands* full, const adx_operands* gops, const MtpShape& sh, int m,
+              int P, int K) {
+  const int64_t R = sh.Bs * m;
+  size_t b = kStatusBytes;
+  b += align_up(static_cast<size_t>(R) * 4, kAlign) + align_up(static_cast<size_t>(sh.ng) * 4, kAlign);
+  b += align_up(static_cast<size_t>(sh.ng) * sh.width * 4, kAlign);  // candidate rows
+  b += ws_prepare(gops, sh.ng) +
+       align_up(static_cast<size_t>(sh.ng) * ld_for(full->S) * 4, kAlign) +  // bank scan scores
+       select_scratch_bytes(sh.ng, full->S, P);
+  b += ws_prepare(full, R) + align_up(static_cast<size_t>(R) * sh.bcp * 4, kAlign) +
+       select_scratch_bytes(R, sh.bcp, K);
+  return b;
+}
+
 }  // namespace
 }  // namespace adx
 
@@ -700,6 +745,112 @@ adx_status adx_bank_refine(const adx_operands* o, int32_t G, int32_t B, int32_t 
                     nullptr, 0, cv, st, s);
   }
   return ADX_OK;
+}
+
+size_t adx_mtp_workspace_size(const adx_operands* full, const adx_operands* grp, int32_t m,
+                              int32_t G, int32_t P, int32_t K) {
+  MtpShape sh;
+  adx_operands gops;
+  if (mtp_check(full, grp, m, G, P, K, sh, gops) != ADX_OK) return 0;
+  return ws_mtp(full, &gops, sh, m, P, K);
+}
+
+adx_status adx_index_mtp(const adx_operands* full, const adx_operands* grp, int32_t m, int32_t G,
+                         int32_t P, int32_t K, int32_t* topk_idx, float* topk_score,
+                         int32_t* bank_out, void* ws, size_t ws_bytes, void* stream) {
+  MtpShape sh;
+  adx_operands gops;
+  adx_status r = mtp_check(full, grp, m, G, P, K, sh, gops);
+  if (r != ADX_OK) return r;
+  if (!topk_idx || !ws) return ADX_EINVAL;
+  if (ws_bytes < ws_mtp(full, &gops, sh, m, P, K)) return ADX_EWORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t R = sh.Bs * m, S = full->S, ld = ld_for(S);
+  const int W = static_cast<int>(sh.width);
+  Carve cv(ws);
+  DeviceStatus* st = cv.take<DeviceStatus>(kStatusBytes);
+  int32_t* pos_q = cv.take<int32_t>(static_cast<size_t>(R) * 4);
+  int32_t* pos_g = cv.take<int32_t>(static_cast<size_t>(sh.ng) * 4);
+  int32_t* cand = cv.take<int32_t>(static_cast<size_t>(sh.ng) * W * 4);
+  if (bank_out != nullptr) cand = bank_out;
+  if (counted(launch_mtp_positions(full->seq_len, static_cast<int32_t>(sh.Bs), m, G, pos_q,
+                                   pos_g, s)) != cudaSuccess)
+    return ADX_ECUDA;
+
+  // banks: each group query scans the history its anchor sees, in its own sequence
+  {
+    Prepared pq;
+    if ((r = prepare(&gops, gops.q, gops.q_scale, gops.w, sh.ng, cv, s, pq)) != ADX_OK) return r;
+    float* scores = cv.take<float>(static_cast<size_t>(sh.ng) * ld * 4);
+    ScorePlan p = base_plan(&gops, pq, score_tokens_per_tile(gops.H));
+    p.a.scores = scores;
+    p.a.score_ld = ld;
+    p.a.R = static_cast<int32_t>(sh.ng);
+    p.a.rows_per_batch = sh.gps;
+    p.a.n_batches = static_cast<int32_t>(sh.Bs);
+    p.a.row_blocks_per_batch = (sh.gps + p.tok - 1) / p.tok;
+    p.a.row_pos = pos_g;
+    p.a.key_batch_stride = S;
+    p.a.keys_per_batch = static_cast<int32_t>(S);
+    p.a.status = st;
+    finish_plan(p, (S + kTileM - 1) / kTileM);
+    if ((r = run_score(p, pq.q, full->k, sh.Bs * S, s)) != ADX_OK) return r;
+    SelectArgs sa{};
+    sa.vals = scores;
+    sa.ld = ld;
+    sa.rows_per_batch = 1;
+    sa.len_mode = 3;
+    sa.row_pos = pos_g;
+    sa.len_off = 0;
+    sa.len_cap = static_cast<int32_t>(S);
+    sa.K = P;
+    sa.out_idx = cand;
+    sa.out_ld = W;
+    sa.rows = static_cast<int32_t>(sh.ng);
+    if ((r = run_select(sa, S, cv, st, s)) != ADX_OK) return r;
+    if (counted(launch_mtp_candidates(cand, static_cast<int32_t>(sh.ng), W, P, G, m,
+                                      full->seq_len, pos_g, s)) != cudaSuccess)
+      return ADX_ECUDA;
+  }
+
+  // refinement: every query scores its group's candidates, gathered from its sequence
+  Prepared pq;
+  if ((r = prepare(full, full->q, full->q_scale, full->w, R, cv, s, pq)) != ADX_OK) return r;
+  float* scores = cv.take<float>(static_cast<size_t>(R) * sh.bcp * 4);
+  ScorePlan p = base_plan(full, pq, score_tokens_per_tile(full->H));
+  p.a.scores = scores;
+  p.a.score_ld = sh.bcp;
+  p.a.R = static_cast<int32_t>(R);
+  p.a.rows_per_batch = G;
+  p.a.n_batches = static_cast<int32_t>(sh.ng);
+  p.a.row_blocks_per_batch = (G + p.tok - 1) / p.tok;
+  p.a.round_robin = 1;
+  p.a.row_pos = pos_q;
+  p.a.key_idx = cand;
+  p.a.key_idx_stride = W;
+  p.a.n_idx = W;
+  p.a.S_valid = static_cast<int32_t>(S);
+  p.a.key_batch_stride = S;
+  p.a.key_batch_div = sh.gps;
+  p.a.keys_per_batch = static_cast<int32_t>(sh.bcp);
+  p.a.status = st;
+  finish_plan(p, sh.bcp / kTileM);
+  if ((r = run_score(p, pq.q, full->k, sh.Bs * S, s)) != ADX_OK) return r;
+  SelectArgs sa{};
+  sa.vals = scores;
+  sa.ld = sh.bcp;
+  sa.idx_map = cand;
+  sa.map_stride = W;
+  sa.rows_per_batch = G;
+  sa.len_mode = 0;
+  sa.len_fixed = static_cast<int32_t>(sh.bcp);
+  sa.len_cap = static_cast<int32_t>(sh.bcp);
+  sa.K = K;
+  sa.out_idx = topk_idx;
+  sa.out_val = topk_score;
+  sa.out_ld = K;
+  sa.rows = static_cast<int32_t>(R);
+  return run_select(sa, sh.bcp, cv, st, s);
 }
 
 adx_status adx_read_device_status(void* ws, void* stream) {

@@ -24,8 +24,9 @@ constexpr int kTileM = 128;  // keys per MMA tile (TMEM lanes)
 //
 // Query rows r = 0..R-1 are split into batches of rows_per_batch rows; every batch owns a
 // key range of keys_per_batch rows in the key tensor map, starting at row
-// b * key_batch_stride. The position of row r is seq_len[b] - 1 when seq_len is given
-// (decode), else pos_base + r * pos_step. Key c of batch b sits at position key_pos[...]
+// (b / key_batch_div) * key_batch_stride (key_batch_div consecutive batches share one range;
+// 0 counts as 1). The position of row r is row_pos[r] when row_pos is given, seq_len[b] - 1
+// when seq_len is given (decode), else pos_base + r * pos_step. Key c of batch b sits at position key_pos[...]
 // when key_pos is given (packed candidate lists), at the position the index list gives for
 // slot c with gathered keys (key_idx), else at position c.
 struct ScoreArgs {
@@ -41,6 +42,7 @@ struct ScoreArgs {
   int32_t n_idx;
   int32_t S_valid;
   const int32_t* seq_len;  // [n_batches] or null
+  const int32_t* row_pos;  // [R] or null
   const int8_t* fold_flag; // [R]: 1 = the row's queries carry its gates already; null = none do
   float* scores;           // [R, score_ld]
   int64_t score_ld;
@@ -50,6 +52,7 @@ struct ScoreArgs {
   int32_t rows_per_batch;
   int32_t n_batches;
   int64_t key_batch_stride;
+  int32_t key_batch_div;
   int32_t keys_per_batch;
   int32_t row_blocks_per_batch;
   int32_t chunks_per_block;
@@ -73,13 +76,16 @@ struct SelectArgs {
   int64_t map_stride;
   int32_t rows_per_batch;
   // row length: len_mode 0 -> fixed len_fixed; 1 -> min(len_cap, pos_base + r*pos_step + 1);
-  //             2 -> min(len_cap, seq_len[r / rows_per_batch])
+  //             2 -> min(len_cap, seq_len[r / rows_per_batch]);
+  //             3 -> min(len_cap, row_pos[r] + 1 + len_off)
   int32_t len_mode;
   int32_t len_fixed;
   int32_t len_cap;
   int64_t pos_base;
   int32_t pos_step;
   const int32_t* seq_len;
+  const int32_t* row_pos;
+  int32_t len_off;
   int32_t K;
   int32_t n_seg;           // split each row into n_seg segments of seg_len (first stage)
   int32_t seg_len;
@@ -108,6 +114,16 @@ cudaError_t launch_pack_candidates(const void* k, const float* k_scale, int64_t 
                                    int32_t n_groups, int32_t n_cand, int32_t n_cand_pad,
                                    int32_t row_bytes, void* packed, float* packed_scale,
                                    int32_t* packed_pos, cudaStream_t s);
+// MTP windows: positions of the window queries (row_pos_q [Bs*m]) and of the group anchors
+// (row_pos_g [Bs*m/G]) from seq_len[b] = keys in sequence b's cache, the window included.
+cudaError_t launch_mtp_positions(const int32_t* seq_len, int32_t Bs, int32_t m, int32_t G,
+                                 int32_t* row_pos_q, int32_t* row_pos_g, cudaStream_t s);
+// MTP windows: completes each group's candidate row cand [n_groups, width] (columns < P hold
+// the bank): a banked window adds the post-anchor positions and pads with -1; a window whose
+// first query sees at most P keys gets every position up to its last member's instead.
+cudaError_t launch_mtp_candidates(int32_t* cand, int32_t n_groups, int32_t width, int32_t P,
+                                  int32_t G, int32_t m, const int32_t* seq_len,
+                                  const int32_t* anchor_pos, cudaStream_t s);
 cudaError_t launch_fill_post_anchor(int32_t* bank, int32_t n_groups, int32_t bank_w,
                                     int32_t first_col, int32_t count, int64_t pos_base,
                                     int32_t pos_step, const int32_t* seq_len, int32_t start_off,

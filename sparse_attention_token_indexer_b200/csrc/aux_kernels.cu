@@ -44,6 +44,41 @@ __global__ void pack_kernel(const uint8_t* __restrict__ k, const float* __restri
   }
 }
 
+// MTP window positions: query j of sequence b at seq_len[b] - m + j; group g's anchor (its
+// first query) at seq_len[b] - m + g*G.
+__global__ void mtp_positions_kernel(const int32_t* __restrict__ seq_len, int32_t Bs, int32_t m,
+                                     int32_t G, int32_t* __restrict__ row_pos_q,
+                                     int32_t* __restrict__ row_pos_g) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= static_cast<int64_t>(Bs) * m) return;
+  const int b = static_cast<int>(i / m), j = static_cast<int>(i % m);
+  const int32_t p = seq_len[b] - m + j;
+  row_pos_q[i] = p;
+  if (j % G == 0) row_pos_g[static_cast<int64_t>(b) * (m / G) + j / G] = p;
+}
+
+// One thread per (group, column) of the MTP candidate rows.
+__global__ void mtp_candidates_kernel(int32_t* __restrict__ cand, int32_t n_groups, int32_t width,
+                                      int32_t P, int32_t G, int32_t m,
+                                      const int32_t* __restrict__ seq_len,
+                                      const int32_t* __restrict__ anchor_pos) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= static_cast<int64_t>(n_groups) * width) return;
+  const int g = static_cast<int>(i / width), c = static_cast<int>(i % width);
+  const int b = g / (m / G);
+  const int32_t first_visible = seq_len[b] - m + 1;  // keys the window's first query sees
+  const int32_t a = anchor_pos[g];
+  int32_t v;
+  if (first_visible <= P) {
+    v = c < a + G ? c : -1;  // plain indexer: every position up to the last member's
+  } else if (c < P) {
+    return;  // the bank
+  } else {
+    v = c < P + G - 1 ? a + 1 + (c - P) : -1;  // post-anchor positions, then padding
+  }
+  cand[i] = v;
+}
+
 __global__ void fill_post_kernel(int32_t* bank, int32_t n_groups, int32_t bank_w, int32_t first_col,
                                  int32_t count, int64_t pos_base, int32_t pos_step,
                                  const int32_t* seq_len, int32_t start_off) {
@@ -214,6 +249,25 @@ cudaError_t launch_pack_candidates(const void* k, const float* k_scale, int64_t 
       static_cast<const uint8_t*>(k), k_scale, key_batch_stride, per_group_keys, S_valid, cand,
       n_groups, n_cand, n_cand_pad, row_bytes, static_cast<uint8_t*>(packed), packed_scale,
       packed_pos);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mtp_positions(const int32_t* seq_len, int32_t Bs, int32_t m, int32_t G,
+                                 int32_t* row_pos_q, int32_t* row_pos_g, cudaStream_t s) {
+  const int64_t total = static_cast<int64_t>(Bs) * m;
+  if (total <= 0) return cudaSuccess;
+  mtp_positions_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, s>>>(
+      seq_len, Bs, m, G, row_pos_q, row_pos_g);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mtp_candidates(int32_t* cand, int32_t n_groups, int32_t width, int32_t P,
+                                  int32_t G, int32_t m, const int32_t* seq_len,
+                                  const int32_t* anchor_pos, cudaStream_t s) {
+  const int64_t total = static_cast<int64_t>(n_groups) * width;
+  if (total <= 0) return cudaSuccess;
+  mtp_candidates_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, s>>>(
+      cand, n_groups, width, P, G, m, seq_len, anchor_pos);
   return cudaGetLastError();
 }
 

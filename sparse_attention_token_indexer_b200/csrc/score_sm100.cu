@@ -98,6 +98,7 @@ struct Block {
 };
 
 __device__ __forceinline__ int64_t row_position(const ScoreArgs& a, int r) {
+  if (a.row_pos != nullptr) return a.row_pos[r];
   if (a.seq_len != nullptr) return static_cast<int64_t>(a.seq_len[r / a.rows_per_batch]) - 1;
   return a.pos_base + static_cast<int64_t>(r) * a.pos_step;
 }
@@ -111,14 +112,15 @@ __device__ __forceinline__ void block_info(const ScoreArgs& a, int i, Block& x) 
   const int rb = rbg % a.row_blocks_per_batch;
   x.row0 = x.b * a.rows_per_batch + rb * TOK;
   x.row_end = min(min(x.row0 + TOK, (x.b + 1) * a.rows_per_batch), a.R);
-  x.key_row0 = static_cast<int64_t>(x.b) * a.key_batch_stride;
+  x.key_row0 = static_cast<int64_t>(x.b / (a.key_batch_div > 1 ? a.key_batch_div : 1)) *
+               a.key_batch_stride;
   x.nkeys = 0;
   x.ntiles = 0;
   if (x.row0 >= x.row_end) return;
   int64_t nk;
   if (a.key_pos != nullptr || a.key_idx != nullptr) {
     nk = a.keys_per_batch;
-  } else if (a.seq_len != nullptr) {
+  } else if (a.seq_len != nullptr && a.row_pos == nullptr) {
     nk = min(static_cast<int64_t>(a.seq_len[x.b]), static_cast<int64_t>(a.keys_per_batch));
   } else {
     nk = min(row_position(a, x.row_end - 1) + 1, static_cast<int64_t>(a.keys_per_batch));

@@ -70,8 +70,10 @@ __device__ __forceinline__ int64_t row_length(const SelectArgs& a, int r) {
     n = a.len_fixed;
   } else if (a.len_mode == 1) {
     n = a.pos_base + static_cast<int64_t>(r) * a.pos_step + 1;
-  } else {
+  } else if (a.len_mode == 2) {
     n = a.seq_len[r / a.rows_per_batch];
+  } else {
+    n = static_cast<int64_t>(a.row_pos[r]) + 1 + a.len_off;
   }
   if (n > a.len_cap) n = a.len_cap;
   return n < 0 ? 0 : n;

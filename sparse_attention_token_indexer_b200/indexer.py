@@ -165,6 +165,32 @@ def bank_refine(q, w, k, bank, G, B, mode, K, q_scale=None, k_scale=None, q_pos0
     return idx, sc
 
 
+def index_mtp(q, w, k, seq_len, qbar, wbar, m, G, P, K, q_scale=None, k_scale=None,
+              qbar_scale=None, with_scores=False, with_banks=False, ws=None, stream=None):
+    """MTP target verification: Bs = len(seq_len) windows of m queries (q [Bs*m, H, d]) against
+    their own caches k [Bs, S, d], with group queries qbar [Bs*m/G, H_g, d]
+    -> (topk_idx [Bs*m, K], topk_score or None, candidate rows [Bs*m/G, P+m-1] or None)."""
+    full = make_operands(q, w, k, q_scale, k_scale, 0, seq_len)
+    _dev(qbar, "qbar"), _dev(wbar, "wbar", torch.float32)
+    _dev(qbar_scale, "qbar_scale", torch.float32)
+    grp = L.Operands()
+    grp.q_dtype, grp.k_dtype = _dtype(qbar), full.k_dtype
+    grp.q, grp.q_scale, grp.w = qbar.data_ptr(), _p(qbar_scale), wbar.data_ptr()
+    grp.T, grp.H, grp.d = qbar.shape
+    idx = torch.empty(full.T, K, dtype=torch.int32, device=q.device)
+    sc = torch.empty(full.T, K, dtype=torch.float32, device=q.device) if with_scores else None
+    banks = (torch.empty(grp.T, P + m - 1, dtype=torch.int32, device=q.device)
+             if with_banks else None)
+    need = L.lib().adx_mtp_workspace_size(ctypes.byref(full), ctypes.byref(grp), m, G, P, K)
+    if need == 0:
+        raise L.AdxError("adx_mtp_workspace_size", L.ADX_EINVAL)
+    buf = _ws(ws, q.device).get(need)
+    L.check("adx_index_mtp", L.lib().adx_index_mtp(
+        ctypes.byref(full), ctypes.byref(grp), m, G, P, K, _p(idx), _p(sc), _p(banks), _p(buf),
+        buf.numel(), _stream(stream)))
+    return idx, sc, banks
+
+
 def read_device_status(ws=None, device=None, stream=None):
     """Synchronises and returns (and clears) the device status of a workspace (0 = ok)."""
     w = _ws(ws, device or torch.device("cuda"))

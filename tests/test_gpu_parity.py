@@ -335,6 +335,65 @@ def test_decode_bank_reuse():
 
 
 # ---------------------------------------------------------------------------------------
+# MTP target verification
+# ---------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("G", [4, 8, 16])
+@pytest.mark.parametrize("k_dtype", ["e4m3", "bf16"])
+def test_mtp_windows(G, k_dtype):
+    """Four windows of m = 16 queries: one falls back (its first query sees P - 5 keys), one
+    is just past the budget, one mid-size, one at the end of the cache."""
+    Bs, S0, m, P, K, Hg = 4, 4096, 16, 512, 128, 16
+    prob = inputs.decode_problem(Bs=Bs, S=S0, H=64, d=128, K=K, Hg=Hg, steps=m, seed=34,
+                                 k_dtype=k_dtype, device="cuda")
+    k, ks = prob["k"], prob["k_scale"]
+    S_cap = k.shape[1]
+    first = [P - 5, P + 3, 2000, S_cap - m + 1]          # keys the first window query sees
+    seq_len = torch.tensor([n + m - 1 for n in first], dtype=torch.int32, device="cuda")
+    q = prob["q_steps"].transpose(0, 1).reshape(Bs * m, 64, 128).contiguous()
+    w = prob["w_steps"].transpose(0, 1).reshape(Bs * m, 64).contiguous()
+    qbar, wbar = inputs.mean_pool_group_queries(q.float(), w, G, Hg)
+    qbar = qbar.to(torch.bfloat16).contiguous()
+    idx, sc, banks = indexer.index_mtp(q, w, k, seq_len, qbar, wbar, m, G, P, K, k_scale=ks,
+                                       with_scores=True, with_banks=True)
+    idx, sc, banks = idx.cpu().numpy(), sc.cpu().numpy(), banks.cpu().numpy()
+    q64, w64, qb64, wb64 = f64(q), w.double().cpu().numpy(), f64(qbar), wbar.double().cpu().numpy()
+    caches = [f64(k[b, :int(n)], None if ks is None else ks[b, :int(n)])
+              for b, n in enumerate(seq_len.tolist())]
+    ref = ox.mtp_topk(q64, w64, caches, qb64, wb64, seq_len.tolist(), m, G, P, K)
+    gps, tol = m // G, RTOL[k_dtype]
+    for b, n in enumerate(seq_len.tolist()):
+        keys = caches[b]
+        for g in range(gps):
+            a = n - m + g * G
+            row = banks[b * gps + g]
+            if first[b] <= P:       # window-level fallback: the plain indexer
+                assert row[:a + G].tolist() == list(range(a + G))
+                assert np.all(row[a + G:] == -1)
+                cands = [np.arange(n - m + j + 1) for j in range(g * G, g * G + G)]
+            else:
+                sb = ox.score_keys(qb64[b * gps + g], wb64[b * gps + g], keys[:a + 1])
+                check_topk(row[:P], np.arange(a + 1), sb,
+                           score_floor(qb64[b * gps + g], wb64[b * gps + g], keys[:a + 1]), P,
+                           tol, what=f"mtp bank {b}/{g}")
+                assert row[P:P + G - 1].tolist() == list(range(a + 1, a + G))
+                assert np.all(row[P + G - 1:] == -1)
+                bank = row[:P][row[:P] >= 0]
+                cands = [np.union1d(bank, np.arange(a + 1, n - m + j + 1))
+                         for j in range(g * G, g * G + G)]
+                exact = set(bank.tolist()) == set(np.asarray(ox.token_bank(
+                    qb64[b * gps + g], wb64[b * gps + g], keys,
+                    ox.GroupPlan("bank", (), a, scan_n=a + 1, bank_k=P))).tolist())
+            for j, cand in zip(range(g * G, g * G + G), cands):
+                r = b * m + j
+                cs = ox.score_keys(q64[r], w64[r], keys[cand])
+                check_topk(idx[r], cand, cs, score_floor(q64[r], w64[r], keys[cand]), K, tol,
+                           sc[r], f"mtp row {b}/{j}")
+                if first[b] <= P or exact:  # same candidates as the oracle's own procedure
+                    assert set(ref[r]) == set(ox.topk(cs, K, positions=cand).tolist())
+
+
+# ---------------------------------------------------------------------------------------
 # full-size workloads, sampled rows, in the configuration bench.py times
 # ---------------------------------------------------------------------------------------
 
