@@ -38,6 +38,8 @@ FLAT_SMALL = dict(T=8192, H=64, d=128, K=2048, seed=1)
 GROUP = dict(T=65536, H=64, d=128, K=2048, G=64, B=8192, Hg=16, seed=2)
 DECODE = dict(Bs=32, S=131072, H=64, d=128, K=2048, Hg=16, B=8192, G=16, seed=3)
 CHUNKED = dict(S=262144, chunk=4096, H=64, d=128, K=2048, G=64, B=8192, Hg=16, seed=4)
+# MTP target verification on the decode caches: one window of m draft tokens per sequence
+MTP = dict(m=16, G=8, P=8192)
 
 
 def flat_pairs(T, q_pos0=0):
@@ -364,6 +366,41 @@ def run_decode(args, dist, cycle=True):
                 bytes_flat=c["Bs"] * c["S"] * key_bytes, steps_per_cycle=c["G"], stages=dstages)
 
 
+def run_mtp(args, dist):
+    """One verification round: each of the 32 sequences checks m = 16 draft tokens whose
+    first one sees 131072 keys. Baseline: the plain indexer for the same 16 queries (16
+    decode steps, one query per sequence each)."""
+    from sparse_attention_token_indexer_b200 import indexer, inputs
+    c, m, G, P = DECODE, MTP["m"], MTP["G"], MTP["P"]
+    prob = inputs.decode_problem(c["Bs"], c["S"], c["H"], c["d"], c["K"], c["Hg"], steps=m,
+                                 seed=c["seed"], device="cuda")
+    ws = indexer.Workspace("cuda")
+    k, ks = prob["k"], prob["k_scale"]
+    q = prob["q_steps"].transpose(0, 1).reshape(c["Bs"] * m, c["H"], c["d"]).contiguous()
+    w = prob["w_steps"].transpose(0, 1).reshape(c["Bs"] * m, c["H"]).contiguous()
+    qbar, wbar = inputs.mean_pool_group_queries(q.float(), w, G, c["Hg"])
+    qbar = qbar.to(torch.bfloat16).contiguous()
+    seq = torch.full((c["Bs"],), c["S"] + m - 1, dtype=torch.int32, device="cuda")
+    seqs = [inputs.decode_seq_len(prob, j) for j in range(m)]
+
+    def mtp_round():
+        indexer.index_mtp(q, w, k, seq, qbar, wbar, m, G, P, c["K"], k_scale=ks, ws=ws)
+
+    def flat_round():
+        for j in range(m):
+            indexer.index_decode(prob["q_steps"][j], prob["w_steps"][j], k, seqs[j], c["K"],
+                                 k_scale=ks, ws=ws)
+
+    ms_mtp, l_mtp = timed(mtp_round, args.steps, args.warmup, dist)
+    ms_flat, l_flat = timed(flat_round, max(2, args.steps // 2), args.warmup, dist)
+    n0 = c["S"]                                   # keys the window's first query sees
+    scan = c["Bs"] * sum(n0 + g * G for g in range(m // G))
+    refine = c["Bs"] * sum(P + (j % G) for j in range(m))
+    flat = c["Bs"] * sum(n0 + j for j in range(m))
+    return dict(ms=ms_mtp, launches=l_mtp, ms_flat=ms_flat, launches_flat=l_flat, scan=scan,
+                refine=refine, flat=flat, rows=c["Bs"] * m)
+
+
 def run_chunked(args, dist):
     """256K-token prefill in query chunks of 4096 against the growing causal key cache, flat
     and in group mode (window bank, G = 64, B = 8192); one step = all 64 chunks."""
@@ -586,6 +623,15 @@ def main():
             "scores_per_s": (ck["scan"] + ck["refine"]) / (ck["ms_group"] * 1e-3),
             "topk_queries_per_s": ck["rows"] / (ck["ms_group"] * 1e-3),
             "speedup_vs_flat": ck["ms_flat"] / ck["ms_group"], "gpu_launches": ck["l_group"]}
+        mt = run_mtp(args, dist)
+        rows[f"mtp_round_Bs32_N131072_m{MTP['m']}_G{MTP['G']}_P{MTP['P']}"] = {
+            "ms_per_round": mt["ms"], "scan_pairs": mt["scan"], "refine_pairs": mt["refine"],
+            "scores_per_s": (mt["scan"] + mt["refine"]) / (mt["ms"] * 1e-3),
+            "topk_queries_per_s": mt["rows"] / (mt["ms"] * 1e-3),
+            "flat_ms_per_round": mt["ms_flat"],
+            "speedup_vs_flat": mt["ms_flat"] / mt["ms"],
+            "score_count_ratio": mt["flat"] / (mt["scan"] + mt["refine"]),
+            "gpu_launches": mt["launches"]}
         rows["decode_bank_reuse_cycle16"] = {
             "ms_per_cycle": dcd["ms_cycle"],
             "ms_per_step": dcd["ms_cycle"] / dcd["steps_per_cycle"],
