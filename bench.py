@@ -493,8 +493,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--rows", action="store_true", help="also time the other hot-path rows")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--case", default="flat", choices=["flat", "flat_small", "decode"],
-                    help="flat_small: T = 8192, for profiler captures; decode: the decode "
+    ap.add_argument("--case", default="flat", choices=["flat", "flat_small", "decode", "mtp"],
+                    help="flat_small: T = 8192, for profiler captures; decode, mtp: that "
                          "workload alone (with --quick)")
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "e4m3"])
     ap.add_argument("--quick", action="store_true",
@@ -552,6 +552,15 @@ def main():
                               "stage_ms": dcd["stages"],
                               "hbm_gbs": dcd["bytes_flat"] / (dcd["ms_flat"] * 1e-3) / 1e9,
                               "gpu_launches": dcd["launches_flat"]}), flush=True)
+        dist.close()
+        return
+    if args.case == "mtp" and args.quick:
+        mt = run_mtp(args, dist)
+        if dist.rank == 0:
+            print(json.dumps({"case": "mtp", "ms_per_round": mt["ms"],
+                              "flat_ms_per_round": mt["ms_flat"],
+                              "speedup_vs_flat": mt["ms_flat"] / mt["ms"],
+                              "gpu_launches": mt["launches"]}), flush=True)
         dist.close()
         return
     flat = run_flat(args, dist, args.dtype, clocks)

@@ -473,6 +473,8 @@ size_t ws_mtp(const adx_operands* full, const adx_operands* gops, const MtpShape
        select_scratch_bytes(sh.ng, full->S, P);
   b += ws_prepare(full, R) + align_up(static_cast<size_t>(R) * sh.bcp * 4, kAlign) +
        select_scratch_bytes(R, sh.bcp, K);
+  b += align_up(static_cast<size_t>(sh.ng) * sh.bcp * row_bytes(full), kAlign) +  // packed keys
+       align_up(static_cast<size_t>(sh.ng) * sh.bcp * 4, kAlign) * 2;            // scales, positions
   return b;
 }
 
@@ -689,7 +691,7 @@ adx_status adx_bank_refine(const adx_operands* o, int32_t G, int32_t B, int32_t 
       uint8_t* packed = cv.take<uint8_t>(static_cast<size_t>(ng) * bcp * rb);
       float* pscale = cv.take<float>(static_cast<size_t>(ng) * bcp * 4);
       int32_t* ppos = cv.take<int32_t>(static_cast<size_t>(ng) * bcp * 4);
-      if (counted(launch_pack_candidates(o->k, o->k_scale, o->S, 0, o->S, bank_idx,
+      if (counted(launch_pack_candidates(o->k, o->k_scale, o->S, 0, 1, o->S, bank_idx,
                                          static_cast<int32_t>(ng), bs.width,
                                          static_cast<int32_t>(bcp), rb, packed,
                                          fp8_keys(o) ? pscale : nullptr, ppos, s)) != cudaSuccess)
@@ -782,7 +784,11 @@ adx_status adx_index_mtp(const adx_operands* full, const adx_operands* grp, int3
     Prepared pq;
     if ((r = prepare(&gops, gops.q, gops.q_scale, gops.w, sh.ng, cv, s, pq)) != ADX_OK) return r;
     float* scores = cv.take<float>(static_cast<size_t>(sh.ng) * ld * 4);
-    ScorePlan p = base_plan(&gops, pq, score_tokens_per_tile(gops.H));
+    // one row block per sequence holds its m/G groups: with 16 heads, tiles of 2 or 4
+    // tokens keep the epilogue from reducing empty token slots
+    const int tok = gops.H == 16 && sh.gps <= 4 ? (sh.gps <= 2 ? 2 : 4)
+                                                : score_tokens_per_tile(gops.H);
+    ScorePlan p = base_plan(&gops, pq, tok);
     p.a.scores = scores;
     p.a.score_ld = ld;
     p.a.R = static_cast<int32_t>(sh.ng);
@@ -813,7 +819,18 @@ adx_status adx_index_mtp(const adx_operands* full, const adx_operands* grp, int3
       return ADX_ECUDA;
   }
 
-  // refinement: every query scores its group's candidates, gathered from its sequence
+  // refinement: every query scores its group's candidates, packed once per group from its
+  // sequence into contiguous rows (a group's G queries share them)
+  const int rb = row_bytes(full);
+  uint8_t* packed = cv.take<uint8_t>(static_cast<size_t>(sh.ng) * sh.bcp * rb);
+  float* pscale = cv.take<float>(static_cast<size_t>(sh.ng) * sh.bcp * 4);
+  int32_t* ppos = cv.take<int32_t>(static_cast<size_t>(sh.ng) * sh.bcp * 4);
+  if (counted(launch_pack_candidates(full->k, full->k_scale, S, 1, sh.gps,
+                                     static_cast<int32_t>(S), cand,
+                                     static_cast<int32_t>(sh.ng), W,
+                                     static_cast<int32_t>(sh.bcp), rb, packed,
+                                     fp8_keys(full) ? pscale : nullptr, ppos, s)) != cudaSuccess)
+    return ADX_ECUDA;
   Prepared pq;
   if ((r = prepare(full, full->q, full->q_scale, full->w, R, cv, s, pq)) != ADX_OK) return r;
   float* scores = cv.take<float>(static_cast<size_t>(R) * sh.bcp * 4);
@@ -824,23 +841,19 @@ adx_status adx_index_mtp(const adx_operands* full, const adx_operands* grp, int3
   p.a.rows_per_batch = G;
   p.a.n_batches = static_cast<int32_t>(sh.ng);
   p.a.row_blocks_per_batch = (G + p.tok - 1) / p.tok;
-  p.a.round_robin = 1;
   p.a.row_pos = pos_q;
-  p.a.key_idx = cand;
-  p.a.key_idx_stride = W;
-  p.a.n_idx = W;
-  p.a.S_valid = static_cast<int32_t>(S);
-  p.a.key_batch_stride = S;
-  p.a.key_batch_div = sh.gps;
+  p.a.k_scale = fp8_keys(full) ? pscale : nullptr;
+  p.a.key_pos = ppos;
+  p.a.key_batch_stride = sh.bcp;
   p.a.keys_per_batch = static_cast<int32_t>(sh.bcp);
   p.a.status = st;
   finish_plan(p, sh.bcp / kTileM);
-  if ((r = run_score(p, pq.q, full->k, sh.Bs * S, s)) != ADX_OK) return r;
+  if ((r = run_score(p, pq.q, packed, sh.ng * sh.bcp, s)) != ADX_OK) return r;
   SelectArgs sa{};
   sa.vals = scores;
   sa.ld = sh.bcp;
-  sa.idx_map = cand;
-  sa.map_stride = W;
+  sa.idx_map = ppos;
+  sa.map_stride = sh.bcp;
   sa.rows_per_batch = G;
   sa.len_mode = 0;
   sa.len_fixed = static_cast<int32_t>(sh.bcp);

@@ -109,8 +109,11 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launched);
 int select_cluster_ctas(int64_t rows, int64_t n_max, int K, int sms);
 // One launch of the cluster select with `ctas` CTAs per row (a.n_seg must be 1).
 cudaError_t launch_select_cluster(const SelectArgs& a, int ctas, cudaStream_t s, int* launched);
+// Packs candidate key rows: slot c of group g is key cand[g * n_cand + c] of key range
+// g / group_div (per_group_keys; else of the one shared range).
 cudaError_t launch_pack_candidates(const void* k, const float* k_scale, int64_t key_batch_stride,
-                                   int32_t per_group_keys, int32_t S_valid, const int32_t* cand,
+                                   int32_t per_group_keys, int32_t group_div, int32_t S_valid,
+                                   const int32_t* cand,
                                    int32_t n_groups, int32_t n_cand, int32_t n_cand_pad,
                                    int32_t row_bytes, void* packed, float* packed_scale,
                                    int32_t* packed_pos, cudaStream_t s);

@@ -20,7 +20,8 @@ namespace {
 
 // One thread per 16-byte piece of a packed candidate row.
 __global__ void pack_kernel(const uint8_t* __restrict__ k, const float* __restrict__ k_scale,
-                            int64_t key_batch_stride, int32_t per_group_keys, int32_t S_valid,
+                            int64_t key_batch_stride, int32_t per_group_keys, int32_t group_div,
+                            int32_t S_valid,
                             const int32_t* __restrict__ cand, int32_t n_groups, int32_t n_cand,
                             int32_t n_cand_pad, int32_t row_bytes, uint8_t* __restrict__ packed,
                             float* __restrict__ packed_scale, int32_t* __restrict__ packed_pos) {
@@ -34,7 +35,8 @@ __global__ void pack_kernel(const uint8_t* __restrict__ k, const float* __restri
   const int c = static_cast<int>(slot % n_cand_pad);
   const int32_t p = c < n_cand ? cand[static_cast<int64_t>(g) * n_cand + c] : -1;
   const bool valid = p >= 0 && p < S_valid;
-  const int64_t krow = (per_group_keys ? static_cast<int64_t>(g) * key_batch_stride : 0) + p;
+  const int64_t krow =
+      (per_group_keys ? static_cast<int64_t>(g / group_div) * key_batch_stride : 0) + p;
   uint4 v = make_uint4(0u, 0u, 0u, 0u);
   if (valid) v = reinterpret_cast<const uint4*>(k + krow * row_bytes)[piece];
   reinterpret_cast<uint4*>(packed + slot * row_bytes)[piece] = v;
@@ -238,7 +240,8 @@ cudaError_t launch_prepare_q(const void* q, const float* q_scale, bool in_e4m3, 
 }
 
 cudaError_t launch_pack_candidates(const void* k, const float* k_scale, int64_t key_batch_stride,
-                                   int32_t per_group_keys, int32_t S_valid, const int32_t* cand,
+                                   int32_t per_group_keys, int32_t group_div, int32_t S_valid,
+                                   const int32_t* cand,
                                    int32_t n_groups, int32_t n_cand, int32_t n_cand_pad,
                                    int32_t row_bytes, void* packed, float* packed_scale,
                                    int32_t* packed_pos, cudaStream_t s) {
@@ -246,7 +249,8 @@ cudaError_t launch_pack_candidates(const void* k, const float* k_scale, int64_t 
   if (total <= 0) return cudaSuccess;
   const int threads = 256;
   pack_kernel<<<static_cast<unsigned>((total + threads - 1) / threads), threads, 0, s>>>(
-      static_cast<const uint8_t*>(k), k_scale, key_batch_stride, per_group_keys, S_valid, cand,
+      static_cast<const uint8_t*>(k), k_scale, key_batch_stride, per_group_keys,
+      group_div > 1 ? group_div : 1, S_valid, cand,
       n_groups, n_cand, n_cand_pad, row_bytes, static_cast<uint8_t*>(packed), packed_scale,
       packed_pos);
   return cudaGetLastError();

@@ -714,10 +714,12 @@ bool score_config_supported(bool fp8, int H, int d) {
   X(false, 16, 16, 64)                                                                 \
   /* one query per key batch (decode and its bank refresh): N = H */                  \
   X(false, 64, 1, 128) X(true, 64, 1, 128) X(false, 16, 1, 128) X(true, 16, 1, 128)   \
-  X(false, 32, 1, 128) X(true, 32, 1, 128)
+  X(false, 32, 1, 128) X(true, 32, 1, 128)                                             \
+  /* a few group queries per key batch (MTP windows): N = 2 or 4 tokens x 16 heads */  \
+  X(false, 16, 2, 128) X(true, 16, 2, 128) X(false, 16, 4, 128) X(true, 16, 4, 128)
 
-// tok: tokens per N tile; either score_tokens_per_tile(H) (prefill) or 1 (one query per
-// key batch: decode and its bank refresh).
+// tok: tokens per N tile; score_tokens_per_tile(H) (prefill), 1 (one query per key batch:
+// decode and its bank refresh), or 2 / 4 with 16 heads (the group queries of an MTP window).
 cudaError_t launch_score(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const ScoreArgs& a,
                          bool fp8, int H, int d, int tok, int grid, cudaStream_t s) {
   const bool gather = a.key_idx != nullptr;
