@@ -232,3 +232,15 @@ def mtp_topk(q, w, caches, qbar, wbar, seq_len, m, G, P, K):
         for j, v in res.items():
             out[b * m + j] = v
     return out
+
+
+# ---------------------------------------------------------------------------------------
+# Layer-wise reuse calibration (ADIndex §4.1)
+# ---------------------------------------------------------------------------------------
+
+def group_union_sizes(topk_rows, G):
+    """ADIndex §4.1, Eq. (4): for every group of G consecutive query rows (rows g*G ..
+    g*G+G-1, complete groups only), the size of the union of their Top-K index sets; -1
+    padding is not an index. U^max of the page is the maximum of these sizes."""
+    rows = [set(int(x) for x in np.asarray(r).ravel() if int(x) >= 0) for r in topk_rows]
+    return [len(set().union(*rows[g0:g0 + G])) for g0 in range(0, len(rows) - G + 1, G)]

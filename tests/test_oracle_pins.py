@@ -343,3 +343,32 @@ def test_mtp_banked_window_matches_the_equations():
                 s = _relu_scores(q[b * m + j], w[b * m + j], k[cand])
                 ref = [cand[i] for i in sorted(range(len(cand)), key=lambda x: (-s[x], cand[x]))[:K]]
                 assert set(out[b * m + j]) == set(ref), (b, j)
+
+
+# ---------------------------------------------------------------------------------------
+# Calibration statistic (ADIndex §4.1, Eq. (4))
+# ---------------------------------------------------------------------------------------
+
+def test_union_sizes_hand_cases():
+    same = [[5, 3, 1]] * 4
+    disjoint = [[4 * i, 4 * i + 1, 4 * i + 2] for i in range(4)]
+    padded = [[7, -1, -1], [7, 8, -1], [9, 8, 7], [-1, -1, -1]]
+    assert ox.group_union_sizes(same, 4) == [3]
+    assert ox.group_union_sizes(disjoint, 4) == [12]
+    assert ox.group_union_sizes(disjoint, 2) == [6, 6]
+    assert ox.group_union_sizes(padded, 2) == [2, 3]
+    assert ox.group_union_sizes(padded + [[1, 2, 3]], 2) == [2, 3]   # incomplete group dropped
+
+
+def test_union_sizes_bounds_and_monotonicity():
+    rng = np.random.default_rng(42)
+    K, T = 6, 32
+    rows = [rng.choice(40, size=K, replace=False) for _ in range(T)]
+    for G in (2, 4, 8):
+        u = ox.group_union_sizes(rows, G)
+        assert len(u) == T // G
+        assert all(K <= x <= min(G * K, 40) for x in u)
+    # a group of 2G contains two groups of G: its union is at least either of theirs
+    u4, u8 = ox.group_union_sizes(rows, 4), ox.group_union_sizes(rows, 8)
+    for g, x in enumerate(u8):
+        assert x >= max(u4[2 * g], u4[2 * g + 1])
