@@ -401,6 +401,23 @@ def run_mtp(args, dist):
                 refine=refine, flat=flat, rows=c["Bs"] * m)
 
 
+def run_calibration(args, dist):
+    """Union sizes (Eq. (4)) of one layer's calibration Top-K rows for G = 4, 8 and 16: the
+    flat prefill's own output at T = 16384, K = 2048."""
+    from sparse_attention_token_indexer_b200 import calibration, indexer, inputs
+    c = FLAT
+    p = inputs.anchor_prefill(c["T"], c["H"], c["d"], c["K"], seed=c["seed"], device="cuda")
+    idx, _, _ = indexer.index_prefill(p["q"], p["w"], p["k"], c["K"])
+    del p
+
+    def step():
+        for G in calibration.GROUP_SIZES:
+            calibration.union_sizes(idx, G, c["T"])
+
+    ms, launches = timed(step, args.steps, args.warmup, dist)
+    return dict(ms=ms, launches=launches, bytes=3 * idx.numel() * 4)
+
+
 def run_chunked(args, dist):
     """256K-token prefill in query chunks of 4096 against the growing causal key cache, flat
     and in group mode (window bank, G = 64, B = 8192); one step = all 64 chunks."""
@@ -641,6 +658,12 @@ def main():
             "speedup_vs_flat": mt["ms_flat"] / mt["ms"],
             "score_count_ratio": mt["flat"] / (mt["scan"] + mt["refine"]),
             "gpu_launches": mt["launches"]}
+        cb = run_calibration(args, dist)
+        rows["calibration_union_sizes_T16384_K2048"] = {
+            "ms_per_layer": cb["ms"], "group_sizes": [4, 8, 16],
+            "gbs_read": cb["bytes"] / (cb["ms"] * 1e-3) / 1e9,
+            "hbm_frac": cb["bytes"] / (cb["ms"] * 1e-3) / 1e9 / pk["hbm"],
+            "gpu_launches": cb["launches"]}
         rows["decode_bank_reuse_cycle16"] = {
             "ms_per_cycle": dcd["ms_cycle"],
             "ms_per_step": dcd["ms_cycle"] / dcd["steps_per_cycle"],

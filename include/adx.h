@@ -172,6 +172,16 @@ adx_status adx_index_mtp(const adx_operands* full, const adx_operands* grp, int3
                          int32_t P, int32_t K, int32_t* topk_idx, float* topk_score,
                          int32_t* bank_out, void* ws, size_t ws_bytes, void* stream);
 
+/* Calibration statistic of layer-wise reuse (ADIndex §4.1, Eq. (4)): for every complete group
+ * of G consecutive rows of topk_idx [T, K] (rows g*G .. g*G+G-1, g < T/G), the number of
+ * distinct positions in [0, S) among the group's Top-K sets (-1 padding and other values
+ * outside [0, S) are not positions). U^max of the page is the maximum over groups.
+ * topk_idx  device, as written by the flat indexer (adx_index_prefill)
+ * union_out [T/G] int32 device out
+ * Needs no workspace; S up to 200 KiB of bitmap (6.5M positions), else ADX_EUNSUPPORTED. */
+adx_status adx_group_union_sizes(const int32_t* topk_idx, int32_t T, int32_t K, int32_t G,
+                                 int32_t S, int32_t* union_out, void* stream);
+
 /* Synchronises `stream`, returns the device status recorded in `ws` (ADX_OK if none) and
  * clears it. */
 adx_status adx_read_device_status(void* ws, void* stream);

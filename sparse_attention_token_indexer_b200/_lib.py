@@ -18,7 +18,8 @@ ADX_STATUS_BYTES = 256
 EXPORTS = ("adx_abi_version", "adx_bank_width", "adx_status_string", "adx_workspace_size",
            "adx_index_prefill", "adx_index_decode", "adx_group_bank", "adx_bank_refine",
            "adx_read_device_status", "adx_set_timing_events", "adx_launch_count",
-           "adx_index_prefill_noalloc", "adx_mtp_workspace_size", "adx_index_mtp")
+           "adx_index_prefill_noalloc", "adx_mtp_workspace_size", "adx_index_mtp",
+           "adx_group_union_sizes")
 
 
 class Operands(ctypes.Structure):
@@ -66,6 +67,7 @@ def _declare(lib):
         "adx_index_prefill_noalloc": (ctypes.c_int, [P, I32, VP, VP, VP, VP]),
         "adx_mtp_workspace_size": (SZ, [P, P, I32, I32, I32, I32]),
         "adx_index_mtp": (ctypes.c_int, [P, P, I32, I32, I32, I32, VP, VP, VP, VP, SZ, VP]),
+        "adx_group_union_sizes": (ctypes.c_int, [VP, I32, I32, I32, I32, VP, VP]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

@@ -866,6 +866,16 @@ adx_status adx_index_mtp(const adx_operands* full, const adx_operands* grp, int3
   return run_select(sa, sh.bcp, cv, st, s);
 }
 
+adx_status adx_group_union_sizes(const int32_t* topk_idx, int32_t T, int32_t K, int32_t G,
+                                 int32_t S, int32_t* union_out, void* stream) {
+  if (!topk_idx || !union_out || T <= 0 || K <= 0 || G <= 0 || S <= 0) return ADX_EINVAL;
+  if (static_cast<int64_t>(G) * K > INT32_MAX) return ADX_EINVAL;
+  if (static_cast<size_t>((S + 31) / 32) * 4 > kUnionMaxBitmapBytes) return ADX_EUNSUPPORTED;
+  const cudaError_t e = counted(launch_union_sizes(topk_idx, K, G, S, T / G, union_out,
+                                                   static_cast<cudaStream_t>(stream)));
+  return e == cudaSuccess ? ADX_OK : ADX_ECUDA;
+}
+
 adx_status adx_read_device_status(void* ws, void* stream) {
   if (!ws) return ADX_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -127,6 +127,11 @@ cudaError_t launch_mtp_positions(const int32_t* seq_len, int32_t Bs, int32_t m, 
 cudaError_t launch_mtp_candidates(int32_t* cand, int32_t n_groups, int32_t width, int32_t P,
                                   int32_t G, int32_t m, const int32_t* seq_len,
                                   const int32_t* anchor_pos, cudaStream_t s);
+// Union sizes of the Top-K sets of n_groups groups of G consecutive rows of topk [*, K]
+// (positions outside [0, S) are not indices). S is limited by the shared-memory bitmap.
+constexpr size_t kUnionMaxBitmapBytes = 200 * 1024;
+cudaError_t launch_union_sizes(const int32_t* topk, int32_t K, int32_t G, int32_t S,
+                               int32_t n_groups, int32_t* out, cudaStream_t s);
 cudaError_t launch_fill_post_anchor(int32_t* bank, int32_t n_groups, int32_t bank_w,
                                     int32_t first_col, int32_t count, int64_t pos_base,
                                     int32_t pos_step, const int32_t* seq_len, int32_t start_off,

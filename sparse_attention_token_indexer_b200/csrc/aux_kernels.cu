@@ -81,6 +81,34 @@ __global__ void mtp_candidates_kernel(int32_t* __restrict__ cand, int32_t n_grou
   cand[i] = v;
 }
 
+// Union size of the Top-K sets of one group of G consecutive rows: a bitmap of the S
+// positions in shared memory, one bit set per index, then a population count.
+__global__ void __launch_bounds__(256)
+union_sizes_kernel(const int32_t* __restrict__ topk, int32_t K, int32_t G, int32_t S,
+                   int32_t* __restrict__ out) {
+  extern __shared__ uint32_t bits[];
+  __shared__ uint32_t red[8];
+  const int nw = (S + 31) / 32;
+  for (int i = threadIdx.x; i < nw; i += blockDim.x) bits[i] = 0u;
+  __syncthreads();
+  const int32_t* rows = topk + static_cast<int64_t>(blockIdx.x) * G * K;
+  for (int i = threadIdx.x; i < G * K; i += blockDim.x) {
+    const int32_t v = rows[i];
+    if (v >= 0 && v < S) atomicOr(&bits[v >> 5], 1u << (v & 31));
+  }
+  __syncthreads();
+  uint32_t c = 0;
+  for (int i = threadIdx.x; i < nw; i += blockDim.x) c += __popc(bits[i]);
+  c = __reduce_add_sync(0xffffffffu, c);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t t = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x / 32); ++w) t += red[w];
+    out[blockIdx.x] = static_cast<int32_t>(t);
+  }
+}
+
 __global__ void fill_post_kernel(int32_t* bank, int32_t n_groups, int32_t bank_w, int32_t first_col,
                                  int32_t count, int64_t pos_base, int32_t pos_step,
                                  const int32_t* seq_len, int32_t start_off) {
@@ -272,6 +300,20 @@ cudaError_t launch_mtp_candidates(int32_t* cand, int32_t n_groups, int32_t width
   if (total <= 0) return cudaSuccess;
   mtp_candidates_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, s>>>(
       cand, n_groups, width, P, G, m, seq_len, anchor_pos);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_union_sizes(const int32_t* topk, int32_t K, int32_t G, int32_t S,
+                               int32_t n_groups, int32_t* out, cudaStream_t s) {
+  if (n_groups <= 0) return cudaSuccess;
+  const size_t smem = static_cast<size_t>((S + 31) / 32) * 4;
+  if (smem > kUnionMaxBitmapBytes) return cudaErrorInvalidValue;
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(
+        union_sizes_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  union_sizes_kernel<<<static_cast<unsigned>(n_groups), 256, smem, s>>>(topk, K, G, S, out);
   return cudaGetLastError();
 }
 
