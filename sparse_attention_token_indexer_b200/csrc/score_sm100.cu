@@ -49,13 +49,12 @@ struct Cfg {
   static constexpr int KC = DB / 128;        // 128-byte K chunks
   static constexpr int ELEMS_PER_CHUNK = FP8 ? 128 : 64;
   static constexpr int KSTEPS = DB / 32;     // 32 bytes of K per MMA instruction
-  // Epilogue warpgroups. With one query token per tile (BUF_SPLIT), the tiles go round the
-  // warpgroups: warpgroup g reduces the tiles whose accumulator buffer index is g modulo EG,
-  // all heads of the one token, so each warp has EG MMA periods per tile (a single warpgroup
-  // cannot keep up with the key stream there). With several tokens per tile the two
-  // warpgroups split the tokens of every tile instead (keeps the per-thread partial sums in
-  // registers).
-  static constexpr bool BUF_SPLIT = TOK == 1;
+  // Epilogue warpgroups. With narrow tiles (one token, or N <= 64: BUF_SPLIT), the tiles go
+  // round the warpgroups: warpgroup g reduces the tiles whose accumulator buffer index is g
+  // modulo EG, all their tokens, so each warp has EG MMA periods per tile (one warpgroup per
+  // tile cannot keep up with the key stream there). With wide tiles the two warpgroups split
+  // the tokens of every tile instead (keeps the per-thread partial sums in registers).
+  static constexpr bool BUF_SPLIT = TOK == 1 || TOK * H <= 64;
   static constexpr int EG = 2;
   static constexpr int EPI_WARPS = 4 * EG;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
