@@ -244,3 +244,26 @@ def group_union_sizes(topk_rows, G):
     padding is not an index. U^max of the page is the maximum of these sizes."""
     rows = [set(int(x) for x in np.asarray(r).ravel() if int(x) >= 0) for r in topk_rows]
     return [len(set().union(*rows[g0:g0 + G])) for g0 in range(0, len(rows) - G + 1, G)]
+
+
+# ---------------------------------------------------------------------------------------
+# Training-free group queries
+# ---------------------------------------------------------------------------------------
+
+def mean_pool_group(q, w, G, Hg):
+    """The proxy group query of the PIVOT baseline the pages compare with (ADIndex,
+    Appendix B, "PIVOT"): per group of G consecutive rows, the member mean of each indexing
+    head and of its gate, for the first Hg heads. q [T, H, d], w [T, H] (float64) ->
+    qbar [T // G, Hg, d], wbar [T // G, Hg]; an incomplete trailing group gets none."""
+    q = np.asarray(q, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    ng = q.shape[0] // G
+    qbar = np.zeros((ng, Hg, q.shape[2]))
+    wbar = np.zeros((ng, Hg))
+    for g in range(ng):
+        for i in range(g * G, g * G + G):
+            qbar[g] += q[i, :Hg]
+            wbar[g] += w[i, :Hg]
+        qbar[g] /= G
+        wbar[g] /= G
+    return qbar, wbar

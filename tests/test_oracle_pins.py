@@ -372,3 +372,20 @@ def test_union_sizes_bounds_and_monotonicity():
     u4, u8 = ox.group_union_sizes(rows, 4), ox.group_union_sizes(rows, 8)
     for g, x in enumerate(u8):
         assert x >= max(u4[2 * g], u4[2 * g + 1])
+
+
+def test_mean_pool_group_hand_values():
+    q = np.zeros((5, 3, 2))
+    w = np.zeros((5, 3))
+    for i in range(5):
+        q[i, :, 0] = i          # head-independent ramp
+        q[i, 1, 1] = 10 * i
+        w[i] = [1, 2, 3 + i]
+    qbar, wbar = ox.mean_pool_group(q, w, 2, 2)
+    assert qbar.shape == (2, 2, 2) and wbar.shape == (2, 2)   # trailing row 4 dropped
+    assert qbar[:, 0, 0].tolist() == [0.5, 2.5]
+    assert qbar[:, 1, 1].tolist() == [5.0, 25.0]
+    assert wbar.tolist() == [[1, 2], [1, 2]]
+    # G = 1 is the identity on the kept heads
+    qb1, wb1 = ox.mean_pool_group(q, w, 1, 3)
+    assert np.array_equal(qb1, q) and np.array_equal(wb1, w)
