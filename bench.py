@@ -296,26 +296,24 @@ def run_group(args, dist):
     steps = max(2, args.steps // 2)
     from sparse_attention_token_indexer_b200 import _lib
     tb, tr = StageTimer(_lib.lib(), steps), StageTimer(_lib.lib(), steps)
-    it = [0]
 
-    def step():
-        i = it[0]
-        if 0 <= i < steps:
-            tb.arm(i)
-        bank = indexer.group_bank(p["qbar"], p["wbar"], p["k"], c["G"], c["B"], "window",
-                                  ws=ws)
-        if 0 <= i < steps:
-            tr.arm(i)
+    def step(stage=None):
+        # the group queries (mean-pooled by the library), the banks, the refinement
+        qbar, wbar = indexer.group_query_mean(p["q"], p["w"], c["G"], c["Hg"])
+        if stage is not None:
+            tb.arm(stage)
+        bank = indexer.group_bank(qbar, wbar, p["k"], c["G"], c["B"], "window", ws=ws)
+        if stage is not None:
+            tr.arm(stage)
         indexer.bank_refine(p["q"], p["w"], p["k"], bank, c["G"], c["B"], "window", c["K"],
                             ws=ws)
-        tr.disarm()
-        it[0] += 1
+        if stage is not None:
+            tr.disarm()
 
-    for _ in range(args.warmup):
-        it[0] = -1
-        step()
-    it[0] = 0
-    ms, launches = timed(step, steps, 0, dist)
+    ms, launches = timed(step, steps, args.warmup, dist)
+    for i in range(steps):         # stage breakdown: a second pass with the events armed
+        step(i)
+    torch.cuda.synchronize()
     stages = {"bank_score_ms": statistics.mean(tb.ms(0, 1)),
               "bank_select_ms": statistics.mean(tb.ms(2, 3)),
               "refine_score_ms": statistics.mean(tr.ms(0, 1)),

@@ -172,6 +172,18 @@ adx_status adx_index_mtp(const adx_operands* full, const adx_operands* grp, int3
                          int32_t P, int32_t K, int32_t* topk_idx, float* topk_score,
                          int32_t* bank_out, void* ws, size_t ws_bytes, void* stream);
 
+/* Training-free group queries: the proxy of the PIVOT baseline the pages compare with
+ * (ADIndex, Appendix B, "PIVOT": the group's indexing queries and gates, mean-pooled). For
+ * every complete group of G consecutive rows (g < T/G) of q [T, H, d] (bf16, or e4m3 codes
+ * with q_scale [T]) and w [T, H]:
+ *   qbar_out [T/G, Hg, d] bf16 out: the member mean of each of the first Hg heads (summed in
+ *            fp32, rounded to nearest even)
+ *   wbar_out [T/G, Hg] fp32 out: the member mean of those heads' gates.
+ * Device pointers; q and qbar_out 16-byte aligned; d a multiple of 8; no workspace. */
+adx_status adx_group_query_mean(int32_t q_dtype, const void* q, const float* q_scale,
+                                const float* w, int32_t T, int32_t H, int32_t d, int32_t G,
+                                int32_t Hg, void* qbar_out, float* wbar_out, void* stream);
+
 /* Calibration statistic of layer-wise reuse (ADIndex §4.1, Eq. (4)): for every complete group
  * of G consecutive rows of topk_idx [T, K] (rows g*G .. g*G+G-1, g < T/G), the number of
  * distinct positions in [0, S) among the group's Top-K sets (-1 padding and other values

@@ -19,7 +19,7 @@ EXPORTS = ("adx_abi_version", "adx_bank_width", "adx_status_string", "adx_worksp
            "adx_index_prefill", "adx_index_decode", "adx_group_bank", "adx_bank_refine",
            "adx_read_device_status", "adx_set_timing_events", "adx_launch_count",
            "adx_index_prefill_noalloc", "adx_mtp_workspace_size", "adx_index_mtp",
-           "adx_group_union_sizes")
+           "adx_group_union_sizes", "adx_group_query_mean")
 
 
 class Operands(ctypes.Structure):
@@ -68,6 +68,8 @@ def _declare(lib):
         "adx_mtp_workspace_size": (SZ, [P, P, I32, I32, I32, I32]),
         "adx_index_mtp": (ctypes.c_int, [P, P, I32, I32, I32, I32, VP, VP, VP, VP, SZ, VP]),
         "adx_group_union_sizes": (ctypes.c_int, [VP, I32, I32, I32, I32, VP, VP]),
+        "adx_group_query_mean": (ctypes.c_int, [I32, VP, VP, VP, I32, I32, I32, I32, I32, VP,
+                                                VP, VP]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

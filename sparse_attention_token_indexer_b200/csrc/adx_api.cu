@@ -866,6 +866,21 @@ adx_status adx_index_mtp(const adx_operands* full, const adx_operands* grp, int3
   return run_select(sa, sh.bcp, cv, st, s);
 }
 
+adx_status adx_group_query_mean(int32_t q_dtype, const void* q, const float* q_scale,
+                                const float* w, int32_t T, int32_t H, int32_t d, int32_t G,
+                                int32_t Hg, void* qbar_out, float* wbar_out, void* stream) {
+  if (!q || !w || !qbar_out || !wbar_out || T <= 0 || H <= 0 || d <= 0 || G <= 0) return ADX_EINVAL;
+  if (Hg <= 0 || Hg > H || d % 8 != 0) return ADX_EINVAL;
+  if (q_dtype != ADX_BF16 && q_dtype != ADX_E4M3) return ADX_EINVAL;
+  if ((q_dtype == ADX_E4M3) != (q_scale != nullptr)) return ADX_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(qbar_out)) % 16 != 0)
+    return ADX_EINVAL;
+  const cudaError_t e = counted(launch_group_mean(q, q_scale, q_dtype == ADX_E4M3, w, T / G, H,
+                                                  d, G, Hg, qbar_out, wbar_out,
+                                                  static_cast<cudaStream_t>(stream)));
+  return e == cudaSuccess ? ADX_OK : ADX_ECUDA;
+}
+
 adx_status adx_group_union_sizes(const int32_t* topk_idx, int32_t T, int32_t K, int32_t G,
                                  int32_t S, int32_t* union_out, void* stream) {
   if (!topk_idx || !union_out || T <= 0 || K <= 0 || G <= 0 || S <= 0) return ADX_EINVAL;

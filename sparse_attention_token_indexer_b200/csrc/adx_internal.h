@@ -127,6 +127,10 @@ cudaError_t launch_mtp_positions(const int32_t* seq_len, int32_t Bs, int32_t m, 
 cudaError_t launch_mtp_candidates(int32_t* cand, int32_t n_groups, int32_t width, int32_t P,
                                   int32_t G, int32_t m, const int32_t* seq_len,
                                   const int32_t* anchor_pos, cudaStream_t s);
+// Mean-pooled group queries qbar [n_groups, Hg, d] bf16 and gates wbar [n_groups, Hg].
+cudaError_t launch_group_mean(const void* q, const float* q_scale, bool in_e4m3, const float* w,
+                              int64_t n_groups, int H, int d, int G, int Hg, void* qbar,
+                              float* wbar, cudaStream_t s);
 // Union sizes of the Top-K sets of n_groups groups of G consecutive rows of topk [*, K]
 // (positions outside [0, S) are not indices). S is limited by the shared-memory bitmap.
 constexpr size_t kUnionMaxBitmapBytes = 200 * 1024;

@@ -229,6 +229,39 @@ prepare_q_kernel(const void* __restrict__ q_in, const float* __restrict__ q_scal
   }
 }
 
+// Mean-pooled group query, one CTA per group of G consecutive rows: each thread owns 8
+// consecutive elements of the first Hg heads and sums them over the members in fp32.
+template <bool IN_E4M3>
+__global__ void __launch_bounds__(256)
+group_mean_kernel(const void* __restrict__ q, const float* __restrict__ q_scale,
+                  const float* __restrict__ w, int H, int d, int G, int Hg,
+                  __nv_bfloat16* __restrict__ qbar, float* __restrict__ wbar) {
+  const int64_t g = blockIdx.x;
+  const int n8 = Hg * d / 8;
+  const float inv = 1.f / static_cast<float>(G);
+  for (int e = threadIdx.x; e < n8; e += blockDim.x) {
+    const int j = (e * 8) / d, c = (e * 8) % d;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int i = 0; i < G; ++i) {
+      const int64_t r = g * G + i;
+      float x[8];
+      load8<IN_E4M3>(q, (r * H + j) * d + c, IN_E4M3 ? q_scale[r] : 1.f, x);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc[u] += x[u];
+    }
+    uint4 v;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) h[u] = __floats2bfloat162_rn(acc[2 * u] * inv, acc[2 * u + 1] * inv);
+    reinterpret_cast<uint4*>(qbar + (g * Hg + j) * d + c)[0] = v;
+  }
+  for (int j = threadIdx.x; j < Hg; j += blockDim.x) {
+    float a = 0.f;
+    for (int i = 0; i < G; ++i) a += w[(g * G + i) * H + j];
+    wbar[g * Hg + j] = a * inv;
+  }
+}
+
 template <bool IN_E4M3, bool OUT_E4M3>
 cudaError_t launch_prepare_rows(const void* q, const float* q_scale, const float* w, int64_t rows,
                                 int H, int d, void* q_out, float* q_scale_out, int8_t* fold_flag,
@@ -300,6 +333,19 @@ cudaError_t launch_mtp_candidates(int32_t* cand, int32_t n_groups, int32_t width
   if (total <= 0) return cudaSuccess;
   mtp_candidates_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, s>>>(
       cand, n_groups, width, P, G, m, seq_len, anchor_pos);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_group_mean(const void* q, const float* q_scale, bool in_e4m3, const float* w,
+                              int64_t n_groups, int H, int d, int G, int Hg, void* qbar,
+                              float* wbar, cudaStream_t s) {
+  if (n_groups <= 0) return cudaSuccess;
+  const unsigned grid = static_cast<unsigned>(n_groups);
+  __nv_bfloat16* qb = static_cast<__nv_bfloat16*>(qbar);
+  if (in_e4m3)
+    group_mean_kernel<true><<<grid, 256, 0, s>>>(q, q_scale, w, H, d, G, Hg, qb, wbar);
+  else
+    group_mean_kernel<false><<<grid, 256, 0, s>>>(q, q_scale, w, H, d, G, Hg, qb, wbar);
   return cudaGetLastError();
 }
 

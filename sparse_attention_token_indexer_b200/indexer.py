@@ -191,6 +191,19 @@ def index_mtp(q, w, k, seq_len, qbar, wbar, m, G, P, K, q_scale=None, k_scale=No
     return idx, sc, banks
 
 
+def group_query_mean(q, w, G, Hg, q_scale=None, stream=None):
+    """Mean-pooled group queries (the PIVOT proxy): q [T, H, d] bf16 or e4m3, w [T, H]
+    -> (qbar [T // G, Hg, d] bf16, wbar [T // G, Hg] fp32)."""
+    _dev(q, "q"), _dev(w, "w", torch.float32), _dev(q_scale, "q_scale", torch.float32)
+    T, H, d = q.shape
+    qbar = torch.empty(T // G, Hg, d, dtype=torch.bfloat16, device=q.device)
+    wbar = torch.empty(T // G, Hg, dtype=torch.float32, device=q.device)
+    L.check("adx_group_query_mean", L.lib().adx_group_query_mean(
+        _dtype(q), q.data_ptr(), _p(q_scale), w.data_ptr(), T, H, d, G, Hg, qbar.data_ptr(),
+        wbar.data_ptr(), _stream(stream)))
+    return qbar, wbar
+
+
 def read_device_status(ws=None, device=None, stream=None):
     """Synchronises and returns (and clears) the device status of a workspace (0 = ok)."""
     w = _ws(ws, device or torch.device("cuda"))

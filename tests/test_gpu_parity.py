@@ -482,3 +482,50 @@ def test_group_mode_on_a_later_chunk(mode):
         n = q_pos0 + r + 1
         check_topk(idx[r], np.arange(n), ox.score_keys(q64[r], w64[r], k64[:n]),
                    score_floor(q64[r], w64[r], k64[:n]), K, RTOL["bf16"], sc[r], f"tail {r}")
+
+
+# ---------------------------------------------------------------------------------------
+# training-free group queries (the PIVOT proxy)
+# ---------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+@pytest.mark.parametrize("G,Hg", [(64, 16), (4, 64), (16, 16), (1, 8)])
+def test_group_query_mean(dtype, G, Hg):
+    """bf16 output of an fp32 member sum: within half a bf16 step of the exact mean plus the
+    fp32 accumulation error relative to the members' magnitudes."""
+    T = 1000
+    p = inputs.anchor_prefill(T, H=64, d=128, K=64, seed=26, device="cuda", dtype=dtype)
+    qbar, wbar = indexer.group_query_mean(p["q"], p["w"], G, Hg, q_scale=p["q_scale"])
+    q64, w64 = f64(p["q"], p["q_scale"]), p["w"].double().cpu().numpy()
+    rq, rw = ox.mean_pool_group(q64, w64, G, Hg)
+    ng = T // G
+    mag = np.abs(q64[:ng * G, :Hg]).reshape(ng, G, Hg, -1).mean(axis=1)
+    got = f64(qbar)
+    assert got.shape == rq.shape
+    assert np.all(np.abs(got - rq) <= 2.0 ** -8 * np.abs(rq) + 2.0 ** -20 * (mag + 1e-30))
+    assert np.allclose(wbar.cpu().double().numpy(), rw, rtol=1e-6, atol=0)
+
+
+def test_group_mode_on_kernel_group_queries():
+    """Group mode end to end with the group queries built by the library itself."""
+    T, G, B, K, Hg = 64 * 12, 64, 256, 128, 16
+    p = _to_cuda(inputs.anchor_prefill(T, H=64, d=128, K=K, seed=27))
+    qbar, wbar = indexer.group_query_mean(p["q"], p["w"], G, Hg)
+    bank = indexer.group_bank(qbar, wbar, p["k"], G, B, "paper")
+    idx, sc = indexer.bank_refine(p["q"], p["w"], p["k"], bank, G, B, "paper", K,
+                                  with_scores=True)
+    q64, k64, w64 = f64(p["q"]), f64(p["k"]), p["w"].double().cpu().numpy()
+    qb64, wb64 = f64(qbar), wbar.double().cpu().numpy()
+    bank, idx, sc = bank.cpu().numpy(), idx.cpu().numpy(), sc.cpu().numpy()
+    for g in range(T // G):
+        a = g * G
+        keys = k64[:a + 1]
+        check_topk(bank[g, :B], np.arange(a + 1), ox.score_keys(qb64[g], wb64[g], keys),
+                   score_floor(qb64[g], wb64[g], keys), B, RTOL["bf16"], what=f"bank {g}")
+        part = bank[g, :B][bank[g, :B] >= 0]
+        for r in range(a, a + G, 9):
+            cand = np.union1d(part, np.arange(a + 1, r + 1)) if a + 1 > B else np.arange(r + 1)
+            cand = cand[cand <= r]
+            check_topk(idx[r], cand, ox.score_keys(q64[r], w64[r], k64[cand]),
+                       score_floor(q64[r], w64[r], k64[cand]), K, RTOL["bf16"], sc[r],
+                       f"refine row {r}")
