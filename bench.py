@@ -38,6 +38,8 @@ FLAT_SMALL = dict(T=8192, H=64, d=128, K=2048, seed=1)
 GROUP = dict(T=65536, H=64, d=128, K=2048, G=64, B=8192, Hg=16, seed=2)
 DECODE = dict(Bs=32, S=131072, H=64, d=128, K=2048, Hg=16, B=8192, G=16, seed=3)
 CHUNKED = dict(S=262144, chunk=4096, H=64, d=128, K=2048, G=64, B=8192, Hg=16, seed=4)
+# rows per chunk of the host-buffer path (copies of one chunk overlap the work on another)
+E2E_ROWS_PER_CHUNK = 2048
 # MTP target verification on the decode caches: one window of m draft tokens per sequence
 MTP = dict(m=16, G=8, P=8192)
 
@@ -263,23 +265,18 @@ def _call_prefill(p, K, idx, ws):
 
 
 def run_e2e(args, dist, p):
-    """Same step through the public API with host buffers: pinned H2D of the inputs, the
-    indexer, and D2H of the Top-K indices, every step inside the timed region."""
+    """Same step through the public API with host buffers (adx_index_prefill_host): pinned
+    H2D of the inputs, the indexer and D2H of the Top-K indices, every step inside the timed
+    region; the library overlaps the copies of one chunk of rows with the indexing of another."""
     from sparse_attention_token_indexer_b200 import indexer
     c = FLAT
     host = {k: p[k].cpu().pin_memory() for k in ("q", "w", "k")}
-    dev = {k: torch.empty_like(p[k]) for k in ("q", "w", "k")}
     out_h = torch.empty(c["T"], c["K"], dtype=torch.int32).pin_memory()
-    idx = torch.empty(c["T"], c["K"], dtype=torch.int32, device="cuda")
     ws = indexer.Workspace("cuda")
-    q = dict(p)
 
     def step():
-        for k in dev:
-            dev[k].copy_(host[k], non_blocking=True)
-        q.update(dev)
-        _call_prefill(q, c["K"], idx, ws)
-        out_h.copy_(idx, non_blocking=True)
+        indexer.index_prefill_host(host["q"], host["w"], host["k"], c["K"],
+                                   rows_per_chunk=E2E_ROWS_PER_CHUNK, out=(out_h, None), ws=ws)
 
     ms, _ = timed(step, args.steps, args.warmup, dist)
     h2d = sum(t.numel() * t.element_size() for t in host.values())

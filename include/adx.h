@@ -13,7 +13,8 @@
  * Conventions shared by every entry point
  *  - Every pointer argument is a DEVICE pointer unless stated otherwise. The caller owns
  *    all memory; the library allocates nothing, keeps no state between calls besides
- *    cached device properties, and launches all work asynchronously on `stream` (a
+ *    cached device properties (and, for adx_index_prefill_host, two copy streams and their
+ *    events per device, created on first use), and launches all work asynchronously on `stream` (a
  *    cudaStream_t passed as void*; NULL = the legacy default stream).
  *  - Argument errors are detected on the host and returned before any launch.
  *  - Errors the device detects (a bounded wait that ran out) are recorded in a status word
@@ -68,7 +69,8 @@ typedef enum {
   ADX_OP_PREFILL = 0,
   ADX_OP_DECODE = 1,
   ADX_OP_GROUP_BANK = 2,
-  ADX_OP_BANK_REFINE = 3
+  ADX_OP_BANK_REFINE = 3,
+  ADX_OP_PREFILL_HOST = 4  /* adx_workspace_size: B = rows_per_chunk */
 } adx_op;
 
 /* One indexer operand set.
@@ -117,6 +119,22 @@ int32_t adx_bank_width(int32_t B, int32_t G, int32_t mode);
 adx_status adx_index_prefill(const adx_operands* ops, int32_t K, int32_t* topk_idx,
                              float* topk_score, float* scores_out, int64_t scores_ld, void* ws,
                              size_t ws_bytes, void* stream);
+
+/* Flat causal indexer over host buffers (same computation as adx_index_prefill, prefill
+ * layout): q, q_scale, w, k, k_scale of `ops` and topk_idx [T, K] / topk_score [T, K] (or NULL)
+ * are HOST pointers, page-locked for the copies to overlap the work. The rows are indexed in
+ * chunks of rows_per_chunk (at most 64 chunks): chunk c's queries and gates are copied in while
+ * chunk c-1 is indexed on `stream`, and chunk c-1's Top-K rows are copied out while chunk c is
+ * indexed, on two copy streams the library keeps per device. The call returns once everything
+ * is queued; the results are in the host arrays when `stream` has completed. Work queued on
+ * `stream` before the call finishes before the first copy starts. Calls on one device must
+ * not be issued from several host threads at the same time.
+ * ws  device workspace of ws_bytes >= adx_workspace_size(ADX_OP_PREFILL_HOST, ops, K,
+ *     rows_per_chunk, 0, 0): device copies of the operands and results, one chunk's indexer
+ *     workspace. */
+adx_status adx_index_prefill_host(const adx_operands* ops, int32_t K, int32_t rows_per_chunk,
+                                  int32_t* topk_idx, float* topk_score, void* ws,
+                                  size_t ws_bytes, void* stream);
 
 /* Flat indexer for one query per sequence against that sequence's key cache (§3,
  * Eqs. (1)-(2), one decode step); decode layout. topk_idx [T, K], topk_score [T, K] or NULL. */

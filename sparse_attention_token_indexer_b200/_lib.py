@@ -11,7 +11,7 @@ LIB_PATH = os.path.join(HERE, "libadx.so")
 ADX_OK, ADX_EINVAL, ADX_EUNSUPPORTED, ADX_EWORKSPACE, ADX_ECUDA, ADX_EOVERFLOW, ADX_ETIMEOUT = range(7)
 ADX_BF16, ADX_E4M3 = 0, 1
 ADX_BANK_PAPER, ADX_BANK_WINDOW = 0, 1
-ADX_OP_PREFILL, ADX_OP_DECODE, ADX_OP_GROUP_BANK, ADX_OP_BANK_REFINE = range(4)
+ADX_OP_PREFILL, ADX_OP_DECODE, ADX_OP_GROUP_BANK, ADX_OP_BANK_REFINE, ADX_OP_PREFILL_HOST = range(5)
 ADX_STATUS_BYTES = 256
 
 # every extern "C" symbol include/adx.h declares
@@ -19,7 +19,7 @@ EXPORTS = ("adx_abi_version", "adx_bank_width", "adx_status_string", "adx_worksp
            "adx_index_prefill", "adx_index_decode", "adx_group_bank", "adx_bank_refine",
            "adx_read_device_status", "adx_set_timing_events", "adx_launch_count",
            "adx_index_prefill_noalloc", "adx_mtp_workspace_size", "adx_index_mtp",
-           "adx_group_union_sizes", "adx_group_query_mean")
+           "adx_group_union_sizes", "adx_group_query_mean", "adx_index_prefill_host")
 
 
 class Operands(ctypes.Structure):
@@ -68,6 +68,7 @@ def _declare(lib):
         "adx_mtp_workspace_size": (SZ, [P, P, I32, I32, I32, I32]),
         "adx_index_mtp": (ctypes.c_int, [P, P, I32, I32, I32, I32, VP, VP, VP, VP, SZ, VP]),
         "adx_group_union_sizes": (ctypes.c_int, [VP, I32, I32, I32, I32, VP, VP]),
+        "adx_index_prefill_host": (ctypes.c_int, [P, I32, I32, VP, VP, VP, SZ, VP]),
         "adx_group_query_mean": (ctypes.c_int, [I32, VP, VP, VP, I32, I32, I32, I32, I32, VP,
                                                 VP, VP]),
     }

@@ -431,6 +431,65 @@ size_t ws_refine(const adx_operands* o, int G, int B, int mode, int K) {
   return b;
 }
 
+// ---- flat prefill from host buffers ---------------------------------------------------
+// Copy engines of a device: two non-blocking streams (host to device, device to host) and the
+// events that chain a chunk's copy-in, indexing and copy-out. Created on first use and kept.
+constexpr int kHostMaxChunks = 64;
+constexpr int kMaxDevices = 64;
+struct CopyEngines {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t in[kHostMaxChunks], done[kHostMaxChunks], out;
+  bool ready = false;
+};
+std::mutex g_copy_mutex;
+CopyEngines g_copy[kMaxDevices];
+
+adx_status copy_engines(CopyEngines** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ADX_ECUDA;
+  std::lock_guard<std::mutex> lock(g_copy_mutex);
+  CopyEngines& c = g_copy[dev];
+  if (!c.ready) {
+    if (cudaStreamCreateWithFlags(&c.h2d, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&c.d2h, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c.out, cudaEventDisableTiming) != cudaSuccess)
+      return ADX_ECUDA;
+    for (int i = 0; i < kHostMaxChunks; ++i)
+      if (cudaEventCreateWithFlags(&c.in[i], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&c.done[i], cudaEventDisableTiming) != cudaSuccess)
+        return ADX_ECUDA;
+    c.ready = true;
+  }
+  *out = &c;
+  return ADX_OK;
+}
+
+struct HostLayout {
+  size_t q_row, k_row;  // bytes of a query row (all heads) and of a key row
+  int64_t C, chunks;
+};
+
+bool host_layout(const adx_operands* o, int C, HostLayout& h) {
+  if (C <= 0) return false;
+  h.q_row = static_cast<size_t>(o->H) * o->d * (o->q_dtype == ADX_E4M3 ? 1 : 2);
+  h.k_row = static_cast<size_t>(o->d) * (o->k_dtype == ADX_E4M3 ? 1 : 2);
+  h.C = C;
+  h.chunks = (o->T + C - 1) / C;
+  return h.chunks <= kHostMaxChunks;
+}
+
+size_t ws_prefill_host(const adx_operands* o, int K, const HostLayout& h) {
+  const size_t T = o->T, S = o->S;
+  size_t b = kStatusBytes;
+  b += align_up(T * h.q_row, kAlign) + (o->q_scale ? align_up(T * 4, kAlign) : 0) +
+       align_up(T * o->H * 4, kAlign);
+  b += align_up(S * h.k_row, kAlign) + (o->k_scale ? align_up(S * 4, kAlign) : 0);
+  b += align_up(T * K * 4, kAlign) * 2;  // indices, scores
+  adx_operands chunk = *o;
+  chunk.T = static_cast<int32_t>(std::min<int64_t>(h.C, o->T));
+  return b + ws_flat(&chunk, K, false) - kStatusBytes;
+}
+
 // ---- MTP target verification ----------------------------------------------------------
 struct MtpShape {
   int64_t Bs, ng, width, bcp;
@@ -528,6 +587,11 @@ size_t adx_workspace_size(int32_t op, const adx_operands* ops, int32_t K, int32_
           check_bank_args(ops, G, B, mode) != ADX_OK)
         return 0;
       return ws_bank(ops, G, B, mode);
+    case ADX_OP_PREFILL_HOST: {
+      HostLayout h;
+      if (K <= 0 || check_operands(ops, false) != ADX_OK || !host_layout(ops, B, h)) return 0;
+      return ws_prefill_host(ops, K, h);
+    }
     case ADX_OP_BANK_REFINE:
       if (K <= 0 || check_operands(ops, ops->seq_len != nullptr) != ADX_OK ||
           check_bank_args(ops, G, B, mode) != ADX_OK)
@@ -755,6 +819,77 @@ size_t adx_mtp_workspace_size(const adx_operands* full, const adx_operands* grp,
   adx_operands gops;
   if (mtp_check(full, grp, m, G, P, K, sh, gops) != ADX_OK) return 0;
   return ws_mtp(full, &gops, sh, m, P, K);
+}
+
+adx_status adx_index_prefill_host(const adx_operands* o, int32_t K, int32_t rows_per_chunk,
+                                  int32_t* topk_idx, float* topk_score, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  adx_status r = check_operands(o, false);
+  if (r != ADX_OK) return r;
+  HostLayout h;
+  if (K <= 0 || !topk_idx || !ws || !host_layout(o, rows_per_chunk, h)) return ADX_EINVAL;
+  if (ws_bytes < ws_prefill_host(o, K, h)) return ADX_EWORKSPACE;
+  CopyEngines* ce = nullptr;
+  if ((r = copy_engines(&ce)) != ADX_OK) return r;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t T = o->T, S = o->S, H = o->H;
+  Carve cv(ws);
+  DeviceStatus* st = cv.take<DeviceStatus>(kStatusBytes);
+  uint8_t* dq = cv.take<uint8_t>(static_cast<size_t>(T) * h.q_row);
+  float* dqs = o->q_scale ? cv.take<float>(static_cast<size_t>(T) * 4) : nullptr;
+  float* dw = cv.take<float>(static_cast<size_t>(T) * H * 4);
+  uint8_t* dk = cv.take<uint8_t>(static_cast<size_t>(S) * h.k_row);
+  float* dks = o->k_scale ? cv.take<float>(static_cast<size_t>(S) * 4) : nullptr;
+  int32_t* didx = cv.take<int32_t>(static_cast<size_t>(T) * K * 4);
+  float* dsc = cv.take<float>(static_cast<size_t>(T) * K * 4);
+  uint8_t* chunk_ws = cv.base + cv.off;
+  auto copy = [](void* dst, const void* src, size_t n, cudaMemcpyKind k, cudaStream_t cs) {
+    return n == 0 || cudaMemcpyAsync(dst, src, n, k, cs) == cudaSuccess;
+  };
+  // the copies start once everything queued on `stream` before this call is done
+  if (cudaEventRecord(ce->out, s) != cudaSuccess ||
+      cudaStreamWaitEvent(ce->h2d, ce->out, 0) != cudaSuccess)
+    return ADX_ECUDA;
+  if (!copy(dk, o->k, static_cast<size_t>(S) * h.k_row, cudaMemcpyHostToDevice, ce->h2d) ||
+      (dks && !copy(dks, o->k_scale, static_cast<size_t>(S) * 4, cudaMemcpyHostToDevice, ce->h2d)))
+    return ADX_ECUDA;
+  for (int64_t c = 0; c < h.chunks; ++c) {
+    const int64_t r0 = c * h.C, r1 = std::min(T, r0 + h.C), n = r1 - r0;
+    // chunk c in, while `stream` indexes chunk c-1
+    if (!copy(dq + r0 * h.q_row, static_cast<const uint8_t*>(o->q) + r0 * h.q_row, n * h.q_row,
+              cudaMemcpyHostToDevice, ce->h2d) ||
+        !copy(dw + r0 * H, o->w + r0 * H, n * H * 4, cudaMemcpyHostToDevice, ce->h2d) ||
+        (dqs && !copy(dqs + r0, o->q_scale + r0, n * 4, cudaMemcpyHostToDevice, ce->h2d)))
+      return ADX_ECUDA;
+    if (cudaEventRecord(ce->in[c], ce->h2d) != cudaSuccess ||
+        cudaStreamWaitEvent(s, ce->in[c], 0) != cudaSuccess)
+      return ADX_ECUDA;
+    adx_operands chunk = *o;
+    chunk.q = dq + r0 * h.q_row;
+    chunk.q_scale = dqs ? dqs + r0 : nullptr;
+    chunk.w = dw + r0 * H;
+    chunk.k = dk;
+    chunk.k_scale = dks;
+    chunk.T = static_cast<int32_t>(n);
+    chunk.q_pos0 = o->q_pos0 + r0;
+    Carve ccv(chunk_ws);
+    if ((r = run_flat(&chunk, K, didx + r0 * K, topk_score ? dsc + r0 * K : nullptr, nullptr, 0,
+                      ccv, st, s)) != ADX_OK)
+      return r;
+    // chunk c out, while `stream` indexes chunk c+1
+    if (cudaEventRecord(ce->done[c], s) != cudaSuccess ||
+        cudaStreamWaitEvent(ce->d2h, ce->done[c], 0) != cudaSuccess)
+      return ADX_ECUDA;
+    if (!copy(topk_idx + r0 * K, didx + r0 * K, n * K * 4, cudaMemcpyDeviceToHost, ce->d2h) ||
+        (topk_score &&
+         !copy(topk_score + r0 * K, dsc + r0 * K, n * K * 4, cudaMemcpyDeviceToHost, ce->d2h)))
+      return ADX_ECUDA;
+  }
+  // `stream` completes only after the last copy out
+  if (cudaEventRecord(ce->out, ce->d2h) != cudaSuccess ||
+      cudaStreamWaitEvent(s, ce->out, 0) != cudaSuccess)
+    return ADX_ECUDA;
+  return ADX_OK;
 }
 
 adx_status adx_index_mtp(const adx_operands* full, const adx_operands* grp, int32_t m, int32_t G,

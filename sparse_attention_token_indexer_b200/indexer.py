@@ -122,6 +122,38 @@ def index_prefill(q, w, k, K, q_scale=None, k_scale=None, q_pos0=0, with_scores=
     return idx, sc, full
 
 
+def index_prefill_host(q, w, k, K, q_scale=None, k_scale=None, q_pos0=0, rows_per_chunk=2048,
+                       with_scores=False, out=None, ws=None, stream=None):
+    """Flat causal indexer over HOST tensors (pinned for the copies to overlap the work):
+    -> (topk_idx [T, K] int32, topk_score or None), host tensors, valid once `stream` (the
+    current one by default) has completed. `out` may pass preallocated (pinned) outputs."""
+    for name, t in (("q", q), ("w", w), ("k", k), ("q_scale", q_scale), ("k_scale", k_scale)):
+        if t is not None and (t.is_cuda or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous host tensor")
+    T, H, d = q.shape
+    o = L.Operands()
+    o.q_dtype, o.k_dtype = _dtype(q), _dtype(k)
+    o.q, o.q_scale, o.w = q.data_ptr(), _p(q_scale), w.data_ptr()
+    o.k, o.k_scale = k.data_ptr(), _p(k_scale)
+    o.T, o.H, o.d, o.S = T, H, d, k.shape[-2]
+    o.q_pos0 = int(q_pos0)
+    o.seq_len = None
+    if out is None:
+        idx = torch.empty(T, K, dtype=torch.int32).pin_memory()
+        sc = torch.empty(T, K, dtype=torch.float32).pin_memory() if with_scores else None
+    else:
+        idx, sc = out
+    need = L.lib().adx_workspace_size(L.ADX_OP_PREFILL_HOST, ctypes.byref(o), K, rows_per_chunk,
+                                      0, 0)
+    if need == 0:
+        raise L.AdxError("adx_workspace_size", L.ADX_EINVAL)
+    buf = _ws(ws, torch.device("cuda")).get(need)
+    L.check("adx_index_prefill_host", L.lib().adx_index_prefill_host(
+        ctypes.byref(o), K, rows_per_chunk, _p(idx), _p(sc), _p(buf), buf.numel(),
+        _stream(stream)))
+    return idx, sc
+
+
 def index_decode(q, w, k, seq_len, K, q_scale=None, k_scale=None, with_scores=False, ws=None,
                  stream=None):
     """One decode step of the flat indexer: row t scores its own cache k[t]."""

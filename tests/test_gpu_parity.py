@@ -529,3 +529,25 @@ def test_group_mode_on_kernel_group_queries():
             check_topk(idx[r], cand, ox.score_keys(q64[r], w64[r], k64[cand]),
                        score_floor(q64[r], w64[r], k64[cand]), K, RTOL["bf16"], sc[r],
                        f"refine row {r}")
+
+
+# ---------------------------------------------------------------------------------------
+# host buffers (copies overlapped with the indexing, chunk by chunk)
+# ---------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_host_buffer_prefill_equals_device_path(dtype):
+    """Chunking only changes how the rows are partitioned: every row's scores and Top-K are
+    the same as on the device-buffer path, bit for bit."""
+    T, K = 5000, 300
+    p = inputs.anchor_prefill(T, H=64, d=128, K=K, seed=28, device="cuda", dtype=dtype, S=5300)
+    ref_idx, ref_sc, _ = indexer.index_prefill(p["q"], p["w"], p["k"], K, p["q_scale"],
+                                               p["k_scale"], q_pos0=p["q_pos0"], with_scores=True)
+    host = {n: (None if p[n] is None else p[n].cpu().pin_memory())
+            for n in ("q", "w", "k", "q_scale", "k_scale")}
+    idx, sc = indexer.index_prefill_host(host["q"], host["w"], host["k"], K, host["q_scale"],
+                                         host["k_scale"], q_pos0=p["q_pos0"],
+                                         rows_per_chunk=1024, with_scores=True)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, ref_idx.cpu())
+    assert torch.equal(sc, ref_sc.cpu())
