@@ -39,7 +39,7 @@ GROUP = dict(T=65536, H=64, d=128, K=2048, G=64, B=8192, Hg=16, seed=2)
 DECODE = dict(Bs=32, S=131072, H=64, d=128, K=2048, Hg=16, B=8192, G=16, seed=3)
 CHUNKED = dict(S=262144, chunk=4096, H=64, d=128, K=2048, G=64, B=8192, Hg=16, seed=4)
 # rows per chunk of the host-buffer path (copies of one chunk overlap the work on another)
-E2E_ROWS_PER_CHUNK = 2048
+E2E_ROWS_PER_CHUNK = 1024
 # MTP target verification on the decode caches: one window of m draft tokens per sequence
 MTP = dict(m=16, G=8, P=8192)
 

@@ -123,9 +123,10 @@ adx_status adx_index_prefill(const adx_operands* ops, int32_t K, int32_t* topk_i
 /* Flat causal indexer over host buffers (same computation as adx_index_prefill, prefill
  * layout): q, q_scale, w, k, k_scale of `ops` and topk_idx [T, K] / topk_score [T, K] (or NULL)
  * are HOST pointers, page-locked for the copies to overlap the work. The rows are indexed in
- * chunks of rows_per_chunk (at most 64 chunks): chunk c's queries and gates are copied in while
- * chunk c-1 is indexed on `stream`, and chunk c-1's Top-K rows are copied out while chunk c is
- * indexed, on two copy streams the library keeps per device. The call returns once everything
+ * chunks of rows_per_chunk (at most 64 chunks), the last (longest) rows first: one chunk's
+ * queries and gates are copied in while the chunk before it is indexed on `stream`, and each
+ * chunk's Top-K rows are copied out while the next one is indexed, on two copy streams the
+ * library keeps per device. The call returns once everything
  * is queued; the results are in the host arrays when `stream` has completed. Work queued on
  * `stream` before the call finishes before the first copy starts. Calls on one device must
  * not be issued from several host threads at the same time.

@@ -853,9 +853,12 @@ adx_status adx_index_prefill_host(const adx_operands* o, int32_t K, int32_t rows
   if (!copy(dk, o->k, static_cast<size_t>(S) * h.k_row, cudaMemcpyHostToDevice, ce->h2d) ||
       (dks && !copy(dks, o->k_scale, static_cast<size_t>(S) * 4, cudaMemcpyHostToDevice, ce->h2d)))
     return ADX_ECUDA;
-  for (int64_t c = 0; c < h.chunks; ++c) {
+  // longest rows first: the indexing work then shrinks chunk by chunk, so what follows the
+  // last copy in is the cheapest chunk and its copy out
+  for (int64_t i = 0; i < h.chunks; ++i) {
+    const int64_t c = h.chunks - 1 - i;
     const int64_t r0 = c * h.C, r1 = std::min(T, r0 + h.C), n = r1 - r0;
-    // chunk c in, while `stream` indexes chunk c-1
+    // chunk c in, while `stream` indexes the chunk before it
     if (!copy(dq + r0 * h.q_row, static_cast<const uint8_t*>(o->q) + r0 * h.q_row, n * h.q_row,
               cudaMemcpyHostToDevice, ce->h2d) ||
         !copy(dw + r0 * H, o->w + r0 * H, n * H * 4, cudaMemcpyHostToDevice, ce->h2d) ||
@@ -876,7 +879,7 @@ adx_status adx_index_prefill_host(const adx_operands* o, int32_t K, int32_t rows
     if ((r = run_flat(&chunk, K, didx + r0 * K, topk_score ? dsc + r0 * K : nullptr, nullptr, 0,
                       ccv, st, s)) != ADX_OK)
       return r;
-    // chunk c out, while `stream` indexes chunk c+1
+    // chunk c out, while `stream` indexes the next one
     if (cudaEventRecord(ce->done[c], s) != cudaSuccess ||
         cudaStreamWaitEvent(ce->d2h, ce->done[c], 0) != cudaSuccess)
       return ADX_ECUDA;
