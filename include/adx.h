@@ -213,6 +213,13 @@ adx_status adx_group_query_mean(int32_t q_dtype, const void* q, const float* q_s
 adx_status adx_group_union_sizes(const int32_t* topk_idx, int32_t T, int32_t K, int32_t G,
                                  int32_t S, int32_t* union_out, void* stream);
 
+/* Failure-detection check (no counterpart in the paper): one CTA waits, with the bounded wait
+ * the indexer's kernels use, on a barrier that nothing completes; after timeout_ns (at most
+ * 1 s) the wait gives up and records ADX_ETIMEOUT in the status word of `ws`, as a real wait
+ * that ran out would. The device stays usable; adx_read_device_status(ws) then returns
+ * ADX_ETIMEOUT (and clears it). */
+adx_status adx_check_wait_timeout(void* ws, uint64_t timeout_ns, void* stream);
+
 /* Synchronises `stream`, returns the device status recorded in `ws` (ADX_OK if none) and
  * clears it. */
 adx_status adx_read_device_status(void* ws, void* stream);

@@ -19,7 +19,8 @@ EXPORTS = ("adx_abi_version", "adx_bank_width", "adx_status_string", "adx_worksp
            "adx_index_prefill", "adx_index_decode", "adx_group_bank", "adx_bank_refine",
            "adx_read_device_status", "adx_set_timing_events", "adx_launch_count",
            "adx_index_prefill_noalloc", "adx_mtp_workspace_size", "adx_index_mtp",
-           "adx_group_union_sizes", "adx_group_query_mean", "adx_index_prefill_host")
+           "adx_group_union_sizes", "adx_group_query_mean", "adx_index_prefill_host",
+           "adx_check_wait_timeout")
 
 
 class Operands(ctypes.Structure):
@@ -69,6 +70,7 @@ def _declare(lib):
         "adx_index_mtp": (ctypes.c_int, [P, P, I32, I32, I32, I32, VP, VP, VP, VP, SZ, VP]),
         "adx_group_union_sizes": (ctypes.c_int, [VP, I32, I32, I32, I32, VP, VP]),
         "adx_index_prefill_host": (ctypes.c_int, [P, I32, I32, VP, VP, VP, SZ, VP]),
+        "adx_check_wait_timeout": (ctypes.c_int, [VP, ctypes.c_uint64, VP]),
         "adx_group_query_mean": (ctypes.c_int, [I32, VP, VP, VP, I32, I32, I32, I32, I32, VP,
                                                 VP, VP]),
     }

@@ -1029,6 +1029,13 @@ adx_status adx_group_union_sizes(const int32_t* topk_idx, int32_t T, int32_t K, 
   return e == cudaSuccess ? ADX_OK : ADX_ECUDA;
 }
 
+adx_status adx_check_wait_timeout(void* ws, uint64_t timeout_ns, void* stream) {
+  if (!ws || timeout_ns == 0 || timeout_ns > 1000000000ull) return ADX_EINVAL;
+  const cudaError_t e = counted(launch_wait_timeout(static_cast<DeviceStatus*>(ws), timeout_ns,
+                                                    static_cast<cudaStream_t>(stream)));
+  return e == cudaSuccess ? ADX_OK : ADX_ECUDA;
+}
+
 adx_status adx_read_device_status(void* ws, void* stream) {
   if (!ws) return ADX_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -17,6 +17,7 @@ struct DeviceStatus {
 constexpr size_t kStatusBytes = 256;
 constexpr int kWhereScore = 1;
 constexpr int kWhereSelect = 2;
+constexpr int kWhereCheck = 3;
 
 constexpr int kTileM = 128;  // keys per MMA tile (TMEM lanes)
 
@@ -127,6 +128,9 @@ cudaError_t launch_mtp_positions(const int32_t* seq_len, int32_t Bs, int32_t m, 
 cudaError_t launch_mtp_candidates(int32_t* cand, int32_t n_groups, int32_t width, int32_t P,
                                   int32_t G, int32_t m, const int32_t* seq_len,
                                   const int32_t* anchor_pos, cudaStream_t s);
+// One CTA whose bounded wait on a barrier nothing completes runs out after timeout_ns and is
+// recorded in *status (code ADX_ETIMEOUT) like a wait of the indexer's kernels.
+cudaError_t launch_wait_timeout(DeviceStatus* status, uint64_t timeout_ns, cudaStream_t s);
 // Mean-pooled group queries qbar [n_groups, Hg, d] bf16 and gates wbar [n_groups, Hg].
 cudaError_t launch_group_mean(const void* q, const float* q_scale, bool in_e4m3, const float* w,
                               int64_t n_groups, int H, int d, int G, int Hg, void* qbar,

@@ -13,6 +13,7 @@
 #include <cstdint>
 
 #include "adx_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace adx {
 
@@ -79,6 +80,25 @@ __global__ void mtp_candidates_kernel(int32_t* __restrict__ cand, int32_t n_grou
     v = c < P + G - 1 ? a + 1 + (c - P) : -1;  // post-anchor positions, then padding
   }
   cand[i] = v;
+}
+
+// Failure-detection check: one thread waits, with the indexer kernels' bounded wait, on an
+// mbarrier that nothing completes, and records the timeout in the status word as they do.
+__global__ void wait_timeout_kernel(DeviceStatus* status, uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait(&bar, 0, &abort_flag, timeout_ns) &&
+      atomicCAS(&status->code, 0, 6 /* ADX_ETIMEOUT */) == 0) {
+    status->where = kWhereCheck;
+    status->info0 = 0;
+    status->info1 = 0;
+  }
 }
 
 // Union size of the Top-K sets of one group of G consecutive rows: a bitmap of the S
@@ -346,6 +366,11 @@ cudaError_t launch_group_mean(const void* q, const float* q_scale, bool in_e4m3,
     group_mean_kernel<true><<<grid, 256, 0, s>>>(q, q_scale, w, H, d, G, Hg, qb, wbar);
   else
     group_mean_kernel<false><<<grid, 256, 0, s>>>(q, q_scale, w, H, d, G, Hg, qb, wbar);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wait_timeout(DeviceStatus* status, uint64_t timeout_ns, cudaStream_t s) {
+  wait_timeout_kernel<<<1, 32, 0, s>>>(status, timeout_ns);
   return cudaGetLastError();
 }
 
