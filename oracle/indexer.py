@@ -267,3 +267,42 @@ def mean_pool_group(q, w, G, Hg):
         qbar[g] /= G
         wbar[g] /= G
     return qbar, wbar
+
+
+def rope(x, pos, rope_dim=64, base=10000.0):
+    """Rotary position embedding at position pos of one head vector x [d]: the pairs
+    (x[2i], x[2i+1]), i < rope_dim/2, are rotated by the angle pos * base^(-2i/rope_dim); the
+    other dimensions are left as they are (reading: the pages name RoPE at the group anchor
+    without its layout; this is the interleaved-pair form over the first rope_dim dims)."""
+    y = np.array(x, dtype=np.float64)
+    if rope_dim > y.shape[0] or rope_dim % 2:
+        raise ValueError("rope_dim must be even and at most the head dimension")
+    for i in range(rope_dim // 2):
+        a = pos * base ** (-2.0 * i / rope_dim)
+        c, s = np.cos(a), np.sin(a)
+        x0, x1 = y[2 * i], y[2 * i + 1]
+        y[2 * i], y[2 * i + 1] = x0 * c - x1 * s, x0 * s + x1 * c
+    return y
+
+
+def group_indexer_queries(cq, h, w_pool, w_q, w_g, G, H_S, d, q_pos0=0, rope_dim=64,
+                          base=10000.0):
+    """ADIndex §4.2, Eqs. (6)-(7): the group indexer's query and gates for each complete group
+    of G consecutive rows (anchor t = q_pos0 + g*G):
+      c-bar = W_pool [max_i c_i ; min_i c_i ; mean_i c_i]   (element-wise over the members)
+      h-bar = mean_i h_i
+      q-bar_j = RoPE_t([W_Q c-bar]_j),   w-bar_j = sigmoid([W_G h-bar]_j).
+    cq [T, d_c], h [T, d_h], w_pool [d_c, 3 d_c], w_q [H_S*d, d_c], w_g [H_S, d_h] ->
+    qbar [T // G, H_S, d], wbar [T // G, H_S]."""
+    cq, h = np.asarray(cq, np.float64), np.asarray(h, np.float64)
+    ng = cq.shape[0] // G
+    qbar, wbar = np.zeros((ng, H_S, d)), np.zeros((ng, H_S))
+    for g in range(ng):
+        c = cq[g * G:(g + 1) * G]
+        cbar = np.asarray(w_pool, np.float64) @ np.concatenate([c.max(0), c.min(0), c.mean(0)])
+        qpre = (np.asarray(w_q, np.float64) @ cbar).reshape(H_S, d)
+        for j in range(H_S):
+            qbar[g, j] = rope(qpre[j], q_pos0 + g * G, rope_dim, base)
+        z = np.asarray(w_g, np.float64) @ h[g * G:(g + 1) * G].mean(0)
+        wbar[g] = 1.0 / (1.0 + np.exp(-z))
+    return qbar, wbar

@@ -389,3 +389,51 @@ def test_mean_pool_group_hand_values():
     # G = 1 is the identity on the kept heads
     qb1, wb1 = ox.mean_pool_group(q, w, 1, 3)
     assert np.array_equal(qb1, q) and np.array_equal(wb1, w)
+
+
+# ---------------------------------------------------------------------------------------
+# Group indexer queries (ADIndex §4.2, Eqs. (6)-(7))
+# ---------------------------------------------------------------------------------------
+
+def test_rope_identity_norms_inverse_and_a_hand_value():
+    rng = np.random.default_rng(43)
+    x = rng.standard_normal(16)
+    assert np.allclose(ox.rope(x, 0, 8), x)
+    y = ox.rope(x, 37, 8)
+    assert np.allclose(y[8:], x[8:])                       # beyond rope_dim: unchanged
+    for i in range(4):                                     # each pair keeps its length
+        assert np.isclose(np.hypot(y[2 * i], y[2 * i + 1]), np.hypot(x[2 * i], x[2 * i + 1]))
+    assert np.allclose(ox.rope(y, -37, 8), x)             # rotating back recovers x
+    e = np.zeros(4)
+    e[0] = 1.0
+    assert np.allclose(ox.rope(e, 1, 4)[:2], [np.cos(1.0), np.sin(1.0)])   # pair 0: angle = pos
+    assert np.allclose(ox.rope(e[[1, 0, 2, 3]], 1, 4)[:2], [-np.sin(1.0), np.cos(1.0)])
+
+
+def test_group_indexer_pools_projects_and_gates():
+    rng = np.random.default_rng(44)
+    T, G, dc, dh, HS, d = 9, 4, 3, 5, 2, 4
+    cq, h = rng.standard_normal((T, dc)), rng.standard_normal((T, dh))
+    eye, zero = np.eye(dc), np.zeros((dc, dc))
+    wq = np.zeros((HS * d, dc))
+    wq[0:3, :] = np.eye(3)                                 # head 0, dims 0..2 <- c-bar
+    for k, sel in enumerate(([eye, zero, zero], [zero, eye, zero], [zero, zero, eye])):
+        qbar, wbar = ox.group_indexer_queries(cq, h, np.hstack(sel), wq, np.zeros((HS, dh)),
+                                              G, HS, d, rope_dim=0)
+        assert qbar.shape == (2, HS, d) and wbar.shape == (2, HS)   # trailing row dropped
+        for g in range(2):
+            members = cq[g * G:(g + 1) * G]
+            want = (members.max(0), members.min(0), members.mean(0))[k]
+            assert np.allclose(qbar[g, 0, :3], want)
+        assert np.allclose(wbar, 0.5)                      # sigmoid(0)
+    wg = np.zeros((HS, dh))
+    wg[1, 2] = 1.0
+    _, wbar = ox.group_indexer_queries(cq, h, np.hstack([eye, zero, zero]), wq, wg, G, HS, d,
+                                       rope_dim=0)
+    assert np.allclose(wbar[:, 1], 1 / (1 + np.exp(-np.array([h[0:4, 2].mean(), h[4:8, 2].mean()]))))
+    # RoPE at each group's anchor position
+    qb, _ = ox.group_indexer_queries(cq, h, np.hstack([eye, zero, zero]), wq, wg, G, HS, d,
+                                     q_pos0=10, rope_dim=4)
+    qn, _ = ox.group_indexer_queries(cq, h, np.hstack([eye, zero, zero]), wq, wg, G, HS, d,
+                                     q_pos0=10, rope_dim=0)
+    assert np.allclose(qb[1, 0], ox.rope(qn[1, 0], 14, 4))
