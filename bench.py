@@ -41,6 +41,7 @@ CHUNKED = dict(S=262144, chunk=4096, H=64, d=128, K=2048, G=64, B=8192, Hg=16, s
 # rows per chunk of the host-buffer path (copies of one chunk overlap the work on another)
 E2E_ROWS_PER_CHUNK = 1024
 # MTP target verification on the decode caches: one window of m draft tokens per sequence
+GROUP_INDEXER = dict(T=65536, G=64, d_c=1536, d_h=7168, H_S=16, d=128, seed=12)
 MTP = dict(m=16, G=8, P=8192)
 
 
@@ -413,6 +414,27 @@ def run_calibration(args, dist):
     return dict(ms=ms, launches=launches, bytes=3 * idx.numel() * 4)
 
 
+def run_group_indexer(args, dist):
+    """The trained group indexer's queries and gates (Eqs. (6)-(7)) for a 65536-token prefill
+    with G = 64: d_c = 1536 query latents, d_h = 7168 hidden states, H_S = 16 heads of d = 128,
+    synthetic weights. One step reads both activations once (1.14 GB, above L2)."""
+    from sparse_attention_token_indexer_b200 import indexer, inputs
+    c = GROUP_INDEXER
+    p = inputs.group_indexer_problem(c["T"], c["d_c"], c["d_h"], c["H_S"], c["d"], seed=c["seed"],
+                                     device="cuda")
+    ws = indexer.Workspace("cuda")
+
+    def step():
+        indexer.group_indexer_queries(p["cq"], p["h"], p["w_pool"], p["w_q"], p["w_g"], c["G"],
+                                      c["H_S"], c["d"], ws=ws)
+
+    ms, launches = timed(step, args.steps, args.warmup, dist)
+    ng = c["T"] // c["G"]
+    flops = 2 * ng * (c["d_c"] * 3 * c["d_c"] + c["H_S"] * c["d"] * c["d_c"] + c["H_S"] * c["d_h"])
+    act = c["T"] * (c["d_c"] + c["d_h"]) * 2
+    return dict(ms=ms, launches=launches, groups=ng, act_bytes=act, flops=flops)
+
+
 def run_chunked(args, dist):
     """256K-token prefill in query chunks of 4096 against the growing causal key cache, flat
     and in group mode (window bank, G = 64, B = 8192); one step = all 64 chunks."""
@@ -505,9 +527,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--rows", action="store_true", help="also time the other hot-path rows")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--case", default="flat", choices=["flat", "flat_small", "decode", "mtp"],
-                    help="flat_small: T = 8192, for profiler captures; decode, mtp: that "
-                         "workload alone (with --quick)")
+    ap.add_argument("--case", default="flat", choices=["flat", "flat_small", "decode", "mtp",
+                                                      "group_indexer"],
+                    help="flat_small: T = 8192, for profiler captures; decode, mtp, "
+                         "group_indexer: that workload alone (with --quick)")
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "e4m3"])
     ap.add_argument("--quick", action="store_true",
                     help="time the kernels only (no e2e, rows or CPU baseline): for profiling")
@@ -573,6 +596,14 @@ def main():
                               "flat_ms_per_round": mt["ms_flat"],
                               "speedup_vs_flat": mt["ms_flat"] / mt["ms"],
                               "gpu_launches": mt["launches"]}), flush=True)
+        dist.close()
+        return
+    if args.case == "group_indexer" and args.quick:
+        gi = run_group_indexer(args, dist)
+        if dist.rank == 0:
+            print(json.dumps({"case": "group_indexer", "ms_per_step": gi["ms"],
+                              "activation_gbs": gi["act_bytes"] / (gi["ms"] * 1e-3) / 1e9,
+                              "gpu_launches": gi["launches"]}), flush=True)
         dist.close()
         return
     flat = run_flat(args, dist, args.dtype, clocks)
@@ -659,6 +690,13 @@ def main():
             "gbs_read": cb["bytes"] / (cb["ms"] * 1e-3) / 1e9,
             "hbm_frac": cb["bytes"] / (cb["ms"] * 1e-3) / 1e9 / pk["hbm"],
             "gpu_launches": cb["launches"]}
+        gi = run_group_indexer(args, dist)
+        rows["group_indexer_queries_T65536_G64"] = {
+            "ms_per_step": gi["ms"], "groups_per_s": gi["groups"] / (gi["ms"] * 1e-3),
+            "activation_gbs": gi["act_bytes"] / (gi["ms"] * 1e-3) / 1e9,
+            "hbm_frac": gi["act_bytes"] / (gi["ms"] * 1e-3) / 1e9 / pk["hbm"],
+            "projection_gflop": gi["flops"] / 1e9, "gpu_launches": gi["launches"],
+            "note": "projections on cuBLAS (not counted in gpu_launches)"}
         rows["decode_bank_reuse_cycle16"] = {
             "ms_per_cycle": dcd["ms_cycle"],
             "ms_per_step": dcd["ms_cycle"] / dcd["steps_per_cycle"],

@@ -203,6 +203,40 @@ adx_status adx_group_query_mean(int32_t q_dtype, const void* q, const float* q_s
                                 const float* w, int32_t T, int32_t H, int32_t d, int32_t G,
                                 int32_t Hg, void* qbar_out, float* wbar_out, void* stream);
 
+/* The group indexer's queries and gates (ADIndex §4.2, Eqs. (6)-(7)) from the backbone's
+ * per-token query latents and hidden states. For each complete group g of G consecutive
+ * tokens (anchor t = q_pos0 + g*G):
+ *   c-bar = W_pool [max_i c_i ; min_i c_i ; mean_i c_i]   (element-wise over the members)
+ *   h-bar = mean_i h_i
+ *   q-bar_j = RoPE_t([W_Q c-bar]_j)   (pairs (2i, 2i+1), i < rope_dim/2, rotated by
+ *                                      t * rope_base^(-2i/rope_dim))
+ *   w-bar_j = sigmoid([W_G h-bar]_j)
+ * All pointers are device pointers to bf16 row-major arrays; weights in the [out, in] layout.
+ * Requires d_c and d_h multiples of 8; cq, h and w_g 16-byte aligned; H_S <= 64;
+ * rope_dim <= 512; T / G <= 65535. Tokens past the last complete group are ignored. Invalid
+ * arguments return ADX_EINVAL. The gate projection is taken from h-bar in fp32 inside the
+ * pooling kernel, as per-column-block partial sums added in a fixed order (deterministic).
+ * The projections run on cuBLAS (bf16 operands, fp32 accumulation) with one handle per device
+ * created on first use; calls on one device must not be issued from several host threads at
+ * the same time. */
+typedef struct {
+  const void* cq;      /* [T, d_c] query latents */
+  const void* h;       /* [T, d_h] normalized hidden states */
+  const void* w_pool;  /* [d_c, 3*d_c] */
+  const void* w_q;     /* [H_S*d, d_c] */
+  const void* w_g;     /* [H_S, d_h] */
+  int32_t T, d_c, d_h, H_S, d, rope_dim;  /* rope_dim even, <= d */
+  float rope_base;
+  int64_t q_pos0;      /* position of token 0 */
+} adx_group_indexer;
+
+/* Workspace bytes for adx_group_indexer_queries, 0 for invalid arguments. */
+size_t adx_group_indexer_workspace_size(const adx_group_indexer* gi, int32_t G);
+
+/* qbar_out [T/G, H_S, d] bf16 out, wbar_out [T/G, H_S] fp32 out (device). */
+adx_status adx_group_indexer_queries(const adx_group_indexer* gi, int32_t G, void* qbar_out,
+                                     float* wbar_out, void* ws, size_t ws_bytes, void* stream);
+
 /* Calibration statistic of layer-wise reuse (ADIndex §4.1, Eq. (4)): for every complete group
  * of G consecutive rows of topk_idx [T, K] (rows g*G .. g*G+G-1, g < T/G), the number of
  * distinct positions in [0, S) among the group's Top-K sets (-1 padding and other values

@@ -20,7 +20,8 @@ EXPORTS = ("adx_abi_version", "adx_bank_width", "adx_status_string", "adx_worksp
            "adx_read_device_status", "adx_set_timing_events", "adx_launch_count",
            "adx_index_prefill_noalloc", "adx_mtp_workspace_size", "adx_index_mtp",
            "adx_group_union_sizes", "adx_group_query_mean", "adx_index_prefill_host",
-           "adx_check_wait_timeout")
+           "adx_check_wait_timeout", "adx_group_indexer_workspace_size",
+           "adx_group_indexer_queries")
 
 
 class Operands(ctypes.Structure):
@@ -38,6 +39,24 @@ class Operands(ctypes.Structure):
         ("S", ctypes.c_int32),
         ("q_pos0", ctypes.c_int64),
         ("seq_len", ctypes.c_void_p),
+    ]
+
+
+class GroupIndexer(ctypes.Structure):
+    _fields_ = [
+        ("cq", ctypes.c_void_p),
+        ("h", ctypes.c_void_p),
+        ("w_pool", ctypes.c_void_p),
+        ("w_q", ctypes.c_void_p),
+        ("w_g", ctypes.c_void_p),
+        ("T", ctypes.c_int32),
+        ("d_c", ctypes.c_int32),
+        ("d_h", ctypes.c_int32),
+        ("H_S", ctypes.c_int32),
+        ("d", ctypes.c_int32),
+        ("rope_dim", ctypes.c_int32),
+        ("rope_base", ctypes.c_float),
+        ("q_pos0", ctypes.c_int64),
     ]
 
 
@@ -71,6 +90,9 @@ def _declare(lib):
         "adx_group_union_sizes": (ctypes.c_int, [VP, I32, I32, I32, I32, VP, VP]),
         "adx_index_prefill_host": (ctypes.c_int, [P, I32, I32, VP, VP, VP, SZ, VP]),
         "adx_check_wait_timeout": (ctypes.c_int, [VP, ctypes.c_uint64, VP]),
+        "adx_group_indexer_workspace_size": (SZ, [ctypes.POINTER(GroupIndexer), I32]),
+        "adx_group_indexer_queries": (ctypes.c_int, [ctypes.POINTER(GroupIndexer), I32, VP, VP,
+                                                     VP, SZ, VP]),
         "adx_group_query_mean": (ctypes.c_int, [I32, VP, VP, VP, I32, I32, I32, I32, I32, VP,
                                                 VP, VP]),
     }

@@ -538,6 +538,9 @@ size_t ws_mtp(const adx_operands* full, const adx_operands* gops, const MtpShape
 }
 
 }  // namespace
+
+void add_launches(int n) { g_launches += n; }
+
 }  // namespace adx
 
 using namespace adx;

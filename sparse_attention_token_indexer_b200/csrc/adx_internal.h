@@ -151,4 +151,7 @@ cudaError_t launch_prepare_q(const void* q, const float* q_scale, bool in_e4m3, 
                              const float* w, int64_t rows, int H, int d, void* q_out,
                              float* q_scale_out, int8_t* fold_flag, cudaStream_t s);
 
+// Adds n to the library's launch counter (kernels launched outside the API file).
+void add_launches(int n);
+
 }  // namespace adx

@@ -236,6 +236,29 @@ def group_query_mean(q, w, G, Hg, q_scale=None, stream=None):
     return qbar, wbar
 
 
+def group_indexer_queries(cq, h, w_pool, w_q, w_g, G, H_S, d, q_pos0=0, rope_dim=64,
+                          rope_base=10000.0, ws=None, stream=None):
+    """The group indexer of Eqs. (6)-(7): cq [T, d_c], h [T, d_h] and the weights (bf16, [out,
+    in]) -> (qbar [T // G, H_S, d] bf16, wbar [T // G, H_S] fp32)."""
+    for name, t in (("cq", cq), ("h", h), ("w_pool", w_pool), ("w_q", w_q), ("w_g", w_g)):
+        _dev(t, name, torch.bfloat16)
+    gi = L.GroupIndexer()
+    gi.cq, gi.h, gi.w_pool, gi.w_q, gi.w_g = (t.data_ptr() for t in (cq, h, w_pool, w_q, w_g))
+    gi.T, gi.d_c = cq.shape
+    gi.d_h = h.shape[1]
+    gi.H_S, gi.d, gi.rope_dim, gi.rope_base, gi.q_pos0 = H_S, d, rope_dim, rope_base, int(q_pos0)
+    need = L.lib().adx_group_indexer_workspace_size(ctypes.byref(gi), G)
+    if need == 0:
+        raise L.AdxError("adx_group_indexer_workspace_size", L.ADX_EINVAL)
+    buf = _ws(ws, cq.device).get(need)
+    ng = gi.T // G
+    qbar = torch.empty(ng, H_S, d, dtype=torch.bfloat16, device=cq.device)
+    wbar = torch.empty(ng, H_S, dtype=torch.float32, device=cq.device)
+    L.check("adx_group_indexer_queries", L.lib().adx_group_indexer_queries(
+        ctypes.byref(gi), G, _p(qbar), _p(wbar), _p(buf), buf.numel(), _stream(stream)))
+    return qbar, wbar
+
+
 def read_device_status(ws=None, device=None, stream=None):
     """Synchronises and returns (and clears) the device status of a workspace (0 = ok)."""
     w = _ws(ws, device or torch.device("cuda"))

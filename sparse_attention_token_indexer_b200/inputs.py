@@ -205,3 +205,18 @@ def decode_seq_len(prob, step):
     """Keys visible to each sequence at decode step ``step`` (int32 [Bs])."""
     return torch.full((prob["Bs"],), prob["S"] + step, dtype=torch.int32,
                       device=prob["k"].device)
+
+
+def group_indexer_problem(T, d_c=1536, d_h=7168, H_S=16, d=128, seed=4, device="cpu"):
+    """Inputs of the trained group indexer (query latents, normalized hidden states) with
+    synthetic weights: cq [T, d_c] and h [T, d_h] ~ N(0, 1) (post-normalization activations),
+    W_pool [d_c, 3 d_c], W_Q [H_S d, d_c] and W_G [H_S, d_h] ~ N(0, 1 / fan-in), all bf16."""
+    gen = _gen(seed, device)
+    bf = torch.bfloat16
+    return dict(
+        cq=_randn(gen, (T, d_c), device).to(bf),
+        h=_randn(gen, (T, d_h), device).to(bf),
+        w_pool=_randn(gen, (d_c, 3 * d_c), device, 1.0 / math.sqrt(3 * d_c)).to(bf),
+        w_q=_randn(gen, (H_S * d, d_c), device, 1.0 / math.sqrt(d_c)).to(bf),
+        w_g=_randn(gen, (H_S, d_h), device, 1.0 / math.sqrt(d_h)).to(bf),
+        H_S=H_S, d=d)

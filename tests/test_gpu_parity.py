@@ -506,6 +506,29 @@ def test_group_query_mean(dtype, G, Hg):
     assert np.allclose(wbar.cpu().double().numpy(), rw, rtol=1e-6, atol=0)
 
 
+@pytest.mark.parametrize("T,G,rope_dim,q_pos0,d_c,d_h,H_S", [
+    (16 * 4 + 3, 4, 64, 0, 192, 320, 4), (8 * 16 + 15, 16, 64, 100000, 192, 320, 4),
+    (5 * 64, 64, 0, 7, 192, 320, 4), (3 * 8, 8, 128, 262143, 192, 320, 4),
+    # two column blocks per group, the first holding latent and hidden-state columns
+    (6 * 16 + 5, 16, 64, 65536, 1536, 2048, 16)])
+def test_group_indexer_queries(T, G, rope_dim, q_pos0, d_c, d_h, H_S):
+    """Eqs. (6)-(7) on cuBLAS + the pooling and RoPE kernels against the oracle in fp64. The
+    path rounds the pooled mean, h-bar, c-bar and q-bar to bf16 (relative 2^-9 each), so a
+    head's error is a few 2^-9 of its rms plus q-bar's own rounding; the gates see h-bar's
+    rounding through a sigmoid of slope at most 1/4."""
+    p = inputs.group_indexer_problem(T, d_c=d_c, d_h=d_h, H_S=H_S, d=128, seed=28, device="cuda")
+    qbar, wbar = indexer.group_indexer_queries(p["cq"], p["h"], p["w_pool"], p["w_q"], p["w_g"],
+                                               G, H_S, 128, q_pos0=q_pos0, rope_dim=rope_dim)
+    cpu = {k: (v.double().cpu().numpy() if torch.is_tensor(v) else v) for k, v in p.items()}
+    rq, rw = ox.group_indexer_queries(cpu["cq"], cpu["h"], cpu["w_pool"], cpu["w_q"],
+                                      cpu["w_g"], G, H_S, 128, q_pos0=q_pos0, rope_dim=rope_dim)
+    got = f64(qbar)
+    assert got.shape == rq.shape == (T // G, H_S, 128)
+    rms = np.sqrt((rq ** 2).mean(axis=2, keepdims=True))
+    assert np.all(np.abs(got - rq) <= 2.0 ** -6 * rms + 2.0 ** -8 * np.abs(rq))
+    assert np.abs(wbar.cpu().double().numpy() - rw).max() <= 2.0 ** -8
+
+
 def test_group_mode_on_kernel_group_queries():
     """Group mode end to end with the group queries built by the library itself."""
     T, G, B, K, Hg = 64 * 12, 64, 256, 128, 16
