@@ -21,6 +21,11 @@ notes of the repository):
       "window" - scan s < a; bank = Top-(B-G) of the scan plus the group's own window
                  a..a+G-1 (total B); query i's candidates are the bank entries <= i.
                  Incomplete trailing groups use the plain indexer.
+  * HISA (the HISA paper's abstract; ADIndex Appendix C.5 for its settings): a block is
+    scored with Eq. (1) applied to its mean-pooled key (pooling keys, not token scores); the
+    query's own block is visible (its tokens up to the query's position); a trailing partial
+    block pools the keys it holds; the forced blocks take budget slots first and the other
+    slots follow the block scores with ties broken by ascending block number.
 """
 
 from dataclasses import dataclass
@@ -306,3 +311,63 @@ def group_indexer_queries(cq, h, w_pool, w_q, w_g, G, H_S, d, q_pos0=0, rope_dim
         z = np.asarray(w_g, np.float64) @ h[g * G:(g + 1) * G].mean(0)
         wbar[g] = 1.0 / (1.0 + np.exp(-z))
     return qbar, wbar
+
+
+# ---------------------------------------------------------------------------------------
+# HISA: block filter, then token refinement (the HISA paper's two-stage indexer, with the
+# reproduction settings of ADIndex Appendix C.5)
+# ---------------------------------------------------------------------------------------
+
+HISA_BLOCK = 128
+
+
+def hisa_block_keys(k, block=HISA_BLOCK):
+    """Mean-pooled block keys: kbar[b] = mean of k[b*block : (b+1)*block]; a trailing partial
+    block is the mean of the keys it holds (HISA abstract: pooled block representations;
+    ADIndex Appendix C.5: mean pooling of indexing keys over 128-token blocks)."""
+    k = np.asarray(k, np.float64)
+    nb = -(-k.shape[0] // block)
+    return np.stack([k[b * block:(b + 1) * block].mean(axis=0) for b in range(nb)]) \
+        if nb else np.zeros((0, k.shape[1]))
+
+
+def hisa_blocks_row(q_t, w_t, kbar, p, n_blocks, block=HISA_BLOCK):
+    """Candidate blocks of a query at position p (ADIndex Appendix C.5, HISA paragraph):
+    blocks 0 .. p // block are visible; when at most n_blocks are, all of them; otherwise the
+    first block and the query's own block, plus the n_blocks - (number forced) highest-scoring
+    other visible blocks, a block scored like a key with its pooled key (Eq. (1) with kbar_b).
+    Returns the block numbers, ascending."""
+    cur = int(p) // block
+    nvis = min(cur + 1, kbar.shape[0])
+    if nvis <= n_blocks:
+        return np.arange(nvis)
+    forced = sorted({0, cur})
+    rest = np.array([b for b in range(nvis) if b not in forced], dtype=np.int64)
+    chosen = topk(score_keys(q_t, w_t, kbar[rest]), n_blocks - len(forced), rest)
+    return np.sort(np.concatenate([np.array(forced, np.int64), chosen]))
+
+
+def hisa_candidates(blocks, p, S, block=HISA_BLOCK):
+    """Tokens of the chosen blocks visible to a query at position p (causal masking)."""
+    lim = min(int(p) + 1, S)
+    parts = [np.arange(b * block, min((b + 1) * block, lim)) for b in blocks]
+    return np.concatenate(parts) if parts else np.zeros(0, np.int64)
+
+
+def hisa_topk_row(q_t, w_t, k, kbar, p, K, n_blocks, block=HISA_BLOCK):
+    """One query: candidate blocks, then Top-K of their visible tokens rescored with all heads
+    (Eq. (1)); a query with at most K visible tokens keeps all of them."""
+    S = k.shape[0]
+    if int(p) + 1 <= K:
+        return np.arange(min(int(p) + 1, S))
+    cand = hisa_candidates(hisa_blocks_row(q_t, w_t, kbar, p, n_blocks, block), p, S, block)
+    return topk(score_keys(q_t, w_t, k[cand]), K, cand)
+
+
+def hisa_topk(q, w, k, pos, K, n_blocks=64, block=HISA_BLOCK, rows=None):
+    """HISA indexer: {row: Top-K positions} for the requested rows (all by default)."""
+    k = np.asarray(k, np.float64)
+    kbar = hisa_block_keys(k, block)
+    rows = range(q.shape[0]) if rows is None else rows
+    return {int(t): hisa_topk_row(q[t], w[t], k, kbar, pos[t], K, n_blocks, block)
+            for t in rows}

@@ -437,3 +437,86 @@ def test_group_indexer_pools_projects_and_gates():
     qn, _ = ox.group_indexer_queries(cq, h, np.hstack([eye, zero, zero]), wq, wg, G, HS, d,
                                      q_pos0=10, rope_dim=0)
     assert np.allclose(qb[1, 0], ox.rope(qn[1, 0], 14, 4))
+
+
+# ---------------------------------------------------------------------------------------
+# HISA (block filter + token refinement)
+# ---------------------------------------------------------------------------------------
+
+def test_hisa_block_keys_are_block_means():
+    k = np.arange(10, dtype=np.float64)[:, None] * np.array([[1.0, -2.0]])   # ramp rows
+    kbar = ox.hisa_block_keys(k, block=4)
+    # block b holds rows 4b..4b+3 (mean 4b + 1.5); the partial block holds rows 8, 9 (8.5)
+    assert np.allclose(kbar[:, 0], [1.5, 5.5, 8.5]) and np.allclose(kbar[:, 1], [-3, -11, -17])
+
+
+def test_hisa_scores_pooled_keys_not_pooled_scores():
+    """Block 1 holds +v and -v (pooled key 0: block score 0, although the mean of its token
+    scores is 1.5); block 2 holds 0.5 v twice (block score 0.5). With one free slot the filter
+    must take block 2."""
+    k = np.zeros((12, 2))
+    k[2], k[3] = [3.0, 0], [-3.0, 0]
+    k[4], k[5] = [0.5, 0], [0.5, 0]
+    q, w = np.array([[1.0, 0.0]]), np.array([1.0])
+    kbar = ox.hisa_block_keys(k, block=2)
+    assert list(ox.hisa_blocks_row(q, w, kbar, 11, n_blocks=3, block=2)) == [0, 2, 5]
+    # the refined candidates are the tokens of those blocks up to the query's position
+    assert list(ox.hisa_candidates([0, 2, 5], 10, 12, block=2)) == [0, 1, 4, 5, 10]
+
+
+def test_hisa_forces_first_and_own_block():
+    """Blocks 0 and the query's own block score lowest yet are kept and count toward the
+    budget; the other slots go to the best-scoring blocks."""
+    d, block = 3, 2
+    scores = [-5.0, 4.0, 1.0, 3.0, 2.0, -6.0]       # desired block score of each block
+    k = np.zeros((12, d))
+    for b, s in enumerate(scores):
+        k[2 * b:2 * b + 2, 0] = s
+    q, w = np.array([[1.0, 0.0, 0.0]]), np.array([1.0])
+    kbar = ox.hisa_block_keys(k, block)
+    assert list(ox.hisa_blocks_row(q, w, kbar, 10, n_blocks=4, block=block)) == [0, 1, 3, 5]
+    # query in block 0: only one forced block; all visible when they fit
+    assert list(ox.hisa_blocks_row(q, w, kbar, 1, n_blocks=4, block=block)) == [0]
+    assert list(ox.hisa_blocks_row(q, w, kbar, 7, n_blocks=4, block=block)) == [0, 1, 2, 3]
+
+
+def test_hisa_equals_flat_indexer_when_every_block_fits():
+    rng = np.random.default_rng(45)
+    T, S, H, d = 24, 24, 3, 5
+    q, w, k = rng.standard_normal((T, H, d)), rng.random((T, H)), rng.standard_normal((S, d))
+    pos = np.arange(T)
+    got = ox.hisa_topk(q, w, k, pos, K=5, n_blocks=6, block=4)
+    want = ox.flat_topk(q, w, k, pos, K=5)
+    for t in range(T):
+        assert set(got[t]) == set(want[t])
+
+
+def test_hisa_matches_brute_force_subsets():
+    """Top-m of distinct scores is the m-subset with the largest sum: brute force over all
+    block subsets (forced blocks included) and then over all K-subsets of the candidates."""
+    rng = np.random.default_rng(46)
+    H, d, block, n_blocks, K = 2, 3, 3, 4, 4
+    S = 7 * block
+    k = rng.standard_normal((S, d))
+    for trial in range(6):
+        q, w = rng.standard_normal((H, d)), rng.random(H)
+        p = int(rng.integers(5 * block, S))
+        cur, nb = p // block, p // block + 1
+        kbar = np.stack([k[b * block:(b + 1) * block].mean(0) for b in range(nb)])
+        bs = [sum(w[j] * max(0.0, q[j] @ kbar[b]) for j in range(H)) for b in range(nb)]
+        others = [b for b in range(nb) if b not in (0, cur)]
+        best = max(itertools.combinations(others, n_blocks - 2), key=lambda c: sum(bs[b] for b in c))
+        blocks = sorted(set(best) | {0, cur})
+        assert list(ox.hisa_blocks_row(q, w, ox.hisa_block_keys(k, block), p, n_blocks,
+                                       block)) == blocks
+        cand = [s for b in blocks for s in range(b * block, (b + 1) * block) if s <= p]
+        ts = {s: sum(w[j] * max(0.0, q[j] @ k[s]) for j in range(H)) for s in cand}
+        top = max(itertools.combinations(cand, K), key=lambda c: sum(ts[s] for s in c))
+        got = ox.hisa_topk(q[None], w[None], k, [p], K, n_blocks, block)[0]
+        assert set(got) == set(top)
+
+
+def test_hisa_short_prefix_keeps_every_token():
+    rng = np.random.default_rng(47)
+    q, w, k = rng.standard_normal((1, 2, 3)), rng.random((1, 2)), rng.standard_normal((40, 3))
+    assert list(ox.hisa_topk(q, w, k, [9], K=10, n_blocks=2, block=4)[0]) == list(range(10))
