@@ -40,8 +40,10 @@ DECODE = dict(Bs=32, S=131072, H=64, d=128, K=2048, Hg=16, B=8192, G=16, seed=3)
 CHUNKED = dict(S=262144, chunk=4096, H=64, d=128, K=2048, G=64, B=8192, Hg=16, seed=4)
 # rows per chunk of the host-buffer path (copies of one chunk overlap the work on another)
 E2E_ROWS_PER_CHUNK = 1024
-# MTP target verification on the decode caches: one window of m draft tokens per sequence
+# HISA at the 64K context of the HISA paper's kernel benchmarks: 128-key blocks, 64 kept
+HISA = dict(T=65536, H=64, d=128, K=2048, n_blocks=64, seed=13)
 GROUP_INDEXER = dict(T=65536, G=64, d_c=1536, d_h=7168, H_S=16, d=128, seed=12)
+# MTP target verification on the decode caches: one window of m draft tokens per sequence
 MTP = dict(m=16, G=8, P=8192)
 
 
@@ -414,6 +416,62 @@ def run_calibration(args, dist):
     return dict(ms=ms, launches=launches, bytes=3 * idx.numel() * 4)
 
 
+def run_hisa(args, dist, with_flat=True):
+    """HISA prefill over 65536 tokens (block keys, block filter, token refinement), and the
+    flat indexer on the same inputs."""
+    from sparse_attention_token_indexer_b200 import _lib, indexer, inputs
+    c = HISA
+    p = inputs.anchor_prefill(c["T"], c["H"], c["d"], c["K"], seed=c["seed"], device="cuda")
+    ws = indexer.Workspace("cuda")
+    steps = max(2, args.steps // 2)
+
+    def step():
+        kbar, _ = indexer.hisa_block_keys(p["q"], p["w"], p["k"])
+        indexer.index_hisa(p["q"], p["w"], p["k"], kbar, c["K"], n_blocks=c["n_blocks"], ws=ws)
+
+    th = StageTimer(_lib.lib(), steps)
+    ms, launches = timed(step, steps, args.warmup, dist, th)
+    # the library's events mark its last score and select launches: the token refinement
+    stages = {"refine_score_ms": statistics.mean(th.ms(0, 1)),
+              "final_select_ms": statistics.mean(th.ms(2, 3))}
+    T, nbk, B = c["T"], c["n_blocks"], 128
+    blk_pairs = sum(t // B + 1 for t in range(T))
+    tok_pairs = sum(min(nbk, t // B + 1) * B for t in range(T))
+    out = dict(ms=ms, launches=launches, stages=stages, blk_pairs=blk_pairs, tok_pairs=tok_pairs,
+               flops=2 * c["H"] * c["d"] * (blk_pairs + tok_pairs), rows=T)
+    if with_flat:
+        def flat():
+            indexer.index_prefill(p["q"], p["w"], p["k"], c["K"], ws=ws)
+        out["ms_flat"], _ = timed(flat, max(2, steps // 2), args.warmup, dist)
+    return out
+
+
+def run_hisa_decode(args, dist):
+    """HISA decode step for 32 sequences of 131072 e4m3 keys: the last block key of every
+    cache refreshed, the block filter, the token refinement (the block keys of the rest of
+    the cache are built once, like the cache itself)."""
+    from sparse_attention_token_indexer_b200 import indexer, inputs
+    c = DECODE
+    prob = inputs.decode_problem(c["Bs"], c["S"], c["H"], c["d"], c["K"], c["Hg"], steps=1,
+                                 seed=c["seed"], device="cuda")
+    ws = indexer.Workspace("cuda")
+    seq0 = inputs.decode_seq_len(prob, 0)
+    q0, w0, k, ks = prob["q_steps"][0], prob["w_steps"][0], prob["k"], prob["k_scale"]
+    kbar, kbs = indexer.hisa_block_keys(q0, w0, k, k_scale=ks, seq_len=seq0)
+
+    def step():
+        indexer.hisa_block_keys(q0, w0, k, k_scale=ks, seq_len=seq0, last_only=True,
+                                out=(kbar, kbs))
+        indexer.index_hisa(q0, w0, k, kbar, c["K"], n_blocks=HISA["n_blocks"], k_scale=ks,
+                           kbar_scale=kbs, seq_len=seq0, ws=ws)
+
+    ms, launches = timed(step, args.steps, args.warmup, dist)
+    nb = (c["S"] + 127) // 128
+    key_bytes = c["d"] + 4
+    bytes_step = c["Bs"] * (HISA["n_blocks"] * 128 + nb + 128) * key_bytes
+    return dict(ms=ms, launches=launches, bytes=bytes_step)
+
+
 def run_group_indexer(args, dist):
     """The trained group indexer's queries and gates (Eqs. (6)-(7)) for a 65536-token prefill
     with G = 64: d_c = 1536 query latents, d_h = 7168 hidden states, H_S = 16 heads of d = 128,
@@ -528,9 +586,11 @@ def main():
     ap.add_argument("--rows", action="store_true", help="also time the other hot-path rows")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--case", default="flat", choices=["flat", "flat_small", "decode", "mtp",
-                                                      "group_indexer"],
+                                                      "group_indexer", "hisa", "hisa_small",
+                                                      "hisa_decode"],
                     help="flat_small: T = 8192, for profiler captures; decode, mtp, "
-                         "group_indexer: that workload alone (with --quick)")
+                         "group_indexer, hisa, hisa_decode: that workload alone (with "
+                         "--quick); hisa_small: HISA prefill at T = 16384")
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "e4m3"])
     ap.add_argument("--quick", action="store_true",
                     help="time the kernels only (no e2e, rows or CPU baseline): for profiling")
@@ -596,6 +656,23 @@ def main():
                               "flat_ms_per_round": mt["ms_flat"],
                               "speedup_vs_flat": mt["ms_flat"] / mt["ms"],
                               "gpu_launches": mt["launches"]}), flush=True)
+        dist.close()
+        return
+    if args.case in ("hisa", "hisa_small") and args.quick:
+        if args.case == "hisa_small":
+            HISA["T"] = 16384
+        hs = run_hisa(args, dist, with_flat=False)
+        if dist.rank == 0:
+            print(json.dumps({"case": args.case, "T": HISA["T"], "ms_per_step": hs["ms"],
+                              "stage_ms": hs["stages"], "gpu_launches": hs["launches"]}),
+                  flush=True)
+        dist.close()
+        return
+    if args.case == "hisa_decode" and args.quick:
+        hd = run_hisa_decode(args, dist)
+        if dist.rank == 0:
+            print(json.dumps({"case": "hisa_decode", "ms_per_step": hd["ms"],
+                              "gpu_launches": hd["launches"]}), flush=True)
         dist.close()
         return
     if args.case == "group_indexer" and args.quick:
@@ -690,6 +767,22 @@ def main():
             "gbs_read": cb["bytes"] / (cb["ms"] * 1e-3) / 1e9,
             "hbm_frac": cb["bytes"] / (cb["ms"] * 1e-3) / 1e9 / pk["hbm"],
             "gpu_launches": cb["launches"]}
+        hs = run_hisa(args, dist)
+        rows["hisa_prefill_T65536_nb64"] = {
+            "ms_per_step": hs["ms"], "flat_ms_per_step": hs["ms_flat"],
+            "speedup_vs_flat": hs["ms_flat"] / hs["ms"],
+            "scores_per_s": (hs["blk_pairs"] + hs["tok_pairs"]) / (hs["ms"] * 1e-3),
+            "topk_queries_per_s": hs["rows"] / (hs["ms"] * 1e-3),
+            "tflops": hs["flops"] / (hs["ms"] * 1e-3) / 1e12, "stage_ms": hs["stages"],
+            "refine_score_tflops": 2 * HISA["H"] * HISA["d"] * hs["tok_pairs"]
+            / (hs["stages"]["refine_score_ms"] * 1e-3) / 1e12,
+            "gpu_launches": hs["launches"]}
+        hd = run_hisa_decode(args, dist)
+        rows["hisa_decode_Bs32_S131072_e4m3_nb64"] = {
+            "ms_per_step": hd["ms"], "flat_ms_per_step": dcd["ms_flat"],
+            "speedup_vs_flat": dcd["ms_flat"] / hd["ms"],
+            "topk_queries_per_s": DECODE["Bs"] / (hd["ms"] * 1e-3),
+            "hbm_gbs": hd["bytes"] / (hd["ms"] * 1e-3) / 1e9, "gpu_launches": hd["launches"]}
         gi = run_group_indexer(args, dist)
         rows["group_indexer_queries_T65536_G64"] = {
             "ms_per_step": gi["ms"], "groups_per_s": gi["groups"] / (gi["ms"] * 1e-3),

@@ -142,6 +142,40 @@ adx_status adx_index_prefill_host(const adx_operands* ops, int32_t K, int32_t ro
 adx_status adx_index_decode(const adx_operands* ops, int32_t K, int32_t* topk_idx,
                             float* topk_score, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- HISA: block filter, then token refinement -----------------------------------------
+ * The hierarchical indexer of "HISA: Efficient Hierarchical Indexing for Fine-Grained Sparse
+ * Attention" (arXiv 2603.28458v3, abstract) with the settings of ADIndex Appendix C.5:
+ * keys are pooled into blocks of ADX_HISA_BLOCK consecutive positions by their mean; a query
+ * at position p sees blocks 0 .. p / ADX_HISA_BLOCK; when more than n_blocks are visible it
+ * keeps block 0, its own block and the n_blocks - 2 best other blocks by Eq. (1) on the
+ * block keys (all visible blocks otherwise); the visible tokens of the kept blocks are then
+ * scored with Eq. (1) and the Top-K of them returned (all of them when at most K).
+ * Both layouts of adx_operands apply: prefill (one key range of S keys, rows at q_pos0 + r)
+ * and decode (row r = sequence r at position seq_len[r] - 1, its own S-row cache). */
+#define ADX_HISA_BLOCK 128
+
+/* Block keys kbar [n_seq, ceil(S / 128), d] in the key format (bf16; or e4m3 codes with
+ * per-block scales kbar_scale [n_seq, ceil(S / 128)], scale = amax / 448, 1 for a zero block),
+ * n_seq = 1 (prefill) or T (decode). A trailing partial block is the mean of the keys it
+ * holds. Prefill: the blocks of the first min(S, q_pos0 + T) keys. Decode: the blocks of the
+ * first seq_len[r] keys of each cache; last_only != 0 recomputes only the block holding each
+ * sequence's last key (the one a decode step's appended key changes). Device pointers. */
+adx_status adx_hisa_block_keys(const adx_operands* ops, int32_t last_only, void* kbar,
+                               float* kbar_scale, void* stream);
+
+/* Workspace bytes for adx_index_hisa (blocks_external: a blocks_out array is given), 0 when
+ * the arguments are invalid. */
+size_t adx_hisa_workspace_size(const adx_operands* ops, int32_t n_blocks, int32_t K,
+                               int32_t blocks_external);
+
+/* HISA indexer step. kbar / kbar_scale from adx_hisa_block_keys (read only). Requires
+ * 2 <= n_blocks, K <= n_blocks * 128, T * n_blocks * 128 < 2^31.
+ * topk_idx [T, K] int32 out: key positions (within the row's key range), -1 padded;
+ * topk_score [T, K] or NULL; blocks_out [T, n_blocks] or NULL: the kept blocks, -1 padded. */
+adx_status adx_index_hisa(const adx_operands* ops, const void* kbar, const float* kbar_scale,
+                          int32_t n_blocks, int32_t K, int32_t* topk_idx, float* topk_score,
+                          int32_t* blocks_out, void* ws, size_t ws_bytes, void* stream);
+
 /* Shared token banks (ADIndex §4.3, Eq. (13)); `grp` holds the group queries: q = q-bar
  * [Ng, H_g, d], w = w-bar [Ng, H_g], with Ng = grp->T.
  *  prefill layout: group g has members at positions q_pos0 + g*G .. q_pos0 + g*G + G-1.

@@ -12,6 +12,7 @@ ADX_OK, ADX_EINVAL, ADX_EUNSUPPORTED, ADX_EWORKSPACE, ADX_ECUDA, ADX_EOVERFLOW, 
 ADX_BF16, ADX_E4M3 = 0, 1
 ADX_BANK_PAPER, ADX_BANK_WINDOW = 0, 1
 ADX_OP_PREFILL, ADX_OP_DECODE, ADX_OP_GROUP_BANK, ADX_OP_BANK_REFINE, ADX_OP_PREFILL_HOST = range(5)
+ADX_HISA_BLOCK = 128
 ADX_STATUS_BYTES = 256
 
 # every extern "C" symbol include/adx.h declares
@@ -21,7 +22,8 @@ EXPORTS = ("adx_abi_version", "adx_bank_width", "adx_status_string", "adx_worksp
            "adx_index_prefill_noalloc", "adx_mtp_workspace_size", "adx_index_mtp",
            "adx_group_union_sizes", "adx_group_query_mean", "adx_index_prefill_host",
            "adx_check_wait_timeout", "adx_group_indexer_workspace_size",
-           "adx_group_indexer_queries")
+           "adx_group_indexer_queries", "adx_hisa_block_keys", "adx_hisa_workspace_size",
+           "adx_index_hisa")
 
 
 class Operands(ctypes.Structure):
@@ -90,6 +92,9 @@ def _declare(lib):
         "adx_group_union_sizes": (ctypes.c_int, [VP, I32, I32, I32, I32, VP, VP]),
         "adx_index_prefill_host": (ctypes.c_int, [P, I32, I32, VP, VP, VP, SZ, VP]),
         "adx_check_wait_timeout": (ctypes.c_int, [VP, ctypes.c_uint64, VP]),
+        "adx_hisa_block_keys": (ctypes.c_int, [P, I32, VP, VP, VP]),
+        "adx_hisa_workspace_size": (SZ, [P, I32, I32, I32]),
+        "adx_index_hisa": (ctypes.c_int, [P, VP, VP, I32, I32, VP, VP, VP, VP, SZ, VP]),
         "adx_group_indexer_workspace_size": (SZ, [ctypes.POINTER(GroupIndexer), I32]),
         "adx_group_indexer_queries": (ctypes.c_int, [ctypes.POINTER(GroupIndexer), I32, VP, VP,
                                                      VP, SZ, VP]),

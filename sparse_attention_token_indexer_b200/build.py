@@ -16,7 +16,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libadx.so")
 SOURCES = ["adx_api.cu", "score_sm100.cu", "select_topk.cu", "aux_kernels.cu", "adx_noalloc.cu",
-           "group_indexer.cu"]
+           "group_indexer.cu", "hisa.cu"]
 HEADERS = ["adx_internal.h", "sm100_ptx.cuh"]
 
 

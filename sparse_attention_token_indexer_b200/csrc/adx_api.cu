@@ -537,6 +537,33 @@ size_t ws_mtp(const adx_operands* full, const adx_operands* gops, const MtpShape
   return b;
 }
 
+// ---- HISA (block filter, then token refinement) ------------------------------------
+constexpr int kHisaShift = 7;  // log2 of the block size (one MMA tile of keys)
+static_assert((1 << kHisaShift) == kTileM, "a HISA block is one key tile");
+
+int64_t hisa_nbmax(const adx_operands* o) { return (o->S + kTileM - 1) / kTileM; }
+
+adx_status hisa_check(const adx_operands* o, int32_t n_blocks, int32_t K) {
+  const adx_status r = check_operands(o, o != nullptr && o->seq_len != nullptr);
+  if (r != ADX_OK) return r;
+  if (n_blocks < 2 || K <= 0 || static_cast<int64_t>(n_blocks) * kTileM > (1ll << 24) ||
+      K > n_blocks * kTileM)
+    return ADX_EINVAL;
+  if (static_cast<int64_t>(o->T) * n_blocks * kTileM > INT32_MAX) return ADX_EINVAL;
+  return ADX_OK;
+}
+
+size_t ws_hisa(const adx_operands* o, int32_t n_blocks, int32_t K, bool blocks_external) {
+  const int64_t T = o->T, nbmax = hisa_nbmax(o), nc = static_cast<int64_t>(n_blocks) * kTileM;
+  size_t b = kStatusBytes + ws_prepare(o, T);
+  b += align_up(static_cast<size_t>(T) * 4, kAlign);                         // row blocks
+  b += align_up(static_cast<size_t>(T) * ld_for(nbmax) * 4, kAlign);         // block scores
+  if (!blocks_external) b += align_up(static_cast<size_t>(T) * n_blocks * 4, kAlign);
+  b += align_up(static_cast<size_t>(T) * nc * 4, kAlign);                    // token scores
+  b += select_scratch_bytes(T, nbmax, n_blocks) + select_scratch_bytes(T, nc, K);
+  return b;
+}
+
 }  // namespace
 
 void add_launches(int n) { g_launches += n; }
@@ -1047,6 +1074,141 @@ adx_status adx_read_device_status(void* ws, void* stream) {
   if (cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return ADX_ECUDA;
   if (cudaMemset(ws, 0, sizeof(h)) != cudaSuccess) return ADX_ECUDA;
   return static_cast<adx_status>(h.code);
+}
+
+size_t adx_hisa_workspace_size(const adx_operands* o, int32_t n_blocks, int32_t K,
+                               int32_t blocks_external) {
+  if (hisa_check(o, n_blocks, K) != ADX_OK) return 0;
+  return ws_hisa(o, n_blocks, K, blocks_external != 0);
+}
+
+adx_status adx_hisa_block_keys(const adx_operands* o, int32_t last_only, void* kbar,
+                               float* kbar_scale, void* stream) {
+  const bool decode = o != nullptr && o->seq_len != nullptr;
+  adx_status r = check_operands(o, decode);
+  if (r != ADX_OK) return r;
+  if (!kbar || (fp8_keys(o) != (kbar_scale != nullptr))) return ADX_EINVAL;
+  const int64_t len = decode ? 0 : std::min<int64_t>(o->S, o->q_pos0 + o->T);
+  const cudaError_t e = counted(launch_block_keys(
+      o->k, o->k_scale, fp8_keys(o), o->S, o->d, decode ? o->T : 1, o->seq_len,
+      static_cast<int32_t>(len), last_only != 0, static_cast<int32_t>(hisa_nbmax(o)), kbar,
+      kbar_scale, static_cast<cudaStream_t>(stream)));
+  if (e == cudaErrorInvalidValue) return ADX_EUNSUPPORTED;
+  return e == cudaSuccess ? ADX_OK : ADX_ECUDA;
+}
+
+adx_status adx_index_hisa(const adx_operands* o, const void* kbar, const float* kbar_scale,
+                          int32_t n_blocks, int32_t K, int32_t* topk_idx, float* topk_score,
+                          int32_t* blocks_out, void* ws, size_t ws_bytes, void* stream) {
+  adx_status r = hisa_check(o, n_blocks, K);
+  if (r != ADX_OK) return r;
+  if (!kbar || (fp8_keys(o) != (kbar_scale != nullptr)) || !topk_idx || !ws) return ADX_EINVAL;
+  if (ws_bytes < ws_hisa(o, n_blocks, K, blocks_out != nullptr)) return ADX_EWORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool decode = o->seq_len != nullptr;
+  const int32_t T = o->T;
+  const int64_t nbmax = hisa_nbmax(o), ldb = ld_for(nbmax);
+  const int32_t nc = n_blocks * kTileM;
+  Carve cv(ws);
+  DeviceStatus* st = cv.take<DeviceStatus>(kStatusBytes);
+  Prepared pq;
+  if ((r = prepare(o, o->q, o->q_scale, o->w, T, cv, s, pq)) != ADX_OK) return r;
+  int32_t* row_blk = cv.take<int32_t>(static_cast<size_t>(T) * 4);
+  float* bsc = cv.take<float>(static_cast<size_t>(T) * ldb * 4);
+  int32_t* blocks =
+      blocks_out ? blocks_out : cv.take<int32_t>(static_cast<size_t>(T) * n_blocks * 4);
+  float* tsc = cv.take<float>(static_cast<size_t>(T) * nc * 4);
+  if (counted(launch_row_blocks(T, o->q_pos0, o->seq_len, row_blk, s)) != cudaSuccess)
+    return ADX_ECUDA;
+
+  // 1. block scores: Eq. (1) on the block keys, block b visible to a row whose position lies
+  //    in block >= b
+  {
+    ScorePlan p = decode ? rowwise_plan(o, pq, bsc, ldb)
+                         : base_plan(o, pq, score_tokens_per_tile(o->H));
+    ScoreArgs& a = p.a;
+    a.k_scale = kbar_scale;
+    a.row_pos = row_blk;
+    a.status = st;
+    a.scores = bsc;
+    a.score_ld = ldb;
+    a.R = T;
+    a.keys_per_batch = static_cast<int32_t>(nbmax);
+    if (decode) {
+      a.key_batch_stride = nbmax;
+    } else {
+      a.rows_per_batch = T;
+      a.n_batches = 1;
+      a.row_blocks_per_batch = (T + p.tok - 1) / p.tok;
+      a.reverse_order = 1;
+    }
+    const int64_t vis_blocks =
+        decode ? nbmax : (std::min<int64_t>(o->S, o->q_pos0 + T) + kTileM - 1) / kTileM;
+    finish_plan(p, (vis_blocks + kTileM - 1) / kTileM);
+    if ((r = run_score(p, pq.q, kbar, (decode ? T : 1) * nbmax, s)) != ADX_OK) return r;
+  }
+  // 2. forced blocks, then the block Top-n
+  if (counted(launch_force_blocks(bsc, ldb, T, row_blk, n_blocks, s)) != cudaSuccess)
+    return ADX_ECUDA;
+  {
+    SelectArgs sa{};
+    sa.vals = bsc;
+    sa.ld = ldb;
+    sa.rows_per_batch = 1;
+    sa.len_mode = 3;
+    sa.row_pos = row_blk;
+    sa.len_cap = static_cast<int32_t>(nbmax);
+    sa.K = n_blocks;
+    sa.out_idx = blocks;
+    sa.out_ld = n_blocks;
+    sa.rows = T;
+    if ((r = run_select(sa, nbmax, cv, st, s)) != ADX_OK) return r;
+  }
+  // 3. token refinement: every row scores the key tiles of its own blocks
+  {
+    ScorePlan p = decode ? rowwise_plan(o, pq, tsc, nc) : base_plan(o, pq, 1);
+    ScoreArgs& a = p.a;
+    a.key_blk = blocks;
+    a.key_blk_stride = n_blocks;
+    a.S_valid = o->S;
+    a.keys_per_batch = nc;
+    a.status = st;
+    if (!decode) {
+      a.scores = tsc;
+      a.score_ld = nc;
+      a.pos_base = o->q_pos0;
+      a.pos_step = 1;
+      a.R = T;
+      a.rows_per_batch = 1;
+      a.n_batches = T;
+      a.key_batch_div = T;
+      a.key_batch_stride = 0;
+      a.row_blocks_per_batch = 1;
+      a.reverse_order = 1;
+    }
+    finish_plan(p, n_blocks);
+    if ((r = run_score(p, pq.q, o->k, decode ? static_cast<int64_t>(T) * o->S : o->S, s)) !=
+        ADX_OK)
+      return r;
+  }
+  // 4. final Top-K over the candidate slots, mapped to key positions through the block list
+  SelectArgs sa{};
+  sa.vals = tsc;
+  sa.ld = nc;
+  sa.rows_per_batch = 1;
+  sa.idx_map = blocks;
+  sa.map_stride = n_blocks;
+  sa.map_shift = kHisaShift;
+  sa.len_mode = 3;
+  sa.row_pos = row_blk;
+  sa.len_mul = kTileM;
+  sa.len_cap = nc;
+  sa.K = K;
+  sa.out_idx = topk_idx;
+  sa.out_val = topk_score;
+  sa.out_ld = K;
+  sa.rows = T;
+  return run_select(sa, nc, cv, st, s);
 }
 
 }  // extern "C"

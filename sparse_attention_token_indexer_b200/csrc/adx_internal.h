@@ -42,6 +42,12 @@ struct ScoreArgs {
   int64_t key_idx_stride;
   int32_t n_idx;
   int32_t S_valid;
+  // Key blocks (one row per key batch, contiguous key rows): tile t of batch b is the 128 key
+  // rows starting at 128 * key_blk[b * key_blk_stride + t] of the batch's key range; a
+  // negative entry is no tile, and rows at or past S_valid are no key. A row block then
+  // scores min(keys_per_batch / 128, row position / 128 + 1) tiles. Null: contiguous tiles.
+  const int32_t* key_blk;
+  int64_t key_blk_stride;
   const int32_t* seq_len;  // [n_batches] or null
   const int32_t* row_pos;  // [R] or null
   const int8_t* fold_flag; // [R]: 1 = the row's queries carry its gates already; null = none do
@@ -78,7 +84,7 @@ struct SelectArgs {
   int32_t rows_per_batch;
   // row length: len_mode 0 -> fixed len_fixed; 1 -> min(len_cap, pos_base + r*pos_step + 1);
   //             2 -> min(len_cap, seq_len[r / rows_per_batch]);
-  //             3 -> min(len_cap, row_pos[r] + 1 + len_off)
+  //             3 -> min(len_cap, (row_pos[r] + 1 + len_off) * max(1, len_mul))
   int32_t len_mode;
   int32_t len_fixed;
   int32_t len_cap;
@@ -87,6 +93,10 @@ struct SelectArgs {
   const int32_t* seq_len;
   const int32_t* row_pos;
   int32_t len_off;
+  int32_t len_mul;
+  // with idx_map: 0 -> element c maps to map[c]; s > 0 -> to (map[c >> s] << s) + (c & (2^s - 1))
+  // (the map lists blocks of 2^s consecutive positions)
+  int32_t map_shift;
   int32_t K;
   int32_t n_seg;           // split each row into n_seg segments of seg_len (first stage)
   int32_t seg_len;
@@ -150,6 +160,22 @@ int score_blocks_per_sm(bool fp8, int H, int d, int tok);
 cudaError_t launch_prepare_q(const void* q, const float* q_scale, bool in_e4m3, bool out_e4m3,
                              const float* w, int64_t rows, int H, int d, void* q_out,
                              float* q_scale_out, int8_t* fold_flag, cudaStream_t s);
+
+// HISA block keys: the mean of each 128-key block of each key range (n_seq ranges of S rows;
+// length seq_len[b], or len_fixed without seq_len), stored like keys in kbar [n_seq, nbmax, d]
+// (e4m3 with per-block scales kbar_scale [n_seq, nbmax]); last_only: just the block holding
+// each range's last key.
+cudaError_t launch_block_keys(const void* k, const float* k_scale, bool fp8, int64_t S, int d,
+                              int32_t n_seq, const int32_t* seq_len, int32_t len_fixed,
+                              bool last_only, int32_t nbmax, void* kbar, float* kbar_scale,
+                              cudaStream_t s);
+// row_blk[r] = block of row r's position (q_pos0 + r, or seq_len[r] - 1 when seq_len is set).
+cudaError_t launch_row_blocks(int32_t R, int64_t q_pos0, const int32_t* seq_len, int32_t* row_blk,
+                              cudaStream_t s);
+// Raises the scores of block 0 and of the row's own block to +inf on rows that see more than
+// n_blocks blocks.
+cudaError_t launch_force_blocks(float* scores, int64_t ld, int32_t R, const int32_t* row_blk,
+                                int32_t n_blocks, cudaStream_t s);
 
 // Adds n to the library's launch counter (kernels launched outside the API file).
 void add_launches(int n);

@@ -1,0 +1,140 @@
+// Kernels of the hierarchical (block, then token) indexer of "HISA: Efficient Hierarchical
+// Indexing for Fine-Grained Sparse Attention" (arXiv 2603.28458v3), with the settings the
+// ADIndex paper uses for it (Appendix C.5): 128-key blocks pooled by their mean, the first
+// block and the query's own block always among the candidates.
+//   * block keys: the mean of each block of 128 keys (decoded with their scales for e4m3),
+//     stored like keys (bf16, or e4m3 with a per-block scale amax / 448);
+//   * row blocks: the block holding each query row's position;
+//   * forcing: the two forced blocks' scores raised to +inf ahead of the block Top-n.
+// The block scores, both selections and the token refinement run on the scoring and select
+// kernels (the refinement in their block-list mode).
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "adx_internal.h"
+
+namespace adx {
+namespace {
+
+constexpr int kBlk = kTileM;  // keys per block: one MMA tile
+constexpr int kBkThreads = 256;
+
+// One CTA per (block, key range). Threads are (row group, column); row group g sums the rows
+// g, g + RG, ... of the block in fp32, then the groups are added in shared memory.
+template <bool FP8>
+__global__ void __launch_bounds__(kBkThreads)
+block_keys_kernel(const uint8_t* __restrict__ k, const float* __restrict__ k_scale, int64_t S,
+                  int d, const int32_t* __restrict__ seq_len, int32_t len_fixed, int last_only,
+                  int nbmax, uint8_t* __restrict__ kbar, float* __restrict__ kbar_scale) {
+  __shared__ float part[kBkThreads];
+  __shared__ float red[kBkThreads / 32];
+  const int64_t b = blockIdx.y;
+  int64_t len = seq_len != nullptr ? seq_len[b] : len_fixed;
+  len = len < S ? len : S;
+  if (len <= 0) return;
+  const int64_t blk = last_only ? (len - 1) / kBlk : blockIdx.x;
+  const int64_t r0 = blk * kBlk;
+  if (r0 >= len || blk >= nbmax) return;
+  const int n = static_cast<int>(len - r0 < kBlk ? len - r0 : kBlk);
+  const int RG = kBkThreads / d;  // d divides kBkThreads (d = 64 or 128)
+  const int g = threadIdx.x / d, e = threadIdx.x % d;
+  const int64_t row0 = b * S + r0;
+  float acc = 0.f;
+  for (int i = g; i < n; i += RG) {
+    const int64_t row = row0 + i;
+    if constexpr (FP8) {
+      const __nv_fp8_e4m3 c = reinterpret_cast<const __nv_fp8_e4m3*>(k)[row * d + e];
+      acc += static_cast<float>(c) * k_scale[row];
+    } else {
+      acc += __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(k)[row * d + e]);
+    }
+  }
+  part[threadIdx.x] = acc;
+  __syncthreads();
+  float mean = 0.f;
+  if (threadIdx.x < d) {
+    float s = 0.f;
+    for (int gg = 0; gg < RG; ++gg) s += part[gg * d + threadIdx.x];
+    mean = s / static_cast<float>(n);
+  }
+  const int64_t out = b * nbmax + blk;
+  if constexpr (FP8) {
+    // per-block scale amax / 448 (1 for an all-zero block), like the key rows
+    float m = threadIdx.x < d ? fabsf(mean) : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    float amax = 0.f;
+    for (int w = 0; w < kBkThreads / 32; ++w) amax = fmaxf(amax, red[w]);
+    const float sc = amax > 0.f ? amax / 448.f : 1.f;
+    if (threadIdx.x < d)
+      kbar[out * d + threadIdx.x] = __nv_cvt_float_to_fp8(mean / sc, __NV_SATFINITE, __NV_E4M3);
+    if (threadIdx.x == 0) kbar_scale[out] = sc;
+  } else {
+    if (threadIdx.x < d)
+      reinterpret_cast<__nv_bfloat16*>(kbar)[out * d + threadIdx.x] = __float2bfloat16_rn(mean);
+  }
+}
+
+// Block of each row's position: prefill rows r at q_pos0 + r, decode rows at seq_len[r] - 1.
+__global__ void row_blocks_kernel(int32_t R, int64_t q_pos0, const int32_t* __restrict__ seq_len,
+                                  int32_t* __restrict__ row_blk) {
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (r >= R) return;
+  const int64_t p = seq_len != nullptr ? static_cast<int64_t>(seq_len[r]) - 1 : q_pos0 + r;
+  row_blk[r] = static_cast<int32_t>(p < 0 ? -1 : p / kBlk);
+}
+
+// Forced blocks: where more than n_blocks blocks are visible, block 0 and the row's own block
+// take +inf so that the block Top-n keeps them and fills the other slots by score.
+__global__ void force_blocks_kernel(float* __restrict__ scores, int64_t ld, int32_t R,
+                                    const int32_t* __restrict__ row_blk, int32_t n_blocks) {
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (r >= R) return;
+  const int32_t cur = row_blk[r];
+  if (cur + 1 <= n_blocks) return;
+  scores[r * ld] = INFINITY;
+  scores[r * ld + cur] = INFINITY;
+}
+
+}  // namespace
+
+cudaError_t launch_block_keys(const void* k, const float* k_scale, bool fp8, int64_t S, int d,
+                              int32_t n_seq, const int32_t* seq_len, int32_t len_fixed,
+                              bool last_only, int32_t nbmax, void* kbar, float* kbar_scale,
+                              cudaStream_t s) {
+  if (n_seq <= 0 || nbmax <= 0) return cudaSuccess;
+  if (kBkThreads % d != 0) return cudaErrorInvalidValue;
+  const dim3 grid(last_only ? 1 : nbmax, n_seq);
+  const uint8_t* kc = static_cast<const uint8_t*>(k);
+  uint8_t* out = static_cast<uint8_t*>(kbar);
+  if (fp8)
+    block_keys_kernel<true><<<grid, kBkThreads, 0, s>>>(kc, k_scale, S, d, seq_len, len_fixed,
+                                                        last_only ? 1 : 0, nbmax, out, kbar_scale);
+  else
+    block_keys_kernel<false><<<grid, kBkThreads, 0, s>>>(kc, k_scale, S, d, seq_len, len_fixed,
+                                                         last_only ? 1 : 0, nbmax, out, kbar_scale);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_row_blocks(int32_t R, int64_t q_pos0, const int32_t* seq_len, int32_t* row_blk,
+                              cudaStream_t s) {
+  if (R <= 0) return cudaSuccess;
+  row_blocks_kernel<<<static_cast<unsigned>((R + 255) / 256), 256, 0, s>>>(R, q_pos0, seq_len,
+                                                                          row_blk);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_force_blocks(float* scores, int64_t ld, int32_t R, const int32_t* row_blk,
+                                int32_t n_blocks, cudaStream_t s) {
+  if (R <= 0) return cudaSuccess;
+  force_blocks_kernel<<<static_cast<unsigned>((R + 255) / 256), 256, 0, s>>>(scores, ld, R,
+                                                                            row_blk, n_blocks);
+  return cudaGetLastError();
+}
+
+}  // namespace adx

@@ -117,7 +117,10 @@ __device__ __forceinline__ void block_info(const ScoreArgs& a, int i, Block& x) 
   x.ntiles = 0;
   if (x.row0 >= x.row_end) return;
   int64_t nk;
-  if (a.key_pos != nullptr || a.key_idx != nullptr) {
+  if (a.key_blk != nullptr) {
+    nk = min((row_position(a, x.row_end - 1) / kTileM + 1) * kTileM,
+             static_cast<int64_t>(a.keys_per_batch));
+  } else if (a.key_pos != nullptr || a.key_idx != nullptr) {
     nk = a.keys_per_batch;
   } else if (a.seq_len != nullptr && a.row_pos == nullptr) {
     nk = min(static_cast<int64_t>(a.seq_len[x.b]), static_cast<int64_t>(a.keys_per_batch));
@@ -448,7 +451,12 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         for (int t = t_lo; t < t_hi; ++t) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_s, a.timeout_ns)) break;
           mbar_arrive_expect_tx(&full[stage], C::KBYTES);
-          const int32_t y = static_cast<int32_t>(x.key_row0 + static_cast<int64_t>(t) * kTileM);
+          int64_t tile_row = static_cast<int64_t>(t) * kTileM;
+          if (a.key_blk != nullptr) {
+            const int32_t bk = __ldg(a.key_blk + static_cast<int64_t>(x.b) * a.key_blk_stride + t);
+            tile_row = bk >= 0 ? static_cast<int64_t>(bk) * kTileM : 0;  // no tile: masked
+          }
+          const int32_t y = static_cast<int32_t>(x.key_row0 + tile_row);
 #pragma unroll
           for (int kc = 0; kc < C::KC; ++kc)
             tma_load_2d(k_s + stage * C::KBYTES + kc * kTileM * 128, &tm_k, &full[stage],
@@ -576,6 +584,15 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
               kpos = p;
               if (a.k_scale != nullptr) ks = a.k_scale[x.key_row0 + p];
             }
+          }
+        } else if (a.key_blk != nullptr) {
+          kpos = INT64_MAX;
+          const int32_t bk =
+              c < x.nkeys ? a.key_blk[static_cast<int64_t>(x.b) * a.key_blk_stride + t] : -1;
+          const int64_t p = static_cast<int64_t>(bk) * kTileM + m;
+          if (bk >= 0 && p < a.S_valid) {
+            kpos = p;
+            if (a.k_scale != nullptr) ks = a.k_scale[x.key_row0 + p];
           }
         } else if (c < x.nkeys) {
           const int64_t kr = x.key_row0 + c;

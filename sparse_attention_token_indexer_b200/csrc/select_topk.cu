@@ -60,6 +60,13 @@ __device__ __forceinline__ uint32_t block_inclusive_scan(uint32_t x, uint32_t* w
   return x + before;
 }
 
+// Position of element id through the row's map (per element, or per block of 2^shift).
+__device__ __forceinline__ int32_t map_id(const int32_t* map, int32_t id, int shift) {
+  if (map == nullptr || id < 0) return id;
+  if (shift == 0) return map[id];
+  return (map[id >> shift] << shift) + (id & ((1 << shift) - 1));
+}
+
 struct RowInfo {
   int64_t lo, hi;  // element range of this CTA
 };
@@ -73,7 +80,7 @@ __device__ __forceinline__ int64_t row_length(const SelectArgs& a, int r) {
   } else if (a.len_mode == 2) {
     n = a.seq_len[r / a.rows_per_batch];
   } else {
-    n = static_cast<int64_t>(a.row_pos[r]) + 1 + a.len_off;
+    n = (static_cast<int64_t>(a.row_pos[r]) + 1 + a.len_off) * (a.len_mul > 1 ? a.len_mul : 1);
   }
   if (n > a.len_cap) n = a.len_cap;
   return n < 0 ? 0 : n;
@@ -194,7 +201,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a)
       if (sel_mask & (1u << j)) {
         const int64_t i = base + threadIdx.x * V + j;
         int32_t id = in_idx ? in_idx[i] : static_cast<int32_t>(i);
-        if (map != nullptr && id >= 0) id = map[id];
+        id = map_id(map, id, a.map_shift);
         if (slot < static_cast<uint32_t>(K)) {
           a.out_idx[out_base + slot] = id;
           if (a.out_val) a.out_val[out_base + slot] = v[j];
@@ -744,7 +751,7 @@ select_reg_kernel(const SelectArgs a, int row0) {
       st_idx[slot - cta_slot0] = static_cast<int32_t>(i);
     } else {
       int32_t id = in_idx ? in_idx[i] : static_cast<int32_t>(lo + i);
-      if (map != nullptr && id >= 0) id = map[id];
+      id = map_id(map, id, a.map_shift);
       a.out_idx[out_base + slot] = id;
       if (a.out_val) a.out_val[out_base + slot] = vals[i];
     }
@@ -757,7 +764,7 @@ select_reg_kernel(const SelectArgs a, int row0) {
     for (uint32_t sl = threadIdx.x; sl < n_out; sl += THREADS) {
       const int32_t i = st_idx[sl];
       int32_t id = in_idx ? in_idx[i] : static_cast<int32_t>(lo + i);
-      if (map != nullptr && id >= 0) id = map[id];
+      id = map_id(map, id, a.map_shift);
       a.out_idx[out_base + cta_slot0 + sl] = id;
       if (a.out_val) a.out_val[out_base + cta_slot0 + sl] = vals[i];
     }

@@ -574,3 +574,96 @@ def test_host_buffer_prefill_equals_device_path(dtype):
     torch.cuda.synchronize()
     assert torch.equal(idx, ref_idx.cpu())
     assert torch.equal(sc, ref_sc.cpu())
+
+
+# ---------------------------------------------------------------------------------------
+# HISA: block filter, then token refinement
+# ---------------------------------------------------------------------------------------
+
+def _check_hisa_row(t, p, q64, w64, k64, kbar64, blocks, idx, sc, n_blocks, K, rtol_blk, rtol,
+                    S):
+    """Row t at position p: the kernel's kept blocks must be the visible blocks (when they
+    fit) or the forced pair plus a valid Top-(n_blocks - 2) of the other visible blocks under
+    the oracle's block scores; its Top-K must be a valid Top-K of those blocks' visible
+    tokens under the oracle's token scores."""
+    cur = p // ox.HISA_BLOCK
+    nvis = cur + 1
+    got = blocks[t][blocks[t] >= 0]
+    assert np.all(blocks[t][len(got):] == -1) and len(set(got.tolist())) == len(got)
+    if nvis <= n_blocks:
+        assert sorted(got.tolist()) == list(range(nvis)), f"row {t}: blocks"
+    else:
+        forced = {0, cur}
+        assert forced <= set(got.tolist()) and len(got) == n_blocks, f"row {t}: forced blocks"
+        rest = np.array([b for b in range(nvis) if b not in forced])
+        chosen = np.array([b for b in got.tolist() if b not in forced])
+        full = np.concatenate([chosen, -np.ones(0, np.int64)])
+        check_topk(full, rest, ox.score_keys(q64[t], w64[t], kbar64[rest]),
+                   score_floor(q64[t], w64[t], kbar64[rest]), n_blocks - len(forced), rtol_blk,
+                   what=f"row {t} blocks")
+    cand = ox.hisa_candidates(sorted(got.tolist()), p, S)
+    check_topk(idx[t], cand, ox.score_keys(q64[t], w64[t], k64[cand]),
+               score_floor(q64[t], w64[t], k64[cand]), K, rtol, sc[t], f"row {t} tokens")
+
+
+@pytest.mark.parametrize("T,S,q_pos0,n_blocks,K", [(1500, 1500, 0, 5, 200),
+                                                    (700, 1900, 1200, 6, 640),
+                                                    (1300, 1300, 0, 64, 256)])
+def test_hisa_prefill(T, S, q_pos0, n_blocks, K):
+    """bf16 prefill: 12 to 15 blocks with a partial last one, a chunk whose rows start at
+    q_pos0 > 0, and a budget that holds every block (the flat indexer then)."""
+    p = inputs.anchor_prefill(T, H=64, d=128, K=K, seed=48, device="cuda", S=S, q_pos0=q_pos0)
+    kbar, _ = indexer.hisa_block_keys(p["q"], p["w"], p["k"], q_pos0=q_pos0)
+    idx, sc, blocks = indexer.index_hisa(p["q"], p["w"], p["k"], kbar, K, n_blocks=n_blocks,
+                                         q_pos0=q_pos0, with_scores=True, with_blocks=True)
+    q64, w64, k64 = f64(p["q"]), p["w"].double().cpu().numpy(), f64(p["k"])
+    ref_bar = ox.hisa_block_keys(k64[:q_pos0 + T])
+    got_bar = f64(kbar)[:ref_bar.shape[0]]
+    assert np.all(np.abs(got_bar - ref_bar) <= 2.0 ** -8 * np.abs(ref_bar) + 1e-6)
+    idx, sc, blocks = idx.cpu().numpy(), sc.cpu().numpy(), blocks.cpu().numpy()
+    rows = sorted(set(range(0, T, 37)) | {0, T - 1, T // 2})
+    for t in rows:
+        _check_hisa_row(t, q_pos0 + t, q64, w64, k64, got_bar, blocks, idx, sc, n_blocks, K,
+                        RTOL["bf16"], RTOL["bf16"], S)
+
+
+def test_hisa_decode_e4m3_and_last_block_update():
+    """e4m3 caches of four lengths; the block keys of the next step, updated in place for the
+    last block only, equal a full recomputation (bit for bit) and index the same way. Block
+    selection tolerance is twice the e4m3 one: the block keys carry their own e4m3 rounding
+    on top of the query's."""
+    Bs, S, n_blocks, K = 4, 3100, 6, 300
+    prob = inputs.decode_problem(Bs=Bs, S=S, H=64, d=128, K=K, Hg=16, steps=2, seed=49,
+                                 device="cuda")
+    k, ks = prob["k"], prob["k_scale"]
+    S_cap = k.shape[1]
+    seq_len = torch.tensor([S, 2049, 130, 1], dtype=torch.int32, device="cuda")
+    q, w = prob["q_steps"][0], prob["w_steps"][0]
+    kbar, kbs = indexer.hisa_block_keys(q, w, k, k_scale=ks, seq_len=seq_len)
+    idx, sc, blocks = indexer.index_hisa(q, w, k, kbar, K, n_blocks=n_blocks, k_scale=ks,
+                                         kbar_scale=kbs, seq_len=seq_len, with_scores=True,
+                                         with_blocks=True)
+    q64, w64 = f64(q), w.double().cpu().numpy()
+    k64 = f64(k.reshape(-1, 128), ks.reshape(-1)).reshape(Bs, S_cap, 128)
+    kb64 = f64(kbar.reshape(-1, 128), kbs.reshape(-1)).reshape(Bs, -1, 128)
+    idx_h, sc_h, blocks_h = idx.cpu().numpy(), sc.cpu().numpy(), blocks.cpu().numpy()
+    for b, n in enumerate(seq_len.tolist()):
+        ref = ox.hisa_block_keys(k64[b, :n])
+        got = kb64[b, :ref.shape[0]]
+        amax = np.abs(ref).max(axis=1, keepdims=True)
+        assert np.all(np.abs(got - ref) <= 2.0 ** -4 * np.abs(ref) + 2.0 ** -9 * amax / 448 * 2)
+        _check_hisa_row(b, n - 1, q64, w64, k64[b], got, blocks_h, idx_h, sc_h, n_blocks, K,
+                        2 * RTOL["e4m3"], RTOL["e4m3"], S_cap)
+    # next step: one more key per sequence, block keys refreshed for the last block only
+    seq2 = seq_len + 1
+    indexer.hisa_block_keys(q, w, k, k_scale=ks, seq_len=seq2, last_only=True, out=(kbar, kbs))
+    full, fulls = indexer.hisa_block_keys(q, w, k, k_scale=ks, seq_len=seq2)
+    for b, n in enumerate(seq2.tolist()):
+        nb = (n + 127) // 128
+        assert torch.equal(kbar[b, :nb], full[b, :nb]) and torch.equal(kbs[b, :nb], fulls[b, :nb])
+    q2, w2 = prob["q_steps"][1], prob["w_steps"][1]
+    a = indexer.index_hisa(q2, w2, k, kbar, K, n_blocks=n_blocks, k_scale=ks, kbar_scale=kbs,
+                           seq_len=seq2)[0]
+    bb = indexer.index_hisa(q2, w2, k, full, K, n_blocks=n_blocks, k_scale=ks,
+                            kbar_scale=fulls, seq_len=seq2)[0]
+    assert torch.equal(a, bb)
