@@ -169,7 +169,9 @@ size_t adx_hisa_workspace_size(const adx_operands* ops, int32_t n_blocks, int32_
                                int32_t blocks_external);
 
 /* HISA indexer step. kbar / kbar_scale from adx_hisa_block_keys (read only). Requires
- * 2 <= n_blocks, K <= n_blocks * 128, T * n_blocks * 128 < 2^31.
+ * 2 <= n_blocks <= 255, K <= n_blocks * 128, T * n_blocks * 128 < 2^31, H = 64 (else
+ * ADX_EUNSUPPORTED). Prefill rows are refined in groups of 4 consecutive rows that score the
+ * union of their kept blocks together; each row's Top-K still ranges over its own blocks.
  * topk_idx [T, K] int32 out: key positions (within the row's key range), -1 padded;
  * topk_score [T, K] or NULL; blocks_out [T, n_blocks] or NULL: the kept blocks, -1 padded. */
 adx_status adx_index_hisa(const adx_operands* ops, const void* kbar, const float* kbar_scale,

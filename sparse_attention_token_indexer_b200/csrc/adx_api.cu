@@ -541,14 +541,17 @@ size_t ws_mtp(const adx_operands* full, const adx_operands* gops, const MtpShape
 constexpr int kHisaShift = 7;  // log2 of the block size (one MMA tile of keys)
 static_assert((1 << kHisaShift) == kTileM, "a HISA block is one key tile");
 
+constexpr int kHisaHeads = 64;  // the block-list scoring configurations
+// prefill rows per union group (the rows of one N = 256 tile)
+constexpr int kHisaGroup = 4;
+
 int64_t hisa_nbmax(const adx_operands* o) { return (o->S + kTileM - 1) / kTileM; }
 
 adx_status hisa_check(const adx_operands* o, int32_t n_blocks, int32_t K) {
   const adx_status r = check_operands(o, o != nullptr && o->seq_len != nullptr);
   if (r != ADX_OK) return r;
-  if (n_blocks < 2 || K <= 0 || static_cast<int64_t>(n_blocks) * kTileM > (1ll << 24) ||
-      K > n_blocks * kTileM)
-    return ADX_EINVAL;
+  if (n_blocks < 2 || n_blocks > 255 || K <= 0 || K > n_blocks * kTileM) return ADX_EINVAL;
+  if (o->H != kHisaHeads) return ADX_EUNSUPPORTED;
   if (static_cast<int64_t>(o->T) * n_blocks * kTileM > INT32_MAX) return ADX_EINVAL;
   return ADX_OK;
 }
@@ -560,6 +563,11 @@ size_t ws_hisa(const adx_operands* o, int32_t n_blocks, int32_t K, bool blocks_e
   b += align_up(static_cast<size_t>(T) * ld_for(nbmax) * 4, kAlign);         // block scores
   if (!blocks_external) b += align_up(static_cast<size_t>(T) * n_blocks * 4, kAlign);
   b += align_up(static_cast<size_t>(T) * nc * 4, kAlign);                    // token scores
+  if (o->seq_len == nullptr) {  // prefill: block unions of groups of rows
+    const size_t ng = static_cast<size_t>((T + kHisaGroup - 1) / kHisaGroup);
+    const size_t width = static_cast<size_t>(kHisaGroup) * n_blocks;
+    b += 2 * align_up(ng * width * 4, kAlign) + align_up(ng * 4, kAlign);
+  }
   b += select_scratch_bytes(T, nbmax, n_blocks) + select_scratch_bytes(T, nc, K);
   return b;
 }
@@ -1164,29 +1172,45 @@ adx_status adx_index_hisa(const adx_operands* o, const void* kbar, const float* 
     sa.rows = T;
     if ((r = run_select(sa, nbmax, cv, st, s)) != ADX_OK) return r;
   }
-  // 3. token refinement: every row scores the key tiles of its own blocks
+  // 3. token refinement: a decode row scores the key tiles of its own blocks; a group of
+  //    kHisaGroup prefill rows scores the union of its rows' blocks in one N = 256 tile, each
+  //    row's scores landing in the slots of its own list (no row sees a block it did not keep)
   {
-    ScorePlan p = decode ? rowwise_plan(o, pq, tsc, nc) : base_plan(o, pq, 1);
+    ScorePlan p = decode ? rowwise_plan(o, pq, tsc, nc) : base_plan(o, pq, kHisaGroup);
     ScoreArgs& a = p.a;
     a.key_blk = blocks;
     a.key_blk_stride = n_blocks;
     a.S_valid = o->S;
     a.keys_per_batch = nc;
     a.status = st;
+    int64_t max_tiles = n_blocks;
     if (!decode) {
+      const int32_t ng = (T + kHisaGroup - 1) / kHisaGroup, width = kHisaGroup * n_blocks;
+      int32_t* uni = cv.take<int32_t>(static_cast<size_t>(ng) * width * 4);
+      int32_t* slot = cv.take<int32_t>(static_cast<size_t>(ng) * width * 4);
+      int32_t* cnt = cv.take<int32_t>(static_cast<size_t>(ng) * 4);
+      if (counted(launch_block_union(blocks, n_blocks, T, kHisaGroup, uni, slot, cnt, s)) !=
+          cudaSuccess)
+        return ADX_ECUDA;
+      a.key_blk = uni;
+      a.key_blk_stride = width;
+      a.key_blk_count = cnt;
+      a.key_blk_slot = slot;
+      a.keys_per_batch = width * kTileM;
       a.scores = tsc;
       a.score_ld = nc;
       a.pos_base = o->q_pos0;
       a.pos_step = 1;
       a.R = T;
-      a.rows_per_batch = 1;
-      a.n_batches = T;
-      a.key_batch_div = T;
+      a.rows_per_batch = kHisaGroup;
+      a.n_batches = ng;
+      a.key_batch_div = ng;
       a.key_batch_stride = 0;
       a.row_blocks_per_batch = 1;
       a.reverse_order = 1;
+      max_tiles = width;
     }
-    finish_plan(p, n_blocks);
+    finish_plan(p, max_tiles);
     if ((r = run_score(p, pq.q, o->k, decode ? static_cast<int64_t>(T) * o->S : o->S, s)) !=
         ADX_OK)
       return r;

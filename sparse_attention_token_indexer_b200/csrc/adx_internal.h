@@ -42,12 +42,17 @@ struct ScoreArgs {
   int64_t key_idx_stride;
   int32_t n_idx;
   int32_t S_valid;
-  // Key blocks (one row per key batch, contiguous key rows): tile t of batch b is the 128 key
-  // rows starting at 128 * key_blk[b * key_blk_stride + t] of the batch's key range; a
-  // negative entry is no tile, and rows at or past S_valid are no key. A row block then
-  // scores min(keys_per_batch / 128, row position / 128 + 1) tiles. Null: contiguous tiles.
+  // Key blocks: tile t of batch b is the 128 key rows starting at
+  // 128 * key_blk[b * key_blk_stride + t] of the batch's key range; a negative entry is no
+  // tile, and rows at or past S_valid are no key. The batch scores key_blk_count[b] tiles
+  // (null: min(keys_per_batch / 128, last row position / 128 + 1)). key_blk_slot (same layout,
+  // or null): byte j is the slot of tile t in the block list of the batch's row j, whose
+  // score row receives the tile at columns [128 * slot, 128 * slot + 128) (0xFF: not one of
+  // that row's blocks); null: slot t for every row. Null key_blk: contiguous tiles.
   const int32_t* key_blk;
   int64_t key_blk_stride;
+  const int32_t* key_blk_count;
+  const int32_t* key_blk_slot;
   const int32_t* seq_len;  // [n_batches] or null
   const int32_t* row_pos;  // [R] or null
   const int8_t* fold_flag; // [R]: 1 = the row's queries carry its gates already; null = none do
@@ -172,6 +177,12 @@ cudaError_t launch_block_keys(const void* k, const float* k_scale, bool fp8, int
 // row_blk[r] = block of row r's position (q_pos0 + r, or seq_len[r] - 1 when seq_len is set).
 cudaError_t launch_row_blocks(int32_t R, int64_t q_pos0, const int32_t* seq_len, int32_t* row_blk,
                               cudaStream_t s);
+// Union of the block lists (blocks [R, n_blocks], -1 padded) of each group of `tok`
+// consecutive rows: uni [groups, tok * n_blocks] distinct blocks, count [groups] how many,
+// slot [groups, tok * n_blocks] byte j = slot of the union entry in row j's list (0xFF: none).
+// tok <= 4, n_blocks <= 255.
+cudaError_t launch_block_union(const int32_t* blocks, int32_t n_blocks, int32_t R, int32_t tok,
+                               int32_t* uni, int32_t* slot, int32_t* count, cudaStream_t s);
 // Raises the scores of block 0 and of the row's own block to +inf on rows that see more than
 // n_blocks blocks.
 cudaError_t launch_force_blocks(float* scores, int64_t ld, int32_t R, const int32_t* row_blk,

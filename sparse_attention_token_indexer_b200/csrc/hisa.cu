@@ -101,7 +101,84 @@ __global__ void force_blocks_kernel(float* __restrict__ scores, int64_t ld, int3
   scores[r * ld + cur] = INFINITY;
 }
 
+// Union of the block lists of `tok` consecutive rows (one CTA per group, one thread per list
+// entry, P = the entry count rounded up to a power of two): the entries, keyed
+// (block, row, slot), are sorted (bitonic, in shared memory); the first entry of each block
+// number gives it its union position, and every entry records its slot in its row's list
+// as byte `row` of the union position's slot word (0xFF where a row lacks the block).
+__global__ void block_union_kernel(const int32_t* __restrict__ blocks, int32_t n_blocks,
+                                   int32_t R, int32_t tok, int32_t stride,
+                                   int32_t* __restrict__ uni, int32_t* __restrict__ slot,
+                                   int32_t* __restrict__ count) {
+  extern __shared__ uint64_t key_s[];  // [P] keys, then [stride] slot words
+  const int P = blockDim.x;
+  uint32_t* slot_s = reinterpret_cast<uint32_t*>(key_s + P);
+  __shared__ int warp_n[32];
+  const int64_t g = blockIdx.x;
+  const int i = threadIdx.x;
+  const int row = i / n_blocks, j = i % n_blocks;
+  const int64_t r = g * tok + row;
+  int32_t v = -1;
+  if (i < tok * n_blocks && r < R) v = blocks[r * n_blocks + j];
+  key_s[i] = v >= 0 ? (static_cast<uint64_t>(v) << 16) | (static_cast<uint64_t>(row) << 8) |
+                          static_cast<uint64_t>(j)
+                    : ~0ull;
+  for (int u = i; u < stride; u += P) slot_s[u] = 0xFFFFFFFFu;
+  __syncthreads();
+  for (int k = 2; k <= P; k <<= 1) {
+    for (int h = k >> 1; h > 0; h >>= 1) {
+      const int o = i ^ h;
+      if (o > i) {
+        const uint64_t a = key_s[i], b = key_s[o];
+        if (((i & k) == 0) == (a > b)) {
+          key_s[i] = b;
+          key_s[o] = a;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  const uint64_t kk = key_s[i];
+  const bool valid = kk != ~0ull;
+  const bool first = valid && (i == 0 || (key_s[i - 1] >> 16) != (kk >> 16));
+  // union position = number of first entries at or before i, minus one
+  const unsigned bal = __ballot_sync(0xffffffffu, first);
+  const int lane = i & 31, wid = i >> 5;
+  if (lane == 31) warp_n[wid] = __popc(bal);
+  __syncthreads();
+  int before = 0, total = 0;
+  for (int w = 0; w < P / 32; ++w) {
+    if (w < wid) before += warp_n[w];
+    total += warp_n[w];
+  }
+  const int u = before + __popc(bal & ((2u << lane) - 1u)) - 1;
+  if (valid) {
+    const int rr = static_cast<int>((kk >> 8) & 0xFF), jj = static_cast<int>(kk & 0xFF);
+    reinterpret_cast<uint8_t*>(slot_s)[u * 4 + rr] = static_cast<uint8_t>(jj);
+    if (first) uni[g * stride + u] = static_cast<int32_t>(kk >> 16);
+  }
+  __syncthreads();
+  for (int q = i; q < total; q += P) slot[g * stride + q] = static_cast<int32_t>(slot_s[q]);
+  if (i == 0) count[g] = total;
+}
+
 }  // namespace
+
+cudaError_t launch_block_union(const int32_t* blocks, int32_t n_blocks, int32_t R, int32_t tok,
+                               int32_t* uni, int32_t* slot, int32_t* count, cudaStream_t s) {
+  if (R <= 0) return cudaSuccess;
+  const int n = tok * n_blocks;
+  if (tok < 1 || tok > 4 || n_blocks < 1 || n_blocks > 255 || n > 1024)
+    return cudaErrorInvalidValue;
+  int P = 32;
+  while (P < n) P <<= 1;
+  const int stride = n;
+  const size_t smem = static_cast<size_t>(P) * 8 + static_cast<size_t>(stride) * 4;
+  const int groups = (R + tok - 1) / tok;
+  block_union_kernel<<<static_cast<unsigned>(groups), P, smem, s>>>(blocks, n_blocks, R, tok,
+                                                                     stride, uni, slot, count);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_block_keys(const void* k, const float* k_scale, bool fp8, int64_t S, int d,
                               int32_t n_seq, const int32_t* seq_len, int32_t len_fixed,

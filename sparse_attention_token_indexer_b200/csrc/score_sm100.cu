@@ -38,13 +38,18 @@ __host__ __device__ constexpr int pow2ceil(int x) {
   return p;
 }
 
-template <int H_, int TOK_, int DB_, bool FP8_, bool GATHER_ = false>
+// Key tiles: contiguous rows (0), rows gathered one by one with tile::gather4 (1), or whole
+// 128-row blocks from a per-batch block list (2).
+constexpr int kKeysContiguous = 0, kKeysGather = 1, kKeysBlocks = 2;
+
+template <int H_, int TOK_, int DB_, bool FP8_, int KM_ = kKeysContiguous>
 struct Cfg {
   static constexpr int H = H_;
   static constexpr int TOK = TOK_;
   static constexpr int DB = DB_;             // bytes per q/k row (d * element size)
   static constexpr bool FP8 = FP8_;
-  static constexpr bool GATHER = GATHER_;    // key tiles gathered row by row (tile::gather4)
+  static constexpr bool GATHER = KM_ == kKeysGather;  // key rows gathered (tile::gather4)
+  static constexpr bool BLOCKS = KM_ == kKeysBlocks;  // key tiles from a block list
   static constexpr int N = TOK * H;          // MMA N
   static constexpr int KC = DB / 128;        // 128-byte K chunks
   static constexpr int ELEMS_PER_CHUNK = FP8 ? 128 : 64;
@@ -118,8 +123,10 @@ __device__ __forceinline__ void block_info(const ScoreArgs& a, int i, Block& x) 
   if (x.row0 >= x.row_end) return;
   int64_t nk;
   if (a.key_blk != nullptr) {
-    nk = min((row_position(a, x.row_end - 1) / kTileM + 1) * kTileM,
-             static_cast<int64_t>(a.keys_per_batch));
+    nk = a.key_blk_count != nullptr
+             ? static_cast<int64_t>(a.key_blk_count[x.b]) * kTileM
+             : (row_position(a, x.row_end - 1) / kTileM + 1) * kTileM;
+    nk = min(nk, static_cast<int64_t>(a.keys_per_batch));
   } else if (a.key_pos != nullptr || a.key_idx != nullptr) {
     nk = a.keys_per_batch;
   } else if (a.seq_len != nullptr && a.row_pos == nullptr) {
@@ -452,7 +459,7 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_s, a.timeout_ns)) break;
           mbar_arrive_expect_tx(&full[stage], C::KBYTES);
           int64_t tile_row = static_cast<int64_t>(t) * kTileM;
-          if (a.key_blk != nullptr) {
+          if constexpr (C::BLOCKS) {
             const int32_t bk = __ldg(a.key_blk + static_cast<int64_t>(x.b) * a.key_blk_stride + t);
             tile_row = bk >= 0 ? static_cast<int64_t>(bk) * kTileM : 0;  // no tile: masked
           }
@@ -572,10 +579,11 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
       // per-key scale and position of the next tile, loaded one tile ahead so their
       // latency hides behind the current tile's wait and reduction
-      auto key_meta = [&](int t, float& ks, int64_t& kpos) {
+      auto key_meta = [&](int t, float& ks, int64_t& kpos, uint32_t& slots) {
         const int c = t * kTileM + m;
         kpos = c;
         ks = 1.f;
+        slots = 0u;
         if constexpr (C::GATHER) {
           kpos = INT64_MAX;  // no key: never visible
           if (c < x.nkeys && c < a.n_idx) {
@@ -585,15 +593,16 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
               if (a.k_scale != nullptr) ks = a.k_scale[x.key_row0 + p];
             }
           }
-        } else if (a.key_blk != nullptr) {
+        } else if constexpr (C::BLOCKS) {
           kpos = INT64_MAX;
-          const int32_t bk =
-              c < x.nkeys ? a.key_blk[static_cast<int64_t>(x.b) * a.key_blk_stride + t] : -1;
+          const int64_t e = static_cast<int64_t>(x.b) * a.key_blk_stride + t;
+          const int32_t bk = c < x.nkeys ? a.key_blk[e] : -1;
           const int64_t p = static_cast<int64_t>(bk) * kTileM + m;
           if (bk >= 0 && p < a.S_valid) {
             kpos = p;
             if (a.k_scale != nullptr) ks = a.k_scale[x.key_row0 + p];
           }
+          if (a.key_blk_slot != nullptr) slots = static_cast<uint32_t>(a.key_blk_slot[e]);
         } else if (c < x.nkeys) {
           const int64_t kr = x.key_row0 + c;
           if (a.key_pos != nullptr) kpos = a.key_pos[kr];
@@ -609,12 +618,14 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       if (C::BUF_SPLIT) t0 += static_cast<int>(((grp - gi_lo) % C::EG + C::EG) % C::EG);
       float ks_next = 1.f;
       int64_t kpos_next = 0;
-      if (t0 < t_hi) key_meta(t0, ks_next, kpos_next);
+      uint32_t slots_next = 0u;
+      if (t0 < t_hi) key_meta(t0, ks_next, kpos_next, slots_next);
       bool ok = true;
       for (int t = t0; t < t_hi; t += TSTEP) {
         const float ks = ks_next;
         const int64_t kpos = kpos_next;
-        if (t + TSTEP < t_hi) key_meta(t + TSTEP, ks_next, kpos_next);
+        const uint32_t slots = slots_next;
+        if (t + TSTEP < t_hi) key_meta(t + TSTEP, ks_next, kpos_next, slots_next);
         const int64_t g = gi_lo + (t - t_lo);
         const int acc = static_cast<int>(g % C::ACC);
         const uint32_t acc_phase = static_cast<uint32_t>((g / C::ACC) & 1);
@@ -675,7 +686,19 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll
             for (int p = 0; p < C::NP; ++p) sc += part[tt][p].x + part[tt][p].y;
             const bool vis = key_ok && kpos <= rpos[tt];
-            a.scores[static_cast<int64_t>(r) * a.score_ld + c] = vis ? (ks * tokf[tt]) * sc : -INFINITY;
+            const float out = vis ? (ks * tokf[tt]) * sc : -INFINITY;
+            if constexpr (C::BLOCKS) {
+              // with a slot table, tile t is block slots.byte[token] of the token's own list
+              // (0xFF: not one of its blocks); without one, every token's slot is t
+              int col = c;
+              if (a.key_blk_slot != nullptr) {
+                const uint32_t sl = (slots >> (8 * (tok0 + tt))) & 0xFFu;
+                col = sl == 0xFFu ? -1 : static_cast<int>(sl) * kTileM + m;
+              }
+              if (col >= 0) a.scores[static_cast<int64_t>(r) * a.score_ld + col] = out;
+            } else {
+              a.scores[static_cast<int64_t>(r) * a.score_ld + c] = out;
+            }
           }
         }
       }
@@ -734,14 +757,27 @@ bool score_config_supported(bool fp8, int H, int d) {
   /* a few group queries per key batch (MTP windows): N = 2 or 4 tokens x 16 heads */  \
   X(false, 16, 2, 128) X(true, 16, 2, 128) X(false, 16, 4, 128) X(true, 16, 4, 128)
 
+// Block-list configurations (HISA refinement): one decode row per key batch, or a group of
+// score_tokens_per_tile(H) prefill rows scoring the union of their blocks.
+#define ADX_BLOCK_CONFIGS(X) \
+  X(false, 64, 1, 128) X(true, 64, 1, 128) X(false, 64, 4, 128) X(true, 64, 4, 128)
+
 // tok: tokens per N tile; score_tokens_per_tile(H) (prefill), 1 (one query per key batch:
 // decode and its bank refresh), or 2 / 4 with 16 heads (the group queries of an MTP window).
 cudaError_t launch_score(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const ScoreArgs& a,
                          bool fp8, int H, int d, int tok, int grid, cudaStream_t s) {
   const bool gather = a.key_idx != nullptr;
+  if (a.key_blk != nullptr) {
 #define ADX_CASE(FP, HH, TT, DD)                                                        \
   if (fp8 == FP && H == HH && tok == TT && d == DD)                                     \
-    return gather ? launch_cfg<Cfg<HH, TT, (FP ? DD : 2 * DD), FP, true>>(tm_q, tm_k, a, grid, s) \
+    return launch_cfg<Cfg<HH, TT, (FP ? DD : 2 * DD), FP, kKeysBlocks>>(tm_q, tm_k, a, grid, s);
+    ADX_BLOCK_CONFIGS(ADX_CASE)
+#undef ADX_CASE
+    return cudaErrorNotSupported;
+  }
+#define ADX_CASE(FP, HH, TT, DD)                                                        \
+  if (fp8 == FP && H == HH && tok == TT && d == DD)                                     \
+    return gather ? launch_cfg<Cfg<HH, TT, (FP ? DD : 2 * DD), FP, kKeysGather>>(tm_q, tm_k, a, grid, s) \
                   : launch_cfg<Cfg<HH, TT, (FP ? DD : 2 * DD), FP>>(tm_q, tm_k, a, grid, s);
   ADX_SCORE_CONFIGS(ADX_CASE)
 #undef ADX_CASE
