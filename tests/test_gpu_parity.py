@@ -606,25 +606,40 @@ def _check_hisa_row(t, p, q64, w64, k64, kbar64, blocks, idx, sc, n_blocks, K, r
                score_floor(q64[t], w64[t], k64[cand]), K, rtol, sc[t], f"row {t} tokens")
 
 
-@pytest.mark.parametrize("T,S,q_pos0,n_blocks,K", [(1500, 1500, 0, 5, 200),
-                                                    (700, 1900, 1200, 6, 640),
-                                                    (1300, 1300, 0, 64, 256)])
-def test_hisa_prefill(T, S, q_pos0, n_blocks, K):
-    """bf16 prefill: 12 to 15 blocks with a partial last one, a chunk whose rows start at
-    q_pos0 > 0, and a budget that holds every block (the flat indexer then)."""
-    p = inputs.anchor_prefill(T, H=64, d=128, K=K, seed=48, device="cuda", S=S, q_pos0=q_pos0)
-    kbar, _ = indexer.hisa_block_keys(p["q"], p["w"], p["k"], q_pos0=q_pos0)
+@pytest.mark.parametrize("T,S,q_pos0,n_blocks,K,dtype", [
+    (1500, 1500, 0, 5, 200, "bf16"), (700, 1900, 1200, 6, 640, "bf16"),
+    (1300, 1300, 0, 64, 256, "bf16"),
+    # a last group of rows shorter than the 4 that share a union, e4m3 operands, and the
+    # smallest budget (the two forced blocks only)
+    (1501, 1501, 0, 4, 300, "bf16"), (1203, 1203, 0, 5, 256, "e4m3"),
+    (1027, 1400, 373, 2, 200, "bf16")])
+def test_hisa_prefill(T, S, q_pos0, n_blocks, K, dtype):
+    """Prefill: 12 to 15 blocks with a partial last one, a chunk whose rows start at
+    q_pos0 > 0, a budget that holds every block (the flat indexer then), ragged row groups,
+    e4m3 operands (block keys e4m3 too: twice the e4m3 tolerance for the block choice)."""
+    p = inputs.anchor_prefill(T, H=64, d=128, K=K, seed=48, device="cuda", S=S, q_pos0=q_pos0,
+                              dtype=dtype)
+    kbar, kbs = indexer.hisa_block_keys(p["q"], p["w"], p["k"], q_scale=p["q_scale"],
+                                        k_scale=p["k_scale"], q_pos0=q_pos0)
     idx, sc, blocks = indexer.index_hisa(p["q"], p["w"], p["k"], kbar, K, n_blocks=n_blocks,
-                                         q_pos0=q_pos0, with_scores=True, with_blocks=True)
-    q64, w64, k64 = f64(p["q"]), p["w"].double().cpu().numpy(), f64(p["k"])
+                                         q_scale=p["q_scale"], k_scale=p["k_scale"],
+                                         kbar_scale=kbs, q_pos0=q_pos0, with_scores=True,
+                                         with_blocks=True)
+    q64, w64 = f64(p["q"], p["q_scale"]), p["w"].double().cpu().numpy()
+    k64 = f64(p["k"], p["k_scale"])
     ref_bar = ox.hisa_block_keys(k64[:q_pos0 + T])
-    got_bar = f64(kbar)[:ref_bar.shape[0]]
-    assert np.all(np.abs(got_bar - ref_bar) <= 2.0 ** -8 * np.abs(ref_bar) + 1e-6)
+    got_bar = f64(kbar, kbs)[:ref_bar.shape[0]]
+    if dtype == "bf16":
+        assert np.all(np.abs(got_bar - ref_bar) <= 2.0 ** -8 * np.abs(ref_bar) + 1e-6)
+    else:
+        amax = np.abs(ref_bar).max(axis=1, keepdims=True)
+        assert np.all(np.abs(got_bar - ref_bar) <= 2.0 ** -4 * np.abs(ref_bar) + 2.0 ** -8 * amax / 448)
     idx, sc, blocks = idx.cpu().numpy(), sc.cpu().numpy(), blocks.cpu().numpy()
-    rows = sorted(set(range(0, T, 37)) | {0, T - 1, T // 2})
+    rows = sorted(set(range(0, T, 37)) | {0, T - 1, T - 2, T - 3, T // 2})
+    rtol = RTOL[dtype]
     for t in rows:
         _check_hisa_row(t, q_pos0 + t, q64, w64, k64, got_bar, blocks, idx, sc, n_blocks, K,
-                        RTOL["bf16"], RTOL["bf16"], S)
+                        rtol if dtype == "bf16" else 2 * rtol, rtol, S)
 
 
 def test_hisa_decode_e4m3_and_last_block_update():
