@@ -228,6 +228,37 @@ def timed(fn, steps, warmup, dist, stage_timer=None):
     return ms, launches
 
 
+def timed_graph(fn, steps, warmup, dist):
+    """Like timed(), with the step captured once in a CUDA graph and replayed: for steps of
+    many short kernels, where the host's launch rate rather than the GPU bounds the plain
+    loop. The launch count is the capture's, once per replayed step."""
+    from sparse_attention_token_indexer_b200 import _lib
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    n0 = _lib.lib().adx_launch_count()
+    with torch.cuda.graph(g):
+        fn()
+    per_step = _lib.lib().adx_launch_count() - n0
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(s)
+    for _ in range(steps):
+        g.replay()
+    end.record(s)
+    torch.cuda.synchronize()
+    dist.barrier()
+    ms = dist.max(start.elapsed_time(end)) / steps
+    del g
+    return ms, per_step * steps
+
+
 # ---------------------------------------------------------------------------------------
 # workloads (our CUDA path)
 # ---------------------------------------------------------------------------------------
@@ -359,9 +390,11 @@ def run_decode(args, dist, cycle=True):
                                 seq_len=seqs[r], ws=ws)
 
     ms_cycle, l_cycle = timed(cycle, max(2, args.steps // 4), args.warmup, dist)
+    ms_cycle_graph, _ = timed_graph(cycle, max(2, args.steps // 4), args.warmup, dist)
     key_bytes = c["d"] + 4
     return dict(ms_flat=ms_flat, launches_flat=l_flat, ms_cycle=ms_cycle, launches_cycle=l_cycle,
-                bytes_flat=c["Bs"] * c["S"] * key_bytes, steps_per_cycle=c["G"], stages=dstages)
+                ms_cycle_graph=ms_cycle_graph, bytes_flat=c["Bs"] * c["S"] * key_bytes,
+                steps_per_cycle=c["G"], stages=dstages)
 
 
 def run_mtp(args, dist):
@@ -466,10 +499,11 @@ def run_hisa_decode(args, dist):
                            kbar_scale=kbs, seq_len=seq0, ws=ws)
 
     ms, launches = timed(step, args.steps, args.warmup, dist)
+    ms_graph, _ = timed_graph(step, args.steps, args.warmup, dist)
     nb = (c["S"] + 127) // 128
     key_bytes = c["d"] + 4
     bytes_step = c["Bs"] * (HISA["n_blocks"] * 128 + nb + 128) * key_bytes
-    return dict(ms=ms, launches=launches, bytes=bytes_step)
+    return dict(ms=ms, ms_graph=ms_graph, launches=launches, bytes=bytes_step)
 
 
 def run_group_indexer(args, dist):
@@ -587,10 +621,10 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--case", default="flat", choices=["flat", "flat_small", "decode", "mtp",
                                                       "group_indexer", "hisa", "hisa_small",
-                                                      "hisa_decode"],
+                                                      "hisa_decode", "decode_cycle"],
                     help="flat_small: T = 8192, for profiler captures; decode, mtp, "
-                         "group_indexer, hisa, hisa_decode: that workload alone (with "
-                         "--quick); hisa_small: HISA prefill at T = 16384")
+                         "group_indexer, hisa, hisa_decode, decode_cycle: that workload alone "
+                         "(with --quick); hisa_small: HISA prefill at T = 16384")
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "e4m3"])
     ap.add_argument("--quick", action="store_true",
                     help="time the kernels only (no e2e, rows or CPU baseline): for profiling")
@@ -649,6 +683,15 @@ def main():
                               "gpu_launches": dcd["launches_flat"]}), flush=True)
         dist.close()
         return
+    if args.case == "decode_cycle" and args.quick:
+        dcd = run_decode(args, dist)
+        if dist.rank == 0:
+            n = dcd["steps_per_cycle"]
+            print(json.dumps({"case": "decode_cycle", "ms_per_step": dcd["ms_cycle"] / n,
+                              "graph_ms_per_step": dcd["ms_cycle_graph"] / n,
+                              "gpu_launches": dcd["launches_cycle"]}), flush=True)
+        dist.close()
+        return
     if args.case == "mtp" and args.quick:
         mt = run_mtp(args, dist)
         if dist.rank == 0:
@@ -672,6 +715,7 @@ def main():
         hd = run_hisa_decode(args, dist)
         if dist.rank == 0:
             print(json.dumps({"case": "hisa_decode", "ms_per_step": hd["ms"],
+                              "graph_ms_per_step": hd["ms_graph"],
                               "gpu_launches": hd["launches"]}), flush=True)
         dist.close()
         return
@@ -779,7 +823,8 @@ def main():
             "gpu_launches": hs["launches"]}
         hd = run_hisa_decode(args, dist)
         rows["hisa_decode_Bs32_S131072_e4m3_nb64"] = {
-            "ms_per_step": hd["ms"], "flat_ms_per_step": dcd["ms_flat"],
+            "ms_per_step": hd["ms"], "graph_ms_per_step": hd["ms_graph"],
+            "flat_ms_per_step": dcd["ms_flat"],
             "speedup_vs_flat": dcd["ms_flat"] / hd["ms"],
             "topk_queries_per_s": DECODE["Bs"] / (hd["ms"] * 1e-3),
             "hbm_gbs": hd["bytes"] / (hd["ms"] * 1e-3) / 1e9, "gpu_launches": hd["launches"]}
@@ -793,6 +838,7 @@ def main():
         rows["decode_bank_reuse_cycle16"] = {
             "ms_per_cycle": dcd["ms_cycle"],
             "ms_per_step": dcd["ms_cycle"] / dcd["steps_per_cycle"],
+            "graph_ms_per_step": dcd["ms_cycle_graph"] / dcd["steps_per_cycle"],
             "topk_queries_per_s": DECODE["Bs"] * dcd["steps_per_cycle"] / (dcd["ms_cycle"] * 1e-3),
             "gpu_launches": dcd["launches_cycle"]}
         line["rows"] = rows
