@@ -527,36 +527,52 @@ def run_group_indexer(args, dist):
     return dict(ms=ms, launches=launches, groups=ng, act_bytes=act, flops=flops)
 
 
-def run_chunked(args, dist):
+def run_chunked(args, dist, dtype="bf16"):
     """256K-token prefill in query chunks of 4096 against the growing causal key cache, flat
-    and in group mode (window bank, G = 64, B = 8192); one step = all 64 chunks."""
+    and in group mode (window bank, G = 64, B = 8192); one step = all 64 chunks. e4m3: q, k
+    and the group queries quantised per token (fp32 scales)."""
     from sparse_attention_token_indexer_b200 import indexer, inputs
     c = CHUNKED
     S, ch, G = c["S"], c["chunk"], c["G"]
     st = inputs.AnchorStructure(c["d"], c["seed"], "cuda")
-    k = st.keys(S).to(torch.bfloat16).contiguous()
+    kf = st.keys(S)
     q = torch.empty(S, c["H"], c["d"], dtype=torch.bfloat16, device="cuda")
     for c0 in range(0, S, 16384):  # generate in slices to bound the fp32 temporaries
         q[c0:c0 + 16384] = st.queries(16384, c["H"], pos0=c0).to(torch.bfloat16)
     w = st.gates(S, c["H"])
     qbar, wbar = inputs.mean_pool_group_queries(q, w, G, c["Hg"])
-    qbar = qbar.to(torch.bfloat16).contiguous()
+    qs = ks = qbs = None
+    if dtype == "e4m3":
+        k, ks = inputs.quantize_e4m3_rows(kf)
+        qc = torch.empty(S, c["H"], c["d"], dtype=torch.uint8, device="cuda")
+        qs = torch.empty(S, dtype=torch.float32, device="cuda")
+        for c0 in range(0, S, 16384):
+            qc[c0:c0 + 16384], qs[c0:c0 + 16384] = inputs.quantize_e4m3_rows(q[c0:c0 + 16384])
+        q = qc
+        qbar, qbs = inputs.quantize_e4m3_rows(qbar)
+    else:
+        k = kf.to(torch.bfloat16).contiguous()
+        qbar = qbar.to(torch.bfloat16).contiguous()
+    del kf
     ws = indexer.Workspace("cuda")
     idx = torch.empty(ch, c["K"], dtype=torch.int32, device="cuda")
     gpc = ch // G
 
     def flat_pass():
         for c0 in range(0, S, ch):
-            _call_prefill({"q": q[c0:c0 + ch], "w": w[c0:c0 + ch], "k": k, "q_scale": None,
-                           "k_scale": None, "q_pos0": c0}, c["K"], idx, ws)
+            _call_prefill({"q": q[c0:c0 + ch], "w": w[c0:c0 + ch], "k": k,
+                           "q_scale": None if qs is None else qs[c0:c0 + ch], "k_scale": ks,
+                           "q_pos0": c0}, c["K"], idx, ws)
 
     def group_pass():
         for c0 in range(0, S, ch):
             g0 = c0 // G
             bank = indexer.group_bank(qbar[g0:g0 + gpc], wbar[g0:g0 + gpc], k, G, c["B"],
-                                      "window", q_pos0=c0, ws=ws)
+                                      "window", qbar_scale=None if qbs is None else
+                                      qbs[g0:g0 + gpc], k_scale=ks, q_pos0=c0, ws=ws)
             indexer.bank_refine(q[c0:c0 + ch], w[c0:c0 + ch], k, bank, G, c["B"], "window",
-                                c["K"], q_pos0=c0, ws=ws)
+                                c["K"], q_scale=None if qs is None else qs[c0:c0 + ch],
+                                k_scale=ks, q_pos0=c0, ws=ws)
 
     ms_flat, l_flat = timed(flat_pass, 1, args.warmup, dist)
     ms_grp, l_grp = timed(group_pass, 1, args.warmup, dist)
@@ -621,7 +637,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--case", default="flat", choices=["flat", "flat_small", "decode", "mtp",
                                                       "group_indexer", "hisa", "hisa_small",
-                                                      "hisa_decode", "decode_cycle"],
+                                                      "hisa_decode", "decode_cycle", "chunked"],
                     help="flat_small: T = 8192, for profiler captures; decode, mtp, "
                          "group_indexer, hisa, hisa_decode, decode_cycle: that workload alone "
                          "(with --quick); hisa_small: HISA prefill at T = 16384")
@@ -681,6 +697,16 @@ def main():
                               "stage_ms": dcd["stages"],
                               "hbm_gbs": dcd["bytes_flat"] / (dcd["ms_flat"] * 1e-3) / 1e9,
                               "gpu_launches": dcd["launches_flat"]}), flush=True)
+        dist.close()
+        return
+    if args.case == "chunked" and args.quick:
+        out = {}
+        for dt in ("bf16", "e4m3"):
+            ck = run_chunked(args, dist, dt)
+            out[dt] = {"flat_ms": ck["ms_flat"], "group_ms": ck["ms_group"]}
+            del ck
+        if dist.rank == 0:
+            print(json.dumps({"case": "chunked", **out}), flush=True)
         dist.close()
         return
     if args.case == "decode_cycle" and args.quick:
@@ -796,6 +822,15 @@ def main():
             "scores_per_s": (ck["scan"] + ck["refine"]) / (ck["ms_group"] * 1e-3),
             "topk_queries_per_s": ck["rows"] / (ck["ms_group"] * 1e-3),
             "speedup_vs_flat": ck["ms_flat"] / ck["ms_group"], "gpu_launches": ck["l_group"]}
+        del ck
+        c8 = run_chunked(args, dist, "e4m3")
+        rows["chunked_prefill_S262144_e4m3"] = {
+            "flat_ms_per_pass": c8["ms_flat"], "group_ms_per_pass": c8["ms_group"],
+            "flat_scores_per_s": c8["pairs"] / (c8["ms_flat"] * 1e-3),
+            "flat_tflops": c8["pairs"] * 2 * CHUNKED["H"] * CHUNKED["d"]
+            / (c8["ms_flat"] * 1e-3) / 1e12,
+            "group_speedup_vs_flat": c8["ms_flat"] / c8["ms_group"],
+            "gpu_launches": c8["l_flat"] + c8["l_group"]}
         mt = run_mtp(args, dist)
         rows[f"mtp_round_Bs32_N131072_m{MTP['m']}_G{MTP['G']}_P{MTP['P']}"] = {
             "ms_per_round": mt["ms"], "scan_pairs": mt["scan"], "refine_pairs": mt["refine"],

@@ -97,10 +97,12 @@ def test_other_head_counts(H, d):
     _check_flat(p, idx, sc, range(p["T"]), f"H={H} d={d}")
 
 
-def test_chunked_prefill_with_offset():
-    p = _to_cuda(inputs.anchor_prefill(700, H=64, d=128, K=512, seed=13, S=3000))
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_chunked_prefill_with_offset(dtype):
+    p = _to_cuda(inputs.anchor_prefill(700, H=64, d=128, K=512, seed=13, S=3000, dtype=dtype))
     assert p["q_pos0"] == 2300
-    idx, sc, _ = indexer.index_prefill(p["q"], p["w"], p["k"], p["K"], q_pos0=p["q_pos0"],
+    idx, sc, _ = indexer.index_prefill(p["q"], p["w"], p["k"], p["K"], q_scale=p["q_scale"],
+                                       k_scale=p["k_scale"], q_pos0=p["q_pos0"],
                                        with_scores=True)
     _check_flat(p, idx, sc, _rows_sample(700, 512), "chunk")
 
@@ -447,20 +449,30 @@ def test_bank_rows_starting_past_a_select_class(q_pos0):
                    score_floor(qb64[g], wb64[g], keys), B, RTOL["bf16"], what=f"bank {g}")
 
 
-@pytest.mark.parametrize("mode", ["window", "paper"])
-def test_group_mode_on_a_later_chunk(mode):
+@pytest.mark.parametrize("mode,dtype", [("window", "bf16"), ("paper", "bf16"),
+                                        ("window", "e4m3"), ("paper", "e4m3")])
+def test_group_mode_on_a_later_chunk(mode, dtype):
     """Group mode for one query chunk of a longer prefix (q_pos0 > 0), as chunked prefill
-    runs it; includes an incomplete trailing group."""
+    runs it; includes an incomplete trailing group; bf16 and e4m3 operands."""
     S, T, q_pos0, G, B, K, Hg = 3000, 64 * 9 + 21, 2300, 64, 512, 128, 16
     p = _to_cuda(inputs.anchor_prefill(T, H=64, d=128, K=K, seed=23, S=S, q_pos0=q_pos0))
     qbar, wbar = inputs.mean_pool_group_queries(p["q"].float(), p["w"], G, Hg)
-    qbar = qbar.to(torch.bfloat16).contiguous()
-    bank = indexer.group_bank(qbar, wbar, p["k"], G, B, mode, q_pos0=q_pos0)
-    idx, sc = indexer.bank_refine(p["q"], p["w"], p["k"], bank, G, B, mode, K, q_pos0=q_pos0,
+    qbs = None
+    if dtype == "e4m3":
+        p.update(inputs.as_operands(p["q"].float(), p["k"].float(), "e4m3"))
+        qbar, qbs = inputs.quantize_e4m3_rows(qbar)
+    else:
+        qbar = qbar.to(torch.bfloat16).contiguous()
+    bank = indexer.group_bank(qbar, wbar, p["k"], G, B, mode, qbar_scale=qbs,
+                              k_scale=p["k_scale"], q_pos0=q_pos0)
+    idx, sc = indexer.bank_refine(p["q"], p["w"], p["k"], bank, G, B, mode, K,
+                                  q_scale=p["q_scale"], k_scale=p["k_scale"], q_pos0=q_pos0,
                                   with_scores=True)
     torch.cuda.synchronize()
-    q64, k64, w64 = f64(p["q"]), f64(p["k"]), p["w"].double().cpu().numpy()
-    qb64, wb64 = f64(qbar), wbar.double().cpu().numpy()
+    q64, k64 = f64(p["q"], p["q_scale"]), f64(p["k"], p["k_scale"])
+    w64 = p["w"].double().cpu().numpy()
+    qb64, wb64 = f64(qbar, qbs), wbar.double().cpu().numpy()
+    rtol = RTOL[dtype]
     bank, idx, sc = bank.cpu().numpy(), idx.cpu().numpy(), sc.cpu().numpy()
     bank_k = B if mode == "paper" else B - G
     for g in range(T // G):
@@ -468,7 +480,7 @@ def test_group_mode_on_a_later_chunk(mode):
         scan_n = a + 1 if mode == "paper" else a
         keys = k64[:scan_n]
         check_topk(bank[g, :bank_k], np.arange(scan_n), ox.score_keys(qb64[g], wb64[g], keys),
-                   score_floor(qb64[g], wb64[g], keys), bank_k, RTOL["bf16"], what=f"bank {g}")
+                   score_floor(qb64[g], wb64[g], keys), bank_k, rtol, what=f"bank {g}")
         lo = a + 1 if mode == "paper" else a
         scan_part = bank[g, :bank_k][bank[g, :bank_k] >= 0]
         for r in range(g * G, g * G + G, 5):
@@ -476,12 +488,12 @@ def test_group_mode_on_a_later_chunk(mode):
             cand = np.union1d(scan_part, np.arange(lo, i + 1))
             cand = cand[cand <= i]
             check_topk(idx[r], cand, ox.score_keys(q64[r], w64[r], k64[cand]),
-                       score_floor(q64[r], w64[r], k64[cand]), K, RTOL["bf16"], sc[r],
+                       score_floor(q64[r], w64[r], k64[cand]), K, rtol, sc[r],
                        f"refine row {r}")
     for r in range(T // G * G, T):
         n = q_pos0 + r + 1
         check_topk(idx[r], np.arange(n), ox.score_keys(q64[r], w64[r], k64[:n]),
-                   score_floor(q64[r], w64[r], k64[:n]), K, RTOL["bf16"], sc[r], f"tail {r}")
+                   score_floor(q64[r], w64[r], k64[:n]), K, rtol, sc[r], f"tail {r}")
 
 
 # ---------------------------------------------------------------------------------------
