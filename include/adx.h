@@ -9,13 +9,18 @@
  *   selection  T_t = TopK_{s <= pos(t)} I[t,s]                        (§3, Eq. (2))
  *   bank       P = TopK over the group query's scores of a scan      (§4.3, Eq. (13))
  *   refine     T_i = TopK_{s in C_i} I[i,s], C_i = bank U post-anchor (§4.3, Eq. (14))
+ *   group indexer  q-bar, w-bar from pooled query latents and hidden states (§4.2, Eqs. (6)-(7))
+ *   HISA       block Top-n over mean-pooled 128-key blocks, then Top-K of the kept blocks'
+ *              tokens ("HISA: Efficient Hierarchical Indexing for Fine-Grained Sparse
+ *              Attention", arXiv 2603.28458v3; ADIndex Appendix C.5)
  *
  * Conventions shared by every entry point
  *  - Every pointer argument is a DEVICE pointer unless stated otherwise. The caller owns
  *    all memory; the library allocates nothing, keeps no state between calls besides
- *    cached device properties (and, for adx_index_prefill_host, two copy streams and their
- *    events per device, created on first use), and launches all work asynchronously on `stream` (a
- *    cudaStream_t passed as void*; NULL = the legacy default stream).
+ *    cached device properties (and, created on first use per device: two copy streams and
+ *    their events for adx_index_prefill_host, a cuBLAS handle for adx_group_indexer_queries),
+ *    and launches all work asynchronously on `stream` (a cudaStream_t passed as void*;
+ *    NULL = the legacy default stream).
  *  - Argument errors are detected on the host and returned before any launch.
  *  - Errors the device detects (a bounded wait that ran out) are recorded in a status word
  *    at the start of the workspace and reported by adx_read_device_status(). The word is
