@@ -132,7 +132,7 @@ void plan_split(int64_t rows, int64_t n, int K, int& n_seg, int& seg_len) {
   n_seg = 1;
   seg_len = static_cast<int>(std::min<int64_t>(n, INT32_MAX));
   const int sms = std::max(sm_count(), 1);
-  if (rows >= sms || n < 8ll * K) return;
+  if (rows >= sms || n < 8ll * K || n <= kWarpSelectMax) return;
   const int64_t want = (2ll * sms + rows - 1) / rows;
   const int64_t most = n / (4ll * K);
   // keep the second stage (n_seg * K candidates per row) inside the register-resident select,

@@ -112,6 +112,10 @@ struct SelectArgs {
   DeviceStatus* status;
 };
 
+// Longest row the one-warp-per-row select holds (32 lanes x 40 keys); launches whose rows all
+// fit (and are not split into segments) take it.
+constexpr int64_t kWarpSelectMax = 32 * 40;
+
 // Launchers (return a cudaError_t from the launch).
 cudaError_t launch_score(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const ScoreArgs& a,
                          bool fp8, int H, int d, int tok, int grid, cudaStream_t s);

@@ -776,6 +776,100 @@ select_reg_kernel(const SelectArgs a, int row0) {
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// Short rows (up to 32 x ITEMS elements, e.g. the block rows of the hierarchical indexer):
+// one warp per row. Lane l holds elements j*32 + l (coalesced loads). The K-th largest key
+// is found bit by bit below the row's common high bits (a warp-wide count of keys at or
+// above each candidate); the keys above it and the lowest-indexed keys equal to it are
+// written in ascending index order, slots from ballot prefix counts.
+// ---------------------------------------------------------------------------------------
+constexpr int kWarpSelRows = 8;  // rows (warps) per CTA
+
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+template <int ITEMS>
+__global__ void __launch_bounds__(32 * kWarpSelRows) select_warp_kernel(const SelectArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int r = static_cast<int>(blockIdx.x) * kWarpSelRows + static_cast<int>(threadIdx.x >> 5);
+  if (r >= a.rows) return;  // the whole warp
+  const int64_t n = row_length(a, r);
+  const float* vals = a.vals + static_cast<int64_t>(r) * a.ld;
+  const int32_t* in_idx = a.in_idx ? a.in_idx + static_cast<int64_t>(r) * a.ld : nullptr;
+  const int32_t* map =
+      a.idx_map ? a.idx_map + static_cast<int64_t>(r / a.rows_per_batch) * a.map_stride : nullptr;
+  const int64_t out_base = static_cast<int64_t>(r) * a.out_ld;
+  const uint32_t K = static_cast<uint32_t>(a.K);
+  uint32_t key[ITEMS];
+  uint32_t nval = 0, kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+  for (int j = 0; j < ITEMS; ++j) {
+    const int64_t i = static_cast<int64_t>(j) * 32 + lane;
+    const float v = i < n ? vals[i] : -INFINITY;
+    const bool ok = is_valid(v);
+    key[j] = ok ? order_key(v) : 0u;  // 0 = invalid (valid keys are > 0)
+    nval += ok;
+    kmin = ok ? min(kmin, key[j]) : kmin;
+    kmax = max(kmax, key[j]);
+  }
+  nval = __reduce_add_sync(0xffffffffu, nval);
+  const bool take_all = nval <= K;
+  uint32_t theta = 1u, need_eq = 0u;
+  if (!take_all) {
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    const uint32_t diff = kmin ^ kmax;
+    const int hb = diff == 0u ? 0 : 32 - __clz(diff);  // bits hb.. are common to every key
+    theta = hb >= 32 ? 0u : (kmax >> hb) << hb;        // count(key >= theta) = nval >= K
+    for (int b = hb - 1; b >= 0; --b) {
+      const uint32_t cand = theta | (1u << b);
+      uint32_t c = 0;
+#pragma unroll
+      for (int j = 0; j < ITEMS; ++j) c += key[j] >= cand;
+      if (__reduce_add_sync(0xffffffffu, c) >= K) theta = cand;
+    }
+    uint32_t gt = 0;
+#pragma unroll
+    for (int j = 0; j < ITEMS; ++j) gt += key[j] > theta;
+    need_eq = K - __reduce_add_sync(0xffffffffu, gt);  // >= 1 equal keys to take
+  }
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  uint32_t base = 0, eq_seen = 0;
+#pragma unroll
+  for (int j = 0; j < ITEMS; ++j) {
+    const uint32_t u = key[j];
+    const bool eq = !take_all && u == theta;
+    const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
+    const bool sel = take_all ? u != 0u : (u > theta || (eq && eq_seen + __popc(eqb & lt_mask) < need_eq));
+    eq_seen += __popc(eqb);
+    const uint32_t sb = __ballot_sync(0xffffffffu, sel);
+    if (sel) {
+      const uint32_t slot = base + __popc(sb & lt_mask);
+      const int32_t i = j * 32 + lane;
+      int32_t id = in_idx ? in_idx[i] : i;
+      id = map_id(map, id, a.map_shift);
+      a.out_idx[out_base + slot] = id;
+      if (a.out_val) a.out_val[out_base + slot] = key_value(u);
+    }
+    base += __popc(sb);
+  }
+  for (uint32_t sl = base + lane; sl < K; sl += 32) {
+    a.out_idx[out_base + sl] = -1;
+    if (a.out_val) a.out_val[out_base + sl] = -INFINITY;
+  }
+}
+
+static_assert(kWarpSelectMax == 32 * 40, "the widest warp select instance");
+
+template <int ITEMS>
+cudaError_t launch_warp_select(const SelectArgs& a, cudaStream_t s, int* launched) {
+  const int64_t grid = (static_cast<int64_t>(a.rows) + kWarpSelRows - 1) / kWarpSelRows;
+  select_warp_kernel<ITEMS><<<static_cast<unsigned>(grid), 32 * kWarpSelRows, 0, s>>>(a);
+  *launched = 1;
+  return cudaGetLastError();
+}
+
 template <int THREADS, int DIGIT, int ITEMS = kRegItems>
 cudaError_t launch_reg(const SelectArgs& a, int row0, int row1, cudaStream_t s, int* launched) {
   const int64_t grid = static_cast<int64_t>(row1 - row0) * a.n_seg;
@@ -849,6 +943,12 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launched) {
   constexpr int64_t cap[NC] = {128 * kRegItems, 256 * kRegItems, 256 * kWideItems,
                                512 * kRegItems};
   constexpr int64_t c1024 = 1024 * kRegItems;
+  if (a.n_seg == 1 && seg <= kWarpSelectMax) {  // short rows: one warp per row
+    if (seg <= 32 * 8) return launch_warp_select<8>(a, s, launched);
+    if (seg <= 32 * 16) return launch_warp_select<16>(a, s, launched);
+    if (seg <= 32 * 32) return launch_warp_select<32>(a, s, launched);
+    return launch_warp_select<40>(a, s, launched);
+  }
   if (seg > c1024) {
     select_kernel<<<static_cast<unsigned>(grid), kSelThreads, 0, s>>>(a);
     *launched = 1;
