@@ -148,6 +148,36 @@ def test_rows_where_most_scores_are_exactly_zero():
     assert len(zero_rows) >= 5, "the K-th score is 0 in too few sampled rows"
 
 
+@pytest.mark.parametrize("S,K", [(1200, 100), (1200, 700), (250, 37), (1280, 1279)])
+def test_exact_ties_short_rows(S, K):
+    """Rows of at most 1280 keys take the one-warp-per-row select. Keys are copies of 24
+    vectors a factor 2 apart (exact scores in a fixed order, many equal at the K-th); its set
+    must be the oracle's exactly, in ascending positions, with exact scores."""
+    T, nd, big = 64, 24, 5
+    p = inputs.anchor_prefill(T, H=64, d=128, K=K, seed=19, device="cuda", S=S)
+    rng = np.random.default_rng(11)
+    which = np.where(rng.random(S) < 0.5, big, rng.integers(0, nd, S))
+    scales = torch.tensor([2.0 ** (nd - 13 - i) for i in range(nd)])
+    v = p["k"][0].float().cpu()
+    distinct = (scales[:, None] * v[None, :]).to(torch.bfloat16)
+    k = distinct[torch.as_tensor(which)].contiguous().cuda()
+    idx, sc, _ = indexer.index_prefill(p["q"], p["w"], k, K, q_pos0=p["q_pos0"],
+                                       with_scores=True)
+    idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+    q64, w64, d64 = f64(p["q"]), p["w"].double().cpu().numpy(), f64(distinct)
+    for t in range(T):
+        vals = ox.score_keys(q64[t], w64[t], d64)
+        n = p["q_pos0"] + t + 1
+        row = vals[which[:n]]
+        order = np.lexsort((np.arange(n), -row))
+        m = min(K, n)
+        assert set(idx[t][:m].tolist()) == set(order[:m].tolist()), f"row {t}"
+        assert np.all(idx[t][m:] == -1) and np.all(np.diff(idx[t][:m]) > 0)
+        keys = d64[which[idx[t][:m]]]
+        check_scores(sc[t][:m], row[idx[t][:m]], score_floor(q64[t], w64[t], keys),
+                     RTOL["bf16"], f"row {t} scores")
+
+
 def test_exact_ties_take_the_lowest_positions():
     """Every key is one of 24 copies of one vector scaled by powers of two (exact in bf16 and
     in every product), so each query's scores take 24 exact values in a fixed order, a factor
