@@ -232,7 +232,7 @@ adx_status adx_index_mtp(const adx_operands* full, const adx_operands* grp, int3
                          int32_t P, int32_t K, int32_t* topk_idx, float* topk_score,
                          int32_t* bank_out, void* ws, size_t ws_bytes, void* stream);
 
-/* Training-free group queries: the proxy of the PIVOT baseline the pages compare with
+/* Training-free group queries: the proxy of the PIVOT baseline the paper compares with
  * (ADIndex, Appendix B, "PIVOT": the group's indexing queries and gates, mean-pooled). For
  * every complete group of G consecutive rows (g < T/G) of q [T, H, d] (bf16, or e4m3 codes
  * with q_scale [T]) and w [T, H]:

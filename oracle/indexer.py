@@ -256,7 +256,7 @@ def group_union_sizes(topk_rows, G):
 # ---------------------------------------------------------------------------------------
 
 def mean_pool_group(q, w, G, Hg):
-    """The proxy group query of the PIVOT baseline the pages compare with (ADIndex,
+    """The proxy group query of the PIVOT baseline the paper compares with (ADIndex,
     Appendix B, "PIVOT"): per group of G consecutive rows, the member mean of each indexing
     head and of its gate, for the first Hg heads. q [T, H, d], w [T, H] (float64) ->
     qbar [T // G, Hg, d], wbar [T // G, Hg]; an incomplete trailing group gets none."""
@@ -277,7 +277,7 @@ def mean_pool_group(q, w, G, Hg):
 def rope(x, pos, rope_dim=64, base=10000.0):
     """Rotary position embedding at position pos of one head vector x [d]: the pairs
     (x[2i], x[2i+1]), i < rope_dim/2, are rotated by the angle pos * base^(-2i/rope_dim); the
-    other dimensions are left as they are (reading: the pages name RoPE at the group anchor
+    other dimensions are left as they are (reading: the paper names RoPE at the group anchor
     without its layout; this is the interleaved-pair form over the first rope_dim dims)."""
     y = np.array(x, dtype=np.float64)
     if rope_dim > y.shape[0] or rope_dim % 2:

@@ -3,7 +3,7 @@
 For one layer, the original indexer's Top-K sets of calibration queries give the bank
 capacity a group size needs (Eq. (4): the union of the Top-K sets of G consecutive queries),
 and the reuse configuration is the (G, P) with the largest scoring speedup whose budget P
-holds that capacity (Eq. (5)). The speedup S(G, P; L) is the pages' joint one (Appendix A,
+holds that capacity (Eq. (5)). The speedup S(G, P; L) is the paper's joint one (Appendix A,
 Table 5 panel c): prefill of L tokens plus R = 32 MTP verification rounds of m = 16 queries,
 round j's first query seeing L + (j-1)*8 keys, every score evaluation counted once whatever
 the number of heads. The union sizes are computed on the GPU (adx_group_union_sizes); the
@@ -36,7 +36,7 @@ def union_sizes(topk_idx, G, S, stream=None):
 
 
 def capacity(unions, criterion="max"):
-    """Bank capacity a layer needs from its union sizes: the maximum (the pages' default),
+    """Bank capacity a layer needs from its union sizes: the maximum (the paper's default),
     the 90th percentile or the mean (the relaxed criteria)."""
     u = np.asarray(unions, dtype=np.float64)
     if u.size == 0:

@@ -1,5 +1,5 @@
 """Layer-wise reuse calibration (ADIndex §4.1): the speedup S(G, P; L) against the oracle's
-plan counts and the pages' Table 5 panel c, the configuration choice of Eq. (5) against a
+plan counts and the paper's Table 5 panel c, the configuration choice of Eq. (5) against a
 brute-force search, the capacity criteria, and (GPU) the union sizes of Eq. (4) against the
 oracle on the indexer's own Top-K output."""
 
