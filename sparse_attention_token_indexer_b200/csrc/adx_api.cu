@@ -164,12 +164,17 @@ size_t ws_prepare(const adx_operands* o, int64_t R) {
 
 // R rows of q / q_scale / w starting at the given pointers.
 adx_status prepare(const adx_operands* o, const void* q, const float* q_scale, const float* w,
-                   int64_t R, Carve& cv, cudaStream_t s, Prepared& out) {
+                   int64_t R, Carve& cv, cudaStream_t s, Prepared& out,
+                   int32_t* row_blk = nullptr) {
   const bool in8 = o->q_dtype == ADX_E4M3, out8 = fp8_keys(o);
   void* qo = cv.take<uint8_t>(static_cast<size_t>(R) * o->H * o->d * (out8 ? 1 : 2));
   float* so = out8 ? cv.take<float>(static_cast<size_t>(R) * 4) : nullptr;
   int8_t* fl = cv.take<int8_t>(static_cast<size_t>(R));
-  if (counted(launch_prepare_q(q, q_scale, in8, out8, w, R, o->H, o->d, qo, so, fl, s)) !=
+  RowBlocks rb;
+  rb.out = row_blk;
+  rb.q_pos0 = o->q_pos0;
+  rb.seq_len = o->seq_len;
+  if (counted(launch_prepare_q(q, q_scale, in8, out8, w, R, o->H, o->d, qo, so, fl, s, rb)) !=
       cudaSuccess)
     return ADX_ECUDA;
   out.q = qo;
@@ -1119,15 +1124,13 @@ adx_status adx_index_hisa(const adx_operands* o, const void* kbar, const float* 
   const int32_t nc = n_blocks * kTileM;
   Carve cv(ws);
   DeviceStatus* st = cv.take<DeviceStatus>(kStatusBytes);
-  Prepared pq;
-  if ((r = prepare(o, o->q, o->q_scale, o->w, T, cv, s, pq)) != ADX_OK) return r;
   int32_t* row_blk = cv.take<int32_t>(static_cast<size_t>(T) * 4);
+  Prepared pq;  // the preparation also writes each row's block
+  if ((r = prepare(o, o->q, o->q_scale, o->w, T, cv, s, pq, row_blk)) != ADX_OK) return r;
   float* bsc = cv.take<float>(static_cast<size_t>(T) * ldb * 4);
   int32_t* blocks =
       blocks_out ? blocks_out : cv.take<int32_t>(static_cast<size_t>(T) * n_blocks * 4);
   float* tsc = cv.take<float>(static_cast<size_t>(T) * nc * 4);
-  if (counted(launch_row_blocks(T, o->q_pos0, o->seq_len, row_blk, s)) != cudaSuccess)
-    return ADX_ECUDA;
 
   // 1. block scores: Eq. (1) on the block keys, block b visible to a row whose position lies
   //    in block >= b
@@ -1155,11 +1158,18 @@ adx_status adx_index_hisa(const adx_operands* o, const void* kbar, const float* 
     finish_plan(p, (vis_blocks + kTileM - 1) / kTileM);
     if ((r = run_score(p, pq.q, kbar, (decode ? T : 1) * nbmax, s)) != ADX_OK) return r;
   }
-  // 2. forced blocks, then the block Top-n
-  if (counted(launch_force_blocks(bsc, ldb, T, row_blk, n_blocks, s)) != cudaSuccess)
+  // 2. forced blocks, then the block Top-n; rows that fit the one-warp select get the forced
+  //    blocks there, longer ones from a kernel that raises their scores first
+  const bool warp_rows = nbmax <= kWarpSelectMax;
+  if (!warp_rows &&
+      counted(launch_force_blocks(bsc, ldb, T, row_blk, n_blocks, s)) != cudaSuccess)
     return ADX_ECUDA;
   {
     SelectArgs sa{};
+    if (warp_rows) {
+      sa.force_blk = row_blk;
+      sa.force_n = n_blocks;
+    }
     sa.vals = bsc;
     sa.ld = ldb;
     sa.rows_per_batch = 1;

@@ -99,6 +99,10 @@ struct SelectArgs {
   const int32_t* row_pos;
   int32_t len_off;
   int32_t len_mul;
+  // Forced elements (one-warp select only): on a row r with force_blk[r] + 1 > force_n,
+  // elements 0 and force_blk[r] count as +inf (HISA's first and own block). Null: none.
+  const int32_t* force_blk;
+  int32_t force_n;
   // with idx_map: 0 -> element c maps to map[c]; s > 0 -> to (map[c >> s] << s) + (c & (2^s - 1))
   // (the map lists blocks of 2^s consecutive positions)
   int32_t map_shift;
@@ -166,9 +170,17 @@ cudaError_t launch_fill_post_anchor(int32_t* bank, int32_t n_groups, int32_t ban
 int score_blocks_per_sm(bool fp8, int H, int d, int tok);
 // Writes the prepared query rows (gate-folded where all gates are >= 0, else as given), with
 // fold flags and, for e4m3 output, one scale per row.
+// Optional by-product of the query preparation: out[r] = block (of kTileM positions) of row
+// r's position, q_pos0 + r, or seq_len[r] - 1 when seq_len is set.
+struct RowBlocks {
+  int32_t* out = nullptr;
+  int64_t q_pos0 = 0;
+  const int32_t* seq_len = nullptr;
+};
 cudaError_t launch_prepare_q(const void* q, const float* q_scale, bool in_e4m3, bool out_e4m3,
                              const float* w, int64_t rows, int H, int d, void* q_out,
-                             float* q_scale_out, int8_t* fold_flag, cudaStream_t s);
+                             float* q_scale_out, int8_t* fold_flag, cudaStream_t s,
+                             RowBlocks rb = RowBlocks{});
 
 // HISA block keys: the mean of each 128-key block of each key range (n_seq ranges of S rows;
 // length seq_len[b], or len_fixed without seq_len), stored like keys in kbar [n_seq, nbmax, d]
@@ -177,9 +189,6 @@ cudaError_t launch_prepare_q(const void* q, const float* q_scale, bool in_e4m3, 
 cudaError_t launch_block_keys(const void* k, const float* k_scale, bool fp8, int64_t S, int d,
                               int32_t n_seq, const int32_t* seq_len, int32_t len_fixed,
                               bool last_only, int32_t nbmax, void* kbar, float* kbar_scale,
-                              cudaStream_t s);
-// row_blk[r] = block of row r's position (q_pos0 + r, or seq_len[r] - 1 when seq_len is set).
-cudaError_t launch_row_blocks(int32_t R, int64_t q_pos0, const int32_t* seq_len, int32_t* row_blk,
                               cudaStream_t s);
 // Union of the block lists (blocks [R, n_blocks], -1 padded) of each group of `tok`
 // consecutive rows: uni [groups, tok * n_blocks] distinct blocks, count [groups] how many,

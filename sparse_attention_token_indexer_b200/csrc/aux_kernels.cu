@@ -172,10 +172,15 @@ template <bool IN_E4M3, bool OUT_E4M3, int THREADS>
 __global__ void __launch_bounds__(THREADS)
 prepare_q_kernel(const void* __restrict__ q_in, const float* __restrict__ q_scale_in,
                  const float* __restrict__ w, int H, int d, void* __restrict__ q_out,
-                 float* __restrict__ q_scale_out, int8_t* __restrict__ fold_flag) {
+                 float* __restrict__ q_scale_out, int8_t* __restrict__ fold_flag,
+                 RowBlocks rb) {
   constexpr int G = 1024 / THREADS;
   __shared__ float red[THREADS / 32];
   const int64_t r = blockIdx.x;
+  if (rb.out != nullptr && threadIdx.x == 0) {
+    const int64_t p = rb.seq_len != nullptr ? static_cast<int64_t>(rb.seq_len[r]) - 1 : rb.q_pos0 + r;
+    rb.out[r] = static_cast<int32_t>(p < 0 ? -1 : p / kTileM);
+  }
   const float* wr = w + r * H;
   const int ng = H * d / 8;  // groups of 8 elements; a group lies within one head
   const int64_t base = r * static_cast<int64_t>(H) * d;
@@ -285,7 +290,7 @@ group_mean_kernel(const void* __restrict__ q, const float* __restrict__ q_scale,
 template <bool IN_E4M3, bool OUT_E4M3>
 cudaError_t launch_prepare_rows(const void* q, const float* q_scale, const float* w, int64_t rows,
                                 int H, int d, void* q_out, float* q_scale_out, int8_t* fold_flag,
-                                cudaStream_t s) {
+                                RowBlocks rb, cudaStream_t s) {
   // few rows (decode): spread each row over more threads
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -294,10 +299,10 @@ cudaError_t launch_prepare_rows(const void* q, const float* q_scale, const float
   const unsigned g = static_cast<unsigned>(rows);
   if (rows < 2ll * sms)
     prepare_q_kernel<IN_E4M3, OUT_E4M3, 1024>
-        <<<g, 1024, 0, s>>>(q, q_scale, w, H, d, q_out, q_scale_out, fold_flag);
+        <<<g, 1024, 0, s>>>(q, q_scale, w, H, d, q_out, q_scale_out, fold_flag, rb);
   else
     prepare_q_kernel<IN_E4M3, OUT_E4M3, 256>
-        <<<g, 256, 0, s>>>(q, q_scale, w, H, d, q_out, q_scale_out, fold_flag);
+        <<<g, 256, 0, s>>>(q, q_scale, w, H, d, q_out, q_scale_out, fold_flag, rb);
   return cudaGetLastError();
 }
 
@@ -305,18 +310,18 @@ cudaError_t launch_prepare_rows(const void* q, const float* q_scale, const float
 
 cudaError_t launch_prepare_q(const void* q, const float* q_scale, bool in_e4m3, bool out_e4m3,
                              const float* w, int64_t rows, int H, int d, void* q_out,
-                             float* q_scale_out, int8_t* fold_flag, cudaStream_t s) {
+                             float* q_scale_out, int8_t* fold_flag, cudaStream_t s, RowBlocks rb) {
   if (rows <= 0) return cudaSuccess;
   if (static_cast<int64_t>(H) * d > 8192 || d % 8 != 0) return cudaErrorNotSupported;
   if (!in_e4m3 && !out_e4m3)
     return launch_prepare_rows<false, false>(q, q_scale, w, rows, H, d, q_out, q_scale_out,
-                                             fold_flag, s);
+                                             fold_flag, rb, s);
   if (in_e4m3 && out_e4m3)
     return launch_prepare_rows<true, true>(q, q_scale, w, rows, H, d, q_out, q_scale_out,
-                                           fold_flag, s);
+                                           fold_flag, rb, s);
   if (!in_e4m3 && out_e4m3)
     return launch_prepare_rows<false, true>(q, q_scale, w, rows, H, d, q_out, q_scale_out,
-                                            fold_flag, s);
+                                            fold_flag, rb, s);
   return cudaErrorNotSupported;
 }
 

@@ -4,8 +4,9 @@
 // block and the query's own block always among the candidates.
 //   * block keys: the mean of each block of 128 keys (decoded with their scales for e4m3),
 //     stored like keys (bf16, or e4m3 with a per-block scale amax / 448);
-//   * row blocks: the block holding each query row's position;
-//   * forcing: the two forced blocks' scores raised to +inf ahead of the block Top-n.
+//   * forcing: the two forced blocks' scores raised to +inf ahead of the block Top-n (for
+//     block rows longer than the one-warp select holds; that select forces them itself).
+// The block of each row's position is a by-product of the query preparation.
 // The block scores, both selections and the token refinement run on the scoring and select
 // kernels (the refinement in their block-list mode).
 #include <cuda_bf16.h>
@@ -78,15 +79,6 @@ block_keys_kernel(const uint8_t* __restrict__ k, const float* __restrict__ k_sca
     if (threadIdx.x < d)
       reinterpret_cast<__nv_bfloat16*>(kbar)[out * d + threadIdx.x] = __float2bfloat16_rn(mean);
   }
-}
-
-// Block of each row's position: prefill rows r at q_pos0 + r, decode rows at seq_len[r] - 1.
-__global__ void row_blocks_kernel(int32_t R, int64_t q_pos0, const int32_t* __restrict__ seq_len,
-                                  int32_t* __restrict__ row_blk) {
-  const int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (r >= R) return;
-  const int64_t p = seq_len != nullptr ? static_cast<int64_t>(seq_len[r]) - 1 : q_pos0 + r;
-  row_blk[r] = static_cast<int32_t>(p < 0 ? -1 : p / kBlk);
 }
 
 // Forced blocks: where more than n_blocks blocks are visible, block 0 and the row's own block
@@ -195,14 +187,6 @@ cudaError_t launch_block_keys(const void* k, const float* k_scale, bool fp8, int
   else
     block_keys_kernel<false><<<grid, kBkThreads, 0, s>>>(kc, k_scale, S, d, seq_len, len_fixed,
                                                          last_only ? 1 : 0, nbmax, out, kbar_scale);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_row_blocks(int32_t R, int64_t q_pos0, const int32_t* seq_len, int32_t* row_blk,
-                              cudaStream_t s) {
-  if (R <= 0) return cudaSuccess;
-  row_blocks_kernel<<<static_cast<unsigned>((R + 255) / 256), 256, 0, s>>>(R, q_pos0, seq_len,
-                                                                          row_blk);
   return cudaGetLastError();
 }
 

@@ -803,10 +803,16 @@ __global__ void __launch_bounds__(32 * kWarpSelRows) select_warp_kernel(const Se
   const uint32_t K = static_cast<uint32_t>(a.K);
   uint32_t key[ITEMS];
   uint32_t nval = 0, kmin = 0xffffffffu, kmax = 0u;
+  int64_t forced = -1;  // besides element 0
+  if (a.force_blk != nullptr) {
+    const int32_t cur = a.force_blk[r];
+    if (cur + 1 > a.force_n) forced = cur;
+  }
 #pragma unroll
   for (int j = 0; j < ITEMS; ++j) {
     const int64_t i = static_cast<int64_t>(j) * 32 + lane;
-    const float v = i < n ? vals[i] : -INFINITY;
+    float v = i < n ? vals[i] : -INFINITY;
+    if (forced >= 0 && (i == 0 || i == forced)) v = INFINITY;
     const bool ok = is_valid(v);
     key[j] = ok ? order_key(v) : 0u;  // 0 = invalid (valid keys are > 0)
     nval += ok;
