@@ -656,7 +656,9 @@ def _check_hisa_row(t, p, q64, w64, k64, kbar64, blocks, idx, sc, n_blocks, K, r
     (1501, 1501, 0, 4, 300, "bf16"), (1203, 1203, 0, 5, 256, "e4m3"),
     (1027, 1400, 373, 2, 200, "bf16"),
     # block rows longer than the one-warp select holds (1329 blocks): forced by a kernel
-    (8, 170000, 169992, 64, 2048, "bf16")])
+    (8, 170000, 169992, 64, 2048, "bf16"),
+    # the largest budget (255 blocks: the union of 4 rows sorts 1020 entries)
+    (11, 40000, 39989, 255, 4096, "bf16")])
 def test_hisa_prefill(T, S, q_pos0, n_blocks, K, dtype):
     """Prefill: 12 to 15 blocks with a partial last one, a chunk whose rows start at
     q_pos0 > 0, a budget that holds every block (the flat indexer then), ragged row groups,
