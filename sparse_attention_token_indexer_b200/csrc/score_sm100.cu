@@ -139,9 +139,21 @@ __device__ __forceinline__ void block_info(const ScoreArgs& a, int i, Block& x) 
   x.ntiles = (x.nkeys + kTileM - 1) / kTileM;
 }
 
-// Balanced static partition: all (row block, key tile) pairs laid end to end in schedule
-// order; CTA c owns the tiles [c*W/grid, (c+1)*W/grid). Computed once per CTA by all its
-// threads; returns the first row block touching the range and the tile offset it starts at.
+// Cost of a row block in tile units: its tiles plus a fixed kRowBlockCost for starting it
+// (its query tile's load into the single query buffer after the previous block's last MMA,
+// the gates): without it the CTAs that get the many short row blocks at the end of a causal
+// schedule finish about a quarter later than the rest. Tile t of a block whose costs start at
+// unit cum is unit cum + kRowBlockCost + t.
+constexpr int64_t kRowBlockCost = 2;
+
+__device__ __forceinline__ int64_t block_cost(const Block& x) {
+  return x.ntiles > 0 ? x.ntiles + kRowBlockCost : 0;
+}
+
+// Balanced static partition: all row blocks laid end to end in schedule order, each as its
+// cost units; CTA c owns the units [c*W/grid, (c+1)*W/grid) and scores the tiles whose units
+// it owns. Computed once per CTA by all its threads; returns the first row block touching the
+// range and the unit at which that block's costs start.
 template <class C>
 __device__ __forceinline__ void partition(const ScoreArgs& a, int64_t* scan_s, int64_t& start,
                                           int64_t& end, int& b0, int64_t& base0) {
@@ -154,7 +166,7 @@ __device__ __forceinline__ void partition(const ScoreArgs& a, int64_t* scan_s, i
   for (int i = lo; i < hi; ++i) {
     Block x;
     block_info<C::TOK>(a, i, x);
-    mine += x.ntiles;
+    mine += block_cost(x);
   }
   int64_t incl = mine;
 #pragma unroll
@@ -179,12 +191,12 @@ __device__ __forceinline__ void partition(const ScoreArgs& a, int64_t* scan_s, i
     for (int i = lo; i < hi; ++i) {
       Block x;
       block_info<C::TOK>(a, i, x);
-      if (start < cum + x.ntiles) {
+      if (start < cum + block_cost(x)) {
         scan_s[0] = i;
         scan_s[1] = cum;
         break;
       }
-      cum += x.ntiles;
+      cum += block_cost(x);
     }
   }
   __syncthreads();
@@ -215,9 +227,10 @@ struct WorkIter {
     while (bi < nblocks && cum < end) {
       block_info<TOK>(a, bi, x);
       ++bi;
-      const int64_t lo = max(start - cum, int64_t(0));
-      const int64_t hi = min(end - cum, static_cast<int64_t>(x.ntiles));
-      cum += x.ntiles;
+      const int64_t t0 = cum + kRowBlockCost;  // unit of the block's first tile
+      const int64_t lo = max(start - t0, int64_t(0));
+      const int64_t hi = min(end - t0, static_cast<int64_t>(x.ntiles));
+      cum += block_cost(x);
       if (lo < hi) {
         t_lo = static_cast<int>(lo);
         t_hi = static_cast<int>(hi);
