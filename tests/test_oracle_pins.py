@@ -217,6 +217,68 @@ def test_candidates_stay_causal_and_in_bank():
                     assert banks[gi].max(initial=-1) < plan.scan_n
 
 
+def test_window_group_cost_closed_form():
+    """WINDOW reading (BASELINE's group workload; ADIndex §4.3, Eqs. (13)-(14)): a bank group
+    whose anchor a has at least B - G keys before it scores a scan of the a keys s < a, then
+    member i = a + r (r = 0 .. G-1) scores the B - G bank keys plus its r + 1 window keys
+    a .. a + r: a + G (B - G) + G (G + 1) / 2 in all. With fewer than B - G keys before the
+    anchor the bank holds all a of them instead."""
+    for G, B, a in ((16, 64, 1000), (64, 8192, 65536 - 64), (8, 40, 32), (8, 40, 20)):
+        plans = ox.plan_groups(G, a, G, B, "window")
+        assert len(plans) == 1 and plans[0].kind == "bank"
+        bank = min(B - G, a)
+        assert cost_model.plan_cost(plans, a) == a + G * bank + G * (G + 1) // 2, (G, B, a)
+
+
+def _window_hand_case():
+    """One WINDOW group (G = 4, B = 8, anchor a = 10) with hand-set keys. The group query
+    reads dimension 0, the members' queries dimension 1.
+      group scores: s < a score s + 1, so the scan's best B - G = 4 keys are 9, 8, 7, 6 and
+                    the fifth (rank B - G + 1) is 5; the anchor's own key scores 100, above
+                    every scanned key.
+      member scores: key 5 scores 50 and the anchor's key 60, every other key at most 1.3."""
+    G, B, a, K = 4, 8, 10, 3
+    S = a + G
+    k = np.zeros((S, 4))
+    k[:a, 0] = np.arange(1, a + 1)
+    k[a, 0] = 100.0
+    k[:, 1] = 0.1 * np.arange(S)
+    k[5, 1], k[a, 1] = 50.0, 60.0
+    qbar, wbar = np.array([[[1.0, 0, 0, 0]]]), np.array([[1.0]])
+    q = np.tile(np.array([[0, 1.0, 0, 0], [0, 0.5, 0, 0]]), (G, 1, 1))   # [G, 2, 4]
+    w = np.ones((G, 2))
+    return q, w, k, qbar, wbar, G, B, a, K
+
+
+def test_window_bank_holds_the_anchor_through_the_window_not_the_scan():
+    """The WINDOW scan covers s < a only: the anchor's key, although the group query's best,
+    is not a scanned bank entry; every member still sees it through the window a .. i."""
+    q, w, k, qbar, wbar, G, B, a, K = _window_hand_case()
+    plans = ox.plan_groups(G, a, G, B, "window")
+    bank = ox.token_bank(qbar[0], wbar[0], k, plans[0])
+    assert a not in bank.tolist()
+    got, _ = ox.group_topk(q, w, k, qbar, wbar, a, G, B, K, "window")
+    for r in range(G):
+        assert a in got[r].tolist(), r
+
+
+def test_window_bank_keeps_exactly_B_minus_G_scan_keys():
+    """The WINDOW bank keeps the scan's best B - G keys and not one more: the key of rank
+    B - G + 1 (position 5) stays out of the bank and out of every member's result, although
+    it would be every member's second-best key."""
+    q, w, k, qbar, wbar, G, B, a, K = _window_hand_case()
+    plans = ox.plan_groups(G, a, G, B, "window")
+    bank = ox.token_bank(qbar[0], wbar[0], k, plans[0])
+    assert sorted(bank.tolist()) == [6, 7, 8, 9]
+    got, banks = ox.group_topk(q, w, k, qbar, wbar, a, G, B, K, "window")
+    assert sorted(banks[0].tolist()) == [6, 7, 8, 9]
+    for r in range(G):
+        assert 5 not in got[r].tolist(), r
+    # the same query against the flat indexer does take key 5: the bank is what drops it
+    flat = ox.flat_topk_row(q[G - 1], w[G - 1], k, a + G - 1, K)
+    assert 5 in flat.tolist()
+
+
 def test_paper_fallback_rule():
     plans = ox.plan_groups(T=40, q_pos0=0, G=8, B=16, mode="paper")
     # anchors 0, 8, 16, 24, 32: reuse needs a + 1 > 16; the last group is complete
