@@ -288,6 +288,22 @@ adx_status adx_group_indexer_queries(const adx_group_indexer* gi, int32_t G, voi
 adx_status adx_group_union_sizes(const int32_t* topk_idx, int32_t T, int32_t K, int32_t G,
                                  int32_t S, int32_t* union_out, void* stream);
 
+/* Shared-bank coverage (ADIndex §1, Figure 1(c), and Appendix B.4: the fraction of a query's
+ * original Top-K selections that its group's shared bank includes). For every query row i of
+ * a complete group g = i / G (g < T / G):
+ *   count_out[i] = the number of positions (entries >= 0) in row i of topk_idx [T, K], the
+ *                  original indexer's Top-K (as written by adx_index_prefill);
+ *   hits_out[i]  = how many of them row g of bank_idx [T / G, bank_w] holds (entries < 0 are
+ *                  padding). Pass the bank rows as adx_group_bank writes them: the bank plus
+ *                  the post-anchor (PAPER) or window (WINDOW) positions every member scans,
+ *                  so hits == count exactly when refinement recovers the full Top-K.
+ * coverage_i = hits_out[i] / count_out[i]. Positions must lie in [0, S); larger ones count as
+ * not held. Device pointers; no workspace; S up to 200 KiB of bitmap (6.5M positions), else
+ * ADX_EUNSUPPORTED. */
+adx_status adx_bank_coverage(const int32_t* topk_idx, int32_t T, int32_t K,
+                             const int32_t* bank_idx, int32_t bank_w, int32_t G, int32_t S,
+                             int32_t* hits_out, int32_t* count_out, void* stream);
+
 /* Failure-detection check (no counterpart in the paper): one CTA waits, with the bounded wait
  * the indexer's kernels use, on a barrier that nothing completes; after timeout_ns (at most
  * 1 s) the wait gives up and records ADX_ETIMEOUT in the status word of `ws`, as a real wait

@@ -251,6 +251,27 @@ def group_union_sizes(topk_rows, G):
     return [len(set().union(*rows[g0:g0 + G])) for g0 in range(0, len(rows) - G + 1, G)]
 
 
+def bank_coverage(topk_rows, bank_rows, G):
+    """Shared-bank coverage (ADIndex §1, Figure 1(c), and Appendix B.4): the fraction of a
+    query's original Top-K selections (the flat indexer's, Eq. (2)) that its group's shared
+    bank includes. Query row i belongs to group i // G (complete groups only); a bank row
+    lists the group's candidate positions - the bank of Eq. (13) and the post-anchor or
+    window positions every member scans under Eq. (14) - and -1 is padding, as in a Top-K
+    row. Reading: the post-anchor positions are counted as included, so coverage 1 is
+    exactly the condition under which refinement recovers the full Top-K.
+
+    Returns (hits, count) per row of the complete groups: hits[i] = |T_i n bank_g|,
+    count[i] = |T_i|; coverage_i = hits[i] / count[i]."""
+    hits, count = [], []
+    ng = len(topk_rows) // G
+    for i in range(ng * G):
+        sel = set(int(x) for x in np.asarray(topk_rows[i]).ravel() if int(x) >= 0)
+        bank = set(int(x) for x in np.asarray(bank_rows[i // G]).ravel() if int(x) >= 0)
+        hits.append(len(sel & bank))
+        count.append(len(sel))
+    return np.asarray(hits, np.int64), np.asarray(count, np.int64)
+
+
 # ---------------------------------------------------------------------------------------
 # Training-free group queries
 # ---------------------------------------------------------------------------------------

@@ -23,7 +23,7 @@ EXPORTS = ("adx_abi_version", "adx_bank_width", "adx_status_string", "adx_worksp
            "adx_group_union_sizes", "adx_group_query_mean", "adx_index_prefill_host",
            "adx_check_wait_timeout", "adx_group_indexer_workspace_size",
            "adx_group_indexer_queries", "adx_hisa_block_keys", "adx_hisa_workspace_size",
-           "adx_index_hisa")
+           "adx_index_hisa", "adx_bank_coverage")
 
 
 class Operands(ctypes.Structure):
@@ -90,6 +90,7 @@ def _declare(lib):
         "adx_mtp_workspace_size": (SZ, [P, P, I32, I32, I32, I32]),
         "adx_index_mtp": (ctypes.c_int, [P, P, I32, I32, I32, I32, VP, VP, VP, VP, SZ, VP]),
         "adx_group_union_sizes": (ctypes.c_int, [VP, I32, I32, I32, I32, VP, VP]),
+        "adx_bank_coverage": (ctypes.c_int, [VP, I32, I32, VP, I32, I32, I32, VP, VP, VP]),
         "adx_index_prefill_host": (ctypes.c_int, [P, I32, I32, VP, VP, VP, SZ, VP]),
         "adx_check_wait_timeout": (ctypes.c_int, [VP, ctypes.c_uint64, VP]),
         "adx_hisa_block_keys": (ctypes.c_int, [P, I32, VP, VP, VP]),

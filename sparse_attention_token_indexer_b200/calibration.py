@@ -35,6 +35,36 @@ def union_sizes(topk_idx, G, S, stream=None):
     return out
 
 
+def bank_coverage(topk_idx, bank_idx, G, S, stream=None):
+    """Shared-bank coverage (ADIndex §1, Figure 1(c); Appendix B.4) of the flat Top-K rows
+    topk_idx [T, K] by the group bank rows bank_idx [T // G, W] (device int32, as written by
+    adx_index_prefill and adx_group_bank): (hits, count) [T // G * G] int32 device tensors,
+    coverage of row i = hits[i] / count[i]."""
+    for t in (topk_idx, bank_idx):
+        if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("topk_idx and bank_idx must be contiguous CUDA int32 tensors")
+    T, K = topk_idx.shape
+    n = T // G * G
+    hits = torch.empty(n, dtype=torch.int32, device=topk_idx.device)
+    count = torch.empty(n, dtype=torch.int32, device=topk_idx.device)
+    s = stream if stream is not None else torch.cuda.current_stream(topk_idx.device)
+    L.check("adx_bank_coverage", L.lib().adx_bank_coverage(
+        ctypes.c_void_p(topk_idx.data_ptr()), T, K, ctypes.c_void_p(bank_idx.data_ptr()),
+        bank_idx.shape[1], G, S, ctypes.c_void_p(hits.data_ptr()),
+        ctypes.c_void_p(count.data_ptr()), ctypes.c_void_p(s.cuda_stream)))
+    return hits, count
+
+
+def coverage_by_position(hits, count, G):
+    """Mean coverage at each member position r = 0 .. G-1 of a group, over the groups (the
+    per-position view of Appendix B.4, Figure 4), and its mean over the positions (the
+    layer summary)."""
+    h = np.asarray(hits, dtype=np.float64).reshape(-1, G)
+    c = np.asarray(count, dtype=np.float64).reshape(-1, G)
+    per_pos = (h / np.maximum(c, 1.0)).mean(axis=0)
+    return per_pos, float(per_pos.mean())
+
+
 def capacity(unions, criterion="max"):
     """Bank capacity a layer needs from its union sizes: the maximum (the paper's default),
     the 90th percentile or the mean (the relaxed criteria)."""

@@ -1072,6 +1072,18 @@ adx_status adx_group_union_sizes(const int32_t* topk_idx, int32_t T, int32_t K, 
   return e == cudaSuccess ? ADX_OK : ADX_ECUDA;
 }
 
+adx_status adx_bank_coverage(const int32_t* topk_idx, int32_t T, int32_t K,
+                             const int32_t* bank_idx, int32_t bank_w, int32_t G, int32_t S,
+                             int32_t* hits_out, int32_t* count_out, void* stream) {
+  if (!topk_idx || !bank_idx || !hits_out || !count_out) return ADX_EINVAL;
+  if (T <= 0 || K <= 0 || bank_w <= 0 || G <= 0 || S <= 0) return ADX_EINVAL;
+  if (static_cast<size_t>((S + 31) / 32) * 4 > kUnionMaxBitmapBytes) return ADX_EUNSUPPORTED;
+  const cudaError_t e = counted(launch_bank_coverage(topk_idx, K, bank_idx, bank_w, G, S, T / G,
+                                                     hits_out, count_out,
+                                                     static_cast<cudaStream_t>(stream)));
+  return e == cudaSuccess ? ADX_OK : ADX_ECUDA;
+}
+
 adx_status adx_check_wait_timeout(void* ws, uint64_t timeout_ns, void* stream) {
   if (!ws || timeout_ns == 0 || timeout_ns > 1000000000ull) return ADX_EINVAL;
   const cudaError_t e = counted(launch_wait_timeout(static_cast<DeviceStatus*>(ws), timeout_ns,

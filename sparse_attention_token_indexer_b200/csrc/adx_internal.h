@@ -163,6 +163,11 @@ cudaError_t launch_group_mean(const void* q, const float* q_scale, bool in_e4m3,
 constexpr size_t kUnionMaxBitmapBytes = 200 * 1024;
 cudaError_t launch_union_sizes(const int32_t* topk, int32_t K, int32_t G, int32_t S,
                                int32_t n_groups, int32_t* out, cudaStream_t s);
+// Coverage of each complete group's bank row (bank [n_groups, bank_w]) over the Top-K rows of
+// its G members (topk [n_groups * G, K]): hits = positions found in the bank, count = positions.
+cudaError_t launch_bank_coverage(const int32_t* topk, int32_t K, const int32_t* bank,
+                                 int32_t bank_w, int32_t G, int32_t S, int32_t n_groups,
+                                 int32_t* hits, int32_t* count, cudaStream_t s);
 cudaError_t launch_fill_post_anchor(int32_t* bank, int32_t n_groups, int32_t bank_w,
                                     int32_t first_col, int32_t count, int64_t pos_base,
                                     int32_t pos_step, const int32_t* seq_len, int32_t start_off,

@@ -129,6 +129,45 @@ union_sizes_kernel(const int32_t* __restrict__ topk, int32_t K, int32_t G, int32
   }
 }
 
+// Shared-bank coverage, one CTA per complete group: the group's bank row is marked in a
+// shared-memory bitmap of the S positions, then each warp takes one member row at a time and
+// counts its Top-K positions (entries >= 0) and how many of them the bitmap holds.
+__global__ void __launch_bounds__(256)
+bank_coverage_kernel(const int32_t* __restrict__ topk, int32_t K,
+                     const int32_t* __restrict__ bank, int32_t bank_w, int32_t G, int32_t S,
+                     int32_t* __restrict__ hits, int32_t* __restrict__ count) {
+  extern __shared__ uint32_t bits[];
+  const int nw = (S + 31) / 32;
+  for (int i = threadIdx.x; i < nw; i += blockDim.x) bits[i] = 0u;
+  __syncthreads();
+  const int32_t* brow = bank + static_cast<int64_t>(blockIdx.x) * bank_w;
+  for (int i = threadIdx.x; i < bank_w; i += blockDim.x) {
+    const int32_t v = brow[i];
+    if (v >= 0 && v < S) atomicOr(&bits[v >> 5], 1u << (v & 31));
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = static_cast<int>(blockDim.x >> 5);
+  for (int m = warp; m < G; m += nwarps) {
+    const int64_t r = static_cast<int64_t>(blockIdx.x) * G + m;
+    const int32_t* row = topk + r * K;
+    uint32_t h = 0, c = 0;
+    for (int j = lane; j < K; j += 32) {
+      const int32_t v = row[j];
+      if (v >= 0) {
+        ++c;
+        if (v < S && ((bits[v >> 5] >> (v & 31)) & 1u)) ++h;
+      }
+    }
+    h = __reduce_add_sync(0xffffffffu, h);
+    c = __reduce_add_sync(0xffffffffu, c);
+    if (lane == 0) {
+      hits[r] = static_cast<int32_t>(h);
+      count[r] = static_cast<int32_t>(c);
+    }
+  }
+}
+
 __global__ void fill_post_kernel(int32_t* bank, int32_t n_groups, int32_t bank_w, int32_t first_col,
                                  int32_t count, int64_t pos_base, int32_t pos_step,
                                  const int32_t* seq_len, int32_t start_off) {
@@ -390,6 +429,22 @@ cudaError_t launch_union_sizes(const int32_t* topk, int32_t K, int32_t G, int32_
     if (e != cudaSuccess) return e;
   }
   union_sizes_kernel<<<static_cast<unsigned>(n_groups), 256, smem, s>>>(topk, K, G, S, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bank_coverage(const int32_t* topk, int32_t K, const int32_t* bank,
+                                 int32_t bank_w, int32_t G, int32_t S, int32_t n_groups,
+                                 int32_t* hits, int32_t* count, cudaStream_t s) {
+  if (n_groups <= 0) return cudaSuccess;
+  const size_t smem = static_cast<size_t>((S + 31) / 32) * 4;
+  if (smem > kUnionMaxBitmapBytes) return cudaErrorInvalidValue;
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(
+        bank_coverage_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  bank_coverage_kernel<<<static_cast<unsigned>(n_groups), 256, smem, s>>>(topk, K, bank, bank_w,
+                                                                         G, S, hits, count);
   return cudaGetLastError();
 }
 

@@ -76,3 +76,35 @@ def test_union_sizes_on_the_indexer_output(G):
     feasible = [(cost_model.speedups(128 * K1, g, P)[2], g, P) for g in cal.GROUP_SIZES
                 for P in cal.BUDGETS if ref_caps[g] <= P]
     assert choice == (max(feasible)[1:] if feasible else None)
+
+
+def test_coverage_by_position_hand_values():
+    hits = [4, 2, 2, 3]
+    count = [4, 2, 4, 4]
+    per_pos, mean = cal.coverage_by_position(hits, count, 2)
+    assert per_pos.tolist() == [0.75, 0.875]
+    assert mean == pytest.approx(0.8125)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("mode", ["window", "paper"])
+def test_bank_coverage_equals_the_oracle(mode):
+    """ADIndex Figure 1(c) / Appendix B.4 coverage on the library's own outputs: the flat
+    Top-K rows and the group banks of a group-mode problem. Integer work: equal to the
+    oracle's counts on the same rows, element for element."""
+    from sparse_attention_token_indexer_b200 import build, indexer, inputs
+    build.build()
+    T, G, B, K, Hg = 64 * 20 + 9, 64, 512, 256, 16
+    p = inputs.group_prefill(T, H=64, d=128, K=K, G=G, B=B, Hg=Hg, seed=29, device="cuda")
+    flat, _, _ = indexer.index_prefill(p["q"], p["w"], p["k"], K)
+    bank = indexer.group_bank(p["qbar"], p["wbar"], p["k"], G, B, mode)
+    hits, count = cal.bank_coverage(flat, bank, G, T)
+    ref_h, ref_c = ox.bank_coverage(flat.cpu().numpy(), bank.cpu().numpy(), G)
+    assert hits.cpu().numpy().tolist() == ref_h.tolist()
+    assert count.cpu().numpy().tolist() == ref_c.tolist()
+    # the groups whose anchors see at most B keys hold their whole prefix: full coverage
+    full = [g for g, pl in enumerate(ox.plan_groups(T, 0, G, B, mode))
+            if pl.kind == "bank" and pl.scan_n <= pl.bank_k]
+    h, c = hits.cpu().numpy().reshape(-1, G), count.cpu().numpy().reshape(-1, G)
+    assert full and all(np.array_equal(h[g], c[g]) for g in full)
+    assert (h < c).any()

@@ -436,6 +436,54 @@ def test_union_sizes_bounds_and_monotonicity():
         assert x >= max(u4[2 * g], u4[2 * g + 1])
 
 
+def test_bank_coverage_hand_cases():
+    """A bank holding a query's whole Top-K covers it fully, a disjoint bank not at all,
+    a bank with half of it one half; padding counts on neither side."""
+    topk = [[3, 5, 7, 9], [3, 5, -1, -1], [1, 2, 4, 6], [0, 8, 10, 12]]
+    banks = [[3, 5, 7, 9, 11, -1], [4, 6, 8, 10, 12, -1]]
+    hits, count = ox.bank_coverage(topk, banks, 2)
+    assert hits.tolist() == [4, 2, 2, 3]
+    assert count.tolist() == [4, 2, 4, 4]
+    # an incomplete trailing group has no bank and no coverage
+    hits, count = ox.bank_coverage(topk[:3], banks[:1], 2)
+    assert len(hits) == len(count) == 2
+
+
+def test_bank_coverage_one_is_exact_recovery():
+    """ADIndex §1: refinement over the bank recovers a query's full Top-K exactly when the bank
+    holds all of it. On random problems, rows whose coverage (against the group's candidates:
+    bank plus post-anchor positions) is 1 refine to the flat Top-K, and rows whose flat
+    Top-K holds a key the candidates lack do not."""
+    rng = np.random.default_rng(21)
+    T, H, Hg, d, G, B, K = 96, 3, 2, 8, 8, 24, 6
+    seen_full = seen_part = 0
+    for trial in range(4):
+        q, w, k = rng.normal(size=(T, H, d)), rng.random((T, H)), rng.normal(size=(T, d))
+        qbar, wbar = rng.normal(size=(T // G, Hg, d)), rng.random((T // G, Hg))
+        for mode in ("paper", "window"):
+            plans = ox.plan_groups(T, 0, G, B, mode)
+            flat = ox.flat_topk(q, w, k, np.arange(T), K)
+            got, banks = ox.group_topk(q, w, k, qbar, wbar, 0, G, B, K, mode)
+            rows, brows = [], []
+            for gi, plan in enumerate(plans):
+                if plan.kind != "bank":
+                    continue
+                cand = np.union1d(banks[gi], np.arange(plan.post_lo, plan.rows[-1] + 1))
+                brows.append(cand)
+                rows.extend(flat[t] for t in plan.rows)
+            hits, count = ox.bank_coverage(rows, brows, G)
+            members = [t for p in plans if p.kind == "bank" for t in p.rows]
+            for j, t in enumerate(members):
+                same = set(got[t].tolist()) == set(flat[t].tolist())
+                if hits[j] == count[j]:
+                    assert same, (mode, t)
+                    seen_full += 1
+                else:
+                    assert not same, (mode, t)
+                    seen_part += 1
+    assert seen_full > 20 and seen_part > 20
+
+
 def test_mean_pool_group_hand_values():
     q = np.zeros((5, 3, 2))
     w = np.zeros((5, 3))
