@@ -21,6 +21,9 @@
  *    their events for adx_index_prefill_host, a cuBLAS handle for adx_group_indexer_queries),
  *    and launches all work asynchronously on `stream` (a cudaStream_t passed as void*;
  *    NULL = the legacy default stream).
+ *    One exception: adx_index_prefill_noalloc runs on a fixed device array of
+ *    ADX_STATIC_SCRATCH_BYTES compiled into the library (held on every GPU that loads it) and
+ *    caches that array's device address per device and context.
  *  - Argument errors are detected on the host and returned before any launch.
  *  - Errors the device detects (a bounded wait that ran out) are recorded in a status word
  *    at the start of the workspace and reported by adx_read_device_status(). The word is
@@ -340,10 +343,11 @@ int64_t adx_launch_count(void);
  * paper has no counterpart; this exists only for such callers.
  * Scratch is a fixed array of ADX_STATIC_SCRATCH_BYTES inside the library; every GPU that
  * loads the library holds it until the process exits. Problems that need more (see
- * adx_workspace_size(ADX_OP_PREFILL, ...)) return ADX_EWORKSPACE before any launch; nothing is
- * ever allocated. The first call on a device looks up the array's device address with that
- * device current: make it before any stream capture. All calls on a device share the array,
- * so calls that overlap on the GPU race; serialise them. Each call clears the status word on
+ * adx_workspace_size(ADX_OP_PREFILL, ...)) return ADX_EWORKSPACE before any launch, invalid
+ * or unsupported operands with the codes adx_index_prefill returns; nothing is ever
+ * allocated. The first call on a device looks up the array's device address with that
+ * device current (again after a device reset): make it before any stream capture. All calls
+ * on a device share the array, so calls that overlap on the GPU race; serialise them. Each call clears the status word on
  * `stream` first; device_status (a device int32, or NULL) receives the call's device status
  * (ADX_OK or ADX_ETIMEOUT) asynchronously on `stream`. */
 adx_status adx_index_prefill_noalloc(const adx_operands* ops, int32_t K, int32_t* topk_idx,

@@ -579,6 +579,12 @@ size_t ws_hisa(const adx_operands* o, int32_t n_blocks, int32_t K, bool blocks_e
 
 }  // namespace
 
+adx_status check_prefill_args(const adx_operands* o, int32_t K) {
+  const adx_status r = check_operands(o, false);
+  if (r != ADX_OK) return r;
+  return K <= 0 ? ADX_EINVAL : ADX_OK;
+}
+
 void add_launches(int n) { g_launches += n; }
 
 }  // namespace adx

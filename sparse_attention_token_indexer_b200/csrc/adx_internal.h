@@ -5,6 +5,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "../../include/adx.h"
+
 namespace adx {
 
 // Device status word at the start of every workspace (sticky until read).
@@ -205,6 +207,10 @@ cudaError_t launch_block_union(const int32_t* blocks, int32_t n_blocks, int32_t 
 // n_blocks blocks.
 cudaError_t launch_force_blocks(float* scores, int64_t ld, int32_t R, const int32_t* row_blk,
                                 int32_t n_blocks, cudaStream_t s);
+
+// Argument checks of adx_index_prefill that need no device: the operands (prefill layout)
+// and K. ADX_OK, ADX_EINVAL or ADX_EUNSUPPORTED, exactly as adx_index_prefill returns them.
+adx_status check_prefill_args(const adx_operands* o, int32_t K);
 
 // Adds n to the library's launch counter (kernels launched outside the API file).
 void add_launches(int n);

@@ -153,3 +153,17 @@ def test_group_helpers_host_validation(lib):
     grp.seq_len = 64
     assert lib.adx_mtp_workspace_size(ctypes.byref(full), ctypes.byref(grp), 16, 5, 512,
                                       64) == 0
+
+
+def test_noalloc_reports_operand_errors_like_the_workspace_entry_point(lib):
+    """adx_index_prefill_noalloc checks the operands before it touches the device, with the
+    codes adx_index_prefill returns: an unsupported head count is ADX_EUNSUPPORTED, not a
+    workspace error."""
+    def noalloc(o, K=4):
+        return lib.adx_index_prefill_noalloc(ctypes.byref(o), K, ctypes.c_void_p(4096), None,
+                                             None, None)
+    assert noalloc(_ops(H=5)) == L.ADX_EUNSUPPORTED
+    assert noalloc(_ops(H=5)) == _prefill(lib, _ops(H=5))
+    assert noalloc(_ops(d=96)) == L.ADX_EUNSUPPORTED
+    assert noalloc(_ops(q=None)) == L.ADX_EINVAL
+    assert noalloc(_ops(), K=0) == L.ADX_EINVAL
