@@ -235,19 +235,26 @@ def test_group_bank_and_refine(mode, dtype):
     bank = bank.cpu().numpy()
     idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
     plans = ox.plan_groups(T, 0, G, B, mode)
-    bank_k = B if mode == "paper" else B - G
     assert bank.shape[1] == indexer.bank_width(B, G, mode)
     n_complete = T // G
     for g in range(n_complete):
         a = g * G
-        scan_n = a + 1 if mode == "paper" else a
-        # stage 1: the bank's scan part against Eq. (13) with the oracle's group scores
-        keys = k64[:scan_n]
-        bs = ox.score_keys(qb64[g], wb64[g], keys)
-        bf = score_floor(qb64[g], wb64[g], keys)
-        check_topk(bank[g, :bank_k], np.arange(scan_n), bs, bf, bank_k, rtol, what=f"bank {g}")
+        plan = plans[g]
+        if plan.kind == "flat":
+            # a PAPER group whose anchor sees at most B keys: the bank path still runs and its
+            # bank must hold the anchor's whole prefix (then refinement is the plain indexer)
+            bank_k = B
+            assert sorted(x for x in bank[g, :bank_k].tolist() if x >= 0) == list(range(a + 1))
+            lo = a + 1
+        else:
+            bank_k, lo = plan.bank_k, plan.post_lo
+            # stage 1: the bank's scan part against Eq. (13) with the oracle's group scores
+            keys = k64[:plan.scan_n]
+            bs = ox.score_keys(qb64[g], wb64[g], keys)
+            bf = score_floor(qb64[g], wb64[g], keys)
+            check_topk(bank[g, :bank_k], np.arange(plan.scan_n), bs, bf, bank_k, rtol,
+                       what=f"bank {g}")
         post = bank[g, bank_k:]
-        lo = a + 1 if mode == "paper" else a
         assert post.tolist() == list(range(lo, lo + len(post)))
         # stage 2: refinement over the GPU's own bank (stage isolation)
         scan_part = bank[g, :bank_k]
@@ -472,10 +479,10 @@ def test_bank_rows_starting_past_a_select_class(q_pos0):
     bank = bank.cpu().numpy()
     k64 = f64(p["k"])
     assert q_pos0 in bank[0, :B].tolist()
-    for g in range(T // G):
-        scan_n = q_pos0 + g * G + 1
-        keys = k64[:scan_n]
-        check_topk(bank[g, :B], np.arange(scan_n), ox.score_keys(qb64[g], wb64[g], keys),
+    for g, plan in enumerate(ox.plan_groups(T, q_pos0, G, B, "paper")):
+        assert plan.kind == "bank" and plan.bank_k == B
+        keys = k64[:plan.scan_n]
+        check_topk(bank[g, :B], np.arange(plan.scan_n), ox.score_keys(qb64[g], wb64[g], keys),
                    score_floor(qb64[g], wb64[g], keys), B, RTOL["bf16"], what=f"bank {g}")
 
 
@@ -504,14 +511,15 @@ def test_group_mode_on_a_later_chunk(mode, dtype):
     qb64, wb64 = f64(qbar, qbs), wbar.double().cpu().numpy()
     rtol = RTOL[dtype]
     bank, idx, sc = bank.cpu().numpy(), idx.cpu().numpy(), sc.cpu().numpy()
-    bank_k = B if mode == "paper" else B - G
+    plans = ox.plan_groups(T, q_pos0, G, B, mode)
     for g in range(T // G):
-        a = q_pos0 + g * G
-        scan_n = a + 1 if mode == "paper" else a
-        keys = k64[:scan_n]
-        check_topk(bank[g, :bank_k], np.arange(scan_n), ox.score_keys(qb64[g], wb64[g], keys),
-                   score_floor(qb64[g], wb64[g], keys), bank_k, rtol, what=f"bank {g}")
-        lo = a + 1 if mode == "paper" else a
+        plan = plans[g]
+        assert plan.kind == "bank"      # every anchor here sees more than B keys
+        bank_k, lo = plan.bank_k, plan.post_lo
+        keys = k64[:plan.scan_n]
+        check_topk(bank[g, :bank_k], np.arange(plan.scan_n),
+                   ox.score_keys(qb64[g], wb64[g], keys), score_floor(qb64[g], wb64[g], keys),
+                   bank_k, rtol, what=f"bank {g}")
         scan_part = bank[g, :bank_k][bank[g, :bank_k] >= 0]
         for r in range(g * G, g * G + G, 5):
             i = q_pos0 + r
