@@ -1,18 +1,22 @@
 #!/usr/bin/env python
 """Throughput of the indexer hot path on B200: query-key scores/s and Top-K queries/s.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--rows]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step = one pass of the flat DSA indexer (score, Eq. (1), + per-query Top-K, Eq. (2))
-over the DSA-shaped prefill workload: T = 16384 causal queries, H_I = 64 heads, d = 128,
-K = 2048, bf16 operands on anchor-structured synthetic data. Inputs are resident in HBM
-before the timed region and larger than L2 (q alone is 256 MiB), so no L2 flush is needed.
-Under torchrun each rank runs its own replica of the workload (weak scaling, no collective
-on the data path); the time is the max over ranks.
+Headline step = one pass of the flat DSA indexer (score, Eq. (1), + per-query Top-K,
+Eq. (2)) over the largest single-GPU workload: a 262144-token causal prefill processed in
+query chunks of 4096 against the growing key cache (H_I = 64 heads, d = 128, K = 2048, bf16
+operands, anchor-structured synthetic data): 64 chunk calls, 3.44e10 (query, key) pairs.
+Inputs are resident in HBM before the timed region and larger than L2 (q alone is 4 GiB), so
+no L2 flush is needed. `e2e` times the same pass through the host-buffer entry point with the
+copies inside the timed region. Under torchrun each rank runs its own replica (weak scaling,
+no collective on the data path); the time is the max over ranks.
 
---rows also times the other hot-path rows on their own workloads (FP8 flat prefill, ADIndex
-group mode on 64K tokens, decode with an FP8 key cache, decode with bank reuse) and adds
-them under "rows". --impl reference times the fp64 CPU oracle on the host cores instead.
+"rows" times every other workload of the hot path in the same run: the 256K prefill in group
+mode and in FP8, the 16K flat prefill (bf16 and FP8), group mode on 64K tokens, decode with an
+FP8 key cache, decode bank reuse (cycle and refine-only steps), MTP verification, calibration,
+HISA and the group indexer. `cpu_baseline` is the fp64 oracle on the host cores (a thread per
+core) on sampled rows of the headline workload; --impl reference times only that.
 """
 
 import argparse
@@ -298,26 +302,6 @@ def _call_prefill(p, K, idx, ws):
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)))
 
 
-def run_e2e(args, dist, p):
-    """Same step through the public API with host buffers (adx_index_prefill_host): pinned
-    H2D of the inputs, the indexer and D2H of the Top-K indices, every step inside the timed
-    region; the library overlaps the copies of one chunk of rows with the indexing of another."""
-    from sparse_attention_token_indexer_b200 import indexer
-    c = FLAT
-    host = {k: p[k].cpu().pin_memory() for k in ("q", "w", "k")}
-    out_h = torch.empty(c["T"], c["K"], dtype=torch.int32).pin_memory()
-    ws = indexer.Workspace("cuda")
-
-    def step():
-        indexer.index_prefill_host(host["q"], host["w"], host["k"], c["K"],
-                                   rows_per_chunk=E2E_ROWS_PER_CHUNK, out=(out_h, None), ws=ws)
-
-    ms, _ = timed(step, args.steps, args.warmup, dist)
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_h.numel() * out_h.element_size()
-    return ms, h2d, d2h
-
-
 def run_group(args, dist):
     from sparse_attention_token_indexer_b200 import indexer, inputs
     c = GROUP
@@ -527,13 +511,12 @@ def run_group_indexer(args, dist):
     return dict(ms=ms, launches=launches, groups=ng, act_bytes=act, flops=flops)
 
 
-def run_chunked(args, dist, dtype="bf16"):
-    """256K-token prefill in query chunks of 4096 against the growing causal key cache, flat
-    and in group mode (window bank, G = 64, B = 8192); one step = all 64 chunks. e4m3: q, k
-    and the group queries quantised per token (fp32 scales)."""
-    from sparse_attention_token_indexer_b200 import indexer, inputs
+def chunked_inputs(dtype="bf16"):
+    """The 256K chunked-prefill workload: q [S, 64, 128], w, k [S, 128] on the device (bf16,
+    or e4m3 codes with per-token scales), and the group queries of every G = 64 tokens."""
+    from sparse_attention_token_indexer_b200 import inputs
     c = CHUNKED
-    S, ch, G = c["S"], c["chunk"], c["G"]
+    S, G = c["S"], c["G"]
     st = inputs.AnchorStructure(c["d"], c["seed"], "cuda")
     kf = st.keys(S)
     q = torch.empty(S, c["H"], c["d"], dtype=torch.bfloat16, device="cuda")
@@ -554,78 +537,360 @@ def run_chunked(args, dist, dtype="bf16"):
         k = kf.to(torch.bfloat16).contiguous()
         qbar = qbar.to(torch.bfloat16).contiguous()
     del kf
-    ws = indexer.Workspace("cuda")
-    idx = torch.empty(ch, c["K"], dtype=torch.int32, device="cuda")
+    return dict(q=q, w=w, k=k, q_scale=qs, k_scale=ks, qbar=qbar, wbar=wbar, qbar_scale=qbs,
+                dtype=dtype)
+
+
+def chunked_flat_pass(inp, ws, idx, timers=None):
+    """One 256K prefill in query chunks of 4096, flat indexer; timers: one StageTimer slot per
+    chunk (the library's events around each chunk's scoring and selection kernels)."""
+    c = CHUNKED
+    S, ch = c["S"], c["chunk"]
+    q, w, k, qs, ks = inp["q"], inp["w"], inp["k"], inp["q_scale"], inp["k_scale"]
+    for j, c0 in enumerate(range(0, S, ch)):
+        if timers is not None:
+            timers.arm(j)
+        _call_prefill({"q": q[c0:c0 + ch], "w": w[c0:c0 + ch], "k": k,
+                       "q_scale": None if qs is None else qs[c0:c0 + ch], "k_scale": ks,
+                       "q_pos0": c0}, c["K"], idx, ws)
+    if timers is not None:
+        timers.disarm()
+
+
+def chunked_group_pass(inp, ws):
+    """One 256K prefill in query chunks of 4096, ADIndex group mode (WINDOW bank, G = 64,
+    B = 8192): per chunk the group banks, then every query's refinement."""
+    from sparse_attention_token_indexer_b200 import indexer
+    c = CHUNKED
+    S, ch, G = c["S"], c["chunk"], c["G"]
     gpc = ch // G
+    q, w, k, qs, ks = inp["q"], inp["w"], inp["k"], inp["q_scale"], inp["k_scale"]
+    qbar, wbar, qbs = inp["qbar"], inp["wbar"], inp["qbar_scale"]
+    for c0 in range(0, S, ch):
+        g0 = c0 // G
+        bank = indexer.group_bank(qbar[g0:g0 + gpc], wbar[g0:g0 + gpc], k, G, c["B"], "window",
+                                  qbar_scale=None if qbs is None else qbs[g0:g0 + gpc],
+                                  k_scale=ks, q_pos0=c0, ws=ws)
+        indexer.bank_refine(q[c0:c0 + ch], w[c0:c0 + ch], k, bank, G, c["B"], "window", c["K"],
+                            q_scale=None if qs is None else qs[c0:c0 + ch], k_scale=ks,
+                            q_pos0=c0, ws=ws)
 
-    def flat_pass():
-        for c0 in range(0, S, ch):
-            _call_prefill({"q": q[c0:c0 + ch], "w": w[c0:c0 + ch], "k": k,
-                           "q_scale": None if qs is None else qs[c0:c0 + ch], "k_scale": ks,
-                           "q_pos0": c0}, c["K"], idx, ws)
 
-    def group_pass():
-        for c0 in range(0, S, ch):
-            g0 = c0 // G
-            bank = indexer.group_bank(qbar[g0:g0 + gpc], wbar[g0:g0 + gpc], k, G, c["B"],
-                                      "window", qbar_scale=None if qbs is None else
-                                      qbs[g0:g0 + gpc], k_scale=ks, q_pos0=c0, ws=ws)
-            indexer.bank_refine(q[c0:c0 + ch], w[c0:c0 + ch], k, bank, G, c["B"], "window",
-                                c["K"], q_scale=None if qs is None else qs[c0:c0 + ch],
-                                k_scale=ks, q_pos0=c0, ws=ws)
-
-    ms_flat, l_flat = timed(flat_pass, 1, args.warmup, dist)
-    ms_grp, l_grp = timed(group_pass, 1, args.warmup, dist)
+def chunked_counts():
+    c = CHUNKED
+    S, G, B = c["S"], c["G"], c["B"]
     pairs = S * (S + 1) // 2
     scan = sum(g * G for g in range(S // G))
-    refine = sum(min(c["B"] - G, g * G) * G + G * (G + 1) // 2 for g in range(S // G))
-    return dict(ms_flat=ms_flat, ms_group=ms_grp, l_flat=l_flat, l_group=l_grp, pairs=pairs,
-                scan=scan, refine=refine, rows=S)
+    refine = sum(min(B - G, g * G) * G + G * (G + 1) // 2 for g in range(S // G))
+    return pairs, scan, refine
+
+
+def run_chunked_flat(args, dist, inp, steps, clocks=None):
+    """Times `steps` flat 256K passes, then one more pass with the per-chunk stage events
+    armed; returns ms per pass, launches, and the summed scoring / selection kernel time of a
+    pass."""
+    from sparse_attention_token_indexer_b200 import _lib, indexer
+    c = CHUNKED
+    ws = indexer.Workspace("cuda")
+    idx = torch.empty(c["chunk"], c["K"], dtype=torch.int32, device="cuda")
+    n_chunks = c["S"] // c["chunk"]
+
+    def step():
+        chunked_flat_pass(inp, ws, idx)
+
+    if clocks is not None:
+        with clocks:
+            ms, launches = timed(step, steps, args.warmup, dist)
+    else:
+        ms, launches = timed(step, steps, args.warmup, dist)
+    timer = StageTimer(_lib.lib(), n_chunks)
+    chunked_flat_pass(inp, ws, idx, timer)
+    torch.cuda.synchronize()
+    score_ms = sum(timer.ms(0, 1))
+    select_ms = sum(timer.ms(2, 3))
+    del ws
+    return dict(ms=ms, launches=launches, score_ms=score_ms, select_ms=select_ms)
+
+
+def run_chunked_group(args, dist, inp, steps):
+    from sparse_attention_token_indexer_b200 import indexer
+    ws = indexer.Workspace("cuda")
+
+    def step():
+        chunked_group_pass(inp, ws)
+
+    ms, launches = timed(step, steps, args.warmup, dist)
+    del ws
+    return dict(ms=ms, launches=launches)
+
+
+def run_chunked_e2e(args, dist, inp, steps):
+    """The flat 256K prefill through the public host-buffer entry point (adx_index_prefill_host):
+    the operands start in pinned host memory, chunks of 4096 rows are indexed longest first
+    while the next chunk's queries and gates are copied in and the previous chunk's Top-K rows
+    are copied out; every copy is inside the timed region."""
+    from sparse_attention_token_indexer_b200 import indexer
+    c = CHUNKED
+    host = {n: inp[n].cpu().pin_memory() for n in ("q", "w", "k")}
+    for n in ("q_scale", "k_scale"):
+        host[n] = None if inp[n] is None else inp[n].cpu().pin_memory()
+    out_h = torch.empty(c["S"], c["K"], dtype=torch.int32).pin_memory()
+    ws = indexer.Workspace("cuda")
+
+    def step():
+        indexer.index_prefill_host(host["q"], host["w"], host["k"], c["K"], host["q_scale"],
+                                   host["k_scale"], rows_per_chunk=c["chunk"], out=(out_h, None),
+                                   ws=ws)
+
+    ms, _ = timed(step, steps, args.warmup, dist)
+    h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
+    d2h = out_h.numel() * out_h.element_size()
+    del ws, host, out_h
+    return ms, h2d, d2h
+
+
+def run_decode_refine(args, dist):
+    """Decode with bank reuse (the decode workload's variant): the refine-only steps between
+    two refreshes, each over the bank of B = 8192 positions plus the keys appended since the
+    refresh; one step = the refinement of all 32 sequences at one decode position."""
+    from sparse_attention_token_indexer_b200 import indexer, inputs
+    c = DECODE
+    prob = inputs.decode_problem(c["Bs"], c["S"], c["H"], c["d"], c["K"], c["Hg"],
+                                 steps=c["G"], seed=c["seed"], device="cuda")
+    ws = indexer.Workspace("cuda")
+    seqs = [inputs.decode_seq_len(prob, r) for r in range(c["G"])]
+    qb = prob["q_steps"][0][:, : c["Hg"]].contiguous()
+    wb = prob["w_steps"][0][:, : c["Hg"]].contiguous()
+    bank = indexer.group_bank(qb, wb, prob["k"], c["G"], c["B"], "paper",
+                              k_scale=prob["k_scale"], seq_len=seqs[0], ws=ws)
+    r_mid = c["G"] // 2
+
+    def refine():
+        indexer.bank_refine(prob["q_steps"][r_mid], prob["w_steps"][r_mid], prob["k"], bank,
+                            c["G"], c["B"], "paper", c["K"], k_scale=prob["k_scale"],
+                            seq_len=seqs[r_mid], ws=ws)
+
+    ms, launches = timed(refine, args.steps, args.warmup, dist)
+    ms_graph, _ = timed_graph(refine, args.steps, args.warmup, dist)
+    # keys the step reads: the bank entries at or before the position plus the new keys
+    keys = c["Bs"] * (c["B"] + r_mid)
+    del prob, ws
+    return dict(ms=ms, ms_graph=ms_graph, launches=launches, bytes=keys * (c["d"] + 4),
+                rows=c["Bs"])
 
 
 # ---------------------------------------------------------------------------------------
 # the oracle on the host cores
 # ---------------------------------------------------------------------------------------
 
-def cpu_cores():
+def cpu_model():
     try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
-        if n and n[0]:
-            return int(n[0])
-    except Exception:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
         pass
-    return os.cpu_count()
+    import platform
+    return platform.processor() or "unknown"
 
 
-def oracle_sample(p, K, seconds, seed=0):
-    """Times the oracle on flat rows drawn across the causal triangle until `seconds` of
-    CPU work are done; returns (pairs scored, rows completed, elapsed seconds)."""
-    from oracle import fp_formats
-    from oracle import indexer as ox
+def affinity_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
 
-    def f64(t, scale=None):
-        t = t.detach().cpu()
-        if t.dtype == torch.bfloat16:
-            return fp_formats.bf16_bits_to_f64(t.view(torch.int16).numpy().view(np.uint16))
-        return fp_formats.dequantize(t.numpy(), scale.detach().cpu().numpy(), "e4m3")
 
-    q64 = f64(p["q"], p["q_scale"])
-    k64 = f64(p["k"], p["k_scale"])
-    w64 = p["w"].double().cpu().numpy()
-    rng = np.random.default_rng(seed)
-    T = q64.shape[0]
-    pairs = rows = 0
-    t0 = time.perf_counter()
-    while time.perf_counter() - t0 < seconds or rows < 4:
-        t = int(rng.integers(T))
-        ox.flat_topk_row(q64[t], w64[t], k64, p["q_pos0"] + t, K)
-        pairs += p["q_pos0"] + t + 1
-        rows += 1
-    return pairs, rows, time.perf_counter() - t0
+class OracleBaseline:
+    """The fp64 oracle (as it stands) on the host cores: one query row per task on a thread
+    pool with one thread per affinity core and one BLAS thread per call (numpy releases the
+    interpreter lock inside its matrix products, maxima and sorts), on a stratified sample of
+    the chunked prefill's query rows: the first and last positions, the rows around K, and
+    positions drawn uniformly; scores/s = pairs scored / wall time."""
+
+    def __init__(self, q, w, k, K, n_rows, seed=0, pos=None):
+        """q, w: the workload's query rows and gates (all rows, or with `pos` given, just the
+        rows sampled at those positions); k: its keys."""
+        from concurrent.futures import ThreadPoolExecutor
+
+        from threadpoolctl import threadpool_limits
+
+        from oracle import fp_formats
+        S = k.shape[0]
+        if pos is None:
+            rng = np.random.default_rng(seed)
+            fixed = [0, 1, K - 1, K, K + 1, S - 2, S - 1]
+            pos = np.array(fixed + rng.integers(0, S, max(0, n_rows - len(fixed))).tolist(),
+                           dtype=np.int64)
+            sel = torch.as_tensor(pos, device=q.device)
+            q, w = q[sel], w[sel]
+
+        def bits(t):
+            return t.cpu().view(torch.int16).numpy().view(np.uint16)
+
+        self.pos = np.asarray(pos, dtype=np.int64)
+        self.k = fp_formats.bf16_bits_to_f64(bits(k))
+        self.q = fp_formats.bf16_bits_to_f64(bits(q))
+        self.w = w.cpu().double().numpy()
+        self.K = K
+        self.cores = affinity_cores()
+        self.limits = threadpool_limits(1)
+        self.pool = ThreadPoolExecutor(self.cores)
+
+    def _row(self, j):
+        from oracle import indexer as ox
+        j %= len(self.pos)
+        p = int(self.pos[j])
+        ox.flat_topk_row(self.q[j], self.w[j], self.k, p, self.K)
+        return p + 1
+
+    def run(self, rows):
+        """Scores the sampled rows with these indices; returns (pairs, rows, wall seconds)."""
+        t0 = time.perf_counter()
+        pairs = sum(self.pool.map(self._row, list(rows)))
+        return pairs, len(rows), time.perf_counter() - t0
+
+    def run_for(self, seconds, start=0):
+        """Rows start, start+1, ... until about `seconds` of wall time: one batch of one row per
+        thread first, to measure the row cost, then the rest in one go."""
+        rows = list(range(start, start + self.cores))
+        pairs, n, wall = self.run(rows)
+        per_batch = max(wall, 1e-3)
+        more = int(max(0.0, seconds - wall) / per_batch) * self.cores
+        nxt = start + self.cores
+        rows2 = list(range(nxt, nxt + more))
+        if rows2:
+            p2, n2, w2 = self.run(rows2)
+            pairs, n, wall = pairs + p2, n + n2, wall + w2
+        return pairs, n, wall, nxt + len(rows2)
+
+    def close(self):
+        self.pool.shutdown()
+        self.limits.unregister()
 
 
 # ---------------------------------------------------------------------------------------
+
+def reference_arm(args, dist):
+    """--impl reference: the fp64 oracle as it stands, on the host cores, on the headline's
+    workload (the 256K chunked flat prefill), rank 0 only; each step a bounded sample of rows."""
+    if dist.rank != 0:
+        dist.close()
+        return
+    c = CHUNKED
+    if torch.cuda.is_available():
+        torch.cuda.set_device(dist.local)
+        inp = chunked_inputs("bf16")      # the very operands the CUDA arm indexes
+        ob = OracleBaseline(inp["q"], inp["w"], inp["k"], c["K"], 8192)
+        del inp
+        torch.cuda.empty_cache()
+        where = "drawn on the GPU, the CUDA arm's operands"
+    else:
+        # no device: the same generator on the host (same shapes and distribution, other
+        # values); query rows do not depend on their position, so only the sample is drawn
+        from sparse_attention_token_indexer_b200 import inputs
+        st = inputs.AnchorStructure(c["d"], c["seed"], "cpu")
+        k = st.keys(c["S"]).to(torch.bfloat16)
+        n = 4 * affinity_cores()
+        rng = np.random.default_rng(0)
+        pos = np.array([0, c["K"], c["S"] - 1] + rng.integers(0, c["S"], n - 3).tolist())
+        ob = OracleBaseline(st.queries(n, c["H"]).to(torch.bfloat16), st.gates(n, c["H"]), k,
+                            c["K"], n, pos=pos)
+        where = "drawn on the host"
+    per_step = min(10.0, max(0.5, args.cpu_seconds / max(1, args.steps)))
+    start = 0
+    for _ in range(args.warmup):
+        _, _, _, start = ob.run_for(0.1, start)
+    tot_pairs = tot_rows = 0
+    tot_s = 0.0
+    for _ in range(args.steps):
+        pr, rw, wall, start = ob.run_for(per_step, start)
+        tot_pairs, tot_rows, tot_s = tot_pairs + pr, tot_rows + rw, tot_s + wall
+    ob.close()
+    value = tot_pairs / tot_s
+    sample = (f"{tot_rows} query rows of the 262144-token chunked prefill (first and last "
+              f"positions, around K, uniform positions; inputs {where}), {tot_s:.1f} s wall "
+              f"on {ob.cores} threads ({cpu_model()})")
+    line = {"impl": "reference", "metric": "indexer query-key scores/s", "value": value,
+            "unit": "scores/s", "n_gpus": dist.world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic (anchor-structured, seeded)",
+            "config": headline_config(dist),
+            "topk_queries_per_s": tot_rows / tot_s,
+            "cpu_baseline": {"value": value, "unit": "scores/s", "cores": ob.cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "scores/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    dist.close()
+
+
+def headline_config(dist):
+    c = CHUNKED
+    return {"workload": "chunked_prefill_flat_S262144_chunk4096_H64_d128_K2048_bf16",
+            "S": c["S"], "chunk": c["chunk"], "H_I": c["H"], "d": c["d"], "K": c["K"],
+            "seq_len": c["S"], "global_batch": dist.world,
+            "parallelism": f"replicas{dist.world}",
+            "l2": "inputs larger than L2 (q 4 GiB; per-chunk scores up to 4 GiB)"}
+
+
+def quick_case(args, dist):
+    """--quick: one workload's kernels only (no e2e, rows or CPU baseline), for profiling."""
+    out = {"case": args.case}
+    if args.case == "decode":
+        dcd = run_decode(args, dist, cycle=False)
+        out.update(ms_per_step=dcd["ms_flat"], stage_ms=dcd["stages"],
+                   hbm_gbs=dcd["bytes_flat"] / (dcd["ms_flat"] * 1e-3) / 1e9,
+                   gpu_launches=dcd["launches_flat"])
+    elif args.case == "decode_refine":
+        dr = run_decode_refine(args, dist)
+        out.update(ms_per_step=dr["ms"], graph_ms_per_step=dr["ms_graph"],
+                   hbm_gbs=dr["bytes"] / (dr["ms"] * 1e-3) / 1e9, gpu_launches=dr["launches"])
+    elif args.case == "chunked":
+        inp = chunked_inputs(args.dtype)
+        fl = run_chunked_flat(args, dist, inp, args.steps)
+        gr = run_chunked_group(args, dist, inp, args.steps)
+        out.update(dtype=args.dtype, flat_ms=fl["ms"], score_ms=fl["score_ms"],
+                   select_ms=fl["select_ms"], group_ms=gr["ms"])
+    elif args.case == "decode_cycle":
+        dcd = run_decode(args, dist)
+        n = dcd["steps_per_cycle"]
+        out.update(ms_per_step=dcd["ms_cycle"] / n, graph_ms_per_step=dcd["ms_cycle_graph"] / n,
+                   gpu_launches=dcd["launches_cycle"])
+    elif args.case == "mtp":
+        mt = run_mtp(args, dist)
+        out.update(ms_per_round=mt["ms"], flat_ms_per_round=mt["ms_flat"],
+                   speedup_vs_flat=mt["ms_flat"] / mt["ms"], gpu_launches=mt["launches"])
+    elif args.case in ("hisa", "hisa_small"):
+        if args.case == "hisa_small":
+            HISA["T"] = 16384
+        hs = run_hisa(args, dist, with_flat=False)
+        out.update(T=HISA["T"], ms_per_step=hs["ms"], stage_ms=hs["stages"],
+                   gpu_launches=hs["launches"])
+    elif args.case == "hisa_decode":
+        hd = run_hisa_decode(args, dist)
+        out.update(ms_per_step=hd["ms"], graph_ms_per_step=hd["ms_graph"],
+                   gpu_launches=hd["launches"])
+    elif args.case == "group_indexer":
+        gi = run_group_indexer(args, dist)
+        out.update(ms_per_step=gi["ms"], activation_gbs=gi["act_bytes"] / (gi["ms"] * 1e-3) / 1e9,
+                   gpu_launches=gi["launches"])
+    elif args.case == "group":
+        g = run_group(args, dist)
+        out.update(ms_per_step=g["ms"], stage_ms=g["stages"],
+                   refine_score_tflops=g["refine_tflops"], gpu_launches=g["launches"])
+    else:  # flat / flat_small
+        clocks = Clocks(dist.local)
+        flat = run_flat(args, dist, args.dtype, clocks)
+        out.update(dtype=args.dtype, ms_per_step=flat["ms"], score_ms=flat["score_ms"],
+                   select_ms=flat["select_ms"],
+                   score_tflops=flat["flops"] / flat["score_ms"] / 1e9,
+                   gpu_launches=flat["launches"], clocks=clocks.summary())
+    if dist.rank == 0:
+        print(json.dumps(out), flush=True)
+
 
 def main():
     ap = argparse.ArgumentParser()
@@ -633,265 +898,178 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--rows", action="store_true", help="also time the other hot-path rows")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--case", default="flat", choices=["flat", "flat_small", "decode", "mtp",
-                                                      "group_indexer", "hisa", "hisa_small",
-                                                      "hisa_decode", "decode_cycle", "chunked"],
-                    help="flat_small: T = 8192, for profiler captures; decode, mtp, "
-                         "group_indexer, hisa, hisa_decode, decode_cycle: that workload alone "
-                         "(with --quick); hisa_small: HISA prefill at T = 16384")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--case", default="all",
+                    choices=["all", "flat", "flat_small", "chunked", "group", "decode",
+                             "decode_refine", "decode_cycle", "mtp", "group_indexer", "hisa",
+                             "hisa_small", "hisa_decode"],
+                    help="all (default): the headline and every row; the others time one "
+                         "workload's kernels alone (with --quick), for profiling")
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "e4m3"])
     ap.add_argument("--quick", action="store_true",
-                    help="time the kernels only (no e2e, rows or CPU baseline): for profiling")
+                    help="with --case: time that workload's kernels only")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
     dist = Dist()
-    if args.impl == "ours":
-        torch.cuda.set_device(dist.local)
-    config = {"workload": "dsa_flat_prefill_T16384_H64_d128_K2048", "T": FLAT["T"],
-              "H_I": FLAT["H"], "d": FLAT["d"], "K": FLAT["K"], "seq_len": FLAT["T"],
-              "global_batch": dist.world, "parallelism": f"replicas{dist.world}",
-              "l2": "inputs larger than L2 (q 256 MiB, scores 1 GiB)"}
-
     if args.impl == "reference":
-        if dist.rank != 0:
-            dist.close()
-            return
-        from sparse_attention_token_indexer_b200 import inputs
-        p = inputs.anchor_prefill(FLAT["T"], FLAT["H"], FLAT["d"], FLAT["K"], seed=FLAT["seed"])
-        per = max(1.0, args.cpu_seconds / max(args.steps, 1))
-        for _ in range(args.warmup):
-            oracle_sample(p, FLAT["K"], 0.2)
-        tot_pairs = tot_rows = 0
-        tot_s = 0.0
-        for i in range(args.steps):
-            pr, rw, s = oracle_sample(p, FLAT["K"], per, seed=i)
-            tot_pairs, tot_rows, tot_s = tot_pairs + pr, tot_rows + rw, tot_s + s
-        value = tot_pairs / tot_s
-        line = {"impl": "reference", "metric": "indexer query-key scores/s", "value": value,
-                "unit": "scores/s", "n_gpus": dist.world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "f64", "data": "synthetic", "config": config,
-                "topk_queries_per_s": tot_rows / tot_s,
-                "cpu_baseline": {"value": value, "unit": "scores/s", "cores": cpu_cores(),
-                                 "kind": "oracle",
-                                 "sample": f"{tot_rows} flat rows drawn uniformly over the "
-                                           f"causal triangle, {tot_s:.1f} s"},
-                "e2e": {"value": value, "unit": "scores/s", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0}}
-        print(json.dumps(line), flush=True)
-        dist.close()
+        reference_arm(args, dist)
         return
-
+    torch.cuda.set_device(dist.local)
     from sparse_attention_token_indexer_b200 import build
     build.build()
+    if args.case != "all" or args.quick:
+        quick_case(args, dist)
+        dist.close()
+        return
+
     pk = peaks()
     clocks = Clocks(dist.local)
-    if args.case == "decode" and args.quick:
-        dcd = run_decode(args, dist, cycle=False)
-        if dist.rank == 0:
-            print(json.dumps({"case": "decode", "ms_per_step": dcd["ms_flat"],
-                              "stage_ms": dcd["stages"],
-                              "hbm_gbs": dcd["bytes_flat"] / (dcd["ms_flat"] * 1e-3) / 1e9,
-                              "gpu_launches": dcd["launches_flat"]}), flush=True)
-        dist.close()
-        return
-    if args.case == "chunked" and args.quick:
-        out = {}
-        for dt in ("bf16", "e4m3"):
-            ck = run_chunked(args, dist, dt)
-            out[dt] = {"flat_ms": ck["ms_flat"], "group_ms": ck["ms_group"]}
-            del ck
-        if dist.rank == 0:
-            print(json.dumps({"case": "chunked", **out}), flush=True)
-        dist.close()
-        return
-    if args.case == "decode_cycle" and args.quick:
-        dcd = run_decode(args, dist)
-        if dist.rank == 0:
-            n = dcd["steps_per_cycle"]
-            print(json.dumps({"case": "decode_cycle", "ms_per_step": dcd["ms_cycle"] / n,
-                              "graph_ms_per_step": dcd["ms_cycle_graph"] / n,
-                              "gpu_launches": dcd["launches_cycle"]}), flush=True)
-        dist.close()
-        return
-    if args.case == "mtp" and args.quick:
-        mt = run_mtp(args, dist)
-        if dist.rank == 0:
-            print(json.dumps({"case": "mtp", "ms_per_round": mt["ms"],
-                              "flat_ms_per_round": mt["ms_flat"],
-                              "speedup_vs_flat": mt["ms_flat"] / mt["ms"],
-                              "gpu_launches": mt["launches"]}), flush=True)
-        dist.close()
-        return
-    if args.case in ("hisa", "hisa_small") and args.quick:
-        if args.case == "hisa_small":
-            HISA["T"] = 16384
-        hs = run_hisa(args, dist, with_flat=False)
-        if dist.rank == 0:
-            print(json.dumps({"case": args.case, "T": HISA["T"], "ms_per_step": hs["ms"],
-                              "stage_ms": hs["stages"], "gpu_launches": hs["launches"]}),
-                  flush=True)
-        dist.close()
-        return
-    if args.case == "hisa_decode" and args.quick:
-        hd = run_hisa_decode(args, dist)
-        if dist.rank == 0:
-            print(json.dumps({"case": "hisa_decode", "ms_per_step": hd["ms"],
-                              "graph_ms_per_step": hd["ms_graph"],
-                              "gpu_launches": hd["launches"]}), flush=True)
-        dist.close()
-        return
-    if args.case == "group_indexer" and args.quick:
-        gi = run_group_indexer(args, dist)
-        if dist.rank == 0:
-            print(json.dumps({"case": "group_indexer", "ms_per_step": gi["ms"],
-                              "activation_gbs": gi["act_bytes"] / (gi["ms"] * 1e-3) / 1e9,
-                              "gpu_launches": gi["launches"]}), flush=True)
-        dist.close()
-        return
-    flat = run_flat(args, dist, args.dtype, clocks)
+    row_steps = max(2, args.steps // 5)
+    n_chunks = CHUNKED["S"] // CHUNKED["chunk"]
+
+    # ---- headline: the 256K chunked prefill, flat indexer, bf16 ---------------------------
+    inp = chunked_inputs("bf16")
+    fl = run_chunked_flat(args, dist, inp, args.steps, clocks)
     clk = clocks.summary()
-    if args.quick:
-        if dist.rank == 0:
-            print(json.dumps({"case": args.case, "dtype": args.dtype, "ms_per_step": flat["ms"],
-                              "score_ms": flat["score_ms"], "select_ms": flat["select_ms"],
-                              "score_tflops": flat["flops"] / flat["score_ms"] / 1e9,
-                              "gpu_launches": flat["launches"], "clocks": clk}), flush=True)
-        dist.close()
-        return
-    value = dist.world * flat["pairs"] / (flat["ms"] * 1e-3)
-    score_tflops = flat["flops"] / (flat["score_ms"] * 1e-3) / 1e12
-    e2e_ms, h2d, d2h = run_e2e(args, dist, flat["p"])
+    pairs, scan, refine = chunked_counts()
+    flops = pairs * 2 * CHUNKED["H"] * CHUNKED["d"]
+    score_tflops = flops / (fl["score_ms"] * 1e-3) / 1e12
+    peak_s = pk["bf16_sustained"] or pk["bf16"]
     line = {
-        "metric": "indexer query-key scores/s", "value": value, "unit": "scores/s",
-        "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": flat["ms"], "higher_is_better": True, "scaling": "weak",
+        "metric": "indexer query-key scores/s", "value": dist.world * pairs / (fl["ms"] * 1e-3),
+        "unit": "scores/s", "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": fl["ms"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (anchor-structured, seeded)",
-        "config": config,
-        "topk_queries_per_s": dist.world * flat["rows"] / (flat["ms"] * 1e-3),
-        "stage_ms": {"score": flat["score_ms"], "select": flat["select_ms"]},
-        "roofline": {"kernel": "score_kernel (tcgen05, bf16)", "bound": "tensor",
-                     "achieved": score_tflops, "peak": pk["bf16"], "unit": "TFLOP/s",
-                     "frac": score_tflops / pk["bf16"],
-                     "peak_source": f"{pk['source']} bf16 burst",
-                     "traffic": kernel_traffic("score_kernel_flat_prefill_T16384_bf16")},
-        "e2e": {"value": dist.world * flat["pairs"] / (e2e_ms * 1e-3), "unit": "scores/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": flat["launches"],
+        "config": headline_config(dist),
+        "topk_queries_per_s": dist.world * CHUNKED["S"] / (fl["ms"] * 1e-3),
+        "stage_ms": {"score": fl["score_ms"], "select": fl["select_ms"]},
+        "roofline": {"kernel": "score_kernel (tcgen05, bf16), 64 launches per step",
+                     "bound": "tensor", "achieved": score_tflops, "peak": peak_s,
+                     "unit": "TFLOP/s", "frac": score_tflops / peak_s,
+                     "peak_source": f"{pk['source']} bf16 sustained (a kernel inside a long step)",
+                     "traffic": kernel_traffic("score_kernel_chunked_prefill_S262144_bf16")},
+        "gpu_launches": fl["launches"],
         "clocks": clk,
     }
-    del flat["p"]
-    if args.rows:
-        rows = {}
-        f8 = run_flat(args, dist, "e4m3")
-        f8.pop("p")
-        rows["flat_prefill_e4m3"] = {
-            "scores_per_s": f8["pairs"] / (f8["ms"] * 1e-3), "ms_per_step": f8["ms"],
-            "score_ms": f8["score_ms"], "select_ms": f8["select_ms"],
-            "score_tflops": f8["flops"] / (f8["score_ms"] * 1e-3) / 1e12,
-            "peak_tflops_e4m3": 2 * pk["bf16"], "gpu_launches": f8["launches"]}
-        g = run_group(args, dist)
-        rows["group_mode_T65536"] = {
-            "ms_per_step": g["ms"], "scan_pairs": g["scan_pairs"],
-            "refine_pairs": g["refine_pairs"],
-            "scores_per_s": (g["scan_pairs"] + g["refine_pairs"]) / (g["ms"] * 1e-3),
-            "topk_queries_per_s": g["rows"] / (g["ms"] * 1e-3),
-            "tflops": g["flops"] / (g["ms"] * 1e-3) / 1e12, "gpu_launches": g["launches"],
-            "stage_ms": g["stages"], "refine_score_tflops": g["refine_tflops"]}
-        dcd = run_decode(args, dist)
-        rows["decode_Bs32_S131072_e4m3"] = {
-            "ms_per_step": dcd["ms_flat"],
-            "scores_per_s": DECODE["Bs"] * DECODE["S"] / (dcd["ms_flat"] * 1e-3),
-            "topk_queries_per_s": DECODE["Bs"] / (dcd["ms_flat"] * 1e-3),
-            "hbm_gbs": dcd["bytes_flat"] / (dcd["ms_flat"] * 1e-3) / 1e9,
-            "hbm_frac": dcd["bytes_flat"] / (dcd["ms_flat"] * 1e-3) / 1e9 / pk["hbm"],
-            "score_kernel_hbm_gbs": dcd["bytes_flat"] / (dcd["stages"]["score_ms"] * 1e-3) / 1e9,
-            "stage_ms": dcd["stages"], "gpu_launches": dcd["launches_flat"]}
-        ck = run_chunked(args, dist)
-        rows["chunked_prefill_S262144_flat"] = {
-            "ms_per_pass": ck["ms_flat"], "scores_per_s": ck["pairs"] / (ck["ms_flat"] * 1e-3),
-            "topk_queries_per_s": ck["rows"] / (ck["ms_flat"] * 1e-3),
-            "tflops": ck["pairs"] * 2 * CHUNKED["H"] * CHUNKED["d"] / (ck["ms_flat"] * 1e-3) / 1e12,
-            "gpu_launches": ck["l_flat"]}
-        rows["chunked_prefill_S262144_group"] = {
-            "ms_per_pass": ck["ms_group"],
-            "scores_per_s": (ck["scan"] + ck["refine"]) / (ck["ms_group"] * 1e-3),
-            "topk_queries_per_s": ck["rows"] / (ck["ms_group"] * 1e-3),
-            "speedup_vs_flat": ck["ms_flat"] / ck["ms_group"], "gpu_launches": ck["l_group"]}
-        del ck
-        c8 = run_chunked(args, dist, "e4m3")
-        rows["chunked_prefill_S262144_e4m3"] = {
-            "flat_ms_per_pass": c8["ms_flat"], "group_ms_per_pass": c8["ms_group"],
-            "flat_scores_per_s": c8["pairs"] / (c8["ms_flat"] * 1e-3),
-            "flat_tflops": c8["pairs"] * 2 * CHUNKED["H"] * CHUNKED["d"]
-            / (c8["ms_flat"] * 1e-3) / 1e12,
-            "group_speedup_vs_flat": c8["ms_flat"] / c8["ms_group"],
-            "gpu_launches": c8["l_flat"] + c8["l_group"]}
-        mt = run_mtp(args, dist)
-        rows[f"mtp_round_Bs32_N131072_m{MTP['m']}_G{MTP['G']}_P{MTP['P']}"] = {
-            "ms_per_round": mt["ms"], "scan_pairs": mt["scan"], "refine_pairs": mt["refine"],
-            "scores_per_s": (mt["scan"] + mt["refine"]) / (mt["ms"] * 1e-3),
-            "topk_queries_per_s": mt["rows"] / (mt["ms"] * 1e-3),
-            "flat_ms_per_round": mt["ms_flat"],
-            "speedup_vs_flat": mt["ms_flat"] / mt["ms"],
-            "score_count_ratio": mt["flat"] / (mt["scan"] + mt["refine"]),
-            "gpu_launches": mt["launches"]}
-        cb = run_calibration(args, dist)
-        rows["calibration_union_sizes_T16384_K2048"] = {
-            "ms_per_layer": cb["ms"], "group_sizes": [4, 8, 16],
-            "gbs_read": cb["bytes"] / (cb["ms"] * 1e-3) / 1e9,
-            "hbm_frac": cb["bytes"] / (cb["ms"] * 1e-3) / 1e9 / pk["hbm"],
-            "gpu_launches": cb["launches"]}
-        hs = run_hisa(args, dist)
-        rows["hisa_prefill_T65536_nb64"] = {
-            "ms_per_step": hs["ms"], "flat_ms_per_step": hs["ms_flat"],
-            "speedup_vs_flat": hs["ms_flat"] / hs["ms"],
-            "scores_per_s": (hs["blk_pairs"] + hs["tok_pairs"]) / (hs["ms"] * 1e-3),
-            "topk_queries_per_s": hs["rows"] / (hs["ms"] * 1e-3),
-            "tflops": hs["flops"] / (hs["ms"] * 1e-3) / 1e12, "stage_ms": hs["stages"],
-            "refine_score_tflops": 2 * HISA["H"] * HISA["d"] * hs["tok_pairs"]
-            / (hs["stages"]["refine_score_ms"] * 1e-3) / 1e12,
-            "gpu_launches": hs["launches"]}
-        hd = run_hisa_decode(args, dist)
-        rows["hisa_decode_Bs32_S131072_e4m3_nb64"] = {
-            "ms_per_step": hd["ms"], "graph_ms_per_step": hd["ms_graph"],
-            "flat_ms_per_step": dcd["ms_flat"],
-            "speedup_vs_flat": dcd["ms_flat"] / hd["ms"],
-            "topk_queries_per_s": DECODE["Bs"] / (hd["ms"] * 1e-3),
-            "hbm_gbs": hd["bytes"] / (hd["ms"] * 1e-3) / 1e9, "gpu_launches": hd["launches"]}
-        gi = run_group_indexer(args, dist)
-        rows["group_indexer_queries_T65536_G64"] = {
-            "ms_per_step": gi["ms"], "groups_per_s": gi["groups"] / (gi["ms"] * 1e-3),
-            "activation_gbs": gi["act_bytes"] / (gi["ms"] * 1e-3) / 1e9,
-            "hbm_frac": gi["act_bytes"] / (gi["ms"] * 1e-3) / 1e9 / pk["hbm"],
-            "projection_gflop": gi["flops"] / 1e9, "gpu_launches": gi["launches"],
-            "note": "projections on cuBLAS (not counted in gpu_launches)"}
-        rows["decode_bank_reuse_cycle16"] = {
-            "ms_per_cycle": dcd["ms_cycle"],
-            "ms_per_step": dcd["ms_cycle"] / dcd["steps_per_cycle"],
-            "graph_ms_per_step": dcd["ms_cycle_graph"] / dcd["steps_per_cycle"],
-            "topk_queries_per_s": DECODE["Bs"] * dcd["steps_per_cycle"] / (dcd["ms_cycle"] * 1e-3),
-            "gpu_launches": dcd["launches_cycle"]}
-        line["rows"] = rows
+    e2e_ms, h2d, d2h = run_chunked_e2e(args, dist, inp, args.steps)
+    line["e2e"] = {"value": dist.world * pairs / (e2e_ms * 1e-3), "unit": "scores/s",
+                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+    rows = {}
+    gr = run_chunked_group(args, dist, inp, row_steps)
+    rows["chunked_prefill_S262144_group_bf16"] = {
+        "ms_per_pass": gr["ms"], "scores_per_s": (scan + refine) / (gr["ms"] * 1e-3),
+        "topk_queries_per_s": CHUNKED["S"] / (gr["ms"] * 1e-3),
+        "speedup_vs_flat": fl["ms"] / gr["ms"], "gpu_launches": gr["launches"]}
+    ob = None
     if dist.rank == 0 and dist.world == 1:
-        pr, rw, s = oracle_sample(_cpu_copy_inputs(), FLAT["K"], args.cpu_seconds)
-        line["cpu_baseline"] = {"value": pr / s, "unit": "scores/s", "cores": cpu_cores(),
-                                "kind": "oracle",
-                                "sample": f"{rw} flat rows drawn uniformly over the causal "
-                                          f"triangle of the same workload, {s:.1f} s"}
+        ob = OracleBaseline(inp["q"], inp["w"], inp["k"], CHUNKED["K"], 8192)
+    del inp
+    torch.cuda.empty_cache()
+    inp8 = chunked_inputs("e4m3")
+    f8 = run_chunked_flat(args, dist, inp8, row_steps)
+    g8 = run_chunked_group(args, dist, inp8, row_steps)
+    t8 = flops / (f8["score_ms"] * 1e-3) / 1e12
+    rows["chunked_prefill_S262144_e4m3"] = {
+        "flat_ms_per_pass": f8["ms"], "flat_scores_per_s": pairs / (f8["ms"] * 1e-3),
+        "flat_stage_ms": {"score": f8["score_ms"], "select": f8["select_ms"]},
+        "score_tflops": t8, "score_frac_e4m3_peak": t8 / (2 * peak_s),
+        "group_ms_per_pass": g8["ms"], "group_speedup_vs_flat": f8["ms"] / g8["ms"],
+        "peak_source": f"{pk['source']} bf16 sustained x 2 (e4m3 dense rate)",
+        "gpu_launches": f8["launches"] + g8["launches"]}
+    del inp8
+    torch.cuda.empty_cache()
+
+    # ---- the other workloads -------------------------------------------------------------
+    for dt in ("bf16", "e4m3"):
+        args.case = "flat"
+        f = run_flat(args, dist, dt)
+        f.pop("p")
+        tf = f["flops"] / (f["score_ms"] * 1e-3) / 1e12
+        pkf = pk["bf16"] * (2 if dt == "e4m3" else 1)
+        rows[f"flat_prefill_T16384_{dt}"] = {
+            "ms_per_step": f["ms"], "scores_per_s": f["pairs"] / (f["ms"] * 1e-3),
+            "topk_queries_per_s": f["rows"] / (f["ms"] * 1e-3),
+            "stage_ms": {"score": f["score_ms"], "select": f["select_ms"]},
+            "score_tflops": tf, "score_frac": tf / pkf,
+            "step_frac": f["flops"] / (f["ms"] * 1e-3) / 1e12 / pkf,
+            "peak_tflops": pkf,
+            "peak_source": f"{pk['source']} bf16 burst" + (" x 2" if dt == "e4m3" else ""),
+            "gpu_launches": f["launches"]}
+    args.case = "all"
+    g = run_group(args, dist)
+    rows["group_mode_T65536"] = {
+        "ms_per_step": g["ms"], "scan_pairs": g["scan_pairs"], "refine_pairs": g["refine_pairs"],
+        "scores_per_s": (g["scan_pairs"] + g["refine_pairs"]) / (g["ms"] * 1e-3),
+        "topk_queries_per_s": g["rows"] / (g["ms"] * 1e-3), "stage_ms": g["stages"],
+        "refine_score_tflops": g["refine_tflops"],
+        "refine_score_frac": g["refine_tflops"] / pk["bf16"], "gpu_launches": g["launches"]}
+    dcd = run_decode(args, dist)
+    rows["decode_Bs32_S131072_e4m3"] = {
+        "ms_per_step": dcd["ms_flat"],
+        "scores_per_s": DECODE["Bs"] * DECODE["S"] / (dcd["ms_flat"] * 1e-3),
+        "topk_queries_per_s": DECODE["Bs"] / (dcd["ms_flat"] * 1e-3),
+        "hbm_gbs": dcd["bytes_flat"] / (dcd["ms_flat"] * 1e-3) / 1e9,
+        "hbm_frac": dcd["bytes_flat"] / (dcd["ms_flat"] * 1e-3) / 1e9 / pk["hbm"],
+        "score_kernel_hbm_frac": dcd["bytes_flat"] / (dcd["stages"]["score_ms"] * 1e-3) / 1e9
+        / pk["hbm"], "stage_ms": dcd["stages"], "gpu_launches": dcd["launches_flat"]}
+    rows["decode_bank_reuse_cycle16"] = {
+        "ms_per_cycle": dcd["ms_cycle"],
+        "ms_per_step": dcd["ms_cycle"] / dcd["steps_per_cycle"],
+        "graph_ms_per_step": dcd["ms_cycle_graph"] / dcd["steps_per_cycle"],
+        "topk_queries_per_s": DECODE["Bs"] * dcd["steps_per_cycle"] / (dcd["ms_cycle"] * 1e-3),
+        "gpu_launches": dcd["launches_cycle"]}
+    dr = run_decode_refine(args, dist)
+    rows["decode_refine_step_Bs32_B8192_e4m3"] = {
+        "ms_per_step": dr["ms"], "graph_ms_per_step": dr["ms_graph"],
+        "bytes_per_step": dr["bytes"], "hbm_gbs": dr["bytes"] / (dr["ms"] * 1e-3) / 1e9,
+        "hbm_frac": dr["bytes"] / (dr["ms"] * 1e-3) / 1e9 / pk["hbm"],
+        "graph_hbm_frac": dr["bytes"] / (dr["ms_graph"] * 1e-3) / 1e9 / pk["hbm"],
+        "topk_queries_per_s": dr["rows"] / (dr["ms"] * 1e-3), "gpu_launches": dr["launches"]}
+    mt = run_mtp(args, dist)
+    rows[f"mtp_round_Bs32_N131072_m{MTP['m']}_G{MTP['G']}_P{MTP['P']}"] = {
+        "ms_per_round": mt["ms"], "scan_pairs": mt["scan"], "refine_pairs": mt["refine"],
+        "scores_per_s": (mt["scan"] + mt["refine"]) / (mt["ms"] * 1e-3),
+        "topk_queries_per_s": mt["rows"] / (mt["ms"] * 1e-3), "flat_ms_per_round": mt["ms_flat"],
+        "speedup_vs_flat": mt["ms_flat"] / mt["ms"],
+        "score_count_ratio": mt["flat"] / (mt["scan"] + mt["refine"]), "gpu_launches": mt["launches"]}
+    cb = run_calibration(args, dist)
+    rows["calibration_union_sizes_T16384_K2048"] = {
+        "ms_per_layer": cb["ms"], "group_sizes": [4, 8, 16],
+        "gbs_read": cb["bytes"] / (cb["ms"] * 1e-3) / 1e9,
+        "hbm_frac": cb["bytes"] / (cb["ms"] * 1e-3) / 1e9 / pk["hbm"], "gpu_launches": cb["launches"]}
+    hs = run_hisa(args, dist)
+    rows["hisa_prefill_T65536_nb64"] = {
+        "ms_per_step": hs["ms"], "flat_ms_per_step": hs["ms_flat"],
+        "speedup_vs_flat": hs["ms_flat"] / hs["ms"],
+        "scores_per_s": (hs["blk_pairs"] + hs["tok_pairs"]) / (hs["ms"] * 1e-3),
+        "topk_queries_per_s": hs["rows"] / (hs["ms"] * 1e-3), "stage_ms": hs["stages"],
+        "refine_score_tflops": 2 * HISA["H"] * HISA["d"] * hs["tok_pairs"]
+        / (hs["stages"]["refine_score_ms"] * 1e-3) / 1e12, "gpu_launches": hs["launches"]}
+    hd = run_hisa_decode(args, dist)
+    rows["hisa_decode_Bs32_S131072_e4m3_nb64"] = {
+        "ms_per_step": hd["ms"], "graph_ms_per_step": hd["ms_graph"],
+        "flat_ms_per_step": dcd["ms_flat"], "speedup_vs_flat": dcd["ms_flat"] / hd["ms"],
+        "topk_queries_per_s": DECODE["Bs"] / (hd["ms"] * 1e-3),
+        "hbm_gbs": hd["bytes"] / (hd["ms"] * 1e-3) / 1e9, "gpu_launches": hd["launches"]}
+    gi = run_group_indexer(args, dist)
+    rows["group_indexer_queries_T65536_G64"] = {
+        "ms_per_step": gi["ms"], "groups_per_s": gi["groups"] / (gi["ms"] * 1e-3),
+        "activation_gbs": gi["act_bytes"] / (gi["ms"] * 1e-3) / 1e9,
+        "hbm_frac": gi["act_bytes"] / (gi["ms"] * 1e-3) / 1e9 / pk["hbm"],
+        "projection_gflop": gi["flops"] / 1e9, "gpu_launches": gi["launches"]}
+    line["rows"] = rows
+    if ob is not None:
+        pr, rw, wall, _ = ob.run_for(args.cpu_seconds)
+        ob.close()
+        line["cpu_baseline"] = {
+            "value": pr / wall, "unit": "scores/s", "cores": ob.cores, "kind": "oracle",
+            "sample": f"{rw} query rows of the same 262144-token workload (first and last "
+                      f"positions, around K, uniform positions), {wall:.1f} s wall on "
+                      f"{ob.cores} threads ({cpu_model()})"}
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
     dist.close()
-
-
-def _cpu_copy_inputs():
-    from sparse_attention_token_indexer_b200 import inputs
-    return inputs.anchor_prefill(FLAT["T"], FLAT["H"], FLAT["d"], FLAT["K"], seed=FLAT["seed"],
-                                 device="cuda", dtype="bf16")
 
 
 if __name__ == "__main__":

@@ -102,9 +102,11 @@ def test_bank_coverage_equals_the_oracle(mode):
     ref_h, ref_c = ox.bank_coverage(flat.cpu().numpy(), bank.cpu().numpy(), G)
     assert hits.cpu().numpy().tolist() == ref_h.tolist()
     assert count.cpu().numpy().tolist() == ref_c.tolist()
-    # the groups whose anchors see at most B keys hold their whole prefix: full coverage
+    # groups whose bank holds the anchor's whole visible prefix cover every member fully: the
+    # PAPER groups that fall back (a + 1 <= B, their bank path keeps every key) and the WINDOW
+    # groups whose scan is no longer than the bank
     full = [g for g, pl in enumerate(ox.plan_groups(T, 0, G, B, mode))
-            if pl.kind == "bank" and pl.scan_n <= pl.bank_k]
+            if len(pl.rows) == G and (pl.kind == "flat" or pl.scan_n <= pl.bank_k)]
     h, c = hits.cpu().numpy().reshape(-1, G), count.cpu().numpy().reshape(-1, G)
     assert full and all(np.array_equal(h[g], c[g]) for g in full)
     assert (h < c).any()
