@@ -474,19 +474,20 @@ def run_hisa_decode(args, dist):
     ws = indexer.Workspace("cuda")
     seq0 = inputs.decode_seq_len(prob, 0)
     q0, w0, k, ks = prob["q_steps"][0], prob["w_steps"][0], prob["k"], prob["k_scale"]
-    kbar, kbs = indexer.hisa_block_keys(q0, w0, k, k_scale=ks, seq_len=seq0)
+    kbar, _ = indexer.hisa_block_keys(q0, w0, k, k_scale=ks, seq_len=seq0)
 
     def step():
         indexer.hisa_block_keys(q0, w0, k, k_scale=ks, seq_len=seq0, last_only=True,
-                                out=(kbar, kbs))
+                                out=(kbar, None))
         indexer.index_hisa(q0, w0, k, kbar, c["K"], n_blocks=HISA["n_blocks"], k_scale=ks,
-                           kbar_scale=kbs, seq_len=seq0, ws=ws)
+                           seq_len=seq0, ws=ws)
 
     ms, launches = timed(step, args.steps, args.warmup, dist)
     ms_graph, _ = timed_graph(step, args.steps, args.warmup, dist)
     nb = (c["S"] + 127) // 128
     key_bytes = c["d"] + 4
-    bytes_step = c["Bs"] * (HISA["n_blocks"] * 128 + nb + 128) * key_bytes
+    # the kept blocks' keys, the bf16 block keys and the refreshed last block's keys
+    bytes_step = c["Bs"] * ((HISA["n_blocks"] * 128 + 128) * key_bytes + nb * c["d"] * 2)
     return dict(ms=ms, ms_graph=ms_graph, launches=launches, bytes=bytes_step)
 
 

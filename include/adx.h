@@ -18,9 +18,8 @@
  *  - Every pointer argument is a DEVICE pointer unless stated otherwise. The caller owns
  *    all memory; the library allocates nothing, keeps no state between calls besides
  *    cached device properties (and, created on first use per device: two copy streams and
- *    their events for adx_index_prefill_host, a cuBLAS handle for adx_group_indexer_queries),
- *    and launches all work asynchronously on `stream` (a cudaStream_t passed as void*;
- *    NULL = the legacy default stream).
+ *    their events for adx_index_prefill_host), and launches all work asynchronously on
+ *    `stream` (a cudaStream_t passed as void*; NULL = the legacy default stream).
  *    One exception: adx_index_prefill_noalloc runs on a fixed device array of
  *    ADX_STATIC_SCRATCH_BYTES compiled into the library (held on every GPU that loads it) and
  *    caches that array's device address per device and context.
@@ -162,12 +161,12 @@ adx_status adx_index_decode(const adx_operands* ops, int32_t K, int32_t* topk_id
  * and decode (row r = sequence r at position seq_len[r] - 1, its own S-row cache). */
 #define ADX_HISA_BLOCK 128
 
-/* Block keys kbar [n_seq, ceil(S / 128), d] in the key format (bf16; or e4m3 codes with
- * per-block scales kbar_scale [n_seq, ceil(S / 128)], scale = amax / 448, 1 for a zero block),
- * n_seq = 1 (prefill) or T (decode). A trailing partial block is the mean of the keys it
- * holds. Prefill: the blocks of the first min(S, q_pos0 + T) keys. Decode: the blocks of the
- * first seq_len[r] keys of each cache; last_only != 0 recomputes only the block holding each
- * sequence's last key (the one a decode step's appended key changes). Device pointers. */
+/* Block keys kbar [n_seq, ceil(S / 128), d] bf16, for either key format (e4m3 keys are decoded
+ * with their scales first): the mean of each block's keys, n_seq = 1 (prefill) or T (decode).
+ * A trailing partial block is the mean of the keys it holds. Prefill: the blocks of the first
+ * min(S, q_pos0 + T) keys. Decode: the blocks of the first seq_len[r] keys of each cache;
+ * last_only != 0 recomputes only the block holding each sequence's last key (the one a decode
+ * step's appended key changes). kbar_scale is ignored (NULL). Device pointers. */
 adx_status adx_hisa_block_keys(const adx_operands* ops, int32_t last_only, void* kbar,
                                float* kbar_scale, void* stream);
 
@@ -176,7 +175,9 @@ adx_status adx_hisa_block_keys(const adx_operands* ops, int32_t last_only, void*
 size_t adx_hisa_workspace_size(const adx_operands* ops, int32_t n_blocks, int32_t K,
                                int32_t blocks_external);
 
-/* HISA indexer step. kbar / kbar_scale from adx_hisa_block_keys (read only). Requires
+/* HISA indexer step. kbar from adx_hisa_block_keys (bf16, read only; kbar_scale is ignored):
+ * the block scores take bf16 queries (e4m3 queries decoded with their scales), the token
+ * refinement the operands as given. Requires
  * 2 <= n_blocks <= 255, K <= n_blocks * 128, T * n_blocks * 128 < 2^31, H = 64 (else
  * ADX_EUNSUPPORTED). Prefill rows are refined in groups of 4 consecutive rows that score the
  * union of their kept blocks together; each row's Top-K still ranges over its own blocks.
@@ -256,13 +257,14 @@ adx_status adx_group_query_mean(int32_t q_dtype, const void* q, const float* q_s
  *                                      t * rope_base^(-2i/rope_dim))
  *   w-bar_j = sigmoid([W_G h-bar]_j)
  * All pointers are device pointers to bf16 row-major arrays; weights in the [out, in] layout.
- * Requires d_c and d_h multiples of 8; cq, h and w_g 16-byte aligned; H_S <= 64;
+ * Requires d_c and d_h multiples of 8; cq, h, w_pool, w_q and w_g 16-byte aligned; H_S <= 64;
  * rope_dim <= 512; T / G <= 65535. Tokens past the last complete group are ignored. Invalid
  * arguments return ADX_EINVAL. The gate projection is taken from h-bar in fp32 inside the
  * pooling kernel, as per-column-block partial sums added in a fixed order (deterministic).
- * The projections run on cuBLAS (bf16 operands, fp32 accumulation) with one handle per device
- * created on first use; calls on one device must not be issued from several host threads at
- * the same time. */
+ * The projections W_pool and W_Q run on the library's tcgen05 GEMM (bf16 operands, fp32
+ * accumulation); c-bar is rounded to bf16 between them. The workspace starts with the device
+ * status word (ADX_STATUS_BYTES, zeroed once before the first call; read it with
+ * adx_read_device_status). */
 typedef struct {
   const void* cq;      /* [T, d_c] query latents */
   const void* h;       /* [T, d_h] normalized hidden states */

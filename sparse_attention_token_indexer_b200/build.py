@@ -3,8 +3,8 @@
     python -m sparse_attention_token_indexer_b200.build [--force]
 
 The library links the CUDA runtime statically and reaches the driver's tensor-map encoder
-through cudaGetDriverEntryPoint, so it needs no -lcuda at link time; cuBLAS (for the group
-indexer's projections) is linked dynamically.
+through cudaGetDriverEntryPoint, so it needs no -lcuda at link time; it links no other CUDA
+library.
 """
 
 import os
@@ -16,7 +16,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libadx.so")
 SOURCES = ["adx_api.cu", "score_sm100.cu", "select_topk.cu", "aux_kernels.cu", "adx_noalloc.cu",
-           "group_indexer.cu", "hisa.cu"]
+           "group_indexer.cu", "gemm_sm100.cu", "hisa.cu"]
 HEADERS = ["adx_internal.h", "sm100_ptx.cuh"]
 
 
@@ -53,9 +53,8 @@ def build(force=False, verbose=False):
                 cmd.insert(1, "-Xptxas=-v")
             subprocess.run(cmd, check=True)
     if force or _stale(LIB, objs):
-        cuda_lib = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "lib64")
         cmd = [nvcc(), "-shared", "-cudart", "static", "-gencode", "arch=compute_100a,code=sm_100a",
-               "-o", LIB] + objs + ["-lcublas", "-Xlinker", f"-rpath,{cuda_lib}"]
+               "-o", LIB] + objs
         subprocess.run(cmd, check=True)
     return LIB
 

@@ -53,6 +53,19 @@ struct Carve {
 // ------------------------------------------------------------------------------------
 // device properties and the driver's tensor-map encoder
 // ------------------------------------------------------------------------------------
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  static int cache[64] = {0};
+  if (dev < 0 || dev >= 64) return 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -72,18 +85,7 @@ EncodeTiledFn encoder() {
   return fn;
 }
 
-int sm_count() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  static int cache[64] = {0};
-  if (dev < 0 || dev >= 64) return 0;
-  if (cache[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    cache[dev] = n;
-  }
-  return cache[dev];
-}
+}  // namespace
 
 // 2-D map over `rows` rows of `d` elements (1 or 2 bytes), 128-byte swizzled boxes of
 // (128 bytes) x box_rows.
@@ -102,6 +104,8 @@ bool encode_rows(CUtensorMap* m, const void* base, bool one_byte, int d, int64_t
              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+namespace {
 
 // ------------------------------------------------------------------------------------
 // validation
@@ -561,9 +565,17 @@ adx_status hisa_check(const adx_operands* o, int32_t n_blocks, int32_t K) {
   return ADX_OK;
 }
 
+// bf16 queries for the block pass, prepared apart when the keys are e4m3 (the block keys are
+// bf16 in both formats)
+size_t ws_prepare_bf16(const adx_operands* o, int64_t R) {
+  return align_up(static_cast<size_t>(R) * o->H * o->d * 2, kAlign) +
+         align_up(static_cast<size_t>(R), kAlign);
+}
+
 size_t ws_hisa(const adx_operands* o, int32_t n_blocks, int32_t K, bool blocks_external) {
   const int64_t T = o->T, nbmax = hisa_nbmax(o), nc = static_cast<int64_t>(n_blocks) * kTileM;
   size_t b = kStatusBytes + ws_prepare(o, T);
+  if (fp8_keys(o)) b += ws_prepare_bf16(o, T);
   b += align_up(static_cast<size_t>(T) * 4, kAlign);                         // row blocks
   b += align_up(static_cast<size_t>(T) * ld_for(nbmax) * 4, kAlign);         // block scores
   if (!blocks_external) b += align_up(static_cast<size_t>(T) * n_blocks * 4, kAlign);
@@ -1118,12 +1130,13 @@ adx_status adx_hisa_block_keys(const adx_operands* o, int32_t last_only, void* k
   const bool decode = o != nullptr && o->seq_len != nullptr;
   adx_status r = check_operands(o, decode);
   if (r != ADX_OK) return r;
-  if (!kbar || (fp8_keys(o) != (kbar_scale != nullptr))) return ADX_EINVAL;
+  (void)kbar_scale;  // block keys are bf16 for either key format
+  if (!kbar) return ADX_EINVAL;
   const int64_t len = decode ? 0 : std::min<int64_t>(o->S, o->q_pos0 + o->T);
   const cudaError_t e = counted(launch_block_keys(
       o->k, o->k_scale, fp8_keys(o), o->S, o->d, decode ? o->T : 1, o->seq_len,
       static_cast<int32_t>(len), last_only != 0, static_cast<int32_t>(hisa_nbmax(o)), kbar,
-      kbar_scale, static_cast<cudaStream_t>(stream)));
+      static_cast<cudaStream_t>(stream)));
   if (e == cudaErrorInvalidValue) return ADX_EUNSUPPORTED;
   return e == cudaSuccess ? ADX_OK : ADX_ECUDA;
 }
@@ -1133,7 +1146,8 @@ adx_status adx_index_hisa(const adx_operands* o, const void* kbar, const float* 
                           int32_t* blocks_out, void* ws, size_t ws_bytes, void* stream) {
   adx_status r = hisa_check(o, n_blocks, K);
   if (r != ADX_OK) return r;
-  if (!kbar || (fp8_keys(o) != (kbar_scale != nullptr)) || !topk_idx || !ws) return ADX_EINVAL;
+  (void)kbar_scale;  // block keys are bf16 for either key format
+  if (!kbar || !topk_idx || !ws) return ADX_EINVAL;
   if (ws_bytes < ws_hisa(o, n_blocks, K, blocks_out != nullptr)) return ADX_EWORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool decode = o->seq_len != nullptr;
@@ -1145,6 +1159,19 @@ adx_status adx_index_hisa(const adx_operands* o, const void* kbar, const float* 
   int32_t* row_blk = cv.take<int32_t>(static_cast<size_t>(T) * 4);
   Prepared pq;  // the preparation also writes each row's block
   if ((r = prepare(o, o->q, o->q_scale, o->w, T, cv, s, pq, row_blk)) != ADX_OK) return r;
+  // the block pass scores bf16 block keys, so it takes bf16 queries: the same preparation
+  // without the e4m3 step when the keys are e4m3
+  Prepared pb = pq;
+  if (fp8_keys(o)) {
+    void* qo = cv.take<uint8_t>(static_cast<size_t>(T) * o->H * o->d * 2);
+    int8_t* fl = cv.take<int8_t>(static_cast<size_t>(T));
+    if (counted(launch_prepare_q(o->q, o->q_scale, o->q_dtype == ADX_E4M3, false, o->w, T, o->H,
+                                 o->d, qo, nullptr, fl, s)) != cudaSuccess)
+      return ADX_ECUDA;
+    pb.q = qo;
+    pb.q_scale = nullptr;
+    pb.fold = fl;
+  }
   float* bsc = cv.take<float>(static_cast<size_t>(T) * ldb * 4);
   int32_t* blocks =
       blocks_out ? blocks_out : cv.take<int32_t>(static_cast<size_t>(T) * n_blocks * 4);
@@ -1153,10 +1180,11 @@ adx_status adx_index_hisa(const adx_operands* o, const void* kbar, const float* 
   // 1. block scores: Eq. (1) on the block keys, block b visible to a row whose position lies
   //    in block >= b
   {
-    ScorePlan p = decode ? rowwise_plan(o, pq, bsc, ldb)
-                         : base_plan(o, pq, score_tokens_per_tile(o->H));
+    ScorePlan p = decode ? rowwise_plan(o, pb, bsc, ldb)
+                         : base_plan(o, pb, score_tokens_per_tile(o->H));
+    p.fp8 = false;
     ScoreArgs& a = p.a;
-    a.k_scale = kbar_scale;
+    a.k_scale = nullptr;
     a.row_pos = row_blk;
     a.status = st;
     a.scores = bsc;
@@ -1174,7 +1202,7 @@ adx_status adx_index_hisa(const adx_operands* o, const void* kbar, const float* 
     const int64_t vis_blocks =
         decode ? nbmax : (std::min<int64_t>(o->S, o->q_pos0 + T) + kTileM - 1) / kTileM;
     finish_plan(p, (vis_blocks + kTileM - 1) / kTileM);
-    if ((r = run_score(p, pq.q, kbar, (decode ? T : 1) * nbmax, s)) != ADX_OK) return r;
+    if ((r = run_score(p, pb.q, kbar, (decode ? T : 1) * nbmax, s)) != ADX_OK) return r;
   }
   // 2. forced blocks, then the block Top-n; rows that fit the one-warp select get the forced
   //    blocks there, longer ones from a kernel that raises their scores first

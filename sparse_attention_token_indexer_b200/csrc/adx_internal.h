@@ -20,6 +20,7 @@ constexpr size_t kStatusBytes = 256;
 constexpr int kWhereScore = 1;
 constexpr int kWhereSelect = 2;
 constexpr int kWhereCheck = 3;
+constexpr int kWhereGemm = 4;
 
 constexpr int kTileM = 128;  // keys per MMA tile (TMEM lanes)
 
@@ -190,13 +191,11 @@ cudaError_t launch_prepare_q(const void* q, const float* q_scale, bool in_e4m3, 
                              RowBlocks rb = RowBlocks{});
 
 // HISA block keys: the mean of each 128-key block of each key range (n_seq ranges of S rows;
-// length seq_len[b], or len_fixed without seq_len), stored like keys in kbar [n_seq, nbmax, d]
-// (e4m3 with per-block scales kbar_scale [n_seq, nbmax]); last_only: just the block holding
-// each range's last key.
+// length seq_len[b], or len_fixed without seq_len; e4m3 keys decoded with their scales), in
+// bf16 in kbar [n_seq, nbmax, d]; last_only: just the block holding each range's last key.
 cudaError_t launch_block_keys(const void* k, const float* k_scale, bool fp8, int64_t S, int d,
                               int32_t n_seq, const int32_t* seq_len, int32_t len_fixed,
-                              bool last_only, int32_t nbmax, void* kbar, float* kbar_scale,
-                              cudaStream_t s);
+                              bool last_only, int32_t nbmax, void* kbar, cudaStream_t s);
 // Union of the block lists (blocks [R, n_blocks], -1 padded) of each group of `tok`
 // consecutive rows: uni [groups, tok * n_blocks] distinct blocks, count [groups] how many,
 // slot [groups, tok * n_blocks] byte j = slot of the union entry in row j's list (0xFF: none).
@@ -211,6 +210,18 @@ cudaError_t launch_force_blocks(float* scores, int64_t ld, int32_t R, const int3
 // Argument checks of adx_index_prefill that need no device: the operands (prefill layout)
 // and K. ADX_OK, ADX_EINVAL or ADX_EUNSUPPORTED, exactly as adx_index_prefill returns them.
 adx_status check_prefill_args(const adx_operands* o, int32_t K);
+
+// 2-D tensor map over `rows` rows of `d` elements (1 or 2 bytes each) with 128-byte swizzled
+// boxes of 128 bytes x box_rows; false when the driver's encoder rejects it.
+bool encode_rows(CUtensorMap* m, const void* base, bool one_byte, int d, int64_t rows,
+                 int box_rows);
+// Y [n, m] (bf16, or fp32 with out_f32) = X [n, k] W^T for bf16 W [m, k] (tm_w) and X [n, k]
+// (tm_x), both mapped by encode_rows with gemm_box_rows() rows per box. Timeouts of the
+// kernel's bounded waits are recorded in *st.
+cudaError_t launch_gemm_bf16(const CUtensorMap& tm_w, const CUtensorMap& tm_x, void* y,
+                             bool out_f32, int m, int n, int k, DeviceStatus* st,
+                             uint64_t timeout_ns, cudaStream_t s);
+int gemm_box_rows();
 
 // Adds n to the library's launch counter (kernels launched outside the API file).
 void add_launches(int n);

@@ -361,7 +361,8 @@ cudaError_t launch_prepare_q(const void* q, const float* q_scale, bool in_e4m3, 
   if (!in_e4m3 && out_e4m3)
     return launch_prepare_rows<false, true>(q, q_scale, w, rows, H, d, q_out, q_scale_out,
                                             fold_flag, rb, s);
-  return cudaErrorNotSupported;
+  return launch_prepare_rows<true, false>(q, q_scale, w, rows, H, d, q_out, q_scale_out,
+                                          fold_flag, rb, s);
 }
 
 cudaError_t launch_pack_candidates(const void* k, const float* k_scale, int64_t key_batch_stride,

@@ -4,11 +4,11 @@
 //   h-bar = mean_i h_i                                       (normalized hidden states)
 //   q-bar_j = RoPE_t([W_Q c-bar]_j),   w-bar_j = sigmoid([W_G h-bar]_j).
 // A pooling kernel (16-byte loads, HBM-bound) builds [max; min; mean] and, from h-bar in fp32,
-// the gate projection's partial sums; the two plain GEMMs (W_pool, W_Q) run on cuBLAS (bf16
-// operands, fp32 accumulation); a last kernel applies RoPE at the anchor and the sigmoid.
+// the gate projection's partial sums; the two projections (W_pool, W_Q) run on this library's
+// tcgen05 GEMM (gemm_sm100.cu: bf16 operands, fp32 accumulation in TMEM); a last kernel
+// applies RoPE at the anchor and the sigmoid.
 // RoPE rotates the pairs (2i, 2i+1), i < rope_dim/2, by the angle t * base^(-2i/rope_dim)
 // (the paper names RoPE at the anchor, not its layout).
-#include <cublas_v2.h>
 #include <cuda_bf16.h>
 
 #include <cstdint>
@@ -21,7 +21,7 @@ namespace adx {
 namespace {
 
 constexpr size_t kAlignGi = 256;
-constexpr size_t kCublasWorkspace = 32u << 20;
+constexpr uint64_t kGemmTimeoutNs = 2000000000ull;  // 2 s per device-side wait
 
 size_t up(size_t x) { return (x + kAlignGi - 1) / kAlignGi * kAlignGi; }
 
@@ -189,30 +189,6 @@ gi_finish_kernel(const float* __restrict__ qpre, const float* __restrict__ gpart
   }
 }
 
-// One cuBLAS handle per device, created on first use.
-constexpr int kMaxDevicesGi = 64;
-std::mutex g_blas_mutex;
-cublasHandle_t g_blas[kMaxDevicesGi] = {nullptr};
-
-cublasHandle_t blas_handle() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevicesGi) return nullptr;
-  std::lock_guard<std::mutex> lock(g_blas_mutex);
-  if (g_blas[dev] == nullptr && cublasCreate(&g_blas[dev]) != CUBLAS_STATUS_SUCCESS)
-    g_blas[dev] = nullptr;
-  return g_blas[dev];
-}
-
-// Row-major Y [n, m] = X [n, k] * W^T with W row-major [m, k]: in cuBLAS's column-major
-// terms Y^T [m, n] = W [m, k] (given as its transpose) * X^T [k, n].
-cublasStatus_t linear(cublasHandle_t hb, const void* W, const void* X, void* Y,
-                      cudaDataType_t ytype, int m, int n, int k) {
-  const float one = 1.f, zero = 0.f;
-  return cublasGemmEx(hb, CUBLAS_OP_T, CUBLAS_OP_N, m, n, k, &one, W, CUDA_R_16BF, k, X,
-                      CUDA_R_16BF, k, &zero, Y, ytype, m, CUBLAS_COMPUTE_32F,
-                      CUBLAS_GEMM_DEFAULT);
-}
-
 int pool_ctas(const adx_group_indexer* gi) {
   return (gi->d_c / 8 + gi->d_h / 8 + kPoolThreads - 1) / kPoolThreads;
 }
@@ -231,8 +207,8 @@ bool gi_valid(const adx_group_indexer* gi, int G) {
 
 size_t gi_workspace(const adx_group_indexer* gi, int G) {
   const size_t ng = gi->T / G;
-  return up(ng * 3 * gi->d_c * 2) + up(ng * pool_ctas(gi) * gi->H_S * 4) +
-         up(ng * gi->d_c * 2) + up(ng * gi->H_S * gi->d * 4) + kCublasWorkspace;
+  return kStatusBytes + up(ng * 3 * gi->d_c * 2) + up(ng * pool_ctas(gi) * gi->H_S * 4) +
+         up(ng * gi->d_c * 2) + up(ng * gi->H_S * gi->d * 4);
 }
 
 }  // namespace
@@ -250,8 +226,6 @@ adx_status adx_group_indexer_queries(const adx_group_indexer* gi, int32_t G, voi
                                      float* wbar_out, void* ws, size_t ws_bytes, void* stream) {
   if (!gi_valid(gi, G) || !qbar_out || !wbar_out || !ws) return ADX_EINVAL;
   if (ws_bytes < gi_workspace(gi, G)) return ADX_EWORKSPACE;
-  cublasHandle_t hb = blas_handle();
-  if (!hb) return ADX_ECUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int ng = gi->T / G, dc = gi->d_c, dh = gi->d_h, HS = gi->H_S, d = gi->d;
   uint8_t* p = static_cast<uint8_t*>(ws);
@@ -260,22 +234,32 @@ adx_status adx_group_indexer_queries(const adx_group_indexer* gi, int32_t G, voi
     p += up(bytes);
     return r;
   };
+  auto* st = reinterpret_cast<DeviceStatus*>(take(kStatusBytes));
   const int nparts = pool_ctas(gi);
   auto* pooled = reinterpret_cast<__nv_bfloat16*>(take(static_cast<size_t>(ng) * 3 * dc * 2));
   auto* gpart = reinterpret_cast<float*>(take(static_cast<size_t>(ng) * nparts * HS * 4));
   auto* cbar = reinterpret_cast<__nv_bfloat16*>(take(static_cast<size_t>(ng) * dc * 2));
   auto* qpre = reinterpret_cast<float*>(take(static_cast<size_t>(ng) * HS * d * 4));
-  void* blas_ws = take(kCublasWorkspace);
+  // tensor maps of both projections: W rows and X rows in boxes of 128 rows x 64 k-elements
+  CUtensorMap tw_pool, tx_pool, tw_q, tx_q;
+  const int box = gemm_box_rows();
+  if (!encode_rows(&tw_pool, gi->w_pool, false, 3 * dc, dc, box) ||
+      !encode_rows(&tx_pool, pooled, false, 3 * dc, ng, box) ||
+      !encode_rows(&tw_q, gi->w_q, false, dc, static_cast<int64_t>(HS) * d, box) ||
+      !encode_rows(&tx_q, cbar, false, dc, ng, box))
+    return ADX_EINVAL;
   gi_pool_kernel<<<dim3(nparts, ng), kPoolThreads, 0, s>>>(
       static_cast<const __nv_bfloat16*>(gi->cq), static_cast<const __nv_bfloat16*>(gi->h),
       static_cast<const __nv_bfloat16*>(gi->w_g), G, dc, dh, HS, pooled, gpart);
   if (cudaGetLastError() != cudaSuccess) return ADX_ECUDA;
   add_launches(1);
-  if (cublasSetStream(hb, s) != CUBLAS_STATUS_SUCCESS ||
-      cublasSetWorkspace(hb, blas_ws, kCublasWorkspace) != CUBLAS_STATUS_SUCCESS ||
-      linear(hb, gi->w_pool, pooled, cbar, CUDA_R_16BF, dc, ng, 3 * dc) != CUBLAS_STATUS_SUCCESS ||
-      linear(hb, gi->w_q, cbar, qpre, CUDA_R_32F, HS * d, ng, dc) != CUBLAS_STATUS_SUCCESS)
+  // c-bar [ng, d_c] = pooled [ng, 3 d_c] W_pool^T;  q-bar before RoPE [ng, H_S d] = c-bar W_Q^T
+  if (launch_gemm_bf16(tw_pool, tx_pool, cbar, false, dc, ng, 3 * dc, st, kGemmTimeoutNs, s) !=
+          cudaSuccess ||
+      launch_gemm_bf16(tw_q, tx_q, qpre, true, HS * d, ng, dc, st, kGemmTimeoutNs, s) !=
+          cudaSuccess)
     return ADX_ECUDA;
+  add_launches(2);
   gi_finish_kernel<<<ng, 256, 0, s>>>(qpre, gpart, nparts, HS, d, gi->rope_dim, gi->rope_base,
                                       gi->q_pos0, G, static_cast<__nv_bfloat16*>(qbar_out),
                                       wbar_out);

@@ -3,7 +3,8 @@
 // ADIndex paper uses for it (Appendix C.5): 128-key blocks pooled by their mean, the first
 // block and the query's own block always among the candidates.
 //   * block keys: the mean of each block of 128 keys (decoded with their scales for e4m3),
-//     stored like keys (bf16, or e4m3 with a per-block scale amax / 448);
+//     stored in bf16 for either key format, so block scores carry no FP8 rounding of their
+//     own (the block pass scores them against bf16 queries);
 //   * forcing: the two forced blocks' scores raised to +inf ahead of the block Top-n (for
 //     block rows longer than the one-warp select holds; that select forces them itself).
 // The block of each row's position is a by-product of the query preparation.
@@ -29,9 +30,8 @@ template <bool FP8>
 __global__ void __launch_bounds__(kBkThreads)
 block_keys_kernel(const uint8_t* __restrict__ k, const float* __restrict__ k_scale, int64_t S,
                   int d, const int32_t* __restrict__ seq_len, int32_t len_fixed, int last_only,
-                  int nbmax, uint8_t* __restrict__ kbar, float* __restrict__ kbar_scale) {
+                  int nbmax, uint8_t* __restrict__ kbar) {
   __shared__ float part[kBkThreads];
-  __shared__ float red[kBkThreads / 32];
   const int64_t b = blockIdx.y;
   int64_t len = seq_len != nullptr ? seq_len[b] : len_fixed;
   len = len < S ? len : S;
@@ -62,23 +62,8 @@ block_keys_kernel(const uint8_t* __restrict__ k, const float* __restrict__ k_sca
     mean = s / static_cast<float>(n);
   }
   const int64_t out = b * nbmax + blk;
-  if constexpr (FP8) {
-    // per-block scale amax / 448 (1 for an all-zero block), like the key rows
-    float m = threadIdx.x < d ? fabsf(mean) : 0.f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-    __syncthreads();
-    float amax = 0.f;
-    for (int w = 0; w < kBkThreads / 32; ++w) amax = fmaxf(amax, red[w]);
-    const float sc = amax > 0.f ? amax / 448.f : 1.f;
-    if (threadIdx.x < d)
-      kbar[out * d + threadIdx.x] = __nv_cvt_float_to_fp8(mean / sc, __NV_SATFINITE, __NV_E4M3);
-    if (threadIdx.x == 0) kbar_scale[out] = sc;
-  } else {
-    if (threadIdx.x < d)
-      reinterpret_cast<__nv_bfloat16*>(kbar)[out * d + threadIdx.x] = __float2bfloat16_rn(mean);
-  }
+  if (threadIdx.x < d)
+    reinterpret_cast<__nv_bfloat16*>(kbar)[out * d + threadIdx.x] = __float2bfloat16_rn(mean);
 }
 
 // Forced blocks: where more than n_blocks blocks are visible, block 0 and the row's own block
@@ -174,8 +159,7 @@ cudaError_t launch_block_union(const int32_t* blocks, int32_t n_blocks, int32_t 
 
 cudaError_t launch_block_keys(const void* k, const float* k_scale, bool fp8, int64_t S, int d,
                               int32_t n_seq, const int32_t* seq_len, int32_t len_fixed,
-                              bool last_only, int32_t nbmax, void* kbar, float* kbar_scale,
-                              cudaStream_t s) {
+                              bool last_only, int32_t nbmax, void* kbar, cudaStream_t s) {
   if (n_seq <= 0 || nbmax <= 0) return cudaSuccess;
   if (kBkThreads % d != 0) return cudaErrorInvalidValue;
   const dim3 grid(last_only ? 1 : nbmax, n_seq);
@@ -183,10 +167,10 @@ cudaError_t launch_block_keys(const void* k, const float* k_scale, bool fp8, int
   uint8_t* out = static_cast<uint8_t*>(kbar);
   if (fp8)
     block_keys_kernel<true><<<grid, kBkThreads, 0, s>>>(kc, k_scale, S, d, seq_len, len_fixed,
-                                                        last_only ? 1 : 0, nbmax, out, kbar_scale);
+                                                        last_only ? 1 : 0, nbmax, out);
   else
     block_keys_kernel<false><<<grid, kBkThreads, 0, s>>>(kc, k_scale, S, d, seq_len, len_fixed,
-                                                         last_only ? 1 : 0, nbmax, out, kbar_scale);
+                                                         last_only ? 1 : 0, nbmax, out);
   return cudaGetLastError();
 }
 

@@ -168,24 +168,22 @@ def index_decode(q, w, k, seq_len, K, q_scale=None, k_scale=None, with_scores=Fa
 
 def hisa_block_keys(q, w, k, q_scale=None, k_scale=None, q_pos0=0, seq_len=None,
                     last_only=False, out=None, stream=None):
-    """HISA block keys (means of 128-key blocks) in the key format -> (kbar, kbar_scale or
-    None): [ceil(S / 128), d] (prefill) or [T, ceil(S / 128), d] (decode). `out` updates an
-    existing (kbar, kbar_scale) pair in place (decode steps use last_only=True)."""
+    """HISA block keys (means of 128-key blocks, bf16 for either key format) -> (kbar, None):
+    [ceil(S / 128), d] (prefill) or [T, ceil(S / 128), d] (decode). `out` updates an existing
+    (kbar, _) pair in place (decode steps use last_only=True)."""
     ops = make_operands(q, w, k, q_scale, k_scale, q_pos0, seq_len)
     nb = (ops.S + L.ADX_HISA_BLOCK - 1) // L.ADX_HISA_BLOCK
     shape = (nb, ops.d) if seq_len is None else (ops.T, nb, ops.d)
     if out is None:
-        kbar = torch.empty(*shape, dtype=k.dtype, device=k.device)
-        ks = torch.empty(*shape[:-1], dtype=torch.float32, device=k.device) \
-            if k.dtype == torch.uint8 else None
+        kbar = torch.empty(*shape, dtype=torch.bfloat16, device=k.device)
     else:
-        kbar, ks = out
-        _dev(kbar, "kbar", k.dtype), _dev(ks, "kbar_scale", torch.float32)
+        kbar = out[0]
+        _dev(kbar, "kbar", torch.bfloat16)
         if tuple(kbar.shape) != shape:
             raise ValueError(f"kbar must be {shape}")
     L.check("adx_hisa_block_keys", L.lib().adx_hisa_block_keys(
-        ctypes.byref(ops), int(bool(last_only)), _p(kbar), _p(ks), _stream(stream)))
-    return kbar, ks
+        ctypes.byref(ops), int(bool(last_only)), _p(kbar), None, _stream(stream)))
+    return kbar, None
 
 
 def index_hisa(q, w, k, kbar, K, n_blocks=64, q_scale=None, k_scale=None, kbar_scale=None,
@@ -194,7 +192,7 @@ def index_hisa(q, w, k, kbar, K, n_blocks=64, q_scale=None, k_scale=None, kbar_s
     """HISA indexer (block filter, then token refinement) -> (topk_idx [T, K] int32,
     topk_score or None, blocks [T, n_blocks] int32 or None)."""
     ops = make_operands(q, w, k, q_scale, k_scale, q_pos0, seq_len)
-    _dev(kbar, "kbar", k.dtype), _dev(kbar_scale, "kbar_scale", torch.float32)
+    _dev(kbar, "kbar", torch.bfloat16)
     idx = torch.empty(ops.T, K, dtype=torch.int32, device=q.device)
     sc = torch.empty(ops.T, K, dtype=torch.float32, device=q.device) if with_scores else None
     blocks = torch.empty(ops.T, n_blocks, dtype=torch.int32, device=q.device) \
@@ -204,7 +202,7 @@ def index_hisa(q, w, k, kbar, K, n_blocks=64, q_scale=None, k_scale=None, kbar_s
         raise L.AdxError("adx_hisa_workspace_size", L.ADX_EINVAL)
     buf = _ws(ws, q.device).get(need)
     L.check("adx_index_hisa", L.lib().adx_index_hisa(
-        ctypes.byref(ops), _p(kbar), _p(kbar_scale), n_blocks, K, _p(idx), _p(sc), _p(blocks),
+        ctypes.byref(ops), _p(kbar), None, n_blocks, K, _p(idx), _p(sc), _p(blocks),
         _p(buf), buf.numel(), _stream(stream)))
     return idx, sc, blocks
 

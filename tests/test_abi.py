@@ -95,7 +95,6 @@ def test_hisa_host_validation(lib):
     assert _hisa(lib, o, n_blocks=256) == L.ADX_EINVAL               # slot bytes hold < 255
     assert _hisa(lib, o, n_blocks=4, K=4 * 128 + 1) == L.ADX_EINVAL  # K beyond the candidates
     assert _hisa(lib, o, kbar=0) == L.ADX_EINVAL
-    assert _hisa(lib, o, kbar_scale=64) == L.ADX_EINVAL               # bf16 keys: no scales
     assert _hisa(lib, _ops(H=16)) == L.ADX_EUNSUPPORTED               # 64 heads only
     assert _hisa(lib, o, ws_bytes=16) == L.ADX_EWORKSPACE
     assert lib.adx_hisa_workspace_size(ctypes.byref(o), 1, 64, 0) == 0
