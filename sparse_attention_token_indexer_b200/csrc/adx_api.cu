@@ -347,7 +347,7 @@ adx_status run_flat(const adx_operands* o, int K, int32_t* topk_idx, float* topk
   sa.ld = ld;
   sa.rows_per_batch = o->T;
   sa.len_mode = 1;
-  sa.len_cap = o->S;
+  sa.len_cap = static_cast<int32_t>(max_keys);  // no row is longer: picks the select class
   sa.pos_base = o->q_pos0;
   sa.pos_step = 1;
   sa.K = K;

@@ -60,6 +60,11 @@ __device__ __forceinline__ uint32_t block_inclusive_scan(uint32_t x, uint32_t* w
   return x + before;
 }
 
+// The fp32 value of an order-preserving key (inverse of order_key).
+__device__ __forceinline__ float key_value_long(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
 // Position of element id through the row's map (per element, or per block of 2^shift).
 __device__ __forceinline__ int32_t map_id(const int32_t* map, int32_t id, int shift) {
   if (map == nullptr || id < 0) return id;
@@ -86,14 +91,13 @@ __device__ __forceinline__ int64_t row_length(const SelectArgs& a, int r) {
   return n < 0 ? 0 : n;
 }
 
-__global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a) {
-  __shared__ uint32_t hist[kBins];
-  __shared__ uint32_t warp_tot[32];
-  __shared__ uint32_t sh_bin, sh_above;
-
-  const int seg = blockIdx.x % a.n_seg;
-  const int r = blockIdx.x / a.n_seg;
-  if (r >= a.rows) return;
+// Multi-pass radix select of one row (or row segment) streamed from global memory: three
+// digit passes (12 + 12 + 8 bits) over the row, then an ordered output pass. hist holds kBins
+// words, warp_tot 32, sh two; all in shared memory, all threads of the CTA take part.
+__device__ void radix_row(const SelectArgs& a, int r, int seg, uint32_t* hist, uint32_t* warp_tot,
+                          uint32_t* sh) {
+  uint32_t& sh_bin = sh[0];
+  uint32_t& sh_above = sh[1];
   const int64_t n = row_length(a, r);
   const int64_t lo = static_cast<int64_t>(seg) * a.seg_len;
   const int64_t hi = a.n_seg == 1 ? n : min(n, lo + a.seg_len);
@@ -216,6 +220,16 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a)
     a.out_idx[out_base + j] = -1;
     if (a.out_val) a.out_val[out_base + j] = -INFINITY;
   }
+}
+
+__global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a) {
+  __shared__ uint32_t hist[kBins];
+  __shared__ uint32_t warp_tot[32];
+  __shared__ uint32_t sh[2];
+  const int seg = blockIdx.x % a.n_seg;
+  const int r = blockIdx.x / a.n_seg;
+  if (r >= a.rows) return;
+  radix_row(a, r, seg, hist, warp_tot, sh);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -777,6 +791,297 @@ select_reg_kernel(const SelectArgs a, int row0) {
 }
 
 // ---------------------------------------------------------------------------------------
+// Many rows longer than a register-resident select holds (chunked prefill past 32K keys):
+// a threshold from a sample, then one streaming pass.
+//   1. Sample: every kSampleStride-th tile of 128 elements (m of the row's n). Its key range
+//      and a 12-bit histogram below the range's common high bits give the bin of the sample's
+//      r-th largest key, r = 5/4 * K * m / n + 8, whose lower edge is the threshold tau: about
+//      5/4 of K elements of the row are expected at or above it.
+//   2. One pass gathers every valid element >= tau into shared memory in index order (a block
+//      scan of per-thread masks per 8192 elements). Fewer than K gathered (the estimate was
+//      too high): tau is lowered (rank 4r, then every element) and the pass repeated; more
+//      than the buffer holds (many equal keys): the row takes the multi-pass radix select.
+//   3. The exact K-th largest among the gathered keys (8-bit digit histograms), and the
+//      selected elements written in index order: every key above it and the lowest-indexed
+//      keys equal to it.
+// ---------------------------------------------------------------------------------------
+constexpr int kSampleStride = 16;
+constexpr int kLongCap = 6144;      // gathered elements
+constexpr int kLongPer = 16;        // elements per thread per gather step
+
+__global__ void __launch_bounds__(kSelThreads) long_select_kernel(const SelectArgs a) {
+  __shared__ uint32_t hist[kBins];
+  __shared__ uint32_t warp_tot[32];
+  __shared__ uint32_t sh[2];
+  extern __shared__ __align__(16) uint32_t long_smem[];
+  uint32_t* ck = long_smem;                                   // gathered keys, index order
+  int32_t* cix = reinterpret_cast<int32_t*>(long_smem + kLongCap);  // their element indices
+  __shared__ uint32_t red_min[kSelWarps], red_max[kSelWarps], red_cnt[kSelWarps];
+  __shared__ uint32_t sh_bin, sh_above, sh_inbin;
+  __shared__ unsigned long long warp_tot64[kSelWarps];
+
+  const int r = blockIdx.x;
+  if (r >= a.rows) return;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t n = row_length(a, r);
+  const float* vals = a.vals + static_cast<int64_t>(r) * a.ld;
+  const int32_t* in_idx = a.in_idx ? a.in_idx + static_cast<int64_t>(r) * a.ld : nullptr;
+  const int32_t* map =
+      a.idx_map ? a.idx_map + static_cast<int64_t>(r / a.rows_per_batch) * a.map_stride : nullptr;
+  const int64_t out_base = static_cast<int64_t>(r) * a.out_ld;
+  const uint32_t K = static_cast<uint32_t>(a.K);
+
+  // ---- 1. the sample's key range, then its histogram below the common high bits
+  const int64_t n_tiles = (n + 127) / 128;
+  const int64_t n_samp = (n_tiles + kSampleStride - 1) / kSampleStride;
+  uint32_t kmin = 0xffffffffu, kmax = 0u, cnt = 0u;
+  for (int64_t t = warp; t < n_samp; t += kSelWarps) {
+    const int64_t base = t * kSampleStride * 128;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = base + u * 32 + lane;
+      const float v = i < n ? vals[i] : -INFINITY;
+      if (is_valid(v)) {
+        const uint32_t k = order_key(v);
+        kmin = min(kmin, k);
+        kmax = max(kmax, k);
+        ++cnt;
+      }
+    }
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  cnt = __reduce_add_sync(0xffffffffu, cnt);
+  if (lane == 0) {
+    red_min[warp] = kmin;
+    red_max[warp] = kmax;
+    red_cnt[warp] = cnt;
+  }
+  __syncthreads();
+  kmin = 0xffffffffu;
+  kmax = 0u;
+  uint32_t m = 0u;
+#pragma unroll
+  for (int w = 0; w < kSelWarps; ++w) {
+    kmin = min(kmin, red_min[w]);
+    kmax = max(kmax, red_max[w]);
+    m += red_cnt[w];
+  }
+  const uint32_t diff = kmin ^ kmax;
+  const int shift = diff == 0u ? 0 : 32 - __clz(diff);   // bits above are common to the sample
+  const int wbits = min(12, shift);
+  const int ns = shift - wbits;
+  const uint32_t top = shift >= 32 ? 0u : (kmax >> shift);
+  for (int i = threadIdx.x; i < kBins; i += kSelThreads) hist[i] = 0;
+  __syncthreads();
+  for (int64_t t = warp; t < n_samp; t += kSelWarps) {
+    const int64_t base = t * kSampleStride * 128;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = base + u * 32 + lane;
+      const float v = i < n ? vals[i] : -INFINITY;
+      if (is_valid(v)) atomicAdd(&hist[(order_key(v) >> ns) & ((1u << wbits) - 1u)], 1u);
+    }
+  }
+  __syncthreads();
+
+  // ---- 2. threshold from the sample, one gathering pass (repeated with a lower threshold if
+  //         it gathered fewer than K elements)
+  uint32_t C = 0;        // valid elements >= tau in the row
+  uint32_t tau = 0u;     // 0: every valid element (valid keys are > 0)
+  const uint64_t r0 = static_cast<uint64_t>(1.25 * K * (static_cast<double>(m) / (n > 0 ? n : 1))) + 8;
+#pragma unroll 1
+  for (int attempt = 0; attempt < 3; ++attempt) {
+    const uint64_t want = attempt == 0 ? r0 : r0 * 4;
+    tau = 0u;
+    if (attempt < 2 && want < m) {
+      // the bin holding the sample's want-th largest key, by a block scan from the top
+      const int nb = 1 << wbits;
+      const int bpt = nb >= kSelThreads ? nb / kSelThreads : 1;
+      const bool owner = static_cast<int>(threadIdx.x) * bpt < nb;
+      const int b0 = nb - (static_cast<int>(threadIdx.x) + 1) * bpt;
+      uint32_t mine = 0;
+      if (owner)
+        for (int q = 0; q < bpt; ++q) mine += hist[b0 + q];
+      uint32_t tot;
+      const uint32_t incl = block_inclusive_scan(mine, warp_tot, tot);
+      const uint32_t excl = incl - mine;
+      if (owner && excl < want && want <= incl) {
+        uint32_t above = excl;
+        for (int q = bpt - 1; q >= 0; --q) {
+          above += hist[b0 + q];
+          if (above >= want) {
+            sh_bin = static_cast<uint32_t>(b0 + q);
+            break;
+          }
+        }
+      }
+      __syncthreads();
+      tau = shift >= 32 ? (sh_bin << ns) : ((top << shift) | (sh_bin << ns));
+      if (tau == 0u) tau = 1u;
+    }
+    // gather every valid element >= tau, in index order
+    C = 0;
+    for (int64_t base = 0; base < n; base += static_cast<int64_t>(kSelThreads) * kLongPer) {
+      const int64_t i0 = base + static_cast<int64_t>(threadIdx.x) * kLongPer;
+      uint32_t key[kLongPer];
+      uint32_t msk = 0;
+#pragma unroll
+      for (int j = 0; j < kLongPer; j += 4) {
+        float v[4];
+        if (i0 + j + 4 <= n) {
+          const float4 f = *reinterpret_cast<const float4*>(vals + i0 + j);
+          v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+        } else {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) v[u] = (i0 + j + u < n) ? vals[i0 + j + u] : -INFINITY;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          key[j + u] = order_key(v[u]);
+          if (is_valid(v[u]) && key[j + u] >= tau) msk |= 1u << (j + u);
+        }
+      }
+      const uint32_t nm = __popc(msk);
+      uint32_t tot;
+      uint32_t at = C + block_inclusive_scan(nm, warp_tot, tot) - nm;
+#pragma unroll
+      for (int j = 0; j < kLongPer; ++j) {
+        if (msk & (1u << j)) {
+          if (at < static_cast<uint32_t>(kLongCap)) {
+            ck[at] = key[j];
+            cix[at] = static_cast<int32_t>(i0 + j);
+          }
+          ++at;
+        }
+      }
+      C += tot;
+    }
+    __syncthreads();
+    if (C >= K || tau == 0u) break;
+  }
+  if (C > static_cast<uint32_t>(kLongCap)) {  // too many equal keys to gather: radix passes
+    radix_row(a, r, 0, hist, warp_tot, sh);
+    return;
+  }
+
+  // ---- 3. the K-th largest gathered key (C > K), then the output in index order
+  uint32_t prefix = 0, need = 0;
+  int sh2 = 32;  // gathered keys compare by their bits above sh2 (32: every one is selected)
+  if (C > K) {
+    // common high bits of the gathered keys
+    uint32_t gmin = 0xffffffffu, gmax = 0u;
+    for (uint32_t i = threadIdx.x; i < C; i += kSelThreads) {
+      gmin = min(gmin, ck[i]);
+      gmax = max(gmax, ck[i]);
+    }
+    gmin = __reduce_min_sync(0xffffffffu, gmin);
+    gmax = __reduce_max_sync(0xffffffffu, gmax);
+    if (lane == 0) {
+      red_min[warp] = gmin;
+      red_max[warp] = gmax;
+    }
+    __syncthreads();
+    gmin = 0xffffffffu;
+    gmax = 0u;
+#pragma unroll
+    for (int w = 0; w < kSelWarps; ++w) {
+      gmin = min(gmin, red_min[w]);
+      gmax = max(gmax, red_max[w]);
+    }
+    const uint32_t gd = gmin ^ gmax;
+    sh2 = gd == 0u ? 0 : 32 - __clz(gd);
+    prefix = sh2 >= 32 ? 0u : (gmax >> sh2);
+    need = K;
+    __syncthreads();  // red_* are read; hist is free
+#pragma unroll 1
+    while (sh2 > 0) {
+      const int wb = min(8, sh2);
+      const int nbs = 1 << wb;
+      const int nsh = sh2 - wb;
+      for (int i = threadIdx.x; i < nbs; i += kSelThreads) hist[i] = 0;
+      __syncthreads();
+      for (uint32_t i = threadIdx.x; i < C; i += kSelThreads) {
+        const uint32_t u = ck[i];
+        if (sh2 >= 32 || (u >> sh2) == prefix) atomicAdd(&hist[(u >> nsh) & (nbs - 1)], 1u);
+      }
+      __syncthreads();
+      if (warp == 0) {  // lane l owns bins nbs-1-l*bpl .. nbs-(l+1)*bpl
+        const int bpl = nbs >= 32 ? nbs / 32 : 1;
+        const bool own = lane * bpl < nbs;
+        const int lb0 = nbs - (lane + 1) * bpl;
+        uint32_t c = 0;
+        if (own)
+          for (int q = 0; q < bpl; ++q) c += hist[lb0 + q];
+        uint32_t incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        if (own && incl - c < need && need <= incl) {
+          uint32_t above = incl - c;
+          for (int q = bpl - 1; q >= 0; --q) {
+            const uint32_t hc = hist[lb0 + q];
+            if (above + hc >= need) {
+              sh_bin = static_cast<uint32_t>(lb0 + q);
+              sh_above = above;
+              sh_inbin = hc;
+              break;
+            }
+            above += hc;
+          }
+        }
+      }
+      __syncthreads();
+      need -= sh_above;
+      prefix = (sh2 >= 32 ? 0u : (prefix << wb)) | sh_bin;
+      sh2 = nsh;
+      const uint32_t ib = sh_inbin;
+      __syncthreads();
+      if (ib == need) break;
+    }
+  }
+  // thread t writes the gathered elements [t * ipt, (t + 1) * ipt) of its share
+  const uint32_t ipt = (C + kSelThreads - 1) / kSelThreads;
+  const uint32_t e0 = min(C, threadIdx.x * ipt), e1 = min(C, e0 + ipt);
+  uint32_t gt = 0, eq = 0;
+  for (uint32_t i = e0; i < e1; ++i) {
+    const uint32_t t = sh2 >= 32 ? 1u : (ck[i] >> sh2);
+    if (sh2 >= 32 || t > prefix) ++gt;
+    else if (t == prefix) ++eq;
+  }
+  unsigned long long tot64;
+  const unsigned long long ex = block_exclusive_scan64<kSelThreads>(
+      (static_cast<unsigned long long>(gt) << 32) | eq, warp_tot64, tot64);
+  uint32_t gt_b = static_cast<uint32_t>(ex >> 32), eq_b = static_cast<uint32_t>(ex & 0xffffffffull);
+  const uint32_t eq_need = sh2 >= 32 ? 0u : need;
+  for (uint32_t i = e0; i < e1; ++i) {
+    const uint32_t u = ck[i];
+    const uint32_t t = sh2 >= 32 ? 1u : (u >> sh2);
+    const bool g = sh2 >= 32 || t > prefix;
+    const bool e = !g && t == prefix;
+    if (g || (e && eq_b < eq_need)) {
+      const uint32_t slot = gt_b + min(eq_b, eq_need);
+      if (slot < K) {
+        int32_t id = in_idx ? in_idx[cix[i]] : cix[i];
+        id = map_id(map, id, a.map_shift);
+        a.out_idx[out_base + slot] = id;
+        if (a.out_val) a.out_val[out_base + slot] = key_value_long(u);
+      }
+    }
+    gt_b += g;
+    eq_b += e;
+  }
+  const uint32_t n_sel = min(K, static_cast<uint32_t>(tot64 >> 32) +
+                                   min(static_cast<uint32_t>(tot64 & 0xffffffffull), eq_need));
+  for (uint32_t j = n_sel + threadIdx.x; j < K; j += kSelThreads) {
+    a.out_idx[out_base + j] = -1;
+    if (a.out_val) a.out_val[out_base + j] = -INFINITY;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
 // Short rows (up to 32 x ITEMS elements, e.g. the block rows of the hierarchical indexer):
 // one warp per row. Lane l holds elements j*32 + l (coalesced loads). The K-th largest key
 // is found bit by bit below the row's common high bits (a warp-wide count of keys at or
@@ -956,7 +1261,17 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launched) {
     return launch_warp_select<40>(a, s, launched);
   }
   if (seg > c1024) {
-    select_kernel<<<static_cast<unsigned>(grid), kSelThreads, 0, s>>>(a);
+    // whole long rows with K small enough for the gather buffer: the sample-threshold select;
+    // segments of split rows and large K: the multi-pass radix select
+    if (a.n_seg == 1 && a.K <= kLongCap / 2) {
+      constexpr int smem = 2 * kLongCap * 4;
+      const cudaError_t e = cudaFuncSetAttribute(
+          long_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      long_select_kernel<<<static_cast<unsigned>(grid), kSelThreads, smem, s>>>(a);
+    } else {
+      select_kernel<<<static_cast<unsigned>(grid), kSelThreads, 0, s>>>(a);
+    }
     *launched = 1;
     return cudaGetLastError();
   }

@@ -146,32 +146,43 @@ def test_group_mode_on_the_last_chunk_of_262144_tokens(dtype):
                   f"c5 group {dtype}", rows_per_group=2)
 
 
-def test_many_long_rows_with_exact_ties():
+@pytest.mark.parametrize("big,skew", [(0.6, 1.0), (0.03, 1.0), (0.03, 4.0)])
+def test_many_long_rows_with_exact_ties(big, skew):
     """160 rows of 39841 to 40000 keys in one launch (more rows than SMs, every row longer than
     32768): keys are copies of 24 vectors a factor 2 apart, so each row's scores take 24 exact
     values and tens to thousands of keys tie at the K-th. The set must be the oracle's exactly
-    (the lowest positions among the tied keys), in ascending positions."""
-    S, T, K, nd, big = 40000, 160, 2048, 24, 3
+    (the lowest positions among the tied keys), in ascending positions. One copy holds a
+    fraction `big` of the positions: 60 % (more keys at the threshold than the long-row select
+    gathers: its radix passes take over) or 3 % (the gathered keys decide). With skew 4 the
+    keys of every 16th tile of 128 positions (the tiles a long row's threshold is estimated
+    from) are scaled by 4, so the estimate is far too high and the select lowers it."""
+    S, T, K, nd, bigc = 40000, 160, 2048, 24, 3
     p = inputs.anchor_prefill(T, H=64, d=128, K=K, seed=18, device="cuda", S=S)
     rng = np.random.default_rng(9)
-    which = np.where(rng.random(S) < 0.6, big, rng.integers(0, nd, S))
+    which = np.where(rng.random(S) < big, bigc, rng.integers(0, nd, S))
     scales = torch.tensor([2.0 ** (nd - 13 - i) for i in range(nd)])
     v = p["k"][0].float().cpu()
     distinct = (scales[:, None] * v[None, :]).to(torch.bfloat16)
-    k = distinct[torch.as_tensor(which)].contiguous().cuda()
+    k = distinct[torch.as_tensor(which)].contiguous()
+    pos = np.arange(S)
+    boost = ((pos // 128) % 16 == 0) & (skew != 1.0)
+    k[torch.as_tensor(boost)] = (k[torch.as_tensor(boost)].float() * skew).to(torch.bfloat16)
+    k = k.cuda()
     idx, sc, _ = indexer.index_prefill(p["q"], p["w"], k, K, q_pos0=p["q_pos0"],
                                        with_scores=True)
     idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
     q64, w64, d64 = f64(p["q"]), p["w"].double().cpu().numpy(), f64(distinct)
+    mult = np.where(boost, skew, 1.0)
     thresholds = set()
     for t in range(T):
         vals = ox.score_keys(q64[t], w64[t], d64)
         n = p["q_pos0"] + t + 1
-        row = vals[which[:n]]
+        row = vals[which[:n]] * mult[:n]    # ReLU(c x) = c ReLU(x) for c > 0: exact
         order = np.lexsort((np.arange(n), -row))
         assert set(idx[t].tolist()) == set(order[:K].tolist()), f"row {t}"
         assert np.all(np.diff(idx[t]) > 0), f"row {t}: positions not ascending"
-        check_scores(sc[t], row[idx[t]], score_floor(q64[t], w64[t], d64[which[idx[t]]]),
-                     RTOL["bf16"], f"row {t} scores")
+        keys = d64[which[idx[t]]] * mult[idx[t]][:, None]
+        check_scores(sc[t], row[idx[t]], score_floor(q64[t], w64[t], keys), RTOL["bf16"],
+                     f"row {t} scores")
         thresholds.add(int(np.sum(row == row[order[K - 1]])))
     assert max(thresholds) > 100       # rows whose K-th score is shared by many keys
