@@ -39,6 +39,9 @@ sys.path.insert(0, ROOT)
 FLAT = dict(T=16384, H=64, d=128, K=2048, seed=1)
 # smaller flat case for ncu captures: its operands (q 128 MiB, scores 256 MiB) still exceed L2
 FLAT_SMALL = dict(T=8192, H=64, d=128, K=2048, seed=1)
+# long rows for profiler captures of the long-row select: 1024 queries at the end of a
+# 65536-token prefix (scores 256 MiB, still larger than L2)
+LONG_ROWS = dict(T=1024, S=65536, H=64, d=128, K=2048, seed=1)
 GROUP = dict(T=65536, H=64, d=128, K=2048, G=64, B=8192, Hg=16, seed=2)
 DECODE = dict(Bs=32, S=131072, H=64, d=128, K=2048, Hg=16, B=8192, G=16, seed=3)
 CHUNKED = dict(S=262144, chunk=4096, H=64, d=128, K=2048, G=64, B=8192, Hg=16, seed=4)
@@ -269,9 +272,9 @@ def timed_graph(fn, steps, warmup, dist):
 
 def run_flat(args, dist, dtype="bf16", clocks=None):
     from sparse_attention_token_indexer_b200 import _lib, indexer, inputs
-    c = FLAT_SMALL if args.case == "flat_small" else FLAT
+    c = {"flat_small": FLAT_SMALL, "long_rows": LONG_ROWS}.get(args.case, FLAT)
     p = inputs.anchor_prefill(c["T"], c["H"], c["d"], c["K"], seed=c["seed"], device="cuda",
-                              dtype=dtype)
+                              dtype=dtype, S=c.get("S"))
     ws = indexer.Workspace("cuda")
     idx = torch.empty(c["T"], c["K"], dtype=torch.int32, device="cuda")
 
@@ -286,7 +289,7 @@ def run_flat(args, dist, dtype="bf16", clocks=None):
         ms, launches = timed(step, args.steps, args.warmup, dist, timer)
     score_ms = statistics.mean(timer.ms(0, 1))
     select_ms = statistics.mean(timer.ms(2, 3))
-    pairs = flat_pairs(c["T"])
+    pairs = flat_pairs(c["T"], p["q_pos0"])
     return dict(p=p, ms=ms, launches=launches, score_ms=score_ms, select_ms=select_ms,
                 pairs=pairs, flops=pairs * 2 * c["H"] * c["d"], rows=c["T"])
 
@@ -653,7 +656,9 @@ def run_chunked_e2e(args, dist, inp, steps):
 def run_decode_refine(args, dist):
     """Decode with bank reuse (the decode workload's variant): the refine-only steps between
     two refreshes, each over the bank of B = 8192 positions plus the keys appended since the
-    refresh; one step = the refinement of all 32 sequences at one decode position."""
+    refresh; one step = the refinement of all 32 sequences at one decode position. Timed two
+    ways: the candidate keys gathered from the cache every step (tile::gather4), and the bank's
+    keys packed once at the refresh and streamed (adx_pack_bank_keys, timed apart)."""
     from sparse_attention_token_indexer_b200 import indexer, inputs
     c = DECODE
     prob = inputs.decode_problem(c["Bs"], c["S"], c["H"], c["d"], c["K"], c["Hg"],
@@ -665,19 +670,33 @@ def run_decode_refine(args, dist):
     bank = indexer.group_bank(qb, wb, prob["k"], c["G"], c["B"], "paper",
                               k_scale=prob["k_scale"], seq_len=seqs[0], ws=ws)
     r_mid = c["G"] // 2
+    q, w, k, ks = prob["q_steps"][r_mid], prob["w_steps"][r_mid], prob["k"], prob["k_scale"]
 
     def refine():
-        indexer.bank_refine(prob["q_steps"][r_mid], prob["w_steps"][r_mid], prob["k"], bank,
-                            c["G"], c["B"], "paper", c["K"], k_scale=prob["k_scale"],
+        indexer.bank_refine(q, w, k, bank, c["G"], c["B"], "paper", c["K"], k_scale=ks,
                             seq_len=seqs[r_mid], ws=ws)
+
+    packed = indexer.pack_bank_keys(q, w, k, bank, c["G"], c["B"], k_scale=ks, seq_len=seqs[0])
+
+    def pack():
+        indexer.pack_bank_keys(q, w, k, bank, c["G"], c["B"], k_scale=ks, seq_len=seqs[0],
+                               out=packed)
+
+    def refine_packed():
+        indexer.bank_refine_packed(q, w, k, bank, packed[0], packed[1], c["G"], c["B"], c["K"],
+                                   k_scale=ks, seq_len=seqs[r_mid], ws=ws)
 
     ms, launches = timed(refine, args.steps, args.warmup, dist)
     ms_graph, _ = timed_graph(refine, args.steps, args.warmup, dist)
+    ms_p, launches_p = timed(refine_packed, args.steps, args.warmup, dist)
+    ms_p_graph, _ = timed_graph(refine_packed, args.steps, args.warmup, dist)
+    ms_pack, _ = timed(pack, args.steps, args.warmup, dist)
     # keys the step reads: the bank entries at or before the position plus the new keys
     keys = c["Bs"] * (c["B"] + r_mid)
-    del prob, ws
-    return dict(ms=ms, ms_graph=ms_graph, launches=launches, bytes=keys * (c["d"] + 4),
-                rows=c["Bs"])
+    del prob, ws, packed
+    return dict(ms=ms, ms_graph=ms_graph, launches=launches, ms_packed=ms_p,
+                ms_packed_graph=ms_p_graph, launches_packed=launches_p, ms_pack=ms_pack,
+                bytes=keys * (c["d"] + 4), rows=c["Bs"])
 
 
 # ---------------------------------------------------------------------------------------
@@ -848,7 +867,11 @@ def quick_case(args, dist):
     elif args.case == "decode_refine":
         dr = run_decode_refine(args, dist)
         out.update(ms_per_step=dr["ms"], graph_ms_per_step=dr["ms_graph"],
-                   hbm_gbs=dr["bytes"] / (dr["ms"] * 1e-3) / 1e9, gpu_launches=dr["launches"])
+                   packed_ms_per_step=dr["ms_packed"],
+                   packed_graph_ms_per_step=dr["ms_packed_graph"], pack_ms=dr["ms_pack"],
+                   hbm_gbs=dr["bytes"] / (dr["ms"] * 1e-3) / 1e9,
+                   packed_hbm_gbs=dr["bytes"] / (dr["ms_packed"] * 1e-3) / 1e9,
+                   gpu_launches=dr["launches"])
     elif args.case == "chunked":
         inp = chunked_inputs(args.dtype)
         fl = run_chunked_flat(args, dist, inp, args.steps)
@@ -901,7 +924,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--case", default="all",
-                    choices=["all", "flat", "flat_small", "chunked", "group", "decode",
+                    choices=["all", "flat", "flat_small", "long_rows", "chunked", "group", "decode",
                              "decode_refine", "decode_cycle", "mtp", "group_indexer", "hisa",
                              "hisa_small", "hisa_decode"],
                     help="all (default): the headline and every row; the others time one "
@@ -1022,11 +1045,16 @@ def main():
         "gpu_launches": dcd["launches_cycle"]}
     dr = run_decode_refine(args, dist)
     rows["decode_refine_step_Bs32_B8192_e4m3"] = {
-        "ms_per_step": dr["ms"], "graph_ms_per_step": dr["ms_graph"],
-        "bytes_per_step": dr["bytes"], "hbm_gbs": dr["bytes"] / (dr["ms"] * 1e-3) / 1e9,
-        "hbm_frac": dr["bytes"] / (dr["ms"] * 1e-3) / 1e9 / pk["hbm"],
-        "graph_hbm_frac": dr["bytes"] / (dr["ms_graph"] * 1e-3) / 1e9 / pk["hbm"],
-        "topk_queries_per_s": dr["rows"] / (dr["ms"] * 1e-3), "gpu_launches": dr["launches"]}
+        "ms_per_step": dr["ms_packed"], "graph_ms_per_step": dr["ms_packed_graph"],
+        "bytes_per_step": dr["bytes"],
+        "hbm_gbs": dr["bytes"] / (dr["ms_packed"] * 1e-3) / 1e9,
+        "hbm_frac": dr["bytes"] / (dr["ms_packed"] * 1e-3) / 1e9 / pk["hbm"],
+        "graph_hbm_frac": dr["bytes"] / (dr["ms_packed_graph"] * 1e-3) / 1e9 / pk["hbm"],
+        "pack_ms_per_refresh": dr["ms_pack"],
+        "gather_path": {"ms_per_step": dr["ms"], "graph_ms_per_step": dr["ms_graph"],
+                        "hbm_frac": dr["bytes"] / (dr["ms"] * 1e-3) / 1e9 / pk["hbm"]},
+        "topk_queries_per_s": dr["rows"] / (dr["ms_packed"] * 1e-3),
+        "gpu_launches": dr["launches_packed"]}
     mt = run_mtp(args, dist)
     rows[f"mtp_round_Bs32_N131072_m{MTP['m']}_G{MTP['G']}_P{MTP['P']}"] = {
         "ms_per_round": mt["ms"], "scan_pairs": mt["scan"], "refine_pairs": mt["refine"],

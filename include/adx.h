@@ -77,7 +77,8 @@ typedef enum {
   ADX_OP_DECODE = 1,
   ADX_OP_GROUP_BANK = 2,
   ADX_OP_BANK_REFINE = 3,
-  ADX_OP_PREFILL_HOST = 4  /* adx_workspace_size: B = rows_per_chunk */
+  ADX_OP_PREFILL_HOST = 4,  /* adx_workspace_size: B = rows_per_chunk */
+  ADX_OP_BANK_REFINE_PACKED = 5
 } adx_op;
 
 /* One indexer operand set.
@@ -208,6 +209,28 @@ adx_status adx_group_bank(const adx_operands* grp, int32_t G, int32_t B, int32_t
 adx_status adx_bank_refine(const adx_operands* full, int32_t G, int32_t B, int32_t mode,
                            const int32_t* bank_idx, int32_t K, int32_t* topk_idx,
                            float* topk_score, void* ws, size_t ws_bytes, void* stream);
+
+/* Decode bank reuse over a packed bank (ADIndex §4.3, Eqs. (13)-(14), decode layout, PAPER
+ * banks): the key rows a refresh's banks hold, copied once into contiguous rows, so that the
+ * refinement of each following decode step streams them instead of gathering them from the
+ * cache.
+ * adx_pack_bank_keys: bank_idx [T, W] as written by adx_group_bank (W = adx_bank_width(B, G,
+ *   ADX_BANK_PAPER)); writes bank_keys [T, W, d] in the key format and, for e4m3 keys,
+ *   bank_kscale [T, W] (else NULL): slot c of row t holds the key at position bank_idx[t, c]
+ *   of cache t (zeros, scale 0, for -1 entries). Slots of positions not yet in the cache are
+ *   filled by each refinement that sees them.
+ * adx_bank_refine_packed: the result of adx_bank_refine (decode layout, same bank_idx) with
+ *   the candidate keys read from bank_keys / bank_kscale; it first copies, for each row, the
+ *   post-anchor keys at or before its position from the cache into their slots (bank_keys is
+ *   updated in place). ws >= adx_workspace_size(ADX_OP_BANK_REFINE_PACKED, full, K, B, G,
+ *   ADX_BANK_PAPER). bank_keys 16-byte aligned. */
+adx_status adx_pack_bank_keys(const adx_operands* ops, int32_t G, int32_t B,
+                              const int32_t* bank_idx, void* bank_keys, float* bank_kscale,
+                              void* stream);
+adx_status adx_bank_refine_packed(const adx_operands* full, int32_t G, int32_t B,
+                                  const int32_t* bank_idx, void* bank_keys, float* bank_kscale,
+                                  int32_t K, int32_t* topk_idx, float* topk_score, void* ws,
+                                  size_t ws_bytes, void* stream);
 
 /* MTP target verification (ADIndex §4.3, "Application to Prefill and MTP", and Appendix A.2,
  * "Bank Sharing During MTP Target Verification"): each of Bs sequences verifies a window of

@@ -11,7 +11,8 @@ LIB_PATH = os.path.join(HERE, "libadx.so")
 ADX_OK, ADX_EINVAL, ADX_EUNSUPPORTED, ADX_EWORKSPACE, ADX_ECUDA, ADX_EOVERFLOW, ADX_ETIMEOUT = range(7)
 ADX_BF16, ADX_E4M3 = 0, 1
 ADX_BANK_PAPER, ADX_BANK_WINDOW = 0, 1
-ADX_OP_PREFILL, ADX_OP_DECODE, ADX_OP_GROUP_BANK, ADX_OP_BANK_REFINE, ADX_OP_PREFILL_HOST = range(5)
+(ADX_OP_PREFILL, ADX_OP_DECODE, ADX_OP_GROUP_BANK, ADX_OP_BANK_REFINE, ADX_OP_PREFILL_HOST,
+ ADX_OP_BANK_REFINE_PACKED) = range(6)
 ADX_HISA_BLOCK = 128
 ADX_STATUS_BYTES = 256
 
@@ -23,7 +24,8 @@ EXPORTS = ("adx_abi_version", "adx_bank_width", "adx_status_string", "adx_worksp
            "adx_group_union_sizes", "adx_group_query_mean", "adx_index_prefill_host",
            "adx_check_wait_timeout", "adx_group_indexer_workspace_size",
            "adx_group_indexer_queries", "adx_hisa_block_keys", "adx_hisa_workspace_size",
-           "adx_index_hisa", "adx_bank_coverage")
+           "adx_index_hisa", "adx_bank_coverage", "adx_pack_bank_keys",
+           "adx_bank_refine_packed")
 
 
 class Operands(ctypes.Structure):
@@ -91,6 +93,9 @@ def _declare(lib):
         "adx_index_mtp": (ctypes.c_int, [P, P, I32, I32, I32, I32, VP, VP, VP, VP, SZ, VP]),
         "adx_group_union_sizes": (ctypes.c_int, [VP, I32, I32, I32, I32, VP, VP]),
         "adx_bank_coverage": (ctypes.c_int, [VP, I32, I32, VP, I32, I32, I32, VP, VP, VP]),
+        "adx_pack_bank_keys": (ctypes.c_int, [P, I32, I32, VP, VP, VP, VP]),
+        "adx_bank_refine_packed": (ctypes.c_int, [P, I32, I32, VP, VP, VP, I32, VP, VP, VP, SZ,
+                                                  VP]),
         "adx_index_prefill_host": (ctypes.c_int, [P, I32, I32, VP, VP, VP, SZ, VP]),
         "adx_check_wait_timeout": (ctypes.c_int, [VP, ctypes.c_uint64, VP]),
         "adx_hisa_block_keys": (ctypes.c_int, [P, I32, VP, VP, VP]),

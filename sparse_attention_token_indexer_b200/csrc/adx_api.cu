@@ -440,6 +440,23 @@ size_t ws_refine(const adx_operands* o, int G, int B, int mode, int K) {
   return b;
 }
 
+// ---- decode refinement over a packed bank ----------------------------------------------
+size_t ws_refine_packed(const adx_operands* o, int G, int B, int K) {
+  const int64_t W = static_cast<int64_t>(B) + G - 1;
+  return kStatusBytes + ws_prepare(o, o->T) +
+         align_up(static_cast<size_t>(o->T) * ld_for(W) * 4, kAlign) +
+         select_scratch_bytes(o->T, W, K);
+}
+
+adx_status check_packed(const adx_operands* o, int G, int B) {
+  adx_status r = check_operands(o, true);
+  if (r != ADX_OK) return r;
+  if (G <= 0 || B <= 0 || static_cast<int64_t>(B) + G - 1 > INT32_MAX / 2) return ADX_EINVAL;
+  if (static_cast<int64_t>(o->T) * (static_cast<int64_t>(B) + G - 1) > INT32_MAX)
+    return ADX_EINVAL;
+  return ADX_OK;
+}
+
 // ---- flat prefill from host buffers ---------------------------------------------------
 // Copy engines of a device: two non-blocking streams (host to device, device to host) and the
 // events that chain a chunk's copy-in, indexing and copy-out. Created on first use and kept.
@@ -658,6 +675,9 @@ size_t adx_workspace_size(int32_t op, const adx_operands* ops, int32_t K, int32_
           check_bank_args(ops, G, B, mode) != ADX_OK)
         return 0;
       return ws_refine(ops, G, B, mode, K);
+    case ADX_OP_BANK_REFINE_PACKED:
+      if (K <= 0 || mode != ADX_BANK_PAPER || check_packed(ops, G, B) != ADX_OK) return 0;
+      return ws_refine_packed(ops, G, B, K);
     default:
       return 0;
   }
@@ -771,6 +791,69 @@ adx_status adx_group_bank(const adx_operands* o, int32_t G, int32_t B, int32_t m
       cudaSuccess)
     return ADX_ECUDA;
   return ADX_OK;
+}
+
+adx_status adx_pack_bank_keys(const adx_operands* o, int32_t G, int32_t B,
+                              const int32_t* bank_idx, void* bank_keys, float* bank_kscale,
+                              void* stream) {
+  adx_status r = check_packed(o, G, B);
+  if (r != ADX_OK) return r;
+  if (!bank_idx || !bank_keys || fp8_keys(o) != (bank_kscale != nullptr)) return ADX_EINVAL;
+  if (reinterpret_cast<uintptr_t>(bank_keys) % 16 != 0) return ADX_EINVAL;
+  const int32_t W = B + G - 1;
+  return counted(launch_pack_candidates(o->k, o->k_scale, o->S, 1, 1, o->S, bank_idx, o->T, W, W,
+                                        row_bytes(o), bank_keys, bank_kscale, nullptr,
+                                        static_cast<cudaStream_t>(stream))) == cudaSuccess
+             ? ADX_OK
+             : ADX_ECUDA;
+}
+
+adx_status adx_bank_refine_packed(const adx_operands* o, int32_t G, int32_t B,
+                                  const int32_t* bank_idx, void* bank_keys, float* bank_kscale,
+                                  int32_t K, int32_t* topk_idx, float* topk_score, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  adx_status r = check_packed(o, G, B);
+  if (r != ADX_OK) return r;
+  if (K <= 0 || !bank_idx || !bank_keys || !topk_idx || !ws ||
+      fp8_keys(o) != (bank_kscale != nullptr))
+    return ADX_EINVAL;
+  if (reinterpret_cast<uintptr_t>(bank_keys) % 16 != 0) return ADX_EINVAL;
+  if (ws_bytes < ws_refine_packed(o, G, B, K)) return ADX_EWORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int32_t W = B + G - 1;
+  const int64_t ld = ld_for(W);
+  Carve cv(ws);
+  DeviceStatus* st = cv.take<DeviceStatus>(kStatusBytes);
+  Prepared pq;
+  if ((r = prepare(o, o->q, o->q_scale, o->w, o->T, cv, s, pq)) != ADX_OK) return r;
+  // the post-anchor keys this step sees, from the cache into their packed slots
+  if (counted(launch_refresh_post(o->k, o->k_scale, o->S, o->seq_len, bank_idx, o->T, W, B,
+                                  row_bytes(o), bank_keys, bank_kscale, s)) != cudaSuccess)
+    return ADX_ECUDA;
+  float* scores = cv.take<float>(static_cast<size_t>(o->T) * ld * 4);
+  ScorePlan p = rowwise_plan(o, pq, scores, ld);
+  p.a.key_batch_stride = W;  // row t streams slots [t W, t W + W) of the packed bank
+  p.a.keys_per_batch = W;
+  p.a.key_pos = bank_idx;
+  p.a.k_scale = bank_kscale;
+  p.a.status = st;
+  finish_plan(p, ld / kTileM);
+  if ((r = run_score(p, pq.q, bank_keys, static_cast<int64_t>(o->T) * W, s)) != ADX_OK) return r;
+  SelectArgs sa{};
+  sa.vals = scores;
+  sa.ld = ld;
+  sa.idx_map = bank_idx;
+  sa.map_stride = W;
+  sa.rows_per_batch = 1;
+  sa.len_mode = 0;
+  sa.len_fixed = W;
+  sa.len_cap = W;
+  sa.K = K;
+  sa.out_idx = topk_idx;
+  sa.out_val = topk_score;
+  sa.out_ld = K;
+  sa.rows = o->T;
+  return run_select(sa, W, cv, st, s);
 }
 
 adx_status adx_bank_refine(const adx_operands* o, int32_t G, int32_t B, int32_t mode,

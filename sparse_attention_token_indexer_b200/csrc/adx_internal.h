@@ -122,6 +122,9 @@ struct SelectArgs {
 // Longest row the one-warp-per-row select holds (32 lanes x 40 keys); launches whose rows all
 // fit (and are not split into segments) take it.
 constexpr int64_t kWarpSelectMax = 32 * 40;
+// Launches of at most this many rows, each longer than kWarpSelectMax and at most 32768, take
+// the bit-search select (one 1024-thread CTA per row).
+constexpr int kBitsearchMaxRows = 128;
 
 // Launchers (return a cudaError_t from the launch).
 cudaError_t launch_score(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const ScoreArgs& a,
@@ -137,7 +140,7 @@ int select_cluster_ctas(int64_t rows, int64_t n_max, int K, int sms);
 // One launch of the cluster select with `ctas` CTAs per row (a.n_seg must be 1).
 cudaError_t launch_select_cluster(const SelectArgs& a, int ctas, cudaStream_t s, int* launched);
 // Packs candidate key rows: slot c of group g is key cand[g * n_cand + c] of key range
-// g / group_div (per_group_keys; else of the one shared range).
+// g / group_div (per_group_keys; else of the one shared range). packed_pos may be null.
 cudaError_t launch_pack_candidates(const void* k, const float* k_scale, int64_t key_batch_stride,
                                    int32_t per_group_keys, int32_t group_div, int32_t S_valid,
                                    const int32_t* cand,
@@ -171,6 +174,12 @@ cudaError_t launch_union_sizes(const int32_t* topk, int32_t K, int32_t G, int32_
 cudaError_t launch_bank_coverage(const int32_t* topk, int32_t K, const int32_t* bank,
                                  int32_t bank_w, int32_t G, int32_t S, int32_t n_groups,
                                  int32_t* hits, int32_t* count, cudaStream_t s);
+// Packed decode banks [rows, width] of key rows: copies the slots c in [first, width) whose
+// position bank[t, c] is at or before row t's position (seq_len[t] - 1) from cache t.
+cudaError_t launch_refresh_post(const void* k, const float* k_scale, int64_t S,
+                                const int32_t* seq_len, const int32_t* bank, int32_t rows,
+                                int32_t width, int32_t first, int32_t row_bytes, void* packed,
+                                float* packed_scale, cudaStream_t s);
 cudaError_t launch_fill_post_anchor(int32_t* bank, int32_t n_groups, int32_t bank_w,
                                     int32_t first_col, int32_t count, int64_t pos_base,
                                     int32_t pos_step, const int32_t* seq_len, int32_t start_off,

@@ -42,9 +42,33 @@ __global__ void pack_kernel(const uint8_t* __restrict__ k, const float* __restri
   if (valid) v = reinterpret_cast<const uint4*>(k + krow * row_bytes)[piece];
   reinterpret_cast<uint4*>(packed + slot * row_bytes)[piece] = v;
   if (piece == 0) {
-    packed_pos[slot] = valid ? p : INT32_MAX;
+    if (packed_pos) packed_pos[slot] = valid ? p : INT32_MAX;
     if (packed_scale) packed_scale[slot] = (valid && k_scale) ? k_scale[krow] : 0.f;
   }
+}
+
+// Post-anchor slots of packed decode banks: slot c in [first, width) of row t holds the key at
+// position bank[t, c] of cache t; the slots at or before the row's position seq_len[t] - 1 are
+// copied from the cache (one thread per 16 bytes of a slot).
+__global__ void refresh_post_kernel(const uint8_t* __restrict__ k, const float* __restrict__ k_scale,
+                                    int64_t S, const int32_t* __restrict__ seq_len,
+                                    const int32_t* __restrict__ bank, int32_t rows, int32_t width,
+                                    int32_t first, int32_t row_bytes, uint8_t* __restrict__ packed,
+                                    float* __restrict__ packed_scale) {
+  const int pieces = row_bytes / 16;
+  const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t per_row = static_cast<int64_t>(width - first) * pieces;
+  if (gid >= rows * per_row) return;
+  const int t = static_cast<int>(gid / per_row);
+  const int c = first + static_cast<int>((gid % per_row) / pieces);
+  const int piece = static_cast<int>(gid % pieces);
+  const int64_t slot = static_cast<int64_t>(t) * width + c;
+  const int32_t p = bank[slot];
+  if (p < 0 || p >= S || p > seq_len[t] - 1) return;
+  const int64_t krow = static_cast<int64_t>(t) * S + p;
+  reinterpret_cast<uint4*>(packed + slot * row_bytes)[piece] =
+      reinterpret_cast<const uint4*>(k + krow * row_bytes)[piece];
+  if (piece == 0 && packed_scale) packed_scale[slot] = k_scale ? k_scale[krow] : 0.f;
 }
 
 // MTP window positions: query j of sequence b at seq_len[b] - m + j; group g's anchor (its
@@ -446,6 +470,18 @@ cudaError_t launch_bank_coverage(const int32_t* topk, int32_t K, const int32_t* 
   }
   bank_coverage_kernel<<<static_cast<unsigned>(n_groups), 256, smem, s>>>(topk, K, bank, bank_w,
                                                                          G, S, hits, count);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_refresh_post(const void* k, const float* k_scale, int64_t S,
+                                const int32_t* seq_len, const int32_t* bank, int32_t rows,
+                                int32_t width, int32_t first, int32_t row_bytes, void* packed,
+                                float* packed_scale, cudaStream_t s) {
+  const int64_t total = static_cast<int64_t>(rows) * (width - first) * (row_bytes / 16);
+  if (total <= 0) return cudaSuccess;
+  refresh_post_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, s>>>(
+      static_cast<const uint8_t*>(k), k_scale, S, seq_len, bank, rows, width, first, row_bytes,
+      static_cast<uint8_t*>(packed), packed_scale);
   return cudaGetLastError();
 }
 

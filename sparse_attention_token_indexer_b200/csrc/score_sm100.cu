@@ -618,7 +618,10 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           if (a.key_blk_slot != nullptr) slots = static_cast<uint32_t>(a.key_blk_slot[e]);
         } else if (c < x.nkeys) {
           const int64_t kr = x.key_row0 + c;
-          if (a.key_pos != nullptr) kpos = a.key_pos[kr];
+          if (a.key_pos != nullptr) {
+            const int32_t pp = a.key_pos[kr];  // negative: an empty slot, never visible
+            kpos = pp < 0 ? INT64_MAX : pp;
+          }
           if (a.k_scale != nullptr) ks = a.k_scale[kr];
         }
       };

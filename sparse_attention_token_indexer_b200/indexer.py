@@ -238,6 +238,40 @@ def bank_refine(q, w, k, bank, G, B, mode, K, q_scale=None, k_scale=None, q_pos0
     return idx, sc
 
 
+def pack_bank_keys(q, w, k, bank, G, B, k_scale=None, seq_len=None, out=None, stream=None):
+    """Contiguous copy of the decode banks' key rows (decode layout, PAPER banks) ->
+    (bank_keys [T, W, d] in the key format, bank_kscale [T, W] fp32 or None), W = B + G - 1.
+    `out` reuses an existing pair."""
+    ops = make_operands(q, w, k, None, k_scale, 0, seq_len)
+    _dev(bank, "bank", torch.int32)
+    W = B + G - 1
+    if out is None:
+        keys = torch.empty(ops.T, W, ops.d, dtype=k.dtype, device=k.device)
+        ks = torch.empty(ops.T, W, dtype=torch.float32, device=k.device) \
+            if k.dtype == torch.uint8 else None
+    else:
+        keys, ks = out
+    L.check("adx_pack_bank_keys", L.lib().adx_pack_bank_keys(
+        ctypes.byref(ops), G, B, _p(bank), _p(keys), _p(ks), _stream(stream)))
+    return keys, ks
+
+
+def bank_refine_packed(q, w, k, bank, bank_keys, bank_kscale, G, B, K, k_scale=None,
+                       seq_len=None, with_scores=False, ws=None, stream=None):
+    """Decode refinement (Eq. (14)) over a packed bank (pack_bank_keys) -> (topk_idx [T, K],
+    topk_score or None); the post-anchor slots of bank_keys are refreshed in place."""
+    ops = make_operands(q, w, k, None, k_scale, 0, seq_len)
+    _dev(bank, "bank", torch.int32), _dev(bank_keys, "bank_keys")
+    _dev(bank_kscale, "bank_kscale", torch.float32)
+    idx = torch.empty(ops.T, K, dtype=torch.int32, device=q.device)
+    sc = torch.empty(ops.T, K, dtype=torch.float32, device=q.device) if with_scores else None
+    buf = _ws(ws, q.device).get(workspace_size(L.ADX_OP_BANK_REFINE_PACKED, ops, K, B, G, PAPER))
+    L.check("adx_bank_refine_packed", L.lib().adx_bank_refine_packed(
+        ctypes.byref(ops), G, B, _p(bank), _p(bank_keys), _p(bank_kscale), K, _p(idx), _p(sc),
+        _p(buf), buf.numel(), _stream(stream)))
+    return idx, sc
+
+
 def index_mtp(q, w, k, seq_len, qbar, wbar, m, G, P, K, q_scale=None, k_scale=None,
               qbar_scale=None, with_scores=False, with_banks=False, ws=None, stream=None):
     """MTP target verification: Bs = len(seq_len) windows of m queries (q [Bs*m, H, d]) against

@@ -373,6 +373,34 @@ def test_decode_bank_reuse():
                        f"dref step {step} seq {b}")
 
 
+@pytest.mark.parametrize("k_dtype,B", [("e4m3", 1024), ("bf16", 1024), ("e4m3", 8192)])
+def test_decode_refine_over_a_packed_bank_equals_the_gather_path(k_dtype, B):
+    """The bank's key rows packed once at the refresh and streamed by every refinement give the
+    same result as gathering them from the cache each step, bit for bit (same keys, same
+    kernels): both Top-K rows and scores, at the refresh step and at later steps whose
+    post-anchor keys the refinement copies into the packed bank; e4m3 and bf16 caches, and a
+    bank larger than the history (empty slots, -1 in the bank row)."""
+    Bs, S, K, G = 4, 6000, 256, 16
+    prob = inputs.decode_problem(Bs=Bs, S=S, H=64, d=128, K=K, Hg=16, steps=G, seed=35,
+                                 device="cuda", k_dtype=k_dtype)
+    k, ks = prob["k"], prob["k_scale"]
+    seq0 = inputs.decode_seq_len(prob, 0)
+    qbar = prob["q_steps"][0][:, :16].contiguous()
+    wbar = prob["w_steps"][0][:, :16].contiguous()
+    bank = indexer.group_bank(qbar, wbar, k, G, B, "paper", k_scale=ks, seq_len=seq0)
+    keys, kss = indexer.pack_bank_keys(prob["q_steps"][0], prob["w_steps"][0], k, bank, G,
+                                       B, k_scale=ks, seq_len=seq0)
+    for step in (0, 1, 5, G - 1):
+        seq = inputs.decode_seq_len(prob, step)
+        q, w = prob["q_steps"][step], prob["w_steps"][step]
+        ref = indexer.bank_refine(q, w, k, bank, G, B, "paper", K, k_scale=ks, seq_len=seq,
+                                  with_scores=True)
+        got = indexer.bank_refine_packed(q, w, k, bank, keys, kss, G, B, K, k_scale=ks,
+                                         seq_len=seq, with_scores=True)
+        assert torch.equal(got[0], ref[0]), (k_dtype, step)
+        assert torch.equal(got[1], ref[1]), (k_dtype, step)
+
+
 # ---------------------------------------------------------------------------------------
 # MTP target verification
 # ---------------------------------------------------------------------------------------
