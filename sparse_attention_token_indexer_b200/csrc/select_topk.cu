@@ -11,6 +11,7 @@
 #include <cooperative_groups.h>
 
 #include <algorithm>
+#include <cfloat>
 #include <cstdint>
 #include <type_traits>
 
@@ -809,7 +810,7 @@ constexpr int kSampleStride = 16;
 constexpr int kLongCap = 6144;      // gathered elements
 constexpr int kLongPer = 16;        // elements per thread per gather step
 
-__global__ void __launch_bounds__(kSelThreads) long_select_kernel(const SelectArgs a) {
+__global__ void __launch_bounds__(kSelThreads) long_select_kernel(const SelectArgs a, int row0) {
   __shared__ uint32_t hist[kBins];
   __shared__ uint32_t warp_tot[32];
   __shared__ uint32_t sh[2];
@@ -820,7 +821,7 @@ __global__ void __launch_bounds__(kSelThreads) long_select_kernel(const SelectAr
   __shared__ uint32_t sh_bin, sh_above, sh_inbin;
   __shared__ unsigned long long warp_tot64[kSelWarps];
 
-  const int r = blockIdx.x;
+  const int r = row0 + static_cast<int>(blockIdx.x);
   if (r >= a.rows) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t n = row_length(a, r);
@@ -920,28 +921,28 @@ __global__ void __launch_bounds__(kSelThreads) long_select_kernel(const SelectAr
       tau = shift >= 32 ? (sh_bin << ns) : ((top << shift) | (sh_bin << ns));
       if (tau == 0u) tau = 1u;
     }
-    // gather every valid element >= tau, in index order
+    // gather every valid element >= tau, in index order. The test is one float compare
+    // against the value whose key is tau (clamped to the finite range: every valid element
+    // passes tau = 1), a superset of key >= tau that differs only at -0.0; keys are formed
+    // for the gathered elements alone.
+    const float tau_f = tau <= 0x00800000u ? -FLT_MAX : key_value_long(tau);
     C = 0;
     for (int64_t base = 0; base < n; base += static_cast<int64_t>(kSelThreads) * kLongPer) {
       const int64_t i0 = base + static_cast<int64_t>(threadIdx.x) * kLongPer;
-      uint32_t key[kLongPer];
+      float v[kLongPer];
       uint32_t msk = 0;
 #pragma unroll
       for (int j = 0; j < kLongPer; j += 4) {
-        float v[4];
         if (i0 + j + 4 <= n) {
           const float4 f = *reinterpret_cast<const float4*>(vals + i0 + j);
-          v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+          v[j] = f.x; v[j + 1] = f.y; v[j + 2] = f.z; v[j + 3] = f.w;
         } else {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) v[u] = (i0 + j + u < n) ? vals[i0 + j + u] : -INFINITY;
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          key[j + u] = order_key(v[u]);
-          if (is_valid(v[u]) && key[j + u] >= tau) msk |= 1u << (j + u);
+          for (int u = 0; u < 4; ++u) v[j + u] = (i0 + j + u < n) ? vals[i0 + j + u] : -INFINITY;
         }
       }
+#pragma unroll
+      for (int j = 0; j < kLongPer; ++j) msk |= static_cast<uint32_t>(v[j] >= tau_f) << j;
       const uint32_t nm = __popc(msk);
       uint32_t tot;
       uint32_t at = C + block_inclusive_scan(nm, warp_tot, tot) - nm;
@@ -949,7 +950,7 @@ __global__ void __launch_bounds__(kSelThreads) long_select_kernel(const SelectAr
       for (int j = 0; j < kLongPer; ++j) {
         if (msk & (1u << j)) {
           if (at < static_cast<uint32_t>(kLongCap)) {
-            ck[at] = key[j];
+            ck[at] = order_key(v[j]);
             cix[at] = static_cast<int32_t>(i0 + j);
           }
           ++at;
@@ -1373,6 +1374,19 @@ cudaError_t launch_reg(const SelectArgs& a, int row0, int row1, cudaStream_t s, 
   return cudaGetLastError();
 }
 
+// Rows [row0, row1) of a launch through the sample-threshold select (whole rows, K <= 3072).
+cudaError_t launch_long(const SelectArgs& a, int row0, int row1, cudaStream_t s, int* launched) {
+  const int64_t grid = static_cast<int64_t>(row1 - row0);
+  if (grid <= 0) return cudaSuccess;
+  constexpr int smem = 2 * kLongCap * 4;
+  const cudaError_t e =
+      cudaFuncSetAttribute(long_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  long_select_kernel<<<static_cast<unsigned>(grid), kSelThreads, smem, s>>>(a, row0);
+  ++*launched;
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 int select_cluster_ctas(int64_t rows, int64_t n_max, int K, int sms) {
@@ -1447,15 +1461,8 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launched) {
   if (seg > c1024) {
     // whole long rows with K small enough for the gather buffer: the sample-threshold select;
     // segments of split rows and large K: the multi-pass radix select
-    if (a.n_seg == 1 && a.K <= kLongCap / 2) {
-      constexpr int smem = 2 * kLongCap * 4;
-      const cudaError_t e = cudaFuncSetAttribute(
-          long_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e != cudaSuccess) return e;
-      long_select_kernel<<<static_cast<unsigned>(grid), kSelThreads, smem, s>>>(a);
-    } else {
-      select_kernel<<<static_cast<unsigned>(grid), kSelThreads, 0, s>>>(a);
-    }
+    if (a.n_seg == 1 && a.K <= kLongCap / 2) return launch_long(a, 0, a.rows, s, launched);
+    select_kernel<<<static_cast<unsigned>(grid), kSelThreads, 0, s>>>(a);
     *launched = 1;
     return cudaGetLastError();
   }

@@ -186,3 +186,31 @@ def test_many_long_rows_with_exact_ties(big, skew):
                      f"row {t} scores")
         thresholds.add(int(np.sum(row == row[order[K - 1]])))
     assert max(thresholds) > 100       # rows whose K-th score is shared by many keys
+
+
+def test_many_long_rows_with_negative_scores():
+    """Negative gates over positive logits make every score negative: the long-row select's
+    threshold then lies among negative scores (the float compare against a negative threshold
+    value, keys below the sign bit). 160 rows of about 40000 keys, bf16, against the oracle
+    with the parity tolerance."""
+    S, T, K = 40000, 160, 2048
+    p = inputs.anchor_prefill(T, H=64, d=128, K=K, seed=17, device="cuda", S=S)
+    k = p["k"].float()
+    k[:, 0] += 3.0                                        # every key shares a large component
+    q = p["q"].float()
+    q[..., 0] = q[..., 0].abs() + 3.0                     # which every query head reads
+    p["k"], p["q"] = k.to(torch.bfloat16).contiguous(), q.to(torch.bfloat16).contiguous()
+    p["w"] = (-p["w"] - 1e-3).contiguous()                # every gate negative
+    idx, sc, _ = indexer.index_prefill(p["q"], p["w"], p["k"], K, q_pos0=p["q_pos0"],
+                                       with_scores=True)
+    idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+    k64 = f64(p["k"])
+    rows = [0, 1, 57, 100, 158, 159]
+    q64 = _rows_f64(p["q"], None, rows)
+    w64 = p["w"][torch.as_tensor(rows, device="cuda")].double().cpu().numpy()
+    for j, t in enumerate(rows):
+        n = p["q_pos0"] + t + 1
+        cs = ox.score_keys(q64[j], w64[j], k64[:n])
+        assert np.sort(cs)[-K] < 0, f"row {t}: the K-th score should be negative"
+        check_topk(idx[t], np.arange(n), cs, score_floor(q64[j], w64[j], k64[:n]), K,
+                   RTOL["bf16"], sc[t], f"negative row {t}")
