@@ -122,7 +122,8 @@ int32_t adx_bank_width(int32_t B, int32_t G, int32_t mode);
  * topk_idx    [T, K] int32 out
  * topk_score  [T, K] fp32 out, or NULL
  * scores_out  [T, scores_ld] fp32 out, or NULL: every score I[t, s] (s <= pos(t); -inf for
- *             invisible keys up to the tile end). scores_ld >= S rounded up to 128.
+ *             invisible keys up to the tile end). scores_ld >= S rounded up to 128 and a
+ *             multiple of 4; scores_out 16-byte aligned (ADX_EINVAL otherwise).
  * ws          workspace of ws_bytes >= adx_workspace_size(ADX_OP_PREFILL, ...) */
 adx_status adx_index_prefill(const adx_operands* ops, int32_t K, int32_t* topk_idx,
                              float* topk_score, float* scores_out, int64_t scores_ld, void* ws,

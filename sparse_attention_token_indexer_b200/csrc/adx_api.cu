@@ -689,7 +689,10 @@ adx_status adx_index_prefill(const adx_operands* o, int32_t K, int32_t* topk_idx
   adx_status r = check_operands(o, false);
   if (r != ADX_OK) return r;
   if (K <= 0 || !topk_idx || !ws) return ADX_EINVAL;
-  if (scores_out && scores_ld < ld_for(o->S)) return ADX_EINVAL;
+  // score rows are read with 16-byte vector loads
+  if (scores_out && (scores_ld < ld_for(o->S) || scores_ld % 4 != 0 ||
+                     (reinterpret_cast<uintptr_t>(scores_out) & 15) != 0))
+    return ADX_EINVAL;
   if (ws_bytes < ws_flat(o, K, scores_out != nullptr)) return ADX_EWORKSPACE;
   Carve cv(ws);
   DeviceStatus* st = cv.take<DeviceStatus>(kStatusBytes);

@@ -68,6 +68,12 @@ def test_host_validation(lib):
                               k_scale=64)) == L.ADX_EUNSUPPORTED    # e4m3 needs d = 128
     assert lib.adx_index_prefill(ctypes.byref(_ops()), 4, ctypes.c_void_p(4096), None, None,
                                  0, ctypes.c_void_p(8192), 16, None) == L.ADX_EWORKSPACE
+    # an external score matrix needs 16-byte rows: stride >= S rounded up to 128, a multiple
+    # of 4, and an aligned base
+    for ptr, ld in ((1 << 16, 64), (1 << 16, 129), (1 << 16 | 8, 128)):
+        assert lib.adx_index_prefill(ctypes.byref(_ops()), 4, ctypes.c_void_p(4096), None,
+                                     ctypes.c_void_p(ptr), ld, ctypes.c_void_p(8192), 1 << 20,
+                                     None) == L.ADX_EINVAL
     # decode layout needs seq_len; bank modes are checked
     assert lib.adx_index_decode(ctypes.byref(_ops()), 4, ctypes.c_void_p(4096), None,
                                 ctypes.c_void_p(8192), 1 << 20, None) == L.ADX_EINVAL
