@@ -16,6 +16,7 @@
 #include <type_traits>
 
 #include "adx_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace adx {
 
@@ -794,32 +795,83 @@ select_reg_kernel(const SelectArgs a, int row0) {
 // ---------------------------------------------------------------------------------------
 // Many rows longer than a register-resident select holds (chunked prefill past 32K keys):
 // a threshold from a sample, then one streaming pass.
-//   1. Sample: every kSampleStride-th tile of 128 elements (m of the row's n). Its key range
-//      and a 12-bit histogram below the range's common high bits give the bin of the sample's
-//      r-th largest key, r = 5/4 * K * m / n + 8, whose lower edge is the threshold tau: about
-//      5/4 of K elements of the row are expected at or above it.
-//   2. One pass gathers every valid element >= tau into shared memory in index order (a block
-//      scan of per-thread masks per 8192 elements). Fewer than K gathered (the estimate was
-//      too high): tau is lowered (rank 4r, then every element) and the pass repeated; more
-//      than the buffer holds (many equal keys): the row takes the multi-pass radix select.
+//   1. Sample: every kSampleStride-th tile of 128 elements (m of the row's n), kept in shared
+//      memory after its first read. Its key range and a 12-bit histogram below the range's
+//      common high bits give the bins of the sample's r-th and 4r-th largest keys,
+//      r = 5/4 * K * m / n + 8, whose lower edges are the thresholds tau: about 5/4 of K
+//      elements of the row are expected at or above the first.
+//   2. One pass gathers every valid element >= tau into shared memory in index order: each
+//      thread tests 16 consecutive elements of a step of 8192 (the next step's loads already in
+//      flight) and a block scan of the per-thread counts gives their slots. Fewer than K
+//      gathered (the estimate was too high): the pass is repeated at the lower tau, then at
+//      every element; more than the buffer holds (many equal keys): the row takes the
+//      multi-pass radix select.
 //   3. The exact K-th largest among the gathered keys (8-bit digit histograms), and the
 //      selected elements written in index order: every key above it and the lowest-indexed
 //      keys equal to it.
 // ---------------------------------------------------------------------------------------
 constexpr int kSampleStride = 16;
-constexpr int kLongCap = 6144;      // gathered elements
-constexpr int kLongPer = 16;        // elements per thread per gather step
+constexpr int kLongCap = 4096;                    // gathered elements
+constexpr int kRingStep = 4096;                   // elements per gather step (8 per thread)
+constexpr int kRingSlots = 5;                     // steps in the copy ring (up to four in flight)
+constexpr int kRingFloats = kRingSlots * kRingStep;
+constexpr int kLongSmem = (kRingFloats + 2 * kLongCap) * 4;
+constexpr uint64_t kLongTimeoutNs = 2000000000ull;  // bound on one copy's wait
+static_assert(kRingStep == 8 * kSelThreads, "eight elements per thread per step");
+static_assert(kRingFloats >= kBins && 2 * kLongCap >= kBins, "histograms fit either region");
 
-__global__ void __launch_bounds__(kSelThreads) long_select_kernel(const SelectArgs a, int row0) {
-  __shared__ uint32_t hist[kBins];
+// Bit j set when element j of (d0, d1) is >= t (a NaN compares false).
+__device__ __forceinline__ uint32_t ge_bits8(const float4& d0, const float4& d1, float t) {
+  const float v[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+  uint32_t m = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    uint32_t r;
+    asm("set.ge.u32.f32 %0, %1, %2;" : "=r"(r) : "f"(v[j]), "f"(t));
+    m |= r & (1u << j);
+  }
+  return m;
+}
+
+// Inclusive prefix sum over the warp (all lanes take part).
+__device__ __forceinline__ uint32_t warp_inclusive_sum(uint32_t x) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .u32 y;\n\t"
+        "shfl.sync.up.b32 y|p, %0, %1, 0, -1;\n\t"
+        "@p add.u32 %0, %0, y;\n\t}"
+        : "+r"(x)
+        : "r"(o));
+  return x;
+}
+
+// One bulk copy (no multicast) of `bytes` from global memory into this CTA's shared memory,
+// completing on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kSelThreads, 2) long_select_kernel(const SelectArgs a, int row0) {
   __shared__ uint32_t warp_tot[32];
+  __shared__ uint32_t step_tot[2][kSelWarps];
   __shared__ uint32_t sh[2];
   extern __shared__ __align__(16) uint32_t long_smem[];
-  uint32_t* ck = long_smem;                                   // gathered keys, index order
-  int32_t* cix = reinterpret_cast<int32_t*>(long_smem + kLongCap);  // their element indices
+  float* ring = reinterpret_cast<float*>(long_smem);    // the sample, then the gather's copies
+  float* samp = ring;
+  uint32_t* hist = long_smem;                            // radix histograms once the ring is idle
+  uint32_t* ck = long_smem + kRingFloats;                // gathered keys, index order
+  int32_t* cix = reinterpret_cast<int32_t*>(ck + kLongCap);  // their element indices
+  uint32_t* hist_s = ck;                                 // the sample's histogram (before gathering)
   __shared__ uint32_t red_min[kSelWarps], red_max[kSelWarps], red_cnt[kSelWarps];
-  __shared__ uint32_t sh_bin, sh_above, sh_inbin;
+  __shared__ uint32_t sh_bin, sh_above, sh_inbin, sh_tau_bin[2];
   __shared__ unsigned long long warp_tot64[kSelWarps];
+  __shared__ __align__(8) uint64_t full[kRingSlots];  // one per ring slot: its copy landed
+  __shared__ int abort_s;
 
   const int r = row0 + static_cast<int>(blockIdx.x);
   if (r >= a.rows) return;
@@ -831,22 +883,54 @@ __global__ void __launch_bounds__(kSelThreads) long_select_kernel(const SelectAr
       a.idx_map ? a.idx_map + static_cast<int64_t>(r / a.rows_per_batch) * a.map_stride : nullptr;
   const int64_t out_base = static_cast<int64_t>(r) * a.out_ld;
   const uint32_t K = static_cast<uint32_t>(a.K);
+  // the copies move whole 16-byte chunks: rows must start aligned and end inside their stride
+  if ((reinterpret_cast<uintptr_t>(vals) & 15) != 0 || (a.ld & 3) != 0 || n > a.ld) {
+    radix_row(a, r, 0, hist, warp_tot, sh);
+    return;
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kRingSlots; ++i) mbar_init(&full[i], 1);
+    abort_s = 0;
+    fence_mbarrier_init();
+  }
 
   // ---- 1. the sample's key range, then its histogram below the common high bits
   const int64_t n_tiles = (n + 127) / 128;
   const int64_t n_samp = (n_tiles + kSampleStride - 1) / kSampleStride;
+  const bool cached = n_samp * 128 <= kRingFloats;  // the sample is kept for the second read
+  // lane l of a warp reads elements 4l .. 4l + 3 of a sampled tile; a warp has four tiles'
+  // loads in flight at once
   uint32_t kmin = 0xffffffffu, kmax = 0u, cnt = 0u;
-  for (int64_t t = warp; t < n_samp; t += kSelWarps) {
-    const int64_t base = t * kSampleStride * 128;
+  for (int64_t t0 = warp; t0 < n_samp; t0 += 4 * kSelWarps) {
+    float4 q[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int64_t i = base + u * 32 + lane;
-      const float v = i < n ? vals[i] : -INFINITY;
-      if (is_valid(v)) {
-        const uint32_t k = order_key(v);
-        kmin = min(kmin, k);
-        kmax = max(kmax, k);
-        ++cnt;
+      const int64_t t = t0 + u * kSelWarps;
+      const int64_t i = t * kSampleStride * 128 + 4 * lane;
+      if (t < n_samp && i + 4 <= n) {
+        q[u] = *reinterpret_cast<const float4*>(vals + i);
+      } else {
+        const bool in = t < n_samp;
+        q[u] = make_float4(in && i < n ? vals[i] : -INFINITY, in && i + 1 < n ? vals[i + 1] : -INFINITY,
+                           in && i + 2 < n ? vals[i + 2] : -INFINITY,
+                           in && i + 3 < n ? vals[i + 3] : -INFINITY);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t t = t0 + u * kSelWarps;
+      if (t < n_samp) {
+        if (cached) reinterpret_cast<float4*>(samp + t * 128)[lane] = q[u];
+        const float v4[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (is_valid(v4[c])) {
+            const uint32_t k = order_key(v4[c]);
+            kmin = min(kmin, k);
+            kmax = max(kmax, k);
+            ++cnt;
+          }
+        }
       }
     }
   }
@@ -858,6 +942,7 @@ __global__ void __launch_bounds__(kSelThreads) long_select_kernel(const SelectAr
     red_max[warp] = kmax;
     red_cnt[warp] = cnt;
   }
+  for (int i = threadIdx.x; i < kBins; i += kSelThreads) hist_s[i] = 0;
   __syncthreads();
   kmin = 0xffffffffu;
   kmax = 0u;
@@ -873,91 +958,162 @@ __global__ void __launch_bounds__(kSelThreads) long_select_kernel(const SelectAr
   const int wbits = min(12, shift);
   const int ns = shift - wbits;
   const uint32_t top = shift >= 32 ? 0u : (kmax >> shift);
-  for (int i = threadIdx.x; i < kBins; i += kSelThreads) hist[i] = 0;
-  __syncthreads();
-  for (int64_t t = warp; t < n_samp; t += kSelWarps) {
-    const int64_t base = t * kSampleStride * 128;
+  const uint32_t bmask = (1u << wbits) - 1u;
+  if (cached) {  // the sample as kept (elements past the row's end are -inf)
+    for (int64_t i = threadIdx.x; i < n_samp * 128; i += kSelThreads) {
+      const float v = samp[i];
+      if (is_valid(v)) atomicAdd(&hist_s[(order_key(v) >> ns) & bmask], 1u);
+    }
+  } else {
+    for (int64_t t = warp; t < n_samp; t += kSelWarps) {
+      const int64_t base = t * kSampleStride * 128;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int64_t i = base + u * 32 + lane;
-      const float v = i < n ? vals[i] : -INFINITY;
-      if (is_valid(v)) atomicAdd(&hist[(order_key(v) >> ns) & ((1u << wbits) - 1u)], 1u);
+      for (int u = 0; u < 4; ++u) {
+        const int64_t i = base + u * 32 + lane;
+        const float v = i < n ? vals[i] : -INFINITY;
+        if (is_valid(v)) atomicAdd(&hist_s[(order_key(v) >> ns) & bmask], 1u);
+      }
     }
   }
   __syncthreads();
 
-  // ---- 2. threshold from the sample, one gathering pass (repeated with a lower threshold if
-  //         it gathered fewer than K elements)
-  uint32_t C = 0;        // valid elements >= tau in the row
-  uint32_t tau = 0u;     // 0: every valid element (valid keys are > 0)
+  // the bins holding the sample's want-th largest key for want = r0 and 4 r0, by one block
+  // scan from the top; a want beyond the sample takes every element (tau = 0: valid keys > 0)
   const uint64_t r0 = static_cast<uint64_t>(1.25 * K * (static_cast<double>(m) / (n > 0 ? n : 1))) + 8;
-#pragma unroll 1
-  for (int attempt = 0; attempt < 3; ++attempt) {
-    const uint64_t want = attempt == 0 ? r0 : r0 * 4;
-    tau = 0u;
-    if (attempt < 2 && want < m) {
-      // the bin holding the sample's want-th largest key, by a block scan from the top
-      const int nb = 1 << wbits;
-      const int bpt = nb >= kSelThreads ? nb / kSelThreads : 1;
-      const bool owner = static_cast<int>(threadIdx.x) * bpt < nb;
-      const int b0 = nb - (static_cast<int>(threadIdx.x) + 1) * bpt;
-      uint32_t mine = 0;
-      if (owner)
-        for (int q = 0; q < bpt; ++q) mine += hist[b0 + q];
-      uint32_t tot;
-      const uint32_t incl = block_inclusive_scan(mine, warp_tot, tot);
-      const uint32_t excl = incl - mine;
-      if (owner && excl < want && want <= incl) {
+  uint32_t tau0 = 0u, tau1 = 0u;
+  {
+    const int nb = 1 << wbits;
+    const int bpt = nb >= kSelThreads ? nb / kSelThreads : 1;
+    const bool owner = static_cast<int>(threadIdx.x) * bpt < nb;
+    const int b0 = nb - (static_cast<int>(threadIdx.x) + 1) * bpt;
+    uint32_t mine = 0;
+    if (owner)
+      for (int q = 0; q < bpt; ++q) mine += hist_s[b0 + q];
+    uint32_t tot;
+    const uint32_t incl = block_inclusive_scan(mine, warp_tot, tot);
+    const uint32_t excl = incl - mine;
+#pragma unroll
+    for (int wi = 0; wi < 2; ++wi) {
+      const uint64_t want = wi == 0 ? r0 : r0 * 4;
+      if (owner && want < m && excl < want && want <= incl) {
         uint32_t above = excl;
         for (int q = bpt - 1; q >= 0; --q) {
-          above += hist[b0 + q];
+          above += hist_s[b0 + q];
           if (above >= want) {
-            sh_bin = static_cast<uint32_t>(b0 + q);
+            sh_tau_bin[wi] = static_cast<uint32_t>(b0 + q);
             break;
           }
         }
       }
-      __syncthreads();
-      tau = shift >= 32 ? (sh_bin << ns) : ((top << shift) | (sh_bin << ns));
-      if (tau == 0u) tau = 1u;
     }
-    // gather every valid element >= tau, in index order. The test is one float compare
-    // against the value whose key is tau (clamped to the finite range: every valid element
-    // passes tau = 1), a superset of key >= tau that differs only at -0.0; keys are formed
-    // for the gathered elements alone.
+    __syncthreads();
+#pragma unroll
+    for (int wi = 0; wi < 2; ++wi) {
+      const uint64_t want = wi == 0 ? r0 : r0 * 4;
+      if (want < m) {
+        const uint32_t b = sh_tau_bin[wi];
+        const uint32_t t = shift >= 32 ? (b << ns) : ((top << shift) | (b << ns));
+        (wi == 0 ? tau0 : tau1) = t == 0u ? 1u : t;
+      }
+    }
+  }
+
+  // ---- 2. one gathering pass (repeated at a lower threshold if it found fewer than K)
+  uint32_t C = 0;        // valid elements >= tau in the row
+  uint32_t tau = 0u;
+  const int64_t n_steps = (n + kRingStep - 1) / kRingStep;
+  // Fill f of the ring (counted over every pass) goes to slot f % kRingSlots and completes
+  // phase (f / kRingSlots) & 1 of that slot's barrier; thread 0 issues the copies and waits.
+  uint32_t fbase = 0;
+  auto fill = [&](int64_t st) {  // thread 0: copy step st of this pass
+    const uint32_t f = fbase + static_cast<uint32_t>(st);
+    const int slot = static_cast<int>(f % kRingSlots);
+    const int64_t e0 = st * kRingStep;
+    const int64_t cnt = min(static_cast<int64_t>(kRingStep), n - e0);
+    const uint32_t bytes = static_cast<uint32_t>((cnt * 4 + 15) & ~static_cast<int64_t>(15));
+    mbar_arrive_expect_tx(&full[slot], bytes);
+    bulk_load(ring + slot * kRingStep, vals + e0, bytes, &full[slot]);
+  };
+  auto landed = [&](int64_t st) {  // thread 0: bounded wait for step st's copy
+    const uint32_t f = fbase + static_cast<uint32_t>(st);
+    return mbar_wait(&full[f % kRingSlots], (f / kRingSlots) & 1u, &abort_s, kLongTimeoutNs);
+  };
+#pragma unroll 1
+  for (int attempt = 0; attempt < 3; ++attempt) {
+    tau = attempt == 0 ? tau0 : (attempt == 1 ? tau1 : 0u);
+    if (attempt == 1 && tau == tau0) continue;  // the same threshold again: take every element
+    // The test is one float compare against the value whose key is tau (clamped to the finite
+    // range: every valid element passes tau = 1), a superset of key >= tau that differs only
+    // at -0.0; keys are formed for the gathered elements alone.
     const float tau_f = tau <= 0x00800000u ? -FLT_MAX : key_value_long(tau);
     C = 0;
-    for (int64_t base = 0; base < n; base += static_cast<int64_t>(kSelThreads) * kLongPer) {
-      const int64_t i0 = base + static_cast<int64_t>(threadIdx.x) * kLongPer;
-      float v[kLongPer];
-      uint32_t msk = 0;
-#pragma unroll
-      for (int j = 0; j < kLongPer; j += 4) {
-        if (i0 + j + 4 <= n) {
-          const float4 f = *reinterpret_cast<const float4*>(vals + i0 + j);
-          v[j] = f.x; v[j + 1] = f.y; v[j + 2] = f.z; v[j + 3] = f.w;
-        } else {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) v[j + u] = (i0 + j + u < n) ? vals[i0 + j + u] : -INFINITY;
+    int ok = 1;
+    if (threadIdx.x == 0) {
+      fence_proxy_async_smem();  // the ring's earlier contents were written by the threads
+      for (int64_t j = 0; j < kRingSlots - 1 && j < n_steps; ++j) fill(j);
+      ok = landed(0);
+    }
+    int64_t s = 0;
+    if (__syncthreads_and(ok)) {
+#pragma unroll 1
+      for (; s < n_steps; ++s) {
+        const uint32_t f = fbase + static_cast<uint32_t>(s);
+        const int slot = static_cast<int>(f % kRingSlots);
+        (void)mbar_try_wait(&full[slot], (f / kRingSlots) & 1u);  // complete: orders the reads
+        const float* mine = ring + slot * kRingStep + 8 * threadIdx.x;
+        const float4 d0 = reinterpret_cast<const float4*>(mine)[0];
+        const float4 d1 = reinterpret_cast<const float4*>(mine)[1];
+        const int64_t i0 = s * kRingStep + 8 * static_cast<int64_t>(threadIdx.x);
+        // bit j: element j of this thread is >= tau (past the row's end on the last step: no)
+        uint32_t msk = ge_bits8(d0, d1, tau_f);
+        if (s + 1 == n_steps) {
+          const int64_t left = n - i0;
+          msk &= left >= 8 ? 0xffu : (left <= 0 ? 0u : ((1u << left) - 1u));
         }
-      }
-#pragma unroll
-      for (int j = 0; j < kLongPer; ++j) msk |= static_cast<uint32_t>(v[j] >= tau_f) << j;
-      const uint32_t nm = __popc(msk);
-      uint32_t tot;
-      uint32_t at = C + block_inclusive_scan(nm, warp_tot, tot) - nm;
-#pragma unroll
-      for (int j = 0; j < kLongPer; ++j) {
-        if (msk & (1u << j)) {
+        const uint32_t nm = __popc(msk);
+        const uint32_t incl = warp_inclusive_sum(nm);
+        uint32_t* st = step_tot[s & 1];
+        if (lane == 31) st[warp] = incl;
+        ok = 1;
+        if (threadIdx.x == 0 && s + 1 < n_steps) ok = landed(s + 1);
+        // every thread is done with the previous step's slot, which takes step s + R - 1
+        if (!__syncthreads_and(ok)) break;
+        if (threadIdx.x == 0 && s + kRingSlots - 1 < n_steps) fill(s + kRingSlots - 1);
+        const uint32_t x = lane < kSelWarps ? st[lane] : 0u;
+        const uint32_t tot = __reduce_add_sync(0xffffffffu, x);
+        const uint32_t before = __reduce_add_sync(0xffffffffu, lane < warp ? x : 0u);
+        // this thread's elements >= tau, in index order; their values are read again from the
+        // slot, which is not refilled before the next step's barrier
+        uint32_t at = C + before + incl - nm;
+        for (uint32_t mm = msk; mm != 0u; mm &= mm - 1u, ++at) {
+          const int j = __ffs(mm) - 1;
           if (at < static_cast<uint32_t>(kLongCap)) {
-            ck[at] = order_key(v[j]);
+            ck[at] = order_key(mine[j]);
             cix[at] = static_cast<int32_t>(i0 + j);
           }
-          ++at;
+        }
+        C += tot;
+      }
+    }
+    if (s < n_steps) {
+      // a copy did not land in time: report it, let every copy of this pass that was issued
+      // land (bounded) before the CTA's shared memory is released, and leave the row
+      if (threadIdx.x == 0) {
+        if (a.status != nullptr && atomicCAS(&a.status->code, 0, static_cast<int>(ADX_ETIMEOUT)) == 0) {
+          a.status->where = kWhereSelect;
+          a.status->info0 = 3;
+          a.status->info1 = r;
+        }
+        volatile int never = 0;
+        const int64_t issued = min(n_steps, s + kRingSlots - 1);  // fills s .. issued-1 may be pending
+        for (int64_t j = s; j < issued; ++j) {
+          const uint32_t f = fbase + static_cast<uint32_t>(j);
+          (void)mbar_wait(&full[f % kRingSlots], (f / kRingSlots) & 1u, &never, kLongTimeoutNs);
         }
       }
-      C += tot;
+      return;
     }
+    fbase += static_cast<uint32_t>(n_steps);
     __syncthreads();
     if (C >= K || tau == 0u) break;
   }
@@ -1378,11 +1534,14 @@ cudaError_t launch_reg(const SelectArgs& a, int row0, int row1, cudaStream_t s, 
 cudaError_t launch_long(const SelectArgs& a, int row0, int row1, cudaStream_t s, int* launched) {
   const int64_t grid = static_cast<int64_t>(row1 - row0);
   if (grid <= 0) return cudaSuccess;
-  constexpr int smem = 2 * kLongCap * 4;
-  const cudaError_t e =
-      cudaFuncSetAttribute(long_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(long_select_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kLongSmem);
   if (e != cudaSuccess) return e;
-  long_select_kernel<<<static_cast<unsigned>(grid), kSelThreads, smem, s>>>(a, row0);
+  // two CTAs per SM need the largest shared-memory carveout
+  e = cudaFuncSetAttribute(long_select_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
+  long_select_kernel<<<static_cast<unsigned>(grid), kSelThreads, kLongSmem, s>>>(a, row0);
   ++*launched;
   return cudaGetLastError();
 }
