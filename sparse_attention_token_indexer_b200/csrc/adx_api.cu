@@ -34,6 +34,8 @@ cudaError_t counted(cudaError_t e, int n = 1) {
   return e;
 }
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per device-side wait
+// Score matrices above this size are stored evict-first (twice the L2 of a B200)
+constexpr double kStreamScoreBytes = 256.0 * (1 << 20);
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int64_t ld_for(int64_t n) { return (n + kTileM - 1) / kTileM * kTileM; }
@@ -238,8 +240,10 @@ adx_status run_score(const ScorePlan& p, const void* q_codes, const void* keys, 
   const int bps = score_blocks_per_sm(p.fp8, p.H, p.d, p.tok);
   const int grid = std::min<int64_t>(p.a.n_items, static_cast<int64_t>(sm_count()) * bps);
   if (grid <= 0) return ADX_EUNSUPPORTED;
+  ScoreArgs a = p.a;
+  a.stream_scores = static_cast<double>(a.R) * static_cast<double>(a.score_ld) * 4.0 > kStreamScoreBytes;
   mark(0, s);
-  const cudaError_t e = counted(launch_score(tq, tk, p.a, p.fp8, p.H, p.d, p.tok, grid, s));
+  const cudaError_t e = counted(launch_score(tq, tk, a, p.fp8, p.H, p.d, p.tok, grid, s));
   mark(1, s);
   if (e == cudaErrorNotSupported) return ADX_EUNSUPPORTED;
   return e == cudaSuccess ? ADX_OK : ADX_ECUDA;
@@ -304,7 +308,12 @@ adx_status run_select(SelectArgs a, int64_t n_max, Carve& cv, DeviceStatus* st, 
   s2.len_cap = s2.len_fixed;
   s2.n_seg = 1;
   s2.seg_len = s2.len_fixed;
-  const cudaError_t e2 = launch_select(s2, s, &nl);
+  // candidates beyond what one CTA holds in registers: one cluster per row, when one holds them
+  const int ctas2 = s2.len_fixed > kSelectRegCapacity
+                        ? select_cluster_ctas(s2.rows, s2.len_fixed, s2.K, sm_count(), true)
+                        : 0;
+  const cudaError_t e2 =
+      ctas2 > 0 ? launch_select_cluster(s2, ctas2, s, &nl) : launch_select(s2, s, &nl);
   const cudaError_t e = counted(e2, nl);
   mark(3, s);
   return e == cudaSuccess ? ADX_OK : ADX_ECUDA;

@@ -61,6 +61,9 @@ struct ScoreArgs {
   const int8_t* fold_flag; // [R]: 1 = the row's queries carry its gates already; null = none do
   float* scores;           // [R, score_ld]
   int64_t score_ld;
+  // 1: score stores bypass the L2's normal retention (evict-first), for score matrices far
+  // larger than the L2 that would otherwise push the key tiles out of it
+  int32_t stream_scores;
   int64_t pos_base;
   int32_t pos_step;
   int32_t R;
@@ -135,8 +138,10 @@ bool score_config_supported(bool fp8, int H, int d);
 // Launches one to three kernels (row-length classes); *launched receives how many.
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launched);
 // Few long rows: CTAs per row of the cluster select (one thread-block cluster per row, the
-// row held in registers across the cluster), or 0 when it does not apply.
-int select_cluster_ctas(int64_t rows, int64_t n_max, int K, int sms);
+// row held in registers across the cluster), or 0 when it does not apply. By default rows of
+// at most 8 K keys are left to the one-CTA selects; any_k drops that rule (the second stage of
+// a split select, whose rows are n_seg * K candidates).
+int select_cluster_ctas(int64_t rows, int64_t n_max, int K, int sms, bool any_k = false);
 // One launch of the cluster select with `ctas` CTAs per row (a.n_seg must be 1).
 cudaError_t launch_select_cluster(const SelectArgs& a, int ctas, cudaStream_t s, int* launched);
 // Packs candidate key rows: slot c of group g is key cand[g * n_cand + c] of key range

@@ -299,6 +299,13 @@ __device__ __forceinline__ void reduce_chunk_folded(const float (&v)[C::CW], int
   }
 }
 
+// One score of the output matrix; streaming (evict-first) stores for matrices far larger
+// than the L2, so that they do not displace the key tiles every row block re-reads.
+__device__ __forceinline__ void store_score(const ScoreArgs& a, int64_t at, float v) {
+  if (a.stream_scores) __stcs(a.scores + at, v);
+  else a.scores[at] = v;
+}
+
 // True when the queries of every row of the block carry their gates already.
 __device__ __forceinline__ bool block_folded(const ScoreArgs& a, const Block& x) {
   if (a.fold_flag == nullptr) return false;
@@ -711,9 +718,9 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 const uint32_t sl = (slots >> (8 * (tok0 + tt))) & 0xFFu;
                 col = sl == 0xFFu ? -1 : static_cast<int>(sl) * kTileM + m;
               }
-              if (col >= 0) a.scores[static_cast<int64_t>(r) * a.score_ld + col] = out;
+              if (col >= 0) store_score(a, static_cast<int64_t>(r) * a.score_ld + col, out);
             } else {
-              a.scores[static_cast<int64_t>(r) * a.score_ld + c] = out;
+              store_score(a, static_cast<int64_t>(r) * a.score_ld + c, out);
             }
           }
         }

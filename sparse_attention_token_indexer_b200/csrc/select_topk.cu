@@ -1548,9 +1548,9 @@ cudaError_t launch_long(const SelectArgs& a, int row0, int row1, cudaStream_t s,
 
 }  // namespace
 
-int select_cluster_ctas(int64_t rows, int64_t n_max, int K, int sms) {
+int select_cluster_ctas(int64_t rows, int64_t n_max, int K, int sms, bool any_k) {
   constexpr int64_t cap = static_cast<int64_t>(kClusterThreads) * kClusterItems;
-  if (rows <= 0 || rows >= sms || n_max <= 8ll * K) return 0;
+  if (rows <= 0 || rows >= sms || (!any_k && n_max <= 8ll * K)) return 0;
   const int64_t need = (n_max + cap - 1) / cap;
   if (need > kClusterMaxCtas) return 0;
   const int64_t fill = (2ll * sms) / rows;       // two CTAs of this class fit on an SM
