@@ -43,6 +43,8 @@ FLAT_SMALL = dict(T=8192, H=64, d=128, K=2048, seed=1)
 # 65536-token prefix (scores 256 MiB, still larger than L2)
 LONG_ROWS = dict(T=1024, S=65536, H=64, d=128, K=2048, seed=1)
 GROUP = dict(T=65536, H=64, d=128, K=2048, G=64, B=8192, Hg=16, seed=2)
+# the same group mode at a quarter of the length (a profiling case)
+GROUP_SMALL = dict(T=16384, H=64, d=128, K=2048, G=64, B=8192, Hg=16, seed=2)
 DECODE = dict(Bs=32, S=131072, H=64, d=128, K=2048, Hg=16, B=8192, G=16, seed=3)
 CHUNKED = dict(S=262144, chunk=4096, H=64, d=128, K=2048, G=64, B=8192, Hg=16, seed=4)
 # rows per chunk of the host-buffer path (copies of one chunk overlap the work on another)
@@ -307,7 +309,7 @@ def _call_prefill(p, K, idx, ws):
 
 def run_group(args, dist):
     from sparse_attention_token_indexer_b200 import indexer, inputs
-    c = GROUP
+    c = GROUP_SMALL if getattr(args, "case", "") == "group_small" else GROUP
     p = inputs.group_prefill(c["T"], c["H"], c["d"], c["K"], c["G"], c["B"], c["Hg"],
                              seed=c["seed"], device="cuda")
     ws = indexer.Workspace("cuda")
@@ -901,7 +903,7 @@ def quick_case(args, dist):
         gi = run_group_indexer(args, dist)
         out.update(ms_per_step=gi["ms"], activation_gbs=gi["act_bytes"] / (gi["ms"] * 1e-3) / 1e9,
                    gpu_launches=gi["launches"])
-    elif args.case == "group":
+    elif args.case in ("group", "group_small"):
         g = run_group(args, dist)
         out.update(ms_per_step=g["ms"], stage_ms=g["stages"],
                    refine_score_tflops=g["refine_tflops"], gpu_launches=g["launches"])
@@ -924,7 +926,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--case", default="all",
-                    choices=["all", "flat", "flat_small", "long_rows", "chunked", "group", "decode",
+                    choices=["all", "flat", "flat_small", "long_rows", "chunked", "group",
+                             "group_small", "decode",
                              "decode_refine", "decode_cycle", "mtp", "group_indexer", "hisa",
                              "hisa_small", "hisa_decode"],
                     help="all (default): the headline and every row; the others time one "

@@ -125,9 +125,6 @@ struct SelectArgs {
 // Longest row the one-warp-per-row select holds (32 lanes x 40 keys); launches whose rows all
 // fit (and are not split into segments) take it.
 constexpr int64_t kWarpSelectMax = 32 * 40;
-// Launches of at most this many rows, each longer than kWarpSelectMax and at most 32768, take
-// the bit-search select (one 1024-thread CTA per row).
-constexpr int kBitsearchMaxRows = 128;
 
 // Launchers (return a cudaError_t from the launch).
 cudaError_t launch_score(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const ScoreArgs& a,

@@ -1328,182 +1328,6 @@ __global__ void __launch_bounds__(32 * kWarpSelRows) select_warp_kernel(const Se
   }
 }
 
-// ---------------------------------------------------------------------------------------
-// Few rows of up to 32768 elements (a decode step's refinement, HISA decode, the second stage
-// of a split select: one row per sequence): one 1024-thread CTA per row holds the row in
-// registers and finds the K-th largest key two bits at a time below the row's common high
-// bits. Each step counts the keys at or above three candidates (warp reductions, one barrier
-// to combine the warps, one to broadcast the choice), so a row takes at most 16 steps and no
-// shared-memory histogram (whose atomics serialise on the few bins a row's top scores share).
-// One block scan of (above, equal) counts then places the selected elements in index order:
-// every key above the K-th and the lowest-indexed keys equal to it.
-// ---------------------------------------------------------------------------------------
-constexpr int kBsThreads = 1024;
-constexpr int kBsWarps = kBsThreads / 32;
-
-template <int ITEMS>
-__global__ void __launch_bounds__(kBsThreads, 1) bitsearch_select_kernel(const SelectArgs a) {
-  __shared__ uint32_t part[kBsWarps][4];
-  __shared__ uint32_t sh_val[4];
-  __shared__ unsigned long long warp_tot64[kBsWarps];
-  const int r = blockIdx.x;
-  if (r >= a.rows) return;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t n = row_length(a, r);
-  const float* vals = a.vals + static_cast<int64_t>(r) * a.ld;
-  const int32_t* in_idx = a.in_idx ? a.in_idx + static_cast<int64_t>(r) * a.ld : nullptr;
-  const int32_t* map =
-      a.idx_map ? a.idx_map + static_cast<int64_t>(r / a.rows_per_batch) * a.map_stride : nullptr;
-  const int64_t out_base = static_cast<int64_t>(r) * a.out_ld;
-  const uint32_t K = static_cast<uint32_t>(a.K);
-
-  // ---- load: thread t owns elements [t*ITEMS, (t+1)*ITEMS); 0 marks an invalid element
-  uint32_t key[ITEMS];
-  const int64_t my0 = static_cast<int64_t>(threadIdx.x) * ITEMS;
-  const bool vec = (reinterpret_cast<uintptr_t>(vals) & 15) == 0;
-  uint32_t kmin = 0xffffffffu, kmax = 0u, nval = 0u;
-#pragma unroll
-  for (int j = 0; j < ITEMS; j += 4) {
-    float v[4];
-    const int64_t i0 = my0 + j;
-    if (vec && i0 + 4 <= n) {
-      const float4 f = *reinterpret_cast<const float4*>(vals + i0);
-      v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
-    } else {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = (i0 + u < n) ? vals[i0 + u] : -INFINITY;
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const bool ok = is_valid(v[u]);
-      const uint32_t k = ok ? order_key(v[u]) : 0u;
-      key[j + u] = k;
-      kmin = ok ? min(kmin, k) : kmin;
-      kmax = max(kmax, k);
-      nval += ok;
-    }
-  }
-  kmin = __reduce_min_sync(0xffffffffu, kmin);
-  kmax = __reduce_max_sync(0xffffffffu, kmax);
-  nval = __reduce_add_sync(0xffffffffu, nval);
-  if (lane == 0) {
-    part[warp][0] = kmin;
-    part[warp][1] = kmax;
-    part[warp][2] = nval;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    const uint32_t mn = __reduce_min_sync(0xffffffffu, part[lane][0]);
-    const uint32_t mx = __reduce_max_sync(0xffffffffu, part[lane][1]);
-    const uint32_t nv = __reduce_add_sync(0xffffffffu, part[lane][2]);
-    if (lane == 0) {
-      sh_val[0] = mn;
-      sh_val[1] = mx;
-      sh_val[2] = nv;
-    }
-  }
-  __syncthreads();
-  kmin = sh_val[0];
-  kmax = sh_val[1];
-  nval = sh_val[2];
-  const bool take_all = nval <= K;
-
-  // ---- the K-th largest key, two bits per step; invariant: K keys are >= theta
-  uint32_t theta = 1u;  // take_all: every valid key (valid keys are > 0)
-  uint32_t need = 0u;
-  if (!take_all) {
-    const uint32_t diff = kmin ^ kmax;
-    int b = diff == 0u ? 0 : 32 - __clz(diff);  // bits b.. are common to every valid key
-    theta = b >= 32 ? 0u : ((kmax >> b) << b);
-#pragma unroll 1
-    while (b > 0) {
-      const int w = b >= 2 ? 2 : 1;
-      b -= w;
-      const uint32_t c1 = theta | (1u << b), c2 = theta | (2u << b), c3 = theta | (3u << b);
-      uint32_t n1 = 0, n2 = 0, n3 = 0;
-#pragma unroll
-      for (int j = 0; j < ITEMS; ++j) {
-        n1 += key[j] >= c1;
-        n2 += key[j] >= c2;
-        n3 += key[j] >= c3;
-      }
-      n1 = __reduce_add_sync(0xffffffffu, n1);
-      n2 = __reduce_add_sync(0xffffffffu, n2);
-      n3 = __reduce_add_sync(0xffffffffu, n3);
-      if (lane == 0) {
-        part[warp][0] = n1;
-        part[warp][1] = n2;
-        part[warp][2] = n3;
-      }
-      __syncthreads();
-      if (warp == 0) {
-        const uint32_t t1 = __reduce_add_sync(0xffffffffu, part[lane][0]);
-        const uint32_t t2 = __reduce_add_sync(0xffffffffu, part[lane][1]);
-        const uint32_t t3 = __reduce_add_sync(0xffffffffu, part[lane][2]);
-        if (lane == 0)
-          sh_val[3] = (w == 2 && t3 >= K) ? c3 : (w == 2 && t2 >= K) ? c2 : (t1 >= K) ? c1 : theta;
-      }
-      __syncthreads();
-      theta = sh_val[3];
-    }
-    uint32_t gt = 0;
-#pragma unroll
-    for (int j = 0; j < ITEMS; ++j) gt += key[j] > theta;
-    gt = __reduce_add_sync(0xffffffffu, gt);
-    if (lane == 0) part[warp][0] = gt;
-    __syncthreads();
-    if (warp == 0) {
-      const uint32_t t = __reduce_add_sync(0xffffffffu, part[lane][0]);
-      if (lane == 0) sh_val[3] = K - t;  // equal keys to take, lowest index first
-    }
-    __syncthreads();
-    need = sh_val[3];
-  }
-
-  // ---- output in index order
-  uint32_t gt_mask = 0, eq_mask = 0;
-#pragma unroll
-  for (int j = 0; j < ITEMS; ++j) {
-    if (key[j] == 0u) continue;
-    if (key[j] > theta || (take_all && key[j] >= theta)) gt_mask |= 1u << j;
-    else if (key[j] == theta) eq_mask |= 1u << j;
-  }
-  unsigned long long tot;
-  const unsigned long long ex = block_exclusive_scan64<kBsThreads>(
-      (static_cast<unsigned long long>(__popc(gt_mask)) << 32) | __popc(eq_mask), warp_tot64, tot);
-  uint32_t gt_b = static_cast<uint32_t>(ex >> 32);
-  uint32_t eq_b = static_cast<uint32_t>(ex & 0xffffffffull);
-#pragma unroll
-  for (int j = 0; j < ITEMS; ++j) {
-    const bool g = (gt_mask >> j) & 1u, e = (eq_mask >> j) & 1u;
-    if (g || (e && eq_b < need)) {
-      const uint32_t slot = gt_b + min(eq_b, need);
-      if (slot < K) {
-        const int64_t i = my0 + j;
-        int32_t id = in_idx ? in_idx[i] : static_cast<int32_t>(i);
-        id = map_id(map, id, a.map_shift);
-        a.out_idx[out_base + slot] = id;
-        if (a.out_val) a.out_val[out_base + slot] = key_value(key[j]);
-      }
-    }
-    gt_b += g;
-    eq_b += e;
-  }
-  const uint32_t n_sel = min(K, static_cast<uint32_t>(tot >> 32) +
-                                   min(static_cast<uint32_t>(tot & 0xffffffffull), need));
-  for (uint32_t j = n_sel + threadIdx.x; j < K; j += kBsThreads) {
-    a.out_idx[out_base + j] = -1;
-    if (a.out_val) a.out_val[out_base + j] = -INFINITY;
-  }
-}
-
-template <int ITEMS>
-cudaError_t launch_bitsearch(const SelectArgs& a, cudaStream_t s, int* launched) {
-  bitsearch_select_kernel<ITEMS><<<static_cast<unsigned>(a.rows), kBsThreads, 0, s>>>(a);
-  *launched = 1;
-  return cudaGetLastError();
-}
-
 static_assert(kWarpSelectMax == 32 * 40, "the widest warp select instance");
 
 template <int ITEMS>
@@ -1603,14 +1427,6 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s, int* launched) {
   constexpr int64_t cap[NC] = {128 * kRegItems, 256 * kRegItems, 256 * kWideItems,
                                512 * kRegItems};
   constexpr int64_t c1024 = 1024 * kRegItems;
-  if (a.n_seg == 1 && a.rows <= kBitsearchMaxRows && seg > kWarpSelectMax && seg <= c1024) {
-    // few rows: one 1024-thread CTA per row, the K-th found two bits per step
-    if (seg <= 1024 * 8) return launch_bitsearch<8>(a, s, launched);
-    if (seg <= 1024 * 12) return launch_bitsearch<12>(a, s, launched);
-    if (seg <= 1024 * 16) return launch_bitsearch<16>(a, s, launched);
-    if (seg <= 1024 * 24) return launch_bitsearch<24>(a, s, launched);
-    return launch_bitsearch<32>(a, s, launched);
-  }
   if (a.n_seg == 1 && seg <= kWarpSelectMax) {  // short rows: one warp per row
     if (seg <= 32 * 8) return launch_warp_select<8>(a, s, launched);
     if (seg <= 32 * 16) return launch_warp_select<16>(a, s, launched);
