@@ -310,7 +310,7 @@ select_reg_kernel(const SelectArgs a, int row0) {
   __shared__ uint32_t red_min[NW], red_max[NW], red_cnt[NW];
   __shared__ uint32_t sh_bin, sh_above, sh_inbin;
   __shared__ uint32_t cl_red[3];         // this CTA's (min, max, count) of valid keys
-  __shared__ unsigned long long cl_tot;  // this CTA's packed (above, equal) counts
+  __shared__ unsigned long long cl_tots[kClusterMaxCtas];  // CTA c's packed (above, equal) counts
   __shared__ uint32_t cl_part[NH][CLUSTER ? THREADS : 1];  // per-thread bin-range counts
   __shared__ uint32_t sh_ccount, sh_theta, sh_needt;
   __shared__ uint32_t c_key[kGatherMax];               // this CTA's keys of the threshold bin
@@ -714,26 +714,21 @@ select_reg_kernel(const SelectArgs a, int row0) {
   // packed counts of the CTAs before this one (cluster) and of the whole row
   unsigned long long off = 0, all = tot;
   if constexpr (CLUSTER) {
-    if (threadIdx.x == 0) cl_tot = tot;
-    cg::this_cluster().sync();  // also a CTA barrier: warp_tot64 is free again
-    if (warp == 0) {  // lane c reads CTA c's counts
-      const unsigned long long v =
-          lane < nparts ? *cg::this_cluster().map_shared_rank(&cl_tot, lane) : 0ull;
-      unsigned long long lower = lane < part ? v : 0ull, sum = v;
+    // every CTA's counts are pushed into every CTA of the cluster; after the barrier each
+    // thread adds them up from its own shared memory. No CTA touches another's shared memory
+    // after this barrier, so a CTA may leave as soon as its own writes are done.
+    if (static_cast<int>(threadIdx.x) < nparts)
+      *cg::this_cluster().map_shared_rank(&cl_tots[part], static_cast<int>(threadIdx.x)) = tot;
+    cg::this_cluster().sync();
+    all = 0ull;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        lower += __shfl_xor_sync(0xffffffffu, lower, o);
-        sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      }
-      if (lane == 0) {
-        warp_tot64[0] = lower;
-        warp_tot64[1] = sum;
+    for (int c = 0; c < kClusterMaxCtas; ++c) {
+      if (c < nparts) {
+        const unsigned long long v = cl_tots[c];
+        off += c < part ? v : 0ull;
+        all += v;
       }
     }
-    // no CTA leaves while another may still read its shared memory; also a CTA barrier
-    cg::this_cluster().sync();
-    off = warp_tot64[0];
-    all = warp_tot64[1];
   }
   const uint32_t gt_before = static_cast<uint32_t>((off + ex) >> 32);
   const uint32_t eq_before = static_cast<uint32_t>((off + ex) & kLow);
@@ -1354,7 +1349,7 @@ cudaError_t launch_reg(const SelectArgs& a, int row0, int row1, cudaStream_t s, 
   return cudaGetLastError();
 }
 
-// Rows [row0, row1) of a launch through the sample-threshold select (whole rows, K <= 3072).
+// Rows [row0, row1) of a launch through the sample-threshold select (whole rows, K <= 2048).
 cudaError_t launch_long(const SelectArgs& a, int row0, int row1, cudaStream_t s, int* launched) {
   const int64_t grid = static_cast<int64_t>(row1 - row0);
   if (grid <= 0) return cudaSuccess;
