@@ -365,10 +365,14 @@ select_reg_kernel(const SelectArgs a, int row0) {
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const bool ok = is_valid(v[u]);
-      const uint32_t k = ok ? order_key(v[u]) : 0u;  // 0 = invalid (valid keys are > 0)
+      // order key; the valid ones (-FLT_MAX .. +inf) are 0x00800000 .. 0xff800000, NaN and
+      // -inf fall outside and become 0
+      const uint32_t b = __float_as_uint(v[u]);
+      const uint32_t kk = b ^ (static_cast<uint32_t>(static_cast<int32_t>(b) >> 31) | 0x80000000u);
+      const bool ok = kk - 0x00800000u <= 0xff000000u;
+      const uint32_t k = ok ? kk : 0u;
       key[j + u] = k;
-      kmin = ok ? min(kmin, k) : kmin;
+      kmin = min(kmin, k - 1u);  // invalid (0) wraps to the largest value: no effect
       kmax = max(kmax, k);
       nval += ok;
     }
@@ -422,6 +426,7 @@ select_reg_kernel(const SelectArgs a, int row0) {
     nval = red_cnt[0];
   }
 
+  kmin += 1u;  // the minimum was taken over key - 1
   uint32_t prefix = 0;
   int shift = 32;            // number of low key bits not yet resolved
   uint32_t need = K;
@@ -693,18 +698,21 @@ select_reg_kernel(const SelectArgs a, int row0) {
   }
 
   // ---- output: one scan of (above, equal) counts, then each thread writes its run ------
+  // the threshold bin as a key range [lo, hi]: above it selected, inside it the lowest-indexed
+  // keys up to need; every valid key is above an empty bin (hi = 0) when all are taken
+  uint32_t bin_lo = 1u, bin_hi = 0u;
+  if (!take_all) {
+    const uint32_t base = shift >= 32 ? 0u : (prefix << shift);
+    bin_hi = shift >= 32 ? 0xffffffffu : (base | ((1u << shift) - 1u));
+    bin_lo = max(base, 1u);
+  }
   Mask gt_mask = 0, eq_mask = 0;
 #pragma unroll
   for (int j = 0; j < ITEMS; ++j) {
     const uint32_t u = key[j];
-    if (u == 0u) continue;
-    if (take_all) {
-      gt_mask |= Mask(1) << j;
-      continue;
-    }
-    const uint32_t top = shift >= 32 ? 0u : (u >> shift);
-    if (top > prefix) gt_mask |= Mask(1) << j;
-    else if (top == prefix) eq_mask |= Mask(1) << j;
+    const bool g = u > bin_hi;
+    gt_mask |= Mask(g) << j;
+    eq_mask |= Mask(!g && u >= bin_lo) << j;
   }
   constexpr unsigned long long kLow = 0xffffffffull;
   unsigned long long tot;
