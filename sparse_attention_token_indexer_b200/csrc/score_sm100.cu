@@ -597,39 +597,54 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         tokf[tt] = (folded && in && a.q_scale != nullptr) ? a.q_scale[rowg + tt] : 1.f;
       }
 
-      // per-key scale and position of the next tile, loaded one tile ahead so their
-      // latency hides behind the current tile's wait and reduction
-      auto key_meta = [&](int t, float& ks, int64_t& kpos, uint32_t& slots) {
+      // Per-key metadata of a tile (position for the causal test, key scale, block slots) in
+      // two steps: the loads are issued a tile ahead into raw registers, and nothing depends
+      // on them until the tile is reduced, when they are turned into (ks, kpos, slots). A test
+      // or conversion right after the load would make the warp wait for it there.
+      struct MetaRaw {
+        int32_t i;       // key position, gathered key row or block (-1: none)
+        float ks;        // key scale (plain layout)
+        uint32_t slots;  // block slots of the tile's tokens
+      };
+      auto meta_load = [&](int t, MetaRaw& r) {
         const int c = t * kTileM + m;
-        kpos = c;
+        r.i = -1;
+        r.ks = 1.f;
+        r.slots = 0u;
+        if constexpr (C::GATHER) {
+          if (c < x.nkeys && c < a.n_idx)
+            r.i = a.key_idx[static_cast<int64_t>(x.b) * a.key_idx_stride + c];
+        } else if constexpr (C::BLOCKS) {
+          const int64_t e = static_cast<int64_t>(x.b) * a.key_blk_stride + t;
+          if (c < x.nkeys) r.i = a.key_blk[e];
+          if (a.key_blk_slot != nullptr) r.slots = static_cast<uint32_t>(a.key_blk_slot[e]);
+        } else if (c < x.nkeys) {
+          const int64_t kr = x.key_row0 + c;
+          if (a.key_pos != nullptr) r.i = a.key_pos[kr];  // negative: an empty slot
+          if (a.k_scale != nullptr) r.ks = a.k_scale[kr];
+        }
+      };
+      auto meta_finish = [&](int t, const MetaRaw& r, float& ks, int64_t& kpos, uint32_t& slots) {
+        const int c = t * kTileM + m;
         ks = 1.f;
-        slots = 0u;
+        slots = r.slots;
         if constexpr (C::GATHER) {
           kpos = INT64_MAX;  // no key: never visible
-          if (c < x.nkeys && c < a.n_idx) {
-            const int32_t p = a.key_idx[static_cast<int64_t>(x.b) * a.key_idx_stride + c];
-            if (p >= 0 && p < a.S_valid) {
-              kpos = p;
-              if (a.k_scale != nullptr) ks = a.k_scale[x.key_row0 + p];
-            }
+          if (r.i >= 0 && r.i < a.S_valid) {
+            kpos = r.i;
+            if (a.k_scale != nullptr) ks = a.k_scale[x.key_row0 + r.i];
           }
         } else if constexpr (C::BLOCKS) {
           kpos = INT64_MAX;
-          const int64_t e = static_cast<int64_t>(x.b) * a.key_blk_stride + t;
-          const int32_t bk = c < x.nkeys ? a.key_blk[e] : -1;
-          const int64_t p = static_cast<int64_t>(bk) * kTileM + m;
-          if (bk >= 0 && p < a.S_valid) {
+          const int64_t p = static_cast<int64_t>(r.i) * kTileM + m;
+          if (r.i >= 0 && p < a.S_valid) {
             kpos = p;
             if (a.k_scale != nullptr) ks = a.k_scale[x.key_row0 + p];
           }
-          if (a.key_blk_slot != nullptr) slots = static_cast<uint32_t>(a.key_blk_slot[e]);
-        } else if (c < x.nkeys) {
-          const int64_t kr = x.key_row0 + c;
-          if (a.key_pos != nullptr) {
-            const int32_t pp = a.key_pos[kr];  // negative: an empty slot, never visible
-            kpos = pp < 0 ? INT64_MAX : pp;
-          }
-          if (a.k_scale != nullptr) ks = a.k_scale[kr];
+        } else {
+          kpos = c;
+          ks = r.ks;
+          if (c < x.nkeys && a.key_pos != nullptr) kpos = r.i < 0 ? INT64_MAX : r.i;
         }
       };
       // tile t of this range is the CTA's tile number g = gi_lo + (t - t_lo); it lands in
@@ -639,16 +654,16 @@ score_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       constexpr int TSTEP = C::BUF_SPLIT ? C::EG : 1;
       int t0 = t_lo;
       if (C::BUF_SPLIT) t0 += static_cast<int>(((grp - gi_lo) % C::EG + C::EG) % C::EG);
-      float ks_next = 1.f;
-      int64_t kpos_next = 0;
-      uint32_t slots_next = 0u;
-      if (t0 < t_hi) key_meta(t0, ks_next, kpos_next, slots_next);
+      MetaRaw raw_next;
+      if (t0 < t_hi) meta_load(t0, raw_next);
       bool ok = true;
       for (int t = t0; t < t_hi; t += TSTEP) {
-        const float ks = ks_next;
-        const int64_t kpos = kpos_next;
-        const uint32_t slots = slots_next;
-        if (t + TSTEP < t_hi) key_meta(t + TSTEP, ks_next, kpos_next, slots_next);
+        const MetaRaw raw = raw_next;
+        if (t + TSTEP < t_hi) meta_load(t + TSTEP, raw_next);
+        float ks;
+        int64_t kpos;
+        uint32_t slots;
+        meta_finish(t, raw, ks, kpos, slots);
         const int64_t g = gi_lo + (t - t_lo);
         const int acc = static_cast<int>(g % C::ACC);
         const uint32_t acc_phase = static_cast<uint32_t>((g / C::ACC) & 1);
