@@ -362,10 +362,12 @@ def run_decode(args, dist, cycle=True):
     td = StageTimer(_lib.lib(), args.steps)
     ms_flat, l_flat = timed(flat_step, args.steps, args.warmup, dist, td)
     dstages = {"score_ms": statistics.mean(td.ms(0, 1)), "select_ms": statistics.mean(td.ms(2, 3))}
+    # the same step replayed from a CUDA graph (how a serving loop issues it)
+    ms_flat_graph, _ = timed_graph(flat_step, args.steps, args.warmup, dist)
     key_bytes = c["d"] + 4
     if not cycle:
         return dict(ms_flat=ms_flat, launches_flat=l_flat, bytes_flat=c["Bs"] * c["S"] * key_bytes,
-                    stages=dstages)
+                    stages=dstages, ms_flat_graph=ms_flat_graph)
     seqs = [inputs.decode_seq_len(prob, r) for r in range(c["G"])]
 
     def cycle():
@@ -383,7 +385,7 @@ def run_decode(args, dist, cycle=True):
     key_bytes = c["d"] + 4
     return dict(ms_flat=ms_flat, launches_flat=l_flat, ms_cycle=ms_cycle, launches_cycle=l_cycle,
                 ms_cycle_graph=ms_cycle_graph, bytes_flat=c["Bs"] * c["S"] * key_bytes,
-                steps_per_cycle=c["G"], stages=dstages)
+                steps_per_cycle=c["G"], stages=dstages, ms_flat_graph=ms_flat_graph)
 
 
 def run_mtp(args, dist):
@@ -865,7 +867,7 @@ def quick_case(args, dist):
         dcd = run_decode(args, dist, cycle=False)
         out.update(ms_per_step=dcd["ms_flat"], stage_ms=dcd["stages"],
                    hbm_gbs=dcd["bytes_flat"] / (dcd["ms_flat"] * 1e-3) / 1e9,
-                   gpu_launches=dcd["launches_flat"])
+                   graph_ms_per_step=dcd["ms_flat_graph"], gpu_launches=dcd["launches_flat"])
     elif args.case == "decode_refine":
         dr = run_decode_refine(args, dist)
         out.update(ms_per_step=dr["ms"], graph_ms_per_step=dr["ms_graph"],
@@ -1039,7 +1041,10 @@ def main():
         "hbm_gbs": dcd["bytes_flat"] / (dcd["ms_flat"] * 1e-3) / 1e9,
         "hbm_frac": dcd["bytes_flat"] / (dcd["ms_flat"] * 1e-3) / 1e9 / pk["hbm"],
         "score_kernel_hbm_frac": dcd["bytes_flat"] / (dcd["stages"]["score_ms"] * 1e-3) / 1e9
-        / pk["hbm"], "stage_ms": dcd["stages"], "gpu_launches": dcd["launches_flat"]}
+        / pk["hbm"], "stage_ms": dcd["stages"],
+        "graph_ms_per_step": dcd["ms_flat_graph"],
+        "graph_hbm_frac": dcd["bytes_flat"] / (dcd["ms_flat_graph"] * 1e-3) / 1e9 / pk["hbm"],
+        "gpu_launches": dcd["launches_flat"]}
     rows["decode_bank_reuse_cycle16"] = {
         "ms_per_cycle": dcd["ms_cycle"],
         "ms_per_step": dcd["ms_cycle"] / dcd["steps_per_cycle"],
