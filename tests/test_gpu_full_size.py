@@ -214,3 +214,19 @@ def test_many_long_rows_with_negative_scores():
         assert np.sort(cs)[-K] < 0, f"row {t}: the K-th score should be negative"
         check_topk(idx[t], np.arange(n), cs, score_floor(q64[j], w64[j], k64[:n]), K,
                    RTOL["bf16"], sc[t], f"negative row {t}")
+
+
+def test_prefill_from_position_0_past_32768_rows():
+    """One call of 36864 queries from position 0: the longest rows exceed what the register
+    selects hold, so every row of the launch, from 1 key up, takes the sample-threshold select
+    (rows shorter than K return all their keys, rows just past K, rows whose sample holds a
+    handful of keys, rows ending a partial step of its copy ring)."""
+    T, K = 36864, 256
+    p = inputs.anchor_prefill(T, H=64, d=128, K=K, seed=61, device="cuda")
+    assert p["q_pos0"] == 0
+    idx, sc, _ = indexer.index_prefill(p["q"], p["w"], p["k"], K, with_scores=True)
+    idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+    k64 = f64(p["k"], p["k_scale"])
+    rows = [0, 1, 2, K - 2, K - 1, K, K + 1, 2047, 2048, 4095, 4096, 4097, 8191, 8193, 20000,
+            32767, 32768, T - 1]
+    _check_flat_rows(p, idx, sc, rows, k64, "from 0")
