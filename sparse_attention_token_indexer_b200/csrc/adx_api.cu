@@ -241,7 +241,10 @@ adx_status run_score(const ScorePlan& p, const void* q_codes, const void* keys, 
   const int grid = std::min<int64_t>(p.a.n_items, static_cast<int64_t>(sm_count()) * bps);
   if (grid <= 0) return ADX_EUNSUPPORTED;
   ScoreArgs a = p.a;
-  a.stream_scores = static_cast<double>(a.R) * static_cast<double>(a.score_ld) * 4.0 > kStreamScoreBytes;
+  // not in the block-list mode, whose rows are written block by block in slot order (plain
+  // stores measured faster there)
+  a.stream_scores = a.key_blk == nullptr &&
+                    static_cast<double>(a.R) * static_cast<double>(a.score_ld) * 4.0 > kStreamScoreBytes;
   mark(0, s);
   const cudaError_t e = counted(launch_score(tq, tk, a, p.fp8, p.H, p.d, p.tok, grid, s));
   mark(1, s);
