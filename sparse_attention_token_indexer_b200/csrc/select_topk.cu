@@ -882,12 +882,15 @@ __global__ void __launch_bounds__(kSelThreads, 2) long_select_kernel(const Selec
   const int64_t n = row_length(a, r);
   const float* vals = a.vals + static_cast<int64_t>(r) * a.ld;
   const int32_t* in_idx = a.in_idx ? a.in_idx + static_cast<int64_t>(r) * a.ld : nullptr;
+  const uint32_t lanes_below = (1u << lane) - 1u;
   const int32_t* map =
       a.idx_map ? a.idx_map + static_cast<int64_t>(r / a.rows_per_batch) * a.map_stride : nullptr;
   const int64_t out_base = static_cast<int64_t>(r) * a.out_ld;
   const uint32_t K = static_cast<uint32_t>(a.K);
   // the copies move whole 16-byte chunks: rows must start aligned and end inside their stride
-  if ((reinterpret_cast<uintptr_t>(vals) & 15) != 0 || (a.ld & 3) != 0 || n > a.ld) {
+  // (and the gathering pass counts elements in 32 bits)
+  if ((reinterpret_cast<uintptr_t>(vals) & 15) != 0 || (a.ld & 3) != 0 || n > a.ld ||
+      n > 0x7fffffff - kRingStep) {
     radix_row(a, r, 0, hist, warp_tot, sh);
     return;
   }
@@ -1054,40 +1057,54 @@ __global__ void __launch_bounds__(kSelThreads, 2) long_select_kernel(const Selec
     if (threadIdx.x == 0) {
       fence_proxy_async_smem();  // the ring's earlier contents were written by the threads
       for (int64_t j = 0; j < kRingSlots - 1 && j < n_steps; ++j) fill(j);
-      ok = landed(0);
+      ok = n_steps < 1 || landed(0);
     }
-    int64_t s = 0;
+    // 32-bit loop state (the row is shorter than 2^31 - kRingStep elements); the slot and its
+    // phase advance with the step
+    const int ns = static_cast<int>(n_steps);
+    int slot = static_cast<int>(fbase % kRingSlots);
+    uint32_t ph = (fbase / kRingSlots) & 1u;
+    uint32_t i0 = 8u * threadIdx.x;  // index of this thread's first element of the step
+    int s = 0;
     if (__syncthreads_and(ok)) {
 #pragma unroll 1
-      for (; s < n_steps; ++s) {
-        const uint32_t f = fbase + static_cast<uint32_t>(s);
-        const int slot = static_cast<int>(f % kRingSlots);
-        (void)mbar_try_wait(&full[slot], (f / kRingSlots) & 1u);  // complete: orders the reads
+      for (; s < ns; ++s, i0 += kRingStep) {
+        (void)mbar_try_wait(&full[slot], ph);  // complete: orders the reads
         const float* mine = ring + slot * kRingStep + 8 * threadIdx.x;
         const float4 d0 = reinterpret_cast<const float4*>(mine)[0];
         const float4 d1 = reinterpret_cast<const float4*>(mine)[1];
-        const int64_t i0 = s * kRingStep + 8 * static_cast<int64_t>(threadIdx.x);
         // bit j: element j of this thread is >= tau (past the row's end on the last step: no)
         uint32_t msk = ge_bits8(d0, d1, tau_f);
-        if (s + 1 == n_steps) {
-          const int64_t left = n - i0;
+        if (s + 1 == ns) {
+          const int left = static_cast<int>(static_cast<uint32_t>(n) - i0);
           msk &= left >= 8 ? 0xffu : (left <= 0 ? 0u : ((1u << left) - 1u));
         }
         const uint32_t nm = __popc(msk);
-        const uint32_t incl = warp_inclusive_sum(nm);
+        // this lane's first slot in the warp and the warp's count: one ballot while no lane
+        // has two or more (the usual case: about 1 % of the elements pass), else a scan
+        uint32_t ex, wt;
+        if (__any_sync(0xffffffffu, nm > 1u)) {
+          const uint32_t incl = warp_inclusive_sum(nm);
+          ex = incl - nm;
+          wt = __shfl_sync(0xffffffffu, incl, 31);
+        } else {
+          const uint32_t b = __ballot_sync(0xffffffffu, nm != 0u);
+          ex = __popc(b & lanes_below);
+          wt = __popc(b);
+        }
         uint32_t* st = step_tot[s & 1];
-        if (lane == 31) st[warp] = incl;
+        if (lane == 0) st[warp] = wt;
         ok = 1;
-        if (threadIdx.x == 0 && s + 1 < n_steps) ok = landed(s + 1);
+        if (threadIdx.x == 0 && s + 1 < ns) ok = landed(s + 1);
         // every thread is done with the previous step's slot, which takes step s + R - 1
         if (!__syncthreads_and(ok)) break;
-        if (threadIdx.x == 0 && s + kRingSlots - 1 < n_steps) fill(s + kRingSlots - 1);
+        if (threadIdx.x == 0 && s + kRingSlots - 1 < ns) fill(s + kRingSlots - 1);
         const uint32_t x = lane < kSelWarps ? st[lane] : 0u;
         const uint32_t tot = __reduce_add_sync(0xffffffffu, x);
         const uint32_t before = __reduce_add_sync(0xffffffffu, lane < warp ? x : 0u);
         // this thread's elements >= tau, in index order; their values are read again from the
         // slot, which is not refilled before the next step's barrier
-        uint32_t at = C + before + incl - nm;
+        uint32_t at = C + before + ex;
         for (uint32_t mm = msk; mm != 0u; mm &= mm - 1u, ++at) {
           const int j = __ffs(mm) - 1;
           if (at < static_cast<uint32_t>(kLongCap)) {
@@ -1096,9 +1113,13 @@ __global__ void __launch_bounds__(kSelThreads, 2) long_select_kernel(const Selec
           }
         }
         C += tot;
+        if (++slot == kRingSlots) {
+          slot = 0;
+          ph ^= 1u;
+        }
       }
     }
-    if (s < n_steps) {
+    if (s < ns) {
       // a copy did not land in time: report it, let every copy of this pass that was issued
       // land (bounded) before the CTA's shared memory is released, and leave the row
       if (threadIdx.x == 0) {
@@ -1108,7 +1129,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) long_select_kernel(const Selec
           a.status->info1 = r;
         }
         volatile int never = 0;
-        const int64_t issued = min(n_steps, s + kRingSlots - 1);  // fills s .. issued-1 may be pending
+        const int64_t issued = min(n_steps, static_cast<int64_t>(s) + kRingSlots - 1);  // fills s .. issued-1 may be pending
         for (int64_t j = s; j < issued; ++j) {
           const uint32_t f = fbase + static_cast<uint32_t>(j);
           (void)mbar_wait(&full[f % kRingSlots], (f / kRingSlots) & 1u, &never, kLongTimeoutNs);
