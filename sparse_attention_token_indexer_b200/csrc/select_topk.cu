@@ -803,9 +803,10 @@ select_reg_kernel(const SelectArgs a, int row0) {
 //      common high bits give the bins of the sample's r-th and 4r-th largest keys,
 //      r = 5/4 * K * m / n + 8, whose lower edges are the thresholds tau: about 5/4 of K
 //      elements of the row are expected at or above the first.
-//   2. One pass gathers every valid element >= tau into shared memory in index order: each
-//      thread tests 16 consecutive elements of a step of 8192 (the next step's loads already in
-//      flight) and a block scan of the per-thread counts gives their slots. Fewer than K
+//   2. One pass gathers every valid element >= tau into shared memory in index order: the
+//      row streams through a ring of 16 KB bulk copies (up to four in flight), each thread
+//      tests 8 consecutive elements of a step, and one warp ballot (a shuffle scan when a lane
+//      has two or more) plus one barrier with warp reductions give their slots. Fewer than K
 //      gathered (the estimate was too high): the pass is repeated at the lower tau, then at
 //      every element; more than the buffer holds (many equal keys): the row takes the
 //      multi-pass radix select.
