@@ -283,6 +283,11 @@ def test_paper_fallback_rule():
     plans = ox.plan_groups(T=40, q_pos0=0, G=8, B=16, mode="paper")
     # anchors 0, 8, 16, 24, 32: reuse needs a + 1 > 16; the last group is complete
     assert [p.kind for p in plans] == ["flat", "flat", "bank", "bank", "bank"]
+    # at the boundary: a bank only when the anchor's visible prefix a + 1 exceeds B (ADIndex
+    # §4.3, Shared Token Bank Construction; Appendix A: a prefix that does not exceed the
+    # budget falls back), so the anchor 16 with a + 1 = B = 17 takes the plain indexer
+    plans = ox.plan_groups(T=40, q_pos0=0, G=8, B=17, mode="paper")
+    assert [p.kind for p in plans] == ["flat", "flat", "flat", "bank", "bank"]
     plans = ox.plan_groups(T=36, q_pos0=0, G=8, B=16, mode="paper")
     assert plans[-1].kind == "flat" and len(plans[-1].rows) == 4   # incomplete group
     # MTP: the whole window falls back when its first query sees <= B keys
@@ -307,6 +312,13 @@ def test_decode_bank_reuse_matches_definitions():
     for b in range(Bs):
         allowed = set(banks[b].tolist()) | set(range(n0[b], n0[b] + 4))
         assert set(got[b].tolist()) <= allowed and len(got[b]) == K
+    # Eq. (13) scans s <= t, the anchor's own key included: a key at the anchor that the group
+    # query scores far above the rest is in the bank
+    c2 = caches.copy()
+    for b in range(Bs):
+        c2[b, n0[b] - 1] = 1000.0 * qbar[b, 0]
+    banks2 = ox.decode_bank(qbar, wbar, c2, n0, B)
+    assert all(int(n0[b]) - 1 in set(banks2[b].tolist()) for b in range(Bs))
 
 
 # ---------------------------------------------------------------------------------------
@@ -518,6 +530,9 @@ def test_rope_identity_norms_inverse_and_a_hand_value():
     e[0] = 1.0
     assert np.allclose(ox.rope(e, 1, 4)[:2], [np.cos(1.0), np.sin(1.0)])   # pair 0: angle = pos
     assert np.allclose(ox.rope(e[[1, 0, 2, 3]], 1, 4)[:2], [-np.sin(1.0), np.cos(1.0)])
+    # pair i turns by pos * base^(-2i / rope_dim): pair 1 of a 4-dim rotary part at position 1
+    # turns by 10000^(-1/2) = 0.01
+    assert np.allclose(ox.rope(e[[2, 3, 0, 1]], 1, 4)[2:], [np.cos(0.01), np.sin(0.01)])
 
 
 def test_group_indexer_pools_projects_and_gates():
