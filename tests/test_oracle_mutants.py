@@ -347,6 +347,33 @@ def hisa_short_prefix_strict(q_t, w_t, k, kbar, p, K, n_blocks, block=ox.HISA_BL
     return ox.topk(ox.score_keys(q_t, w_t, k[cand]), K, cand)
 
 
+def decode_topk_one_early(q, w, caches, seq_len, K):  # the row placed at seq_len - 2
+    return {b: ox.flat_topk_row(q[b], w[b], caches[b], int(seq_len[b]) - 2, K)
+            for b in range(q.shape[0])}
+
+
+def base_cost_no_self(T, q_pos0):  # the plain indexer's own-position score not counted
+    return sum(q_pos0 + t for t in range(T))
+
+
+def mtp_round_cost_late(N, G, P, m=16, mode="paper"):  # the window's first query sees N + 1 keys
+    return cost_model.plan_cost(ox.plan_groups(m, N, G, P, mode, fallback="window"), N)
+
+
+_base_cost, _prefill_cost, _mtp_round_cost = (cost_model.base_cost, cost_model.prefill_cost,
+                                              cost_model.mtp_round_cost)
+
+
+def speedups_rounds_from_one(L, G, P, R=32, m=16, a=8):  # round j's prefix L + j a, not L + (j-1) a
+    pre_b, pre_r = _base_cost(L, 0), _prefill_cost(L, G, P)
+    jb, jr = pre_b, pre_r
+    for j in range(1, R + 1):
+        n = L + j * a
+        jb += _base_cost(m, n - 1)
+        jr += _mtp_round_cost(n, G, P, m)
+    return pre_b / pre_r, _base_cost(m, L - 1) / _mtp_round_cost(L, G, P, m), jb / jr
+
+
 # (module, attribute, planted mistake, pins that must catch it)
 CASES = [
     ("score: no ReLU", ox, "score_keys", score_no_relu,
@@ -423,6 +450,14 @@ CASES = [
      [tp.test_candidates_stay_causal_and_in_bank, tp.test_mtp_banked_window_matches_the_equations]),
     ("HISA: a prefix of K tokens filtered", ox, "hisa_topk_row", hisa_short_prefix_strict,
      [tp.test_hisa_short_prefix_keeps_every_token, tp.test_hisa_matches_brute_force_subsets]),
+    ("decode: row one position early", ox, "decode_topk", decode_topk_one_early,
+     [tp.test_decode_bank_reuse_matches_definitions]),
+    ("cost: own position not counted", cost_model, "base_cost", base_cost_no_self,
+     [tp.test_cost_closed_forms_of_appendix_a, tp.test_table5_reproduced_by_the_group_plan, tc.test_speedup_reproduces_table5_panel_c]),
+    ("cost: MTP window one key late", cost_model, "mtp_round_cost", mtp_round_cost_late,
+     [tp.test_cost_closed_forms_of_appendix_a, tp.test_table5_reproduced_by_the_group_plan, tc.test_speedup_reproduces_table5_panel_c]),
+    ("cost: MTP rounds from L + a", cost_model, "speedups", speedups_rounds_from_one,
+     [tp.test_cost_closed_forms_of_appendix_a, tp.test_table5_reproduced_by_the_group_plan, tc.test_speedup_reproduces_table5_panel_c]),
     ("cost: post-anchor keys not counted", cost_model, "plan_cost", plan_cost_no_post,
      [tp.test_table5_reproduced_by_the_group_plan, tc.test_speedup_reproduces_table5_panel_c]),
 ]

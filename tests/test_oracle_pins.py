@@ -335,6 +335,33 @@ def _table5():
     return rows
 
 
+def test_cost_closed_forms_of_appendix_a():
+    """ADIndex Appendix A, exact: a verification round's baseline count m N + m (m - 1) / 2
+    (Eq. (16), query r of the round sees N + r keys); an active round's count
+    sum over its m / G groups b of N + bG + GP + G (G - 1) / 2 (Eq. (20)); the prefill baseline
+    sum_t (t + 1) = L (L + 1) / 2 (the discrete sum Eq. (15) integrates); and the joint
+    workload's rounds at N_j = L + (j - 1) a, so sum_j N_j = R L + a R (R - 1) / 2 (Eqs. (28),
+    (29)), which fixes the joint speedup given the prefill counts."""
+    m = 16
+    for N in (5000, 16384, 70001):
+        assert cost_model.base_cost(m, N - 1) == m * N + m * (m - 1) // 2
+        for G in (4, 8, 16):
+            for P in (1024, 4096):
+                assert cost_model.mtp_round_cost(N, G, P, m) == sum(
+                    N + b * G + G * P + G * (G - 1) // 2 for b in range(m // G))
+    for L in (4096, 20000):
+        assert cost_model.base_cost(L, 0) == L * (L + 1) // 2
+    L, R, a = 65536, 32, 8
+    S = R * L + a * R * (R - 1) // 2
+    for G in (4, 8, 16):
+        for P in (4096, 16384):
+            nb = m // G
+            jb = L * (L + 1) // 2 + m * S + R * m * (m - 1) // 2
+            jr = cost_model.prefill_cost(L, G, P) + nb * S + R * (
+                G * nb * (nb - 1) // 2 + nb * (G * P + G * (G - 1) // 2))
+            assert cost_model.speedups(L, G, P, R, m, a)[2] == pytest.approx(jb / jr, rel=1e-12)
+
+
 def test_group_cost_matches_eq17():
     # one bank group with anchor visible prefix N: N + G P + G (G - 1) / 2
     G, P, a = 16, 4096, 10000
