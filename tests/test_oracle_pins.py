@@ -218,7 +218,7 @@ def test_candidates_stay_causal_and_in_bank():
 
 
 def test_window_group_cost_closed_form():
-    """WINDOW reading (BASELINE's group workload; ADIndex §4.3, Eqs. (13)-(14)): a bank group
+    """WINDOW reading (the group-mode workloads; ADIndex §4.3, Eqs. (13)-(14)): a bank group
     whose anchor a has at least B - G keys before it scores a scan of the a keys s < a, then
     member i = a + r (r = 0 .. G-1) scores the B - G bank keys plus its r + 1 window keys
     a .. a + r: a + G (B - G) + G (G + 1) / 2 in all. With fewer than B - G keys before the
